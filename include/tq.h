@@ -1,0 +1,224 @@
+/*
+ * tq.h — C ABI of a compressed KV-cache library for NVIDIA B200 (sm_100a).
+ *
+ * The library does two things on the GPU:
+ *   1. tq_encode   — compress K/V head vectors: FP16 norm, seeded randomized
+ *                    Hadamard rotation, Lloyd-Max scalar codebook, bit-packing.
+ *   2. tq_attend   — decode attention that reads only the packed cache.
+ * plus tq_dequant (verification) and tq_build_codebook (host-side solver).
+ *
+ * Sources (cited below by the key in brackets, then the section):
+ *   [TQAI]   "We Built a Python Library That Cuts LLM Memory Usage by 80%"
+ *            (dev.to, tqai library post)
+ *   [ADAPTQ] "AdapTQ — Adaptive Streaming Vector Quantization KV Cache for
+ *            LLMs" (PyPI project page, adaptq 0.2.3)
+ *   [TQPLUS] "TurboQuant+: Compresión de Caché KV 6.4x para LLMs" (aibit.im)
+ *
+ * Conventions shared by every entry point
+ *   - Pointers are DEVICE pointers unless marked "host".
+ *   - The caller owns every buffer. No entry point allocates device memory;
+ *     scratch space for tq_attend is passed in by the caller.
+ *   - GPU entry points are asynchronous on `stream` (a cudaStream_t passed as
+ *     void*; NULL means the legacy default stream). They validate arguments
+ *     on the host, enqueue kernels and return without synchronizing. A
+ *     TQ_ERR_CUDA return reports a launch failure (cudaGetLastError);
+ *     execution errors surface at the caller's next synchronization.
+ *   - Entry points hold no global state: codebooks and the sign vector travel
+ *     to the kernels as launch parameters, so calls are thread-safe.
+ *   - Kernels never trap and never spin. Device-side conditions set bits in
+ *     the optional *dev_status word (atomicOr; the caller zeroes it).
+ *
+ * Frozen format definitions (the pages leave these open; these readings are
+ * the library's own and the test oracle implements the same definitions):
+ *   - Codebook: Lloyd-Max quantizer for N(0,1) with 2^b levels, symmetric,
+ *     ascending; thresholds are the midpoints between adjacent centroids.
+ *     The N(0,1/d) codebook of [TQAI §The Paper] is that codebook / sqrt(d).
+ *     Kernels compare zeta = z/||x|| against the N(0,1) thresholds, where
+ *     z = H·(D⊙x) with the unnormalized Hadamard matrix, so zeta = sqrt(d)·y.
+ *   - Index: idx_i = #{ j : zeta_i >= t_j } (a value on a threshold goes to
+ *     the upper cell).
+ *   - Sign vector D: SplitMix64 (Steele, Lea & Flood 2014) with state = seed;
+ *     D_i = -1 iff bit 63 of the i-th output (i = 0..d-1) is set. The same D
+ *     serves K, V, all heads and the query; pass one seed per layer.
+ *   - Hadamard: Sylvester order, H[i][j] = (-1)^popcount(i & j).
+ *   - Packing: LSB-first contiguous. Row bit (i·b + k) is bit k of idx_i;
+ *     row byte j holds row bits 8j..8j+7. One row of d·b/8 bytes per
+ *     (sequence, kv head, token).
+ *   - Norm: ||x||_2 of the fp16/bf16 input promoted to float, stored as IEEE
+ *     fp16 with round-to-nearest-even, saturated to 65504 (TQ_DEV_NORM_SATURATED).
+ *     The unit vector is formed with the unrounded norm.
+ *   - Sparse-V gate [TQPLUS §2 Sparse V]: with tau = sparse_v_thresh > 0, the
+ *     V row at position t is left out of query head h's accumulation iff
+ *     exp(s_t - M_blk(t)) < tau, where M_blk(t) is the maximum score of head h
+ *     over the aligned block of TQ_SPARSE_V_BLOCK positions containing t
+ *     (blocks start at position 0). Gated positions still count in the
+ *     softmax denominator. tau <= 0 disables the gate.
+ *
+ * Cache layout (attend/dequant):
+ *   packed_k : uint8 [batch][n_kv_heads][cap_tok][d*bits_k/8]
+ *   packed_v : uint8 [batch][n_kv_heads][cap_tok][d*bits_v/8]
+ *   norms_k, norms_v : fp16 bits (uint16) [batch][n_kv_heads][cap_tok]
+ * tq_encode writes one sequence (batch index 0 of that layout, i.e. pass the
+ * base pointers of the sequence you are filling).
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TQ_ABI_VERSION 1
+
+/* Tokens per sparse-V block; split boundaries are multiples of this. */
+#define TQ_SPARSE_V_BLOCK 64
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARG = 1,    /* a null pointer, a size out of range, ... */
+  TQ_ERR_UNSUPPORTED = 2,    /* valid in principle, not built (e.g. d != 128) */
+  TQ_ERR_CUDA = 3,           /* a CUDA runtime call or launch failed */
+  TQ_ERR_NO_CONVERGENCE = 4  /* the Lloyd-Max iteration did not converge */
+} tq_status;
+
+typedef enum { TQ_F16 = 0, TQ_BF16 = 1, TQ_F32 = 2 } tq_dtype;
+
+/* Bits of *dev_status (device int, zeroed by the caller, set with atomicOr). */
+#define TQ_DEV_CTX_CLAMPED    1  /* some ctx_lens[b] > cap_tok; clamped     */
+#define TQ_DEV_NORM_SATURATED 2  /* some norm > 65504; stored as 65504      */
+#define TQ_DEV_CTX_EMPTY      4  /* some ctx_lens[b] <= 0; output set to 0  */
+
+/* Library ABI version (TQ_ABI_VERSION of the build). */
+int tq_abi_version(void);
+
+/* Static, human-readable name of a status code. */
+const char* tq_status_string(int status);
+
+/*
+ * tq_build_codebook — host-side Lloyd-Max solver for the post-rotation
+ * coordinate distribution N(0, 1/d) [TQAI §The Paper: after the rotation a
+ * coordinate is modelled as Gaussian with variance 1/d, so the optimal
+ * scalar quantizer is fixed in advance and needs no data; ADAPTQ §How it
+ * works, item 2].
+ *
+ *   bits        1..8; the codebook has N = 2^bits levels.
+ *   d           head dimension >= 1 (d = 1 gives the N(0,1) codebook).
+ *   centroids   host, N doubles, ascending, symmetric about 0.
+ *   thresholds  host, N-1 doubles, t_j = (c_{j-1} + c_j)/2, ascending.
+ *   mse         host, nullable: expected squared error of a rotated unit
+ *               vector, i.e. the per-coordinate MSE in N(0,1) units
+ *               (0.1175 / 0.03454 / 0.009497 at 2 / 3 / 4 bits).
+ * Pure host computation: needs no GPU. Returns TQ_ERR_INVALID_ARG on bad
+ * arguments, TQ_ERR_NO_CONVERGENCE if the fixed point is not reached.
+ */
+int tq_build_codebook(int bits, int d, double* centroids, double* thresholds,
+                      double* mse);
+
+/*
+ * tq_encode — compress n_tok tokens of one sequence into a packed cache
+ * [TQAI §The Paper (rotate, quantize each coordinate, store the norm in
+ * FP16); ADAPTQ §How it works, items 1-2 (y = (1/sqrt d)·H·D·x via FWHT,
+ * Max-Lloyd codebook); TQAI §Compression numbers (K4/V2, K3/V2, K4/V3) and
+ * §What's Next (bit-packing)].
+ *
+ *   kv          [2][n_tok][n_kv_heads][d] of `dtype` (TQ_F16 or TQ_BF16):
+ *               the K block followed by the V block, token-major as a
+ *               projection produces them. 16-byte aligned.
+ *   n_tok       >= 0 tokens to encode (0 is a no-op).
+ *   n_kv_heads  >= 1.
+ *   d           head dimension; this build supports d = 128
+ *               (other powers of two in [64, 256]: TQ_ERR_UNSUPPORTED).
+ *   bits_k, bits_v  2..4 bits per coordinate for K and for V.
+ *   seed        sign-vector seed (see "Sign vector D" above).
+ *   packed_k    [n_kv_heads][cap_tok][d*bits_k/8] bytes, 16-byte aligned.
+ *   packed_v    [n_kv_heads][cap_tok][d*bits_v/8] bytes, 16-byte aligned.
+ *   norms_k, norms_v  [n_kv_heads][cap_tok] fp16 bits.
+ *   cap_tok     token capacity of the cache rows (>= 1).
+ *   tok_offset  first row written; rows tok_offset .. tok_offset+n_tok-1.
+ *               tok_offset + n_tok <= cap_tok, else TQ_ERR_INVALID_ARG.
+ *   dev_status  device int, nullable; TQ_DEV_NORM_SATURATED may be set.
+ *   stream      cudaStream_t.
+ * Rows outside the written range are untouched.
+ */
+int tq_encode(const void* kv, int dtype, int n_tok, int n_kv_heads, int d,
+              int bits_k, int bits_v, uint64_t seed,
+              uint8_t* packed_k, uint8_t* packed_v,
+              uint16_t* norms_k, uint16_t* norms_v,
+              int cap_tok, int tok_offset, int* dev_status, void* stream);
+
+/*
+ * tq_dequant — reconstruct vectors from one packed cache (K or V) for
+ * verification; not used by tq_attend.
+ *
+ *   packed      [n_kv_heads][cap_tok][d*bits/8] bytes.
+ *   norms       [n_kv_heads][cap_tok] fp16 bits.
+ *   n_tok       rows 0..n_tok-1 of each head are reconstructed (<= cap_tok).
+ *   domain      0: original space, x_hat = fp16norm · D⊙(H·c[idx]) / d;
+ *               1: rotated unit-vector coordinates c[idx] / sqrt(d)
+ *               (the N(0,1/d) codebook values, norm not applied).
+ *   out         float [n_kv_heads][n_tok][d].
+ */
+int tq_dequant(const uint8_t* packed, const uint16_t* norms, int n_tok,
+               int n_kv_heads, int d, int bits, uint64_t seed, int cap_tok,
+               int domain, float* out, void* stream);
+
+/*
+ * tq_attend_workspace_size — bytes of scratch tq_attend needs for these
+ * sizes and this split_tokens argument (0 = the library's choice). The
+ * split-K partials are (m, l, acc[d]) in fp32 per (batch, query head, split).
+ */
+size_t tq_attend_workspace_size(int batch, int n_q_heads, int cap_tok, int d,
+                                int split_tokens);
+
+/*
+ * tq_attend — single-query decode attention over the packed cache
+ * [ADAPTQ §How it works, item 3: the query is rotated a single time and the
+ * scores are formed from the packed indices, never materializing the
+ * dequantized cache; TQAI §What's Next: fused decode over compressed data;
+ * TQAI §Test Suite: the attention being approximated is
+ * softmax(Q·K^T/sqrt d)·V; TQPLUS §2 Sparse V].
+ *
+ * For batch b and query head h (kv head g = h / gqa_ratio, i.e. consecutive
+ * query heads share a kv head) with L = min(ctx_lens[b], cap_tok):
+ *   q~   = H·(D⊙q) / sqrt(d)                       (rotated once)
+ *   s_t  = (1/sqrt d) · nK_t · sum_i q~_i · cK[idxK_t,i] / sqrt(d),  t < L
+ *   w_t  = exp(s_t - max s),  l = sum_t w_t
+ *   acc  = sum_{t not gated} w_t · nV_t · cV[idxV_t] / sqrt(d)
+ *   out  = D⊙(H·(acc / l)) / sqrt(d)               (inverse-rotated once)
+ * where c are the N(0,1) codebooks and nK, nV the stored fp16 norms.
+ *
+ *   q           [batch][n_q_heads][d] of q_dtype (TQ_F16 | TQ_BF16 | TQ_F32).
+ *   packed_*, norms_*  the cache layout above, with a leading batch dim.
+ *   ctx_lens    int32 [batch] on the device. Values > cap_tok are clamped
+ *               (TQ_DEV_CTX_CLAMPED); values <= 0 give out = 0
+ *               (TQ_DEV_CTX_EMPTY).
+ *   batch >= 1; n_q_heads >= 1; gqa_ratio >= 1 divides n_q_heads.
+ *   d, bits_k, bits_v, seed   as used by tq_encode for this cache.
+ *   sparse_v_thresh  tau of the sparse-V gate; <= 0 disables it.
+ *   split_tokens     tokens per split-K work item: 0 = library's choice,
+ *                    else a positive multiple of TQ_SPARSE_V_BLOCK.
+ *   workspace, workspace_bytes  >= tq_attend_workspace_size(...) bytes,
+ *                    16-byte aligned; contents on entry are ignored.
+ *   dev_status  device int, nullable.
+ *   sparse_v_skipped  device uint64, nullable: atomically incremented by the
+ *               number of (b, h, t) positions the gate left out.
+ *   out         [batch][n_q_heads][d] of out_dtype (TQ_F16 | TQ_BF16 | TQ_F32).
+ */
+int tq_attend(const void* q, int q_dtype,
+              const uint8_t* packed_k, const uint16_t* norms_k,
+              const uint8_t* packed_v, const uint16_t* norms_v,
+              const int32_t* ctx_lens, int batch, int n_q_heads,
+              int gqa_ratio, int d, int bits_k, int bits_v, uint64_t seed,
+              int cap_tok, float sparse_v_thresh, int split_tokens,
+              void* workspace, size_t workspace_bytes, int* dev_status,
+              unsigned long long* sparse_v_skipped,
+              void* out, int out_dtype, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

@@ -1,0 +1,99 @@
+"""The pins catch plausible oracle mistakes (CPU).
+
+Each case plants one mistake in the oracle (monkeypatched for the duration of
+the case only) and checks that at least one pin test then fails.
+"""
+import numpy as np
+import pytest
+
+import test_oracle_attention as ta
+import test_oracle_codebook as tcb
+import test_oracle_codec as tc
+import test_oracle_rotation as tr
+from oracle import attention, codebook, codec, rotation
+
+
+def _fails(fn, *args):
+    with pytest.raises(AssertionError):
+        fn(*args)
+
+
+def test_sign_bit_choice_is_pinned(monkeypatch):
+    real = rotation.splitmix64
+    monkeypatch.setattr(rotation, "sign_vector", lambda seed, d: np.array(
+        [-1.0 if (v >> 62) & 1 else 1.0 for v in real(seed, d)]))
+    _fails(tr.test_sign_vector_definition)
+
+
+def test_missing_sign_flip_in_encode(monkeypatch):
+    # the encoder loses D; the closed-form input is still built with the real D
+    real_signs = rotation.sign_vector
+    real_helper = tc._x_from_zeta
+    def helper(z, s):
+        monkeypatch.setattr(rotation, "sign_vector", real_signs)
+        try:
+            return real_helper(z, s)
+        finally:
+            monkeypatch.setattr(rotation, "sign_vector", lambda seed, d: np.ones(d))
+    monkeypatch.setattr(tc, "_x_from_zeta", helper)
+    monkeypatch.setattr(rotation, "sign_vector", lambda seed, d: np.ones(d))
+    _fails(tc.test_closed_form_indices, 4)
+
+
+def test_query_rotation_without_signs(monkeypatch):
+    real_rotate = rotation.rotate
+    monkeypatch.setattr(rotation, "rotate",
+                        lambda x, seed: x @ rotation.hadamard(x.shape[-1]).T / np.sqrt(x.shape[-1]))
+    _fails(ta.test_matches_dense_brute_force, 4, 2, 1)
+    monkeypatch.setattr(rotation, "rotate", real_rotate)
+
+
+def test_dropped_score_scale(monkeypatch):
+    real = codec.dequant_rotated
+    monkeypatch.setattr(codec, "dequant_rotated", lambda idx, bits: real(idx, bits) * np.sqrt(idx.shape[-1]))
+    _fails(ta.test_matches_dense_brute_force, 4, 2, 1)
+
+
+def test_ties_to_lower_cell(monkeypatch):
+    monkeypatch.setattr(codec, "quantize_index",
+                        lambda z, t: np.searchsorted(t, z, side="left").astype(np.int64))
+    _fails(tc.test_ties_go_to_upper_cell)
+
+
+def test_msb_first_packing(monkeypatch):
+    def pack_msb(idx, bits):
+        n, d = idx.shape
+        planes = (idx[:, :, None] >> np.arange(bits)[::-1]) & 1
+        return np.packbits(planes.reshape(n, d * bits).astype(np.uint8), axis=1)
+    monkeypatch.setattr(codec, "pack", pack_msb)
+    _fails(tc.test_packing_golden_bytes)
+
+
+def test_wrong_threshold_rule(monkeypatch):
+    real = codebook.lloyd_max_normal
+    def bad(bits, **kw):
+        c, t = real(bits)
+        return c, t * 1.01
+    monkeypatch.setattr(codebook, "lloyd_max_normal", bad)
+    _fails(tcb.test_fixed_point_with_independent_normal, 3)
+
+
+def test_gate_with_global_max(monkeypatch):
+    monkeypatch.setattr(attention, "GATE_BLOCK", 1 << 20)
+    _fails(ta.test_gate_matches_brute_force, 0.05)
+
+
+def test_wrong_gqa_mapping(monkeypatch):
+    real = attention.attend_head_group
+    def swapped(qs, *a, **k):
+        return real(qs[::-1].copy(), *a, **k)
+    monkeypatch.setattr(attention, "attend_head_group", swapped)
+    _fails(ta.test_matches_dense_brute_force, 4, 3, 4)
+
+
+def test_norm_not_saturated(monkeypatch):
+    def unsaturated(n):
+        with np.errstate(over="ignore"):
+            return np.asarray(n).astype(np.float16).view(np.uint16)
+    monkeypatch.setattr(codec, "fp16_norm_bits", unsaturated)
+    _fails(tc.test_norm_rounding_and_saturation)
