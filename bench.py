@@ -1,0 +1,506 @@
+#!/usr/bin/env python3
+"""Benchmark: decode attention over the packed KV cache, and bulk encode.
+
+One step = one decode step of a 32-layer Llama-3-8B-shaped model (batch 1,
+32 query heads, 8 kv heads, d = 128, 32768 cached tokens, K4/V2, fp16): for
+every layer, tq_encode appends the new token's K/V to that layer's packed
+cache and tq_attend attends over all 32768 positions. The 32 layer caches
+(839 MB) are distinct, so successive reads of a layer are far apart and the
+126 MB L2 cannot hold them. Steps are CUDA-graph replays.
+
+  value   packed-KV GB/s: algorithmic bytes of the step (packed K/V rows,
+          fp16 norms, q and out, plus the encode's input/output) / step time
+  e2e     the same bytes over a step that also copies the step's inputs from
+          pinned host memory and its output back
+  encode  bulk prefill encode of the same 32 x 8 x 32768 K/V (4.29 GB of fp16
+          input): Mtok/s (model tokens/s and token-head vectors/s)
+
+`--impl reference` times the CPU oracle (float64 numpy) on a bounded sample
+of the same workload instead.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own replica of
+the workload (weak scaling, no collective on the data path); the step time is
+the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic as S  # noqa: E402
+
+METRIC = "decode-attn packed-KV GB/s & % HBM roofline; encode Mtok/s (1×B200)"
+WORKLOAD = "llama3_8b_decode"
+ENCODE_WORKLOAD = "bulk_prefill_encode"
+LAYERS = 32
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------------ helpers
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def attend_bytes(w, ctx_total, q_bytes=2, out_bytes=2):
+    """Algorithmic bytes of one tq_attend call: packed rows + norms + q + out."""
+    row = w.d * w.bits_k // 8 + w.d * w.bits_v // 8 + 4
+    return ctx_total * w.n_kv_heads * row + w.batch * w.n_q_heads * w.d * (q_bytes + out_bytes)
+
+
+def encode_bytes(w, n_vec_pairs):
+    """Algorithmic bytes of tq_encode over n (token, kv head) K/V pairs."""
+    return n_vec_pairs * (2 * w.d * 2 + w.d * w.bits_k // 8 + w.d * w.bits_v // 8 + 4)
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for fn in ("attend.cu", "device_common.cuh", "tq_internal.h"):
+        with open(os.path.join(ROOT, "compressed_decode_attention_b200", "csrc", fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """dram bytes per launch from the last ncu capture, if the kernel source
+    is unchanged since (profiles/traffic.json), else None."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+        if t.get("kernel_source_sha") == kernel_source_sha():
+            return t
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init_dist(world, backend):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def reduce_max(x: float, device=None) -> float:
+    """Maximum of a per-rank float over all ranks (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and str(device).startswith("cuda"):
+            dist.barrier(device_ids=[int(str(device).split(":")[1])])
+        else:
+            dist.barrier()
+
+
+# ------------------------------------------------------------------ GPU arm
+class LayerCaches:
+    """Device buffers of the 32-layer decode workload."""
+
+    def __init__(self, w, layers, stream):
+        import torch
+        self.w = w
+        d, H, cap = w.d, w.n_kv_heads, w.cap_tok
+        dev = "cuda"
+        self.rk, self.rv = d * w.bits_k // 8, d * w.bits_v // 8
+        self.pk = [torch.empty((1, H, cap, self.rk), dtype=torch.uint8, device=dev) for _ in range(layers)]
+        self.pv = [torch.empty((1, H, cap, self.rv), dtype=torch.uint8, device=dev) for _ in range(layers)]
+        self.nk = [torch.empty((1, H, cap), dtype=torch.int16, device=dev) for _ in range(layers)]
+        self.nv = [torch.empty((1, H, cap), dtype=torch.int16, device=dev) for _ in range(layers)]
+        self.stream = stream
+
+
+def device_kv(w, layer, n_tok, gen):
+    """fp16 K/V [2][n][H][d] on the device: N(0,1) with the workload's x20
+    outlier K channels (same recipe as synthetic.kv_f32, torch's generator)."""
+    import torch
+    x = torch.randn((2, n_tok, w.n_kv_heads, w.d), generator=gen, device="cuda",
+                    dtype=torch.float32)
+    ch = S.outlier_channels(w, layer)
+    for h in range(w.n_kv_heads):
+        x[0, :, h, torch.as_tensor(ch[h], device="cuda")] *= 20.0
+    return x.half().view(torch.int16)
+
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import compressed_decode_attention_b200 as tq
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    w = S.WORKLOADS[WORKLOAD]
+    we = S.WORKLOADS[ENCODE_WORKLOAD]
+    assert (we.n_kv_heads, we.ctx, we.bits_k, we.bits_v) == (w.n_kv_heads, w.ctx, w.bits_k, w.bits_v)
+    L = args.layers
+    stream = torch.cuda.Stream(device)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(S.DATA_SEED + 7919 * rank)
+    seed = S.SIGN_SEED
+    caches = LayerCaches(w, L, stream)
+    H, d, ctx, cap = w.n_kv_heads, w.d, w.ctx, w.cap_tok
+    launches = 0
+
+    # ---------------- bulk encode (prefill) of every layer: the encode metric
+    kv_all = [device_kv(we, l, ctx, gen) for l in range(L)]
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def encode_all():
+        for l in range(L):
+            tq.tq_encode(kv_all[l], tq.TQ_F16, ctx, H, d, w.bits_k, w.bits_v, seed,
+                         caches.pk[l], caches.pv[l], caches.nk[l], caches.nv[l], cap, 0,
+                         status, stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            encode_all()
+    torch.cuda.synchronize()
+    enc_steps = max(3, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(device)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(enc_steps):
+            encode_all()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    enc_ms = reduce_max(e0.elapsed_time(e1) / enc_steps, device)
+    enc_launches = enc_steps * L
+    del kv_all
+    torch.cuda.empty_cache()
+
+    # ---------------- decode step graphs
+    q = [torch.randn((1, w.n_q_heads, d), generator=gen, device=device).half() for _ in range(L)]
+    kv_new = [device_kv(w, l, 1, gen) for l in range(L)]
+    outs = [torch.empty((1, w.n_q_heads, d), dtype=torch.float16, device=device) for _ in range(L)]
+    ctx_dev = torch.full((1,), ctx, dtype=torch.int32, device=device)
+    ws_bytes = tq.tq_attend_workspace_size(1, w.n_q_heads, cap, d, 0)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
+
+    def step(events=None):
+        for l in range(L):
+            tq.tq_encode(kv_new[l], tq.TQ_F16, 1, H, d, w.bits_k, w.bits_v, seed,
+                         caches.pk[l], caches.pv[l], caches.nk[l], caches.nv[l], cap, ctx - 1,
+                         status, stream)
+            if events is not None:
+                events[l][0].record(stream)
+            tq.tq_attend(q[l], tq.TQ_F16, caches.pk[l], caches.nk[l], caches.pv[l], caches.nv[l],
+                         ctx_dev, 1, w.n_q_heads, w.gqa, d, w.bits_k, w.bits_v, seed, cap, 0.0, 0,
+                         ws, ws_bytes, outs[l], tq.TQ_F16, dev_status=status, stream=stream)
+            if events is not None:
+                events[l][1].record(stream)
+
+    kernels_per_step = L * 3   # encode + attend split-K + combine per layer
+
+    def capture(with_events):
+        evs = None
+        if with_events:
+            evs = [(torch.cuda.Event(enable_timing=True, external=True),
+                    torch.cuda.Event(enable_timing=True, external=True)) for _ in range(L)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(evs)
+        return g, evs
+
+    with torch.cuda.stream(stream):
+        step()                       # eager warm-up of the exact sequence
+    torch.cuda.synchronize()
+    warm_graph, _ = capture(False)
+    timed = [capture(True) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        warm_graph.replay()
+    torch.cuda.synchronize()
+
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[local_rank]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else local_rank
+    barrier(device)
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_index) as clk:
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            for g, _ in timed:
+                g.replay()
+            t1.record(stream)
+        torch.cuda.synchronize()
+    ms_total = t0.elapsed_time(t1)
+    ms_step = reduce_max(ms_total / args.steps, device)
+    attend_ms = [e[0].elapsed_time(e[1]) for _, evs in timed for e in evs]
+    attend_ms_mean = reduce_max(float(np.mean(attend_ms)), device)
+    launches += kernels_per_step * args.steps
+
+    # ---------------- end to end: host inputs in, host output back, every step
+    q_host = torch.empty((L, 1, w.n_q_heads, d), dtype=torch.float16).pin_memory()
+    kv_host = torch.empty((L, 2, 1, H, d), dtype=torch.int16).pin_memory()
+    out_host = torch.empty((L, 1, w.n_q_heads, d), dtype=torch.float16).pin_memory()
+    q_host.copy_(torch.stack([x.cpu() for x in q]))
+    kv_host.copy_(torch.stack([x.cpu() for x in kv_new]))
+    e2e_graph, _ = capture(False)
+    torch.cuda.synchronize()
+
+    def e2e_step():
+        for l in range(L):
+            q[l].copy_(q_host[l], non_blocking=True)
+            kv_new[l].copy_(kv_host[l], non_blocking=True)
+        e2e_graph.replay()
+        for l in range(L):
+            out_host[l].copy_(outs[l], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            e2e_step()
+    torch.cuda.synchronize()
+    barrier(device)
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        x0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        x1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(x0.elapsed_time(x1) / args.steps, device)
+    launches += kernels_per_step * args.steps
+    st = int(status.item())
+
+    per_layer_attend = attend_bytes(w, ctx)
+    per_layer_encode = encode_bytes(w, H)
+    step_bytes = L * (per_layer_attend + per_layer_encode)
+    peak, peak_kind = measured_peak()
+    achieved = per_layer_attend / (attend_ms_mean * 1e-3) / 1e9
+    enc_bytes = L * encode_bytes(we, ctx * H)
+    enc_gbs = enc_bytes / (enc_ms * 1e-3) / 1e9
+    traffic = recorded_traffic()
+    res = {
+        "metric": METRIC,
+        "value": round(world * step_bytes / (ms_step * 1e-3) / 1e9, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic (seeded N(0,1) fp16 K/V with x20 outlier K channels; torch generator on device)",
+        "config": {"workload": WORKLOAD, "layers": L, "batch": w.batch, "n_q_heads": w.n_q_heads,
+                   "n_kv_heads": H, "d": d, "ctx": ctx, "bits": f"K{w.bits_k}/V{w.bits_v}",
+                   "kv_dtype": "fp16", "q_out_dtype": "fp16", "per_gpu": "one model replica",
+                   "l2": f"inputs larger than L2: {L} distinct layer caches, "
+                         f"{L * per_layer_attend / 1e6:.0f} MB per step",
+                   "step": "per layer: tq_encode(1 new token) + tq_attend(ctx positions), CUDA graph"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                     "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+                     "kernel": "tq_attend (split-K + combine)",
+                     "bytes_per_launch": per_layer_attend,
+                     "launch_ms": round(attend_ms_mean, 5),
+                     "traffic": traffic["traffic_bytes_per_launch"] if traffic else None},
+        "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 4),
+                "h2d_bytes_per_step": int(q_host.numel() * 2 + kv_host.numel() * 2),
+                "d2h_bytes_per_step": int(out_host.numel() * 2)},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+        "encode": {"workload": ENCODE_WORKLOAD, "metric": "encode Mtok/s",
+                   "value": round(world * L * ctx / (enc_ms * 1e-3) / 1e6, 3), "unit": "Mtok/s",
+                   "token_head_vectors_per_s": round(world * L * ctx * H / (enc_ms * 1e-3), 0),
+                   "ms_per_step": round(enc_ms, 4), "steps": enc_steps,
+                   "roofline": {"bound": "hbm", "achieved": round(enc_gbs, 1), "peak": peak,
+                                "unit": "GB/s", "frac": round(enc_gbs / peak, 4),
+                                "frac_of_nominal_8tbs": round(enc_gbs / NOMINAL_HBM_GBS, 4),
+                                "bytes_per_step": enc_bytes},
+                   "gpu_launches": enc_launches},
+        "device_status": st,
+    }
+    for g, _ in timed:
+        del g
+    return res
+
+
+# ------------------------------------------------------------------ CPU oracle arm
+def oracle_sample(budget_s=12.0):
+    """Time the oracle on a bounded sample of the decode workload: whole
+    (kv head, query group) units of one layer at full context, plus a block of
+    encode vectors. Returns dict with GB/s and Mtok/s on the same byte basis."""
+    import threadpoolctl
+    from oracle import attention, codec
+    w = S.WORKLOADS[WORKLOAD]
+    cores = max(i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()) \
+        if threadpoolctl.threadpool_info() else 1
+    # inputs (not timed): one kv head's K/V at full context, encoded by the oracle
+    kv = S.kv_bits(w, 0, w.ctx)[:, :, :1]
+    x_k = codec.promote(kv[0, :, 0], w.dtype)
+    x_v = codec.promote(kv[1, :, 0], w.dtype)
+    t = time.perf_counter()
+    rk, nk = codec.encode_rows(x_k, w.bits_k, S.SIGN_SEED)
+    rv, nv = codec.encode_rows(x_v, w.bits_v, S.SIGN_SEED)
+    enc_s = time.perf_counter() - t
+    enc_vecs = 2 * w.ctx
+    qb = S.query_bits(w)[:, :w.gqa]
+    q64 = codec.promote(qb, w.dtype)
+    units, att_s = 0, 0.0
+    while att_s < budget_s and units < 64:
+        t = time.perf_counter()
+        attention.attend(q64, rk[None, None], nk[None, None], rv[None, None], nv[None, None],
+                         np.array([w.ctx]), w.gqa, w.bits_k, w.bits_v, S.SIGN_SEED)
+        att_s += time.perf_counter() - t
+        units += 1
+    unit_bytes = w.ctx * (w.d * w.bits_k // 8 + w.d * w.bits_v // 8 + 4) + w.gqa * w.d * 4
+    return {"attend_gbs": units * unit_bytes / att_s / 1e9, "attend_units": units,
+            "attend_s": att_s, "encode_mtoks": (enc_vecs / 2 / w.n_kv_heads) / enc_s / 1e6,
+            "encode_vectors_per_s": enc_vecs / enc_s, "cores": cores,
+            "sample": f"{units} x (1 kv head + its {w.gqa} query heads, ctx {w.ctx}) attention; "
+                      f"{enc_vecs} vector encodes"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    w = S.WORKLOADS[WORKLOAD]
+    per_step = []
+    o = None
+    for i in range(args.warmup + args.steps):
+        o = oracle_sample(budget_s=2.0)
+        if i >= args.warmup:
+            per_step.append(o)
+    gbs = float(np.mean([p["attend_gbs"] for p in per_step]))
+    step_bytes = LAYERS * (attend_bytes(w, w.ctx) + encode_bytes(w, w.n_kv_heads))
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(step_bytes / (gbs * 1e9) * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "layers": LAYERS, "batch": w.batch,
+                   "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "d": w.d,
+                   "ctx": w.ctx, "bits": f"K{w.bits_k}/V{w.bits_v}"},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": o["cores"],
+                         "kind": "oracle", "sample": "per step: " + o["sample"]},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--layers", type=int, default=LAYERS)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, world, local_rank = dist_env()
+    if args.gpus > 1 and world == 1:
+        ap.error("--gpus N > 1 runs under torch.distributed.run (one process per GPU)")
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+
+    init_dist(world, "nccl")
+    res = run_gpu(args, rank, world, local_rank)
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            o = oracle_sample()
+            res["cpu_baseline"] = {"value": round(o["attend_gbs"], 4), "unit": "GB/s",
+                                   "cores": o["cores"], "kind": "oracle", "sample": o["sample"],
+                                   "encode_mtoks": round(o["encode_mtoks"], 6)}
+        print(json.dumps(res), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,138 @@
+"""Python binding of the compressed decode-attention library (libtq.so).
+
+Thin ctypes marshalling around the C ABI declared in include/tq.h: every
+function here has the name of the C entry point it calls, accepts torch
+tensors (device buffers) or raw integer addresses for the pointer arguments,
+and raises TQError on a non-zero status. All computation runs in the CUDA
+kernels of libtq.so; there is no fallback — if the library is not built,
+importing any entry point raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtq.so")
+
+TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_CUDA, TQ_ERR_NO_CONVERGENCE = range(5)
+TQ_F16, TQ_BF16, TQ_F32 = 0, 1, 2
+TQ_DEV_CTX_CLAMPED, TQ_DEV_NORM_SATURATED, TQ_DEV_CTX_EMPTY = 1, 2, 4
+TQ_SPARSE_V_BLOCK = 64
+
+_lib = None
+
+
+class TQError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn} returned {status_string(status)} ({status})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libtq.so (built in-tree). Raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is not built; run "
+                              "`python -m compressed_decode_attention_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, U64, SZ, F, D = (ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64,
+                               ctypes.c_size_t, ctypes.c_float, ctypes.POINTER(ctypes.c_double))
+        L.tq_abi_version.restype = I
+        L.tq_abi_version.argtypes = []
+        L.tq_status_string.restype = ctypes.c_char_p
+        L.tq_status_string.argtypes = [I]
+        L.tq_build_codebook.restype = I
+        L.tq_build_codebook.argtypes = [I, I, D, D, D]
+        L.tq_encode.restype = I
+        L.tq_encode.argtypes = [P, I, I, I, I, I, I, U64, P, P, P, P, I, I, P, P]
+        L.tq_dequant.restype = I
+        L.tq_dequant.argtypes = [P, P, I, I, I, I, U64, I, I, P, P]
+        L.tq_attend_workspace_size.restype = SZ
+        L.tq_attend_workspace_size.argtypes = [I, I, I, I, I]
+        L.tq_attend.restype = I
+        L.tq_attend.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F, I,
+                                P, SZ, P, P, P, I, P]
+        _lib = L
+    return _lib
+
+
+def _ptr(x):
+    """Device address of a torch tensor, an int address, or None (NULL)."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(fn, st):
+    if st != TQ_OK:
+        raise TQError(fn, st)
+
+
+def tq_status_string(status: int) -> str:
+    return lib().tq_status_string(status).decode()
+
+
+status_string = tq_status_string
+
+
+def tq_abi_version() -> int:
+    return lib().tq_abi_version()
+
+
+def tq_build_codebook(bits: int, d: int):
+    """(centroids[2^bits], thresholds[2^bits-1], mse) of the N(0,1/d) codebook."""
+    n = 1 << bits
+    c = np.zeros(n, dtype=np.float64)
+    t = np.zeros(max(n - 1, 1), dtype=np.float64)
+    m = ctypes.c_double()
+    dp = ctypes.POINTER(ctypes.c_double)
+    _check("tq_build_codebook", lib().tq_build_codebook(
+        bits, d, c.ctypes.data_as(dp), t.ctypes.data_as(dp), ctypes.byref(m)))
+    return c, t[:n - 1], m.value
+
+
+def tq_encode(kv, dtype, n_tok, n_kv_heads, d, bits_k, bits_v, seed, packed_k,
+              packed_v, norms_k, norms_v, cap_tok, tok_offset, dev_status=None,
+              stream=None):
+    _check("tq_encode", lib().tq_encode(
+        _ptr(kv), dtype, n_tok, n_kv_heads, d, bits_k, bits_v, seed,
+        _ptr(packed_k), _ptr(packed_v), _ptr(norms_k), _ptr(norms_v), cap_tok,
+        tok_offset, _ptr(dev_status), _stream(stream)))
+
+
+def tq_dequant(packed, norms, n_tok, n_kv_heads, d, bits, seed, cap_tok, domain,
+               out, stream=None):
+    _check("tq_dequant", lib().tq_dequant(
+        _ptr(packed), _ptr(norms), n_tok, n_kv_heads, d, bits, seed, cap_tok,
+        domain, _ptr(out), _stream(stream)))
+
+
+def tq_attend_workspace_size(batch, n_q_heads, cap_tok, d, split_tokens=0) -> int:
+    return lib().tq_attend_workspace_size(batch, n_q_heads, cap_tok, d, split_tokens)
+
+
+def tq_attend(q, q_dtype, packed_k, norms_k, packed_v, norms_v, ctx_lens, batch,
+              n_q_heads, gqa_ratio, d, bits_k, bits_v, seed, cap_tok,
+              sparse_v_thresh, split_tokens, workspace, workspace_bytes, out,
+              out_dtype, dev_status=None, sparse_v_skipped=None, stream=None):
+    _check("tq_attend", lib().tq_attend(
+        _ptr(q), q_dtype, _ptr(packed_k), _ptr(norms_k), _ptr(packed_v),
+        _ptr(norms_v), _ptr(ctx_lens), batch, n_q_heads, gqa_ratio, d, bits_k,
+        bits_v, seed, cap_tok, float(sparse_v_thresh), split_tokens,
+        _ptr(workspace), workspace_bytes, _ptr(dev_status),
+        _ptr(sparse_v_skipped), _ptr(out), out_dtype, _stream(stream)))

@@ -1,0 +1,205 @@
+// C ABI entry points: argument validation on the host, then kernel launches
+// on the caller's stream. Declarations and contracts: include/tq.h.
+#include <math.h>
+#include <stdint.h>
+
+#include "tq.h"
+#include "tq_internal.h"
+
+using namespace tq;
+
+namespace {
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+int check_head_dim(int d) {
+  if (d <= 0 || (d & (d - 1))) return TQ_ERR_INVALID_ARG;
+  if (d < 64 || d > 256) return TQ_ERR_INVALID_ARG;
+  if (d != kHeadDim) return TQ_ERR_UNSUPPORTED;
+  return TQ_OK;
+}
+
+bool bits_ok(int b) { return b >= 2 && b <= 4; }
+
+constexpr int kMaxGridYZ = 65535;   // CUDA grid y/z limit (heads, batch)
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA; }
+
+}  // namespace
+
+namespace tq {
+
+int choose_split_tokens(int batch, int n_q_heads, int cap_tok, int requested) {
+  if (requested > 0) return requested;
+  (void)batch;
+  (void)n_q_heads;
+  // One gate block for tiny caches, else 512 tokens per split-K work item.
+  if (cap_tok <= kGateBlock) return kGateBlock;
+  return 512;
+}
+
+}  // namespace tq
+
+extern "C" {
+
+int tq_abi_version(void) { return TQ_ABI_VERSION; }
+
+const char* tq_status_string(int status) {
+  switch (status) {
+    case TQ_OK: return "TQ_OK";
+    case TQ_ERR_INVALID_ARG: return "TQ_ERR_INVALID_ARG";
+    case TQ_ERR_UNSUPPORTED: return "TQ_ERR_UNSUPPORTED";
+    case TQ_ERR_CUDA: return "TQ_ERR_CUDA";
+    case TQ_ERR_NO_CONVERGENCE: return "TQ_ERR_NO_CONVERGENCE";
+    default: return "unknown tq_status";
+  }
+}
+
+int tq_build_codebook(int bits, int d, double* centroids, double* thresholds,
+                      double* mse) {
+  if (bits < 1 || bits > 8 || d < 1 || !centroids || !thresholds)
+    return TQ_ERR_INVALID_ARG;
+  const int st = solve_lloyd_max(bits, centroids, thresholds, mse);
+  if (st != TQ_OK) return st;
+  const double s = 1.0 / sqrt((double)d);
+  for (int j = 0; j < (1 << bits); ++j) centroids[j] *= s;
+  for (int j = 0; j < (1 << bits) - 1; ++j) thresholds[j] *= s;
+  return TQ_OK;
+}
+
+int tq_encode(const void* kv, int dtype, int n_tok, int n_kv_heads, int d,
+              int bits_k, int bits_v, uint64_t seed, uint8_t* packed_k,
+              uint8_t* packed_v, uint16_t* norms_k, uint16_t* norms_v,
+              int cap_tok, int tok_offset, int* dev_status, void* stream) {
+  if (n_tok < 0 || n_kv_heads < 1 || cap_tok < 1 || tok_offset < 0)
+    return TQ_ERR_INVALID_ARG;
+  if ((long long)tok_offset + n_tok > cap_tok) return TQ_ERR_INVALID_ARG;
+  if (n_kv_heads > kMaxGridYZ) return TQ_ERR_UNSUPPORTED;
+  if (dtype != TQ_F16 && dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
+  if (!bits_ok(bits_k) || !bits_ok(bits_v)) return TQ_ERR_INVALID_ARG;
+  const int hd = check_head_dim(d);
+  if (hd != TQ_OK) return hd;
+  if (!kv || !packed_k || !packed_v || !norms_k || !norms_v) return TQ_ERR_INVALID_ARG;
+  if (!aligned16(kv) || !aligned16(packed_k) || !aligned16(packed_v))
+    return TQ_ERR_INVALID_ARG;
+  if (n_tok == 0) return TQ_OK;
+  const Codebook* cbk = codebook_for(bits_k);
+  const Codebook* cbv = codebook_for(bits_v);
+  if (!cbk || !cbv) return TQ_ERR_NO_CONVERGENCE;
+  EncodeArgs a;
+  a.kv = (const uint16_t*)kv;
+  a.is_bf16 = dtype == TQ_BF16;
+  a.n_tok = n_tok;
+  a.n_kv_heads = n_kv_heads;
+  a.bits_k = bits_k;
+  a.bits_v = bits_v;
+  a.packed_k = packed_k;
+  a.packed_v = packed_v;
+  a.norms_k = norms_k;
+  a.norms_v = norms_v;
+  a.cap_tok = cap_tok;
+  a.tok_offset = tok_offset;
+  a.dev_status = dev_status;
+  return from_cuda(launch_encode(a, *cbk, *cbv, sign_mask(seed), (cudaStream_t)stream));
+}
+
+int tq_dequant(const uint8_t* packed, const uint16_t* norms, int n_tok,
+               int n_kv_heads, int d, int bits, uint64_t seed, int cap_tok,
+               int domain, float* out, void* stream) {
+  if (n_tok < 0 || n_kv_heads < 1 || cap_tok < 1 || n_tok > cap_tok)
+    return TQ_ERR_INVALID_ARG;
+  if (n_kv_heads > kMaxGridYZ) return TQ_ERR_UNSUPPORTED;
+  if (bits < 2 || bits > 4 || (domain != 0 && domain != 1)) return TQ_ERR_INVALID_ARG;
+  const int hd = check_head_dim(d);
+  if (hd != TQ_OK) return hd;
+  if (!packed || !norms || !out) return TQ_ERR_INVALID_ARG;
+  if (!aligned16(packed) || !aligned16(out)) return TQ_ERR_INVALID_ARG;
+  if (n_tok == 0) return TQ_OK;
+  const Codebook* cb = codebook_for(bits);
+  if (!cb) return TQ_ERR_NO_CONVERGENCE;
+  DequantArgs a;
+  a.packed = packed;
+  a.norms = norms;
+  a.n_tok = n_tok;
+  a.n_kv_heads = n_kv_heads;
+  a.bits = bits;
+  a.cap_tok = cap_tok;
+  a.domain = domain;
+  a.out = out;
+  return from_cuda(launch_dequant(a, *cb, sign_mask(seed), (cudaStream_t)stream));
+}
+
+size_t tq_attend_workspace_size(int batch, int n_q_heads, int cap_tok, int d,
+                                int split_tokens) {
+  if (batch < 1 || n_q_heads < 1 || cap_tok < 1 || d != kHeadDim) return 0;
+  if (split_tokens < 0 || split_tokens % kGateBlock) return 0;
+  const int s = choose_split_tokens(batch, n_q_heads, cap_tok, split_tokens);
+  return attend_workspace_bytes(batch, n_q_heads, num_splits(cap_tok, s));
+}
+
+int tq_attend(const void* q, int q_dtype, const uint8_t* packed_k,
+              const uint16_t* norms_k, const uint8_t* packed_v,
+              const uint16_t* norms_v, const int32_t* ctx_lens, int batch,
+              int n_q_heads, int gqa_ratio, int d, int bits_k, int bits_v,
+              uint64_t seed, int cap_tok, float sparse_v_thresh,
+              int split_tokens, void* workspace, size_t workspace_bytes,
+              int* dev_status, unsigned long long* sparse_v_skipped, void* out,
+              int out_dtype, void* stream) {
+  if (batch < 1 || n_q_heads < 1 || gqa_ratio < 1 || cap_tok < 1)
+    return TQ_ERR_INVALID_ARG;
+  if (n_q_heads % gqa_ratio) return TQ_ERR_INVALID_ARG;
+  if (gqa_ratio > kMaxGroup) return TQ_ERR_UNSUPPORTED;
+  if (batch > kMaxGridYZ || n_q_heads / gqa_ratio > kMaxGridYZ) return TQ_ERR_UNSUPPORTED;
+  if (q_dtype < TQ_F16 || q_dtype > TQ_F32 || out_dtype < TQ_F16 || out_dtype > TQ_F32)
+    return TQ_ERR_INVALID_ARG;
+  if (!bits_ok(bits_k) || !bits_ok(bits_v)) return TQ_ERR_INVALID_ARG;
+  if (split_tokens < 0 || split_tokens % kGateBlock) return TQ_ERR_INVALID_ARG;
+  if (isnan(sparse_v_thresh)) return TQ_ERR_INVALID_ARG;
+  const int hd = check_head_dim(d);
+  if (hd != TQ_OK) return hd;
+  if (!q || !packed_k || !norms_k || !packed_v || !norms_v || !ctx_lens || !out ||
+      !workspace)
+    return TQ_ERR_INVALID_ARG;
+  if (!aligned16(packed_k) || !aligned16(packed_v) || !aligned16(workspace))
+    return TQ_ERR_INVALID_ARG;
+  const uintptr_t qa = q_dtype == TQ_F32 ? 3u : 1u, oa = out_dtype == TQ_F32 ? 3u : 1u;
+  if (((uintptr_t)q & qa) || ((uintptr_t)out & oa) || ((uintptr_t)ctx_lens & 3u) ||
+      ((uintptr_t)norms_k & 1u) || ((uintptr_t)norms_v & 1u) ||
+      ((uintptr_t)sparse_v_skipped & 7u) || ((uintptr_t)dev_status & 3u))
+    return TQ_ERR_INVALID_ARG;
+  const int split = choose_split_tokens(batch, n_q_heads, cap_tok, split_tokens);
+  const int ns = num_splits(cap_tok, split);
+  if (workspace_bytes < attend_workspace_bytes(batch, n_q_heads, ns))
+    return TQ_ERR_INVALID_ARG;
+  const Codebook* cbk = codebook_for(bits_k);
+  const Codebook* cbv = codebook_for(bits_v);
+  if (!cbk || !cbv) return TQ_ERR_NO_CONVERGENCE;
+  AttendArgs a;
+  a.q = q;
+  a.q_dtype = q_dtype;
+  a.packed_k = packed_k;
+  a.norms_k = norms_k;
+  a.packed_v = packed_v;
+  a.norms_v = norms_v;
+  a.ctx_lens = ctx_lens;
+  a.batch = batch;
+  a.n_q_heads = n_q_heads;
+  a.gqa = gqa_ratio;
+  a.n_kv_heads = n_q_heads / gqa_ratio;
+  a.bits_k = bits_k;
+  a.bits_v = bits_v;
+  a.cap_tok = cap_tok;
+  a.tau = sparse_v_thresh;
+  a.split_tokens = split;
+  a.n_splits = ns;
+  const size_t units = (size_t)batch * n_q_heads * ns;
+  a.part_acc = (float*)workspace;
+  a.part_ml = (float*)workspace + units * kHeadDim;
+  a.dev_status = dev_status;
+  a.skipped = sparse_v_skipped;
+  a.out = out;
+  a.out_dtype = out_dtype;
+  return from_cuda(launch_attend(a, *cbk, *cbv, sign_mask(seed), (cudaStream_t)stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,142 @@
+// tq_encode kernel: FP16 norm, randomized Hadamard rotation, Lloyd-Max
+// index, LSB-first bit-packing — one pass over each K/V head vector.
+//
+// [TQAI §The Paper]: keep the norm in FP16, rotate the unit vector,
+// quantize each coordinate with the precomputed Lloyd-Max codebook.
+// [ADAPTQ §How it works, item 1]: y = (1/sqrt d)·H·D·x applied with a fast
+// Walsh-Hadamard transform. [TQAI §What's Next]: indices bit-packed at
+// 2/3/4 bits.
+//
+// Thread layout: four lanes per vector, 32 consecutive coordinates per lane
+// (d = 128). A 256-thread block encodes 64 consecutive tokens of one kv head
+// (K or V), so its packed rows and norms form one contiguous range.
+//   load    4 x 16-byte loads per lane (the vector's 256 bytes, coalesced)
+//   norm    32 FMAs + 2 shuffles
+//   rotate  5 in-register butterfly stages + 2 cross-lane stages
+//   index   zeta = z/n compared as z against n·t (symmetric half table)
+//   pack    the lane's 32 indices are 4·bits contiguous bytes of the row
+#include "device_common.cuh"
+
+namespace tq {
+namespace {
+
+constexpr int kEncThreads = 256;
+constexpr int kEncTokens = kEncThreads / 4;
+
+template <int BITS>
+__device__ __forceinline__ void encode_vector(
+    float (&x)[32], const Codebook& cb, int sub, unsigned gmask,
+    uint8_t* row_dst, uint16_t* norm_dst, int* dev_status) {
+  constexpr int kHalf = 1 << (BITS - 1);
+  // ||x||^2 over the group of four lanes
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) ss = fmaf(x[i], x[i], ss);
+  ss += __shfl_xor_sync(gmask, ss, 1);
+  ss += __shfl_xor_sync(gmask, ss, 2);
+  const float n = sqrtf(ss);
+
+  // z = H·(D⊙x): coordinate 32·sub + i lives in register i of lane sub.
+  fwht_registers<32>(x);
+  fwht_cross_lane<32>(x, gmask, 1, (sub & 1) != 0);   // stride 32
+  fwht_cross_lane<32>(x, gmask, 2, (sub & 2) != 0);   // stride 64
+
+  // idx = #{j : z/n >= t_j}, evaluated as z against n·t_j. Positive half of
+  // the table: T_k = n·t_{half-1+k}, k = 1..half-1 (t_{half-1} = 0).
+  // z >= 0: idx = half + #{k : T_k <= z};  z < 0: idx = half-1 - #{k : T_k < |z|}.
+  // The strict comparison uses |z| lowered by one ulp. A zero vector keeps
+  // n = 0, z = 0 and must land on idx = half: scale the table by 1 instead.
+  const float sc = n > 0.f ? n : 1.f;
+  float T[kHalf > 1 ? kHalf - 1 : 1];
+#pragma unroll
+  for (int k = 1; k < kHalf; ++k) T[k - 1] = sc * cb.threshold[kHalf - 1 + k];
+
+  uint32_t words[BITS] = {};
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float z = x[i];
+    const bool neg = z < 0.f;
+    const float a = __uint_as_float((__float_as_uint(z) & 0x7FFFFFFFu) - (neg ? 1u : 0u));
+    int cnt = 0;
+#pragma unroll
+    for (int k = 0; k < kHalf - 1; ++k) cnt += (a >= T[k]) ? 1 : 0;
+    const uint32_t idx = neg ? (uint32_t)(kHalf - 1 - cnt) : (uint32_t)(kHalf + cnt);
+    const int p = i * BITS, w = p >> 5, off = p & 31;
+    words[w] |= idx << off;
+    if (off + BITS > 32) words[w + 1] |= idx >> (32 - off);
+  }
+
+  if constexpr (BITS == 4) {
+    *reinterpret_cast<uint4*>(row_dst + 16 * sub) =
+        make_uint4(words[0], words[1], words[2], words[3]);
+  } else if constexpr (BITS == 2) {
+    *reinterpret_cast<uint2*>(row_dst + 8 * sub) = make_uint2(words[0], words[1]);
+  } else {
+    uint32_t* d32 = reinterpret_cast<uint32_t*>(row_dst + 12 * sub);
+    d32[0] = words[0];
+    d32[1] = words[1];
+    d32[2] = words[2];
+  }
+  if (sub == 0) {
+    *norm_dst = f32_to_f16_bits(fminf(n, 65504.f));
+    if (n > 65504.f && dev_status) atomicOr(dev_status, TQ_DEV_NORM_SATURATED);
+  }
+}
+
+__global__ void __launch_bounds__(kEncThreads)
+encode_kernel(const __grid_constant__ EncodeArgs a,
+              const __grid_constant__ Codebook cbk,
+              const __grid_constant__ Codebook cbv,
+              const __grid_constant__ SignMask sm) {
+  const int is_v = blockIdx.z;
+  const int h = blockIdx.y;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane & 3;
+  const int tok = blockIdx.x * kEncTokens + (threadIdx.x >> 2);
+  if (tok >= a.n_tok) return;                       // whole groups of four
+  const unsigned gmask = 0xFu << (lane & ~3);
+
+  const uint16_t* src = a.kv +
+      ((size_t)(is_v * a.n_tok + tok) * a.n_kv_heads + h) * kHeadDim + 32 * sub;
+  uint4 raw[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) raw[k] = __ldcs(reinterpret_cast<const uint4*>(src) + k);
+  float x[32];
+  const uint32_t m = sm.w[sub];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t w4[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = unpack16x2(w4[j], a.is_bf16);
+      const int i = 8 * k + 2 * j;
+      x[i] = apply_sign(f.x, m, i);
+      x[i + 1] = apply_sign(f.y, m, i + 1);
+    }
+  }
+
+  const size_t row = (size_t)h * a.cap_tok + a.tok_offset + tok;
+  const int bits = is_v ? a.bits_v : a.bits_k;
+  const Codebook& cb = is_v ? cbv : cbk;
+  uint8_t* packed = is_v ? a.packed_v : a.packed_k;
+  uint16_t* norms = (is_v ? a.norms_v : a.norms_k) + row;
+  const size_t rb = (size_t)kHeadDim * bits / 8;
+  if (bits == 4)
+    encode_vector<4>(x, cb, sub, gmask, packed + row * rb, norms, a.dev_status);
+  else if (bits == 3)
+    encode_vector<3>(x, cb, sub, gmask, packed + row * rb, norms, a.dev_status);
+  else
+    encode_vector<2>(x, cb, sub, gmask, packed + row * rb, norms, a.dev_status);
+}
+
+}  // namespace
+
+cudaError_t launch_encode(const EncodeArgs& a, const Codebook& cbk,
+                          const Codebook& cbv, const SignMask& sm,
+                          cudaStream_t stream) {
+  dim3 grid((a.n_tok + kEncTokens - 1) / kEncTokens, a.n_kv_heads, 2);
+  encode_kernel<<<grid, kEncThreads, 0, stream>>>(a, cbk, cbv, sm);
+  return cudaGetLastError();
+}
+
+}  // namespace tq

@@ -1,0 +1,97 @@
+// Internal definitions shared by the host layer (api.cpp) and the kernels.
+// Not part of the public ABI (include/tq.h is).
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime.h>
+
+namespace tq {
+
+constexpr int kHeadDim = 128;          // d supported by this build
+constexpr int kMaxLevels = 16;         // 2^4: widest code on the hot path
+constexpr int kGateBlock = 64;         // sparse-V block (TQ_SPARSE_V_BLOCK)
+constexpr int kMaxGroup = 8;           // largest GQA group handled per CTA
+
+// Codebook in N(0,1) units, as float for the kernels.
+struct Codebook {
+  float centroid[kMaxLevels];          // 2^bits ascending levels
+  float threshold[kMaxLevels];         // 2^bits - 1 ascending thresholds
+  int bits;
+};
+
+// Sign vector D as a bit mask: bit i of word i/32 set <=> D_i = -1.
+struct SignMask {
+  uint32_t w[kHeadDim / 32];
+};
+
+// ---------------------------------------------------------------- host side
+// Lloyd-Max solver (codebook.cpp). Returns 0 on success, else a tq_status.
+int solve_lloyd_max(int bits, double* centroids, double* thresholds,
+                    double* mse);
+// Cached float codebook for bits in 1..4 (computed once, immutable after).
+const Codebook* codebook_for(int bits);
+SignMask sign_mask(uint64_t seed);
+
+// ---------------------------------------------------------------- launchers
+struct EncodeArgs {
+  const uint16_t* kv;        // [2][n_tok][n_kv_heads][d]
+  int is_bf16;
+  int n_tok, n_kv_heads;
+  int bits_k, bits_v;
+  uint8_t* packed_k;
+  uint8_t* packed_v;
+  uint16_t* norms_k;
+  uint16_t* norms_v;
+  int cap_tok, tok_offset;
+  int* dev_status;
+};
+cudaError_t launch_encode(const EncodeArgs& a, const Codebook& cbk,
+                          const Codebook& cbv, const SignMask& sm,
+                          cudaStream_t stream);
+
+struct DequantArgs {
+  const uint8_t* packed;
+  const uint16_t* norms;
+  int n_tok, n_kv_heads, bits, cap_tok, domain;
+  float* out;
+};
+cudaError_t launch_dequant(const DequantArgs& a, const Codebook& cb,
+                           const SignMask& sm, cudaStream_t stream);
+
+struct AttendArgs {
+  const void* q;
+  int q_dtype;
+  const uint8_t* packed_k;
+  const uint16_t* norms_k;
+  const uint8_t* packed_v;
+  const uint16_t* norms_v;
+  const int32_t* ctx_lens;
+  int batch, n_q_heads, gqa, n_kv_heads;
+  int bits_k, bits_v;
+  int cap_tok;
+  float tau;
+  int split_tokens, n_splits;
+  float* part_acc;           // [batch][n_q_heads][n_splits][d]
+  float* part_ml;            // [batch][n_q_heads][n_splits][2]
+  int* dev_status;
+  unsigned long long* skipped;
+  void* out;
+  int out_dtype;
+};
+cudaError_t launch_attend(const AttendArgs& a, const Codebook& cbk,
+                          const Codebook& cbv, const SignMask& sm,
+                          cudaStream_t stream);
+
+// Split-K geometry shared by tq_attend and tq_attend_workspace_size.
+int choose_split_tokens(int batch, int n_q_heads, int cap_tok, int requested);
+inline int num_splits(int cap_tok, int split_tokens) {
+  return (cap_tok + split_tokens - 1) / split_tokens;
+}
+inline size_t attend_workspace_bytes(int batch, int n_q_heads, int n_splits) {
+  const size_t units = (size_t)batch * n_q_heads * n_splits;
+  return units * kHeadDim * sizeof(float) + units * 2 * sizeof(float);
+}
+
+}  // namespace tq

@@ -159,7 +159,8 @@ int tq_encode(const void* kv, int dtype, int n_tok, int n_kv_heads, int d,
  *   domain      0: original space, x_hat = fp16norm · D⊙(H·c[idx]) / d;
  *               1: rotated unit-vector coordinates c[idx] / sqrt(d)
  *               (the N(0,1/d) codebook values, norm not applied).
- *   out         float [n_kv_heads][n_tok][d].
+ *   out         float [n_kv_heads][n_tok][d], 16-byte aligned.
+ * packed must be 16-byte aligned.
  */
 int tq_dequant(const uint8_t* packed, const uint16_t* norms, int n_tok,
                int n_kv_heads, int d, int bits, uint64_t seed, int cap_tok,

@@ -1,0 +1,227 @@
+"""Helpers for the GPU parity tests: oracle-built inputs and device buffers.
+
+Every expected value comes from the oracle on seeded synthetic inputs; the
+packed caches fed to the GPU attention are built by the oracle's encoder, so
+no oracle input ever comes from the CUDA path. The oracle work runs in a
+process pool started with 'spawn' (before any CUDA call in the workers).
+"""
+from __future__ import annotations
+
+import functools
+import multiprocessing as mp
+import os
+from concurrent.futures import ProcessPoolExecutor
+
+import numpy as np
+
+import synthetic as S
+
+_POOL = None
+
+
+def pool() -> ProcessPoolExecutor:
+    global _POOL
+    if _POOL is None:
+        n = max(1, min(32, (os.cpu_count() or 2) - 1))
+        _POOL = ProcessPoolExecutor(max_workers=n, mp_context=mp.get_context("spawn"),
+                                    initializer=_worker_init)
+    return _POOL
+
+
+def _worker_init():
+    os.environ["OPENBLAS_NUM_THREADS"] = "1"
+    os.environ["OMP_NUM_THREADS"] = "1"
+    try:
+        import threadpoolctl
+        threadpoolctl.threadpool_limits(1)
+    except Exception:
+        pass
+
+
+# ------------------------------------------------------------ oracle side
+def oracle_encode_heads(kv_bits: np.ndarray, dtype: str, which: int, bits: int,
+                        seed: int, chunk: int = 32768):
+    """Oracle encode of kv_bits[which] ([n][H][d] 16-bit patterns).
+
+    Returns idx uint8 [H][n][d], norm bits uint16 [H][n], margin float32
+    [H][n][d] (distance of zeta to the nearest threshold, N(0,1) units).
+    """
+    from oracle import codec
+    n, H, d = kv_bits.shape[1:]
+    idx = np.empty((H, n, d), np.uint8)
+    nb = np.empty((H, n), np.uint16)
+    mg = np.empty((H, n, d), np.float32)
+    for h in range(H):
+        for s in range(0, n, chunk):
+            x = codec.promote(kv_bits[which, s:s + chunk, h], dtype)
+            i, _, b, _, m = codec.encode(x, bits, seed)
+            idx[h, s:s + chunk] = i
+            nb[h, s:s + chunk] = b
+            mg[h, s:s + chunk] = m
+    return idx, nb, mg
+
+
+def _seq_cache(name: str, seq: int, n_tok: int, seed: int):
+    """Worker: oracle-encoded packed rows of one sequence (all kv heads)."""
+    from oracle import codec
+    w = S.WORKLOADS[name]
+    kv = S.kv_bits(w, seq, n_tok)
+    out = []
+    for which, bits in ((0, w.bits_k), (1, w.bits_v)):
+        idx, nb, _ = oracle_encode_heads(kv, w.dtype, which, bits, seed)
+        rows = np.stack([codec.pack(idx[h].astype(np.int64), bits) for h in range(w.n_kv_heads)])
+        out += [rows, nb]
+    return out
+
+
+@functools.lru_cache(maxsize=4)
+def oracle_cache(name: str, seed: int = S.SIGN_SEED):
+    """(packed_k, norms_k, packed_v, norms_v, ctx) for a workload, built by
+    the oracle from the workload's synthetic K/V ([B][H][cap][row] layout;
+    rows past each sequence's context are zero)."""
+    w = S.WORKLOADS[name]
+    ctx = S.ctx_lens(w)
+    B, H, cap, d = w.batch, w.n_kv_heads, w.cap_tok, w.d
+    pk = np.zeros((B, H, cap, d * w.bits_k // 8), np.uint8)
+    pv = np.zeros((B, H, cap, d * w.bits_v // 8), np.uint8)
+    nk = np.zeros((B, H, cap), np.uint16)
+    nv = np.zeros((B, H, cap), np.uint16)
+    futs = [pool().submit(_seq_cache, name, b, int(ctx[b]), seed) for b in range(B)]
+    for b, f in enumerate(futs):
+        rk, bk, rv, bv = f.result()
+        L = int(ctx[b])
+        pk[b, :, :L], nk[b, :, :L], pv[b, :, :L], nv[b, :, :L] = rk, bk, rv, bv
+    return pk, nk, pv, nv, ctx
+
+
+def _oracle_attend_part(q, pk, nk, pv, nv, ctx, gqa, bk, bv, seed, tau):
+    from oracle import attention
+    return attention.attend(q, pk, nk, pv, nv, ctx, gqa, bk, bv, seed, tau)
+
+
+def oracle_attend(q64, pk, nk, pv, nv, ctx, gqa, bk, bv, seed, tau=0.0):
+    """Oracle attention; each (batch, kv head) pair is one pool task that
+    receives only its own slice of the cache."""
+    B, H = pk.shape[:2]
+    out = np.zeros(q64.shape)
+    futs = []
+    for b in range(B):
+        L = int(min(max(int(ctx[b]), 0), pk.shape[2]))
+        for g in range(H):
+            hs = slice(g * gqa, (g + 1) * gqa)
+            futs.append((b, hs, pool().submit(
+                _oracle_attend_part, q64[b:b + 1, hs], pk[b:b + 1, g:g + 1, :L],
+                nk[b:b + 1, g:g + 1, :L], pv[b:b + 1, g:g + 1, :L], nv[b:b + 1, g:g + 1, :L],
+                np.array([L]), gqa, bk, bv, seed, tau)))
+    n_gated = 0
+    for b, hs, f in futs:
+        o, ng = f.result()
+        out[b, hs] = o[0]
+        n_gated += ng
+    return out, n_gated
+
+
+# ------------------------------------------------------------ device side
+def dev(a: np.ndarray):
+    """numpy -> CUDA tensor (16-bit patterns travel as int16)."""
+    import torch
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    return torch.from_numpy(a).cuda()
+
+
+def host(t) -> np.ndarray:
+    a = t.cpu().numpy()
+    return a.view(np.uint16) if a.dtype == np.int16 else a
+
+
+def gpu_encode(kv_bits, dtype, bits_k, bits_v, seed, cap=None, tok_offset=0,
+               fill=0, status=None):
+    """Run tq_encode on kv_bits [2][n][H][d]; returns host copies of the cache."""
+    import torch
+    import compressed_decode_attention_b200 as tq
+    _, n, H, d = kv_bits.shape
+    cap = cap or n + tok_offset
+    pk = torch.full((H, cap, d * bits_k // 8), fill, dtype=torch.uint8, device="cuda")
+    pv = torch.full((H, cap, d * bits_v // 8), fill, dtype=torch.uint8, device="cuda")
+    nk = torch.full((H, cap), fill, dtype=torch.int16, device="cuda")
+    nv = torch.full((H, cap), fill, dtype=torch.int16, device="cuda")
+    st = status if status is not None else torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq.tq_encode(dev(kv_bits), tq.TQ_F16 if dtype == "f16" else tq.TQ_BF16, n, H, d,
+                 bits_k, bits_v, seed, pk, pv, nk, nv, cap, tok_offset, st)
+    torch.cuda.synchronize()
+    return host(pk), host(nk), host(pv), host(nv), int(st.item())
+
+
+def gpu_attend(q_bits, q_dtype, pk, nk, pv, nv, ctx, gqa, bk, bv, seed, tau=0.0,
+               split=0, out_dtype=None, want_skipped=False):
+    """tq_attend on host arrays; returns (out float32/bits, status, skipped)."""
+    import torch
+    import compressed_decode_attention_b200 as tq
+    B, H, cap = pk.shape[:3]
+    Hq = q_bits.shape[1]
+    d = q_bits.shape[2]
+    out_dtype = tq.TQ_F32 if out_dtype is None else out_dtype
+    ws_bytes = tq.tq_attend_workspace_size(B, Hq, cap, d, split)
+    ws = torch.empty(ws_bytes // 4, dtype=torch.float32, device="cuda")
+    if out_dtype == tq.TQ_F32:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device="cuda")
+    else:
+        out = torch.empty((B, Hq, d), dtype=torch.int16, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sk = torch.zeros(1, dtype=torch.int64, device="cuda")
+    qt = dev(q_bits)
+    q_enum = {"f16": tq.TQ_F16, "bf16": tq.TQ_BF16, "f32": tq.TQ_F32}[q_dtype]
+    tq.tq_attend(qt, q_enum, dev(pk), dev(nk), dev(pv), dev(nv),
+                 dev(np.asarray(ctx, np.int32)), B, Hq, gqa, d, bk, bv, seed, cap, tau,
+                 split, ws, ws_bytes, out, out_dtype, dev_status=st, sparse_v_skipped=sk)
+    torch.cuda.synchronize()
+    return host(out), int(st.item()), int(sk.item())
+
+
+def _encode_slice(kv_slice, dtype, bits, seed):
+    """Worker: oracle encode of [n][d] 16-bit patterns."""
+    kv = kv_slice[None, :, None, :]
+    idx, nb, mg = oracle_encode_heads(np.stack([kv[0], kv[0]]), dtype, 0, bits, seed)
+    return idx[0], nb[0], mg[0]
+
+
+def oracle_encode_parallel(kv_bits, dtype, which, bits, seed, chunk=65536):
+    """oracle_encode_heads spread over the pool by (head, token chunk)."""
+    n, H, d = kv_bits.shape[1:]
+    idx = np.empty((H, n, d), np.uint8)
+    nb = np.empty((H, n), np.uint16)
+    mg = np.empty((H, n, d), np.float32)
+    futs = []
+    for h in range(H):
+        for s in range(0, n, chunk):
+            sl = np.ascontiguousarray(kv_bits[which, s:s + chunk, h])
+            futs.append((h, s, pool().submit(_encode_slice, sl, dtype, bits, seed)))
+    for h, s, f in futs:
+        i, b, m = f.result()
+        idx[h, s:s + len(b)], nb[h, s:s + len(b)], mg[h, s:s + len(b)] = i, b, m
+    return idx, nb, mg
+
+
+# Comparison rule for encoded indices: bit-exact except at coordinates whose
+# rotated value lies within this distance (N(0,1) units, i.e. 1e-5/sqrt(d) in
+# the N(0,1/d) units of the codebook) of a threshold; those must be at most
+# NEAR_FRACTION of all coordinates.
+NEAR_WINDOW = 1e-5
+NEAR_FRACTION = 1e-4
+
+
+def check_indices(idx_gpu, idx_oracle, margin):
+    near = margin < NEAR_WINDOW
+    bad = (idx_gpu != idx_oracle) & ~near
+    assert not bad.any(), f"{int(bad.sum())} index mismatches outside the boundary window"
+    assert near.sum() <= NEAR_FRACTION * near.size, (int(near.sum()), near.size)
+    return int((idx_gpu != idx_oracle).sum()), int(near.sum())
+
+
+def check_norms(nb_gpu, nb_oracle):
+    """Stored fp16 norms within one ulp (non-negative fp16 bit patterns are
+    ordered like the values they encode)."""
+    diff = np.abs(nb_gpu.astype(np.int64) - nb_oracle.astype(np.int64))
+    assert diff.max(initial=0) <= 1, int(diff.max())

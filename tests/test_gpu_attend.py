@@ -1,0 +1,165 @@
+"""GPU parity of tq_attend against the float64 oracle on the same packed
+cache (built by the oracle's encoder), B200.
+
+Bar: max |out_gpu - out_oracle| <= 2e-3 on float32 output; fp16/bf16 output
+equals the round-to-nearest-even of the float32 output within one ulp; the
+sparse-V skip count matches the oracle's except at positions whose gate value
+exp(s - M_blk) lies within GATE_WINDOW (relative) of tau.
+"""
+import numpy as np
+import pytest
+
+import synthetic as S
+from gpu_support import gpu_attend, oracle_attend, oracle_cache, pool
+from oracle import attention, codec
+
+pytestmark = pytest.mark.gpu
+SEED = S.SIGN_SEED
+ATOL = 2e-3
+# Relative band around tau inside which the kernel's float32 scores and the
+# oracle's float64 scores may decide the gate differently.
+GATE_WINDOW = 1e-3
+
+
+def _gate_values(q64, pk, nk, ctx, gqa, bk, seed):
+    vals = []
+    B, H = pk.shape[:2]
+    for b in range(B):
+        L = int(min(ctx[b], pk.shape[2]))
+        for g in range(H):
+            if L <= 0:
+                continue
+            idx = codec.unpack(pk[b, g, :L], bk, q64.shape[-1])
+            vals.append(attention.gate_values(q64[b, g * gqa:(g + 1) * gqa], idx, nk[b, g, :L], bk, seed).ravel())
+    return np.concatenate(vals)
+
+
+def _ambiguous(q64, pk, nk, ctx, gqa, bk, seed, tau):
+    gv = _gate_values(q64, pk, nk, ctx, gqa, bk, seed)
+    return int(np.sum(np.abs(gv / tau - 1.0) < GATE_WINDOW))
+
+
+def _run(name, scale=1.0, tau=None, split=0):
+    w = S.WORKLOADS[name]
+    pk, nk, pv, nv, ctx = oracle_cache(name)
+    qb = S.query_bits(w, scale=scale)
+    q64 = codec.promote(qb, w.dtype)
+    tau = w.tau if tau is None else tau
+    want, ng_o = oracle_attend(q64, pk, nk, pv, nv, ctx, w.gqa, w.bits_k, w.bits_v, SEED, tau)
+    got, st, ng_g = gpu_attend(qb, w.dtype, pk, nk, pv, nv, ctx, w.gqa, w.bits_k, w.bits_v,
+                               SEED, tau=tau, split=split)
+    return w, q64, (pk, nk, pv, nv, ctx), want, got, st, ng_o, ng_g, tau
+
+
+@pytest.mark.parametrize("name", ["single_head_1k", "llama3_8b_decode", "qwen14b_decode",
+                                  "batched_serving"])
+def test_attend_full_workload(name):
+    w, q64, cache, want, got, st, ng_o, ng_g, tau = _run(name)
+    err = np.abs(got - want).max()
+    print(f"{name}: max|err| = {err:.3e}, gated oracle {ng_o} gpu {ng_g}")
+    assert err <= ATOL
+    assert st == 0
+    if tau > 0:
+        amb = _ambiguous(q64, cache[0], cache[1], cache[4], w.gqa, w.bits_k, SEED, tau)
+        assert abs(ng_g - ng_o) <= amb
+
+
+def test_forced_gate_batched_serving():
+    """Queries scaled x8 sharpen the softmax so the 1e-6 gate fires often."""
+    w, q64, cache, want, got, st, ng_o, ng_g, tau = _run("batched_serving", scale=8.0)
+    assert ng_o > 1000
+    amb = _ambiguous(q64, cache[0], cache[1], cache[4], w.gqa, w.bits_k, SEED, tau)
+    print(f"forced gate: oracle {ng_o}, gpu {ng_g}, ambiguous {amb}")
+    assert abs(ng_g - ng_o) <= amb
+    assert np.abs(got - want).max() <= ATOL
+
+
+@pytest.mark.parametrize("tau", [1e-2, 0.5, 1.0, 2.0])
+def test_gate_thresholds_single_head(tau):
+    w, q64, cache, want, got, st, ng_o, ng_g, tau = _run("single_head_1k", scale=3.0, tau=tau)
+    amb = _ambiguous(q64, cache[0], cache[1], cache[4], w.gqa, w.bits_k, SEED, tau)
+    assert abs(ng_g - ng_o) <= amb
+    assert np.abs(got - want).max() <= ATOL
+    if tau > 1:
+        assert ng_g == 1024 and np.all(got == 0)
+
+
+@pytest.mark.parametrize("split", [64, 128, 448, 1024])
+def test_split_sizes(split):
+    _, _, _, want, got, _, _, _, _ = _run("single_head_1k", split=split)
+    assert np.abs(got - want).max() <= ATOL
+
+
+def _small_cache(bk, bv, B, Hkv, cap, ctx, seed, rng, dtype="f16"):
+    pk = np.zeros((B, Hkv, cap, 128 * bk // 8), np.uint8)
+    pv = np.zeros((B, Hkv, cap, 128 * bv // 8), np.uint8)
+    nk = np.zeros((B, Hkv, cap), np.uint16)
+    nv = np.zeros((B, Hkv, cap), np.uint16)
+    for b in range(B):
+        for g in range(Hkv):
+            L = int(min(max(ctx[b], 0), cap))
+            k = rng.standard_normal((L, 128)) * 2
+            v = rng.standard_normal((L, 128))
+            kx = codec.promote(S.to_bits(k, dtype), dtype)
+            vx = codec.promote(S.to_bits(v, dtype), dtype)
+            pk[b, g, :L], nk[b, g, :L] = codec.encode_rows(kx, bk, seed)
+            pv[b, g, :L], nv[b, g, :L] = codec.encode_rows(vx, bv, seed)
+    return pk, nk, pv, nv
+
+
+@pytest.mark.parametrize("bk,bv,gqa", [(2, 2, 1), (3, 3, 8), (4, 4, 2), (2, 4, 3),
+                                       (3, 4, 6), (2, 3, 7), (4, 2, 5), (3, 2, 4), (4, 3, 1)])
+def test_bit_widths_and_group_sizes(bk, bv, gqa):
+    rng = np.random.default_rng(bk * 100 + bv * 10 + gqa)
+    ctx = np.array([300, 77])
+    pk, nk, pv, nv = _small_cache(bk, bv, 2, 2, 320, ctx, 99, rng)
+    qb = S.f16_bits(rng.standard_normal((2, 2 * gqa, 128)))
+    q64 = codec.promote(qb, "f16")
+    want, _ = oracle_attend(q64, pk, nk, pv, nv, ctx, gqa, bk, bv, 99)
+    got, st, _ = gpu_attend(qb, "f16", pk, nk, pv, nv, ctx, gqa, bk, bv, 99)
+    assert np.abs(got - want).max() <= ATOL
+
+
+def test_context_edge_cases_and_status():
+    rng = np.random.default_rng(8)
+    cap = 256
+    ctx = np.array([1, 0, 65, 5000, -4, 256, 64, 129])
+    pk, nk, pv, nv = _small_cache(4, 2, len(ctx), 1, cap, ctx, 3, rng)
+    qb = S.f16_bits(rng.standard_normal((len(ctx), 2, 128)))
+    q64 = codec.promote(qb, "f16")
+    want, _ = oracle_attend(q64, pk, nk, pv, nv, ctx, 2, 4, 2, 3)
+    got, st, _ = gpu_attend(qb, "f16", pk, nk, pv, nv, ctx, 2, 4, 2, 3)
+    assert np.abs(got - want).max() <= ATOL
+    assert np.all(got[1] == 0) and np.all(got[4] == 0)
+    assert st == (1 | 4)   # clamped and empty
+    # context of one position returns that position's value
+    v0 = codec.dequant(codec.unpack(pv[0, 0, :1], 2, 128), nv[0, 0, :1], 2, 3)[0]
+    np.testing.assert_allclose(got[0, 0], v0, atol=ATOL)
+
+
+@pytest.mark.parametrize("q_dtype", ["f16", "bf16", "f32"])
+def test_query_dtypes(q_dtype):
+    rng = np.random.default_rng(12)
+    ctx = np.array([200])
+    pk, nk, pv, nv = _small_cache(4, 2, 1, 2, 200, ctx, 5, rng)
+    qf = rng.standard_normal((1, 8, 128)).astype(np.float32)
+    if q_dtype == "f32":
+        qb, q64 = qf, qf.astype(np.float64)
+    else:
+        qb = S.to_bits(qf, q_dtype)
+        q64 = codec.promote(qb, q_dtype)
+    want, _ = oracle_attend(q64, pk, nk, pv, nv, ctx, 4, 4, 2, 5)
+    got, _, _ = gpu_attend(qb, q_dtype, pk, nk, pv, nv, ctx, 4, 4, 2, 5)
+    assert np.abs(got - want).max() <= ATOL
+
+
+@pytest.mark.parametrize("out_dtype", [0, 1])
+def test_output_dtypes_round_float32_result(out_dtype):
+    import torch
+    w = S.WORKLOADS["single_head_1k"]
+    pk, nk, pv, nv, ctx = oracle_cache("single_head_1k")
+    qb = S.query_bits(w)
+    f32, _, _ = gpu_attend(qb, "f16", pk, nk, pv, nv, ctx, 1, 4, 2, SEED)
+    lo, _, _ = gpu_attend(qb, "f16", pk, nk, pv, nv, ctx, 1, 4, 2, SEED, out_dtype=out_dtype)
+    ref = S.f16_bits(f32) if out_dtype == 0 else S.bf16_bits(f32)
+    assert np.abs(lo.astype(np.int64) - ref.astype(np.int64)).max() <= 1

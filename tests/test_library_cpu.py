@@ -1,0 +1,131 @@
+"""Host-side checks of libtq.so that need no GPU: it loads, exports every
+entry point include/tq.h declares, its Lloyd-Max solver agrees with the
+oracle's (two independent implementations), and bad arguments are rejected
+on the host before any CUDA call."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import compressed_decode_attention_b200 as tq
+from oracle import codebook as ocb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(tq_\w+)\s*\(", src))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared_functions()
+    assert {"tq_build_codebook", "tq_encode", "tq_dequant", "tq_attend",
+            "tq_attend_workspace_size"} <= set(names)
+    lib = ctypes.CDLL(tq.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+        assert hasattr(tq, n), f"binding lacks {n}"
+
+
+def test_abi_version_and_status_strings():
+    assert tq.tq_abi_version() == 1
+    assert tq.status_string(0) == "TQ_OK"
+    assert tq.status_string(2) == "TQ_ERR_UNSUPPORTED"
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5])
+@pytest.mark.parametrize("d", [1, 64, 128])
+def test_host_codebook_matches_oracle(bits, d):
+    c, t, mse = tq.tq_build_codebook(bits, d)
+    oc, ot = ocb.lloyd_max_normal(bits)
+    np.testing.assert_allclose(c * np.sqrt(d), oc, atol=1e-12)
+    np.testing.assert_allclose(t * np.sqrt(d), ot, atol=1e-12)
+    assert mse == pytest.approx(ocb.quantizer_mse(oc, ot), abs=1e-12)
+
+
+def test_codebook_rejects_bad_arguments():
+    for bits, d in [(0, 128), (9, 128), (4, 0)]:
+        with pytest.raises(tq.TQError) as e:
+            tq.tq_build_codebook(bits, d)
+        assert e.value.status == tq.TQ_ERR_INVALID_ARG
+
+
+FAKE = 1 << 20  # 16-byte aligned dummy address; never dereferenced
+
+
+def _encode(**kw):
+    args = dict(kv=FAKE, dtype=tq.TQ_F16, n_tok=4, n_kv_heads=2, d=128, bits_k=4,
+                bits_v=2, seed=0, packed_k=FAKE, packed_v=FAKE, norms_k=FAKE,
+                norms_v=FAKE, cap_tok=8, tok_offset=0, dev_status=None, stream=0)
+    args.update(kw)
+    return tq.lib().tq_encode(args["kv"], args["dtype"], args["n_tok"], args["n_kv_heads"],
+                              args["d"], args["bits_k"], args["bits_v"], args["seed"],
+                              args["packed_k"], args["packed_v"], args["norms_k"],
+                              args["norms_v"], args["cap_tok"], args["tok_offset"],
+                              args["dev_status"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(kv=None), tq.TQ_ERR_INVALID_ARG),
+    (dict(packed_v=None), tq.TQ_ERR_INVALID_ARG),
+    (dict(kv=FAKE + 2), tq.TQ_ERR_INVALID_ARG),           # misaligned
+    (dict(bits_k=5), tq.TQ_ERR_INVALID_ARG),
+    (dict(bits_v=1), tq.TQ_ERR_INVALID_ARG),
+    (dict(d=96), tq.TQ_ERR_INVALID_ARG),                  # not a power of two
+    (dict(d=64), tq.TQ_ERR_UNSUPPORTED),
+    (dict(d=256), tq.TQ_ERR_UNSUPPORTED),
+    (dict(dtype=tq.TQ_F32), tq.TQ_ERR_INVALID_ARG),
+    (dict(tok_offset=5), tq.TQ_ERR_INVALID_ARG),          # 5 + 4 > 8
+    (dict(n_tok=-1), tq.TQ_ERR_INVALID_ARG),
+    (dict(n_kv_heads=0), tq.TQ_ERR_INVALID_ARG),
+    (dict(n_tok=0), tq.TQ_OK),                            # no-op, no launch
+])
+def test_encode_validation(kw, want):
+    assert _encode(**kw) == want
+
+
+def _attend(**kw):
+    a = dict(q=FAKE, q_dtype=tq.TQ_F16, pk=FAKE, nk=FAKE, pv=FAKE, nv=FAKE, ctx=FAKE,
+             batch=2, hq=8, gqa=4, d=128, bk=4, bv=2, seed=0, cap=256, tau=0.0,
+             split=0, ws=FAKE, wsb=1 << 30, status=None, skipped=None, out=FAKE,
+             out_dtype=tq.TQ_F32, stream=0)
+    a.update(kw)
+    return tq.lib().tq_attend(a["q"], a["q_dtype"], a["pk"], a["nk"], a["pv"], a["nv"],
+                              a["ctx"], a["batch"], a["hq"], a["gqa"], a["d"], a["bk"],
+                              a["bv"], a["seed"], a["cap"], a["tau"], a["split"], a["ws"],
+                              a["wsb"], a["status"], a["skipped"], a["out"], a["out_dtype"],
+                              a["stream"])
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(q=None), tq.TQ_ERR_INVALID_ARG),
+    (dict(ws=None), tq.TQ_ERR_INVALID_ARG),
+    (dict(gqa=3), tq.TQ_ERR_INVALID_ARG),                 # 8 % 3 != 0
+    (dict(hq=16, gqa=16), tq.TQ_ERR_UNSUPPORTED),         # group wider than 8
+    (dict(split=100), tq.TQ_ERR_INVALID_ARG),             # not a multiple of 64
+    (dict(wsb=16), tq.TQ_ERR_INVALID_ARG),                # workspace too small
+    (dict(bk=1), tq.TQ_ERR_INVALID_ARG),
+    (dict(d=64), tq.TQ_ERR_UNSUPPORTED),
+    (dict(tau=float("nan")), tq.TQ_ERR_INVALID_ARG),
+    (dict(out_dtype=7), tq.TQ_ERR_INVALID_ARG),
+    (dict(batch=0), tq.TQ_ERR_INVALID_ARG),
+    (dict(pk=FAKE + 8), tq.TQ_ERR_INVALID_ARG),
+])
+def test_attend_validation(kw, want):
+    assert _attend(**kw) == want
+
+
+def test_workspace_size_formula():
+    # (batch · heads · splits) units of d + 2 floats; 512-token splits by default
+    assert tq.tq_attend_workspace_size(1, 32, 32768, 128) == 32 * 64 * 130 * 4
+    assert tq.tq_attend_workspace_size(2, 4, 1000, 128, 256) == 2 * 4 * 4 * 130 * 4
+    assert tq.tq_attend_workspace_size(1, 1, 10, 128) == 130 * 4
+    assert tq.tq_attend_workspace_size(1, 1, 10, 128, 100) == 0
