@@ -257,8 +257,8 @@ def run_gpu(args, rank, world, local_rank):
     kv_new = [device_kv(w, l, 1, gen) for l in range(L)]
     outs = [torch.empty((1, w.n_q_heads, d), dtype=torch.float16, device=device) for _ in range(L)]
     ctx_dev = torch.full((1,), ctx, dtype=torch.int32, device=device)
-    ws_bytes = tq.tq_attend_workspace_size(1, w.n_q_heads, cap, d, 0)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
+    ws_bytes = tq.tq_attend_workspace_size(1, w.n_q_heads, cap, d)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=device)
 
     def step(events=None):
         for l in range(L):
@@ -273,7 +273,7 @@ def run_gpu(args, rank, world, local_rank):
             if events is not None:
                 events[l][1].record(stream)
 
-    kernels_per_step = L * 3   # encode + attend split-K + combine per layer
+    kernels_per_step = L * 2   # encode + attend per layer
 
     def capture(with_events):
         evs = None
@@ -377,7 +377,7 @@ def run_gpu(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                      "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
-                     "kernel": "tq_attend (split-K + combine)",
+                     "kernel": "tq_attend (attend_kernel, one launch)",
                      "bytes_per_launch": per_layer_attend,
                      "launch_ms": round(attend_ms_mean, 5),
                      "traffic": traffic["traffic_bytes_per_launch"] if traffic else None},

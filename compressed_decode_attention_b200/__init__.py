@@ -52,7 +52,7 @@ def lib() -> ctypes.CDLL:
         L.tq_dequant.restype = I
         L.tq_dequant.argtypes = [P, P, I, I, I, I, U64, I, I, P, P]
         L.tq_attend_workspace_size.restype = SZ
-        L.tq_attend_workspace_size.argtypes = [I, I, I, I, I]
+        L.tq_attend_workspace_size.argtypes = [I, I, I, I]
         L.tq_attend.restype = I
         L.tq_attend.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F, I,
                                 P, SZ, P, P, P, I, P]
@@ -122,17 +122,19 @@ def tq_dequant(packed, norms, n_tok, n_kv_heads, d, bits, seed, cap_tok, domain,
         domain, _ptr(out), _stream(stream)))
 
 
-def tq_attend_workspace_size(batch, n_q_heads, cap_tok, d, split_tokens=0) -> int:
-    return lib().tq_attend_workspace_size(batch, n_q_heads, cap_tok, d, split_tokens)
+def tq_attend_workspace_size(batch, n_q_heads, cap_tok, d) -> int:
+    return lib().tq_attend_workspace_size(batch, n_q_heads, cap_tok, d)
 
 
 def tq_attend(q, q_dtype, packed_k, norms_k, packed_v, norms_v, ctx_lens, batch,
               n_q_heads, gqa_ratio, d, bits_k, bits_v, seed, cap_tok,
-              sparse_v_thresh, split_tokens, workspace, workspace_bytes, out,
+              sparse_v_thresh, n_ctas, workspace, workspace_bytes, out,
               out_dtype, dev_status=None, sparse_v_skipped=None, stream=None):
+    """Decode attention. The workspace's counter region must be zero before
+    its first use (allocate it with torch.zeros); calls keep it zero."""
     _check("tq_attend", lib().tq_attend(
         _ptr(q), q_dtype, _ptr(packed_k), _ptr(norms_k), _ptr(packed_v),
         _ptr(norms_v), _ptr(ctx_lens), batch, n_q_heads, gqa_ratio, d, bits_k,
-        bits_v, seed, cap_tok, float(sparse_v_thresh), split_tokens,
+        bits_v, seed, cap_tok, float(sparse_v_thresh), n_ctas,
         _ptr(workspace), workspace_bytes, _ptr(dev_status),
         _ptr(sparse_v_skipped), _ptr(out), out_dtype, _stream(stream)))

@@ -27,18 +27,6 @@ int from_cuda(cudaError_t e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA; }
 
 }  // namespace
 
-namespace tq {
-
-int choose_split_tokens(int batch, int n_q_heads, int cap_tok, int requested) {
-  if (requested > 0) return requested;
-  (void)batch;
-  (void)n_q_heads;
-  // One gate block for tiny caches, else 512 tokens per split-K work item.
-  if (cap_tok <= kGateBlock) return kGateBlock;
-  return 512;
-}
-
-}  // namespace tq
 
 extern "C" {
 
@@ -129,48 +117,40 @@ int tq_dequant(const uint8_t* packed, const uint16_t* norms, int n_tok,
   return from_cuda(launch_dequant(a, *cb, sign_mask(seed), (cudaStream_t)stream));
 }
 
-size_t tq_attend_workspace_size(int batch, int n_q_heads, int cap_tok, int d,
-                                int split_tokens) {
+size_t tq_attend_workspace_size(int batch, int n_q_heads, int cap_tok, int d) {
   if (batch < 1 || n_q_heads < 1 || cap_tok < 1 || d != kHeadDim) return 0;
-  if (split_tokens < 0 || split_tokens % kGateBlock) return 0;
-  const int s = choose_split_tokens(batch, n_q_heads, cap_tok, split_tokens);
-  return attend_workspace_bytes(batch, n_q_heads, num_splits(cap_tok, s));
+  return attend_workspace_bytes(batch, n_q_heads);
 }
 
 int tq_attend(const void* q, int q_dtype, const uint8_t* packed_k,
               const uint16_t* norms_k, const uint8_t* packed_v,
               const uint16_t* norms_v, const int32_t* ctx_lens, int batch,
               int n_q_heads, int gqa_ratio, int d, int bits_k, int bits_v,
-              uint64_t seed, int cap_tok, float sparse_v_thresh,
-              int split_tokens, void* workspace, size_t workspace_bytes,
-              int* dev_status, unsigned long long* sparse_v_skipped, void* out,
-              int out_dtype, void* stream) {
+              uint64_t seed, int cap_tok, float sparse_v_thresh, int n_ctas,
+              void* workspace, size_t workspace_bytes, int* dev_status,
+              unsigned long long* sparse_v_skipped, void* out, int out_dtype,
+              void* stream) {
   if (batch < 1 || n_q_heads < 1 || gqa_ratio < 1 || cap_tok < 1)
     return TQ_ERR_INVALID_ARG;
   if (n_q_heads % gqa_ratio) return TQ_ERR_INVALID_ARG;
   if (gqa_ratio > kMaxGroup) return TQ_ERR_UNSUPPORTED;
-  if (batch > kMaxGridYZ || n_q_heads / gqa_ratio > kMaxGridYZ) return TQ_ERR_UNSUPPORTED;
   if (q_dtype < TQ_F16 || q_dtype > TQ_F32 || out_dtype < TQ_F16 || out_dtype > TQ_F32)
     return TQ_ERR_INVALID_ARG;
   if (!bits_ok(bits_k) || !bits_ok(bits_v)) return TQ_ERR_INVALID_ARG;
-  if (split_tokens < 0 || split_tokens % kGateBlock) return TQ_ERR_INVALID_ARG;
+  if (n_ctas < 0 || n_ctas > kMaxCtas) return TQ_ERR_INVALID_ARG;
   if (isnan(sparse_v_thresh)) return TQ_ERR_INVALID_ARG;
   const int hd = check_head_dim(d);
   if (hd != TQ_OK) return hd;
+  if (cap_tok % 8) return TQ_ERR_UNSUPPORTED;
   if (!q || !packed_k || !norms_k || !packed_v || !norms_v || !ctx_lens || !out ||
       !workspace)
     return TQ_ERR_INVALID_ARG;
-  if (!aligned16(packed_k) || !aligned16(packed_v) || !aligned16(workspace))
+  if (!aligned16(q) || !aligned16(out) || !aligned16(packed_k) || !aligned16(packed_v) ||
+      !aligned16(norms_k) || !aligned16(norms_v) || !aligned16(workspace) ||
+      ((uintptr_t)ctx_lens & 3u) || ((uintptr_t)sparse_v_skipped & 7u) ||
+      ((uintptr_t)dev_status & 3u))
     return TQ_ERR_INVALID_ARG;
-  const uintptr_t qa = q_dtype == TQ_F32 ? 3u : 1u, oa = out_dtype == TQ_F32 ? 3u : 1u;
-  if (((uintptr_t)q & qa) || ((uintptr_t)out & oa) || ((uintptr_t)ctx_lens & 3u) ||
-      ((uintptr_t)norms_k & 1u) || ((uintptr_t)norms_v & 1u) ||
-      ((uintptr_t)sparse_v_skipped & 7u) || ((uintptr_t)dev_status & 3u))
-    return TQ_ERR_INVALID_ARG;
-  const int split = choose_split_tokens(batch, n_q_heads, cap_tok, split_tokens);
-  const int ns = num_splits(cap_tok, split);
-  if (workspace_bytes < attend_workspace_bytes(batch, n_q_heads, ns))
-    return TQ_ERR_INVALID_ARG;
+  if (workspace_bytes < attend_workspace_bytes(batch, n_q_heads)) return TQ_ERR_INVALID_ARG;
   const Codebook* cbk = codebook_for(bits_k);
   const Codebook* cbv = codebook_for(bits_v);
   if (!cbk || !cbv) return TQ_ERR_NO_CONVERGENCE;
@@ -190,16 +170,14 @@ int tq_attend(const void* q, int q_dtype, const uint8_t* packed_k,
   a.bits_v = bits_v;
   a.cap_tok = cap_tok;
   a.tau = sparse_v_thresh;
-  a.split_tokens = split;
-  a.n_splits = ns;
-  const size_t units = (size_t)batch * n_q_heads * ns;
-  a.part_acc = (float*)workspace;
-  a.part_ml = (float*)workspace + units * kHeadDim;
+  a.counters = (int*)workspace;
+  a.slots = (float*)((uint8_t*)workspace + attend_counter_bytes(batch, n_q_heads));
   a.dev_status = dev_status;
   a.skipped = sparse_v_skipped;
   a.out = out;
   a.out_dtype = out_dtype;
-  return from_cuda(launch_attend(a, *cbk, *cbv, sign_mask(seed), (cudaStream_t)stream));
+  return from_cuda(launch_attend(a, *cbk, *cbv, sign_mask(seed), n_ctas,
+                                 (cudaStream_t)stream));
 }
 
 }  // extern "C"

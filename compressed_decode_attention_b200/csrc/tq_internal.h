@@ -72,26 +72,28 @@ struct AttendArgs {
   int bits_k, bits_v;
   int cap_tok;
   float tau;
-  int split_tokens, n_splits;
-  float* part_acc;           // [batch][n_q_heads][n_splits][d]
-  float* part_ml;            // [batch][n_q_heads][n_splits][2]
+  int* counters;             // [batch * n_kv_heads], zero between calls
+  float* slots;              // partial (acc[gqa][d], m/l[gqa][2]) per slot
   int* dev_status;
   unsigned long long* skipped;
   void* out;
   int out_dtype;
 };
 cudaError_t launch_attend(const AttendArgs& a, const Codebook& cbk,
-                          const Codebook& cbv, const SignMask& sm,
+                          const Codebook& cbv, const SignMask& sm, int n_ctas,
                           cudaStream_t stream);
 
-// Split-K geometry shared by tq_attend and tq_attend_workspace_size.
-int choose_split_tokens(int batch, int n_q_heads, int cap_tok, int requested);
-inline int num_splits(int cap_tok, int split_tokens) {
-  return (cap_tok + split_tokens - 1) / split_tokens;
+// Workspace of tq_attend: a counter region (zero on first use; every call
+// leaves it zero) followed by partial-result slots. Sized for up to
+// kMaxCtas CTAs, independent of the device.
+constexpr int kMaxCtas = 1024;
+constexpr int kSlotFloats = kHeadDim + 2;   // per query head
+inline size_t attend_counter_bytes(int batch, int n_q_heads) {
+  return ((size_t)batch * n_q_heads * sizeof(int) + 255) & ~(size_t)255;
 }
-inline size_t attend_workspace_bytes(int batch, int n_q_heads, int n_splits) {
-  const size_t units = (size_t)batch * n_q_heads * n_splits;
-  return units * kHeadDim * sizeof(float) + units * 2 * sizeof(float);
+inline size_t attend_workspace_bytes(int batch, int n_q_heads) {
+  const size_t slots = (size_t)kMaxCtas * kMaxGroup + (size_t)batch * n_q_heads;
+  return attend_counter_bytes(batch, n_q_heads) + slots * kSlotFloats * sizeof(float);
 }
 
 }  // namespace tq

@@ -167,12 +167,13 @@ int tq_dequant(const uint8_t* packed, const uint16_t* norms, int n_tok,
                int domain, float* out, void* stream);
 
 /*
- * tq_attend_workspace_size — bytes of scratch tq_attend needs for these
- * sizes and this split_tokens argument (0 = the library's choice). The
- * split-K partials are (m, l, acc[d]) in fp32 per (batch, query head, split).
+ * tq_attend_workspace_size — bytes of device scratch tq_attend needs for
+ * this batch and head count: a counter region of
+ * round_up(4·batch·n_q_heads, 256) bytes, then per-split partial results
+ * (running max, sum and d accumulators in fp32 per query head) for up to 1024
+ * CTAs. Returns 0 for invalid arguments.
  */
-size_t tq_attend_workspace_size(int batch, int n_q_heads, int cap_tok, int d,
-                                int split_tokens);
+size_t tq_attend_workspace_size(int batch, int n_q_heads, int cap_tok, int d);
 
 /*
  * tq_attend — single-query decode attention over the packed cache
@@ -191,29 +192,37 @@ size_t tq_attend_workspace_size(int batch, int n_q_heads, int cap_tok, int d,
  *   out  = D⊙(H·(acc / l)) / sqrt(d)               (inverse-rotated once)
  * where c are the N(0,1) codebooks and nK, nV the stored fp16 norms.
  *
- *   q           [batch][n_q_heads][d] of q_dtype (TQ_F16 | TQ_BF16 | TQ_F32).
- *   packed_*, norms_*  the cache layout above, with a leading batch dim.
+ *   q           [batch][n_q_heads][d] of q_dtype (TQ_F16 | TQ_BF16 | TQ_F32),
+ *               16-byte aligned.
+ *   packed_*, norms_*  the cache layout above with a leading batch dim, all
+ *               four 16-byte aligned; cap_tok must be a multiple of 8
+ *               (TQ_ERR_UNSUPPORTED otherwise).
  *   ctx_lens    int32 [batch] on the device. Values > cap_tok are clamped
  *               (TQ_DEV_CTX_CLAMPED); values <= 0 give out = 0
  *               (TQ_DEV_CTX_EMPTY).
- *   batch >= 1; n_q_heads >= 1; gqa_ratio >= 1 divides n_q_heads.
+ *   batch >= 1; n_q_heads >= 1; gqa_ratio in 1..8 divides n_q_heads.
  *   d, bits_k, bits_v, seed   as used by tq_encode for this cache.
  *   sparse_v_thresh  tau of the sparse-V gate; <= 0 disables it.
- *   split_tokens     tokens per split-K work item: 0 = library's choice,
- *                    else a positive multiple of TQ_SPARSE_V_BLOCK.
+ *   n_ctas      0: one CTA per SM (the intended setting); 1..1024 forces the
+ *               number of CTAs the 64-position blocks are balanced over.
  *   workspace, workspace_bytes  >= tq_attend_workspace_size(...) bytes,
- *                    16-byte aligned; contents on entry are ignored.
+ *               16-byte aligned. Its counter region (the first
+ *               round_up(4·batch·n_q_heads, 256) bytes) must be zero before
+ *               the first call that uses it (e.g. cudaMemset once); every call
+ *               leaves it zero again when it completes on the stream. The
+ *               rest is scratch. One workspace per concurrently running call.
  *   dev_status  device int, nullable.
  *   sparse_v_skipped  device uint64, nullable: atomically incremented by the
  *               number of (b, h, t) positions the gate left out.
- *   out         [batch][n_q_heads][d] of out_dtype (TQ_F16 | TQ_BF16 | TQ_F32).
+ *   out         [batch][n_q_heads][d] of out_dtype (TQ_F16 | TQ_BF16 | TQ_F32),
+ *               16-byte aligned.
  */
 int tq_attend(const void* q, int q_dtype,
               const uint8_t* packed_k, const uint16_t* norms_k,
               const uint8_t* packed_v, const uint16_t* norms_v,
               const int32_t* ctx_lens, int batch, int n_q_heads,
               int gqa_ratio, int d, int bits_k, int bits_v, uint64_t seed,
-              int cap_tok, float sparse_v_thresh, int split_tokens,
+              int cap_tok, float sparse_v_thresh, int n_ctas,
               void* workspace, size_t workspace_bytes, int* dev_status,
               unsigned long long* sparse_v_skipped,
               void* out, int out_dtype, void* stream);

@@ -132,7 +132,8 @@ def kv_f32(w: Workload, seq: int, n_tok: int, layer: int = 0,
         elif w.outlier == "laplace":
             lap = rng.laplace(0.0, 1.0, size=(chunk, w.n_kv_heads, w.n_outlier))
             for h in range(w.n_kv_heads):
-                blk[0, :, h, chans[h]] = lap[:, h, :].astype(np.float32)
+                for j, ch in enumerate(chans[h]):
+                    blk[0, :, h, ch] = lap[:, h, j]
         lo = max(tok_start, c * chunk)
         hi = min(tok_start + n_tok, (c + 1) * chunk)
         out[:, lo - tok_start:hi - tok_start] = blk[:, lo - c * chunk:hi - c * chunk]

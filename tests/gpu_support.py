@@ -155,7 +155,7 @@ def gpu_encode(kv_bits, dtype, bits_k, bits_v, seed, cap=None, tok_offset=0,
 
 
 def gpu_attend(q_bits, q_dtype, pk, nk, pv, nv, ctx, gqa, bk, bv, seed, tau=0.0,
-               split=0, out_dtype=None, want_skipped=False):
+               n_ctas=0, out_dtype=None, workspace=None):
     """tq_attend on host arrays; returns (out float32/bits, status, skipped)."""
     import torch
     import compressed_decode_attention_b200 as tq
@@ -163,8 +163,9 @@ def gpu_attend(q_bits, q_dtype, pk, nk, pv, nv, ctx, gqa, bk, bv, seed, tau=0.0,
     Hq = q_bits.shape[1]
     d = q_bits.shape[2]
     out_dtype = tq.TQ_F32 if out_dtype is None else out_dtype
-    ws_bytes = tq.tq_attend_workspace_size(B, Hq, cap, d, split)
-    ws = torch.empty(ws_bytes // 4, dtype=torch.float32, device="cuda")
+    ws_bytes = tq.tq_attend_workspace_size(B, Hq, cap, d)
+    ws = workspace if workspace is not None else \
+        torch.zeros(ws_bytes // 4, dtype=torch.float32, device="cuda")
     if out_dtype == tq.TQ_F32:
         out = torch.empty((B, Hq, d), dtype=torch.float32, device="cuda")
     else:
@@ -175,7 +176,7 @@ def gpu_attend(q_bits, q_dtype, pk, nk, pv, nv, ctx, gqa, bk, bv, seed, tau=0.0,
     q_enum = {"f16": tq.TQ_F16, "bf16": tq.TQ_BF16, "f32": tq.TQ_F32}[q_dtype]
     tq.tq_attend(qt, q_enum, dev(pk), dev(nk), dev(pv), dev(nv),
                  dev(np.asarray(ctx, np.int32)), B, Hq, gqa, d, bk, bv, seed, cap, tau,
-                 split, ws, ws_bytes, out, out_dtype, dev_status=st, sparse_v_skipped=sk)
+                 n_ctas, ws, ws_bytes, out, out_dtype, dev_status=st, sparse_v_skipped=sk)
     torch.cuda.synchronize()
     return host(out), int(st.item()), int(sk.item())
 
@@ -213,11 +214,20 @@ NEAR_FRACTION = 1e-4
 
 
 def check_indices(idx_gpu, idx_oracle, margin):
+    """Bit-exact outside the boundary window. Returns (mismatches, near, total)
+    so the caller can bound the exempted count over a whole encode call."""
     near = margin < NEAR_WINDOW
     bad = (idx_gpu != idx_oracle) & ~near
     assert not bad.any(), f"{int(bad.sum())} index mismatches outside the boundary window"
-    assert near.sum() <= NEAR_FRACTION * near.size, (int(near.sum()), near.size)
-    return int((idx_gpu != idx_oracle).sum()), int(near.sum())
+    return int((idx_gpu != idx_oracle).sum()), int(near.sum()), int(near.size)
+
+
+def check_near_fraction(stats):
+    """The exempted (near-threshold) coordinates of one encode call, K and V
+    together, are at most NEAR_FRACTION of all its coordinates."""
+    near = sum(s[1] for s in stats)
+    total = sum(s[2] for s in stats)
+    assert near <= NEAR_FRACTION * total, (near, total)
 
 
 def check_norms(nb_gpu, nb_oracle):

@@ -39,7 +39,7 @@ def _ambiguous(q64, pk, nk, ctx, gqa, bk, seed, tau):
     return int(np.sum(np.abs(gv / tau - 1.0) < GATE_WINDOW))
 
 
-def _run(name, scale=1.0, tau=None, split=0):
+def _run(name, scale=1.0, tau=None, n_ctas=0):
     w = S.WORKLOADS[name]
     pk, nk, pv, nv, ctx = oracle_cache(name)
     qb = S.query_bits(w, scale=scale)
@@ -47,7 +47,7 @@ def _run(name, scale=1.0, tau=None, split=0):
     tau = w.tau if tau is None else tau
     want, ng_o = oracle_attend(q64, pk, nk, pv, nv, ctx, w.gqa, w.bits_k, w.bits_v, SEED, tau)
     got, st, ng_g = gpu_attend(qb, w.dtype, pk, nk, pv, nv, ctx, w.gqa, w.bits_k, w.bits_v,
-                               SEED, tau=tau, split=split)
+                               SEED, tau=tau, n_ctas=n_ctas)
     return w, q64, (pk, nk, pv, nv, ctx), want, got, st, ng_o, ng_g, tau
 
 
@@ -84,10 +84,47 @@ def test_gate_thresholds_single_head(tau):
         assert ng_g == 1024 and np.all(got == 0)
 
 
-@pytest.mark.parametrize("split", [64, 128, 448, 1024])
-def test_split_sizes(split):
-    _, _, _, want, got, _, _, _, _ = _run("single_head_1k", split=split)
+@pytest.mark.parametrize("n_ctas", [1, 3, 7, 16, 1024])
+def test_cta_counts_single_head(n_ctas):
+    """1024 positions = 16 blocks: ranges that split the sequence unevenly,
+    one block per CTA, and more CTAs than blocks."""
+    _, _, _, want, got, _, _, _, _ = _run("single_head_1k", n_ctas=n_ctas)
     assert np.abs(got - want).max() <= ATOL
+
+
+@pytest.mark.parametrize("n_ctas", [5, 37, 300])
+def test_cta_counts_ragged_batch(n_ctas):
+    """CTA ranges that cross sequence and kv-head boundaries, ragged lengths."""
+    rng = np.random.default_rng(n_ctas)
+    ctx = np.array([1, 700, 64, 0, 129, 1000, 63, 512])
+    pk, nk, pv, nv = _small_cache(4, 2, len(ctx), 2, 1024, ctx, 21, rng)
+    qb = S.f16_bits(rng.standard_normal((len(ctx), 8, 128)))
+    q64 = codec.promote(qb, "f16")
+    want, _ = oracle_attend(q64, pk, nk, pv, nv, ctx, 4, 4, 2, 21)
+    got, st, _ = gpu_attend(qb, "f16", pk, nk, pv, nv, ctx, 4, 4, 2, 21, n_ctas=n_ctas)
+    assert np.abs(got - want).max() <= ATOL
+    assert st == 4
+
+
+def test_workspace_counters_return_to_zero_and_calls_repeat():
+    import torch
+    import compressed_decode_attention_b200 as tq
+    rng = np.random.default_rng(31)
+    ctx = np.array([900, 2000, 5])
+    pk, nk, pv, nv = _small_cache(3, 2, 1, 3, 2048, ctx, 2, rng)
+    qb = S.f16_bits(rng.standard_normal((3, 6, 128)))
+    ws_bytes = tq.tq_attend_workspace_size(3, 6, 2048, 128)
+    ws = torch.zeros(ws_bytes // 4, dtype=torch.float32, device="cuda")
+    outs = []
+    for n_ctas in (0, 9, 9, 0):
+        o, _, _ = gpu_attend(qb, "f16", pk, nk, pv, nv, ctx, 2, 3, 2, 2, n_ctas=n_ctas,
+                             workspace=ws)
+        counters = ws[: (3 * 6 * 4 + 255) // 256 * 64].view(torch.int32)
+        assert int(counters.abs().sum().item()) == 0
+        outs.append(o)
+    np.testing.assert_array_equal(outs[0], outs[3])
+    np.testing.assert_array_equal(outs[1], outs[2])
+    assert np.abs(outs[0] - outs[1]).max() <= 1e-5
 
 
 def _small_cache(bk, bv, B, Hkv, cap, ctx, seed, rng, dtype="f16"):

@@ -9,15 +9,18 @@ import numpy as np
 import pytest
 
 import synthetic as S
-from gpu_support import (check_indices, check_norms, dev, gpu_encode, host,
-                         oracle_encode_heads, oracle_encode_parallel)
+from gpu_support import (check_indices, check_near_fraction, check_norms, dev,
+                         gpu_encode, host, oracle_encode_heads, oracle_encode_parallel)
 from oracle import codec
 
 pytestmark = pytest.mark.gpu
 SEED = S.SIGN_SEED
 
 
-def _compare(kv, dtype, bk, bv, seed, pk, nk, pv, nv, lo=0, parallel=False):
+def _compare(kv, dtype, bk, bv, seed, pk, nk, pv, nv, lo=0, parallel=False,
+             count_rule=False):
+    """count_rule: also bound the exempted fraction (workload-scale calls;
+    on a few hundred vectors the expected count is below one)."""
     n, H, d = kv.shape[1:]
     enc = oracle_encode_parallel if parallel else oracle_encode_heads
     stats = []
@@ -27,6 +30,9 @@ def _compare(kv, dtype, bk, bv, seed, pk, nk, pv, nv, lo=0, parallel=False):
         idx_g = codec.unpack(r, bits, d).reshape(H, n, d)
         stats.append(check_indices(idx_g, idx_o, mg))
         check_norms(nb[:, lo:lo + n], nb_o)
+    if count_rule:
+        check_near_fraction(stats)
+    print(f"mismatches/near/total per K,V: {stats}")
     return stats
 
 
@@ -36,7 +42,8 @@ def test_encode_full_workload(name):
     kv = S.kv_bits(w, 0, w.ctx)
     pk, nk, pv, nv, st = gpu_encode(kv, w.dtype, w.bits_k, w.bits_v, SEED)
     assert st == 0
-    _compare(kv, w.dtype, w.bits_k, w.bits_v, SEED, pk, nk, pv, nv, parallel=True)
+    _compare(kv, w.dtype, w.bits_k, w.bits_v, SEED, pk, nk, pv, nv, parallel=True,
+             count_rule=True)
 
 
 def test_encode_k4v3_batched_serving_sequence():
@@ -44,7 +51,8 @@ def test_encode_k4v3_batched_serving_sequence():
     n = int(S.ctx_lens(w)[0])
     kv = S.kv_bits(w, 0, n)
     pk, nk, pv, nv, st = gpu_encode(kv, w.dtype, w.bits_k, w.bits_v, SEED, cap=w.cap_tok)
-    _compare(kv, w.dtype, w.bits_k, w.bits_v, SEED, pk, nk, pv, nv, parallel=True)
+    _compare(kv, w.dtype, w.bits_k, w.bits_v, SEED, pk, nk, pv, nv, parallel=True,
+             count_rule=True)
 
 
 @pytest.mark.parametrize("layer", [0, 31])
@@ -56,11 +64,13 @@ def test_encode_bulk_prefill_layer_sampled(layer):
     rng = np.random.default_rng(layer)
     toks = np.sort(rng.choice(w.ctx, size=2048, replace=False))
     sub = kv[:, toks]
+    stats = []
     for which, bits, rows, nb in ((0, w.bits_k, pk, nk), (1, w.bits_v, pv, nv)):
         idx_o, nb_o, mg = oracle_encode_heads(sub, w.dtype, which, bits, SEED)
         idx_g = codec.unpack(rows[:, toks].reshape(-1, rows.shape[-1]), bits, w.d)
-        check_indices(idx_g.reshape(idx_o.shape), idx_o, mg)
+        stats.append(check_indices(idx_g.reshape(idx_o.shape), idx_o, mg))
         check_norms(nb[:, toks], nb_o)
+    check_near_fraction(stats)
 
 
 @pytest.mark.parametrize("bk,bv", [(2, 2), (3, 3), (4, 4), (2, 4), (3, 2)])
@@ -79,7 +89,7 @@ def test_ragged_range_with_offset_leaves_other_rows():
     for rows in (pk, pv):
         assert np.all(rows[:, :37] == 0x5A) and np.all(rows[:, 1037:] == 0x5A)
     for nb in (nk, nv):
-        assert np.all(nb[:, :37] == 0x5A5A) and np.all(nb[:, 1037:] == 0x5A5A)
+        assert np.all(nb[:, :37] == 0x5A) and np.all(nb[:, 1037:] == 0x5A)
 
 
 def test_single_token_append():

@@ -95,12 +95,12 @@ def test_encode_validation(kw, want):
 def _attend(**kw):
     a = dict(q=FAKE, q_dtype=tq.TQ_F16, pk=FAKE, nk=FAKE, pv=FAKE, nv=FAKE, ctx=FAKE,
              batch=2, hq=8, gqa=4, d=128, bk=4, bv=2, seed=0, cap=256, tau=0.0,
-             split=0, ws=FAKE, wsb=1 << 30, status=None, skipped=None, out=FAKE,
+             ctas=0, ws=FAKE, wsb=1 << 30, status=None, skipped=None, out=FAKE,
              out_dtype=tq.TQ_F32, stream=0)
     a.update(kw)
     return tq.lib().tq_attend(a["q"], a["q_dtype"], a["pk"], a["nk"], a["pv"], a["nv"],
                               a["ctx"], a["batch"], a["hq"], a["gqa"], a["d"], a["bk"],
-                              a["bv"], a["seed"], a["cap"], a["tau"], a["split"], a["ws"],
+                              a["bv"], a["seed"], a["cap"], a["tau"], a["ctas"], a["ws"],
                               a["wsb"], a["status"], a["skipped"], a["out"], a["out_dtype"],
                               a["stream"])
 
@@ -110,7 +110,11 @@ def _attend(**kw):
     (dict(ws=None), tq.TQ_ERR_INVALID_ARG),
     (dict(gqa=3), tq.TQ_ERR_INVALID_ARG),                 # 8 % 3 != 0
     (dict(hq=16, gqa=16), tq.TQ_ERR_UNSUPPORTED),         # group wider than 8
-    (dict(split=100), tq.TQ_ERR_INVALID_ARG),             # not a multiple of 64
+    (dict(ctas=-1), tq.TQ_ERR_INVALID_ARG),
+    (dict(ctas=1025), tq.TQ_ERR_INVALID_ARG),             # more CTAs than slots
+    (dict(cap=260), tq.TQ_ERR_UNSUPPORTED),               # capacity not a multiple of 8
+    (dict(out=FAKE + 4), tq.TQ_ERR_INVALID_ARG),          # misaligned output
+    (dict(nk=FAKE + 2), tq.TQ_ERR_INVALID_ARG),
     (dict(wsb=16), tq.TQ_ERR_INVALID_ARG),                # workspace too small
     (dict(bk=1), tq.TQ_ERR_INVALID_ARG),
     (dict(d=64), tq.TQ_ERR_UNSUPPORTED),
@@ -124,8 +128,11 @@ def test_attend_validation(kw, want):
 
 
 def test_workspace_size_formula():
-    # (batch · heads · splits) units of d + 2 floats; 512-token splits by default
-    assert tq.tq_attend_workspace_size(1, 32, 32768, 128) == 32 * 64 * 130 * 4
-    assert tq.tq_attend_workspace_size(2, 4, 1000, 128, 256) == 2 * 4 * 4 * 130 * 4
-    assert tq.tq_attend_workspace_size(1, 1, 10, 128) == 130 * 4
-    assert tq.tq_attend_workspace_size(1, 1, 10, 128, 100) == 0
+    # counters (4·batch·heads bytes, rounded to 256) + slots of d + 2 floats for
+    # 1024 CTAs x 8 heads plus one per (batch, query head)
+    def want(b, h):
+        return -(-4 * b * h // 256) * 256 + (1024 * 8 + b * h) * 130 * 4
+    assert tq.tq_attend_workspace_size(1, 32, 32768, 128) == want(1, 32)
+    assert tq.tq_attend_workspace_size(64, 32, 16384, 128) == want(64, 32)
+    assert tq.tq_attend_workspace_size(1, 1, 10, 128) == want(1, 1)
+    assert tq.tq_attend_workspace_size(1, 1, 10, 64) == 0
