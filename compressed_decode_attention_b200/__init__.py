@@ -56,6 +56,9 @@ def lib() -> ctypes.CDLL:
         L.tq_attend.restype = I
         L.tq_attend.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F, I,
                                 P, SZ, P, P, P, I, P]
+        L.tq_attend_noalloc.restype = I
+        L.tq_attend_noalloc.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F, I,
+                                        P, P, P, I, P]
         _lib = L
     return _lib
 
@@ -137,4 +140,19 @@ def tq_attend(q, q_dtype, packed_k, norms_k, packed_v, norms_v, ctx_lens, batch,
         _ptr(norms_v), _ptr(ctx_lens), batch, n_q_heads, gqa_ratio, d, bits_k,
         bits_v, seed, cap_tok, float(sparse_v_thresh), n_ctas,
         _ptr(workspace), workspace_bytes, _ptr(dev_status),
+        _ptr(sparse_v_skipped), _ptr(out), out_dtype, _stream(stream)))
+
+
+def tq_attend_noalloc(q, q_dtype, packed_k, norms_k, packed_v, norms_v, ctx_lens,
+                      batch, n_q_heads, gqa_ratio, d, bits_k, bits_v, seed, cap_tok,
+                      sparse_v_thresh, n_ctas, out, out_dtype, dev_status=None,
+                      sparse_v_skipped=None, stream=None):
+    """tq_attend with the library's fixed internal scratch instead of a
+    workspace (for callers that cannot allocate). Calls on one device must
+    not overlap on the GPU; the first call per device must precede any
+    stream capture."""
+    _check("tq_attend_noalloc", lib().tq_attend_noalloc(
+        _ptr(q), q_dtype, _ptr(packed_k), _ptr(norms_k), _ptr(packed_v),
+        _ptr(norms_v), _ptr(ctx_lens), batch, n_q_heads, gqa_ratio, d, bits_k,
+        bits_v, seed, cap_tok, float(sparse_v_thresh), n_ctas, _ptr(dev_status),
         _ptr(sparse_v_skipped), _ptr(out), out_dtype, _stream(stream)))

@@ -227,6 +227,37 @@ int tq_attend(const void* q, int q_dtype,
               unsigned long long* sparse_v_skipped,
               void* out, int out_dtype, void* stream);
 
+/*
+ * tq_attend_noalloc — tq_attend for callers that cannot allocate device
+ * memory when they run attention (a fixed memory budget set at start-up, a
+ * runtime that forbids allocations after initialization because they can
+ * synchronize the device, or a plugin whose host owns every allocation).
+ * None of the source pages has a counterpart; this is a library convenience.
+ *
+ * Same arguments and results as tq_attend, without workspace and
+ * workspace_bytes: the scratch is one fixed 8 MiB device array inside the
+ * library, allocated when the library is loaded, on every device that loads
+ * it, and kept until the process exits. This call allocates and frees no
+ * memory.
+ *   - Limit: batch · n_q_heads <= 7879 (the problem's
+ *     tq_attend_workspace_size must fit 8 MiB); larger problems return
+ *     TQ_ERR_UNSUPPORTED.
+ *   - The first call on a device looks up the array's device address (a
+ *     host-side set-up); make that first call before any stream capture.
+ *   - Every call on a device shares the array. Each call first clears the
+ *     array's counter region on `stream`; calls whose execution overlaps on
+ *     the GPU (other streams, other threads) race on it and give undefined
+ *     results. Serialize them.
+ */
+int tq_attend_noalloc(const void* q, int q_dtype,
+                      const uint8_t* packed_k, const uint16_t* norms_k,
+                      const uint8_t* packed_v, const uint16_t* norms_v,
+                      const int32_t* ctx_lens, int batch, int n_q_heads,
+                      int gqa_ratio, int d, int bits_k, int bits_v, uint64_t seed,
+                      int cap_tok, float sparse_v_thresh, int n_ctas,
+                      int* dev_status, unsigned long long* sparse_v_skipped,
+                      void* out, int out_dtype, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
