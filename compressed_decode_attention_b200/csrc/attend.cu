@@ -8,27 +8,30 @@
 // weight are left out (block-local rule, include/tq.h).
 //
 // Work decomposition. The cache is a flat list of 64-position blocks in
-// (batch, kv head, block) order; CTA c of G (one per SM) owns blocks
-// [c·NB/G, (c+1)·NB/G). A CTA walks the (batch, kv head) segments of its range;
-// its 8 warps split each segment, merge in shared memory, and either write
-// the output directly (segment = whole sequence) or leave a partial in a
-// workspace slot; the last CTA to finish a sequence (atomic counter, no
-// waiting) merges the partials and writes the output. No separate combine
-// launch, no spin-waits.
+// (batch, kv head, block) order; CTA c of Geff = min(grid, #blocks) owns
+// blocks [c·NB/Geff, (c+1)·NB/Geff). A CTA walks the (batch, kv head)
+// segments of its range; its warps split each segment, merge in shared
+// memory, and either write the output (segment = whole sequence) or leave a
+// partial in a workspace slot; the last CTA to finish a sequence (atomic
+// counter, no waiting) merges the partials and writes the output. No separate
+// combine launch, no spin-waits.
 //
-// Per warp and 64-position block (GQA group of g <= 8 query heads):
+// Per warp and 64-position block (GQA group of g <= 8 query heads), in four
+// 16-position steps:
 //   stage   cp.async of the packed K/V rows and fp16 norms (per-warp ring)
-//   scores  mma.m16n8k16 (fp16 in, fp32 accumulate). A = rotated query:
-//           rows 0-7 its fp16 high part, rows 8-15 its fp16 low part (the
-//           group fills at most 8 rows), B = K codebook values as fp16
-//           high/low pairs from a shared-memory table indexed by the packed
-//           byte (one copy per lane, conflict-free). score = row h + row h+8,
-//           so the query and codebook keep ~22 significant bits.
-//   softmax fp32, log2 domain; block maximum = sparse-V reference
-//   PV      mma.m16n8k16: A = V codebook values (fp16) as the transposed
-//           tile, B = softmax weights · V norm (fp16) taken straight from the
-//           score accumulators. V2: token pairs by byte permutes of a 4-entry
-//           register table; V3/V4: pair table + movmatrix transpose.
+//   scores  mma.m16n8k16, fp16 in, fp32 accumulate. A = K codebook values of
+//           16 positions (rows) x 16 coordinates, read as fp16 high/low pairs
+//           from a shared table indexed by the packed byte (one copy per
+//           half-warp lane); B = rotated query, fp16 high and low parts in
+//           the 8 columns (g <= 4: 4 heads x {high, low}; g <= 8: two column
+//           tiles). K high, K low and query low are summed, so scores keep
+//           ~22 significant bits (fp16-only operands measured up to 1.2e-2
+//           output error with x20 outlier channels).
+//   softmax fp32, log2 domain; block maximum = sparse-V reference.
+//   PV      mma.m16n8k16: A = V codebook values (fp16), coordinates x
+//           positions; B = softmax weight x V norm (fp16), moved from the
+//           score layout with movmatrix. V2: position pairs by byte permutes
+//           of a 4-entry register table; V3/V4: pair table + movmatrix.
 // Output, once per (batch, query head): D⊙(H·(acc/l))/d with shuffles.
 #include <math.h>
 
@@ -37,12 +40,18 @@
 namespace tq {
 namespace {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 12;
 constexpr int kThreads = 32 * kWarps;
 constexpr int kBlk = kGateBlock;                // positions per block
 constexpr float kLog2e = 1.44269504088896340736f;
 constexpr float kKScale = 256.f;                // K codebook scale inside the MMA
 constexpr int kSmemBudget = 227 * 1024;
+
+constexpr int ceil_pow2(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
 
 template <int BK, int BV>
 struct Geo {
@@ -53,11 +62,17 @@ struct Geo {
   static constexpr int VB = kBlk * RVS;
   static constexpr int NKOFF = KB + VB;
   static constexpr int STAGE = KB + VB + 2 * kBlk * 2;
-  static constexpr int LUTK = (1 << (2 * BK)) * 32 * 8;  // uint2 per (pair, lane)
-  static constexpr int LUTV = BV == 2 ? 0 : (1 << (2 * BV)) * 32 * 4;
+  // K table: uint2 (high pair, low pair) per (pair code, lane & 15): 128 B per code.
+  static constexpr int LUTK = (1 << (2 * BK)) * 128;
+  // V table (3/4 bits): uint32 fp16 pair per (pair code, lane): 128 B per code.
+  static constexpr int LUTV = BV == 2 ? 0 : (1 << (2 * BV)) * 128;
+  // The V table sits at a power-of-two offset no smaller than either table,
+  // so entry addresses are formed with OR.
+  static constexpr int LUTV_OFF = BV == 2 ? LUTK : ceil_pow2(LUTK > LUTV ? LUTK : LUTV);
+  static constexpr int QOFF = LUTV_OFF + LUTV;
   static constexpr int QS = kMaxGroup * kHeadDim * 2 * 2;  // q~ high and low, fp16
-  static constexpr int MISC = 512;                      // 128 words
-  static constexpr int FIXED = LUTK + LUTV + QS + MISC;
+  static constexpr int MISC = 1024;                     // kMiscWords words
+  static constexpr int FIXED = QOFF + QS + MISC;
   static constexpr int NFIT = (kSmemBudget - FIXED) / (kWarps * STAGE);
   static constexpr int NSTAGE = NFIT > 3 ? 3 : NFIT;
   static constexpr int MERGE = kWarps * (kMaxGroup * kHeadDim + 2 * kMaxGroup) * 4;
@@ -68,19 +83,22 @@ struct Geo {
 };
 
 // misc words
-constexpr int kMiscSeg = 0;      // b, g, blk0, nseg, nb, L, flat0 (7 ints)
+constexpr int kMiscSeg = 0;      // b, g, blk0, nseg, nb, L
 constexpr int kMiscLast = 8;     // last-CTA flag
-constexpr int kMiscNB = 9;       // flat block count (2 ints: lo, hi)
+constexpr int kMiscNB = 9;       // flat block count (lo, hi)
 constexpr int kMiscState = 12;   // scan state: sb, sP (lo, hi)
 constexpr int kMiscQInv = 16;    // 8 floats: 1/(query scale · kKScale)
 constexpr int kMiscM = 32;       // 8 floats: merged max
 constexpr int kMiscL = 40;       // 8 floats: merged sum
+constexpr int kMiscCb = 64;      // 32 words: staged codebooks
+constexpr int kMiscWt = 128;     // kWarps x 8 floats: per-warp merge weights
+constexpr int kMiscWords = 256;  // Geo::MISC / 4
+static_assert(kMiscWt + kWarps * kMaxGroup <= kMiscWords, "misc words");
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1,
                                          uint32_t a2, uint32_t a3, uint32_t b0,
                                          uint32_t b1) {
-  asm(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, "
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, "
       "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -89,6 +107,12 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 __device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
   uint32_t y;
   asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+  return y;
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {   // ex2.approx: -inf -> 0
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
   return y;
 }
 
@@ -108,13 +132,9 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-// Plain shared-memory loads at a byte offset from the dynamic smem base, so
-// the compiler can schedule them (the cp.async waits carry memory clobbers).
-__device__ __forceinline__ uint2 lds64(const uint8_t* base, uint32_t off) {
-  return *reinterpret_cast<const uint2*>(base + off);
-}
-__device__ __forceinline__ uint32_t lds32(const uint8_t* base, uint32_t off) {
-  return *reinterpret_cast<const uint32_t*>(base + off);
+template <typename T>
+__device__ __forceinline__ T lds(const uint8_t* base, uint32_t off) {
+  return *reinterpret_cast<const T*>(base + off);
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
@@ -170,52 +190,53 @@ __device__ __forceinline__ int pv_coord(int r, int m) {
   return 32 * ((m & 7) >> 1) + 4 * r + (m & 1) + 2 * (m >> 3);
 }
 
-// Shared-memory address of pair-table entry `field` in this lane's copy
-// (lane_base = table address + lane · entry size).
-template <int ENTRY_SHIFT>
-__device__ __forceinline__ uint32_t lut_off(uint32_t field, uint32_t lane_base) {
-  return (field << ENTRY_SHIFT) + lane_base;
-}
-
-// Field p (2·BITS bits: coordinates 2p, 2p+1) of a lane's chunk of packed words.
-template <int BITS>
-__device__ __forceinline__ uint32_t pair_field(const uint32_t* w, int p) {
+// (pair code p of a lane's chunk of packed words) << SHIFT, for a table
+// whose entries are 2^SHIFT bytes apart. Codes are 2·BITS bits wide
+// (coordinates 2p, 2p+1), little-endian in the chunk.
+template <int BITS, int SHIFT>
+__device__ __forceinline__ uint32_t pair_code_shifted(const uint32_t* w, int p) {
   constexpr int FB = 2 * BITS;
+  constexpr uint32_t MASK = ((1u << FB) - 1u) << SHIFT;
   const int bit = p * FB;
   const int k = bit >> 5, off = bit & 31;
-  uint32_t v;
-  if (off + FB <= 32) v = w[k] >> off;
-  else v = __funnelshift_r(w[k], w[k + 1], off);
-  return v & ((1u << FB) - 1u);
+  if (off + FB > 32) return (__funnelshift_r(w[k], w[k + 1], off) << SHIFT) & MASK;
+  if (off >= SHIFT) return (w[k] >> (off - SHIFT)) & MASK;
+  return (w[k] << (SHIFT - off)) & MASK;
 }
 
-template <int BK, int BV>
+template <int BK, int BV, int NT>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_kernel(const __grid_constant__ AttendArgs a,
               const __grid_constant__ Codebook cbk,
               const __grid_constant__ Codebook cbv,
               const __grid_constant__ SignMask sm) {
   using Gm = Geo<BK, BV>;
+  constexpr int NR = NT == 1 ? 1 : 2;       // score rows (positions) per lane and step
   extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* lutK = smem;
-  uint8_t* lutV = smem + Gm::LUTK;
-  __half* qhi = reinterpret_cast<__half*>(smem + Gm::LUTK + Gm::LUTV);
+  uint8_t* lutK = smem;                                   // offset 0
+  uint8_t* lutV = smem + Gm::LUTV_OFF;
+  __half* qhi = reinterpret_cast<__half*>(smem + Gm::QOFF);
   __half* qlo = qhi + kMaxGroup * kHeadDim;
   float* fin = reinterpret_cast<float*>(qhi);             // reuses q~ after a segment
-  int* misc = reinterpret_cast<int*>(smem + Gm::LUTK + Gm::LUTV + Gm::QS);
+  int* misc = reinterpret_cast<int*>(smem + Gm::QOFF + Gm::QS);
   float* miscf = reinterpret_cast<float*>(misc);
-  uint8_t* ring = smem + Gm::FIXED;
-  float* merge = reinterpret_cast<float*>(ring);
+  float* merge = reinterpret_cast<float*>(smem + Gm::FIXED);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, tq = lane & 3;
   const int H = a.n_kv_heads, GQ = a.gqa, B = a.batch;
   const int Gc = gridDim.x, cta = blockIdx.x;   // Gc <= kMaxCtas (host check)
-  const uint32_t lutK_base = 0, lutV_base = Gm::LUTK;    // byte offsets in smem
+  const uint32_t lbK = (lane & 15) * 8;                   // K table lane offset
+  const uint32_t lbV = Gm::LUTV_OFF | (lane * 4);         // V table lane base
 
-  // ---- codebook tables: fp16 high/low parts of the scaled K levels and
+  // Lengths of the first 32 sequences, loaded by warp 0 now so the latency
+  // overlaps the table build; the block count and the first segment search
+  // reuse them.
+  const int len0 = (warp == 0 && lane < B) ? min(max(a.ctx_lens[lane], 0), a.cap_tok) : 0;
+
+  // ---- codebook tables: fp16 high/low parts of the scaled K levels and the
   // fp16 V levels are staged in misc first (uniform lookups afterwards).
-  uint32_t* cbs = reinterpret_cast<uint32_t*>(misc) + 64;   // 16 K (hi|lo<<16), 16 V
+  uint32_t* cbs = reinterpret_cast<uint32_t*>(misc) + kMiscCb;
   if (tid < 16) {
     const float c = cbk.centroid[tid] * kKScale;
     const __half h = __float2half_rn(c), l = __float2half_rn(c - __half2float(h));
@@ -223,19 +244,19 @@ attend_kernel(const __grid_constant__ AttendArgs a,
     cbs[16 + tid] = __half_as_ushort(__float2half_rn(cbv.centroid[tid]));
   }
   __syncthreads();
-  for (int e = tid; e < (1 << (2 * BK)) * 32; e += kThreads) {
-    const int entry = e >> 5, copy = e & 31;
-    const uint32_t c0 = cbs[entry & ((1 << BK) - 1)], c1 = cbs[entry >> BK];
+  for (int e = tid; e < (1 << (2 * BK)) * 16; e += kThreads) {
+    const int code = e >> 4, copy = e & 15;
+    const uint32_t c0 = cbs[code & ((1 << BK) - 1)], c1 = cbs[code >> BK];
     uint2 v;
-    v.x = (c0 & 0xFFFFu) | (c1 << 16);
-    v.y = (c0 >> 16) | (c1 & 0xFFFF0000u);
-    *reinterpret_cast<uint2*>(lutK + entry * 256 + copy * 8) = v;
+    v.x = (c0 & 0xFFFFu) | (c1 << 16);              // high parts (even, odd coord)
+    v.y = (c0 >> 16) | (c1 & 0xFFFF0000u);          // low parts
+    *reinterpret_cast<uint2*>(lutK + code * 128 + copy * 8) = v;
   }
   if (BV != 2) {
     for (int e = tid; e < (1 << (2 * BV)) * 32; e += kThreads) {
-      const int entry = e >> 5, copy = e & 31;
-      *reinterpret_cast<uint32_t*>(lutV + entry * 128 + copy * 4) =
-          cbs[16 + (entry & ((1 << BV) - 1))] | (cbs[16 + (entry >> BV)] << 16);
+      const int code = e >> 5, copy = e & 31;
+      *reinterpret_cast<uint32_t*>(lutV + code * 128 + copy * 4) =
+          cbs[16 + (code & ((1 << BV) - 1))] | (cbs[16 + (code >> BV)] << 16);
     }
   }
   // V2 byte tables: low bytes of the 4 fp16 levels, then their high bytes.
@@ -271,7 +292,7 @@ attend_kernel(const __grid_constant__ AttendArgs a,
   if (warp == 0) {
     long long tot = 0;
     for (int b0 = 0; b0 < B; b0 += 32) {
-      int nb = (b0 + lane < B) ? seq_blocks(a, b0 + lane) : 0;
+      int nb = b0 == 0 ? (len0 + kBlk - 1) / kBlk : ((b0 + lane < B) ? seq_blocks(a, b0 + lane) : 0);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) nb += __shfl_xor_sync(0xFFFFFFFFu, nb, o);
       tot += nb;
@@ -280,9 +301,9 @@ attend_kernel(const __grid_constant__ AttendArgs a,
       const long long nbt = tot * H;
       misc[kMiscNB] = (int)(nbt & 0xFFFFFFFF);
       misc[kMiscNB + 1] = (int)(nbt >> 32);
-      misc[kMiscState] = 0;       // sb
-      misc[kMiscState + 1] = 0;   // sP low word
-      misc[kMiscState + 2] = 0;   // sP high word
+      misc[kMiscState] = 0;
+      misc[kMiscState + 1] = 0;
+      misc[kMiscState + 2] = 0;
     }
   }
   __syncthreads();
@@ -296,6 +317,16 @@ attend_kernel(const __grid_constant__ AttendArgs a,
   unsigned nskip = 0;
   const float log2tau = a.tau > 0.f ? log2f(a.tau) : -INFINITY;
 
+  // Lane roles in the score / softmax layout:
+  //   NT = 1: the lane holds position gq (tq < 2) or gq + 8 (tq >= 2) of each
+  //           16-position step, for heads hs0 = 2·(tq & 1) and hs0 + 1;
+  //   NT = 2: positions gq and gq + 8, heads hs0 = 2·tq and hs0 + 1.
+  const int hs0 = NT == 1 ? 2 * (tq & 1) : 2 * tq;
+  const bool hv0 = hs0 < GQ, hv1 = hs0 + 1 < GQ;
+  auto pos_of = [&](int mt, int rr) {
+    return 16 * mt + gq + (NT == 1 ? 8 * (tq >> 1) : 8 * rr);
+  };
+
   while (pos < r1) {
     // ---- next segment (warp 0): first sequence whose flat range holds pos
     if (warp == 0) {
@@ -307,7 +338,8 @@ attend_kernel(const __grid_constant__ AttendArgs a,
           break;
         }
         const int b = sb + lane;
-        const int nb = b < B ? seq_blocks(a, b) : 0;
+        const int len = sb == 0 ? len0 : (b < B ? min(max(a.ctx_lens[b], 0), a.cap_tok) : 0);
+        const int nb = (len + kBlk - 1) / kBlk;
         int incl = nb;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -319,28 +351,26 @@ attend_kernel(const __grid_constant__ AttendArgs a,
         if (hit) {
           const int l = __ffs(hit) - 1;
           const int nbl = __shfl_sync(0xFFFFFFFFu, nb, l);
+          const int lenl = __shfl_sync(0xFFFFFFFFu, len, l);
           const int excl = __shfl_sync(0xFFFFFFFFu, incl - nb, l);
           sb += l;
           sP += excl;
           if (lane == 0) {
-            const long long start = (long long)H * sP;
-            const long long rel = pos - start;
+            const long long rel = pos - (long long)H * sP;
             const int g = (int)(rel / nbl), blk0 = (int)(rel % nbl);
-            const int nseg = (int)min((long long)(nbl - blk0), r1 - pos);
             misc[kMiscSeg + 0] = sb;
             misc[kMiscSeg + 1] = g;
             misc[kMiscSeg + 2] = blk0;
-            misc[kMiscSeg + 3] = nseg;
+            misc[kMiscSeg + 3] = (int)min((long long)(nbl - blk0), r1 - pos);
             misc[kMiscSeg + 4] = nbl;
-            misc[kMiscSeg + 5] = min(max(a.ctx_lens[sb], 0), a.cap_tok);
+            misc[kMiscSeg + 5] = lenl;
             misc[kMiscState] = sb;
             misc[kMiscState + 1] = (int)(sP & 0xFFFFFFFF);
             misc[kMiscState + 2] = (int)(sP >> 32);
           }
           break;
         }
-        const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
-        sP += total;
+        sP += __shfl_sync(0xFFFFFFFFu, incl, 31);
         sb += 32;
       }
     }
@@ -351,14 +381,77 @@ attend_kernel(const __grid_constant__ AttendArgs a,
     const long long sP_seg = (long long)(unsigned)misc[kMiscState + 1] | ((long long)misc[kMiscState + 2] << 32);
     const long long seg_first = (long long)H * sP_seg + (long long)g * nbl;
 
+    // query values of the group (warp h < g loads head h), issued before the
+    // block loads so that both latencies overlap
+    float qraw[4] = {0.f, 0.f, 0.f, 0.f};
+    if (warp < GQ) {
+      const size_t qo = ((size_t)b * a.n_q_heads + (size_t)g * GQ + warp) * kHeadDim + 4 * lane;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) qraw[k] = load_elem(a.q, a.q_dtype, qo + k);
+    }
+
+    // ---- this warp's blocks of the segment; their first loads go out
+    // before the query rotation so that the two overlap
+    const int wb0 = blk0 + (int)((long long)nseg * warp / kWarps);
+    const int wb1 = blk0 + (int)((long long)nseg * (warp + 1) / kWarps);
+    const int nw = wb1 - wb0;
+
+    float acc[8][4];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+
+    const size_t seq_row = ((size_t)b * H + g) * a.cap_tok;
+    const uint8_t* gk = a.packed_k + seq_row * Gm::RK;
+    const uint8_t* gv = a.packed_v + seq_row * Gm::RV;
+    const uint16_t* gnk = a.norms_k + seq_row;
+    const uint16_t* gnv = a.norms_v + seq_row;
+    const uint32_t wring = Gm::FIXED + warp * Gm::NSTAGE * Gm::STAGE;   // smem offset
+    const uint32_t wring_s = smem_addr(smem) + wring;                    // shared address
+
+    // cp.async of block `blk` into ring slot `slot`. K and V blocks are
+    // contiguous in global memory; chunk c of K lands at byte 16c, chunk c of
+    // V at row (c / BV) · RVS + (c % BV) · 16. Chunks past the sequence are
+    // zero-filled without reading.
+    auto issue = [&](int blk, int slot) {
+      const int t0 = blk * kBlk;
+      const int kvalid = min(kBlk, L - t0) * BK;
+      const int vvalid = min(kBlk, L - t0) * BV;
+      const uint32_t dst = wring_s + slot * Gm::STAGE;
+      const uint8_t* ksrc = gk + (size_t)t0 * Gm::RK;
+      const uint8_t* vsrc = gv + (size_t)t0 * Gm::RV;
+#pragma unroll
+      for (int i = 0; i < BK * 2; ++i) {
+        const int ch = lane + 32 * i;
+        const bool ok = ch < kvalid;
+        cp_async16(dst + 16 * ch, ksrc + (ok ? 16 * ch : 0), ok ? 16 : 0);
+      }
+#pragma unroll
+      for (int i = 0; i < BV * 2; ++i) {
+        const int ch = lane + 32 * i;
+        const bool ok = ch < vvalid;
+        cp_async16(dst + Gm::KB + (ch / BV) * Gm::RVS + (ch % BV) * 16,
+                   vsrc + (ok ? 16 * ch : 0), ok ? 16 : 0);
+      }
+      if (lane < 16) {
+        const int c8 = lane & 7;
+        const bool ok = t0 + 8 * c8 < L;
+        const uint16_t* src = (lane < 8 ? gnk : gnv) + t0 + (ok ? 8 * c8 : 0);
+        cp_async16(dst + Gm::NKOFF + (lane >> 3) * (2 * kBlk) + 16 * c8, src, ok ? 16 : 0);
+      }
+    };
+
+#pragma unroll
+    for (int p = 0; p < Gm::NSTAGE - 1; ++p) {
+      if (p < nw) issue(wb0 + p, p);
+      cp_async_commit();
+    }
     // ---- rotated query of the group: warp h handles query head h
     if (warp < GQ) {
-      const size_t qb = ((size_t)b * a.n_q_heads + (size_t)g * GQ + warp) * kHeadDim + 4 * lane;
       float x[4];
       const uint32_t m = sm.w[lane >> 3];
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        x[k] = apply_sign(load_elem(a.q, a.q_dtype, qb + k), m, (4 * lane + k) & 31);
+      for (int k = 0; k < 4; ++k) x[k] = apply_sign(qraw[k], m, (4 * lane + k) & 31);
       fwht128_warp(x, lane);
       // log2(e)/d^{3/2} folds the rotation normalization, the codebook's
       // 1/sqrt(d) and the softmax 1/sqrt(d); a power-of-two scale keeps the
@@ -387,68 +480,27 @@ attend_kernel(const __grid_constant__ AttendArgs a,
     }
     __syncthreads();
 
-    // ---- this warp's blocks of the segment
-    const int wb0 = blk0 + (int)((long long)nseg * warp / kWarps);
-    const int wb1 = blk0 + (int)((long long)nseg * (warp + 1) / kWarps);
-    const int nw = wb1 - wb0;
-    const bool hv = gq < GQ;                       // this lane's score row is a real head
-    uint32_t qa[8][4];
+    // ---- query fragments (B operand of the score MMA), column n = gq.
+    //   NT = 1: columns 0-3 hold the high part of heads 0-3, 4-7 their low part.
+    //   NT = 2: tile 0 column n = high part of head n, tile 1 = low part.
+    // The K-low product reuses tile 0 (for NT = 1 it also picks up the
+    // negligible query-low x K-low term).
+    uint32_t qb[NT][8][2];
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      const int c0 = 32 * tq + 4 * s;
-      if (hv) {
-        qa[s][0] = *reinterpret_cast<const uint32_t*>(qhi + gq * kHeadDim + c0);
-        qa[s][1] = *reinterpret_cast<const uint32_t*>(qlo + gq * kHeadDim + c0);
-        qa[s][2] = *reinterpret_cast<const uint32_t*>(qhi + gq * kHeadDim + c0 + 2);
-        qa[s][3] = *reinterpret_cast<const uint32_t*>(qlo + gq * kHeadDim + c0 + 2);
-      } else {
-        qa[s][0] = qa[s][1] = qa[s][2] = qa[s][3] = 0u;
+    for (int t = 0; t < NT; ++t) {
+      const int head = NT == 1 ? (gq & 3) : gq;
+      const __half* src = (NT == 1 ? (gq < 4) : (t == 0)) ? qhi : qlo;
+      const bool ok = head < GQ;
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        const int c0 = 32 * tq + 4 * s;
+        qb[t][s][0] = ok ? *reinterpret_cast<const uint32_t*>(src + head * kHeadDim + c0) : 0u;
+        qb[t][s][1] = ok ? *reinterpret_cast<const uint32_t*>(src + head * kHeadDim + c0 + 2) : 0u;
       }
     }
-    const float sinv = hv ? miscf[kMiscQInv + gq] : 0.f;
+    const float sinv0 = hv0 ? miscf[kMiscQInv + hs0] : 0.f;
+    const float sinv1 = hv1 ? miscf[kMiscQInv + hs0 + 1] : 0.f;
 
-    float acc[8][4];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
-    float m_run = -INFINITY, l_run = 0.f;
-
-    const size_t seq_row = ((size_t)b * H + g) * a.cap_tok;
-    const uint8_t* gk = a.packed_k + seq_row * Gm::RK;
-    const uint8_t* gv = a.packed_v + seq_row * Gm::RV;
-    const uint16_t* gnk = a.norms_k + seq_row;
-    const uint16_t* gnv = a.norms_v + seq_row;
-    const uint32_t wring = Gm::FIXED + warp * Gm::NSTAGE * Gm::STAGE;   // smem offset
-    const uint32_t wring_s = smem_addr(smem) + wring;                    // shared address
-
-    auto issue = [&](int blk, int slot) {
-      const int t0 = blk * kBlk;
-      const int nvalid = min(kBlk, L - t0);
-      const uint32_t dst = wring_s + slot * Gm::STAGE;
-      for (int ch = lane; ch < kBlk * BK; ch += 32) {
-        const int row = ch / BK, col = ch % BK;
-        const bool ok = row < nvalid;
-        const uint8_t* src = gk + (size_t)(t0 + (ok ? row : 0)) * Gm::RK + col * 16;
-        cp_async16(dst + row * Gm::RK + col * 16, src, ok ? 16 : 0);
-      }
-      for (int ch = lane; ch < kBlk * BV; ch += 32) {
-        const int row = ch / BV, col = ch % BV;
-        const bool ok = row < nvalid;
-        const uint8_t* src = gv + (size_t)(t0 + (ok ? row : 0)) * Gm::RV + col * 16;
-        cp_async16(dst + Gm::KB + row * Gm::RVS + col * 16, src, ok ? 16 : 0);
-      }
-      if (lane < 16) {
-        const int c8 = lane & 7;
-        const bool ok = t0 + 8 * c8 < L;
-        const uint16_t* src = (lane < 8 ? gnk : gnv) + t0 + (ok ? 8 * c8 : 0);
-        cp_async16(dst + Gm::NKOFF + (lane >> 3) * (2 * kBlk) + 16 * c8, src, ok ? 16 : 0);
-      }
-    };
-
-#pragma unroll
-    for (int p = 0; p < Gm::NSTAGE - 1; ++p) {
-      if (p < nw) issue(wb0 + p, p);
-      cp_async_commit();
-    }
     for (int i = 0; i < nw; ++i) {
       {
         const int nxt = i + Gm::NSTAGE - 1;
@@ -457,96 +509,167 @@ attend_kernel(const __grid_constant__ AttendArgs a,
       }
       cp_async_wait<Gm::NSTAGE - 1>();
       __syncwarp();
-      const uint32_t st = wring + (i % Gm::NSTAGE) * Gm::STAGE;          // smem offset
+      const uint32_t st = wring + (i % Gm::NSTAGE) * Gm::STAGE;         // smem offset
       const int t0 = (wb0 + i) * kBlk;
+      const bool partial = t0 + kBlk > L;
 
-      // -- scores for 8 tiles of 8 positions; high and low codebook parts
-      //    accumulate in separate chains
-      float sc[8][2];
+      // -- scores: 4 steps of 16 positions
+      float sc[4][NR][2];               // [step][row][head hs0 + e]
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        uint32_t kw[BK + 1];
-        const uint32_t krow = st + (8 * j + gq) * Gm::RK + 4 * BK * tq;
+      for (int mt = 0; mt < 4; ++mt) {
+        uint32_t kw0[BK + 1], kw1[BK + 1];   // rows gq and gq + 8, chunk tq
+        const uint32_t r0 = st + (16 * mt + gq) * Gm::RK + 4 * BK * tq;
+        const uint32_t r1 = r0 + 8 * Gm::RK;
+        if (BK == 4) {                       // one 16-byte load per row chunk
+          const uint4 u0 = lds<uint4>(smem, r0), u1 = lds<uint4>(smem, r1);
+          kw0[0] = u0.x; kw0[1] = u0.y; kw0[2 % (BK + 1)] = u0.z; kw0[3 % (BK + 1)] = u0.w;
+          kw1[0] = u1.x; kw1[1] = u1.y; kw1[2 % (BK + 1)] = u1.z; kw1[3 % (BK + 1)] = u1.w;
+        } else if (BK == 2) {
+          const uint2 u0 = lds<uint2>(smem, r0), u1 = lds<uint2>(smem, r1);
+          kw0[0] = u0.x; kw0[1] = u0.y;
+          kw1[0] = u1.x; kw1[1] = u1.y;
+        } else {
 #pragma unroll
-        for (int w = 0; w < BK; ++w) kw[w] = lds32(smem, krow + 4 * w);
-        kw[BK] = 0;
-        float dh[4] = {0.f, 0.f, 0.f, 0.f}, dl[4] = {0.f, 0.f, 0.f, 0.f};
-        const uint32_t lo = lutK_base + lane * 8;
-        uint2 e[16];
+          for (int w = 0; w < BK; ++w) {
+            kw0[w] = lds<uint32_t>(smem, r0 + 4 * w);
+            kw1[w] = lds<uint32_t>(smem, r1 + 4 * w);
+          }
+        }
+        kw0[BK] = kw1[BK] = 0;
+        // two accumulator sets (even / odd k-steps) halve the MMA chains
+        float dh[2][NT][4], dl[2][4];
 #pragma unroll
-        for (int p = 0; p < 16; ++p) e[p] = lds64(smem, lut_off<8>(pair_field<BK>(kw, p), lo));
+        for (int c = 0; c < 2; ++c) {
+#pragma unroll
+          for (int t = 0; t < NT; ++t) dh[c][t][0] = dh[c][t][1] = dh[c][t][2] = dh[c][t][3] = 0.f;
+          dl[c][0] = dl[c][1] = dl[c][2] = dl[c][3] = 0.f;
+        }
 #pragma unroll
         for (int s2 = 0; s2 < 8; ++s2) {
-          mma16816(dh, qa[s2][0], qa[s2][1], qa[s2][2], qa[s2][3], e[2 * s2].x, e[2 * s2 + 1].x);
-          mma16816(dl, qa[s2][0], qa[s2][1], qa[s2][2], qa[s2][3], e[2 * s2].y, e[2 * s2 + 1].y);
+          const uint2 e00 = lds<uint2>(smem, pair_code_shifted<BK, 7>(kw0, 2 * s2) | lbK);
+          const uint2 e10 = lds<uint2>(smem, pair_code_shifted<BK, 7>(kw1, 2 * s2) | lbK);
+          const uint2 e01 = lds<uint2>(smem, pair_code_shifted<BK, 7>(kw0, 2 * s2 + 1) | lbK);
+          const uint2 e11 = lds<uint2>(smem, pair_code_shifted<BK, 7>(kw1, 2 * s2 + 1) | lbK);
+#pragma unroll
+          for (int t = 0; t < NT; ++t)
+            mma16816(dh[s2 & 1][t], e00.x, e10.x, e01.x, e11.x, qb[t][s2][0], qb[t][s2][1]);
+          mma16816(dl[s2 & 1], e00.y, e10.y, e01.y, e11.y, qb[0][s2][0], qb[0][s2][1]);
         }
-        const uint32_t n2 = lds32(smem, st + Gm::NKOFF + (8 * j + 2 * tq) * 2);
-        const float n0 = __half2float(__ushort_as_half((uint16_t)(n2 & 0xFFFF)));
-        const float n1 = __half2float(__ushort_as_half((uint16_t)(n2 >> 16)));
-        const int tok = t0 + 8 * j + 2 * tq;
-        sc[j][0] = tok < L ? ((dh[0] + dl[0]) + (dh[2] + dl[2])) * sinv * n0 : -INFINITY;
-        sc[j][1] = tok + 1 < L ? ((dh[1] + dl[1]) + (dh[3] + dl[3])) * sinv * n1 : -INFINITY;
+        float dsum[NT][4];
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            dsum[t][k] = (dh[0][t][k] + dh[1][t][k]) + (t == 0 ? dl[0][k] + dl[1][k] : 0.f);
+        // d[0], d[1]: position gq, columns 2tq, 2tq+1; d[2], d[3]: position gq+8
+        if (NT == 1) {
+          // Columns 2tq, 2tq+1 are the high part of heads 2tq, 2tq+1 (tq < 2)
+          // or the low part of heads 2(tq-2), +1 (tq >= 2); lane ^ 2 holds
+          // the other part. Lanes tq < 2 keep position gq, tq >= 2 keep gq+8.
+          const float d0 = dsum[0][0], d1 = dsum[0][1];
+          const float d2 = dsum[0][2], d3 = dsum[0][3];
+          const bool lowq = tq >= 2;
+          const float s0 = __shfl_xor_sync(0xFFFFFFFFu, lowq ? d0 : d2, 2);
+          const float s1 = __shfl_xor_sync(0xFFFFFFFFu, lowq ? d1 : d3, 2);
+          sc[mt][0][0] = (lowq ? d2 : d0) + s0;
+          sc[mt][0][1] = (lowq ? d3 : d1) + s1;
+        } else {
+          sc[mt][0][0] = dsum[0][0] + dsum[NT - 1][0];
+          sc[mt][0][1] = dsum[0][1] + dsum[NT - 1][1];
+          sc[mt][NR - 1][0] = dsum[0][2] + dsum[NT - 1][2];
+          sc[mt][NR - 1][1] = dsum[0][3] + dsum[NT - 1][3];
+        }
       }
 
-      // -- softmax statistics of the block (head = gq)
-      float mb = -INFINITY;
+      // -- scale by the K norm and query scale, mask, block maximum per head
+      float mb0 = -INFINITY, mb1 = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) mb = fmaxf(mb, fmaxf(sc[j][0], sc[j][1]));
-      mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 1));
-      mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 2));
-      const float m_new = fmaxf(m_run, mb);
-      const float alpha = exp2f(m_run - m_new);
-      l_run *= alpha;
-      m_run = m_new;
-      uint32_t pb[8];
+      for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint32_t n2 = lds32(smem, st + Gm::NKOFF + 2 * kBlk + (8 * j + 2 * tq) * 2);
-        float p[2];
+        for (int rr = 0; rr < NR; ++rr) {
+          const int p = pos_of(mt, rr);
+          const float nk = __half2float(__ushort_as_half(lds<uint16_t>(smem, st + Gm::NKOFF + 2 * p)));
+          float v0 = sc[mt][rr][0] * (sinv0 * nk);
+          float v1 = sc[mt][rr][1] * (sinv1 * nk);
+          if (partial && t0 + p >= L) v0 = v1 = -INFINITY;
+          sc[mt][rr][0] = v0;
+          sc[mt][rr][1] = v1;
+          mb0 = fmaxf(mb0, v0);
+          mb1 = fmaxf(mb1, v1);
+        }
+      // lanes holding the same heads: NT = 1 -> lane bits 1-4; NT = 2 -> bits 2-4
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float w = exp2f(sc[j][e] - m_new);
-          l_run += w;
-          const float nv = __half2float(__ushort_as_half((uint16_t)(e ? n2 >> 16 : n2 & 0xFFFF)));
-          float pv = w * nv;
-          if (sc[j][e] - mb < log2tau) {       // exp(s - M_blk) < tau, log2 domain
-            if (hv && sc[j][e] != -INFINITY) ++nskip;
-            pv = 0.f;
+      for (int o = (NT == 1 ? 2 : 4); o < 32; o <<= 1) {
+        mb0 = fmaxf(mb0, __shfl_xor_sync(0xFFFFFFFFu, mb0, o));
+        mb1 = fmaxf(mb1, __shfl_xor_sync(0xFFFFFFFFu, mb1, o));
+      }
+      const float mn0 = fmaxf(m_run[0], mb0), mn1 = fmaxf(m_run[1], mb1);
+      const float al0 = fast_exp2(m_run[0] - mn0), al1 = fast_exp2(m_run[1] - mn1);
+      m_run[0] = mn0;
+      m_run[1] = mn1;
+      l_run[0] *= al0;
+      l_run[1] *= al1;
+
+      // -- weights, gate, P' = w · nV packed as fp16 pairs (heads hs0, hs0+1)
+      uint32_t pk[4][NR];
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int rr = 0; rr < NR; ++rr) {
+          const int p = pos_of(mt, rr);
+          const float nv = __half2float(__ushort_as_half(lds<uint16_t>(smem, st + Gm::NKOFF + 2 * kBlk + 2 * p)));
+          const float s0 = sc[mt][rr][0], s1 = sc[mt][rr][1];
+          const float w0 = fast_exp2(s0 - mn0), w1 = fast_exp2(s1 - mn1);
+          l_run[0] += w0;
+          l_run[1] += w1;
+          float p0 = w0 * nv, p1 = w1 * nv;
+          const bool g0 = s0 - mb0 < log2tau, g1 = s1 - mb1 < log2tau;   // exp(s - M_blk) < tau
+          if (g0) p0 = 0.f;
+          if (g1) p1 = 0.f;
+          nskip += (g0 && hv0 && s0 != -INFINITY) + (g1 && hv1 && s1 != -INFINITY);
+          pk[mt][rr] = pack_half2(hv0 ? p0 : 0.f, hv1 ? p1 : 0.f);
+        }
+      // rescale the PV accumulators (PV layout: heads 2tq, 2tq+1)
+      {
+        float a0 = al0, a1 = al1;
+        if (NT == 1 && tq >= 2) a0 = a1 = 1.f;      // heads 4-7: padding
+        if (__any_sync(0xFFFFFFFFu, a0 != 1.f || a1 != 1.f)) {
+#pragma unroll
+          for (int r = 0; r < 8; ++r) {
+            acc[r][0] *= a0;
+            acc[r][1] *= a1;
+            acc[r][2] *= a0;
+            acc[r][3] *= a1;
           }
-          p[e] = hv ? pv : 0.f;
-        }
-        pb[j] = pack_half2(p[0], p[1]);
-      }
-      // rescale the accumulators of heads 2tq, 2tq+1
-      const float a0 = __shfl_sync(0xFFFFFFFFu, alpha, 8 * tq);
-      const float a1 = __shfl_sync(0xFFFFFFFFu, alpha, 8 * tq + 4);
-      if (__any_sync(0xFFFFFFFFu, a0 != 1.f || a1 != 1.f)) {
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          acc[r][0] *= a0;
-          acc[r][1] *= a1;
-          acc[r][2] *= a0;
-          acc[r][3] *= a1;
         }
       }
 
-      // -- P·V over four 16-position k-steps
+      // -- P·V over the four 16-position steps
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint32_t b0 = pb[2 * kk], b1 = pb[2 * kk + 1];
-        if (!__any_sync(0xFFFFFFFFu, (b0 | b1) != 0u)) continue;   // whole step gated
+      for (int mt = 0; mt < 4; ++mt) {
+        uint32_t x0, x1;   // P' of positions 0-7 / 8-15 x heads 0-7, standard layout
+        if (NT == 1) {
+          const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, pk[mt][0], 2);
+          x0 = tq < 2 ? pk[mt][0] : 0u;
+          x1 = tq < 2 ? other : 0u;
+        } else {
+          x0 = pk[mt][0];
+          x1 = pk[mt][NR - 1];
+        }
+        if (!__any_sync(0xFFFFFFFFu, (x0 | x1) != 0u)) continue;   // whole step gated
+        const uint32_t b0 = transpose8x8(x0), b1 = transpose8x8(x1);
         if (BV == 2) {
-          const uint32_t vrow = st + Gm::KB + (16 * kk + 2 * tq) * Gm::RVS + 4 * gq;
-          const uint32_t wA = lds32(smem, vrow), wB = lds32(smem, vrow + Gm::RVS);
-          const uint32_t wC = lds32(smem, vrow + 8 * Gm::RVS), wD = lds32(smem, vrow + 9 * Gm::RVS);
+          const uint32_t vrow = st + Gm::KB + (16 * mt + 2 * tq) * Gm::RVS + 4 * gq;
+          const uint32_t wA = lds<uint32_t>(smem, vrow), wB = lds<uint32_t>(smem, vrow + Gm::RVS);
+          const uint32_t wC = lds<uint32_t>(smem, vrow + 8 * Gm::RVS);
+          const uint32_t wD = lds<uint32_t>(smem, vrow + 9 * Gm::RVS);
           const uint32_t xab[2] = {__byte_perm(wA, wB, 0x5140), __byte_perm(wA, wB, 0x7362)};
           const uint32_t xcd[2] = {__byte_perm(wC, wD, 0x5140), __byte_perm(wC, wD, 0x7362)};
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
-            // original bytes 2·half (low 16 bits) and 2·half+1 (high 16 bits)
 #pragma unroll
             for (int odd = 0; odd < 2; ++odd) {
-              const int f0 = 4 * odd, f1 = 4 * odd + 2;   // fields of coords 2r, 2r+1
+              const int f0 = 4 * odd, f1 = 4 * odd + 2;   // codes of coords 2r, 2r+1
               const uint32_t s0 = ((xab[half] >> f0) & 0x03030303u) * 0x11u + 0x40404040u;
               const uint32_t s1 = ((xab[half] >> f1) & 0x03030303u) * 0x11u + 0x40404040u;
               const uint32_t s2 = ((xcd[half] >> f0) & 0x03030303u) * 0x11u + 0x40404040u;
@@ -555,33 +678,30 @@ attend_kernel(const __grid_constant__ AttendArgs a,
               for (int hb = 0; hb < 2; ++hb) {
                 const int r = 2 * (2 * half + hb) + odd;
                 const int sh = 16 * hb;
-                const uint32_t va0 = __byte_perm(vt_lo, vt_hi, s0 >> sh);
-                const uint32_t va1 = __byte_perm(vt_lo, vt_hi, s1 >> sh);
-                const uint32_t va2 = __byte_perm(vt_lo, vt_hi, s2 >> sh);
-                const uint32_t va3 = __byte_perm(vt_lo, vt_hi, s3 >> sh);
-                mma16816(acc[r], va0, va1, va2, va3, b0, b1);
+                mma16816(acc[r], __byte_perm(vt_lo, vt_hi, s0 >> sh),
+                         __byte_perm(vt_lo, vt_hi, s1 >> sh), __byte_perm(vt_lo, vt_hi, s2 >> sh),
+                         __byte_perm(vt_lo, vt_hi, s3 >> sh), b0, b1);
               }
             }
           }
         } else {
           uint32_t v0[BV + 1], v1[BV + 1];
-          const uint32_t r0p = st + Gm::KB + (16 * kk + gq) * Gm::RVS + 4 * BV * tq;
+          const uint32_t r0p = st + Gm::KB + (16 * mt + gq) * Gm::RVS + 4 * BV * tq;
           const uint32_t r1p = r0p + 8 * Gm::RVS;
 #pragma unroll
           for (int w = 0; w < BV; ++w) {
-            v0[w] = lds32(smem, r0p + 4 * w);
-            v1[w] = lds32(smem, r1p + 4 * w);
+            v0[w] = lds<uint32_t>(smem, r0p + 4 * w);
+            v1[w] = lds<uint32_t>(smem, r1p + 4 * w);
           }
           v0[BV] = v1[BV] = 0;
-          const uint32_t lo = lutV_base + lane * 4;
 #pragma unroll
           for (int r = 0; r < 8; ++r) {
-            const uint32_t x0 = lds32(smem, lut_off<7>(pair_field<BV>(v0, 2 * r), lo));
-            const uint32_t x1 = lds32(smem, lut_off<7>(pair_field<BV>(v0, 2 * r + 1), lo));
-            const uint32_t x2 = lds32(smem, lut_off<7>(pair_field<BV>(v1, 2 * r), lo));
-            const uint32_t x3 = lds32(smem, lut_off<7>(pair_field<BV>(v1, 2 * r + 1), lo));
-            mma16816(acc[r], transpose8x8(x0), transpose8x8(x1), transpose8x8(x2),
-                     transpose8x8(x3), b0, b1);
+            const uint32_t y0 = lds<uint32_t>(smem, pair_code_shifted<BV, 7>(v0, 2 * r) | lbV);
+            const uint32_t y1 = lds<uint32_t>(smem, pair_code_shifted<BV, 7>(v0, 2 * r + 1) | lbV);
+            const uint32_t y2 = lds<uint32_t>(smem, pair_code_shifted<BV, 7>(v1, 2 * r) | lbV);
+            const uint32_t y3 = lds<uint32_t>(smem, pair_code_shifted<BV, 7>(v1, 2 * r + 1) | lbV);
+            mma16816(acc[r], transpose8x8(y0), transpose8x8(y1), transpose8x8(y2),
+                     transpose8x8(y3), b0, b1);
           }
         }
       }
@@ -589,15 +709,27 @@ attend_kernel(const __grid_constant__ AttendArgs a,
     }
     cp_async_wait<0>();
 
+    // ---- per-warp softmax sums over the lanes holding the same heads
+#pragma unroll
+    for (int o = (NT == 1 ? 2 : 4); o < 32; o <<= 1) {
+      l_run[0] += __shfl_xor_sync(0xFFFFFFFFu, l_run[0], o);
+      l_run[1] += __shfl_xor_sync(0xFFFFFFFFu, l_run[1], o);
+    }
+
     // ---- merge the warps of this segment
-    l_run += __shfl_xor_sync(0xFFFFFFFFu, l_run, 1);
-    l_run += __shfl_xor_sync(0xFFFFFFFFu, l_run, 2);
+    constexpr int WS = kMaxGroup * kHeadDim + 2 * kMaxGroup;
     __syncthreads();                                  // all warps done with the ring
     {
-      float* wm = merge + warp * (kMaxGroup * kHeadDim + 2 * kMaxGroup);
-      if (tq == 0 && hv) {
-        wm[kMaxGroup * kHeadDim + gq] = nw > 0 ? m_run : -INFINITY;
-        wm[kMaxGroup * kHeadDim + kMaxGroup + gq] = nw > 0 ? l_run : 0.f;
+      float* wm = merge + warp * WS;
+      if (gq == 0 && (NT == 2 || tq < 2)) {
+        if (hv0) {
+          wm[kMaxGroup * kHeadDim + hs0] = nw > 0 ? m_run[0] : -INFINITY;
+          wm[kMaxGroup * kHeadDim + kMaxGroup + hs0] = nw > 0 ? l_run[0] : 0.f;
+        }
+        if (hv1) {
+          wm[kMaxGroup * kHeadDim + hs0 + 1] = nw > 0 ? m_run[1] : -INFINITY;
+          wm[kMaxGroup * kHeadDim + kMaxGroup + hs0 + 1] = nw > 0 ? l_run[1] : 0.f;
+        }
       }
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
@@ -614,25 +746,29 @@ attend_kernel(const __grid_constant__ AttendArgs a,
       }
     }
     __syncthreads();
-    constexpr int WS = kMaxGroup * kHeadDim + 2 * kMaxGroup;
+    // per-head maximum and sum over the warps, then per-(warp, head) weights
+    float* wt = miscf + kMiscWt;                      // [kWarps][GQ] <= 96 floats
     if (tid < GQ) {
       float mx = -INFINITY;
       for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, merge[w * WS + kMaxGroup * kHeadDim + tid]);
       float ls = 0.f;
-      for (int w = 0; w < kWarps; ++w)
-        ls += merge[w * WS + kMaxGroup * kHeadDim + kMaxGroup + tid] *
-              exp2f(merge[w * WS + kMaxGroup * kHeadDim + tid] - mx);
+      for (int w = 0; w < kWarps; ++w) {
+        const float mw = merge[w * WS + kMaxGroup * kHeadDim + tid];
+        const float f = mw == -INFINITY ? 0.f : exp2f(mw - mx);
+        wt[w * GQ + tid] = f;
+        ls += merge[w * WS + kMaxGroup * kHeadDim + kMaxGroup + tid] * f;
+      }
       miscf[kMiscM + tid] = mx;
       miscf[kMiscL + tid] = ls;
     }
     __syncthreads();
     for (int i = tid; i < GQ * kHeadDim; i += kThreads) {
       const int h = i / kHeadDim;
-      const float mx = miscf[kMiscM + h];
       float s = 0.f;
+#pragma unroll
       for (int w = 0; w < kWarps; ++w) {
-        const float mw = merge[w * WS + kMaxGroup * kHeadDim + h];
-        if (mw != -INFINITY) s += merge[w * WS + i] * exp2f(mw - mx);
+        const float f = wt[w * GQ + h];
+        if (f != 0.f) s += merge[w * WS + i] * f;
       }
       fin[i] = s;
     }
@@ -659,27 +795,54 @@ attend_kernel(const __grid_constant__ AttendArgs a,
       __syncthreads();
       finalize = misc[kMiscLast] != 0;
       if (finalize) {
+        // Merge the n_parts partials of this sequence. Their (max, sum) pairs
+        // are read in one parallel pass and turned into weights in shared
+        // memory (the ring area is free here: n_parts <= 1024 CTAs x 8 heads
+        // x 2 floats = 64 KB); the accumulators are then summed with up to 16
+        // independent loads in flight per thread.
         __threadfence();
         const float* s0 = a.slots + (size_t)(c_first + sigma) * GQ * kSlotFloats;
         const size_t stride = (size_t)GQ * kSlotFloats;
+        float* pm = merge;                       // [n_parts][GQ] max, then weight
+        float* pl = merge + n_parts * GQ;        // [n_parts][GQ] sum
+        for (int j = tid; j < n_parts * GQ; j += kThreads) {
+          const int p = j / GQ, h = j - p * GQ;
+          pm[j] = __ldcg(s0 + p * stride + GQ * kHeadDim + 2 * h);
+          pl[j] = __ldcg(s0 + p * stride + GQ * kHeadDim + 2 * h + 1);
+        }
+        __syncthreads();
         if (tid < GQ) {
           float mx = -INFINITY;
-          for (int p = 0; p < n_parts; ++p) mx = fmaxf(mx, __ldcg(s0 + p * stride + GQ * kHeadDim + 2 * tid));
+          for (int p = 0; p < n_parts; ++p) mx = fmaxf(mx, pm[p * GQ + tid]);
           float ls = 0.f;
-          for (int p = 0; p < n_parts; ++p)
-            ls += __ldcg(s0 + p * stride + GQ * kHeadDim + 2 * tid + 1) *
-                  exp2f(__ldcg(s0 + p * stride + GQ * kHeadDim + 2 * tid) - mx);
+          for (int p = 0; p < n_parts; ++p) ls += pl[p * GQ + tid] * exp2f(pm[p * GQ + tid] - mx);
           miscf[kMiscM + tid] = mx;
           miscf[kMiscL + tid] = ls;
         }
         __syncthreads();
+        for (int j = tid; j < n_parts * GQ; j += kThreads)
+          pm[j] = exp2f(pm[j] - miscf[kMiscM + j % GQ]);
+        __syncthreads();
         for (int i = tid; i < GQ * kHeadDim; i += kThreads) {
           const int h = i / kHeadDim;
-          const float mx = miscf[kMiscM + h];
-          float s = 0.f;
-          for (int p = 0; p < n_parts; ++p)
-            s += __ldcg(s0 + p * stride + i) * exp2f(__ldcg(s0 + p * stride + GQ * kHeadDim + 2 * h) - mx);
-          fin[i] = s;
+          float sum = 0.f;
+          int p = 0;
+          for (; p + 16 <= n_parts; p += 16) {
+            float v[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) v[k] = __ldcg(s0 + (p + k) * stride + i);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) sum += v[k] * pm[(p + k) * GQ + h];
+          }
+          for (; p + 4 <= n_parts; p += 4) {
+            float v[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) v[k] = __ldcg(s0 + (p + k) * stride + i);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) sum += v[k] * pm[(p + k) * GQ + h];
+          }
+          for (; p < n_parts; ++p) sum += __ldcg(s0 + p * stride + i) * pm[p * GQ + h];
+          fin[i] = sum;
         }
         if (tid == 0) atomicExch(a.counters + sigma, 0);
         __syncthreads();
@@ -730,22 +893,29 @@ int sm_count() {
   return cached[dev];
 }
 
-template <int BK, int BV>
-cudaError_t launch_pair(const AttendArgs& a, const Codebook& cbk, const Codebook& cbv,
-                        const SignMask& sm, int n_ctas, cudaStream_t stream) {
+template <int BK, int BV, int NT>
+cudaError_t launch_one(const AttendArgs& a, const Codebook& cbk, const Codebook& cbv,
+                       const SignMask& sm, int n_ctas, cudaStream_t stream) {
   using Gm = Geo<BK, BV>;
   static bool configured[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || !configured[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(attend_kernel<BK, BV>,
+    const cudaError_t e = cudaFuncSetAttribute(attend_kernel<BK, BV, NT>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, Gm::SMEM);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }
   const int grid = n_ctas > 0 ? n_ctas : sm_count();
-  attend_kernel<BK, BV><<<grid, kThreads, Gm::SMEM, stream>>>(a, cbk, cbv, sm);
+  attend_kernel<BK, BV, NT><<<grid, kThreads, Gm::SMEM, stream>>>(a, cbk, cbv, sm);
   return cudaGetLastError();
+}
+
+template <int BK, int BV>
+cudaError_t launch_pair(const AttendArgs& a, const Codebook& cbk, const Codebook& cbv,
+                        const SignMask& sm, int n_ctas, cudaStream_t stream) {
+  return a.gqa <= 4 ? launch_one<BK, BV, 1>(a, cbk, cbv, sm, n_ctas, stream)
+                    : launch_one<BK, BV, 2>(a, cbk, cbv, sm, n_ctas, stream);
 }
 
 }  // namespace
