@@ -8,8 +8,11 @@
 // weight are left out (block-local rule, include/tq.h).
 //
 // Work decomposition. The cache is a flat list of 64-position blocks in
-// (batch, kv head, block) order; CTA c of Geff = min(grid, #blocks) owns
-// blocks [c·NB/Geff, (c+1)·NB/Geff). A CTA walks the (batch, kv head)
+// (batch, kv head, block) order; CTA c of Geff owns blocks
+// [c·NB/Geff, (c+1)·NB/Geff). Geff = min(grid, #blocks), except that when all
+// S (batch, kv head) segments have the same block count and S <= grid, Geff
+// is the largest multiple of S within the grid (at most one CTA per block),
+// so every CTA stays inside one segment. A CTA walks the (batch, kv head)
 // segments of its range; its warps split each segment, merge in shared
 // memory, and either write the output (segment = whole sequence) or leave a
 // partial in a workspace slot; the last CTA to finish a sequence (atomic
@@ -85,7 +88,7 @@ struct Geo {
 // misc words
 constexpr int kMiscSeg = 0;      // b, g, blk0, nseg, nb, L
 constexpr int kMiscLast = 8;     // last-CTA flag
-constexpr int kMiscNB = 9;       // flat block count (lo, hi)
+constexpr int kMiscNB = 9;       // flat block count (lo, hi), common length
 constexpr int kMiscState = 12;   // scan state: sb, sP (lo, hi)
 constexpr int kMiscQInv = 16;    // 8 floats: 1/(query scale · kKScale)
 constexpr int kMiscM = 32;       // 8 floats: merged max
@@ -288,19 +291,29 @@ attend_kernel(const __grid_constant__ AttendArgs a,
     }
   }
 
-  // ---- flat block count
+  // ---- flat block count, and whether all sequences have the same length
   if (warp == 0) {
     long long tot = 0;
+    int nmin = 0x7FFFFFFF, nmax = 0;
     for (int b0 = 0; b0 < B; b0 += 32) {
-      int nb = b0 == 0 ? (len0 + kBlk - 1) / kBlk : ((b0 + lane < B) ? seq_blocks(a, b0 + lane) : 0);
+      const bool in = b0 + lane < B;
+      const int nb = b0 == 0 ? (len0 + kBlk - 1) / kBlk : (in ? seq_blocks(a, b0 + lane) : 0);
+      int sum = nb, lo = in ? nb : 0x7FFFFFFF, hi = nb;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) nb += __shfl_xor_sync(0xFFFFFFFFu, nb, o);
-      tot += nb;
+      for (int o = 16; o > 0; o >>= 1) {
+        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+        lo = min(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, o));
+        hi = max(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, o));
+      }
+      tot += sum;
+      nmin = min(nmin, lo);
+      nmax = max(nmax, hi);
     }
     if (lane == 0) {
       const long long nbt = tot * H;
       misc[kMiscNB] = (int)(nbt & 0xFFFFFFFF);
       misc[kMiscNB + 1] = (int)(nbt >> 32);
+      misc[kMiscNB + 2] = nmin == nmax ? nmax : -1;   // common length in blocks
       misc[kMiscState] = 0;
       misc[kMiscState + 1] = 0;
       misc[kMiscState + 2] = 0;
@@ -308,9 +321,16 @@ attend_kernel(const __grid_constant__ AttendArgs a,
   }
   __syncthreads();
   const long long NB = (long long)(unsigned)misc[kMiscNB] | ((long long)misc[kMiscNB + 1] << 32);
-  // Balance over Geff = min(grid, NB) CTAs so every participating CTA owns at
-  // least one block; the partial count of a sequence relies on it.
-  const int Geff = (int)min((long long)Gc, NB);
+  // Balance over Geff CTAs, each owning at least one block (the partial count
+  // of a sequence relies on it): min(grid, NB), or, when every (sequence, kv
+  // head) segment has the same length and there are no more segments than
+  // CTAs, a multiple of the segment count so that no CTA spans two segments.
+  int Geff = (int)min((long long)Gc, NB);
+  {
+    const int common = misc[kMiscNB + 2];
+    const long long S = (long long)B * H;
+    if (common > 0 && S <= Gc) Geff = (int)(S * min((long long)(Gc / S), (long long)common));
+  }
   const long long r0 = cta < Geff ? NB * cta / Geff : 0;
   const long long r1 = cta < Geff ? NB * (cta + 1) / Geff : 0;
   long long pos = r0;

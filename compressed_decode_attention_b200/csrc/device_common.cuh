@@ -72,3 +72,39 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits(float x) {
 }
 
 }  // namespace tq
+
+namespace tq {
+
+// Packed two-wide fp32 arithmetic (sm_100: add/sub/fma .f32x2), round to
+// nearest per lane: bit-identical to the scalar operations.
+__device__ __forceinline__ float2 f2add(float2 a, float2 b) {
+  float2 r;
+  asm("{.reg .b64 ra, rb, rc;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rc, ra, rb;\n\tmov.b64 {%0, %1}, rc;}\n"
+      : "=f"(r.x), "=f"(r.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+__device__ __forceinline__ float2 f2sub(float2 a, float2 b) {
+  float2 r;
+  asm("{.reg .b64 ra, rb, rc;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rc, ra, rb;\n\tmov.b64 {%0, %1}, rc;}\n"
+      : "=f"(r.x), "=f"(r.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+__device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) {
+  float2 r;
+  asm("{.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;}\n"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return r;
+}
+
+// 0xFFFFFFFF if a >= b else 0 (one compare-and-set).
+__device__ __forceinline__ uint32_t set_ge(float a, float b) {
+  uint32_t r;
+  asm("set.ge.u32.f32 %0, %1, %2;\n" : "=r"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+}  // namespace tq

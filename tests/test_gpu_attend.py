@@ -106,6 +106,23 @@ def test_cta_counts_ragged_batch(n_ctas):
     assert st == 4
 
 
+@pytest.mark.parametrize("n_ctas", [5, 12, 37, 300, 0])
+def test_cta_counts_equal_block_counts(n_ctas):
+    """Every (sequence, kv head) segment has 11 blocks (lengths 641..704):
+    the partition then aligns CTA ranges with segments when the grid allows
+    (5 CTAs for 12 segments does not, 37 gives three CTAs per segment over
+    11 blocks, 300 one block per CTA)."""
+    rng = np.random.default_rng(100 + n_ctas)
+    ctx = np.array([704, 641, 700, 650, 683, 704])
+    pk, nk, pv, nv = _small_cache(4, 2, len(ctx), 2, 768, ctx, 22, rng)
+    qb = S.f16_bits(rng.standard_normal((len(ctx), 8, 128)))
+    q64 = codec.promote(qb, "f16")
+    want, _ = oracle_attend(q64, pk, nk, pv, nv, ctx, 4, 4, 2, 22)
+    got, st, _ = gpu_attend(qb, "f16", pk, nk, pv, nv, ctx, 4, 4, 2, 22, n_ctas=n_ctas)
+    assert np.abs(got - want).max() <= ATOL
+    assert st == 0
+
+
 def test_workspace_counters_return_to_zero_and_calls_repeat():
     import torch
     import compressed_decode_attention_b200 as tq
