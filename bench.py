@@ -268,40 +268,33 @@ def run_gpu(args, rank, world, local_rank):
     ws_bytes = tq.tq_attend_workspace_size(1, w.n_q_heads, cap, d)
     ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=device)
 
-    def step(events=None):
+    def attend_layer(l):
+        tq.tq_attend(q[l], tq.TQ_F16, caches.pk[l], caches.nk[l], caches.pv[l], caches.nv[l],
+                     ctx_dev, 1, w.n_q_heads, w.gqa, d, w.bits_k, w.bits_v, seed, cap, 0.0, 0,
+                     ws, ws_bytes, outs[l], tq.TQ_F16, dev_status=status, stream=stream)
+
+    def step():
         for l in range(L):
             tq.tq_encode(kv_new[l], tq.TQ_F16, 1, H, d, w.bits_k, w.bits_v, seed,
                          caches.pk[l], caches.pv[l], caches.nk[l], caches.nv[l], cap, ctx - 1,
                          status, stream)
-            if events is not None:
-                events[l][0].record(stream)
-            tq.tq_attend(q[l], tq.TQ_F16, caches.pk[l], caches.nk[l], caches.pv[l], caches.nv[l],
-                         ctx_dev, 1, w.n_q_heads, w.gqa, d, w.bits_k, w.bits_v, seed, cap, 0.0, 0,
-                         ws, ws_bytes, outs[l], tq.TQ_F16, dev_status=status, stream=stream)
-            if events is not None:
-                events[l][1].record(stream)
+            attend_layer(l)
 
     kernels_per_step = L * 2   # encode + attend per layer
 
-    def capture(with_events):
-        evs = None
-        if with_events:
-            evs = [(torch.cuda.Event(enable_timing=True, external=True),
-                    torch.cuda.Event(enable_timing=True, external=True)) for _ in range(L)]
+    def capture(fn):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            step(evs)
-        return g, evs
+            fn()
+        return g
 
     with torch.cuda.stream(stream):
         step()                       # eager warm-up of the exact sequence
     torch.cuda.synchronize()
-    warm_graph, _ = capture(False)
-    timed = [capture(True) for _ in range(args.steps)]
+    step_graph = capture(step)
     torch.cuda.synchronize()
-
     for _ in range(args.warmup):
-        warm_graph.replay()
+        step_graph.replay()
     torch.cuda.synchronize()
 
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -310,15 +303,35 @@ def run_gpu(args, rank, world, local_rank):
     with ClockSampler(local_rank) as clk:
         with torch.cuda.stream(stream):
             t0.record(stream)
-            for g, _ in timed:
-                g.replay()
+            for _ in range(args.steps):
+                step_graph.replay()
             t1.record(stream)
         torch.cuda.synchronize()
     ms_total = t0.elapsed_time(t1)
     ms_step = reduce_max(ms_total / args.steps, device)
-    attend_ms = [e[0].elapsed_time(e[1]) for _, evs in timed for e in evs]
-    attend_ms_mean = reduce_max(float(np.mean(attend_ms)), device)
     launches += kernels_per_step * args.steps
+
+    # ---------------- the attention kernel alone: per-launch time = a graph
+    # of the L layers' launches (distinct caches, larger than L2) / L
+    def attend_all():
+        for l in range(L):
+            attend_layer(l)
+
+    attend_graph = capture(attend_all)
+    for _ in range(args.warmup):
+        attend_graph.replay()
+    torch.cuda.synchronize()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(device)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        a0.record(stream)
+        for _ in range(args.steps):
+            attend_graph.replay()
+        a1.record(stream)
+    torch.cuda.synchronize()
+    attend_ms_mean = reduce_max(a0.elapsed_time(a1) / (args.steps * L), device)
+    launches += L * args.steps
 
     # ---------------- end to end: host inputs in, host output back, every step
     q_host = torch.empty((L, 1, w.n_q_heads, d), dtype=torch.float16).pin_memory()
@@ -326,7 +339,7 @@ def run_gpu(args, rank, world, local_rank):
     out_host = torch.empty((L, 1, w.n_q_heads, d), dtype=torch.float16).pin_memory()
     q_host.copy_(torch.stack([x.cpu() for x in q]))
     kv_host.copy_(torch.stack([x.cpu() for x in kv_new]))
-    e2e_graph, _ = capture(False)
+    e2e_graph = capture(step)
     torch.cuda.synchronize()
 
     def e2e_step():
@@ -383,7 +396,8 @@ def run_gpu(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                      "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
-                     "kernel": "tq_attend (attend_kernel, one launch)",
+                     "kernel": "tq_attend (attend_kernel): per-launch time from a CUDA graph of "
+                               f"{L} back-to-back launches over distinct layer caches, / {L}",
                      "bytes_per_launch": per_layer_attend,
                      "launch_ms": round(attend_ms_mean, 5),
                      "traffic": traffic["traffic_bytes_per_launch"] if traffic else None},
@@ -404,8 +418,7 @@ def run_gpu(args, rank, world, local_rank):
                    "gpu_launches": enc_launches},
         "device_status": st,
     }
-    for g, _ in timed:
-        del g
+    del step_graph, attend_graph, e2e_graph
     return res
 
 

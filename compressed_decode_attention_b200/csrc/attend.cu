@@ -13,24 +13,27 @@
 // S (batch, kv head) segments have the same block count and S <= grid, Geff
 // is the largest multiple of S within the grid (at most one CTA per block),
 // so every CTA stays inside one segment. A CTA walks the (batch, kv head)
-// segments of its range; its warps split each segment, merge in shared
-// memory, and either write the output (segment = whole sequence) or leave a
-// partial in a workspace slot; the last CTA to finish a sequence (atomic
-// counter, no waiting) merges the partials and writes the output. No separate
-// combine launch, no spin-waits.
+// segments of its range. Its 12 warps split each segment in whole blocks,
+// merge in shared memory, and
+// either write the output (segment = whole sequence) or leave a partial in a
+// workspace slot; the last CTA to finish a sequence (atomic counter, no
+// waiting) merges the partials and writes the output. No separate combine
+// launch, no spin-waits on other CTAs.
 //
-// Per warp and 64-position block (GQA group of g <= 8 query heads), in four
-// 16-position steps:
-//   stage   cp.async of the packed K/V rows and fp16 norms (per-warp ring)
-//   scores  mma.m16n8k16, fp16 in, fp32 accumulate. A = K codebook values of
-//           16 positions (rows) x 16 coordinates, read as fp16 high/low pairs
-//           from a shared table indexed by the packed byte (one copy per
-//           half-warp lane); B = rotated query, fp16 high and low parts in
-//           the 8 columns (g <= 4: 4 heads x {high, low}; g <= 8: two column
-//           tiles). K high, K low and query low are summed, so scores keep
-//           ~22 significant bits (fp16-only operands measured up to 1.2e-2
-//           output error with x20 outlier channels).
-//   softmax fp32, log2 domain; block maximum = sparse-V reference.
+// Per warp and chunk of up to 64 positions (GQA group of g <= 8 query heads),
+// in four 16-position steps:
+//   stage   bulk copies (cp.async.bulk, one lane) of the packed K/V rows and
+//           fp16 norms into a per-warp ring of shared-memory slots, each
+//           completed on its own mbarrier (bounded wait)
+//   scores  mma.m16n8k16, fp16 in, fp32 accumulate, per 8 positions: A rows
+//           0-7 = K codebook high parts, rows 8-15 = low parts of the same
+//           positions (one shared-table entry per packed byte fills two
+//           fragment registers); B = rotated query, fp16 high and low parts
+//           in the 8 columns (g <= 4: 4 heads x {high, low}; g <= 8: two
+//           column tiles). K high, K low and query low are summed, so scores
+//           keep ~22 significant bits (fp16-only operands measured up to
+//           1.2e-2 output error with x20 outlier channels).
+//   softmax fp32, log2 domain; chunk maximum = sparse-V block maximum.
 //   PV      mma.m16n8k16: A = V codebook values (fp16), coordinates x
 //           positions; B = softmax weight x V norm (fp16), moved from the
 //           score layout with movmatrix. V2: position pairs by byte permutes
@@ -49,6 +52,10 @@ constexpr int kBlk = kGateBlock;                // positions per block
 constexpr float kLog2e = 1.44269504088896340736f;
 constexpr float kKScale = 256.f;                // K codebook scale inside the MMA
 constexpr int kSmemBudget = 227 * 1024;
+constexpr int kMaxStages = 3;                   // ring slots per warp
+constexpr int kMergeChunk = 16;                 // partials per round of loads
+// Give up on a staged-data wait after this many cycles (~1 s at 2 GHz).
+constexpr long long kWaitLimitCycles = 2000000000LL;
 
 constexpr int ceil_pow2(int x) {
   int p = 1;
@@ -56,11 +63,31 @@ constexpr int ceil_pow2(int x) {
   return p;
 }
 
+// misc words
+constexpr int kMiscSeg = 0;      // b, g, blk0, nseg, nb, L
+constexpr int kMiscLast = 8;     // last-CTA flag
+constexpr int kMiscNB = 9;       // flat block count (lo, hi), common length
+constexpr int kMiscState = 12;   // scan state: sb, sP (lo, hi)
+constexpr int kMiscQInv = 16;    // 8 floats: 1/(query scale · kKScale)
+constexpr int kMiscM = 32;       // 8 floats: merged max
+constexpr int kMiscL = 40;       // 8 floats: merged sum
+constexpr int kMiscCb = 64;      // 32 words: staged codebooks
+constexpr int kMiscWt = 128;     // kWarps x 8 floats: per-warp merge weights
+constexpr int kMiscWords = 256;  // Geo::MISC / 4
+// Per-warp merge buffer (floats): accumulators (in register order 32 per
+// lane at a stride of kMergeLane, which keeps 16-byte stores of consecutive
+// lanes on distinct banks; or in output order), then per-head max and sum.
+constexpr int kMergeLane = 36;
+constexpr int kMergeM = 32 * kMergeLane;
+constexpr int kMergeL = kMergeM + kMaxGroup;
+constexpr int kMergeStride = kMergeL + kMaxGroup;
+static_assert(kMiscWt + kWarps * kMaxGroup <= kMiscWords, "misc words");
+
 template <int BK, int BV>
 struct Geo {
   static constexpr int RK = 16 * BK;                    // packed K row bytes
   static constexpr int RV = 16 * BV;
-  static constexpr int RVS = BV == 2 ? RV + 16 : RV;    // V row stride in smem
+  static constexpr int RVS = RV;                        // V row stride in smem
   static constexpr int KB = kBlk * RK;
   static constexpr int VB = kBlk * RVS;
   static constexpr int NKOFF = KB + VB;
@@ -75,28 +102,17 @@ struct Geo {
   static constexpr int QOFF = LUTV_OFF + LUTV;
   static constexpr int QS = kMaxGroup * kHeadDim * 2 * 2;  // q~ high and low, fp16
   static constexpr int MISC = 1024;                     // kMiscWords words
-  static constexpr int FIXED = QOFF + QS + MISC;
+  static constexpr int MBAR = kWarps * kMaxStages * 8;  // per-warp ring barriers
+  static constexpr int FIXED = QOFF + QS + MISC + MBAR;
   static constexpr int NFIT = (kSmemBudget - FIXED) / (kWarps * STAGE);
-  static constexpr int NSTAGE = NFIT > 3 ? 3 : NFIT;
-  static constexpr int MERGE = kWarps * (kMaxGroup * kHeadDim + 2 * kMaxGroup) * 4;
+  static constexpr int NSTAGE = NFIT > kMaxStages ? kMaxStages : NFIT;
+  static constexpr int MERGE = kWarps * kMergeStride * 4;
   static constexpr int RING = NSTAGE * kWarps * STAGE;
   static constexpr int SMEM = FIXED + (RING > MERGE ? RING : MERGE);
   static_assert(NSTAGE >= 1, "stage ring does not fit");
   static_assert(SMEM <= kSmemBudget, "shared memory budget");
 };
 
-// misc words
-constexpr int kMiscSeg = 0;      // b, g, blk0, nseg, nb, L
-constexpr int kMiscLast = 8;     // last-CTA flag
-constexpr int kMiscNB = 9;       // flat block count (lo, hi), common length
-constexpr int kMiscState = 12;   // scan state: sb, sP (lo, hi)
-constexpr int kMiscQInv = 16;    // 8 floats: 1/(query scale · kKScale)
-constexpr int kMiscM = 32;       // 8 floats: merged max
-constexpr int kMiscL = 40;       // 8 floats: merged sum
-constexpr int kMiscCb = 64;      // 32 words: staged codebooks
-constexpr int kMiscWt = 128;     // kWarps x 8 floats: per-warp merge weights
-constexpr int kMiscWords = 256;  // Geo::MISC / 4
-static_assert(kMiscWt + kWarps * kMaxGroup <= kMiscWords, "misc words");
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1,
                                          uint32_t a2, uint32_t a3, uint32_t b0,
@@ -133,6 +149,44 @@ __device__ __forceinline__ void cp_async_commit() {
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// Shared-memory barrier with a transaction count, completed by bulk copies.
+__device__ __forceinline__ void mbar_init(uint32_t bar) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(done) : "r"(bar), "r"(parity) : "memory");
+  return done != 0;
+}
+// Slow path of mbar_wait, out of line: keeps polling until the phase
+// completes or kWaitLimitCycles have passed.
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try(bar, parity))
+    if (clock64() - t0 > kWaitLimitCycles) return false;
+  return true;
+}
+// Waits for the phase with the given parity to complete; false if it does
+// not within kWaitLimitCycles.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  return mbar_try(bar, parity) || mbar_wait_slow(bar, parity);
+}
+// Bulk copy global -> this CTA's shared memory (16-byte aligned, size a
+// multiple of 16), completing on `bar`.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+      ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
 
 template <typename T>
@@ -193,6 +247,23 @@ __device__ __forceinline__ int pv_coord(int r, int m) {
   return 32 * ((m & 7) >> 1) + 4 * r + (m & 1) + 2 * (m >> 3);
 }
 
+// Position of output (head h, coordinate c) in a warp's accumulators as
+// stored lane-major (register acc[r][k] of a lane at 4r + k):
+// the inverse of pv_coord together with the head columns 2tq, 2tq + 1.
+template <int BV>
+__device__ __forceinline__ int pv_slot(int c, int h) {
+  int m, r;
+  if (BV == 2) {
+    m = (c >> 4) + 8 * (c & 1);
+    r = (c & 15) >> 1;
+  } else {
+    m = 2 * (c >> 5) + (c & 1) + 8 * ((c >> 1) & 1);
+    r = (c & 31) >> 2;
+  }
+  const int lane = 4 * (m & 7) + (h >> 1);
+  return lane * kMergeLane + 4 * r + (h & 1) + 2 * (m >> 3);
+}
+
 // (pair code p of a lane's chunk of packed words) << SHIFT, for a table
 // whose entries are 2^SHIFT bytes apart. Codes are 2·BITS bits wide
 // (coordinates 2p, 2p+1), little-endian in the chunk.
@@ -205,6 +276,17 @@ __device__ __forceinline__ uint32_t pair_code_shifted(const uint32_t* w, int p) 
   if (off + FB > 32) return (__funnelshift_r(w[k], w[k + 1], off) << SHIFT) & MASK;
   if (off >= SHIFT) return (w[k] >> (off - SHIFT)) & MASK;
   return (w[k] << (SHIFT - off)) & MASK;
+}
+
+// Byte offset of the K table entry for pair code p of a lane's chunk (entries
+// 128 bytes apart). For 4-bit codes the pair code is a whole byte: one byte
+// permute and one multiply-add; narrower codes straddle bytes.
+template <int BK>
+__device__ __forceinline__ uint32_t k_entry(const uint32_t* w, int p) {
+  if constexpr (BK == 4)
+    return (uint32_t)__byte_perm(w[p >> 2], 0u, 0x4440u | (uint32_t)(p & 3)) * 128u;
+  else
+    return pair_code_shifted<BK, 7>(w, p);
 }
 
 template <int BK, int BV, int NT>
@@ -226,19 +308,30 @@ attend_kernel(const __grid_constant__ AttendArgs a,
   float* merge = reinterpret_cast<float*>(smem + Gm::FIXED);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // this warp's ring barriers: one per slot, phases counted over all blocks
+  // the warp stages in this launch (jdone)
+  const uint32_t wbar = smem_addr(smem) + Gm::QOFF + Gm::QS + Gm::MISC + warp * kMaxStages * 8;
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < Gm::NSTAGE; ++s) mbar_init(wbar + 8 * s);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  __syncwarp();
+  int jdone = 0;
+  bool stalled = false;                       // a staged-data wait gave up
   const int gq = lane >> 2, tq = lane & 3;
   const int H = a.n_kv_heads, GQ = a.gqa, B = a.batch;
   const int Gc = gridDim.x, cta = blockIdx.x;   // Gc <= kMaxCtas (host check)
   const uint32_t lbK = (lane & 15) * 8;                   // K table lane offset
   const uint32_t lbV = Gm::LUTV_OFF | (lane * 4);         // V table lane base
 
-  // Lengths of the first 32 sequences, loaded by warp 0 now so the latency
-  // overlaps the table build; the block count and the first segment search
-  // reuse them.
-  const int len0 = (warp == 0 && lane < B) ? min(max(a.ctx_lens[lane], 0), a.cap_tok) : 0;
+  // Launches that follow in the stream may start their own set-up now; they
+  // wait for this grid before touching memory (programmatic dependent
+  // launch; a no-op without it).
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 
-  // ---- codebook tables: fp16 high/low parts of the scaled K levels and the
-  // fp16 V levels are staged in misc first (uniform lookups afterwards).
+  // ---- codebooks staged in misc (launch parameters only): fp16 high/low
+  // parts of the scaled K levels and the fp16 V levels
   uint32_t* cbs = reinterpret_cast<uint32_t*>(misc) + kMiscCb;
   if (tid < 16) {
     const float c = cbk.centroid[tid] * kKScale;
@@ -247,12 +340,13 @@ attend_kernel(const __grid_constant__ AttendArgs a,
     cbs[16 + tid] = __half_as_ushort(__float2half_rn(cbv.centroid[tid]));
   }
   __syncthreads();
+  // ---- K table: uint2 (high pair, low pair) per (pair code, copy)
   for (int e = tid; e < (1 << (2 * BK)) * 16; e += kThreads) {
     const int code = e >> 4, copy = e & 15;
     const uint32_t c0 = cbs[code & ((1 << BK) - 1)], c1 = cbs[code >> BK];
     uint2 v;
-    v.x = (c0 & 0xFFFFu) | (c1 << 16);              // high parts (even, odd coord)
-    v.y = (c0 >> 16) | (c1 & 0xFFFF0000u);          // low parts
+    v.x = (c0 & 0xFFFFu) | (c1 << 16);                // high parts (even, odd coord)
+    v.y = (c0 >> 16) | (c1 & 0xFFFF0000u);            // low parts
     *reinterpret_cast<uint2*>(lutK + code * 128 + copy * 8) = v;
   }
   if (BV != 2) {
@@ -267,32 +361,93 @@ attend_kernel(const __grid_constant__ AttendArgs a,
   if (BV == 2) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const uint32_t h = __half_as_ushort(__float2half_rn(cbv.centroid[j]));
+      const uint32_t h = cbs[16 + j];
       vt_lo |= (h & 0xFFu) << (8 * j);
       vt_hi |= (h >> 8) << (8 * j);
     }
   }
 
-  // ---- status words and empty sequences (CTA 0)
-  if (cta == 0) {
-    for (int b = 0; b < B; ++b) {
-      const int raw = a.ctx_lens[b];
-      if (tid == 0 && a.dev_status) {
-        if (raw > a.cap_tok) atomicOr(a.dev_status, TQ_DEV_CTX_CLAMPED);
-        if (raw <= 0) atomicOr(a.dev_status, TQ_DEV_CTX_EMPTY);
-      }
-      if (raw <= 0) {
-        const size_t n = (size_t)a.n_q_heads * kHeadDim, base = (size_t)b * n;
-        for (size_t i = tid; i < n; i += kThreads) {
-          if (a.out_dtype == TQ_F32) reinterpret_cast<float*>(a.out)[base + i] = 0.f;
-          else reinterpret_cast<uint16_t*>(a.out)[base + i] = 0;
-        }
-      }
-    }
+  // Everything below reads inputs that an earlier launch may have written.
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+
+  // Lengths of the first 32 sequences, loaded by warp 0 first; the block
+  // count and the first segment search use them.
+  const int len0 = (warp == 0 && lane < B) ? min(max(a.ctx_lens[lane], 0), a.cap_tok) : 0;
+  // The queries (small next to the cache) are pulled into L2 now, spread
+  // over the CTAs, so that their later loads do not queue behind the cache
+  // stream in DRAM.
+  {
+    const size_t qbytes = (size_t)B * a.n_q_heads * kHeadDim * (a.q_dtype == TQ_F32 ? 4 : 2);
+    const char* qc = reinterpret_cast<const char*>(a.q);
+    for (size_t off = ((size_t)cta * kThreads + tid) * 128; off < qbytes;
+         off += (size_t)Gc * kThreads * 128)
+      asm volatile("prefetch.global.L2 [%0];\n" ::"l"(qc + off));
   }
 
-  // ---- flat block count, and whether all sequences have the same length
+  // Segment search (warp 0): the first sequence whose flat block range holds
+  // flat block `at`, continuing from the scan state in misc. Writes the
+  // segment (b, g, first block, block count, blocks of the sequence, length).
+  auto find_segment = [&](long long at, long long end) {
+    int sb = misc[kMiscState];
+    long long sP = (long long)(unsigned)misc[kMiscState + 1] | ((long long)misc[kMiscState + 2] << 32);
+    while (true) {
+      if (sb >= B) {                      // inconsistent lengths: stop this CTA
+        if (lane == 0) misc[kMiscSeg + 3] = 0;
+        break;
+      }
+      const int bb = sb + lane;
+      const int len = sb == 0 ? len0 : (bb < B ? min(max(a.ctx_lens[bb], 0), a.cap_tok) : 0);
+      const int nb = (len + kBlk - 1) / kBlk;
+      int incl = nb;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const long long segend = (long long)H * (sP + incl);
+      const unsigned hit = __ballot_sync(0xFFFFFFFFu, segend > at && bb < B);
+      if (hit) {
+        const int l = __ffs(hit) - 1;
+        const int nbl = __shfl_sync(0xFFFFFFFFu, nb, l);
+        const int lenl = __shfl_sync(0xFFFFFFFFu, len, l);
+        const int excl = __shfl_sync(0xFFFFFFFFu, incl - nb, l);
+        sb += l;
+        sP += excl;
+        if (lane == 0) {
+          const long long rel = at - (long long)H * sP;
+          const int g = (int)(rel / nbl), blk0 = (int)(rel % nbl);
+          misc[kMiscSeg + 0] = sb;
+          misc[kMiscSeg + 1] = g;
+          misc[kMiscSeg + 2] = blk0;
+          misc[kMiscSeg + 3] = (int)min((long long)(nbl - blk0), end - at);
+          misc[kMiscSeg + 4] = nbl;
+          misc[kMiscSeg + 5] = lenl;
+          misc[kMiscState] = sb;
+          misc[kMiscState + 1] = (int)(sP & 0xFFFFFFFF);
+          misc[kMiscState + 2] = (int)(sP >> 32);
+        }
+        break;
+      }
+      sP += __shfl_sync(0xFFFFFFFFu, incl, 31);
+      sb += 32;
+    }
+  };
+
+  // Balanced split over Geff CTAs, each owning at least one block (the
+  // partial count of a sequence relies on it): min(grid, NB), or, when every
+  // (sequence, kv head) segment has the same block count and there are no
+  // more segments than CTAs, a multiple of the segment count so that no CTA
+  // spans two segments.
+  auto effective_ctas = [&](long long nbt, int common) {
+    int ge = (int)min((long long)Gc, nbt);
+    const long long S = (long long)B * H;
+    if (common > 0 && S <= Gc) ge = (int)(S * min((long long)(Gc / S), (long long)common));
+    return ge;
+  };
+
   if (warp == 0) {
+    // ---- flat block count, whether all sequences have the same length, and
+    // the first segment of this CTA
     long long tot = 0;
     int nmin = 0x7FFFFFFF, nmax = 0;
     for (int b0 = 0; b0 < B; b0 += 32) {
@@ -309,33 +464,46 @@ attend_kernel(const __grid_constant__ AttendArgs a,
       nmin = min(nmin, lo);
       nmax = max(nmax, hi);
     }
+    const long long nbt = tot * H;
+    const int common = nmin == nmax ? nmax : -1;
     if (lane == 0) {
-      const long long nbt = tot * H;
       misc[kMiscNB] = (int)(nbt & 0xFFFFFFFF);
       misc[kMiscNB + 1] = (int)(nbt >> 32);
-      misc[kMiscNB + 2] = nmin == nmax ? nmax : -1;   // common length in blocks
+      misc[kMiscNB + 2] = common;
       misc[kMiscState] = 0;
       misc[kMiscState + 1] = 0;
       misc[kMiscState + 2] = 0;
+      misc[kMiscSeg + 3] = 0;
     }
+    __syncwarp();
+    const int ge = effective_ctas(nbt, common);
+    if (cta < ge) find_segment(nbt * cta / ge, nbt * (cta + 1) / ge);
   }
   __syncthreads();
+
   const long long NB = (long long)(unsigned)misc[kMiscNB] | ((long long)misc[kMiscNB + 1] << 32);
-  // Balance over Geff CTAs, each owning at least one block (the partial count
-  // of a sequence relies on it): min(grid, NB), or, when every (sequence, kv
-  // head) segment has the same length and there are no more segments than
-  // CTAs, a multiple of the segment count so that no CTA spans two segments.
-  int Geff = (int)min((long long)Gc, NB);
-  {
-    const int common = misc[kMiscNB + 2];
-    const long long S = (long long)B * H;
-    if (common > 0 && S <= Gc) Geff = (int)(S * min((long long)(Gc / S), (long long)common));
-  }
+  const int Geff = effective_ctas(NB, misc[kMiscNB + 2]);
   const long long r0 = cta < Geff ? NB * cta / Geff : 0;
   const long long r1 = cta < Geff ? NB * (cta + 1) / Geff : 0;
   long long pos = r0;
   unsigned nskip = 0;
   const float log2tau = a.tau > 0.f ? log2f(a.tau) : -INFINITY;
+
+  // ---- status words and empty sequences (CTA 0, one sequence per thread)
+  if (cta == 0) {
+    for (int b = tid; b < B; b += kThreads) {
+      const int raw = a.ctx_lens[b];
+      if (a.dev_status && (raw > a.cap_tok || raw <= 0))
+        atomicOr(a.dev_status, raw <= 0 ? TQ_DEV_CTX_EMPTY : TQ_DEV_CTX_CLAMPED);
+      if (raw <= 0) {
+        const int es = a.out_dtype == TQ_F32 ? 4 : 2;
+        const size_t n16 = (size_t)a.n_q_heads * kHeadDim * es / 16;
+        uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(a.out) +
+                                            (size_t)b * a.n_q_heads * kHeadDim * es);
+        for (size_t i = 0; i < n16; ++i) o[i] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+  }
 
   // Lane roles in the score / softmax layout:
   //   NT = 1: the lane holds position gq (tq < 2) or gq + 8 (tq >= 2) of each
@@ -347,54 +515,49 @@ attend_kernel(const __grid_constant__ AttendArgs a,
     return 16 * mt + gq + (NT == 1 ? 8 * (tq >> 1) : 8 * rr);
   };
 
-  while (pos < r1) {
-    // ---- next segment (warp 0): first sequence whose flat range holds pos
-    if (warp == 0) {
-      int sb = misc[kMiscState];
-      long long sP = (long long)(unsigned)misc[kMiscState + 1] | ((long long)misc[kMiscState + 2] << 32);
-      while (true) {
-        if (sb >= B) {                    // inconsistent lengths: stop this CTA
-          if (lane == 0) misc[kMiscSeg + 3] = 0;
-          break;
-        }
-        const int b = sb + lane;
-        const int len = sb == 0 ? len0 : (b < B ? min(max(a.ctx_lens[b], 0), a.cap_tok) : 0);
-        const int nb = (len + kBlk - 1) / kBlk;
-        int incl = nb;
+  // Combines the kWarps merge buffers into fin[] (GQ x d) and the merged
+  // per-head maximum and softmax sum (misc). A buffer holds accumulators in
+  // register order (natural = false: lane-major, 32 per lane) or in output
+  // order (natural = true), then the per-head maxima and sums.
+  float* wts = miscf + kMiscWt;                       // [kWarps][GQ] weights
+  auto merge_buffers = [&](bool natural) {
+    if (tid < kWarps * GQ) {
+      const int w = tid / GQ, h = tid - w * GQ;
+      float mx = -INFINITY;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-          if (lane >= o) incl += v;
+      for (int v = 0; v < kWarps; ++v) mx = fmaxf(mx, merge[v * kMergeStride + kMergeM + h]);
+      const float mw = merge[w * kMergeStride + kMergeM + h];
+      wts[tid] = mw == -INFINITY ? 0.f : fast_exp2(mw - mx);
+      if (w == 0) {
+        float ls = 0.f;
+#pragma unroll
+        for (int v = 0; v < kWarps; ++v) {
+          const float m = merge[v * kMergeStride + kMergeM + h];
+          if (m != -INFINITY) ls += merge[v * kMergeStride + kMergeL + h] * fast_exp2(m - mx);
         }
-        const long long end = (long long)H * (sP + incl);
-        const unsigned hit = __ballot_sync(0xFFFFFFFFu, end > pos && b < B);
-        if (hit) {
-          const int l = __ffs(hit) - 1;
-          const int nbl = __shfl_sync(0xFFFFFFFFu, nb, l);
-          const int lenl = __shfl_sync(0xFFFFFFFFu, len, l);
-          const int excl = __shfl_sync(0xFFFFFFFFu, incl - nb, l);
-          sb += l;
-          sP += excl;
-          if (lane == 0) {
-            const long long rel = pos - (long long)H * sP;
-            const int g = (int)(rel / nbl), blk0 = (int)(rel % nbl);
-            misc[kMiscSeg + 0] = sb;
-            misc[kMiscSeg + 1] = g;
-            misc[kMiscSeg + 2] = blk0;
-            misc[kMiscSeg + 3] = (int)min((long long)(nbl - blk0), r1 - pos);
-            misc[kMiscSeg + 4] = nbl;
-            misc[kMiscSeg + 5] = lenl;
-            misc[kMiscState] = sb;
-            misc[kMiscState + 1] = (int)(sP & 0xFFFFFFFF);
-            misc[kMiscState + 2] = (int)(sP >> 32);
-          }
-          break;
-        }
-        sP += __shfl_sync(0xFFFFFFFFu, incl, 31);
-        sb += 32;
+        miscf[kMiscM + h] = mx;
+        miscf[kMiscL + h] = ls;
       }
     }
     __syncthreads();
+    for (int i = tid; i < GQ * kHeadDim; i += kThreads) {
+      const int h = i / kHeadDim;
+      const int idx = natural ? i : pv_slot<BV>(i - h * kHeadDim, h);
+      float sum = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) sum += merge[w * kMergeStride + idx] * wts[w * GQ + h];
+      fin[i] = sum;
+    }
+    __syncthreads();
+  };
+
+  bool first = true;
+  while (pos < r1) {
+    if (!first) {
+      if (warp == 0) find_segment(pos, r1);
+      __syncthreads();
+    }
+    first = false;
     const int b = misc[kMiscSeg + 0], g = misc[kMiscSeg + 1], blk0 = misc[kMiscSeg + 2];
     const int nseg = misc[kMiscSeg + 3], nbl = misc[kMiscSeg + 4], L = misc[kMiscSeg + 5];
     if (nseg <= 0) break;
@@ -402,19 +565,33 @@ attend_kernel(const __grid_constant__ AttendArgs a,
     const long long seg_first = (long long)H * sP_seg + (long long)g * nbl;
 
     // query values of the group (warp h < g loads head h), issued before the
-    // block loads so that both latencies overlap
+    // block loads
     float qraw[4] = {0.f, 0.f, 0.f, 0.f};
     if (warp < GQ) {
       const size_t qo = ((size_t)b * a.n_q_heads + (size_t)g * GQ + warp) * kHeadDim + 4 * lane;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) qraw[k] = load_elem(a.q, a.q_dtype, qo + k);
+      if (a.q_dtype == TQ_F32) {
+        const float4 v = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.q) + qo);
+        qraw[0] = v.x; qraw[1] = v.y; qraw[2] = v.z; qraw[3] = v.w;
+      } else {
+        const uint2 v = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(a.q) + qo);
+        const bool bf = a.q_dtype == TQ_BF16;
+        const float2 f0 = unpack16x2(v.x, bf), f1 = unpack16x2(v.y, bf);
+        qraw[0] = f0.x; qraw[1] = f0.y; qraw[2] = f1.x; qraw[3] = f1.y;
+      }
     }
 
-    // ---- this warp's blocks of the segment; their first loads go out
-    // before the query rotation so that the two overlap
-    const int wb0 = blk0 + (int)((long long)nseg * warp / kWarps);
-    const int wb1 = blk0 + (int)((long long)nseg * (warp + 1) / kWarps);
-    const int nw = wb1 - wb0;
+    // ---- this warp's blocks of the segment
+    // The warps split the segment in whole 64-position blocks (the sparse-V
+    // gate's block maximum needs the full block; measured, a 16-position
+    // split was no faster without the gate either: the SM is throughput
+    // bound in this phase). A warp walks its range in chunks of up to 64
+    // positions starting at wp0.
+    const int sp0 = blk0 * kBlk, sp1 = min(L, (blk0 + nseg) * kBlk);
+    const int unit = kBlk;
+    const int nun = (sp1 - sp0 + unit - 1) / unit;
+    const int wp0 = sp0 + unit * (int)((long long)nun * warp / kWarps);
+    const int wp1 = min(sp1, sp0 + unit * (int)((long long)nun * (warp + 1) / kWarps));
+    const int nw = wp1 > wp0 ? (wp1 - wp0 + kBlk - 1) / kBlk : 0;
 
     float acc[8][4];
 #pragma unroll
@@ -429,43 +606,39 @@ attend_kernel(const __grid_constant__ AttendArgs a,
     const uint32_t wring = Gm::FIXED + warp * Gm::NSTAGE * Gm::STAGE;   // smem offset
     const uint32_t wring_s = smem_addr(smem) + wring;                    // shared address
 
-    // cp.async of block `blk` into ring slot `slot`. K and V blocks are
-    // contiguous in global memory; chunk c of K lands at byte 16c, chunk c of
-    // V at row (c / BV) · RVS + (c % BV) · 16. Chunks past the sequence are
-    // zero-filled without reading.
-    auto issue = [&](int blk, int slot) {
-      const int t0 = blk * kBlk;
-      const int kvalid = min(kBlk, L - t0) * BK;
-      const int vvalid = min(kBlk, L - t0) * BV;
-      const uint32_t dst = wring_s + slot * Gm::STAGE;
-      const uint8_t* ksrc = gk + (size_t)t0 * Gm::RK;
-      const uint8_t* vsrc = gv + (size_t)t0 * Gm::RV;
-#pragma unroll
-      for (int i = 0; i < BK * 2; ++i) {
-        const int ch = lane + 32 * i;
-        const bool ok = ch < kvalid;
-        cp_async16(dst + 16 * ch, ksrc + (ok ? 16 * ch : 0), ok ? 16 : 0);
-      }
-#pragma unroll
-      for (int i = 0; i < BV * 2; ++i) {
-        const int ch = lane + 32 * i;
-        const bool ok = ch < vvalid;
-        cp_async16(dst + Gm::KB + (ch / BV) * Gm::RVS + (ch % BV) * 16,
-                   vsrc + (ok ? 16 * ch : 0), ok ? 16 : 0);
-      }
-      if (lane < 16) {
-        const int c8 = lane & 7;
-        const bool ok = t0 + 8 * c8 < L;
-        const uint16_t* src = (lane < 8 ? gnk : gnv) + t0 + (ok ? 8 * c8 : 0);
-        cp_async16(dst + Gm::NKOFF + (lane >> 3) * (2 * kBlk) + 16 * c8, src, ok ? 16 : 0);
+    // Bulk copies of chunk c of the warp's range (its j-th staged chunk)
+    // into ring slot j % NSTAGE, issued by lane 0: K rows, V rows and the
+    // two norm runs are contiguous in global memory. Rows past the range are
+    // not copied; their slot bytes are stale and masked out below (norms are
+    // copied in whole 16-byte runs, which stay inside cap_tok).
+    auto issue = [&](int c, int j) {
+      if (lane == 0) {
+        const int t0 = wp0 + c * kBlk;
+        const int rows = min(kBlk, wp1 - t0);
+        const int nrows = min(kBlk, (rows + 7) & ~7);
+        const int slot = j % Gm::NSTAGE;
+        const uint32_t dst = wring_s + slot * Gm::STAGE, bar = wbar + 8 * slot;
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+        mbar_expect(bar, rows * (Gm::RK + Gm::RV) + 4 * nrows);
+        bulk_g2s(dst, gk + (size_t)t0 * Gm::RK, rows * Gm::RK, bar);
+        bulk_g2s(dst + Gm::KB, gv + (size_t)t0 * Gm::RV, rows * Gm::RV, bar);
+        bulk_g2s(dst + Gm::NKOFF, gnk + t0, 2 * nrows, bar);
+        bulk_g2s(dst + Gm::NKOFF + 2 * kBlk, gnv + t0, 2 * nrows, bar);
       }
     };
 
+    // every slot of the ring gets a block (or an empty group); the warps
+    // that rotate the query fill theirs afterwards, so that the query loads
+    // do not wait behind their block loads
+    auto fill_ring = [&]() {
 #pragma unroll
-    for (int p = 0; p < Gm::NSTAGE - 1; ++p) {
-      if (p < nw) issue(wb0 + p, p);
-      cp_async_commit();
-    }
+      for (int p = 0; p < Gm::NSTAGE; ++p)
+        if (!stalled && p < nw) issue(p, jdone + p);
+    };
+    int issued = stalled ? 0 : min(nw, Gm::NSTAGE);
+    auto bar_of = [&](int jj) { return wbar + 8 * (jj % Gm::NSTAGE); };
+    auto par_of = [&](int jj) { return (uint32_t)(jj / Gm::NSTAGE) & 1u; };
+    if (warp >= GQ) fill_ring();
     // ---- rotated query of the group: warp h handles query head h
     if (warp < GQ) {
       float x[4];
@@ -497,14 +670,13 @@ attend_kernel(const __grid_constant__ AttendArgs a,
       *reinterpret_cast<uint2*>(qhi + warp * kHeadDim + 4 * lane) = make_uint2(hi2[0], hi2[1]);
       *reinterpret_cast<uint2*>(qlo + warp * kHeadDim + 4 * lane) = make_uint2(lo2[0], lo2[1]);
       if (lane == 0) miscf[kMiscQInv + warp] = 1.f / (qs * kKScale);
+      fill_ring();
     }
     __syncthreads();
 
     // ---- query fragments (B operand of the score MMA), column n = gq.
     //   NT = 1: columns 0-3 hold the high part of heads 0-3, 4-7 their low part.
     //   NT = 2: tile 0 column n = high part of head n, tile 1 = low part.
-    // The K-low product reuses tile 0 (for NT = 1 it also picks up the
-    // negligible query-low x K-low term).
     uint32_t qb[NT][8][2];
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
@@ -521,86 +693,86 @@ attend_kernel(const __grid_constant__ AttendArgs a,
     const float sinv0 = hv0 ? miscf[kMiscQInv + hs0] : 0.f;
     const float sinv1 = hv1 ? miscf[kMiscQInv + hs0 + 1] : 0.f;
 
-    for (int i = 0; i < nw; ++i) {
-      {
-        const int nxt = i + Gm::NSTAGE - 1;
-        if (nxt < nw) issue(wb0 + nxt, nxt % Gm::NSTAGE);
-        cp_async_commit();
+    for (int i = 0; i < nw && !stalled; ++i) {
+      const int j = jdone + i;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar_of(j), par_of(j)))) {
+        // give up: report, wait (bounded) for the copies still in flight,
+        // issue nothing more
+        stalled = true;
+        if (lane == 0 && a.dev_status) atomicOr(a.dev_status, TQ_DEV_WAIT_TIMEOUT);
+        for (int k = i + 1; k < issued; ++k) mbar_wait(bar_of(jdone + k), par_of(jdone + k));
+        __syncwarp();
+        break;
       }
-      cp_async_wait<Gm::NSTAGE - 1>();
-      __syncwarp();
-      const uint32_t st = wring + (i % Gm::NSTAGE) * Gm::STAGE;         // smem offset
-      const int t0 = (wb0 + i) * kBlk;
-      const bool partial = t0 + kBlk > L;
+      const uint32_t st = wring + (j % Gm::NSTAGE) * Gm::STAGE;         // smem offset
+      const int t0 = wp0 + i * kBlk;                // chunk [t0, cend)
+      const int cend = min(wp1, t0 + kBlk);
+      const bool partial = cend < t0 + kBlk;
 
-      // -- scores: 4 steps of 16 positions
+      // -- scores: 4 steps of 16 positions, each as two 8-position groups.
+      // A operand rows 0-7 are the K codebook high parts of the group's
+      // positions, rows 8-15 the low parts of the same positions, so one
+      // table entry (high pair, low pair) fills two adjacent fragment
+      // registers; D rows r and r + 8 add up to the score of position r.
       float sc[4][NR][2];               // [step][row][head hs0 + e]
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
-        uint32_t kw0[BK + 1], kw1[BK + 1];   // rows gq and gq + 8, chunk tq
-        const uint32_t r0 = st + (16 * mt + gq) * Gm::RK + 4 * BK * tq;
-        const uint32_t r1 = r0 + 8 * Gm::RK;
-        if (BK == 4) {                       // one 16-byte load per row chunk
-          const uint4 u0 = lds<uint4>(smem, r0), u1 = lds<uint4>(smem, r1);
-          kw0[0] = u0.x; kw0[1] = u0.y; kw0[2 % (BK + 1)] = u0.z; kw0[3 % (BK + 1)] = u0.w;
-          kw1[0] = u1.x; kw1[1] = u1.y; kw1[2 % (BK + 1)] = u1.z; kw1[3 % (BK + 1)] = u1.w;
-        } else if (BK == 2) {
-          const uint2 u0 = lds<uint2>(smem, r0), u1 = lds<uint2>(smem, r1);
-          kw0[0] = u0.x; kw0[1] = u0.y;
-          kw1[0] = u1.x; kw1[1] = u1.y;
-        } else {
+        if (16 * mt >= cend - t0) {          // step past the chunk: all masked
 #pragma unroll
-          for (int w = 0; w < BK; ++w) {
-            kw0[w] = lds<uint32_t>(smem, r0 + 4 * w);
-            kw1[w] = lds<uint32_t>(smem, r1 + 4 * w);
+          for (int rr = 0; rr < NR; ++rr) sc[mt][rr][0] = sc[mt][rr][1] = -INFINITY;
+          continue;
+        }
+        uint32_t kw[2][BK + 1];              // positions gq and gq + 8, chunk tq
+#pragma unroll
+        for (int gr = 0; gr < 2; ++gr) {
+          const uint32_t rp = st + (16 * mt + 8 * gr + gq) * Gm::RK + 4 * BK * tq;
+          if constexpr (BK == 4) {
+            const uint4 u = lds<uint4>(smem, rp);
+            kw[gr][0] = u.x; kw[gr][1] = u.y; kw[gr][2] = u.z; kw[gr][3] = u.w;
+          } else if constexpr (BK == 2) {
+            const uint2 u = lds<uint2>(smem, rp);
+            kw[gr][0] = u.x; kw[gr][1] = u.y;
+          } else {
+#pragma unroll
+            for (int w = 0; w < BK; ++w) kw[gr][w] = lds<uint32_t>(smem, rp + 4 * w);
           }
+          kw[gr][BK] = 0;
         }
-        kw0[BK] = kw1[BK] = 0;
-        // two accumulator sets (even / odd k-steps) halve the MMA chains
-        float dh[2][NT][4], dl[2][4];
+        float d[2][NT][4];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int gr = 0; gr < 2; ++gr)
 #pragma unroll
-          for (int t = 0; t < NT; ++t) dh[c][t][0] = dh[c][t][1] = dh[c][t][2] = dh[c][t][3] = 0.f;
-          dl[c][0] = dl[c][1] = dl[c][2] = dl[c][3] = 0.f;
-        }
+          for (int t = 0; t < NT; ++t) d[gr][t][0] = d[gr][t][1] = d[gr][t][2] = d[gr][t][3] = 0.f;
 #pragma unroll
         for (int s2 = 0; s2 < 8; ++s2) {
-          const uint2 e00 = lds<uint2>(smem, pair_code_shifted<BK, 7>(kw0, 2 * s2) | lbK);
-          const uint2 e10 = lds<uint2>(smem, pair_code_shifted<BK, 7>(kw1, 2 * s2) | lbK);
-          const uint2 e01 = lds<uint2>(smem, pair_code_shifted<BK, 7>(kw0, 2 * s2 + 1) | lbK);
-          const uint2 e11 = lds<uint2>(smem, pair_code_shifted<BK, 7>(kw1, 2 * s2 + 1) | lbK);
 #pragma unroll
-          for (int t = 0; t < NT; ++t)
-            mma16816(dh[s2 & 1][t], e00.x, e10.x, e01.x, e11.x, qb[t][s2][0], qb[t][s2][1]);
-          mma16816(dl[s2 & 1], e00.y, e10.y, e01.y, e11.y, qb[0][s2][0], qb[0][s2][1]);
+          for (int gr = 0; gr < 2; ++gr) {
+            const uint2 e0 = lds<uint2>(smem, k_entry<BK>(kw[gr], 2 * s2) + lbK);
+            const uint2 e1 = lds<uint2>(smem, k_entry<BK>(kw[gr], 2 * s2 + 1) + lbK);
+#pragma unroll
+            for (int t = 0; t < NT; ++t)
+              mma16816(d[gr][t], e0.x, e0.y, e1.x, e1.y, qb[t][s2][0], qb[t][s2][1]);
+          }
         }
-        float dsum[NT][4];
-#pragma unroll
-        for (int t = 0; t < NT; ++t)
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            dsum[t][k] = (dh[0][t][k] + dh[1][t][k]) + (t == 0 ? dl[0][k] + dl[1][k] : 0.f);
-        // d[0], d[1]: position gq, columns 2tq, 2tq+1; d[2], d[3]: position gq+8
         if (NT == 1) {
-          // Columns 2tq, 2tq+1 are the high part of heads 2tq, 2tq+1 (tq < 2)
-          // or the low part of heads 2(tq-2), +1 (tq >= 2); lane ^ 2 holds
-          // the other part. Lanes tq < 2 keep position gq, tq >= 2 keep gq+8.
-          const float d0 = dsum[0][0], d1 = dsum[0][1];
-          const float d2 = dsum[0][2], d3 = dsum[0][3];
+          // Columns 2tq, 2tq+1: the high part of heads 2tq, 2tq+1 (tq < 2) or
+          // the low part of heads 2(tq-2), +1 (tq >= 2); lane ^ 2 holds the
+          // other part. Lanes tq < 2 keep group 0, tq >= 2 keep group 1.
+          const float a0 = d[0][0][0] + d[0][0][2], a1 = d[0][0][1] + d[0][0][3];
+          const float c0 = d[1][0][0] + d[1][0][2], c1 = d[1][0][1] + d[1][0][3];
           const bool lowq = tq >= 2;
-          const float s0 = __shfl_xor_sync(0xFFFFFFFFu, lowq ? d0 : d2, 2);
-          const float s1 = __shfl_xor_sync(0xFFFFFFFFu, lowq ? d1 : d3, 2);
-          sc[mt][0][0] = (lowq ? d2 : d0) + s0;
-          sc[mt][0][1] = (lowq ? d3 : d1) + s1;
+          const float s0 = __shfl_xor_sync(0xFFFFFFFFu, lowq ? a0 : c0, 2);
+          const float s1 = __shfl_xor_sync(0xFFFFFFFFu, lowq ? a1 : c1, 2);
+          sc[mt][0][0] = (lowq ? c0 : a0) + s0;
+          sc[mt][0][1] = (lowq ? c1 : a1) + s1;
         } else {
-          sc[mt][0][0] = dsum[0][0] + dsum[NT - 1][0];
-          sc[mt][0][1] = dsum[0][1] + dsum[NT - 1][1];
-          sc[mt][NR - 1][0] = dsum[0][2] + dsum[NT - 1][2];
-          sc[mt][NR - 1][1] = dsum[0][3] + dsum[NT - 1][3];
+#pragma unroll
+          for (int gr = 0; gr < 2; ++gr) {
+            sc[mt][gr][0] = (d[gr][0][0] + d[gr][0][2]) + d[gr][NT - 1][0];
+            sc[mt][gr][1] = (d[gr][0][1] + d[gr][0][3]) + d[gr][NT - 1][1];
+          }
         }
       }
-
       // -- scale by the K norm and query scale, mask, block maximum per head
       float mb0 = -INFINITY, mb1 = -INFINITY;
 #pragma unroll
@@ -611,7 +783,7 @@ attend_kernel(const __grid_constant__ AttendArgs a,
           const float nk = __half2float(__ushort_as_half(lds<uint16_t>(smem, st + Gm::NKOFF + 2 * p)));
           float v0 = sc[mt][rr][0] * (sinv0 * nk);
           float v1 = sc[mt][rr][1] * (sinv1 * nk);
-          if (partial && t0 + p >= L) v0 = v1 = -INFINITY;
+          if (partial && t0 + p >= cend) v0 = v1 = -INFINITY;
           sc[mt][rr][0] = v0;
           sc[mt][rr][1] = v1;
           mb0 = fmaxf(mb0, v0);
@@ -646,6 +818,7 @@ attend_kernel(const __grid_constant__ AttendArgs a,
           const bool g0 = s0 - mb0 < log2tau, g1 = s1 - mb1 < log2tau;   // exp(s - M_blk) < tau
           if (g0) p0 = 0.f;
           if (g1) p1 = 0.f;
+          if (partial && t0 + p >= cend) p0 = p1 = 0.f;   // stale slot bytes
           nskip += (g0 && hv0 && s0 != -INFINITY) + (g1 && hv1 && s1 != -INFINITY);
           pk[mt][rr] = pack_half2(hv0 ? p0 : 0.f, hv1 ? p1 : 0.f);
         }
@@ -725,9 +898,13 @@ attend_kernel(const __grid_constant__ AttendArgs a,
           }
         }
       }
-      __syncwarp();
+      __syncwarp();                                  // the slot is free again
+      if (i + Gm::NSTAGE < nw) {
+        issue(i + Gm::NSTAGE, j + Gm::NSTAGE);
+        ++issued;
+      }
     }
-    cp_async_wait<0>();
+    jdone += nw;
 
     // ---- per-warp softmax sums over the lanes holding the same heads
 #pragma unroll
@@ -736,63 +913,29 @@ attend_kernel(const __grid_constant__ AttendArgs a,
       l_run[1] += __shfl_xor_sync(0xFFFFFFFFu, l_run[1], o);
     }
 
-    // ---- merge the warps of this segment
-    constexpr int WS = kMaxGroup * kHeadDim + 2 * kMaxGroup;
+    // ---- merge the warps of this segment. Each warp leaves its partial in
+    // a merge buffer (accumulators as stored in its registers, then the
+    // per-head maximum and sum); the buffers are combined per output element.
     __syncthreads();                                  // all warps done with the ring
     {
-      float* wm = merge + warp * WS;
+      float* wm = merge + warp * kMergeStride;
       if (gq == 0 && (NT == 2 || tq < 2)) {
         if (hv0) {
-          wm[kMaxGroup * kHeadDim + hs0] = nw > 0 ? m_run[0] : -INFINITY;
-          wm[kMaxGroup * kHeadDim + kMaxGroup + hs0] = nw > 0 ? l_run[0] : 0.f;
+          wm[kMergeM + hs0] = nw > 0 ? m_run[0] : -INFINITY;
+          wm[kMergeL + hs0] = nw > 0 ? l_run[0] : 0.f;
         }
         if (hv1) {
-          wm[kMaxGroup * kHeadDim + hs0 + 1] = nw > 0 ? m_run[1] : -INFINITY;
-          wm[kMaxGroup * kHeadDim + kMaxGroup + hs0 + 1] = nw > 0 ? l_run[1] : 0.f;
+          wm[kMergeM + hs0 + 1] = nw > 0 ? m_run[1] : -INFINITY;
+          wm[kMergeL + hs0 + 1] = nw > 0 ? l_run[1] : 0.f;
         }
       }
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        const int c0 = pv_coord<BV>(r, gq), c1 = pv_coord<BV>(r, gq + 8);
-        const int h0 = 2 * tq, h1 = 2 * tq + 1;
-        if (h0 < GQ) {
-          wm[h0 * kHeadDim + c0] = acc[r][0];
-          wm[h0 * kHeadDim + c1] = acc[r][2];
-        }
-        if (h1 < GQ) {
-          wm[h1 * kHeadDim + c0] = acc[r][1];
-          wm[h1 * kHeadDim + c1] = acc[r][3];
-        }
-      }
+      for (int r = 0; r < 8; ++r)
+        *reinterpret_cast<float4*>(wm + lane * kMergeLane + 4 * r) =
+            make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
     }
     __syncthreads();
-    // per-head maximum and sum over the warps, then per-(warp, head) weights
-    float* wt = miscf + kMiscWt;                      // [kWarps][GQ] <= 96 floats
-    if (tid < GQ) {
-      float mx = -INFINITY;
-      for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, merge[w * WS + kMaxGroup * kHeadDim + tid]);
-      float ls = 0.f;
-      for (int w = 0; w < kWarps; ++w) {
-        const float mw = merge[w * WS + kMaxGroup * kHeadDim + tid];
-        const float f = mw == -INFINITY ? 0.f : exp2f(mw - mx);
-        wt[w * GQ + tid] = f;
-        ls += merge[w * WS + kMaxGroup * kHeadDim + kMaxGroup + tid] * f;
-      }
-      miscf[kMiscM + tid] = mx;
-      miscf[kMiscL + tid] = ls;
-    }
-    __syncthreads();
-    for (int i = tid; i < GQ * kHeadDim; i += kThreads) {
-      const int h = i / kHeadDim;
-      float s = 0.f;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const float f = wt[w * GQ + h];
-        if (f != 0.f) s += merge[w * WS + i] * f;
-      }
-      fin[i] = s;
-    }
-    __syncthreads();
+    merge_buffers(false);
 
     bool finalize = nseg == nbl;                      // this CTA saw the whole sequence
     if (!finalize) {
@@ -810,62 +953,66 @@ attend_kernel(const __grid_constant__ AttendArgs a,
       if (tid == 0) {
         __threadfence();
         const int prev = atomicAdd(a.counters + sigma, 1);
-        misc[kMiscLast] = prev == n_parts - 1;
+        const bool is_last = prev == n_parts - 1;
+        if (is_last) __threadfence();
+        misc[kMiscLast] = is_last;
       }
       __syncthreads();
       finalize = misc[kMiscLast] != 0;
       if (finalize) {
-        // Merge the n_parts partials of this sequence. Their (max, sum) pairs
-        // are read in one parallel pass and turned into weights in shared
-        // memory (the ring area is free here: n_parts <= 1024 CTAs x 8 heads
-        // x 2 floats = 64 KB); the accumulators are then summed with up to 16
-        // independent loads in flight per thread.
-        __threadfence();
+        // Merge the n_parts partials of this sequence: warp w folds partials
+        // w, w + kWarps, ... (two per round of loads) into a merge buffer in
+        // output order, then the buffers are combined as above.
         const float* s0 = a.slots + (size_t)(c_first + sigma) * GQ * kSlotFloats;
         const size_t stride = (size_t)GQ * kSlotFloats;
-        float* pm = merge;                       // [n_parts][GQ] max, then weight
-        float* pl = merge + n_parts * GQ;        // [n_parts][GQ] sum
-        for (int j = tid; j < n_parts * GQ; j += kThreads) {
-          const int p = j / GQ, h = j - p * GQ;
-          pm[j] = __ldcg(s0 + p * stride + GQ * kHeadDim + 2 * h);
-          pl[j] = __ldcg(s0 + p * stride + GQ * kHeadDim + 2 * h + 1);
-        }
-        __syncthreads();
-        if (tid < GQ) {
-          float mx = -INFINITY;
-          for (int p = 0; p < n_parts; ++p) mx = fmaxf(mx, pm[p * GQ + tid]);
-          float ls = 0.f;
-          for (int p = 0; p < n_parts; ++p) ls += pl[p * GQ + tid] * exp2f(pm[p * GQ + tid] - mx);
-          miscf[kMiscM + tid] = mx;
-          miscf[kMiscL + tid] = ls;
-        }
-        __syncthreads();
-        for (int j = tid; j < n_parts * GQ; j += kThreads)
-          pm[j] = exp2f(pm[j] - miscf[kMiscM + j % GQ]);
-        __syncthreads();
-        for (int i = tid; i < GQ * kHeadDim; i += kThreads) {
-          const int h = i / kHeadDim;
-          float sum = 0.f;
-          int p = 0;
-          for (; p + 16 <= n_parts; p += 16) {
-            float v[16];
+        const int nk = GQ * kHeadDim / 32;            // outputs per lane: lane + 32k
+        float S[kMaxGroup * kHeadDim / 32];
+        float Mh = -INFINITY, Lh = 0.f;               // lane h < GQ: head h
 #pragma unroll
-            for (int k = 0; k < 16; ++k) v[k] = __ldcg(s0 + (p + k) * stride + i);
+        for (int k = 0; k < kMaxGroup * kHeadDim / 32; ++k) S[k] = 0.f;
+        for (int p = warp; p < n_parts; p += 2 * kWarps) {
+          const bool two = p + kWarps < n_parts;
+          const float* pa = s0 + (size_t)p * stride;
+          const float* pb = s0 + (size_t)(two ? p + kWarps : p) * stride;
+          float va[kMaxGroup * kHeadDim / 32], vb[kMaxGroup * kHeadDim / 32];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) sum += v[k] * pm[(p + k) * GQ + h];
+          for (int k = 0; k < kMaxGroup * kHeadDim / 32; ++k) {
+            va[k] = k < nk ? __ldcg(pa + lane + 32 * k) : 0.f;
+            vb[k] = k < nk && two ? __ldcg(pb + lane + 32 * k) : 0.f;
           }
-          for (; p + 4 <= n_parts; p += 4) {
-            float v[4];
+          const bool hl = lane < GQ;
+          const float ma = hl ? __ldcg(pa + GQ * kHeadDim + 2 * lane) : -INFINITY;
+          const float la = hl ? __ldcg(pa + GQ * kHeadDim + 2 * lane + 1) : 0.f;
+          const float mb = hl && two ? __ldcg(pb + GQ * kHeadDim + 2 * lane) : -INFINITY;
+          const float lb = hl && two ? __ldcg(pb + GQ * kHeadDim + 2 * lane + 1) : 0.f;
+          // per head (lane h): new maximum and the three rescale factors
+          const float Mn = fmaxf(Mh, fmaxf(ma, mb));
+          const float fo = Mh == -INFINITY ? 0.f : fast_exp2(Mh - Mn);
+          const float fa = ma == -INFINITY ? 0.f : fast_exp2(ma - Mn);
+          const float fb = mb == -INFINITY ? 0.f : fast_exp2(mb - Mn);
+          Lh = Lh * fo + la * fa + lb * fb;
+          Mh = Mn;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) v[k] = __ldcg(s0 + (p + k) * stride + i);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) sum += v[k] * pm[(p + k) * GQ + h];
+          for (int k = 0; k < kMaxGroup * kHeadDim / 32; ++k) {
+            const int h = k >> 2;                       // 32k / kHeadDim
+            const float go = __shfl_sync(0xFFFFFFFFu, fo, h);
+            const float ga = __shfl_sync(0xFFFFFFFFu, fa, h);
+            const float gb = __shfl_sync(0xFFFFFFFFu, fb, h);
+            S[k] = S[k] * go + va[k] * ga + vb[k] * gb;
           }
-          for (; p < n_parts; ++p) sum += __ldcg(s0 + p * stride + i) * pm[p * GQ + h];
-          fin[i] = sum;
         }
+        __syncthreads();                              // merge buffers are free
+        float* wm = merge + warp * kMergeStride;
+#pragma unroll
+        for (int k = 0; k < kMaxGroup * kHeadDim / 32; ++k)
+          if (k < nk) wm[lane + 32 * k] = S[k];
+        if (lane < GQ) {
+          wm[kMergeM + lane] = Mh;
+          wm[kMergeL + lane] = Lh;
+        }
+        __syncthreads();
+        merge_buffers(true);
         if (tid == 0) atomicExch(a.counters + sigma, 0);
-        __syncthreads();
       }
     }
     if (finalize && warp < GQ) {
@@ -927,8 +1074,20 @@ cudaError_t launch_one(const AttendArgs& a, const Codebook& cbk, const Codebook&
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }
   const int grid = n_ctas > 0 ? n_ctas : sm_count();
-  attend_kernel<BK, BV, NT><<<grid, kThreads, Gm::SMEM, stream>>>(a, cbk, cbv, sm);
-  return cudaGetLastError();
+  // Programmatic dependent launch: the kernel's set-up may overlap the tail
+  // of the previous launch in the stream; it waits for that launch before
+  // reading any input (griddepcontrol.wait).
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Gm::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attend_kernel<BK, BV, NT>, a, cbk, cbv, sm);
 }
 
 template <int BK, int BV>

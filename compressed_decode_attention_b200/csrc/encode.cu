@@ -130,6 +130,10 @@ encode_kernel(const __grid_constant__ EncodeArgs a,
               const __grid_constant__ Codebook cbk,
               const __grid_constant__ Codebook cbv,
               const __grid_constant__ SignMask sm) {
+  // Programmatic dependent launch (a no-op without it): the next launch may
+  // start; the input may come from the previous one, so wait before reading.
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int sub = lane & 3;
   const unsigned gmask = 0xFu << (lane & ~3);
@@ -199,8 +203,16 @@ cudaError_t launch_encode(const EncodeArgs& a, const Codebook& cbk,
   }
   const long long units = (long long)((a.n_tok + kEncTokens - 1) / kEncTokens) * a.n_kv_heads * 2;
   const int grid = (int)(units < (long long)sms * 8 ? units : (long long)sms * 8);
-  encode_kernel<<<grid, kEncThreads, 0, stream>>>(a, cbk, cbv, sm);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kEncThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, encode_kernel, a, cbk, cbv, sm);
 }
 
 }  // namespace tq

@@ -90,6 +90,8 @@ typedef enum { TQ_F16 = 0, TQ_BF16 = 1, TQ_F32 = 2 } tq_dtype;
 #define TQ_DEV_CTX_CLAMPED    1  /* some ctx_lens[b] > cap_tok; clamped     */
 #define TQ_DEV_NORM_SATURATED 2  /* some norm > 65504; stored as 65504      */
 #define TQ_DEV_CTX_EMPTY      4  /* some ctx_lens[b] <= 0; output set to 0  */
+#define TQ_DEV_WAIT_TIMEOUT   8  /* a wait for staged cache data gave up    */
+                                 /* after ~1 s; the output is not valid     */
 
 /* Library ABI version (TQ_ABI_VERSION of the build). */
 int tq_abi_version(void);
@@ -211,7 +213,9 @@ size_t tq_attend_workspace_size(int batch, int n_q_heads, int cap_tok, int d);
  *               the first call that uses it (e.g. cudaMemset once); every call
  *               leaves it zero again when it completes on the stream. The
  *               rest is scratch. One workspace per concurrently running call.
- *   dev_status  device int, nullable.
+ *   dev_status  device int, nullable. TQ_DEV_WAIT_TIMEOUT reports a copy of
+ *               cache data into shared memory that did not complete within
+ *               about a second (the kernel then gives up instead of hanging).
  *   sparse_v_skipped  device uint64, nullable: atomically incremented by the
  *               number of (b, h, t) positions the gate left out.
  *   out         [batch][n_q_heads][d] of out_dtype (TQ_F16 | TQ_BF16 | TQ_F32),

@@ -141,7 +141,11 @@ def test_workspace_counters_return_to_zero_and_calls_repeat():
         outs.append(o)
     np.testing.assert_array_equal(outs[0], outs[3])
     np.testing.assert_array_equal(outs[1], outs[2])
-    assert np.abs(outs[0] - outs[1]).max() <= 1e-5
+    # Different CTA counts split the positions differently; the softmax
+    # weights x V norms enter the P.V product rounded to fp16 (relative step
+    # 2^-11) against each chunk's own maximum, so the two splits agree to
+    # about 1e-4, ten times inside the oracle bar.
+    assert np.abs(outs[0] - outs[1]).max() <= 2e-4
 
 
 def _small_cache(bk, bv, B, Hkv, cap, ctx, seed, rng, dtype="f16"):
