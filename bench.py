@@ -3,13 +3,16 @@
 
 One step = one decode step of a 32-layer Llama-3-8B-shaped model (batch 1,
 32 query heads, 8 kv heads, d = 128, 32768 cached tokens, K4/V2, fp16): for
-every layer, tq_encode appends the new token's K/V to that layer's packed
-cache and tq_attend attends over all 32768 positions. The 32 layer caches
-(839 MB) are distinct, so successive reads of a layer are far apart and the
-126 MB L2 cannot hold them. Steps are CUDA-graph replays.
+every layer, one tq_attend_append launch appends the new token's K/V to that
+layer's packed cache and attends over all 32768 positions. The 32 layer
+caches (839 MB) are distinct, so successive reads of a layer are far apart
+and the 126 MB L2 cannot hold them. Steps are CUDA-graph replays.
 
   value   packed-KV GB/s: algorithmic bytes of the step (packed K/V rows,
-          fp16 norms, q and out, plus the encode's input/output) / step time
+          fp16 norms, q and out, plus the appended token's input/output) /
+          step time
+  roofline  the attention kernel alone (tq_attend over the same caches): a
+          CUDA graph of the 32 layer launches, time / 32 per launch
   e2e     the same bytes over a step that also copies the step's inputs from
           pinned host memory and its output back
   encode  bulk prefill encode of the same 32 x 8 x 32768 K/V (4.29 GB of fp16
@@ -274,13 +277,16 @@ def run_gpu(args, rank, world, local_rank):
                      ws, ws_bytes, outs[l], tq.TQ_F16, dev_status=status, stream=stream)
 
     def step():
+        # one decode step: per layer, the new token is appended to the
+        # compressed cache and attention runs over ctx positions, one launch
         for l in range(L):
-            tq.tq_encode(kv_new[l], tq.TQ_F16, 1, H, d, w.bits_k, w.bits_v, seed,
-                         caches.pk[l], caches.pv[l], caches.nk[l], caches.nv[l], cap, ctx - 1,
-                         status, stream)
-            attend_layer(l)
+            tq.tq_attend_append(q[l], tq.TQ_F16, kv_new[l], tq.TQ_F16, caches.pk[l],
+                                caches.nk[l], caches.pv[l], caches.nv[l], ctx_dev, 1,
+                                w.n_q_heads, w.gqa, d, w.bits_k, w.bits_v, seed, cap, 0.0, 0,
+                                ws, ws_bytes, outs[l], tq.TQ_F16, dev_status=status,
+                                stream=stream)
 
-    kernels_per_step = L * 2   # encode + attend per layer
+    kernels_per_step = L       # one tq_attend_append per layer
 
     def capture(fn):
         g = torch.cuda.CUDAGraph()
@@ -392,7 +398,8 @@ def run_gpu(args, rank, world, local_rank):
                    "kv_dtype": "fp16", "q_out_dtype": "fp16", "per_gpu": "one model replica",
                    "l2": f"inputs larger than L2: {L} distinct layer caches, "
                          f"{L * per_layer_attend / 1e6:.0f} MB per step",
-                   "step": "per layer: tq_encode(1 new token) + tq_attend(ctx positions), CUDA graph"},
+                   "step": "per layer: tq_attend_append (append the new token, attend over "
+                           "ctx positions; one launch), CUDA graph"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                      "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),

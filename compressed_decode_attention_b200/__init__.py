@@ -56,6 +56,9 @@ def lib() -> ctypes.CDLL:
         L.tq_attend.restype = I
         L.tq_attend.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F, I,
                                 P, SZ, P, P, P, I, P]
+        L.tq_attend_append.restype = I
+        L.tq_attend_append.argtypes = [P, I, P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F,
+                                       I, P, SZ, P, P, P, I, P]
         L.tq_attend_noalloc.restype = I
         L.tq_attend_noalloc.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F, I,
                                         P, P, P, I, P]
@@ -141,6 +144,21 @@ def tq_attend(q, q_dtype, packed_k, norms_k, packed_v, norms_v, ctx_lens, batch,
         bits_v, seed, cap_tok, float(sparse_v_thresh), n_ctas,
         _ptr(workspace), workspace_bytes, _ptr(dev_status),
         _ptr(sparse_v_skipped), _ptr(out), out_dtype, _stream(stream)))
+
+
+def tq_attend_append(q, q_dtype, new_kv, kv_dtype, packed_k, norms_k, packed_v, norms_v,
+                     ctx_lens, batch, n_q_heads, gqa_ratio, d, bits_k, bits_v, seed,
+                     cap_tok, sparse_v_thresh, n_ctas, workspace, workspace_bytes, out,
+                     out_dtype, dev_status=None, sparse_v_skipped=None, stream=None):
+    """One decode step: encode new_kv [2][batch][n_kv_heads][d] into cache row
+    ctx_lens[b] - 1 of every sequence, then attend over ctx_lens[b]
+    positions (the workspace contract of tq_attend)."""
+    _check("tq_attend_append", lib().tq_attend_append(
+        _ptr(q), q_dtype, _ptr(new_kv), kv_dtype, _ptr(packed_k), _ptr(norms_k),
+        _ptr(packed_v), _ptr(norms_v), _ptr(ctx_lens), batch, n_q_heads, gqa_ratio, d,
+        bits_k, bits_v, seed, cap_tok, float(sparse_v_thresh), n_ctas,
+        _ptr(workspace), workspace_bytes, _ptr(dev_status), _ptr(sparse_v_skipped),
+        _ptr(out), out_dtype, _stream(stream)))
 
 
 def tq_attend_noalloc(q, q_dtype, packed_k, norms_k, packed_v, norms_v, ctx_lens,

@@ -28,6 +28,70 @@ int from_cuda(cudaError_t e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA; }
 }  // namespace
 
 
+namespace tq {
+
+// Validation and launch shared by tq_attend and tq_attend_append.
+int attend_common(const void* q, int q_dtype, const void* new_kv, int kv_dtype,
+                  uint8_t* packed_k, uint16_t* norms_k, uint8_t* packed_v,
+                  uint16_t* norms_v, const int32_t* ctx_lens, int batch, int n_q_heads,
+                  int gqa_ratio, int d, int bits_k, int bits_v, uint64_t seed, int cap_tok,
+                  float sparse_v_thresh, int n_ctas, void* workspace, size_t workspace_bytes,
+                  int* dev_status, unsigned long long* sparse_v_skipped, void* out,
+                  int out_dtype, void* stream) {
+  if (batch < 1 || n_q_heads < 1 || gqa_ratio < 1 || cap_tok < 1)
+    return TQ_ERR_INVALID_ARG;
+  if (n_q_heads % gqa_ratio) return TQ_ERR_INVALID_ARG;
+  if (gqa_ratio > kMaxGroup) return TQ_ERR_UNSUPPORTED;
+  if (q_dtype < TQ_F16 || q_dtype > TQ_F32 || out_dtype < TQ_F16 || out_dtype > TQ_F32)
+    return TQ_ERR_INVALID_ARG;
+  if (!bits_ok(bits_k) || !bits_ok(bits_v)) return TQ_ERR_INVALID_ARG;
+  if (n_ctas < 0 || n_ctas > kMaxCtas) return TQ_ERR_INVALID_ARG;
+  if (isnan(sparse_v_thresh)) return TQ_ERR_INVALID_ARG;
+  const int hd = check_head_dim(d);
+  if (hd != TQ_OK) return hd;
+  if (cap_tok % 8) return TQ_ERR_UNSUPPORTED;
+  if (!q || !packed_k || !norms_k || !packed_v || !norms_v || !ctx_lens || !out ||
+      !workspace)
+    return TQ_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(packed_k) || !aligned16(packed_v) ||
+      !aligned16(norms_k) || !aligned16(norms_v) || !aligned16(workspace) ||
+      ((uintptr_t)ctx_lens & 3u) || ((uintptr_t)sparse_v_skipped & 7u) ||
+      ((uintptr_t)dev_status & 3u))
+    return TQ_ERR_INVALID_ARG;
+  if (workspace_bytes < attend_workspace_bytes(batch, n_q_heads)) return TQ_ERR_INVALID_ARG;
+  const Codebook* cbk = codebook_for(bits_k);
+  const Codebook* cbv = codebook_for(bits_v);
+  if (!cbk || !cbv) return TQ_ERR_NO_CONVERGENCE;
+  AttendArgs a;
+  a.q = q;
+  a.q_dtype = q_dtype;
+  a.packed_k = packed_k;
+  a.norms_k = norms_k;
+  a.packed_v = packed_v;
+  a.norms_v = norms_v;
+  a.new_kv = (const uint16_t*)new_kv;
+  a.new_kv_bf16 = kv_dtype == TQ_BF16;
+  a.ctx_lens = ctx_lens;
+  a.batch = batch;
+  a.n_q_heads = n_q_heads;
+  a.gqa = gqa_ratio;
+  a.n_kv_heads = n_q_heads / gqa_ratio;
+  a.bits_k = bits_k;
+  a.bits_v = bits_v;
+  a.cap_tok = cap_tok;
+  a.tau = sparse_v_thresh;
+  a.counters = (int*)workspace;
+  a.slots = (float*)((uint8_t*)workspace + attend_counter_bytes(batch, n_q_heads));
+  a.dev_status = dev_status;
+  a.skipped = sparse_v_skipped;
+  a.out = out;
+  a.out_dtype = out_dtype;
+  return from_cuda(launch_attend(a, *cbk, *cbv, sign_mask(seed), n_ctas,
+                                 (cudaStream_t)stream));
+}
+
+}  // namespace tq
+
 extern "C" {
 
 int tq_abi_version(void) { return TQ_ABI_VERSION; }
@@ -130,54 +194,29 @@ int tq_attend(const void* q, int q_dtype, const uint8_t* packed_k,
               void* workspace, size_t workspace_bytes, int* dev_status,
               unsigned long long* sparse_v_skipped, void* out, int out_dtype,
               void* stream) {
-  if (batch < 1 || n_q_heads < 1 || gqa_ratio < 1 || cap_tok < 1)
-    return TQ_ERR_INVALID_ARG;
-  if (n_q_heads % gqa_ratio) return TQ_ERR_INVALID_ARG;
-  if (gqa_ratio > kMaxGroup) return TQ_ERR_UNSUPPORTED;
-  if (q_dtype < TQ_F16 || q_dtype > TQ_F32 || out_dtype < TQ_F16 || out_dtype > TQ_F32)
-    return TQ_ERR_INVALID_ARG;
-  if (!bits_ok(bits_k) || !bits_ok(bits_v)) return TQ_ERR_INVALID_ARG;
-  if (n_ctas < 0 || n_ctas > kMaxCtas) return TQ_ERR_INVALID_ARG;
-  if (isnan(sparse_v_thresh)) return TQ_ERR_INVALID_ARG;
-  const int hd = check_head_dim(d);
-  if (hd != TQ_OK) return hd;
-  if (cap_tok % 8) return TQ_ERR_UNSUPPORTED;
-  if (!q || !packed_k || !norms_k || !packed_v || !norms_v || !ctx_lens || !out ||
-      !workspace)
-    return TQ_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(out) || !aligned16(packed_k) || !aligned16(packed_v) ||
-      !aligned16(norms_k) || !aligned16(norms_v) || !aligned16(workspace) ||
-      ((uintptr_t)ctx_lens & 3u) || ((uintptr_t)sparse_v_skipped & 7u) ||
-      ((uintptr_t)dev_status & 3u))
-    return TQ_ERR_INVALID_ARG;
-  if (workspace_bytes < attend_workspace_bytes(batch, n_q_heads)) return TQ_ERR_INVALID_ARG;
-  const Codebook* cbk = codebook_for(bits_k);
-  const Codebook* cbv = codebook_for(bits_v);
-  if (!cbk || !cbv) return TQ_ERR_NO_CONVERGENCE;
-  AttendArgs a;
-  a.q = q;
-  a.q_dtype = q_dtype;
-  a.packed_k = packed_k;
-  a.norms_k = norms_k;
-  a.packed_v = packed_v;
-  a.norms_v = norms_v;
-  a.ctx_lens = ctx_lens;
-  a.batch = batch;
-  a.n_q_heads = n_q_heads;
-  a.gqa = gqa_ratio;
-  a.n_kv_heads = n_q_heads / gqa_ratio;
-  a.bits_k = bits_k;
-  a.bits_v = bits_v;
-  a.cap_tok = cap_tok;
-  a.tau = sparse_v_thresh;
-  a.counters = (int*)workspace;
-  a.slots = (float*)((uint8_t*)workspace + attend_counter_bytes(batch, n_q_heads));
-  a.dev_status = dev_status;
-  a.skipped = sparse_v_skipped;
-  a.out = out;
-  a.out_dtype = out_dtype;
-  return from_cuda(launch_attend(a, *cbk, *cbv, sign_mask(seed), n_ctas,
-                                 (cudaStream_t)stream));
+  return tq::attend_common(q, q_dtype, nullptr, TQ_F16, const_cast<uint8_t*>(packed_k),
+                           const_cast<uint16_t*>(norms_k), const_cast<uint8_t*>(packed_v),
+                           const_cast<uint16_t*>(norms_v), ctx_lens, batch, n_q_heads,
+                           gqa_ratio, d, bits_k, bits_v, seed, cap_tok, sparse_v_thresh,
+                           n_ctas, workspace, workspace_bytes, dev_status, sparse_v_skipped,
+                           out, out_dtype, stream);
+}
+
+int tq_attend_append(const void* q, int q_dtype, const void* new_kv, int kv_dtype,
+                     uint8_t* packed_k, uint16_t* norms_k, uint8_t* packed_v,
+                     uint16_t* norms_v, const int32_t* ctx_lens, int batch,
+                     int n_q_heads, int gqa_ratio, int d, int bits_k, int bits_v,
+                     uint64_t seed, int cap_tok, float sparse_v_thresh, int n_ctas,
+                     void* workspace, size_t workspace_bytes, int* dev_status,
+                     unsigned long long* sparse_v_skipped, void* out, int out_dtype,
+                     void* stream) {
+  if (!new_kv) return TQ_ERR_INVALID_ARG;
+  if (kv_dtype != TQ_F16 && kv_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
+  if (!aligned16(new_kv)) return TQ_ERR_INVALID_ARG;
+  return tq::attend_common(q, q_dtype, new_kv, kv_dtype, packed_k, norms_k, packed_v, norms_v,
+                           ctx_lens, batch, n_q_heads, gqa_ratio, d, bits_k, bits_v, seed,
+                           cap_tok, sparse_v_thresh, n_ctas, workspace, workspace_bytes,
+                           dev_status, sparse_v_skipped, out, out_dtype, stream);
 }
 
 }  // extern "C"

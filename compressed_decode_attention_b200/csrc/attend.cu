@@ -41,7 +41,7 @@
 // Output, once per (batch, query head): D⊙(H·(acc/l))/d with shuffles.
 #include <math.h>
 
-#include "device_common.cuh"
+#include "encode_common.cuh"
 
 namespace tq {
 namespace {
@@ -103,7 +103,9 @@ struct Geo {
   static constexpr int QS = kMaxGroup * kHeadDim * 2 * 2;  // q~ high and low, fp16
   static constexpr int MISC = 1024;                     // kMiscWords words
   static constexpr int MBAR = kWarps * kMaxStages * 8;  // per-warp ring barriers
-  static constexpr int FIXED = QOFF + QS + MISC + MBAR;
+  static constexpr int APPOFF = QOFF + QS + MISC + MBAR;  // decode-step append:
+  static constexpr int APP = 256;                       //   K row, V row, norms
+  static constexpr int FIXED = APPOFF + APP;
   static constexpr int NFIT = (kSmemBudget - FIXED) / (kWarps * STAGE);
   static constexpr int NSTAGE = NFIT > kMaxStages ? kMaxStages : NFIT;
   static constexpr int MERGE = kWarps * kMergeStride * 4;
@@ -672,6 +674,42 @@ attend_kernel(const __grid_constant__ AttendArgs a,
       if (lane == 0) miscf[kMiscQInv + warp] = 1.f / (qs * kKScale);
       fill_ring();
     }
+    // ---- decode-step append: the warp whose range ends at the sequence's
+    // last position encodes the new token of (b, g) (lanes 0-3: K, 4-7: V;
+    // the encode kernel's per-vector code), stores it in cache row L - 1 and
+    // keeps a copy to patch into its staged last chunk.
+    const bool app = a.new_kv != nullptr && blk0 + nseg == nbl && nw > 0 && wp1 == L;
+    uint8_t* app_k = smem + Gm::APPOFF;
+    uint8_t* app_v = app_k + 64;
+    uint16_t* app_n = reinterpret_cast<uint16_t*>(app_k + 128);
+    if (app) {
+      if (lane < 8) {
+        const int sub = lane & 3;
+        const bool isv = lane >= 4;
+        uint32_t smask[16];
+        sign_masks(sm, sub, smask);
+        const uint16_t* src = a.new_kv + ((size_t)((isv ? B : 0) + b) * H + g) * kHeadDim;
+        float x[32];
+        load_signed(src, sub, a.new_kv_bf16 != 0, smask, x);
+        const unsigned gmask = 0xFu << (lane & ~3);
+        if (isv)
+          encode_vector<BV>(x, cbv, sub, gmask, app_v, app_n + 1, a.dev_status);
+        else
+          encode_vector<BK>(x, cbk, sub, gmask, app_k, app_n, a.dev_status);
+      }
+      __syncwarp();
+      const size_t row = seq_row + (size_t)(L - 1);
+      if (lane < Gm::RK / 4)
+        reinterpret_cast<uint32_t*>(a.packed_k + row * Gm::RK)[lane] =
+            reinterpret_cast<const uint32_t*>(app_k)[lane];
+      if (lane < Gm::RV / 4)
+        reinterpret_cast<uint32_t*>(a.packed_v + row * Gm::RV)[lane] =
+            reinterpret_cast<const uint32_t*>(app_v)[lane];
+      if (lane == 0) {
+        a.norms_k[row] = app_n[0];
+        a.norms_v[row] = app_n[1];
+      }
+    }
     __syncthreads();
 
     // ---- query fragments (B operand of the score MMA), column n = gq.
@@ -708,6 +746,20 @@ attend_kernel(const __grid_constant__ AttendArgs a,
       const int t0 = wp0 + i * kBlk;                // chunk [t0, cend)
       const int cend = min(wp1, t0 + kBlk);
       const bool partial = cend < t0 + kBlk;
+      if (app && cend == L) {                       // the staged row L - 1 is stale
+        const int r = L - 1 - t0;
+        if (lane < Gm::RK / 4)
+          *reinterpret_cast<uint32_t*>(smem + st + r * Gm::RK + 4 * lane) =
+              reinterpret_cast<const uint32_t*>(app_k)[lane];
+        if (lane < Gm::RV / 4)
+          *reinterpret_cast<uint32_t*>(smem + st + Gm::KB + r * Gm::RV + 4 * lane) =
+              reinterpret_cast<const uint32_t*>(app_v)[lane];
+        if (lane == 0) {
+          *reinterpret_cast<uint16_t*>(smem + st + Gm::NKOFF + 2 * r) = app_n[0];
+          *reinterpret_cast<uint16_t*>(smem + st + Gm::NKOFF + 2 * kBlk + 2 * r) = app_n[1];
+        }
+        __syncwarp();
+      }
 
       // -- scores: 4 steps of 16 positions, each as two 8-position groups.
       // A operand rows 0-7 are the K codebook high parts of the group's

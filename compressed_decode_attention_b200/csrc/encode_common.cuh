@@ -1,0 +1,142 @@
+// Per-vector encode shared by the encode kernel and the fused decode-step
+// append: FP16 norm, randomized Hadamard rotation, Lloyd-Max index and
+// LSB-first packing of one d = 128 vector held by a group of four lanes
+// (32 consecutive coordinates per lane).
+//
+// [TQAI §The Paper]: keep the norm in FP16, rotate the unit vector,
+// quantize each coordinate with the precomputed Lloyd-Max codebook.
+// [ADAPTQ §How it works, item 1]: y = (1/sqrt d)·H·D·x with a fast
+// Walsh-Hadamard transform. [TQAI §What's Next]: indices bit-packed at
+// 2/3/4 bits.
+#pragma once
+
+#include "device_common.cuh"
+
+namespace tq {
+
+// XOR masks that flip the fp16/bf16 sign bits of coordinates 2j (bit 15) and
+// 2j+1 (bit 31) of lane `sub`'s 16 half2 words where D = -1.
+__device__ __forceinline__ void sign_masks(const SignMask& sm, int sub, uint32_t (&smask)[16]) {
+  const uint32_t m = sm.w[sub];
+#pragma unroll
+  for (int j = 0; j < 16; ++j)
+    smask[j] = (((m >> (2 * j)) & 1u) << 15) | (((m >> (2 * j + 1)) & 1u) << 31);
+}
+
+// Coordinates 32·sub .. 32·sub + 31 of the vector at src (fp16 or bf16),
+// multiplied by D, as float.
+__device__ __forceinline__ void load_signed(const uint16_t* src, int sub, bool bf16,
+                                            const uint32_t (&smask)[16], float (&x)[32]) {
+  const uint4* p = reinterpret_cast<const uint4*>(src + 32 * sub);
+  uint4 raw[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) raw[k] = __ldcs(p + k);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t w4[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = unpack16x2(w4[j] ^ smask[4 * k + j], bf16);
+      x[8 * k + 2 * j] = f.x;
+      x[8 * k + 2 * j + 1] = f.y;
+    }
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ void encode_vector(
+    float (&x)[32], const Codebook& cb, int sub, unsigned gmask,
+    uint8_t* row_dst, uint16_t* norm_dst, int* dev_status) {
+  constexpr int kHalf = 1 << (BITS - 1);
+  // ||x||^2 over the group of four lanes (pairs of coordinates per fma)
+  float2 ss2 = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const float2 v = make_float2(x[2 * j], x[2 * j + 1]);
+    ss2 = f2fma(v, v, ss2);
+  }
+  float ss = ss2.x + ss2.y;
+  ss += __shfl_xor_sync(gmask, ss, 1);
+  ss += __shfl_xor_sync(gmask, ss, 2);
+  const float n = sqrtf(ss);
+
+  // z = H·(D⊙x): coordinate 32·sub + i lives in register i of lane sub.
+  // Stride 1 in scalar form, strides 2..16 on register pairs, strides 32 and
+  // 64 across the four lanes (x' = partner + sign·x, sign = -1 on the upper
+  // lane); every step rounds exactly like a scalar add or subtract.
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const float u = x[2 * j], v = x[2 * j + 1];
+    x[2 * j] = u + v;
+    x[2 * j + 1] = u - v;
+  }
+#pragma unroll
+  for (int s = 2; s < 32; s <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      if ((i & s) == 0) {
+        const float2 u = make_float2(x[i], x[i + 1]), v = make_float2(x[i + s], x[i + s + 1]);
+        const float2 p = f2add(u, v), m = f2sub(u, v);
+        x[i] = p.x; x[i + 1] = p.y;
+        x[i + s] = m.x; x[i + s + 1] = m.y;
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 1; o <= 2; o <<= 1) {
+    const float sg = (sub & o) ? -1.f : 1.f;
+    const float2 sg2 = make_float2(sg, sg);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float2 v = make_float2(x[2 * j], x[2 * j + 1]);
+      const float2 p = make_float2(__shfl_xor_sync(gmask, v.x, o), __shfl_xor_sync(gmask, v.y, o));
+      const float2 r = f2fma(v, sg2, p);
+      x[2 * j] = r.x;
+      x[2 * j + 1] = r.y;
+    }
+  }
+
+  // idx = #{j : z/n >= t_j}, evaluated as z against n·t_j. Positive half of
+  // the table: T_k = n·t_{half-1+k}, k = 1..half-1 (t_{half-1} = 0).
+  // z >= 0: idx = half + #{k : T_k <= z};  z < 0: idx = half-1 - #{k : T_k < |z|}.
+  // The strict comparison uses |z| lowered by one ulp. A zero vector keeps
+  // n = 0, z = 0 and must land on idx = half: scale the table by 1 instead.
+  // Counts are sums of compare results (0 or -1).
+  const float sc = n > 0.f ? n : 1.f;
+  float T[kHalf > 1 ? kHalf - 1 : 1];
+#pragma unroll
+  for (int k = 1; k < kHalf; ++k) T[k - 1] = sc * cb.threshold[kHalf - 1 + k];
+
+  uint32_t words[BITS] = {};
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float z = x[i];
+    const bool neg = z < 0.f;
+    const float a = __uint_as_float((__float_as_uint(z) & 0x7FFFFFFFu) - (neg ? 1u : 0u));
+    uint32_t s = 0;                                   // = -count
+#pragma unroll
+    for (int k = 0; k < kHalf - 1; ++k) s += set_ge(a, T[k]);
+    const uint32_t idx = neg ? (uint32_t)(kHalf - 1) + s : (uint32_t)kHalf - s;
+    const int p = i * BITS, w = p >> 5, off = p & 31;
+    words[w] += idx << off;                           // fields do not overlap
+    if (off + BITS > 32) words[w + 1] += idx >> (32 - off);
+  }
+
+  if constexpr (BITS == 4) {
+    *reinterpret_cast<uint4*>(row_dst + 16 * sub) =
+        make_uint4(words[0], words[1], words[2], words[3]);
+  } else if constexpr (BITS == 2) {
+    *reinterpret_cast<uint2*>(row_dst + 8 * sub) = make_uint2(words[0], words[1]);
+  } else {
+    uint32_t* d32 = reinterpret_cast<uint32_t*>(row_dst + 12 * sub);
+    d32[0] = words[0];
+    d32[1] = words[1];
+    d32[2] = words[2];
+  }
+  if (sub == 0) {
+    *norm_dst = f32_to_f16_bits(fminf(n, 65504.f));
+    if (n > 65504.f && dev_status) atomicOr(dev_status, TQ_DEV_NORM_SATURATED);
+  }
+}
+
+}  // namespace tq

@@ -63,10 +63,15 @@ cudaError_t launch_dequant(const DequantArgs& a, const Codebook& cb,
 struct AttendArgs {
   const void* q;
   int q_dtype;
-  const uint8_t* packed_k;
-  const uint16_t* norms_k;
-  const uint8_t* packed_v;
-  const uint16_t* norms_v;
+  // The cache; written only by the decode-step append (new_kv != nullptr).
+  uint8_t* packed_k;
+  uint16_t* norms_k;
+  uint8_t* packed_v;
+  uint16_t* norms_v;
+  // Decode-step append: [2][batch][n_kv_heads][d] fp16/bf16 new K/V (one
+  // token per sequence), encoded into row ctx_lens[b] - 1; nullptr = none.
+  const uint16_t* new_kv;
+  int new_kv_bf16;
   const int32_t* ctx_lens;
   int batch, n_q_heads, gqa, n_kv_heads;
   int bits_k, bits_v;

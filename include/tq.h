@@ -71,7 +71,7 @@
 extern "C" {
 #endif
 
-#define TQ_ABI_VERSION 1
+#define TQ_ABI_VERSION 2
 
 /* Tokens per sparse-V block; split boundaries are multiples of this. */
 #define TQ_SPARSE_V_BLOCK 64
@@ -230,6 +230,40 @@ int tq_attend(const void* q, int q_dtype,
               void* workspace, size_t workspace_bytes, int* dev_status,
               unsigned long long* sparse_v_skipped,
               void* out, int out_dtype, void* stream);
+
+/*
+ * tq_attend_append — one decode step in one launch: append the new token of
+ * every sequence to the compressed cache, then attend over the cache
+ * including it. The pages' decode loop updates the cache with the new
+ * key/value pair before attention runs ("We Built a Python Library That Cuts
+ * LLM Memory Usage by 80%", §The Paper: cache.update() ahead of the
+ * attention call); this entry point does both steps in one kernel.
+ *
+ * Equivalent, bit for bit in the cache and within the attention tolerance in
+ * out, to: for every b with L_b = min(ctx_lens[b], cap_tok) >= 1,
+ *   tq_encode(new_kv[:, b], n_tok = 1, tok_offset = L_b - 1) on sequence b's
+ *   cache, followed by tq_attend(...) with the same arguments.
+ *
+ *   new_kv      [2][batch][n_kv_heads][d] of kv_dtype (TQ_F16 | TQ_BF16),
+ *               16-byte aligned: the new key (index 0) and value (index 1)
+ *               of each sequence. ctx_lens counts the new token.
+ *   packed_*, norms_*  the cache (written: row L_b - 1 of every kv head of
+ *               every sequence with L_b >= 1). Sequences with ctx_lens[b] <= 0
+ *               append nothing (out = 0, TQ_DEV_CTX_EMPTY); ctx_lens[b] >
+ *               cap_tok writes row cap_tok - 1 (TQ_DEV_CTX_CLAMPED).
+ *   TQ_DEV_NORM_SATURATED is set as in tq_encode.
+ * All other arguments, the workspace contract and the errors are those of
+ * tq_attend; a null new_kv or another kv_dtype is TQ_ERR_INVALID_ARG.
+ */
+int tq_attend_append(const void* q, int q_dtype, const void* new_kv, int kv_dtype,
+                     uint8_t* packed_k, uint16_t* norms_k,
+                     uint8_t* packed_v, uint16_t* norms_v,
+                     const int32_t* ctx_lens, int batch, int n_q_heads,
+                     int gqa_ratio, int d, int bits_k, int bits_v, uint64_t seed,
+                     int cap_tok, float sparse_v_thresh, int n_ctas,
+                     void* workspace, size_t workspace_bytes, int* dev_status,
+                     unsigned long long* sparse_v_skipped,
+                     void* out, int out_dtype, void* stream);
 
 /*
  * tq_attend_noalloc — tq_attend for callers that cannot allocate device
