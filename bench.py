@@ -73,7 +73,7 @@ def encode_bytes(w, n_vec_pairs):
 
 def kernel_source_sha():
     h = hashlib.sha256()
-    for fn in ("attend.cu", "encode_common.cuh", "device_common.cuh", "tq_internal.h"):
+    for fn in ("attend_kernel.cuh", "encode_common.cuh", "device_common.cuh", "tq_internal.h"):
         with open(os.path.join(ROOT, "compressed_decode_attention_b200", "csrc", fn), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

@@ -15,8 +15,7 @@ bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 int check_head_dim(int d) {
   if (d <= 0 || (d & (d - 1))) return TQ_ERR_INVALID_ARG;
   if (d < 64 || d > 256) return TQ_ERR_INVALID_ARG;
-  if (d != kHeadDim) return TQ_ERR_UNSUPPORTED;
-  return TQ_OK;
+  return TQ_OK;                              // 64, 128, 256
 }
 
 bool bits_ok(int b) { return b >= 2 && b <= 4; }
@@ -58,7 +57,7 @@ int attend_common(const void* q, int q_dtype, const void* new_kv, int kv_dtype,
       ((uintptr_t)ctx_lens & 3u) || ((uintptr_t)sparse_v_skipped & 7u) ||
       ((uintptr_t)dev_status & 3u))
     return TQ_ERR_INVALID_ARG;
-  if (workspace_bytes < attend_workspace_bytes(batch, n_q_heads)) return TQ_ERR_INVALID_ARG;
+  if (workspace_bytes < attend_workspace_bytes(batch, n_q_heads, d)) return TQ_ERR_INVALID_ARG;
   const Codebook* cbk = codebook_for(bits_k);
   const Codebook* cbv = codebook_for(bits_v);
   if (!cbk || !cbv) return TQ_ERR_NO_CONVERGENCE;
@@ -72,6 +71,7 @@ int attend_common(const void* q, int q_dtype, const void* new_kv, int kv_dtype,
   a.new_kv = (const uint16_t*)new_kv;
   a.new_kv_bf16 = kv_dtype == TQ_BF16;
   a.ctx_lens = ctx_lens;
+  a.d = d;
   a.batch = batch;
   a.n_q_heads = n_q_heads;
   a.gqa = gqa_ratio;
@@ -140,6 +140,7 @@ int tq_encode(const void* kv, int dtype, int n_tok, int n_kv_heads, int d,
   if (!cbk || !cbv) return TQ_ERR_NO_CONVERGENCE;
   EncodeArgs a;
   a.kv = (const uint16_t*)kv;
+  a.d = d;
   a.is_bf16 = dtype == TQ_BF16;
   a.n_tok = n_tok;
   a.n_kv_heads = n_kv_heads;
@@ -170,6 +171,7 @@ int tq_dequant(const uint8_t* packed, const uint16_t* norms, int n_tok,
   const Codebook* cb = codebook_for(bits);
   if (!cb) return TQ_ERR_NO_CONVERGENCE;
   DequantArgs a;
+  a.d = d;
   a.packed = packed;
   a.norms = norms;
   a.n_tok = n_tok;
@@ -182,8 +184,8 @@ int tq_dequant(const uint8_t* packed, const uint16_t* norms, int n_tok,
 }
 
 size_t tq_attend_workspace_size(int batch, int n_q_heads, int cap_tok, int d) {
-  if (batch < 1 || n_q_heads < 1 || cap_tok < 1 || d != kHeadDim) return 0;
-  return attend_workspace_bytes(batch, n_q_heads);
+  if (batch < 1 || n_q_heads < 1 || cap_tok < 1 || check_head_dim(d) != TQ_OK) return 0;
+  return attend_workspace_bytes(batch, n_q_heads, d);
 }
 
 int tq_attend(const void* q, int q_dtype, const uint8_t* packed_k,

@@ -1,5 +1,6 @@
 // tq_attend: decode attention over the packed cache in one persistent,
-// load-balanced kernel on the B200 tensor cores.
+// load-balanced kernel on the B200 tensor cores. The kernel template is in
+// attend_kernel.cuh; this file dispatches on the head dimension.
 //
 // [ADAPTQ §How it works, item 3]: the query is rotated once; scores are
 // formed from the packed indices through the codebook, without materializing
@@ -39,1132 +40,18 @@
 //           score layout with movmatrix. V2: position pairs by byte permutes
 //           of a 4-entry register table; V3/V4: pair table + movmatrix.
 // Output, once per (batch, query head): D⊙(H·(acc/l))/d with shuffles.
-#include <math.h>
-
-#include "encode_common.cuh"
+#include "tq_internal.h"
 
 namespace tq {
-namespace {
-
-constexpr int kWarps = 12;
-constexpr int kThreads = 32 * kWarps;
-constexpr int kBlk = kGateBlock;                // positions per block
-constexpr float kLog2e = 1.44269504088896340736f;
-constexpr float kKScale = 256.f;                // K codebook scale inside the MMA
-constexpr int kSmemBudget = 227 * 1024;
-constexpr int kMaxStages = 3;                   // ring slots per warp
-constexpr int kMergeChunk = 16;                 // partials per round of loads
-// Give up on a staged-data wait after this many cycles (~1 s at 2 GHz).
-constexpr long long kWaitLimitCycles = 2000000000LL;
-
-constexpr int ceil_pow2(int x) {
-  int p = 1;
-  while (p < x) p <<= 1;
-  return p;
-}
-
-// misc words
-constexpr int kMiscSeg = 0;      // b, g, blk0, nseg, nb, L
-constexpr int kMiscLast = 8;     // last-CTA flag
-constexpr int kMiscNB = 9;       // flat block count (lo, hi), common length
-constexpr int kMiscState = 12;   // scan state: sb, sP (lo, hi)
-constexpr int kMiscQInv = 16;    // 8 floats: 1/(query scale · kKScale)
-constexpr int kMiscM = 32;       // 8 floats: merged max
-constexpr int kMiscL = 40;       // 8 floats: merged sum
-constexpr int kMiscCb = 64;      // 32 words: staged codebooks
-constexpr int kMiscWt = 128;     // kWarps x 8 floats: per-warp merge weights
-constexpr int kMiscWords = 256;  // Geo::MISC / 4
-// Per-warp merge buffer (floats): accumulators (in register order 32 per
-// lane at a stride of kMergeLane, which keeps 16-byte stores of consecutive
-// lanes on distinct banks; or in output order), then per-head max and sum.
-constexpr int kMergeLane = 36;
-constexpr int kMergeM = 32 * kMergeLane;
-constexpr int kMergeL = kMergeM + kMaxGroup;
-constexpr int kMergeStride = kMergeL + kMaxGroup;
-static_assert(kMiscWt + kWarps * kMaxGroup <= kMiscWords, "misc words");
-
-template <int BK, int BV>
-struct Geo {
-  static constexpr int RK = 16 * BK;                    // packed K row bytes
-  static constexpr int RV = 16 * BV;
-  static constexpr int RVS = RV;                        // V row stride in smem
-  static constexpr int KB = kBlk * RK;
-  static constexpr int VB = kBlk * RVS;
-  static constexpr int NKOFF = KB + VB;
-  static constexpr int STAGE = KB + VB + 2 * kBlk * 2;
-  // K table: uint2 (high pair, low pair) per (pair code, lane & 15): 128 B per code.
-  static constexpr int LUTK = (1 << (2 * BK)) * 128;
-  // V table (3/4 bits): uint32 fp16 pair per (pair code, lane): 128 B per code.
-  static constexpr int LUTV = BV == 2 ? 0 : (1 << (2 * BV)) * 128;
-  // The V table sits at a power-of-two offset no smaller than either table,
-  // so entry addresses are formed with OR.
-  static constexpr int LUTV_OFF = BV == 2 ? LUTK : ceil_pow2(LUTK > LUTV ? LUTK : LUTV);
-  static constexpr int QOFF = LUTV_OFF + LUTV;
-  static constexpr int QS = kMaxGroup * kHeadDim * 2 * 2;  // q~ high and low, fp16
-  static constexpr int MISC = 1024;                     // kMiscWords words
-  static constexpr int MBAR = kWarps * kMaxStages * 8;  // per-warp ring barriers
-  static constexpr int APPOFF = QOFF + QS + MISC + MBAR;  // decode-step append:
-  static constexpr int APP = 256;                       //   K row, V row, norms
-  static constexpr int FIXED = APPOFF + APP;
-  static constexpr int NFIT = (kSmemBudget - FIXED) / (kWarps * STAGE);
-  static constexpr int NSTAGE = NFIT > kMaxStages ? kMaxStages : NFIT;
-  static constexpr int MERGE = kWarps * kMergeStride * 4;
-  static constexpr int RING = NSTAGE * kWarps * STAGE;
-  static constexpr int SMEM = FIXED + (RING > MERGE ? RING : MERGE);
-  static_assert(NSTAGE >= 1, "stage ring does not fit");
-  static_assert(SMEM <= kSmemBudget, "shared memory budget");
-};
-
-
-__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1,
-                                         uint32_t a2, uint32_t a3, uint32_t b0,
-                                         uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, "
-      "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
-  uint32_t y;
-  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
-  return y;
-}
-
-__device__ __forceinline__ float fast_exp2(float x) {   // ex2.approx: -inf -> 0
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
-  return y;
-}
-
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
-               "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;\n" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
-}
-
-// Shared-memory barrier with a transaction count, completed by bulk copies.
-__device__ __forceinline__ void mbar_init(uint32_t bar) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_expect(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(done) : "r"(bar), "r"(parity) : "memory");
-  return done != 0;
-}
-// Slow path of mbar_wait, out of line: keeps polling until the phase
-// completes or kWaitLimitCycles have passed.
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (!mbar_try(bar, parity))
-    if (clock64() - t0 > kWaitLimitCycles) return false;
-  return true;
-}
-// Waits for the phase with the given parity to complete; false if it does
-// not within kWaitLimitCycles.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-  return mbar_try(bar, parity) || mbar_wait_slow(bar, parity);
-}
-// Bulk copy global -> this CTA's shared memory (16-byte aligned, size a
-// multiple of 16), completing on `bar`.
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
-                                         uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
-      ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
-}
-
-template <typename T>
-__device__ __forceinline__ T lds(const uint8_t* base, uint32_t off) {
-  return *reinterpret_cast<const T*>(base + off);
-}
-
-__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
-  __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
-__device__ __forceinline__ float load_elem(const void* p, int dtype, size_t i) {
-  if (dtype == TQ_F32) return reinterpret_cast<const float*>(p)[i];
-  const uint16_t v = reinterpret_cast<const uint16_t*>(p)[i];
-  if (dtype == TQ_BF16) return __uint_as_float((uint32_t)v << 16);
-  return __half2float(__ushort_as_half(v));
-}
-
-__device__ __forceinline__ int seq_blocks(const AttendArgs& a, int b) {
-  const int L = min(max(a.ctx_lens[b], 0), a.cap_tok);
-  return (L + kBlk - 1) / kBlk;
-}
-
-// CTA owning flat block `blk` when NB blocks are split over G CTAs as
-// [c·NB/G, (c+1)·NB/G): the largest c with floor(c·NB/G) <= blk.
-__device__ __forceinline__ int cta_of(long long blk, long long nb, int g) {
-  return (int)(((blk + 1) * g - 1) / nb);
-}
-
-// Walsh-Hadamard transform of 128 values spread as 4 per lane (coordinate
-// 4·lane + k in x[k]): two in-register stages, five shuffle stages.
-__device__ __forceinline__ void fwht128_warp(float (&x)[4], int lane) {
-#pragma unroll
-  for (int s = 1; s < 4; s <<= 1)
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-      if (!(k & s)) {
-        const float u = x[k], v = x[k + s];
-        x[k] = u + v;
-        x[k + s] = u - v;
-      }
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const bool upper = lane & o;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float p = __shfl_xor_sync(0xFFFFFFFFu, x[k], o);
-      x[k] = upper ? p - x[k] : x[k] + p;
-    }
-  }
-}
-
-// Output coordinate held by accumulator register (m-tile r, m-slot m) of PV.
-template <int BV>
-__device__ __forceinline__ int pv_coord(int r, int m) {
-  if (BV == 2) return 16 * (m & 7) + 2 * r + (m >> 3);
-  return 32 * ((m & 7) >> 1) + 4 * r + (m & 1) + 2 * (m >> 3);
-}
-
-// Position of output (head h, coordinate c) in a warp's accumulators as
-// stored lane-major (register acc[r][k] of a lane at 4r + k):
-// the inverse of pv_coord together with the head columns 2tq, 2tq + 1.
-template <int BV>
-__device__ __forceinline__ int pv_slot(int c, int h) {
-  int m, r;
-  if (BV == 2) {
-    m = (c >> 4) + 8 * (c & 1);
-    r = (c & 15) >> 1;
-  } else {
-    m = 2 * (c >> 5) + (c & 1) + 8 * ((c >> 1) & 1);
-    r = (c & 31) >> 2;
-  }
-  const int lane = 4 * (m & 7) + (h >> 1);
-  return lane * kMergeLane + 4 * r + (h & 1) + 2 * (m >> 3);
-}
-
-// (pair code p of a lane's chunk of packed words) << SHIFT, for a table
-// whose entries are 2^SHIFT bytes apart. Codes are 2·BITS bits wide
-// (coordinates 2p, 2p+1), little-endian in the chunk.
-template <int BITS, int SHIFT>
-__device__ __forceinline__ uint32_t pair_code_shifted(const uint32_t* w, int p) {
-  constexpr int FB = 2 * BITS;
-  constexpr uint32_t MASK = ((1u << FB) - 1u) << SHIFT;
-  const int bit = p * FB;
-  const int k = bit >> 5, off = bit & 31;
-  if (off + FB > 32) return (__funnelshift_r(w[k], w[k + 1], off) << SHIFT) & MASK;
-  if (off >= SHIFT) return (w[k] >> (off - SHIFT)) & MASK;
-  return (w[k] << (SHIFT - off)) & MASK;
-}
-
-// Byte offset of the K table entry for pair code p of a lane's chunk (entries
-// 128 bytes apart). For 4-bit codes the pair code is a whole byte: one byte
-// permute and one multiply-add; narrower codes straddle bytes.
-template <int BK>
-__device__ __forceinline__ uint32_t k_entry(const uint32_t* w, int p) {
-  if constexpr (BK == 4)
-    return (uint32_t)__byte_perm(w[p >> 2], 0u, 0x4440u | (uint32_t)(p & 3)) * 128u;
-  else
-    return pair_code_shifted<BK, 7>(w, p);
-}
-
-template <int BK, int BV, int NT>
-__global__ void __launch_bounds__(kThreads, 1)
-attend_kernel(const __grid_constant__ AttendArgs a,
-              const __grid_constant__ Codebook cbk,
-              const __grid_constant__ Codebook cbv,
-              const __grid_constant__ SignMask sm) {
-  using Gm = Geo<BK, BV>;
-  constexpr int NR = NT == 1 ? 1 : 2;       // score rows (positions) per lane and step
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* lutK = smem;                                   // offset 0
-  uint8_t* lutV = smem + Gm::LUTV_OFF;
-  __half* qhi = reinterpret_cast<__half*>(smem + Gm::QOFF);
-  __half* qlo = qhi + kMaxGroup * kHeadDim;
-  float* fin = reinterpret_cast<float*>(qhi);             // reuses q~ after a segment
-  int* misc = reinterpret_cast<int*>(smem + Gm::QOFF + Gm::QS);
-  float* miscf = reinterpret_cast<float*>(misc);
-  float* merge = reinterpret_cast<float*>(smem + Gm::FIXED);
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // this warp's ring barriers: one per slot, phases counted over all blocks
-  // the warp stages in this launch (jdone)
-  const uint32_t wbar = smem_addr(smem) + Gm::QOFF + Gm::QS + Gm::MISC + warp * kMaxStages * 8;
-  if (lane == 0) {
-#pragma unroll
-    for (int s = 0; s < Gm::NSTAGE; ++s) mbar_init(wbar + 8 * s);
-    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-  }
-  __syncwarp();
-  int jdone = 0;
-  bool stalled = false;                       // a staged-data wait gave up
-  const int gq = lane >> 2, tq = lane & 3;
-  const int H = a.n_kv_heads, GQ = a.gqa, B = a.batch;
-  const int Gc = gridDim.x, cta = blockIdx.x;   // Gc <= kMaxCtas (host check)
-  const uint32_t lbK = (lane & 15) * 8;                   // K table lane offset
-  const uint32_t lbV = Gm::LUTV_OFF | (lane * 4);         // V table lane base
-
-  // Launches that follow in the stream may start their own set-up now; they
-  // wait for this grid before touching memory (programmatic dependent
-  // launch; a no-op without it).
-  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-
-  // ---- codebooks staged in misc (launch parameters only): fp16 high/low
-  // parts of the scaled K levels and the fp16 V levels
-  uint32_t* cbs = reinterpret_cast<uint32_t*>(misc) + kMiscCb;
-  if (tid < 16) {
-    const float c = cbk.centroid[tid] * kKScale;
-    const __half h = __float2half_rn(c), l = __float2half_rn(c - __half2float(h));
-    cbs[tid] = (uint32_t)__half_as_ushort(h) | ((uint32_t)__half_as_ushort(l) << 16);
-    cbs[16 + tid] = __half_as_ushort(__float2half_rn(cbv.centroid[tid]));
-  }
-  __syncthreads();
-  // ---- K table: uint2 (high pair, low pair) per (pair code, copy)
-  for (int e = tid; e < (1 << (2 * BK)) * 16; e += kThreads) {
-    const int code = e >> 4, copy = e & 15;
-    const uint32_t c0 = cbs[code & ((1 << BK) - 1)], c1 = cbs[code >> BK];
-    uint2 v;
-    v.x = (c0 & 0xFFFFu) | (c1 << 16);                // high parts (even, odd coord)
-    v.y = (c0 >> 16) | (c1 & 0xFFFF0000u);            // low parts
-    *reinterpret_cast<uint2*>(lutK + code * 128 + copy * 8) = v;
-  }
-  if (BV != 2) {
-    for (int e = tid; e < (1 << (2 * BV)) * 32; e += kThreads) {
-      const int code = e >> 5, copy = e & 31;
-      *reinterpret_cast<uint32_t*>(lutV + code * 128 + copy * 4) =
-          cbs[16 + (code & ((1 << BV) - 1))] | (cbs[16 + (code >> BV)] << 16);
-    }
-  }
-  // V2 byte tables: low bytes of the 4 fp16 levels, then their high bytes.
-  uint32_t vt_lo = 0, vt_hi = 0;
-  if (BV == 2) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t h = cbs[16 + j];
-      vt_lo |= (h & 0xFFu) << (8 * j);
-      vt_hi |= (h >> 8) << (8 * j);
-    }
-  }
-
-  // Everything below reads inputs that an earlier launch may have written.
-  asm volatile("griddepcontrol.wait;\n" ::: "memory");
-
-  // Lengths of the first 32 sequences, loaded by warp 0 first; the block
-  // count and the first segment search use them.
-  const int len0 = (warp == 0 && lane < B) ? min(max(a.ctx_lens[lane], 0), a.cap_tok) : 0;
-  // The queries (small next to the cache) are pulled into L2 now, spread
-  // over the CTAs, so that their later loads do not queue behind the cache
-  // stream in DRAM.
-  {
-    const size_t qbytes = (size_t)B * a.n_q_heads * kHeadDim * (a.q_dtype == TQ_F32 ? 4 : 2);
-    const char* qc = reinterpret_cast<const char*>(a.q);
-    for (size_t off = ((size_t)cta * kThreads + tid) * 128; off < qbytes;
-         off += (size_t)Gc * kThreads * 128)
-      asm volatile("prefetch.global.L2 [%0];\n" ::"l"(qc + off));
-  }
-
-  // Segment search (warp 0): the first sequence whose flat block range holds
-  // flat block `at`, continuing from the scan state in misc. Writes the
-  // segment (b, g, first block, block count, blocks of the sequence, length).
-  auto find_segment = [&](long long at, long long end) {
-    int sb = misc[kMiscState];
-    long long sP = (long long)(unsigned)misc[kMiscState + 1] | ((long long)misc[kMiscState + 2] << 32);
-    while (true) {
-      if (sb >= B) {                      // inconsistent lengths: stop this CTA
-        if (lane == 0) misc[kMiscSeg + 3] = 0;
-        break;
-      }
-      const int bb = sb + lane;
-      const int len = sb == 0 ? len0 : (bb < B ? min(max(a.ctx_lens[bb], 0), a.cap_tok) : 0);
-      const int nb = (len + kBlk - 1) / kBlk;
-      int incl = nb;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      const long long segend = (long long)H * (sP + incl);
-      const unsigned hit = __ballot_sync(0xFFFFFFFFu, segend > at && bb < B);
-      if (hit) {
-        const int l = __ffs(hit) - 1;
-        const int nbl = __shfl_sync(0xFFFFFFFFu, nb, l);
-        const int lenl = __shfl_sync(0xFFFFFFFFu, len, l);
-        const int excl = __shfl_sync(0xFFFFFFFFu, incl - nb, l);
-        sb += l;
-        sP += excl;
-        if (lane == 0) {
-          const long long rel = at - (long long)H * sP;
-          const int g = (int)(rel / nbl), blk0 = (int)(rel % nbl);
-          misc[kMiscSeg + 0] = sb;
-          misc[kMiscSeg + 1] = g;
-          misc[kMiscSeg + 2] = blk0;
-          misc[kMiscSeg + 3] = (int)min((long long)(nbl - blk0), end - at);
-          misc[kMiscSeg + 4] = nbl;
-          misc[kMiscSeg + 5] = lenl;
-          misc[kMiscState] = sb;
-          misc[kMiscState + 1] = (int)(sP & 0xFFFFFFFF);
-          misc[kMiscState + 2] = (int)(sP >> 32);
-        }
-        break;
-      }
-      sP += __shfl_sync(0xFFFFFFFFu, incl, 31);
-      sb += 32;
-    }
-  };
-
-  // Balanced split over Geff CTAs, each owning at least one block (the
-  // partial count of a sequence relies on it): min(grid, NB), or, when every
-  // (sequence, kv head) segment has the same block count and there are no
-  // more segments than CTAs, a multiple of the segment count so that no CTA
-  // spans two segments.
-  auto effective_ctas = [&](long long nbt, int common) {
-    int ge = (int)min((long long)Gc, nbt);
-    const long long S = (long long)B * H;
-    if (common > 0 && S <= Gc) ge = (int)(S * min((long long)(Gc / S), (long long)common));
-    return ge;
-  };
-
-  if (warp == 0) {
-    // ---- flat block count, whether all sequences have the same length, and
-    // the first segment of this CTA
-    long long tot = 0;
-    int nmin = 0x7FFFFFFF, nmax = 0;
-    for (int b0 = 0; b0 < B; b0 += 32) {
-      const bool in = b0 + lane < B;
-      const int nb = b0 == 0 ? (len0 + kBlk - 1) / kBlk : (in ? seq_blocks(a, b0 + lane) : 0);
-      int sum = nb, lo = in ? nb : 0x7FFFFFFF, hi = nb;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-        lo = min(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, o));
-        hi = max(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, o));
-      }
-      tot += sum;
-      nmin = min(nmin, lo);
-      nmax = max(nmax, hi);
-    }
-    const long long nbt = tot * H;
-    const int common = nmin == nmax ? nmax : -1;
-    if (lane == 0) {
-      misc[kMiscNB] = (int)(nbt & 0xFFFFFFFF);
-      misc[kMiscNB + 1] = (int)(nbt >> 32);
-      misc[kMiscNB + 2] = common;
-      misc[kMiscState] = 0;
-      misc[kMiscState + 1] = 0;
-      misc[kMiscState + 2] = 0;
-      misc[kMiscSeg + 3] = 0;
-    }
-    __syncwarp();
-    const int ge = effective_ctas(nbt, common);
-    if (cta < ge) find_segment(nbt * cta / ge, nbt * (cta + 1) / ge);
-  }
-  __syncthreads();
-
-  const long long NB = (long long)(unsigned)misc[kMiscNB] | ((long long)misc[kMiscNB + 1] << 32);
-  const int Geff = effective_ctas(NB, misc[kMiscNB + 2]);
-  const long long r0 = cta < Geff ? NB * cta / Geff : 0;
-  const long long r1 = cta < Geff ? NB * (cta + 1) / Geff : 0;
-  long long pos = r0;
-  unsigned nskip = 0;
-  const float log2tau = a.tau > 0.f ? log2f(a.tau) : -INFINITY;
-
-  // ---- status words and empty sequences (CTA 0, one sequence per thread)
-  if (cta == 0) {
-    for (int b = tid; b < B; b += kThreads) {
-      const int raw = a.ctx_lens[b];
-      if (a.dev_status && (raw > a.cap_tok || raw <= 0))
-        atomicOr(a.dev_status, raw <= 0 ? TQ_DEV_CTX_EMPTY : TQ_DEV_CTX_CLAMPED);
-      if (raw <= 0) {
-        const int es = a.out_dtype == TQ_F32 ? 4 : 2;
-        const size_t n16 = (size_t)a.n_q_heads * kHeadDim * es / 16;
-        uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(a.out) +
-                                            (size_t)b * a.n_q_heads * kHeadDim * es);
-        for (size_t i = 0; i < n16; ++i) o[i] = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
-  }
-
-  // Lane roles in the score / softmax layout:
-  //   NT = 1: the lane holds position gq (tq < 2) or gq + 8 (tq >= 2) of each
-  //           16-position step, for heads hs0 = 2·(tq & 1) and hs0 + 1;
-  //   NT = 2: positions gq and gq + 8, heads hs0 = 2·tq and hs0 + 1.
-  const int hs0 = NT == 1 ? 2 * (tq & 1) : 2 * tq;
-  const bool hv0 = hs0 < GQ, hv1 = hs0 + 1 < GQ;
-  auto pos_of = [&](int mt, int rr) {
-    return 16 * mt + gq + (NT == 1 ? 8 * (tq >> 1) : 8 * rr);
-  };
-
-  // Combines the kWarps merge buffers into fin[] (GQ x d) and the merged
-  // per-head maximum and softmax sum (misc). A buffer holds accumulators in
-  // register order (natural = false: lane-major, 32 per lane) or in output
-  // order (natural = true), then the per-head maxima and sums.
-  float* wts = miscf + kMiscWt;                       // [kWarps][GQ] weights
-  auto merge_buffers = [&](bool natural) {
-    if (tid < kWarps * GQ) {
-      const int w = tid / GQ, h = tid - w * GQ;
-      float mx = -INFINITY;
-#pragma unroll
-      for (int v = 0; v < kWarps; ++v) mx = fmaxf(mx, merge[v * kMergeStride + kMergeM + h]);
-      const float mw = merge[w * kMergeStride + kMergeM + h];
-      wts[tid] = mw == -INFINITY ? 0.f : fast_exp2(mw - mx);
-      if (w == 0) {
-        float ls = 0.f;
-#pragma unroll
-        for (int v = 0; v < kWarps; ++v) {
-          const float m = merge[v * kMergeStride + kMergeM + h];
-          if (m != -INFINITY) ls += merge[v * kMergeStride + kMergeL + h] * fast_exp2(m - mx);
-        }
-        miscf[kMiscM + h] = mx;
-        miscf[kMiscL + h] = ls;
-      }
-    }
-    __syncthreads();
-    for (int i = tid; i < GQ * kHeadDim; i += kThreads) {
-      const int h = i / kHeadDim;
-      const int idx = natural ? i : pv_slot<BV>(i - h * kHeadDim, h);
-      float sum = 0.f;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) sum += merge[w * kMergeStride + idx] * wts[w * GQ + h];
-      fin[i] = sum;
-    }
-    __syncthreads();
-  };
-
-  bool first = true;
-  while (pos < r1) {
-    if (!first) {
-      if (warp == 0) find_segment(pos, r1);
-      __syncthreads();
-    }
-    first = false;
-    const int b = misc[kMiscSeg + 0], g = misc[kMiscSeg + 1], blk0 = misc[kMiscSeg + 2];
-    const int nseg = misc[kMiscSeg + 3], nbl = misc[kMiscSeg + 4], L = misc[kMiscSeg + 5];
-    if (nseg <= 0) break;
-    const long long sP_seg = (long long)(unsigned)misc[kMiscState + 1] | ((long long)misc[kMiscState + 2] << 32);
-    const long long seg_first = (long long)H * sP_seg + (long long)g * nbl;
-
-    // query values of the group (warp h < g loads head h), issued before the
-    // block loads
-    float qraw[4] = {0.f, 0.f, 0.f, 0.f};
-    if (warp < GQ) {
-      const size_t qo = ((size_t)b * a.n_q_heads + (size_t)g * GQ + warp) * kHeadDim + 4 * lane;
-      if (a.q_dtype == TQ_F32) {
-        const float4 v = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.q) + qo);
-        qraw[0] = v.x; qraw[1] = v.y; qraw[2] = v.z; qraw[3] = v.w;
-      } else {
-        const uint2 v = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(a.q) + qo);
-        const bool bf = a.q_dtype == TQ_BF16;
-        const float2 f0 = unpack16x2(v.x, bf), f1 = unpack16x2(v.y, bf);
-        qraw[0] = f0.x; qraw[1] = f0.y; qraw[2] = f1.x; qraw[3] = f1.y;
-      }
-    }
-
-    // ---- this warp's blocks of the segment
-    // The warps split the segment in whole 64-position blocks (the sparse-V
-    // gate's block maximum needs the full block; measured, a 16-position
-    // split was no faster without the gate either: the SM is throughput
-    // bound in this phase). A warp walks its range in chunks of up to 64
-    // positions starting at wp0.
-    const int sp0 = blk0 * kBlk, sp1 = min(L, (blk0 + nseg) * kBlk);
-    const int unit = kBlk;
-    const int nun = (sp1 - sp0 + unit - 1) / unit;
-    const int wp0 = sp0 + unit * (int)((long long)nun * warp / kWarps);
-    const int wp1 = min(sp1, sp0 + unit * (int)((long long)nun * (warp + 1) / kWarps));
-    const int nw = wp1 > wp0 ? (wp1 - wp0 + kBlk - 1) / kBlk : 0;
-
-    float acc[8][4];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
-    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
-
-    const size_t seq_row = ((size_t)b * H + g) * a.cap_tok;
-    const uint8_t* gk = a.packed_k + seq_row * Gm::RK;
-    const uint8_t* gv = a.packed_v + seq_row * Gm::RV;
-    const uint16_t* gnk = a.norms_k + seq_row;
-    const uint16_t* gnv = a.norms_v + seq_row;
-    const uint32_t wring = Gm::FIXED + warp * Gm::NSTAGE * Gm::STAGE;   // smem offset
-    const uint32_t wring_s = smem_addr(smem) + wring;                    // shared address
-
-    // Bulk copies of chunk c of the warp's range (its j-th staged chunk)
-    // into ring slot j % NSTAGE, issued by lane 0: K rows, V rows and the
-    // two norm runs are contiguous in global memory. Rows past the range are
-    // not copied; their slot bytes are stale and masked out below (norms are
-    // copied in whole 16-byte runs, which stay inside cap_tok).
-    auto issue = [&](int c, int j) {
-      if (lane == 0) {
-        const int t0 = wp0 + c * kBlk;
-        const int rows = min(kBlk, wp1 - t0);
-        const int nrows = min(kBlk, (rows + 7) & ~7);
-        const int slot = j % Gm::NSTAGE;
-        const uint32_t dst = wring_s + slot * Gm::STAGE, bar = wbar + 8 * slot;
-        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-        mbar_expect(bar, rows * (Gm::RK + Gm::RV) + 4 * nrows);
-        bulk_g2s(dst, gk + (size_t)t0 * Gm::RK, rows * Gm::RK, bar);
-        bulk_g2s(dst + Gm::KB, gv + (size_t)t0 * Gm::RV, rows * Gm::RV, bar);
-        bulk_g2s(dst + Gm::NKOFF, gnk + t0, 2 * nrows, bar);
-        bulk_g2s(dst + Gm::NKOFF + 2 * kBlk, gnv + t0, 2 * nrows, bar);
-      }
-    };
-
-    // every slot of the ring gets a block (or an empty group); the warps
-    // that rotate the query fill theirs afterwards, so that the query loads
-    // do not wait behind their block loads
-    auto fill_ring = [&]() {
-#pragma unroll
-      for (int p = 0; p < Gm::NSTAGE; ++p)
-        if (!stalled && p < nw) issue(p, jdone + p);
-    };
-    int issued = stalled ? 0 : min(nw, Gm::NSTAGE);
-    auto bar_of = [&](int jj) { return wbar + 8 * (jj % Gm::NSTAGE); };
-    auto par_of = [&](int jj) { return (uint32_t)(jj / Gm::NSTAGE) & 1u; };
-    if (warp >= GQ) fill_ring();
-    // ---- rotated query of the group: warp h handles query head h
-    if (warp < GQ) {
-      float x[4];
-      const uint32_t m = sm.w[lane >> 3];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) x[k] = apply_sign(qraw[k], m, (4 * lane + k) & 31);
-      fwht128_warp(x, lane);
-      // log2(e)/d^{3/2} folds the rotation normalization, the codebook's
-      // 1/sqrt(d) and the softmax 1/sqrt(d); a power-of-two scale keeps the
-      // fp16 high part near 2^14 so that the low part stays normal.
-      float amax = 0.f;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        x[k] *= kLog2e / (128.0f * 11.3137084989847603904f);
-        amax = fmaxf(amax, fabsf(x[k]));
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-      const int e = amax > 0.f ? ilogbf(amax) : 0;
-      const float qs = ldexpf(1.f, min(14 - e, 120));
-      uint32_t hi2[2], lo2[2];
-#pragma unroll
-      for (int k = 0; k < 4; k += 2) {
-        const float v0 = x[k] * qs, v1 = x[k + 1] * qs;
-        const __half h0 = __float2half_rn(v0), h1 = __float2half_rn(v1);
-        hi2[k / 2] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
-        lo2[k / 2] = pack_half2(v0 - __half2float(h0), v1 - __half2float(h1));
-      }
-      *reinterpret_cast<uint2*>(qhi + warp * kHeadDim + 4 * lane) = make_uint2(hi2[0], hi2[1]);
-      *reinterpret_cast<uint2*>(qlo + warp * kHeadDim + 4 * lane) = make_uint2(lo2[0], lo2[1]);
-      if (lane == 0) miscf[kMiscQInv + warp] = 1.f / (qs * kKScale);
-      fill_ring();
-    }
-    // ---- decode-step append: the warp whose range ends at the sequence's
-    // last position encodes the new token of (b, g) (lanes 0-3: K, 4-7: V;
-    // the encode kernel's per-vector code), stores it in cache row L - 1 and
-    // keeps a copy to patch into its staged last chunk.
-    const bool app = a.new_kv != nullptr && blk0 + nseg == nbl && nw > 0 && wp1 == L;
-    uint8_t* app_k = smem + Gm::APPOFF;
-    uint8_t* app_v = app_k + 64;
-    uint16_t* app_n = reinterpret_cast<uint16_t*>(app_k + 128);
-    if (app) {
-      if (lane < 8) {
-        const int sub = lane & 3;
-        const bool isv = lane >= 4;
-        uint32_t smask[16];
-        sign_masks(sm, sub, smask);
-        const uint16_t* src = a.new_kv + ((size_t)((isv ? B : 0) + b) * H + g) * kHeadDim;
-        float x[32];
-        load_signed(src, sub, a.new_kv_bf16 != 0, smask, x);
-        const unsigned gmask = 0xFu << (lane & ~3);
-        if (isv)
-          encode_vector<BV>(x, cbv, sub, gmask, app_v, app_n + 1, a.dev_status);
-        else
-          encode_vector<BK>(x, cbk, sub, gmask, app_k, app_n, a.dev_status);
-      }
-      __syncwarp();
-      const size_t row = seq_row + (size_t)(L - 1);
-      if (lane < Gm::RK / 4)
-        reinterpret_cast<uint32_t*>(a.packed_k + row * Gm::RK)[lane] =
-            reinterpret_cast<const uint32_t*>(app_k)[lane];
-      if (lane < Gm::RV / 4)
-        reinterpret_cast<uint32_t*>(a.packed_v + row * Gm::RV)[lane] =
-            reinterpret_cast<const uint32_t*>(app_v)[lane];
-      if (lane == 0) {
-        a.norms_k[row] = app_n[0];
-        a.norms_v[row] = app_n[1];
-      }
-    }
-    __syncthreads();
-
-    // ---- query fragments (B operand of the score MMA), column n = gq.
-    //   NT = 1: columns 0-3 hold the high part of heads 0-3, 4-7 their low part.
-    //   NT = 2: tile 0 column n = high part of head n, tile 1 = low part.
-    uint32_t qb[NT][8][2];
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      const int head = NT == 1 ? (gq & 3) : gq;
-      const __half* src = (NT == 1 ? (gq < 4) : (t == 0)) ? qhi : qlo;
-      const bool ok = head < GQ;
-#pragma unroll
-      for (int s = 0; s < 8; ++s) {
-        const int c0 = 32 * tq + 4 * s;
-        qb[t][s][0] = ok ? *reinterpret_cast<const uint32_t*>(src + head * kHeadDim + c0) : 0u;
-        qb[t][s][1] = ok ? *reinterpret_cast<const uint32_t*>(src + head * kHeadDim + c0 + 2) : 0u;
-      }
-    }
-    const float sinv0 = hv0 ? miscf[kMiscQInv + hs0] : 0.f;
-    const float sinv1 = hv1 ? miscf[kMiscQInv + hs0 + 1] : 0.f;
-
-    for (int i = 0; i < nw && !stalled; ++i) {
-      const int j = jdone + i;
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar_of(j), par_of(j)))) {
-        // give up: report, wait (bounded) for the copies still in flight,
-        // issue nothing more
-        stalled = true;
-        if (lane == 0 && a.dev_status) atomicOr(a.dev_status, TQ_DEV_WAIT_TIMEOUT);
-        for (int k = i + 1; k < issued; ++k) mbar_wait(bar_of(jdone + k), par_of(jdone + k));
-        __syncwarp();
-        break;
-      }
-      const uint32_t st = wring + (j % Gm::NSTAGE) * Gm::STAGE;         // smem offset
-      const int t0 = wp0 + i * kBlk;                // chunk [t0, cend)
-      const int cend = min(wp1, t0 + kBlk);
-      const bool partial = cend < t0 + kBlk;
-      if (app && cend == L) {                       // the staged row L - 1 is stale
-        const int r = L - 1 - t0;
-        if (lane < Gm::RK / 4)
-          *reinterpret_cast<uint32_t*>(smem + st + r * Gm::RK + 4 * lane) =
-              reinterpret_cast<const uint32_t*>(app_k)[lane];
-        if (lane < Gm::RV / 4)
-          *reinterpret_cast<uint32_t*>(smem + st + Gm::KB + r * Gm::RV + 4 * lane) =
-              reinterpret_cast<const uint32_t*>(app_v)[lane];
-        if (lane == 0) {
-          *reinterpret_cast<uint16_t*>(smem + st + Gm::NKOFF + 2 * r) = app_n[0];
-          *reinterpret_cast<uint16_t*>(smem + st + Gm::NKOFF + 2 * kBlk + 2 * r) = app_n[1];
-        }
-        __syncwarp();
-      }
-
-      // -- scores: 4 steps of 16 positions, each as two 8-position groups.
-      // A operand rows 0-7 are the K codebook high parts of the group's
-      // positions, rows 8-15 the low parts of the same positions, so one
-      // table entry (high pair, low pair) fills two adjacent fragment
-      // registers; D rows r and r + 8 add up to the score of position r.
-      float sc[4][NR][2];               // [step][row][head hs0 + e]
-#pragma unroll
-      for (int mt = 0; mt < 4; ++mt) {
-        if (16 * mt >= cend - t0) {          // step past the chunk: all masked
-#pragma unroll
-          for (int rr = 0; rr < NR; ++rr) sc[mt][rr][0] = sc[mt][rr][1] = -INFINITY;
-          continue;
-        }
-        uint32_t kw[2][BK + 1];              // positions gq and gq + 8, chunk tq
-#pragma unroll
-        for (int gr = 0; gr < 2; ++gr) {
-          const uint32_t rp = st + (16 * mt + 8 * gr + gq) * Gm::RK + 4 * BK * tq;
-          if constexpr (BK == 4) {
-            const uint4 u = lds<uint4>(smem, rp);
-            kw[gr][0] = u.x; kw[gr][1] = u.y; kw[gr][2] = u.z; kw[gr][3] = u.w;
-          } else if constexpr (BK == 2) {
-            const uint2 u = lds<uint2>(smem, rp);
-            kw[gr][0] = u.x; kw[gr][1] = u.y;
-          } else {
-#pragma unroll
-            for (int w = 0; w < BK; ++w) kw[gr][w] = lds<uint32_t>(smem, rp + 4 * w);
-          }
-          kw[gr][BK] = 0;
-        }
-        float d[2][NT][4];
-#pragma unroll
-        for (int gr = 0; gr < 2; ++gr)
-#pragma unroll
-          for (int t = 0; t < NT; ++t) d[gr][t][0] = d[gr][t][1] = d[gr][t][2] = d[gr][t][3] = 0.f;
-#pragma unroll
-        for (int s2 = 0; s2 < 8; ++s2) {
-#pragma unroll
-          for (int gr = 0; gr < 2; ++gr) {
-            const uint2 e0 = lds<uint2>(smem, k_entry<BK>(kw[gr], 2 * s2) + lbK);
-            const uint2 e1 = lds<uint2>(smem, k_entry<BK>(kw[gr], 2 * s2 + 1) + lbK);
-#pragma unroll
-            for (int t = 0; t < NT; ++t)
-              mma16816(d[gr][t], e0.x, e0.y, e1.x, e1.y, qb[t][s2][0], qb[t][s2][1]);
-          }
-        }
-        if (NT == 1) {
-          // Columns 2tq, 2tq+1: the high part of heads 2tq, 2tq+1 (tq < 2) or
-          // the low part of heads 2(tq-2), +1 (tq >= 2); lane ^ 2 holds the
-          // other part. Lanes tq < 2 keep group 0, tq >= 2 keep group 1.
-          const float a0 = d[0][0][0] + d[0][0][2], a1 = d[0][0][1] + d[0][0][3];
-          const float c0 = d[1][0][0] + d[1][0][2], c1 = d[1][0][1] + d[1][0][3];
-          const bool lowq = tq >= 2;
-          const float s0 = __shfl_xor_sync(0xFFFFFFFFu, lowq ? a0 : c0, 2);
-          const float s1 = __shfl_xor_sync(0xFFFFFFFFu, lowq ? a1 : c1, 2);
-          sc[mt][0][0] = (lowq ? c0 : a0) + s0;
-          sc[mt][0][1] = (lowq ? c1 : a1) + s1;
-        } else {
-#pragma unroll
-          for (int gr = 0; gr < 2; ++gr) {
-            sc[mt][gr][0] = (d[gr][0][0] + d[gr][0][2]) + d[gr][NT - 1][0];
-            sc[mt][gr][1] = (d[gr][0][1] + d[gr][0][3]) + d[gr][NT - 1][1];
-          }
-        }
-      }
-      // -- scale by the K norm and query scale, mask, block maximum per head
-      float mb0 = -INFINITY, mb1 = -INFINITY;
-#pragma unroll
-      for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-        for (int rr = 0; rr < NR; ++rr) {
-          const int p = pos_of(mt, rr);
-          const float nk = __half2float(__ushort_as_half(lds<uint16_t>(smem, st + Gm::NKOFF + 2 * p)));
-          float v0 = sc[mt][rr][0] * (sinv0 * nk);
-          float v1 = sc[mt][rr][1] * (sinv1 * nk);
-          if (partial && t0 + p >= cend) v0 = v1 = -INFINITY;
-          sc[mt][rr][0] = v0;
-          sc[mt][rr][1] = v1;
-          mb0 = fmaxf(mb0, v0);
-          mb1 = fmaxf(mb1, v1);
-        }
-      // lanes holding the same heads: NT = 1 -> lane bits 1-4; NT = 2 -> bits 2-4
-#pragma unroll
-      for (int o = (NT == 1 ? 2 : 4); o < 32; o <<= 1) {
-        mb0 = fmaxf(mb0, __shfl_xor_sync(0xFFFFFFFFu, mb0, o));
-        mb1 = fmaxf(mb1, __shfl_xor_sync(0xFFFFFFFFu, mb1, o));
-      }
-      const float mn0 = fmaxf(m_run[0], mb0), mn1 = fmaxf(m_run[1], mb1);
-      const float al0 = fast_exp2(m_run[0] - mn0), al1 = fast_exp2(m_run[1] - mn1);
-      m_run[0] = mn0;
-      m_run[1] = mn1;
-      l_run[0] *= al0;
-      l_run[1] *= al1;
-
-      // -- weights, gate, P' = w · nV packed as fp16 pairs (heads hs0, hs0+1)
-      uint32_t pk[4][NR];
-#pragma unroll
-      for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-        for (int rr = 0; rr < NR; ++rr) {
-          const int p = pos_of(mt, rr);
-          const float nv = __half2float(__ushort_as_half(lds<uint16_t>(smem, st + Gm::NKOFF + 2 * kBlk + 2 * p)));
-          const float s0 = sc[mt][rr][0], s1 = sc[mt][rr][1];
-          const float w0 = fast_exp2(s0 - mn0), w1 = fast_exp2(s1 - mn1);
-          l_run[0] += w0;
-          l_run[1] += w1;
-          float p0 = w0 * nv, p1 = w1 * nv;
-          const bool g0 = s0 - mb0 < log2tau, g1 = s1 - mb1 < log2tau;   // exp(s - M_blk) < tau
-          if (g0) p0 = 0.f;
-          if (g1) p1 = 0.f;
-          if (partial && t0 + p >= cend) p0 = p1 = 0.f;   // stale slot bytes
-          nskip += (g0 && hv0 && s0 != -INFINITY) + (g1 && hv1 && s1 != -INFINITY);
-          pk[mt][rr] = pack_half2(hv0 ? p0 : 0.f, hv1 ? p1 : 0.f);
-        }
-      // rescale the PV accumulators (PV layout: heads 2tq, 2tq+1)
-      {
-        float a0 = al0, a1 = al1;
-        if (NT == 1 && tq >= 2) a0 = a1 = 1.f;      // heads 4-7: padding
-        if (__any_sync(0xFFFFFFFFu, a0 != 1.f || a1 != 1.f)) {
-#pragma unroll
-          for (int r = 0; r < 8; ++r) {
-            acc[r][0] *= a0;
-            acc[r][1] *= a1;
-            acc[r][2] *= a0;
-            acc[r][3] *= a1;
-          }
-        }
-      }
-
-      // -- P·V over the four 16-position steps
-#pragma unroll
-      for (int mt = 0; mt < 4; ++mt) {
-        uint32_t x0, x1;   // P' of positions 0-7 / 8-15 x heads 0-7, standard layout
-        if (NT == 1) {
-          const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, pk[mt][0], 2);
-          x0 = tq < 2 ? pk[mt][0] : 0u;
-          x1 = tq < 2 ? other : 0u;
-        } else {
-          x0 = pk[mt][0];
-          x1 = pk[mt][NR - 1];
-        }
-        if (!__any_sync(0xFFFFFFFFu, (x0 | x1) != 0u)) continue;   // whole step gated
-        const uint32_t b0 = transpose8x8(x0), b1 = transpose8x8(x1);
-        if (BV == 2) {
-          const uint32_t vrow = st + Gm::KB + (16 * mt + 2 * tq) * Gm::RVS + 4 * gq;
-          const uint32_t wA = lds<uint32_t>(smem, vrow), wB = lds<uint32_t>(smem, vrow + Gm::RVS);
-          const uint32_t wC = lds<uint32_t>(smem, vrow + 8 * Gm::RVS);
-          const uint32_t wD = lds<uint32_t>(smem, vrow + 9 * Gm::RVS);
-          const uint32_t xab[2] = {__byte_perm(wA, wB, 0x5140), __byte_perm(wA, wB, 0x7362)};
-          const uint32_t xcd[2] = {__byte_perm(wC, wD, 0x5140), __byte_perm(wC, wD, 0x7362)};
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-#pragma unroll
-            for (int odd = 0; odd < 2; ++odd) {
-              const int f0 = 4 * odd, f1 = 4 * odd + 2;   // codes of coords 2r, 2r+1
-              const uint32_t s0 = ((xab[half] >> f0) & 0x03030303u) * 0x11u + 0x40404040u;
-              const uint32_t s1 = ((xab[half] >> f1) & 0x03030303u) * 0x11u + 0x40404040u;
-              const uint32_t s2 = ((xcd[half] >> f0) & 0x03030303u) * 0x11u + 0x40404040u;
-              const uint32_t s3 = ((xcd[half] >> f1) & 0x03030303u) * 0x11u + 0x40404040u;
-#pragma unroll
-              for (int hb = 0; hb < 2; ++hb) {
-                const int r = 2 * (2 * half + hb) + odd;
-                const int sh = 16 * hb;
-                mma16816(acc[r], __byte_perm(vt_lo, vt_hi, s0 >> sh),
-                         __byte_perm(vt_lo, vt_hi, s1 >> sh), __byte_perm(vt_lo, vt_hi, s2 >> sh),
-                         __byte_perm(vt_lo, vt_hi, s3 >> sh), b0, b1);
-              }
-            }
-          }
-        } else {
-          uint32_t v0[BV + 1], v1[BV + 1];
-          const uint32_t r0p = st + Gm::KB + (16 * mt + gq) * Gm::RVS + 4 * BV * tq;
-          const uint32_t r1p = r0p + 8 * Gm::RVS;
-#pragma unroll
-          for (int w = 0; w < BV; ++w) {
-            v0[w] = lds<uint32_t>(smem, r0p + 4 * w);
-            v1[w] = lds<uint32_t>(smem, r1p + 4 * w);
-          }
-          v0[BV] = v1[BV] = 0;
-#pragma unroll
-          for (int r = 0; r < 8; ++r) {
-            const uint32_t y0 = lds<uint32_t>(smem, pair_code_shifted<BV, 7>(v0, 2 * r) | lbV);
-            const uint32_t y1 = lds<uint32_t>(smem, pair_code_shifted<BV, 7>(v0, 2 * r + 1) | lbV);
-            const uint32_t y2 = lds<uint32_t>(smem, pair_code_shifted<BV, 7>(v1, 2 * r) | lbV);
-            const uint32_t y3 = lds<uint32_t>(smem, pair_code_shifted<BV, 7>(v1, 2 * r + 1) | lbV);
-            mma16816(acc[r], transpose8x8(y0), transpose8x8(y1), transpose8x8(y2),
-                     transpose8x8(y3), b0, b1);
-          }
-        }
-      }
-      __syncwarp();                                  // the slot is free again
-      if (i + Gm::NSTAGE < nw) {
-        issue(i + Gm::NSTAGE, j + Gm::NSTAGE);
-        ++issued;
-      }
-    }
-    jdone += nw;
-
-    // ---- per-warp softmax sums over the lanes holding the same heads
-#pragma unroll
-    for (int o = (NT == 1 ? 2 : 4); o < 32; o <<= 1) {
-      l_run[0] += __shfl_xor_sync(0xFFFFFFFFu, l_run[0], o);
-      l_run[1] += __shfl_xor_sync(0xFFFFFFFFu, l_run[1], o);
-    }
-
-    // ---- merge the warps of this segment. Each warp leaves its partial in
-    // a merge buffer (accumulators as stored in its registers, then the
-    // per-head maximum and sum); the buffers are combined per output element.
-    __syncthreads();                                  // all warps done with the ring
-    {
-      float* wm = merge + warp * kMergeStride;
-      if (gq == 0 && (NT == 2 || tq < 2)) {
-        if (hv0) {
-          wm[kMergeM + hs0] = nw > 0 ? m_run[0] : -INFINITY;
-          wm[kMergeL + hs0] = nw > 0 ? l_run[0] : 0.f;
-        }
-        if (hv1) {
-          wm[kMergeM + hs0 + 1] = nw > 0 ? m_run[1] : -INFINITY;
-          wm[kMergeL + hs0 + 1] = nw > 0 ? l_run[1] : 0.f;
-        }
-      }
-#pragma unroll
-      for (int r = 0; r < 8; ++r)
-        *reinterpret_cast<float4*>(wm + lane * kMergeLane + 4 * r) =
-            make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
-    }
-    __syncthreads();
-    merge_buffers(false);
-
-    bool finalize = nseg == nbl;                      // this CTA saw the whole sequence
-    if (!finalize) {
-      const int sigma = b * H + g;
-      const long long last = seg_first + nbl - 1;
-      const int c_first = cta_of(seg_first, NB, Geff), c_last = cta_of(last, NB, Geff);
-      const int n_parts = c_last - c_first + 1;
-      float* slot = a.slots + (size_t)(cta + sigma) * GQ * kSlotFloats;
-      for (int i = tid; i < GQ * kHeadDim; i += kThreads) slot[i] = fin[i];
-      if (tid < GQ) {
-        slot[GQ * kHeadDim + 2 * tid] = miscf[kMiscM + tid];
-        slot[GQ * kHeadDim + 2 * tid + 1] = miscf[kMiscL + tid];
-      }
-      __syncthreads();
-      if (tid == 0) {
-        __threadfence();
-        const int prev = atomicAdd(a.counters + sigma, 1);
-        const bool is_last = prev == n_parts - 1;
-        if (is_last) __threadfence();
-        misc[kMiscLast] = is_last;
-      }
-      __syncthreads();
-      finalize = misc[kMiscLast] != 0;
-      if (finalize) {
-        // Merge the n_parts partials of this sequence: warp w folds partials
-        // w, w + kWarps, ... (two per round of loads) into a merge buffer in
-        // output order, then the buffers are combined as above.
-        const float* s0 = a.slots + (size_t)(c_first + sigma) * GQ * kSlotFloats;
-        const size_t stride = (size_t)GQ * kSlotFloats;
-        const int nk = GQ * kHeadDim / 32;            // outputs per lane: lane + 32k
-        float S[kMaxGroup * kHeadDim / 32];
-        float Mh = -INFINITY, Lh = 0.f;               // lane h < GQ: head h
-#pragma unroll
-        for (int k = 0; k < kMaxGroup * kHeadDim / 32; ++k) S[k] = 0.f;
-        for (int p = warp; p < n_parts; p += 2 * kWarps) {
-          const bool two = p + kWarps < n_parts;
-          const float* pa = s0 + (size_t)p * stride;
-          const float* pb = s0 + (size_t)(two ? p + kWarps : p) * stride;
-          float va[kMaxGroup * kHeadDim / 32], vb[kMaxGroup * kHeadDim / 32];
-#pragma unroll
-          for (int k = 0; k < kMaxGroup * kHeadDim / 32; ++k) {
-            va[k] = k < nk ? __ldcg(pa + lane + 32 * k) : 0.f;
-            vb[k] = k < nk && two ? __ldcg(pb + lane + 32 * k) : 0.f;
-          }
-          const bool hl = lane < GQ;
-          const float ma = hl ? __ldcg(pa + GQ * kHeadDim + 2 * lane) : -INFINITY;
-          const float la = hl ? __ldcg(pa + GQ * kHeadDim + 2 * lane + 1) : 0.f;
-          const float mb = hl && two ? __ldcg(pb + GQ * kHeadDim + 2 * lane) : -INFINITY;
-          const float lb = hl && two ? __ldcg(pb + GQ * kHeadDim + 2 * lane + 1) : 0.f;
-          // per head (lane h): new maximum and the three rescale factors
-          const float Mn = fmaxf(Mh, fmaxf(ma, mb));
-          const float fo = Mh == -INFINITY ? 0.f : fast_exp2(Mh - Mn);
-          const float fa = ma == -INFINITY ? 0.f : fast_exp2(ma - Mn);
-          const float fb = mb == -INFINITY ? 0.f : fast_exp2(mb - Mn);
-          Lh = Lh * fo + la * fa + lb * fb;
-          Mh = Mn;
-#pragma unroll
-          for (int k = 0; k < kMaxGroup * kHeadDim / 32; ++k) {
-            const int h = k >> 2;                       // 32k / kHeadDim
-            const float go = __shfl_sync(0xFFFFFFFFu, fo, h);
-            const float ga = __shfl_sync(0xFFFFFFFFu, fa, h);
-            const float gb = __shfl_sync(0xFFFFFFFFu, fb, h);
-            S[k] = S[k] * go + va[k] * ga + vb[k] * gb;
-          }
-        }
-        __syncthreads();                              // merge buffers are free
-        float* wm = merge + warp * kMergeStride;
-#pragma unroll
-        for (int k = 0; k < kMaxGroup * kHeadDim / 32; ++k)
-          if (k < nk) wm[lane + 32 * k] = S[k];
-        if (lane < GQ) {
-          wm[kMergeM + lane] = Mh;
-          wm[kMergeL + lane] = Lh;
-        }
-        __syncthreads();
-        merge_buffers(true);
-        if (tid == 0) atomicExch(a.counters + sigma, 0);
-      }
-    }
-    if (finalize && warp < GQ) {
-      const float inv_l = 1.f / miscf[kMiscL + warp];
-      float x[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) x[k] = fin[warp * kHeadDim + 4 * lane + k] * inv_l;
-      fwht128_warp(x, lane);
-      const uint32_t m = sm.w[lane >> 3];
-      const size_t ob = ((size_t)b * a.n_q_heads + (size_t)g * GQ + warp) * kHeadDim + 4 * lane;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) x[k] = apply_sign(x[k], m, (4 * lane + k) & 31) * (1.f / kHeadDim);
-      if (a.out_dtype == TQ_F32) {
-        *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + ob) = make_float4(x[0], x[1], x[2], x[3]);
-      } else {
-        uint16_t h[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          h[k] = a.out_dtype == TQ_BF16 ? f32_to_bf16_bits(x[k]) : f32_to_f16_bits(x[k]);
-        *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.out) + ob) =
-            make_uint2(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16));
-      }
-    }
-    pos += nseg;
-    __syncthreads();                                  // misc / fin / q~ reuse
-  }
-
-  if (a.skipped) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) nskip += __shfl_xor_sync(0xFFFFFFFFu, nskip, o);
-    if (lane == 0 && nskip) atomicAdd(a.skipped, (unsigned long long)nskip);
-  }
-}
-
-int sm_count() {
-  static int cached[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!cached[dev]) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      n = 148;
-    cached[dev] = n;
-  }
-  return cached[dev];
-}
-
-template <int BK, int BV, int NT>
-cudaError_t launch_one(const AttendArgs& a, const Codebook& cbk, const Codebook& cbv,
-                       const SignMask& sm, int n_ctas, cudaStream_t stream) {
-  using Gm = Geo<BK, BV>;
-  static bool configured[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64 || !configured[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(attend_kernel<BK, BV, NT>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, Gm::SMEM);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) configured[dev] = true;
-  }
-  const int grid = n_ctas > 0 ? n_ctas : sm_count();
-  // Programmatic dependent launch: the kernel's set-up may overlap the tail
-  // of the previous launch in the stream; it waits for that launch before
-  // reading any input (griddepcontrol.wait).
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = Gm::SMEM;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attend_kernel<BK, BV, NT>, a, cbk, cbv, sm);
-}
-
-template <int BK, int BV>
-cudaError_t launch_pair(const AttendArgs& a, const Codebook& cbk, const Codebook& cbv,
-                        const SignMask& sm, int n_ctas, cudaStream_t stream) {
-  return a.gqa <= 4 ? launch_one<BK, BV, 1>(a, cbk, cbv, sm, n_ctas, stream)
-                    : launch_one<BK, BV, 2>(a, cbk, cbv, sm, n_ctas, stream);
-}
-
-}  // namespace
 
 cudaError_t launch_attend(const AttendArgs& a, const Codebook& cbk,
                           const Codebook& cbv, const SignMask& sm, int n_ctas,
                           cudaStream_t stream) {
   if (n_ctas > kMaxCtas) return cudaErrorInvalidValue;
-  switch (a.bits_k * 8 + a.bits_v) {
-    case 4 * 8 + 2: return launch_pair<4, 2>(a, cbk, cbv, sm, n_ctas, stream);
-    case 3 * 8 + 2: return launch_pair<3, 2>(a, cbk, cbv, sm, n_ctas, stream);
-    case 4 * 8 + 3: return launch_pair<4, 3>(a, cbk, cbv, sm, n_ctas, stream);
-    case 2 * 8 + 2: return launch_pair<2, 2>(a, cbk, cbv, sm, n_ctas, stream);
-    case 3 * 8 + 3: return launch_pair<3, 3>(a, cbk, cbv, sm, n_ctas, stream);
-    case 4 * 8 + 4: return launch_pair<4, 4>(a, cbk, cbv, sm, n_ctas, stream);
-    case 2 * 8 + 3: return launch_pair<2, 3>(a, cbk, cbv, sm, n_ctas, stream);
-    case 2 * 8 + 4: return launch_pair<2, 4>(a, cbk, cbv, sm, n_ctas, stream);
-    case 3 * 8 + 4: return launch_pair<3, 4>(a, cbk, cbv, sm, n_ctas, stream);
+  switch (a.d) {
+    case 64: return launch_attend_d<64>(a, cbk, cbv, sm, n_ctas, stream);
+    case 128: return launch_attend_d<128>(a, cbk, cbv, sm, n_ctas, stream);
+    case 256: return launch_attend_d<256>(a, cbk, cbv, sm, n_ctas, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -9,7 +9,8 @@
 //
 // The array lives for as long as the library is loaded, on every device that
 // loads it, and is shared by every call on that device. Its size caps the
-// problem: batch · n_q_heads <= 7879 (see kNoAllocScratchBytes).
+// problem: batch · n_q_heads <= 54530 / 23887 / 8033 at d = 64 / 128 / 256
+// (see kNoAllocScratchBytes).
 #include <mutex>
 
 #include "tq.h"
@@ -18,9 +19,9 @@
 namespace tq {
 namespace {
 
-// 8 MiB: partial-result slots for up to 1024 CTAs plus the counters and the
-// per-(batch, query head) slots, which fits batch · n_q_heads <= 7879.
-constexpr size_t kNoAllocScratchBytes = 8u << 20;
+// 16 MiB: partial-result slots (d + 2 floats per query head) for up to 1024
+// CTAs plus the counters and the per-(batch, query head) slots.
+constexpr size_t kNoAllocScratchBytes = 16u << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;

@@ -113,7 +113,7 @@ const Codebook* codebook_for(int bits) {
 SignMask sign_mask(uint64_t seed) {
   SignMask m{};
   uint64_t state = seed;
-  for (int i = 0; i < kHeadDim; ++i) {
+  for (int i = 0; i < kMaxHeadDim; ++i) {   // d-bit masks are prefixes
     state += 0x9E3779B97F4A7C15ull;
     uint64_t z = state;
     z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;

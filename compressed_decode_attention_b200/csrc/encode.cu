@@ -1,10 +1,11 @@
 // tq_encode kernel: FP16 norm, randomized Hadamard rotation, Lloyd-Max
 // index, LSB-first bit-packing — one pass over each K/V head vector.
 //
-// Thread layout: four lanes per vector, 32 consecutive coordinates per lane
-// (d = 128). A 256-thread block encodes 64 consecutive tokens of one kv head
-// (K or V) per step, so its packed rows and norms form one contiguous range;
-// blocks stride over the (tile, head, K/V) units. The per-vector arithmetic
+// Thread layout: d/32 lanes per vector (2, 4 or 8 for d = 64, 128, 256), 32
+// consecutive coordinates per lane. A 256-thread block encodes 256/(d/32)
+// consecutive tokens of one kv head (K or V) per step, so its packed rows and
+// norms form one contiguous range; blocks stride over the (tile, head, K/V)
+// units. The per-vector arithmetic
 // (encode_common.cuh) uses two-wide fp32 operations, since the kernel is
 // bound by instruction issue:
 //   load    4 x 16-byte loads per lane (the vector's 256 bytes, coalesced),
@@ -20,10 +21,10 @@ namespace tq {
 namespace {
 
 constexpr int kEncThreads = 256;
-constexpr int kEncTokens = kEncThreads / 4;
 
 // Grid-stride over (token tile, kv head, K/V): each group of four lanes
 // encodes one vector per iteration; its half2 sign masks are built once.
+template <int D>
 __global__ void __launch_bounds__(kEncThreads)
 encode_kernel(const __grid_constant__ EncodeArgs a,
               const __grid_constant__ Codebook cbk,
@@ -33,21 +34,23 @@ encode_kernel(const __grid_constant__ EncodeArgs a,
   // start; the input may come from the previous one, so wait before reading.
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  constexpr int LPV = D / 32;                 // lanes per vector
+  constexpr int kTokens = kEncThreads / LPV;  // tokens per tile
   const int lane = threadIdx.x & 31;
-  const int sub = lane & 3;
-  const unsigned gmask = 0xFu << (lane & ~3);
+  const int sub = lane & (LPV - 1);
+  const unsigned gmask = ((1u << LPV) - 1u) << (lane & ~(LPV - 1));
   uint32_t smask[16];
   sign_masks(sm, sub, smask);
-  const int tiles = (a.n_tok + kEncTokens - 1) / kEncTokens;
+  const int tiles = (a.n_tok + kTokens - 1) / kTokens;
   const long long units = (long long)tiles * a.n_kv_heads * 2;
   for (long long u = blockIdx.x; u < units; u += gridDim.x) {
     const int tile = (int)(u % tiles);
     const int h = (int)((u / tiles) % a.n_kv_heads);
     const int is_v = (int)(u / ((long long)tiles * a.n_kv_heads));
-    const int tok = tile * kEncTokens + (threadIdx.x >> 2);
-    if (tok >= a.n_tok) continue;                     // whole groups of four
+    const int tok = tile * kTokens + threadIdx.x / LPV;
+    if (tok >= a.n_tok) continue;                     // whole lane groups
 
-    const uint16_t* src = a.kv + ((size_t)(is_v * a.n_tok + tok) * a.n_kv_heads + h) * kHeadDim;
+    const uint16_t* src = a.kv + ((size_t)(is_v * a.n_tok + tok) * a.n_kv_heads + h) * D;
     float x[32];
     load_signed(src, sub, a.is_bf16, smask, x);
 
@@ -56,21 +59,19 @@ encode_kernel(const __grid_constant__ EncodeArgs a,
     const Codebook& cb = is_v ? cbv : cbk;
     uint8_t* packed = is_v ? a.packed_v : a.packed_k;
     uint16_t* norms = (is_v ? a.norms_v : a.norms_k) + row;
-    const size_t rb = (size_t)kHeadDim * bits / 8;
+    const size_t rb = (size_t)D * bits / 8;
     if (bits == 4)
-      encode_vector<4>(x, cb, sub, gmask, packed + row * rb, norms, a.dev_status);
+      encode_vector<4, LPV>(x, cb, sub, gmask, packed + row * rb, norms, a.dev_status);
     else if (bits == 3)
-      encode_vector<3>(x, cb, sub, gmask, packed + row * rb, norms, a.dev_status);
+      encode_vector<3, LPV>(x, cb, sub, gmask, packed + row * rb, norms, a.dev_status);
     else
-      encode_vector<2>(x, cb, sub, gmask, packed + row * rb, norms, a.dev_status);
+      encode_vector<2, LPV>(x, cb, sub, gmask, packed + row * rb, norms, a.dev_status);
   }
 }
 
-}  // namespace
-
-cudaError_t launch_encode(const EncodeArgs& a, const Codebook& cbk,
-                          const Codebook& cbv, const SignMask& sm,
-                          cudaStream_t stream) {
+template <int D>
+cudaError_t launch_encode_d(const EncodeArgs& a, const Codebook& cbk, const Codebook& cbv,
+                            const SignMask& sm, cudaStream_t stream) {
   // Enough resident blocks to cover every SM several times; each block then
   // strides over the (tile, head, K/V) units.
   static int sms = 0;
@@ -80,7 +81,8 @@ cudaError_t launch_encode(const EncodeArgs& a, const Codebook& cbk,
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       sms = 148;
   }
-  const long long units = (long long)((a.n_tok + kEncTokens - 1) / kEncTokens) * a.n_kv_heads * 2;
+  constexpr int kTokens = kEncThreads / (D / 32);
+  const long long units = (long long)((a.n_tok + kTokens - 1) / kTokens) * a.n_kv_heads * 2;
   const int grid = (int)(units < (long long)sms * 8 ? units : (long long)sms * 8);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -91,7 +93,20 @@ cudaError_t launch_encode(const EncodeArgs& a, const Codebook& cbk,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, encode_kernel, a, cbk, cbv, sm);
+  return cudaLaunchKernelEx(&cfg, encode_kernel<D>, a, cbk, cbv, sm);
+}
+
+}  // namespace
+
+cudaError_t launch_encode(const EncodeArgs& a, const Codebook& cbk,
+                          const Codebook& cbv, const SignMask& sm,
+                          cudaStream_t stream) {
+  switch (a.d) {
+    case 64: return launch_encode_d<64>(a, cbk, cbv, sm, stream);
+    case 128: return launch_encode_d<128>(a, cbk, cbv, sm, stream);
+    case 256: return launch_encode_d<256>(a, cbk, cbv, sm, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace tq

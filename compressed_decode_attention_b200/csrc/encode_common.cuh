@@ -1,7 +1,7 @@
 // Per-vector encode shared by the encode kernel and the fused decode-step
 // append: FP16 norm, randomized Hadamard rotation, Lloyd-Max index and
-// LSB-first packing of one d = 128 vector held by a group of four lanes
-// (32 consecutive coordinates per lane).
+// LSB-first packing of one d-dimensional vector (d = 32·LPV: 64, 128 or 256)
+// held by a group of LPV lanes, 32 consecutive coordinates per lane.
 //
 // [TQAI §The Paper]: keep the norm in FP16, rotate the unit vector,
 // quantize each coordinate with the precomputed Lloyd-Max codebook.
@@ -43,12 +43,12 @@ __device__ __forceinline__ void load_signed(const uint16_t* src, int sub, bool b
   }
 }
 
-template <int BITS>
+template <int BITS, int LPV>
 __device__ __forceinline__ void encode_vector(
     float (&x)[32], const Codebook& cb, int sub, unsigned gmask,
     uint8_t* row_dst, uint16_t* norm_dst, int* dev_status) {
   constexpr int kHalf = 1 << (BITS - 1);
-  // ||x||^2 over the group of four lanes (pairs of coordinates per fma)
+  // ||x||^2 over the group of LPV lanes (pairs of coordinates per fma)
   float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
@@ -56,14 +56,14 @@ __device__ __forceinline__ void encode_vector(
     ss2 = f2fma(v, v, ss2);
   }
   float ss = ss2.x + ss2.y;
-  ss += __shfl_xor_sync(gmask, ss, 1);
-  ss += __shfl_xor_sync(gmask, ss, 2);
+#pragma unroll
+  for (int o = 1; o < LPV; o <<= 1) ss += __shfl_xor_sync(gmask, ss, o);
   const float n = sqrtf(ss);
 
   // z = H·(D⊙x): coordinate 32·sub + i lives in register i of lane sub.
-  // Stride 1 in scalar form, strides 2..16 on register pairs, strides 32 and
-  // 64 across the four lanes (x' = partner + sign·x, sign = -1 on the upper
-  // lane); every step rounds exactly like a scalar add or subtract.
+  // Stride 1 in scalar form, strides 2..16 on register pairs, strides
+  // 32 .. 16·LPV across the lanes (x' = partner + sign·x, sign = -1 on the
+  // upper lane); every step rounds exactly like a scalar add or subtract.
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const float u = x[2 * j], v = x[2 * j + 1];
@@ -83,7 +83,7 @@ __device__ __forceinline__ void encode_vector(
     }
   }
 #pragma unroll
-  for (int o = 1; o <= 2; o <<= 1) {
+  for (int o = 1; o < LPV; o <<= 1) {
     const float sg = (sub & o) ? -1.f : 1.f;
     const float2 sg2 = make_float2(sg, sg);
 #pragma unroll

@@ -9,7 +9,7 @@
 
 namespace tq {
 
-constexpr int kHeadDim = 128;          // d supported by this build
+constexpr int kMaxHeadDim = 256;       // d in {64, 128, 256}
 constexpr int kMaxLevels = 16;         // 2^4: widest code on the hot path
 constexpr int kGateBlock = 64;         // sparse-V block (TQ_SPARSE_V_BLOCK)
 constexpr int kMaxGroup = 8;           // largest GQA group handled per CTA
@@ -23,7 +23,7 @@ struct Codebook {
 
 // Sign vector D as a bit mask: bit i of word i/32 set <=> D_i = -1.
 struct SignMask {
-  uint32_t w[kHeadDim / 32];
+  uint32_t w[kMaxHeadDim / 32];        // the first d bits are used
 };
 
 // ---------------------------------------------------------------- host side
@@ -37,6 +37,7 @@ SignMask sign_mask(uint64_t seed);
 // ---------------------------------------------------------------- launchers
 struct EncodeArgs {
   const uint16_t* kv;        // [2][n_tok][n_kv_heads][d]
+  int d;
   int is_bf16;
   int n_tok, n_kv_heads;
   int bits_k, bits_v;
@@ -52,6 +53,7 @@ cudaError_t launch_encode(const EncodeArgs& a, const Codebook& cbk,
                           cudaStream_t stream);
 
 struct DequantArgs {
+  int d;
   const uint8_t* packed;
   const uint16_t* norms;
   int n_tok, n_kv_heads, bits, cap_tok, domain;
@@ -73,6 +75,7 @@ struct AttendArgs {
   const uint16_t* new_kv;
   int new_kv_bf16;
   const int32_t* ctx_lens;
+  int d;
   int batch, n_q_heads, gqa, n_kv_heads;
   int bits_k, bits_v;
   int cap_tok;
@@ -87,18 +90,22 @@ struct AttendArgs {
 cudaError_t launch_attend(const AttendArgs& a, const Codebook& cbk,
                           const Codebook& cbv, const SignMask& sm, int n_ctas,
                           cudaStream_t stream);
+// Per head dimension (attend_d64.cu, attend_d128.cu, attend_d256.cu).
+template <int D>
+cudaError_t launch_attend_d(const AttendArgs& a, const Codebook& cbk, const Codebook& cbv,
+                            const SignMask& sm, int n_ctas, cudaStream_t stream);
 
 // Workspace of tq_attend: a counter region (zero on first use; every call
 // leaves it zero) followed by partial-result slots. Sized for up to
 // kMaxCtas CTAs, independent of the device.
 constexpr int kMaxCtas = 1024;
-constexpr int kSlotFloats = kHeadDim + 2;   // per query head
+// A slot holds, per query head, d accumulators then (max, sum).
 inline size_t attend_counter_bytes(int batch, int n_q_heads) {
   return ((size_t)batch * n_q_heads * sizeof(int) + 255) & ~(size_t)255;
 }
-inline size_t attend_workspace_bytes(int batch, int n_q_heads) {
+inline size_t attend_workspace_bytes(int batch, int n_q_heads, int d) {
   const size_t slots = (size_t)kMaxCtas * kMaxGroup + (size_t)batch * n_q_heads;
-  return attend_counter_bytes(batch, n_q_heads) + slots * kSlotFloats * sizeof(float);
+  return attend_counter_bytes(batch, n_q_heads) + slots * (size_t)(d + 2) * sizeof(float);
 }
 
 }  // namespace tq

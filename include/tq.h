@@ -273,13 +273,13 @@ int tq_attend_append(const void* q, int q_dtype, const void* new_kv, int kv_dtyp
  * None of the source pages has a counterpart; this is a library convenience.
  *
  * Same arguments and results as tq_attend, without workspace and
- * workspace_bytes: the scratch is one fixed 8 MiB device array inside the
+ * workspace_bytes: the scratch is one fixed 16 MiB device array inside the
  * library, allocated when the library is loaded, on every device that loads
  * it, and kept until the process exits. This call allocates and frees no
  * memory.
- *   - Limit: batch · n_q_heads <= 7879 (the problem's
- *     tq_attend_workspace_size must fit 8 MiB); larger problems return
- *     TQ_ERR_UNSUPPORTED.
+ *   - Limit: the problem's tq_attend_workspace_size must fit 16 MiB, i.e.
+ *     batch · n_q_heads <= 54530 / 23887 / 8033 at d = 64 / 128 / 256;
+ *     larger problems return TQ_ERR_UNSUPPORTED.
  *   - The first call on a device looks up the array's device address (a
  *     host-side set-up); make that first call before any stream capture.
  *   - Every call on a device shares the array. Each call first clears the

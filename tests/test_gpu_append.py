@@ -20,10 +20,9 @@ from oracle import codec
 
 pytestmark = pytest.mark.gpu
 ATOL = 2e-3
-D = 128
 
 
-def _cache(bk, bv, B, Hkv, cap, ctx, seed, rng):
+def _cache(bk, bv, B, Hkv, cap, ctx, seed, rng, D=128):
     """Oracle-encoded random cache with rows 0 .. L_b - 2 filled; row L_b - 1
     holds unrelated bytes that the append must replace."""
     pk = rng.integers(0, 256, (B, Hkv, cap, D * bk // 8), dtype=np.uint8)
@@ -45,13 +44,13 @@ def _cache(bk, bv, B, Hkv, cap, ctx, seed, rng):
 
 
 def _run(bk, bv, ctx, cap, Hkv, gqa, kv_dtype, seed, tau=0.0, n_ctas=0, qscale=1.0,
-         rng_seed=0):
+         rng_seed=0, D=128):
     import torch
     import compressed_decode_attention_b200 as tq
     rng = np.random.default_rng(rng_seed)
     ctx = np.asarray(ctx, np.int32)
     B, Hq = len(ctx), Hkv * gqa
-    pk, nk, pv, nv = _cache(bk, bv, B, Hkv, cap, ctx, seed, rng)
+    pk, nk, pv, nv = _cache(bk, bv, B, Hkv, cap, ctx, seed, rng, D)
     new = rng.standard_normal((2, B, Hkv, D))
     new[0, :, :, :4] *= 20.0                       # outlier K channels
     new_bits = S.to_bits(new, kv_dtype)
@@ -131,3 +130,11 @@ def test_append_k4v3_gate():
 
 def test_append_single_sequence_eight_heads():
     _run(4, 2, [4096], 4096, 8, 4, "f16", 0, rng_seed=4)
+
+
+@pytest.mark.parametrize("d,bk,bv,gqa", [(64, 4, 2, 4), (64, 3, 2, 5), (256, 4, 3, 4),
+                                         (256, 3, 2, 5)])
+def test_append_head_dims(d, bk, bv, gqa):
+    """d = 64 and 256: the new token's rows (d/32 lanes per vector) and the
+    attention over the updated cache."""
+    _run(bk, bv, [700, 64, 1, 1000], 768, 2, gqa, "f16", 0, rng_seed=10 + d + bk, D=d)

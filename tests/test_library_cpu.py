@@ -80,8 +80,8 @@ def _encode(**kw):
     (dict(bits_k=5), tq.TQ_ERR_INVALID_ARG),
     (dict(bits_v=1), tq.TQ_ERR_INVALID_ARG),
     (dict(d=96), tq.TQ_ERR_INVALID_ARG),                  # not a power of two
-    (dict(d=64), tq.TQ_ERR_UNSUPPORTED),
-    (dict(d=256), tq.TQ_ERR_UNSUPPORTED),
+    (dict(d=32), tq.TQ_ERR_INVALID_ARG),                  # below the supported 64..256
+    (dict(d=512), tq.TQ_ERR_INVALID_ARG),
     (dict(dtype=tq.TQ_F32), tq.TQ_ERR_INVALID_ARG),
     (dict(tok_offset=5), tq.TQ_ERR_INVALID_ARG),          # 5 + 4 > 8
     (dict(n_tok=-1), tq.TQ_ERR_INVALID_ARG),
@@ -117,7 +117,8 @@ def _attend(**kw):
     (dict(nk=FAKE + 2), tq.TQ_ERR_INVALID_ARG),
     (dict(wsb=16), tq.TQ_ERR_INVALID_ARG),                # workspace too small
     (dict(bk=1), tq.TQ_ERR_INVALID_ARG),
-    (dict(d=64), tq.TQ_ERR_UNSUPPORTED),
+    (dict(d=512), tq.TQ_ERR_INVALID_ARG),
+    (dict(d=100), tq.TQ_ERR_INVALID_ARG),
     (dict(tau=float("nan")), tq.TQ_ERR_INVALID_ARG),
     (dict(out_dtype=7), tq.TQ_ERR_INVALID_ARG),
     (dict(batch=0), tq.TQ_ERR_INVALID_ARG),
@@ -130,9 +131,12 @@ def test_attend_validation(kw, want):
 def test_workspace_size_formula():
     # counters (4·batch·heads bytes, rounded to 256) + slots of d + 2 floats for
     # 1024 CTAs x 8 heads plus one per (batch, query head)
-    def want(b, h):
-        return -(-4 * b * h // 256) * 256 + (1024 * 8 + b * h) * 130 * 4
+    def want(b, h, d=128):
+        return -(-4 * b * h // 256) * 256 + (1024 * 8 + b * h) * (d + 2) * 4
     assert tq.tq_attend_workspace_size(1, 32, 32768, 128) == want(1, 32)
     assert tq.tq_attend_workspace_size(64, 32, 16384, 128) == want(64, 32)
     assert tq.tq_attend_workspace_size(1, 1, 10, 128) == want(1, 1)
-    assert tq.tq_attend_workspace_size(1, 1, 10, 64) == 0
+    assert tq.tq_attend_workspace_size(3, 8, 10, 64) == want(3, 8, 64)
+    assert tq.tq_attend_workspace_size(3, 8, 10, 256) == want(3, 8, 256)
+    assert tq.tq_attend_workspace_size(1, 1, 10, 96) == 0
+    assert tq.tq_attend_workspace_size(1, 1, 10, 512) == 0

@@ -67,10 +67,14 @@ def test_noalloc_matches_workspace_entry_point_twice():
     assert int(status.item()) == 0
 
 
-def test_noalloc_rejects_problems_beyond_its_scratch():
+@pytest.mark.parametrize("batch,d", [(187, 128), (64, 256), (427, 64)])
+def test_noalloc_rejects_problems_beyond_its_scratch(batch, d):
+    """batch x 128 query heads just beyond the 16 MiB scratch at each head
+    dimension (23887 / 8033 / 54530 pairs fit at d = 128 / 256 / 64); the
+    call is rejected on the host before any launch."""
     import compressed_decode_attention_b200 as tq
     FAKE = 1 << 20
-    # 64 x 128 = 8192 (batch, query head) pairs need more than the 8 MiB scratch
-    st = tq.lib().tq_attend_noalloc(FAKE, 0, FAKE, FAKE, FAKE, FAKE, FAKE, 64, 128, 4,
-                                    128, 4, 2, 0, 1024, 0.0, 0, None, None, FAKE, 2, None)
+    assert tq.tq_attend_workspace_size(batch, 128, 1024, d) > 16 << 20
+    st = tq.lib().tq_attend_noalloc(FAKE, 0, FAKE, FAKE, FAKE, FAKE, FAKE, batch, 128, 4,
+                                    d, 4, 2, 0, 1024, 0.0, 0, None, None, FAKE, 2, None)
     assert st == tq.TQ_ERR_UNSUPPORTED
