@@ -138,3 +138,43 @@ def test_append_head_dims(d, bk, bv, gqa):
     """d = 64 and 256: the new token's rows (d/32 lanes per vector) and the
     attention over the updated cache."""
     _run(bk, bv, [700, 64, 1, 1000], 768, 2, gqa, "f16", 0, rng_seed=10 + d + bk, D=d)
+
+
+def test_per_layer_bit_choice_in_one_step():
+    """A decode step over layers with different bit widths (K4/V2, K3/V2,
+    K4/V3, K2/V4), sharing one workspace, each layer one tq_attend_append
+    call: every layer's output and appended rows match the oracle (a model
+    may choose the bits per layer)."""
+    import torch
+    import compressed_decode_attention_b200 as tq
+    rng = np.random.default_rng(77)
+    B, Hkv, gqa, cap, seed = 2, 2, 4, 512, 3
+    Hq = Hkv * gqa
+    ctx = np.array([300, 97], np.int32)
+    ws_bytes = tq.tq_attend_workspace_size(B, Hq, cap, 128)
+    ws = torch.zeros(ws_bytes // 4, dtype=torch.float32, device="cuda")
+    layers = [(4, 2), (3, 2), (4, 3), (2, 4)]
+    caches, news, qs, outs = [], [], [], []
+    for bk, bv in layers:
+        pk, nk, pv, nv = _cache(bk, bv, B, Hkv, cap, ctx, seed, rng)
+        caches.append([dev(x) for x in (pk, nk, pv, nv)])
+        news.append(S.f16_bits(rng.standard_normal((2, B, Hkv, 128))))
+        qs.append(S.f16_bits(rng.standard_normal((B, Hq, 128))))
+        outs.append(torch.empty((B, Hq, 128), dtype=torch.float32, device="cuda"))
+    ctx_d = dev(ctx)
+    for l, (bk, bv) in enumerate(layers):
+        c = caches[l]
+        tq.tq_attend_append(dev(qs[l]), tq.TQ_F16, dev(news[l]), tq.TQ_F16, c[0], c[1], c[2],
+                            c[3], ctx_d, B, Hq, gqa, 128, bk, bv, seed, cap, 0.0, 0, ws, ws_bytes,
+                            outs[l], tq.TQ_F32)
+    torch.cuda.synchronize()
+    for l, (bk, bv) in enumerate(layers):
+        gk, gnk, gv, gnv = [host(x) for x in caches[l]]
+        for b in range(B):
+            for which, bits, rows in ((0, bk, gk), (1, bv, gv)):
+                x = codec.promote(news[l][which, b], "f16")
+                idx, _, _, _, margin = codec.encode(x, bits, seed)
+                check_indices(codec.unpack(rows[b, :, ctx[b] - 1], bits, 128), idx, margin)
+        want, _ = oracle_attend(codec.promote(qs[l], "f16"), gk, gnk, gv, gnv, ctx, gqa, bk, bv,
+                                seed)
+        assert np.abs(host(outs[l]) - want).max() <= ATOL, (bk, bv)
