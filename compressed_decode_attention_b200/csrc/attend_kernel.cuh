@@ -53,13 +53,14 @@ namespace {
 
 // Warps per CTA: 12, or 8 at d = 256 where a 64-position stage of the K and
 // V rows is twice as large.
-template <int D>
-constexpr int warps_for() { return D == 256 ? 8 : 12; }
+
 constexpr int kMaxWarps = 12;
 constexpr int kBlk = kGateBlock;                // positions per block
 constexpr float kLog2e = 1.44269504088896340736f;
 constexpr float kKScale = 256.f;                // K codebook scale inside the MMA
-constexpr int kSmemBudget = 227 * 1024;
+// Shared memory of one CTA when `per_sm` CTAs share an SM's 228 KB (1 KB of
+// each CTA's share is reserved by the system).
+constexpr int smem_budget(int per_sm) { return per_sm == 1 ? 227 * 1024 : 228 * 1024 / per_sm - 1024; }
 constexpr int kMaxStages = 3;                   // ring slots per warp
 // Give up on a staged-data wait after this many cycles (~1 s at 2 GHz).
 constexpr long long kWaitLimitCycles = 2000000000LL;
@@ -102,15 +103,14 @@ struct Dm {
 
 template <int BK, int BV, int D>
 struct Geo {
-  static constexpr int NW = warps_for<D>();
-  // rows per 16-byte multiple of a bulk copy of K / V rows
-  static constexpr int KROWS = (D * BK / 8) % 16 == 0 ? 1 : 16 / ((D * BK / 8) % 16);
-  static constexpr int VROWS = (D * BV / 8) % 16 == 0 ? 1 : 16 / ((D * BV / 8) % 16);
-  static_assert((KROWS * D * BK / 8) % 16 == 0 && (VROWS * D * BV / 8) % 16 == 0, "row multiple");
-  static_assert(kGateBlock % KROWS == 0 && kGateBlock % VROWS == 0 && 8 % KROWS == 0 &&
-                8 % VROWS == 0, "rounded row counts stay inside a block and cap_tok");
   static constexpr int RK = D * BK / 8;                 // packed K row bytes
   static constexpr int RV = D * BV / 8;
+  // rows per 16-byte multiple of a bulk copy of K / V rows
+  static constexpr int KROWS = RK % 16 == 0 ? 1 : 16 / (RK % 16);
+  static constexpr int VROWS = RV % 16 == 0 ? 1 : 16 / (RV % 16);
+  static_assert((KROWS * RK) % 16 == 0 && (VROWS * RV) % 16 == 0, "row multiple");
+  static_assert(kGateBlock % KROWS == 0 && kGateBlock % VROWS == 0 && 8 % KROWS == 0 &&
+                8 % VROWS == 0, "rounded row counts stay inside a block and cap_tok");
   static constexpr int RVS = RV;                        // V row stride in smem
   static constexpr int KB = kBlk * RK;
   static constexpr int VB = kBlk * RVS;
@@ -126,17 +126,23 @@ struct Geo {
   static constexpr int QOFF = LUTV_OFF + LUTV;
   static constexpr int QS = kMaxGroup * D * 2 * 2;      // q~ high and low, fp16
   static constexpr int MISC = 1024;                     // kMiscWords words
-  static constexpr int MBAR = NW * kMaxStages * 8;  // per-warp ring barriers
+  static constexpr int MBAR = kMaxWarps * kMaxStages * 8;  // per-warp ring barriers
   static constexpr int APPOFF = QOFF + QS + MISC + MBAR;  // decode-step append:
   static constexpr int APP = D + 64;                    //   K row, V row, norms
   static constexpr int FIXED = APPOFF + APP;
-  static constexpr int NFIT = (kSmemBudget - FIXED) / (NW * STAGE);
+  // One CTA of 12 warps per SM (8 at d = 256, where a stage of K/V rows is
+  // twice as large). Measured: two 6-warp CTAs per SM (halved shared memory)
+  // made the attention launch 9% slower on the Llama-3-8B-shaped layer.
+  static constexpr int PER_SM = 1;
+  static constexpr int NW = D == 256 ? 8 : 12;
+  static constexpr int BUDGET = smem_budget(PER_SM);
+  static constexpr int NFIT = (BUDGET - FIXED) / (NW * STAGE);
   static constexpr int NSTAGE = NFIT > kMaxStages ? kMaxStages : NFIT;
   static constexpr int MERGE = NW * Dm<D>::STRIDE * 4;
   static constexpr int RING = NSTAGE * NW * STAGE;
   static constexpr int SMEM = FIXED + (RING > MERGE ? RING : MERGE);
   static_assert(NSTAGE >= 1, "stage ring does not fit");
-  static_assert(SMEM <= kSmemBudget, "shared memory budget");
+  static_assert(SMEM <= BUDGET, "shared memory budget");
 };
 
 
@@ -341,14 +347,14 @@ __device__ __forceinline__ uint32_t k_entry(const uint32_t* w, int p) {
 }
 
 template <int BK, int BV, int NT, int D>
-__global__ void __launch_bounds__(32 * warps_for<D>(), 1)
+__global__ void __launch_bounds__(32 * Geo<BK, BV, D>::NW, Geo<BK, BV, D>::PER_SM)
 attend_kernel(const __grid_constant__ AttendArgs a,
               const __grid_constant__ Codebook cbk,
               const __grid_constant__ Codebook cbv,
               const __grid_constant__ SignMask sm) {
   using Gm = Geo<BK, BV, D>;
   using Dd = Dm<D>;
-  constexpr int kWarps = warps_for<D>(), kThreads = 32 * kWarps;
+  constexpr int kWarps = Gm::NW, kThreads = 32 * kWarps;
   constexpr int QPL = Dd::QPL, KS = Dd::KS, NPV = Dd::NPV;
   constexpr int CBK = D * BK / 32, CBV = D * BV / 32;   // chunk bytes per tq lane
   constexpr int NR = NT == 1 ? 1 : 2;       // score rows (positions) per lane and step
@@ -621,18 +627,16 @@ attend_kernel(const __grid_constant__ AttendArgs a,
 
     // query values of the group (warp h < g loads head h), issued before the
     // block loads
-    float qraw[QPL];
-#pragma unroll
-    for (int k = 0; k < QPL; ++k) qraw[k] = 0.f;
-    if (warp < GQ) {       // coordinates QPL·lane .. QPL·lane + QPL - 1
-      const size_t qo = ((size_t)b * a.n_q_heads + (size_t)g * GQ + warp) * D + QPL * lane;
+    // query head h of the group: coordinates QPL·lane .. QPL·lane + QPL - 1
+    auto load_q = [&](int h, float (&qr)[QPL]) {
+      const size_t qo = ((size_t)b * a.n_q_heads + (size_t)g * GQ + h) * D + QPL * lane;
       if (a.q_dtype == TQ_F32) {
         const float2* src = reinterpret_cast<const float2*>(reinterpret_cast<const float*>(a.q) + qo);
 #pragma unroll
         for (int k = 0; k < QPL / 2; ++k) {
           const float2 v = src[k];
-          qraw[2 * k] = v.x;
-          qraw[2 * k + 1] = v.y;
+          qr[2 * k] = v.x;
+          qr[2 * k + 1] = v.y;
         }
       } else {
         const uint32_t* src = reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint16_t*>(a.q) + qo);
@@ -640,11 +644,15 @@ attend_kernel(const __grid_constant__ AttendArgs a,
 #pragma unroll
         for (int k = 0; k < QPL / 2; ++k) {
           const float2 f = unpack16x2(src[k], bf);
-          qraw[2 * k] = f.x;
-          qraw[2 * k + 1] = f.y;
+          qr[2 * k] = f.x;
+          qr[2 * k + 1] = f.y;
         }
       }
-    }
+    };
+    float qraw[QPL];
+#pragma unroll
+    for (int k = 0; k < QPL; ++k) qraw[k] = 0.f;
+    if (warp < GQ) load_q(warp, qraw);
 
     // ---- this warp's blocks of the segment
     // The warps split the segment in whole 64-position blocks (the sparse-V
@@ -711,13 +719,14 @@ attend_kernel(const __grid_constant__ AttendArgs a,
     auto bar_of = [&](int jj) { return wbar + 8 * (jj % Gm::NSTAGE); };
     auto par_of = [&](int jj) { return (uint32_t)(jj / Gm::NSTAGE) & 1u; };
     if (warp >= GQ) fill_ring();
-    // ---- rotated query of the group: warp h handles query head h
-    if (warp < GQ) {
+    // ---- rotated query of the group: warp w handles query heads w, w +
+    // kWarps, ... (the first one's values are already loaded)
+    auto rotate_q = [&](int h, const float (&qr)[QPL]) {
       float x[QPL];
 #pragma unroll
       for (int k = 0; k < QPL; ++k) {
         const int c = QPL * lane + k;
-        x[k] = apply_sign(qraw[k], sm.w[c >> 5], c & 31);
+        x[k] = apply_sign(qr[k], sm.w[c >> 5], c & 31);
       }
       fwht_warp<QPL>(x, lane);
       // log2(e)/d^{3/2} folds the rotation normalization, the codebook's
@@ -733,8 +742,8 @@ attend_kernel(const __grid_constant__ AttendArgs a,
       for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
       const int e = amax > 0.f ? ilogbf(amax) : 0;
       const float qs = ldexpf(1.f, min(14 - e, 120));
-      uint32_t* hdst = reinterpret_cast<uint32_t*>(qhi + warp * D + QPL * lane);
-      uint32_t* ldst = reinterpret_cast<uint32_t*>(qlo + warp * D + QPL * lane);
+      uint32_t* hdst = reinterpret_cast<uint32_t*>(qhi + h * D + QPL * lane);
+      uint32_t* ldst = reinterpret_cast<uint32_t*>(qlo + h * D + QPL * lane);
 #pragma unroll
       for (int k = 0; k < QPL; k += 2) {
         const float v0 = x[k] * qs, v1 = x[k + 1] * qs;
@@ -742,7 +751,15 @@ attend_kernel(const __grid_constant__ AttendArgs a,
         hdst[k / 2] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
         ldst[k / 2] = pack_half2(v0 - __half2float(h0), v1 - __half2float(h1));
       }
-      if (lane == 0) miscf[kMiscQInv + warp] = 1.f / (qs * kKScale);
+      if (lane == 0) miscf[kMiscQInv + h] = 1.f / (qs * kKScale);
+    };
+    if (warp < GQ) {
+      rotate_q(warp, qraw);
+      for (int h = warp + kWarps; h < GQ; h += kWarps) {
+        float q2[QPL];
+        load_q(h, q2);
+        rotate_q(h, q2);
+      }
       fill_ring();
     }
     // ---- decode-step append: the warp whose range ends at the sequence's
@@ -1147,13 +1164,13 @@ attend_kernel(const __grid_constant__ AttendArgs a,
         if (tid == 0) atomicExch(a.counters + sigma, 0);
       }
     }
-    if (finalize && warp < GQ) {
-      const float inv_l = 1.f / miscf[kMiscL + warp];
+    for (int h = warp; finalize && h < GQ; h += kWarps) {
+      const float inv_l = 1.f / miscf[kMiscL + h];
       float x[QPL];
 #pragma unroll
-      for (int k = 0; k < QPL; ++k) x[k] = fin[warp * D + QPL * lane + k] * inv_l;
+      for (int k = 0; k < QPL; ++k) x[k] = fin[h * D + QPL * lane + k] * inv_l;
       fwht_warp<QPL>(x, lane);
-      const size_t ob = ((size_t)b * a.n_q_heads + (size_t)g * GQ + warp) * D + QPL * lane;
+      const size_t ob = ((size_t)b * a.n_q_heads + (size_t)g * GQ + h) * D + QPL * lane;
 #pragma unroll
       for (int k = 0; k < QPL; ++k) {
         const int c = QPL * lane + k;
@@ -1211,13 +1228,13 @@ cudaError_t launch_one(const AttendArgs& a, const Codebook& cbk, const Codebook&
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }
-  const int grid = n_ctas > 0 ? n_ctas : sm_count();
+  const int grid = n_ctas > 0 ? n_ctas : Gm::PER_SM * sm_count();
   // Programmatic dependent launch: the kernel's set-up may overlap the tail
   // of the previous launch in the stream; it waits for that launch before
   // reading any input (griddepcontrol.wait).
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(32 * warps_for<D>());
+  cfg.blockDim = dim3(32 * Gm::NW);
   cfg.dynamicSmemBytes = Gm::SMEM;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
