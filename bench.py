@@ -28,6 +28,7 @@ the maximum over ranks.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -48,6 +49,9 @@ ENCODE_WORKLOAD = "bulk_prefill_encode"
 LAYERS = 32
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+PREFILL_CTX = 8192       # prefill measurement: context length after the chunk
+PREFILL_TOKENS = 1024    # tokens in the chunk
 
 
 # ------------------------------------------------------------------ helpers
@@ -60,10 +64,28 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def measured_tensor_peak():
+    """Dense bf16 tensor TFLOP/s measured on this machine (burst: the prefill
+    kernel is timed on its own)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return FALLBACK_BF16_TFLOPS
+
+
 def attend_bytes(w, ctx_total, q_bytes=2, out_bytes=2):
     """Algorithmic bytes of one tq_attend call: packed rows + norms + q + out."""
     row = w.d * w.bits_k // 8 + w.d * w.bits_v // 8 + 4
     return ctx_total * w.n_kv_heads * row + w.batch * w.n_q_heads * w.d * (q_bytes + out_bytes)
+
+
+def prefill_flops(w, ctx, n_tok):
+    """Algorithmic FLOPs of one tq_prefill_attend call: 2·d for q·k and 2·d
+    for the weighted V sum per (query token, head, visible position); token
+    i of the chunk sees ctx - n_tok + i + 1 positions."""
+    visible = sum(ctx - n_tok + i + 1 for i in range(n_tok))
+    return 4 * w.d * w.n_q_heads * visible
 
 
 def encode_bytes(w, n_vec_pairs):
@@ -263,6 +285,52 @@ def run_gpu(args, rank, world, local_rank):
     del kv_all
     torch.cuda.empty_cache()
 
+    # ---------------- prefill attention: a 1024-token chunk at the end of an
+    # 8192-token context (the chunk's rows are in the cache), 4 layers
+    pf_layers, pf_ctx, pf_T = 4, PREFILL_CTX, PREFILL_TOKENS
+    pf = LayerCaches(dataclasses.replace(w, ctx=pf_ctx, cap_tok=pf_ctx), pf_layers, stream)
+    for l in range(pf_layers):
+        kv_pf = device_kv(w, l, pf_ctx, gen)
+        tq.tq_encode(kv_pf, tq.TQ_F16, pf_ctx, H, d, w.bits_k, w.bits_v, seed, pf.pk[l], pf.pv[l],
+                     pf.nk[l], pf.nv[l], pf_ctx, 0, status, stream)
+        del kv_pf
+    pf_q = [torch.randn((1, pf_T, w.n_q_heads, d), generator=gen, device=device).half()
+            for _ in range(pf_layers)]
+    pf_out = [torch.empty((1, pf_T, w.n_q_heads, d), dtype=torch.float16, device=device)
+              for _ in range(pf_layers)]
+    pf_ctx_dev = torch.full((1,), pf_ctx, dtype=torch.int32, device=device)
+
+    def prefill_all():
+        for l in range(pf_layers):
+            tq.tq_prefill_attend(pf_q[l], tq.TQ_F16, pf.pk[l], pf.nk[l], pf.pv[l], pf.nv[l],
+                                 pf_ctx_dev, 1, pf_T, w.n_q_heads, w.gqa, d, w.bits_k, w.bits_v,
+                                 seed, pf_ctx, pf_out[l], tq.TQ_F16, dev_status=status,
+                                 stream=stream)
+
+    with torch.cuda.stream(stream):
+        prefill_all()
+    torch.cuda.synchronize()
+    pf_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(pf_graph, stream=stream):
+        prefill_all()
+    for _ in range(max(3, args.warmup)):
+        pf_graph.replay()
+    torch.cuda.synchronize()
+    pf_steps = max(3, min(args.steps, 10))
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(device)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        p0.record(stream)
+        for _ in range(pf_steps):
+            pf_graph.replay()
+        p1.record(stream)
+    torch.cuda.synchronize()
+    pf_ms = reduce_max(p0.elapsed_time(p1) / (pf_steps * pf_layers), device)
+    pf_flops = prefill_flops(w, pf_ctx, pf_T)
+    del pf_graph, pf, pf_q, pf_out
+    torch.cuda.empty_cache()
+
     # ---------------- decode step graphs
     q = [torch.randn((1, w.n_q_heads, d), generator=gen, device=device).half() for _ in range(L)]
     kv_new = [device_kv(w, l, 1, gen) for l in range(L)]
@@ -423,6 +491,18 @@ def run_gpu(args, rank, world, local_rank):
                                 "frac_of_nominal_8tbs": round(enc_gbs / NOMINAL_HBM_GBS, 4),
                                 "bytes_per_step": enc_bytes},
                    "gpu_launches": enc_launches},
+        "prefill": {"workload": f"{WORKLOAD} prefill chunk: {pf_T} tokens at the end of a "
+                                f"{pf_ctx}-token context (32 q / 8 kv heads, d=128, "
+                                f"K{w.bits_k}/V{w.bits_v}), {pf_layers} layer caches",
+                    "metric": "prefill attention TFLOP/s", "unit": "TFLOP/s",
+                    "value": round(world * pf_flops / (pf_ms * 1e-3) / 1e12, 2),
+                    "ms_per_call": round(pf_ms, 4),
+                    "roofline": {"bound": "tensor", "achieved": round(pf_flops / (pf_ms * 1e-3) / 1e12, 2),
+                                 "peak": measured_tensor_peak(), "unit": "TFLOP/s",
+                                 "frac": round(pf_flops / (pf_ms * 1e-3) / 1e12 / measured_tensor_peak(), 4),
+                                 "peak_kind": "measured dense bf16 (fp16 mma runs at the same rate)",
+                                 "flops_per_call": pf_flops},
+                    "gpu_launches": pf_steps * pf_layers},
         "device_status": st,
     }
     del step_graph, attend_graph, e2e_graph

@@ -59,6 +59,9 @@ def lib() -> ctypes.CDLL:
         L.tq_attend_append.restype = I
         L.tq_attend_append.argtypes = [P, I, P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F,
                                        I, P, SZ, P, P, P, I, P]
+        L.tq_prefill_attend.restype = I
+        L.tq_prefill_attend.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, I, U64, I, P, P,
+                                        I, P]
         L.tq_attend_noalloc.restype = I
         L.tq_attend_noalloc.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F, I,
                                         P, P, P, I, P]
@@ -159,6 +162,18 @@ def tq_attend_append(q, q_dtype, new_kv, kv_dtype, packed_k, norms_k, packed_v, 
         bits_k, bits_v, seed, cap_tok, float(sparse_v_thresh), n_ctas,
         _ptr(workspace), workspace_bytes, _ptr(dev_status), _ptr(sparse_v_skipped),
         _ptr(out), out_dtype, _stream(stream)))
+
+
+def tq_prefill_attend(q, q_dtype, packed_k, norms_k, packed_v, norms_v, ctx_lens, batch,
+                      n_tok, n_q_heads, gqa_ratio, d, bits_k, bits_v, seed, cap_tok, out,
+                      out_dtype, dev_status=None, stream=None):
+    """Causal attention of n_tok new query tokens per sequence over the cache
+    (q, out: [batch][n_tok][n_q_heads][d]; token i sits at position
+    ctx_lens[b] - n_tok + i)."""
+    _check("tq_prefill_attend", lib().tq_prefill_attend(
+        _ptr(q), q_dtype, _ptr(packed_k), _ptr(norms_k), _ptr(packed_v), _ptr(norms_v),
+        _ptr(ctx_lens), batch, n_tok, n_q_heads, gqa_ratio, d, bits_k, bits_v, seed, cap_tok,
+        _ptr(dev_status), _ptr(out), out_dtype, _stream(stream)))
 
 
 def tq_attend_noalloc(q, q_dtype, packed_k, norms_k, packed_v, norms_v, ctx_lens,

@@ -221,4 +221,52 @@ int tq_attend_append(const void* q, int q_dtype, const void* new_kv, int kv_dtyp
                            dev_status, sparse_v_skipped, out, out_dtype, stream);
 }
 
+int tq_prefill_attend(const void* q, int q_dtype, const uint8_t* packed_k,
+                      const uint16_t* norms_k, const uint8_t* packed_v,
+                      const uint16_t* norms_v, const int32_t* ctx_lens, int batch,
+                      int n_tok, int n_q_heads, int gqa_ratio, int d, int bits_k,
+                      int bits_v, uint64_t seed, int cap_tok, int* dev_status, void* out,
+                      int out_dtype, void* stream) {
+  if (batch < 1 || n_tok < 1 || n_q_heads < 1 || gqa_ratio < 1 || cap_tok < 1)
+    return TQ_ERR_INVALID_ARG;
+  if (n_q_heads % gqa_ratio) return TQ_ERR_INVALID_ARG;
+  if (gqa_ratio > kMaxGroup) return TQ_ERR_UNSUPPORTED;
+  if (q_dtype < TQ_F16 || q_dtype > TQ_F32 || out_dtype < TQ_F16 || out_dtype > TQ_F32)
+    return TQ_ERR_INVALID_ARG;
+  if (!bits_ok(bits_k) || !bits_ok(bits_v)) return TQ_ERR_INVALID_ARG;
+  const int hd = check_head_dim(d);
+  if (hd != TQ_OK) return hd;
+  if (d != 128) return TQ_ERR_UNSUPPORTED;       // prefill: d = 128
+  if (cap_tok % 8) return TQ_ERR_UNSUPPORTED;
+  if (!q || !packed_k || !norms_k || !packed_v || !norms_v || !ctx_lens || !out)
+    return TQ_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(packed_k) || !aligned16(packed_v) ||
+      !aligned16(norms_k) || !aligned16(norms_v) || ((uintptr_t)ctx_lens & 3u) ||
+      ((uintptr_t)dev_status & 3u))
+    return TQ_ERR_INVALID_ARG;
+  const Codebook* cbk = codebook_for(bits_k);
+  const Codebook* cbv = codebook_for(bits_v);
+  if (!cbk || !cbv) return TQ_ERR_NO_CONVERGENCE;
+  PrefillArgs a;
+  a.q = q;
+  a.q_dtype = q_dtype;
+  a.packed_k = packed_k;
+  a.norms_k = norms_k;
+  a.packed_v = packed_v;
+  a.norms_v = norms_v;
+  a.ctx_lens = ctx_lens;
+  a.batch = batch;
+  a.n_tok = n_tok;
+  a.n_q_heads = n_q_heads;
+  a.gqa = gqa_ratio;
+  a.n_kv_heads = n_q_heads / gqa_ratio;
+  a.bits_k = bits_k;
+  a.bits_v = bits_v;
+  a.cap_tok = cap_tok;
+  a.dev_status = dev_status;
+  a.out = out;
+  a.out_dtype = out_dtype;
+  return from_cuda(launch_prefill(a, *cbk, *cbv, sign_mask(seed), (cudaStream_t)stream));
+}
+
 }  // extern "C"

@@ -95,6 +95,24 @@ template <int D>
 cudaError_t launch_attend_d(const AttendArgs& a, const Codebook& cbk, const Codebook& cbv,
                             const SignMask& sm, int n_ctas, cudaStream_t stream);
 
+struct PrefillArgs {
+  const void* q;             // [batch][n_tok][n_q_heads][d]
+  int q_dtype;
+  const uint8_t* packed_k;
+  const uint16_t* norms_k;
+  const uint8_t* packed_v;
+  const uint16_t* norms_v;
+  const int32_t* ctx_lens;
+  int batch, n_tok, n_q_heads, gqa, n_kv_heads;
+  int bits_k, bits_v;
+  int cap_tok;
+  int* dev_status;
+  void* out;                 // [batch][n_tok][n_q_heads][d]
+  int out_dtype;
+};
+cudaError_t launch_prefill(const PrefillArgs& a, const Codebook& cbk, const Codebook& cbv,
+                           const SignMask& sm, cudaStream_t stream);
+
 // Workspace of tq_attend: a counter region (zero on first use; every call
 // leaves it zero) followed by partial-result slots. Sized for up to
 // kMaxCtas CTAs, independent of the device.

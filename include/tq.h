@@ -71,7 +71,7 @@
 extern "C" {
 #endif
 
-#define TQ_ABI_VERSION 2
+#define TQ_ABI_VERSION 3
 
 /* Tokens per sparse-V block; split boundaries are multiples of this. */
 #define TQ_SPARSE_V_BLOCK 64
@@ -264,6 +264,35 @@ int tq_attend_append(const void* q, int q_dtype, const void* new_kv, int kv_dtyp
                      void* workspace, size_t workspace_bytes, int* dev_status,
                      unsigned long long* sparse_v_skipped,
                      void* out, int out_dtype, void* stream);
+
+/*
+ * tq_prefill_attend — causal attention of a chunk of n_tok new query tokens
+ * per sequence over the compressed cache, the prefill counterpart of
+ * tq_attend (TurboQuant+ §3 reports prefill with the compressed cache; the
+ * scores and weighted sum follow AdapTQ §How it works, item 3). The chunk's
+ * K/V rows must already be in the cache (tq_encode at tok_offset
+ * ctx_lens[b] - n_tok). Runs on tensor cores: each CTA dequantizes a cache
+ * chunk once into shared memory for up to 128 query rows.
+ *
+ *   q           [batch][n_tok][n_q_heads][d] of q_dtype, 16-byte aligned.
+ *               Token i of sequence b sits at position
+ *               p = ctx_lens[b] - n_tok + i and attends to positions 0..p.
+ *   out         [batch][n_tok][n_q_heads][d] of out_dtype, 16-byte aligned.
+ *   packed_*, norms_*, ctx_lens, batch, n_q_heads, gqa_ratio, bits_k,
+ *               bits_v, seed, cap_tok, dev_status   as for tq_attend.
+ *               Tokens with p < 0 (ctx_lens[b] < n_tok) get out = 0 and set
+ *               TQ_DEV_CTX_EMPTY; ctx_lens[b] > cap_tok is clamped
+ *               (TQ_DEV_CTX_CLAMPED).
+ *   d           128 (TQ_ERR_UNSUPPORTED for 64 and 256).
+ * No sparse-V gate and no workspace. Errors as for tq_attend.
+ */
+int tq_prefill_attend(const void* q, int q_dtype,
+                      const uint8_t* packed_k, const uint16_t* norms_k,
+                      const uint8_t* packed_v, const uint16_t* norms_v,
+                      const int32_t* ctx_lens, int batch, int n_tok, int n_q_heads,
+                      int gqa_ratio, int d, int bits_k, int bits_v, uint64_t seed,
+                      int cap_tok, int* dev_status, void* out, int out_dtype,
+                      void* stream);
 
 /*
  * tq_attend_noalloc — tq_attend for callers that cannot allocate device
