@@ -23,6 +23,20 @@ Readings where the pages are silent or open (the library uses the same):
     score over the aligned 64-position block holding t. Since
     exp(s_t - M_blk) >= exp(s_t - max s) >= w_t / l, a gated position has
     softmax weight below tau. Gated positions stay in l. tau <= 0: no gate.
+
+Context parallelism (the pages describe one device; splitting the context
+is the library's extension): each device attends over a contiguous slice of
+the positions and reports a log-sum-exp record per query head,
+  m2  = log2(e) · max_t s_t
+  l   = sum_t exp(s_t - max s)
+  acc = sum over ungated t of exp(s_t - max s) · nV_t · cV[idx'_t]
+with cV the N(0,1) codebook, i.e. acc lives in the unnormalized Hadamard
+domain z = H·(D⊙v) of the encoder. An empty slice reports acc = 0,
+m2 = -inf, l = 0. Records of disjoint slices merge exactly:
+  M = max_p m2_p,  l = sum_p 2^(m2_p - M) · l_p,  acc likewise,
+  out = D⊙(H·(acc / l)) / d.
+Slices start at multiples of 64 positions so that the gate's blocks are the
+same as in one pass over the whole context.
 """
 from __future__ import annotations
 
@@ -101,6 +115,80 @@ def attend(q: np.ndarray, packed_k: np.ndarray, norms_k: np.ndarray,
         out[b, hs] = o
         n_gated += int(gated.sum())
     return out, n_gated
+
+
+def partial_head_group(qs: np.ndarray, idx_k: np.ndarray, nk_bits: np.ndarray,
+                       idx_v: np.ndarray, nv_bits: np.ndarray, bits_k: int,
+                       bits_v: int, seed: int, tau: float):
+    """Log-sum-exp record of the query heads qs[g, d] over the L rows of one
+    kv head in one context slice. Returns (rec[g, d + 2], gated[g, L]) with
+    rec[:, :d] = acc, rec[:, d] = m2, rec[:, d + 1] = l (module docstring)."""
+    qs = np.asarray(qs, dtype=np.float64)
+    g, d = qs.shape
+    L = idx_k.shape[0]
+    rec = np.zeros((g, d + 2))
+    if L <= 0:
+        rec[:, d] = -np.inf
+        return rec, np.zeros((g, 0), dtype=bool)
+    nk = np.asarray(nk_bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+    nv = np.asarray(nv_bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+    q_rot = _rot.rotate(qs, seed)
+    s = (q_rot @ _codec.dequant_rotated(idx_k, bits_k).T) * nk[None, :] / np.sqrt(d)
+    m = s.max(axis=1, keepdims=True)
+    w = np.exp(s - m)
+    if tau > 0.0:
+        nblk = (L + GATE_BLOCK - 1) // GATE_BLOCK
+        pad = np.full((g, nblk * GATE_BLOCK), -np.inf)
+        pad[:, :L] = s
+        mblk = pad.reshape(g, nblk, GATE_BLOCK).max(axis=2)
+        gated = np.exp(s - np.repeat(mblk, GATE_BLOCK, axis=1)[:, :L]) < tau
+    else:
+        gated = np.zeros((g, L), dtype=bool)
+    # codebook values in N(0,1) units: sqrt(d) times the rotated unit coordinates
+    cv = _codec.dequant_rotated(idx_v, bits_v) * np.sqrt(d)
+    rec[:, :d] = (np.where(gated, 0.0, w) * nv[None, :]) @ cv
+    rec[:, d] = m[:, 0] / np.log(2.0)
+    rec[:, d + 1] = w.sum(axis=1)
+    return rec, gated
+
+
+def attend_partial(q: np.ndarray, packed_k: np.ndarray, norms_k: np.ndarray,
+                   packed_v: np.ndarray, norms_v: np.ndarray, ctx_lens: np.ndarray,
+                   gqa: int, bits_k: int, bits_v: int, seed: int, tau: float = 0.0):
+    """Records [B, Hq, d + 2] of one context slice (the cache arrays and
+    ctx_lens describe the slice: its rows start at local position 0)."""
+    q = np.asarray(q, dtype=np.float64)
+    B, Hq, d = q.shape
+    Hkv, cap = packed_k.shape[1], packed_k.shape[2]
+    rec = np.zeros((B, Hq, d + 2))
+    n_gated = 0
+    for b in range(B):
+        L = max(int(min(int(ctx_lens[b]), cap)), 0)
+        for g in range(Hkv):
+            ik = _codec.unpack(packed_k[b, g, :L], bits_k, d)
+            iv = _codec.unpack(packed_v[b, g, :L], bits_v, d)
+            hs = slice(g * gqa, (g + 1) * gqa)
+            rec[b, hs], gated = partial_head_group(q[b, hs], ik, norms_k[b, g, :L], iv,
+                                                   norms_v[b, g, :L], bits_k, bits_v, seed, tau)
+            n_gated += int(gated.sum())
+    return rec, n_gated
+
+
+def combine(recs: np.ndarray, seed: int) -> np.ndarray:
+    """Merge the records [P, B, Hq, d + 2] of P disjoint slices into the
+    attention output [B, Hq, d]; heads whose every slice is empty give 0."""
+    recs = np.asarray(recs, dtype=np.float64)
+    d = recs.shape[-1] - 2
+    m2 = recs[..., d]
+    M = m2.max(axis=0)                                          # [B, Hq]
+    live = np.isfinite(M)
+    f = np.where(np.isfinite(m2), np.exp2(m2 - np.where(live, M, 0.0)[None]), 0.0)
+    l = (f * recs[..., d + 1]).sum(axis=0)
+    acc = (f[..., None] * recs[..., :d]).sum(axis=0)
+    y = acc / np.where(live, l, 1.0)[..., None]
+    # D ⊙ (H · y) / d = R^T · y / sqrt(d)
+    out = _rot.unrotate(y, seed) / np.sqrt(d)
+    return np.where(live[..., None], out, 0.0)
 
 
 def gate_values(qs, idx_k, nk_bits, bits_k, seed):

@@ -174,3 +174,64 @@ def test_context_clamp_and_empty():
     b, _ = attention.attend(q, pk, nk, pv, nv, np.array([70, 0, 0]), 1, 4, 2, 0)
     np.testing.assert_array_equal(a, b)
     np.testing.assert_array_equal(a[1:], 0.0)
+
+
+# ---- context parallelism: per-slice log-sum-exp records and their merge
+
+def _slice(arrs, ctx, a, b):
+    """The cache rows [a, b) of every sequence as a cache of its own, and the
+    number of valid rows each sequence has in it."""
+    pk, nk, pv, nv = arrs
+    loc = np.clip(np.minimum(ctx, pk.shape[2]) - a, 0, b - a)
+    return (pk[:, :, a:b], nk[:, :, a:b], pv[:, :, a:b], nv[:, :, a:b]), loc
+
+
+@pytest.mark.parametrize("tau", [0.0, 0.05])
+def test_context_slices_combine_to_whole(tau):
+    """Records of 64-aligned slices (one of them empty for every sequence)
+    merge to the dense brute-force attention over the whole context."""
+    rng = np.random.default_rng(11)
+    B, Hkv, cap, d, seed, gqa, bk, bv = 3, 2, 300, 128, 4, 2, 4, 2
+    arrs = _cache(B, Hkv, cap, d, bk, bv, seed, rng)
+    q = rng.standard_normal((B, Hkv * gqa, d)) * 3
+    ctx = np.array([300, 130, 0])
+    recs = []
+    for a, b in [(0, 64), (64, 192), (192, 300), (300, 300)]:
+        part, loc = _slice(arrs, ctx, a, b)
+        rec, _ = attention.attend_partial(q, *part, loc, gqa, bk, bv, seed, tau)
+        recs.append(rec)
+    got = attention.combine(np.stack(recs), seed)
+    want = _brute(q, *arrs, ctx, gqa, bk, bv, seed, tau)
+    np.testing.assert_allclose(got, want, atol=1e-12)
+    np.testing.assert_array_equal(got[2], 0.0)
+    # slice order does not matter
+    np.testing.assert_allclose(attention.combine(np.stack(recs[::-1]), seed), got, atol=1e-14)
+
+
+def test_partial_record_closed_form():
+    """One slice's record against the original-space quantities: 2^m2 · l is
+    sum_t exp(s_t), and D⊙(H·acc)/d is sum_t exp(s_t - max s) · v_hat_t."""
+    rng = np.random.default_rng(12)
+    d, L, seed = 128, 90, 6
+    pk, nk, pv, nv = _cache(1, 1, L, d, 3, 3, seed, rng)
+    q = rng.standard_normal((1, 1, d)) * 2
+    rec, _ = attention.attend_partial(q, pk, nk, pv, nv, np.array([L]), 1, 3, 3, seed)
+    kh = codec.dequant(codec.unpack(pk[0, 0], 3, d), nk[0, 0], 3, seed)
+    vh = codec.dequant(codec.unpack(pv[0, 0], 3, d), nv[0, 0], 3, seed)
+    s = kh @ q[0, 0] / np.sqrt(d)
+    w = np.exp(s - s.max())
+    assert rec[0, 0, d] == pytest.approx(s.max() * np.log2(np.e), abs=1e-12)
+    assert np.exp2(rec[0, 0, d]) * rec[0, 0, d + 1] == pytest.approx(np.exp(s).sum(), rel=1e-12)
+    h = scipy.linalg.hadamard(d).astype(np.float64)
+    sv = rotation.sign_vector(seed, d)
+    np.testing.assert_allclose(sv * (h @ rec[0, 0, :d]) / d, w @ vh, atol=1e-11)
+
+
+def test_empty_slice_record_and_all_empty_combine():
+    rng = np.random.default_rng(13)
+    pk, nk, pv, nv = _cache(2, 1, 64, 128, 4, 2, 0, rng)
+    q = rng.standard_normal((2, 2, 128))
+    rec, _ = attention.attend_partial(q, pk, nk, pv, nv, np.array([0, -5]), 2, 4, 2, 0)
+    np.testing.assert_array_equal(rec[..., :128], 0.0)
+    assert np.all(rec[..., 128] == -np.inf) and np.all(rec[..., 129] == 0.0)
+    np.testing.assert_array_equal(attention.combine(np.stack([rec, rec]), 0), 0.0)

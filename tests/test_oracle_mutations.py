@@ -97,3 +97,25 @@ def test_norm_not_saturated(monkeypatch):
             return np.asarray(n).astype(np.float16).view(np.uint16)
     monkeypatch.setattr(codec, "fp16_norm_bits", unsaturated)
     _fails(tc.test_norm_rounding_and_saturation)
+
+
+def test_combine_without_rescaling(monkeypatch):
+    real_exp2 = np.exp2
+    monkeypatch.setattr(attention.np, "exp2", lambda x: np.where(np.isfinite(x), 1.0, 0.0))
+    try:
+        _fails(ta.test_context_slices_combine_to_whole, 0.0)
+    finally:
+        monkeypatch.setattr(attention.np, "exp2", real_exp2)
+
+
+def test_record_max_in_natural_units(monkeypatch):
+    real = attention.partial_head_group
+    def natural(*args):
+        rec, gated = real(*args)
+        d = rec.shape[-1] - 2
+        rec = rec.copy()
+        rec[:, d] *= np.log(2.0)
+        return rec, gated
+    monkeypatch.setattr(attention, "partial_head_group", natural)
+    _fails(ta.test_partial_record_closed_form)
+    _fails(ta.test_context_slices_combine_to_whole, 0.0)
