@@ -62,6 +62,11 @@ def lib() -> ctypes.CDLL:
         L.tq_prefill_attend.restype = I
         L.tq_prefill_attend.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, I, U64, I, P, P,
                                         I, P]
+        L.tq_attend_partial.restype = I
+        L.tq_attend_partial.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F, I,
+                                        P, SZ, P, P, P, P]
+        L.tq_attend_combine.restype = I
+        L.tq_attend_combine.argtypes = [P, I, I, I, I, U64, P, P, I, P]
         L.tq_attend_noalloc.restype = I
         L.tq_attend_noalloc.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F, I,
                                         P, P, P, I, P]
@@ -174,6 +179,29 @@ def tq_prefill_attend(q, q_dtype, packed_k, norms_k, packed_v, norms_v, ctx_lens
         _ptr(q), q_dtype, _ptr(packed_k), _ptr(norms_k), _ptr(packed_v), _ptr(norms_v),
         _ptr(ctx_lens), batch, n_tok, n_q_heads, gqa_ratio, d, bits_k, bits_v, seed, cap_tok,
         _ptr(dev_status), _ptr(out), out_dtype, _stream(stream)))
+
+
+def tq_attend_partial(q, q_dtype, packed_k, norms_k, packed_v, norms_v, ctx_lens, batch,
+                      n_q_heads, gqa_ratio, d, bits_k, bits_v, seed, cap_tok,
+                      sparse_v_thresh, n_ctas, workspace, workspace_bytes, partial,
+                      dev_status=None, sparse_v_skipped=None, stream=None):
+    """Attention over one context slice, leaving log-sum-exp records
+    (float [batch][n_q_heads][d + 2]) in `partial` for tq_attend_combine."""
+    _check("tq_attend_partial", lib().tq_attend_partial(
+        _ptr(q), q_dtype, _ptr(packed_k), _ptr(norms_k), _ptr(packed_v),
+        _ptr(norms_v), _ptr(ctx_lens), batch, n_q_heads, gqa_ratio, d, bits_k,
+        bits_v, seed, cap_tok, float(sparse_v_thresh), n_ctas,
+        _ptr(workspace), workspace_bytes, _ptr(dev_status),
+        _ptr(sparse_v_skipped), _ptr(partial), _stream(stream)))
+
+
+def tq_attend_combine(partials, n_parts, batch, n_q_heads, d, seed, out, out_dtype,
+                      dev_status=None, stream=None):
+    """Merge n_parts slices' records ([n_parts][batch][n_q_heads][d + 2])
+    into the attention output."""
+    _check("tq_attend_combine", lib().tq_attend_combine(
+        _ptr(partials), n_parts, batch, n_q_heads, d, seed, _ptr(dev_status), _ptr(out),
+        out_dtype, _stream(stream)))
 
 
 def tq_attend_noalloc(q, q_dtype, packed_k, norms_k, packed_v, norms_v, ctx_lens,

@@ -29,14 +29,15 @@ int from_cuda(cudaError_t e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA; }
 
 namespace tq {
 
-// Validation and launch shared by tq_attend and tq_attend_append.
+// Validation and launch shared by tq_attend, tq_attend_append and
+// tq_attend_partial (partial_out: out receives log-sum-exp records).
 int attend_common(const void* q, int q_dtype, const void* new_kv, int kv_dtype,
                   uint8_t* packed_k, uint16_t* norms_k, uint8_t* packed_v,
                   uint16_t* norms_v, const int32_t* ctx_lens, int batch, int n_q_heads,
                   int gqa_ratio, int d, int bits_k, int bits_v, uint64_t seed, int cap_tok,
                   float sparse_v_thresh, int n_ctas, void* workspace, size_t workspace_bytes,
                   int* dev_status, unsigned long long* sparse_v_skipped, void* out,
-                  int out_dtype, void* stream) {
+                  int out_dtype, int partial_out, void* stream) {
   if (batch < 1 || n_q_heads < 1 || gqa_ratio < 1 || cap_tok < 1)
     return TQ_ERR_INVALID_ARG;
   if (n_q_heads % gqa_ratio) return TQ_ERR_INVALID_ARG;
@@ -52,7 +53,9 @@ int attend_common(const void* q, int q_dtype, const void* new_kv, int kv_dtype,
   if (!q || !packed_k || !norms_k || !packed_v || !norms_v || !ctx_lens || !out ||
       !workspace)
     return TQ_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(out) || !aligned16(packed_k) || !aligned16(packed_v) ||
+  // records (partial_out) are written two floats at a time: 8-byte alignment
+  const bool out_ok = partial_out ? ((uintptr_t)out & 7u) == 0 : aligned16(out);
+  if (!aligned16(q) || !out_ok || !aligned16(packed_k) || !aligned16(packed_v) ||
       !aligned16(norms_k) || !aligned16(norms_v) || !aligned16(workspace) ||
       ((uintptr_t)ctx_lens & 3u) || ((uintptr_t)sparse_v_skipped & 7u) ||
       ((uintptr_t)dev_status & 3u))
@@ -86,6 +89,7 @@ int attend_common(const void* q, int q_dtype, const void* new_kv, int kv_dtype,
   a.skipped = sparse_v_skipped;
   a.out = out;
   a.out_dtype = out_dtype;
+  a.partial_out = partial_out;
   return from_cuda(launch_attend(a, *cbk, *cbv, sign_mask(seed), n_ctas,
                                  (cudaStream_t)stream));
 }
@@ -201,7 +205,7 @@ int tq_attend(const void* q, int q_dtype, const uint8_t* packed_k,
                            const_cast<uint16_t*>(norms_v), ctx_lens, batch, n_q_heads,
                            gqa_ratio, d, bits_k, bits_v, seed, cap_tok, sparse_v_thresh,
                            n_ctas, workspace, workspace_bytes, dev_status, sparse_v_skipped,
-                           out, out_dtype, stream);
+                           out, out_dtype, 0, stream);
 }
 
 int tq_attend_append(const void* q, int q_dtype, const void* new_kv, int kv_dtype,
@@ -218,7 +222,44 @@ int tq_attend_append(const void* q, int q_dtype, const void* new_kv, int kv_dtyp
   return tq::attend_common(q, q_dtype, new_kv, kv_dtype, packed_k, norms_k, packed_v, norms_v,
                            ctx_lens, batch, n_q_heads, gqa_ratio, d, bits_k, bits_v, seed,
                            cap_tok, sparse_v_thresh, n_ctas, workspace, workspace_bytes,
-                           dev_status, sparse_v_skipped, out, out_dtype, stream);
+                           dev_status, sparse_v_skipped, out, out_dtype, 0, stream);
+}
+
+int tq_attend_partial(const void* q, int q_dtype, const uint8_t* packed_k,
+                      const uint16_t* norms_k, const uint8_t* packed_v,
+                      const uint16_t* norms_v, const int32_t* ctx_lens, int batch,
+                      int n_q_heads, int gqa_ratio, int d, int bits_k, int bits_v,
+                      uint64_t seed, int cap_tok, float sparse_v_thresh, int n_ctas,
+                      void* workspace, size_t workspace_bytes, int* dev_status,
+                      unsigned long long* sparse_v_skipped, float* partial, void* stream) {
+  return tq::attend_common(q, q_dtype, nullptr, TQ_F16, const_cast<uint8_t*>(packed_k),
+                           const_cast<uint16_t*>(norms_k), const_cast<uint8_t*>(packed_v),
+                           const_cast<uint16_t*>(norms_v), ctx_lens, batch, n_q_heads,
+                           gqa_ratio, d, bits_k, bits_v, seed, cap_tok, sparse_v_thresh,
+                           n_ctas, workspace, workspace_bytes, dev_status, sparse_v_skipped,
+                           partial, TQ_F32, 1, stream);
+}
+
+int tq_attend_combine(const float* partials, int n_parts, int batch, int n_q_heads, int d,
+                      uint64_t seed, int* dev_status, void* out, int out_dtype,
+                      void* stream) {
+  if (n_parts < 1 || batch < 1 || n_q_heads < 1) return TQ_ERR_INVALID_ARG;
+  if ((long long)batch * n_q_heads > (1LL << 30)) return TQ_ERR_UNSUPPORTED;
+  if (out_dtype < TQ_F16 || out_dtype > TQ_F32) return TQ_ERR_INVALID_ARG;
+  const int hd = check_head_dim(d);
+  if (hd != TQ_OK) return hd;
+  if (!partials || !out) return TQ_ERR_INVALID_ARG;
+  if (((uintptr_t)partials & 7u) || !aligned16(out) || ((uintptr_t)dev_status & 3u))
+    return TQ_ERR_INVALID_ARG;
+  CombineArgs a;
+  a.partials = partials;
+  a.n_parts = n_parts;
+  a.n_rec = batch * n_q_heads;
+  a.d = d;
+  a.dev_status = dev_status;
+  a.out = out;
+  a.out_dtype = out_dtype;
+  return from_cuda(launch_combine(a, sign_mask(seed), (cudaStream_t)stream));
 }
 
 int tq_prefill_attend(const void* q, int q_dtype, const uint8_t* packed_k,

@@ -556,7 +556,13 @@ attend_kernel(const __grid_constant__ AttendArgs a,
       const int raw = a.ctx_lens[b];
       if (a.dev_status && (raw > a.cap_tok || raw <= 0))
         atomicOr(a.dev_status, raw <= 0 ? TQ_DEV_CTX_EMPTY : TQ_DEV_CTX_CLAMPED);
-      if (raw <= 0) {
+      if (raw <= 0 && a.partial_out) {              // empty slice record
+        float* r = reinterpret_cast<float*>(a.out) + (size_t)b * a.n_q_heads * (D + 2);
+        for (int h = 0; h < a.n_q_heads; ++h, r += D + 2) {
+          for (int i = 0; i < D; i += 2) *reinterpret_cast<float2*>(r + i) = make_float2(0.f, 0.f);
+          *reinterpret_cast<float2*>(r + D) = make_float2(-INFINITY, 0.f);
+        }
+      } else if (raw <= 0) {
         const int es = a.out_dtype == TQ_F32 ? 4 : 2;
         const size_t n16 = (size_t)a.n_q_heads * D * es / 16;
         uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(a.out) +
@@ -1164,7 +1170,18 @@ attend_kernel(const __grid_constant__ AttendArgs a,
         if (tid == 0) atomicExch(a.counters + sigma, 0);
       }
     }
-    for (int h = warp; finalize && h < GQ; h += kWarps) {
+    for (int h = warp; finalize && a.partial_out && h < GQ; h += kWarps) {
+      // context-parallel slice: the record (acc, base-2 maximum, sum)
+      float* r = reinterpret_cast<float*>(a.out) +
+                 ((size_t)b * a.n_q_heads + (size_t)g * GQ + h) * (D + 2);
+#pragma unroll
+      for (int k = 0; k < QPL; k += 2)
+        *reinterpret_cast<float2*>(r + QPL * lane + k) =
+            make_float2(fin[h * D + QPL * lane + k], fin[h * D + QPL * lane + k + 1]);
+      if (lane == 0)
+        *reinterpret_cast<float2*>(r + D) = make_float2(miscf[kMiscM + h], miscf[kMiscL + h]);
+    }
+    for (int h = warp; finalize && !a.partial_out && h < GQ; h += kWarps) {
       const float inv_l = 1.f / miscf[kMiscL + h];
       float x[QPL];
 #pragma unroll

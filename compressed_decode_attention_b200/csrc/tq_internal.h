@@ -86,6 +86,10 @@ struct AttendArgs {
   unsigned long long* skipped;
   void* out;
   int out_dtype;
+  // Context-parallel slice: out is float [batch][n_q_heads][d + 2] of
+  // log-sum-exp records (acc in the unnormalized Hadamard domain, then the
+  // base-2 maximum and the sum) instead of the attention output.
+  int partial_out;
 };
 cudaError_t launch_attend(const AttendArgs& a, const Codebook& cbk,
                           const Codebook& cbv, const SignMask& sm, int n_ctas,
@@ -112,6 +116,17 @@ struct PrefillArgs {
 };
 cudaError_t launch_prefill(const PrefillArgs& a, const Codebook& cbk, const Codebook& cbv,
                            const SignMask& sm, cudaStream_t stream);
+
+struct CombineArgs {
+  const float* partials;     // [n_parts][n_rec][d + 2]
+  int n_parts;
+  int n_rec;                 // batch * n_q_heads
+  int d;
+  int* dev_status;
+  void* out;                 // [n_rec][d] of out_dtype
+  int out_dtype;
+};
+cudaError_t launch_combine(const CombineArgs& a, const SignMask& sm, cudaStream_t stream);
 
 // Workspace of tq_attend: a counter region (zero on first use; every call
 // leaves it zero) followed by partial-result slots. Sized for up to

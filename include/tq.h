@@ -71,7 +71,7 @@
 extern "C" {
 #endif
 
-#define TQ_ABI_VERSION 3
+#define TQ_ABI_VERSION 4
 
 /* Tokens per sparse-V block; split boundaries are multiples of this. */
 #define TQ_SPARSE_V_BLOCK 64
@@ -131,8 +131,7 @@ int tq_build_codebook(int bits, int d, double* centroids, double* thresholds,
  *               projection produces them. 16-byte aligned.
  *   n_tok       >= 0 tokens to encode (0 is a no-op).
  *   n_kv_heads  >= 1.
- *   d           head dimension; this build supports d = 128
- *               (other powers of two in [64, 256]: TQ_ERR_UNSUPPORTED).
+ *   d           head dimension: 64, 128 or 256 (else TQ_ERR_INVALID_ARG).
  *   bits_k, bits_v  2..4 bits per coordinate for K and for V.
  *   seed        sign-vector seed (see "Sign vector D" above).
  *   packed_k    [n_kv_heads][cap_tok][d*bits_k/8] bytes, 16-byte aligned.
@@ -292,6 +291,67 @@ int tq_prefill_attend(const void* q, int q_dtype,
                       const int32_t* ctx_lens, int batch, int n_tok, int n_q_heads,
                       int gqa_ratio, int d, int bits_k, int bits_v, uint64_t seed,
                       int cap_tok, int* dev_status, void* out, int out_dtype,
+                      void* stream);
+
+/*
+ * Context parallelism: the positions of every sequence are split over the
+ * devices of a group, each device attends over its own slice and the
+ * per-slice results are merged. The source pages run on one device; this
+ * split is the library's extension, and it is exact (the log-sum-exp
+ * identity), so the merged output equals tq_attend over the whole context
+ * within the attention tolerance.
+ *
+ * Record layout (one per (sequence, query head), float32, d + 2 values):
+ *   acc[0..d-1]  sum over the slice's ungated positions t of
+ *                2^(s_t·log2(e) - m2) · nV_t · cV[idxV_t], cV the N(0,1)
+ *                codebook: the value sum in the unnormalized Hadamard
+ *                domain z = H·(D⊙v) of the encoder, not yet rotated back.
+ *   acc[d]       m2 = log2(e) · max_t s_t (base-2 maximum score).
+ *   acc[d + 1]   l = sum over ALL the slice's positions of 2^(s_t·log2(e) - m2).
+ * A slice with no position gives acc = 0, m2 = -inf, l = 0.
+ * s_t, nV_t, idxV_t and the gate are those of tq_attend.
+ *
+ * tq_attend_partial — tq_attend over one slice, writing records.
+ *   The cache arguments describe the slice as a cache of its own: row 0 of
+ *   each (sequence, kv head) is the slice's first position, ctx_lens[b] is
+ *   the number of positions sequence b has in the slice (<= 0: an empty
+ *   record and TQ_DEV_CTX_EMPTY, which is normal for a short sequence).
+ *   For the sparse-V gate to act as in one pass over the whole context, a
+ *   slice must start at a multiple of TQ_SPARSE_V_BLOCK positions (its
+ *   blocks are aligned to its own row 0).
+ *   partial     float [batch][n_q_heads][d + 2] records, 8-byte aligned (so
+ *               row p of a gathered [n_parts][...] buffer always qualifies).
+ *   All other arguments, the workspace contract and the errors are those of
+ *   tq_attend.
+ */
+int tq_attend_partial(const void* q, int q_dtype,
+                      const uint8_t* packed_k, const uint16_t* norms_k,
+                      const uint8_t* packed_v, const uint16_t* norms_v,
+                      const int32_t* ctx_lens, int batch, int n_q_heads,
+                      int gqa_ratio, int d, int bits_k, int bits_v, uint64_t seed,
+                      int cap_tok, float sparse_v_thresh, int n_ctas,
+                      void* workspace, size_t workspace_bytes, int* dev_status,
+                      unsigned long long* sparse_v_skipped,
+                      float* partial, void* stream);
+
+/*
+ * tq_attend_combine — merge the records of n_parts disjoint slices and
+ * rotate the result back once:
+ *   M = max_p m2_p, f_p = 2^(m2_p - M) (0 for an empty slice),
+ *   l = sum_p f_p·l_p, acc = sum_p f_p·acc_p, out = D⊙(H·(acc / l)) / d.
+ *   partials    float [n_parts][batch][n_q_heads][d + 2], 8-byte aligned
+ *               (e.g. the all-gather of every device's tq_attend_partial
+ *               output, in any order of the parts).
+ *   n_parts >= 1; batch, n_q_heads >= 1; d = 64, 128 or 256.
+ *   seed        the sign-vector seed of the cache.
+ *   dev_status  device int, nullable: TQ_DEV_CTX_EMPTY when a (sequence,
+ *               head) had no position in any slice (its output is 0).
+ *   out         [batch][n_q_heads][d] of out_dtype, 16-byte aligned.
+ * Errors: TQ_ERR_INVALID_ARG for a null or misaligned pointer or a bad
+ * size or dtype; TQ_ERR_CUDA for a failed launch.
+ */
+int tq_attend_combine(const float* partials, int n_parts, int batch, int n_q_heads,
+                      int d, uint64_t seed, int* dev_status, void* out, int out_dtype,
                       void* stream);
 
 /*

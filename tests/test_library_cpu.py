@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_status_strings():
-    assert tq.tq_abi_version() == 3
+    assert tq.tq_abi_version() == 4
     assert tq.status_string(0) == "TQ_OK"
     assert tq.status_string(2) == "TQ_ERR_UNSUPPORTED"
 
@@ -140,3 +140,51 @@ def test_workspace_size_formula():
     assert tq.tq_attend_workspace_size(3, 8, 10, 256) == want(3, 8, 256)
     assert tq.tq_attend_workspace_size(1, 1, 10, 96) == 0
     assert tq.tq_attend_workspace_size(1, 1, 10, 512) == 0
+
+
+def _combine(**kw):
+    a = dict(parts=FAKE, n=2, batch=2, hq=8, d=128, seed=0, status=None, out=FAKE,
+             out_dtype=tq.TQ_F32, stream=0)
+    a.update(kw)
+    return tq.lib().tq_attend_combine(a["parts"], a["n"], a["batch"], a["hq"], a["d"],
+                                      a["seed"], a["status"], a["out"], a["out_dtype"],
+                                      a["stream"])
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(parts=None), tq.TQ_ERR_INVALID_ARG),
+    (dict(out=None), tq.TQ_ERR_INVALID_ARG),
+    (dict(n=0), tq.TQ_ERR_INVALID_ARG),
+    (dict(batch=0), tq.TQ_ERR_INVALID_ARG),
+    (dict(hq=-1), tq.TQ_ERR_INVALID_ARG),
+    (dict(d=96), tq.TQ_ERR_INVALID_ARG),
+    (dict(d=512), tq.TQ_ERR_INVALID_ARG),
+    (dict(parts=FAKE + 4), tq.TQ_ERR_INVALID_ARG),       # records need 8-byte alignment
+    (dict(out=FAKE + 4), tq.TQ_ERR_INVALID_ARG),
+    (dict(out_dtype=3), tq.TQ_ERR_INVALID_ARG),
+    (dict(status=FAKE + 2), tq.TQ_ERR_INVALID_ARG),
+])
+def test_combine_validation(kw, want):
+    assert _combine(**kw) == want
+
+
+def _partial(**kw):
+    a = dict(q=FAKE, pk=FAKE, ws=FAKE, wsb=1 << 30, part=FAKE, d=128, gqa=4, bk=4)
+    a.update(kw)
+    return tq.lib().tq_attend_partial(a["q"], tq.TQ_F16, a["pk"], FAKE, FAKE, FAKE, FAKE, 2, 8,
+                                      a["gqa"], a["d"], a["bk"], 2, 0, 256, 0.0, 0, a["ws"],
+                                      a["wsb"], None, None, a["part"], 0)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(part=None), tq.TQ_ERR_INVALID_ARG),
+    (dict(part=FAKE + 4), tq.TQ_ERR_INVALID_ARG),         # records need 8-byte alignment
+    (dict(q=None), tq.TQ_ERR_INVALID_ARG),
+    (dict(ws=None), tq.TQ_ERR_INVALID_ARG),
+    (dict(wsb=16), tq.TQ_ERR_INVALID_ARG),
+    (dict(gqa=3), tq.TQ_ERR_INVALID_ARG),
+    (dict(d=100), tq.TQ_ERR_INVALID_ARG),
+    (dict(bk=5), tq.TQ_ERR_INVALID_ARG),
+])
+def test_partial_validation(kw, want):
+    assert _partial(**kw) == want
