@@ -17,6 +17,11 @@ and the 126 MB L2 cannot hold them. Steps are CUDA-graph replays.
           pinned host memory and its output back
   encode  bulk prefill encode of the same 32 x 8 x 32768 K/V (4.29 GB of fp16
           input): Mtok/s (model tokens/s and token-head vectors/s)
+  prefill causal attention of a 1024-token chunk over an 8192-token
+          compressed context (tensor cores): TFLOP/s
+  context_parallel  the same attention split into 4 slices of the context,
+          emulated on one GPU: 4 tq_attend_partial launches + tq_attend_combine
+          per layer, against the one-pass launch
 
 `--impl reference` times the CPU oracle (float64 numpy) on a bounded sample
 of the same workload instead.
@@ -50,6 +55,7 @@ LAYERS = 32
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+CP_SLICES = 4            # context-parallel measurement: slices per sequence
 PREFILL_CTX = 8192       # prefill measurement: context length after the chunk
 PREFILL_TOKENS = 1024    # tokens in the chunk
 
@@ -407,6 +413,60 @@ def run_gpu(args, rank, world, local_rank):
     attend_ms_mean = reduce_max(a0.elapsed_time(a1) / (args.steps * L), device)
     launches += L * args.steps
 
+    # ---------------- context parallelism, P slices emulated on this GPU: per
+    # layer, one tq_attend_partial per slice of whole 64-position blocks
+    # (views into the layer cache: row offset, cap_tok kept as the head
+    # stride), then tq_attend_combine of the P records. On P GPUs the
+    # partials run concurrently and an all-gather of the records precedes
+    # the combine; here they run back to back.
+    from compressed_decode_attention_b200.context_parallel import slice_bounds
+    P = CP_SLICES
+    spans = [slice_bounds(ctx, P, r) for r in range(P)]
+    cp_lens = [torch.full((1,), b - a, dtype=torch.int32, device=device) for a, b in spans]
+    rec = torch.empty((P, 1, w.n_q_heads, d + 2), dtype=torch.float32, device=device)
+    rk, rv = d * w.bits_k // 8, d * w.bits_v // 8
+
+    def cp_partials(l):
+        for r, (a, _) in enumerate(spans):
+            tq.tq_attend_partial(q[l], tq.TQ_F16, caches.pk[l].data_ptr() + a * rk,
+                                 caches.nk[l].data_ptr() + 2 * a,
+                                 caches.pv[l].data_ptr() + a * rv,
+                                 caches.nv[l].data_ptr() + 2 * a, cp_lens[r], 1, w.n_q_heads,
+                                 w.gqa, d, w.bits_k, w.bits_v, seed, cap, 0.0, 0, ws, ws_bytes,
+                                 rec[r], dev_status=status, stream=stream)
+
+    def cp_combine(l):
+        tq.tq_attend_combine(rec, P, 1, w.n_q_heads, d, seed, outs[l], tq.TQ_F16,
+                             dev_status=status, stream=stream)
+
+    def cp_all():
+        for l in range(L):
+            cp_partials(l)
+            cp_combine(l)
+
+    def combine_all():
+        for l in range(L):
+            cp_combine(l)
+
+    cp_times = {}
+    for name, fn, per in (("layer", cp_all, P + 1), ("combine", combine_all, 1)):
+        g = capture(fn)
+        for _ in range(args.warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(device)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            c0.record(stream)
+            for _ in range(args.steps):
+                g.replay()
+            c1.record(stream)
+        torch.cuda.synchronize()
+        cp_times[name] = reduce_max(c0.elapsed_time(c1) / (args.steps * L), device)
+        launches += per * L * args.steps
+        del g
+
     # ---------------- end to end: host inputs in, host output back, every step
     q_host = torch.empty((L, 1, w.n_q_heads, d), dtype=torch.float16).pin_memory()
     kv_host = torch.empty((L, 2, 1, H, d), dtype=torch.int16).pin_memory()
@@ -503,6 +563,15 @@ def run_gpu(args, rank, world, local_rank):
                                  "peak_kind": "measured dense bf16 (fp16 mma runs at the same rate)",
                                  "flops_per_call": pf_flops},
                     "gpu_launches": pf_steps * pf_layers},
+        "context_parallel": {
+            "slices": P, "emulated_on_one_gpu": True,
+            "per_layer": f"{P} x tq_attend_partial over {ctx // P}-position slices + "
+                         "tq_attend_combine of the records (no all-gather on one GPU)",
+            "layer_ms": round(cp_times["layer"], 5),
+            "one_pass_layer_ms": round(attend_ms_mean, 5),
+            "achieved_gbs": round(per_layer_attend / (cp_times["layer"] * 1e-3) / 1e9, 1),
+            "combine_ms": round(cp_times["combine"], 5),
+            "record_bytes_per_slice": int(w.n_q_heads * (d + 2) * 4)},
         "device_status": st,
     }
     del step_graph, attend_graph, e2e_graph
