@@ -100,6 +100,13 @@ __device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) {
   return r;
 }
 
+// sat(a·b + c): the fused multiply-add clamped to [0, 1] (one rounding).
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float r;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // 0xFFFFFFFF if a >= b else 0 (one compare-and-set).
 __device__ __forceinline__ uint32_t set_ge(float a, float b) {
   uint32_t r;

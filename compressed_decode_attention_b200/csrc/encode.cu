@@ -4,8 +4,8 @@
 // Thread layout: d/32 lanes per vector (2, 4 or 8 for d = 64, 128, 256), 32
 // consecutive coordinates per lane. A 256-thread block encodes 256/(d/32)
 // consecutive tokens of one kv head (K or V) per step, so its packed rows and
-// norms form one contiguous range; blocks stride over the (tile, head, K/V)
-// units. The per-vector arithmetic
+// norms form one contiguous range; the grid is (tile blocks, kv head, K/V)
+// and a block strides over its head's tiles. The per-vector arithmetic
 // (encode_common.cuh) uses two-wide fp32 operations, since the kernel is
 // bound by instruction issue:
 //   load    4 x 16-byte loads per lane (the vector's 256 bytes, coalesced),
@@ -22,8 +22,9 @@ namespace {
 
 constexpr int kEncThreads = 256;
 
-// Grid-stride over (token tile, kv head, K/V): each group of four lanes
-// encodes one vector per iteration; its half2 sign masks are built once.
+// Grid (tile blocks, kv head, K/V): block (x, h, is_v) strides over the
+// token tiles of one kv head's K or V; each group of d/32 lanes encodes one
+// vector per iteration; its half2 sign masks are built once.
 template <int D>
 __global__ void __launch_bounds__(kEncThreads)
 encode_kernel(const __grid_constant__ EncodeArgs a,
@@ -41,39 +42,31 @@ encode_kernel(const __grid_constant__ EncodeArgs a,
   const unsigned gmask = ((1u << LPV) - 1u) << (lane & ~(LPV - 1));
   uint32_t smask[16];
   sign_masks(sm, sub, smask);
-  const int tiles = (a.n_tok + kTokens - 1) / kTokens;
-  const long long units = (long long)tiles * a.n_kv_heads * 2;
-  for (long long u = blockIdx.x; u < units; u += gridDim.x) {
-    const int tile = (int)(u % tiles);
-    const int h = (int)((u / tiles) % a.n_kv_heads);
-    const int is_v = (int)(u / ((long long)tiles * a.n_kv_heads));
-    const int tok = tile * kTokens + threadIdx.x / LPV;
-    if (tok >= a.n_tok) continue;                     // whole lane groups
-
-    const uint16_t* src = a.kv + ((size_t)(is_v * a.n_tok + tok) * a.n_kv_heads + h) * D;
+  const int h = blockIdx.y;
+  const int is_v = blockIdx.z;
+  const int bits = is_v ? a.bits_v : a.bits_k;
+  const Codebook& cb = is_v ? cbv : cbk;
+  const size_t rb = (size_t)D * bits / 8;
+  uint8_t* packed = (is_v ? a.packed_v : a.packed_k) + ((size_t)h * a.cap_tok + a.tok_offset) * rb;
+  uint16_t* norms = (is_v ? a.norms_v : a.norms_k) + (size_t)h * a.cap_tok + a.tok_offset;
+  const uint16_t* src0 = a.kv + ((size_t)is_v * a.n_tok * a.n_kv_heads + h) * D;
+  const size_t tok_stride = (size_t)a.n_kv_heads * D;
+  for (int tok = blockIdx.x * kTokens + threadIdx.x / LPV; tok < a.n_tok;
+       tok += gridDim.x * kTokens) {
     float x[32];
-    load_signed(src, sub, a.is_bf16, smask, x);
-
-    const size_t row = (size_t)h * a.cap_tok + a.tok_offset + tok;
-    const int bits = is_v ? a.bits_v : a.bits_k;
-    const Codebook& cb = is_v ? cbv : cbk;
-    uint8_t* packed = is_v ? a.packed_v : a.packed_k;
-    uint16_t* norms = (is_v ? a.norms_v : a.norms_k) + row;
-    const size_t rb = (size_t)D * bits / 8;
+    load_signed(src0 + tok * tok_stride, sub, a.is_bf16, smask, x);
     if (bits == 4)
-      encode_vector<4, LPV>(x, cb, sub, gmask, packed + row * rb, norms, a.dev_status);
+      encode_vector<4, LPV>(x, cb, sub, gmask, packed + tok * rb, norms + tok, a.dev_status);
     else if (bits == 3)
-      encode_vector<3, LPV>(x, cb, sub, gmask, packed + row * rb, norms, a.dev_status);
+      encode_vector<3, LPV>(x, cb, sub, gmask, packed + tok * rb, norms + tok, a.dev_status);
     else
-      encode_vector<2, LPV>(x, cb, sub, gmask, packed + row * rb, norms, a.dev_status);
+      encode_vector<2, LPV>(x, cb, sub, gmask, packed + tok * rb, norms + tok, a.dev_status);
   }
 }
 
 template <int D>
 cudaError_t launch_encode_d(const EncodeArgs& a, const Codebook& cbk, const Codebook& cbv,
                             const SignMask& sm, cudaStream_t stream) {
-  // Enough resident blocks to cover every SM several times; each block then
-  // strides over the (tile, head, K/V) units.
   static int sms = 0;
   if (!sms) {
     int dev = 0;
@@ -81,11 +74,15 @@ cudaError_t launch_encode_d(const EncodeArgs& a, const Codebook& cbk, const Code
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       sms = 148;
   }
+  // grid.x: enough tile blocks that all (head, K/V) pairs cover every SM
+  // about eight times; each block strides over its head's tiles
   constexpr int kTokens = kEncThreads / (D / 32);
-  const long long units = (long long)((a.n_tok + kTokens - 1) / kTokens) * a.n_kv_heads * 2;
-  const int grid = (int)(units < (long long)sms * 8 ? units : (long long)sms * 8);
+  const int tiles = (a.n_tok + kTokens - 1) / kTokens;
+  const int pairs = a.n_kv_heads * 2;
+  int gx = (sms * 8 + pairs - 1) / pairs;
+  if (gx > tiles) gx = tiles;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
+  cfg.gridDim = dim3(gx, a.n_kv_heads, 2);
   cfg.blockDim = dim3(kEncThreads);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

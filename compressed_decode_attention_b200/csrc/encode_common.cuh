@@ -96,30 +96,61 @@ __device__ __forceinline__ void encode_vector(
     }
   }
 
-  // idx = #{j : z/n >= t_j}, evaluated as z against n·t_j. Positive half of
-  // the table: T_k = n·t_{half-1+k}, k = 1..half-1 (t_{half-1} = 0).
-  // z >= 0: idx = half + #{k : T_k <= z};  z < 0: idx = half-1 - #{k : T_k < |z|}.
-  // The strict comparison uses |z| lowered by one ulp. A zero vector keeps
-  // n = 0, z = 0 and must land on idx = half: scale the table by 1 instead.
-  // Counts are sums of compare results (0 or -1).
-  const float sc = n > 0.f ? n : 1.f;
-  float T[kHalf > 1 ? kHalf - 1 : 1];
+  // idx = #{j : z/n >= t_j} over the symmetric table (t_{half-1} = 0), on
+  // the FMA pipe. With a = |z| and the positive thresholds t_k (k = 1 ..
+  // half-1, N(0,1) units), each indicator [a < n·t_k] is the saturated
+  //   y_k = sat(t_k·2^24 - a·(2^24/n))
+  // (1 below the threshold, 0 at or above it, fractional only within
+  // 2^-24 of it in zeta = z/n: inside the comparison window, where either
+  // index is acceptable). With the odd number
+  // w = 2·count + 1 = (2·half - 1) - 2·sum_k y_k:
+  //   z >= 0: 2·idx = 2·(half + count)     = (2·half - 1) + w
+  //   z <  0: 2·idx = 2·(half - 1 - count) = (2·half - 1) - w
+  // so u = copysign(w, z) + (2·half - 1) = 2·idx, and 2^24 + u rounds to
+  // an even number (fp32 spacing 2 there) whose mantissa bits are idx. A
+  // zero vector keeps n = 0, z = 0 (made +0 by adding +0) and lands on
+  // idx = half: its scale uses n = 1.
+  constexpr float kTwo24 = 16777216.f;
+  constexpr int NTH = kHalf - 1;                      // positive thresholds
+  const float big = __frcp_rn(n > 0.f ? n : 1.f) * kTwo24;
+  float C[NTH];
 #pragma unroll
-  for (int k = 1; k < kHalf; ++k) T[k - 1] = sc * cb.threshold[kHalf - 1 + k];
+  for (int k = 0; k < NTH; ++k) C[k] = cb.threshold[kHalf + k] * kTwo24;
+  constexpr float kOdd = (float)(2 * kHalf - 1);
+  constexpr uint32_t kMagic = 0x4B800000u;            // bits of 2^24
 
+  // words[w] accumulates bits(v) << off = (kMagic + idx) << off; the kMagic
+  // parts are removed after the loop
   uint32_t words[BITS] = {};
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const float z = x[i];
-    const bool neg = z < 0.f;
-    const float a = __uint_as_float((__float_as_uint(z) & 0x7FFFFFFFu) - (neg ? 1u : 0u));
-    uint32_t s = 0;                                   // = -count
+  for (int i = 0; i < 32; i += 2) {
+    float2 w2 = make_float2(kOdd, kOdd);
+    const float a0 = fabsf(x[i]), a1 = fabsf(x[i + 1]);
 #pragma unroll
-    for (int k = 0; k < kHalf - 1; ++k) s += set_ge(a, T[k]);
-    const uint32_t idx = neg ? (uint32_t)(kHalf - 1) + s : (uint32_t)kHalf - s;
-    const int p = i * BITS, w = p >> 5, off = p & 31;
-    words[w] += idx << off;                           // fields do not overlap
-    if (off + BITS > 32) words[w + 1] += idx >> (32 - off);
+    for (int k = 0; k < NTH; ++k)
+      w2 = f2fma(make_float2(fma_sat(a0, -big, C[k]), fma_sat(a1, -big, C[k])),
+                 make_float2(-2.f, -2.f), w2);
+    const float2 sg = f2add(make_float2(x[i], x[i + 1]), make_float2(0.f, 0.f));
+    const float2 u = f2add(make_float2(copysignf(w2.x, sg.x), copysignf(w2.y, sg.y)),
+                           make_float2(kOdd, kOdd));
+    const float2 v = f2add(u, make_float2(kTwo24, kTwo24));
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const uint32_t b = __float_as_uint(e ? v.y : v.x);    // kMagic + idx
+      const int p = (i + e) * BITS, w = p >> 5, off = p & 31;
+      words[w] += b << off;
+      if (off + BITS > 32) words[w + 1] += (b - kMagic) >> (32 - off);
+    }
+  }
+#pragma unroll
+  for (int w = 0; w < BITS; ++w) {
+    uint32_t c = 0;                                   // the kMagic parts, mod 2^32
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int p = i * BITS;
+      if ((p >> 5) == w) c += kMagic << (p & 31);
+    }
+    words[w] -= c;
   }
 
   if constexpr (BITS == 4) {
