@@ -161,3 +161,10 @@ def ctx_lens(w: Workload) -> np.ndarray:
     rng = rng_for(w.name, "ctx-lens")
     return rng.integers(lo, hi + 1, size=w.batch).astype(np.int32)
 
+
+
+def projection_matrix(d: int, index: int = 0) -> np.ndarray:
+    """[d][d] float32 with i.i.d. N(0, 1) entries: the random projection of
+    the residual sketch, drawn by the caller and passed to both sides."""
+    return rng_for("residual-sketch", "projection", d, index).standard_normal((d, d)) \
+        .astype(np.float32)

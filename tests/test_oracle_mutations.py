@@ -119,3 +119,36 @@ def test_record_max_in_natural_units(monkeypatch):
     monkeypatch.setattr(attention, "partial_head_group", natural)
     _fails(ta.test_partial_record_closed_form)
     _fails(ta.test_context_slices_combine_to_whole, 0.0)
+
+
+def test_sketch_without_the_sqrt_pi_over_2_factor(monkeypatch):
+    from oracle import qjl
+    real = qjl.correction
+    monkeypatch.setattr(qjl, "correction",
+                        lambda *a: real(*a) / np.sqrt(np.pi / 2.0))
+    import test_oracle_qjl as tq
+    _fails(tq.test_correction_is_unbiased_with_the_closed_form_variance, 4)
+
+
+def test_sketch_bit_convention_flipped(monkeypatch):
+    from oracle import qjl
+    real = qjl.sketch
+    def flipped(r_rot, Sm):
+        rows, u, gb = real(r_rot, Sm)
+        return np.invert(rows), u, gb
+    monkeypatch.setattr(qjl, "sketch", flipped)
+    import test_oracle_qjl as tq
+    _fails(tq.test_correction_is_unbiased_with_the_closed_form_variance, 2)
+    _fails(tq.test_sketch_bits_by_hand)
+
+
+def test_sketch_of_the_unrotated_residual(monkeypatch):
+    from oracle import qjl
+    real = qjl.residual_rotated
+    def unrotated(x, bits, seed):
+        idx, nb, r_rot = real(x, bits, seed)
+        return idx, nb, rotation.unrotate(r_rot, seed)
+    monkeypatch.setattr(qjl, "residual_rotated", unrotated)
+    import test_oracle_qjl as tq
+    _fails(tq.test_residual_is_the_original_space_difference)
+    _fails(tq.test_rotated_sketch_equals_original_space_sketch_with_S_R)
