@@ -67,6 +67,10 @@ def lib() -> ctypes.CDLL:
                                         P, SZ, P, P, P, P]
         L.tq_attend_combine.restype = I
         L.tq_attend_combine.argtypes = [P, I, I, I, I, U64, P, P, I, P]
+        L.tq_qjl_encode.restype = I
+        L.tq_qjl_encode.argtypes = [P, I, I, I, I, I, U64, P, P, P, P, P, I, I, P, P]
+        L.tq_qjl_scores.restype = I
+        L.tq_qjl_scores.argtypes = [P, I, P, P, P, P, P, P, I, I, I, I, I, U64, I, I, P, P, P]
         L.tq_attend_noalloc.restype = I
         L.tq_attend_noalloc.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F, I,
                                         P, P, P, I, P]
@@ -202,6 +206,27 @@ def tq_attend_combine(partials, n_parts, batch, n_q_heads, d, seed, out, out_dty
     _check("tq_attend_combine", lib().tq_attend_combine(
         _ptr(partials), n_parts, batch, n_q_heads, d, seed, _ptr(dev_status), _ptr(out),
         out_dtype, _stream(stream)))
+
+
+def tq_qjl_encode(k, dtype, n_tok, n_kv_heads, d, bits_k, seed, projection, packed_k, norms_k,
+                  sketch, gamma, cap_tok, tok_offset, dev_status=None, stream=None):
+    """Residual sketch rows (d/8 bytes) and fp16 residual norms of n_tok keys
+    ([n_tok][n_kv_heads][d]) whose stage-1 rows are in packed_k / norms_k."""
+    _check("tq_qjl_encode", lib().tq_qjl_encode(
+        _ptr(k), dtype, n_tok, n_kv_heads, d, bits_k, seed, _ptr(projection), _ptr(packed_k),
+        _ptr(norms_k), _ptr(sketch), _ptr(gamma), cap_tok, tok_offset, _ptr(dev_status),
+        _stream(stream)))
+
+
+def tq_qjl_scores(q, q_dtype, packed_k, norms_k, sketch, gamma, projection, ctx_lens, batch,
+                  n_q_heads, gqa_ratio, d, bits_k, seed, cap_tok, with_sketch, scores,
+                  dev_status=None, stream=None):
+    """Estimated scores [batch][n_q_heads][cap_tok] (float) of the first
+    ctx_lens[b] keys; with_sketch adds the unbiased residual correction."""
+    _check("tq_qjl_scores", lib().tq_qjl_scores(
+        _ptr(q), q_dtype, _ptr(packed_k), _ptr(norms_k), _ptr(sketch), _ptr(gamma),
+        _ptr(projection), _ptr(ctx_lens), batch, n_q_heads, gqa_ratio, d, bits_k, seed, cap_tok,
+        int(with_sketch), _ptr(dev_status), _ptr(scores), _stream(stream)))
 
 
 def tq_attend_noalloc(q, q_dtype, packed_k, norms_k, packed_v, norms_v, ctx_lens,

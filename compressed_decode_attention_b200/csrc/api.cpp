@@ -310,4 +310,84 @@ int tq_prefill_attend(const void* q, int q_dtype, const uint8_t* packed_k,
   return from_cuda(launch_prefill(a, *cbk, *cbv, sign_mask(seed), (cudaStream_t)stream));
 }
 
+int tq_qjl_encode(const void* k, int dtype, int n_tok, int n_kv_heads, int d, int bits_k,
+                  uint64_t seed, const float* projection, const uint8_t* packed_k,
+                  const uint16_t* norms_k, uint8_t* sketch, uint16_t* gamma, int cap_tok,
+                  int tok_offset, int* dev_status, void* stream) {
+  if (n_tok < 0 || n_kv_heads < 1 || cap_tok < 1 || tok_offset < 0)
+    return TQ_ERR_INVALID_ARG;
+  if ((long long)tok_offset + n_tok > cap_tok) return TQ_ERR_INVALID_ARG;
+  if (n_kv_heads > kMaxGridYZ) return TQ_ERR_UNSUPPORTED;
+  if (dtype != TQ_F16 && dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
+  if (!bits_ok(bits_k)) return TQ_ERR_INVALID_ARG;
+  const int hd = check_head_dim(d);
+  if (hd != TQ_OK) return hd;
+  if (!k || !projection || !packed_k || !norms_k || !sketch || !gamma) return TQ_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(projection) || !aligned16(packed_k) ||
+      ((uintptr_t)norms_k & 1u) || ((uintptr_t)gamma & 1u) || ((uintptr_t)dev_status & 3u))
+    return TQ_ERR_INVALID_ARG;
+  if (n_tok == 0) return TQ_OK;
+  const Codebook* cb = codebook_for(bits_k);
+  if (!cb) return TQ_ERR_NO_CONVERGENCE;
+  QjlEncodeArgs a;
+  a.k = (const uint16_t*)k;
+  a.is_bf16 = dtype == TQ_BF16;
+  a.d = d;
+  a.n_tok = n_tok;
+  a.n_kv_heads = n_kv_heads;
+  a.bits_k = bits_k;
+  a.packed_k = packed_k;
+  a.norms_k = norms_k;
+  a.S = projection;
+  a.sketch = sketch;
+  a.gamma = gamma;
+  a.cap_tok = cap_tok;
+  a.tok_offset = tok_offset;
+  a.dev_status = dev_status;
+  return from_cuda(launch_qjl_encode(a, *cb, sign_mask(seed), (cudaStream_t)stream));
+}
+
+int tq_qjl_scores(const void* q, int q_dtype, const uint8_t* packed_k, const uint16_t* norms_k,
+                  const uint8_t* sketch, const uint16_t* gamma, const float* projection,
+                  const int32_t* ctx_lens, int batch, int n_q_heads, int gqa_ratio, int d,
+                  int bits_k, uint64_t seed, int cap_tok, int with_sketch, int* dev_status,
+                  float* scores, void* stream) {
+  if (batch < 1 || n_q_heads < 1 || gqa_ratio < 1 || cap_tok < 1) return TQ_ERR_INVALID_ARG;
+  if (n_q_heads % gqa_ratio) return TQ_ERR_INVALID_ARG;
+  if (gqa_ratio > kMaxGroup) return TQ_ERR_UNSUPPORTED;
+  if (batch > kMaxGridYZ || n_q_heads / gqa_ratio > kMaxGridYZ) return TQ_ERR_UNSUPPORTED;
+  if (q_dtype < TQ_F16 || q_dtype > TQ_F32) return TQ_ERR_INVALID_ARG;
+  if (!bits_ok(bits_k) || (with_sketch != 0 && with_sketch != 1)) return TQ_ERR_INVALID_ARG;
+  const int hd = check_head_dim(d);
+  if (hd != TQ_OK) return hd;
+  if (!q || !packed_k || !norms_k || !ctx_lens || !scores) return TQ_ERR_INVALID_ARG;
+  if (with_sketch && (!sketch || !gamma || !projection)) return TQ_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(packed_k) || !aligned16(projection) ||
+      ((uintptr_t)sketch & 7u) || ((uintptr_t)norms_k & 1u) || ((uintptr_t)gamma & 1u) ||
+      ((uintptr_t)ctx_lens & 3u) || ((uintptr_t)scores & 3u) || ((uintptr_t)dev_status & 3u))
+    return TQ_ERR_INVALID_ARG;
+  const Codebook* cb = codebook_for(bits_k);
+  if (!cb) return TQ_ERR_NO_CONVERGENCE;
+  QjlScoresArgs a;
+  a.q = q;
+  a.q_dtype = q_dtype;
+  a.packed_k = packed_k;
+  a.norms_k = norms_k;
+  a.sketch = sketch;
+  a.gamma = gamma;
+  a.S = projection;
+  a.ctx_lens = ctx_lens;
+  a.d = d;
+  a.batch = batch;
+  a.n_q_heads = n_q_heads;
+  a.gqa = gqa_ratio;
+  a.n_kv_heads = n_q_heads / gqa_ratio;
+  a.bits_k = bits_k;
+  a.cap_tok = cap_tok;
+  a.with_sketch = with_sketch;
+  a.dev_status = dev_status;
+  a.out = scores;
+  return from_cuda(launch_qjl_scores(a, *cb, sign_mask(seed), (cudaStream_t)stream));
+}
+
 }  // extern "C"

@@ -43,27 +43,13 @@ __device__ __forceinline__ void load_signed(const uint16_t* src, int sub, bool b
   }
 }
 
-template <int BITS, int LPV>
-__device__ __forceinline__ void encode_vector(
-    float (&x)[32], const Codebook& cb, int sub, unsigned gmask,
-    uint8_t* row_dst, uint16_t* norm_dst, int* dev_status) {
-  constexpr int kHalf = 1 << (BITS - 1);
-  // ||x||^2 over the group of LPV lanes (pairs of coordinates per fma)
-  float2 ss2 = make_float2(0.f, 0.f);
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const float2 v = make_float2(x[2 * j], x[2 * j + 1]);
-    ss2 = f2fma(v, v, ss2);
-  }
-  float ss = ss2.x + ss2.y;
-#pragma unroll
-  for (int o = 1; o < LPV; o <<= 1) ss += __shfl_xor_sync(gmask, ss, o);
-  const float n = sqrtf(ss);
-
-  // z = H·(D⊙x): coordinate 32·sub + i lives in register i of lane sub.
-  // Stride 1 in scalar form, strides 2..16 on register pairs, strides
-  // 32 .. 16·LPV across the lanes (x' = partner + sign·x, sign = -1 on the
-  // upper lane); every step rounds exactly like a scalar add or subtract.
+// z = H·(D⊙x) in place for the vector held by a group of LPV lanes:
+// coordinate 32·sub + i lives in register i of lane sub.
+// Stride 1 in scalar form, strides 2..16 on register pairs, strides
+// 32 .. 16·LPV across the lanes (x' = partner + sign·x, sign = -1 on the
+// upper lane); every step rounds exactly like a scalar add or subtract.
+template <int LPV>
+__device__ __forceinline__ void rotate_vector(float (&x)[32], int sub, unsigned gmask) {
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const float u = x[2 * j], v = x[2 * j + 1];
@@ -95,6 +81,26 @@ __device__ __forceinline__ void encode_vector(
       x[2 * j + 1] = r.y;
     }
   }
+}
+
+template <int BITS, int LPV>
+__device__ __forceinline__ void encode_vector(
+    float (&x)[32], const Codebook& cb, int sub, unsigned gmask,
+    uint8_t* row_dst, uint16_t* norm_dst, int* dev_status) {
+  constexpr int kHalf = 1 << (BITS - 1);
+  // ||x||^2 over the group of LPV lanes (pairs of coordinates per fma)
+  float2 ss2 = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const float2 v = make_float2(x[2 * j], x[2 * j + 1]);
+    ss2 = f2fma(v, v, ss2);
+  }
+  float ss = ss2.x + ss2.y;
+#pragma unroll
+  for (int o = 1; o < LPV; o <<= 1) ss += __shfl_xor_sync(gmask, ss, o);
+  const float n = sqrtf(ss);
+
+  rotate_vector<LPV>(x, sub, gmask);
 
   // idx = #{j : z/n >= t_j} over the symmetric table (t_{half-1} = 0), on
   // the FMA pipe. With a = |z| and the positive thresholds t_k (k = 1 ..

@@ -128,6 +128,39 @@ struct CombineArgs {
 };
 cudaError_t launch_combine(const CombineArgs& a, const SignMask& sm, cudaStream_t stream);
 
+// Stage-2 residual sketch of keys (one kv head block per grid row).
+struct QjlEncodeArgs {
+  const uint16_t* k;         // [n_tok][n_kv_heads][d] fp16/bf16 keys
+  int is_bf16;
+  int d, n_tok, n_kv_heads, bits_k;
+  const uint8_t* packed_k;   // stage-1 rows [n_kv_heads][cap_tok][d*bits_k/8] (read)
+  const uint16_t* norms_k;   // [n_kv_heads][cap_tok]
+  const float* S;            // [d][d] projection, row i = projection i
+  uint8_t* sketch;           // [n_kv_heads][cap_tok][d/8]
+  uint16_t* gamma;           // [n_kv_heads][cap_tok] fp16 residual norms
+  int cap_tok, tok_offset;
+  int* dev_status;
+};
+cudaError_t launch_qjl_encode(const QjlEncodeArgs& a, const Codebook& cb, const SignMask& sm,
+                              cudaStream_t stream);
+
+struct QjlScoresArgs {
+  const void* q;             // [batch][n_q_heads][d]
+  int q_dtype;
+  const uint8_t* packed_k;   // [batch][n_kv_heads][cap_tok][d*bits_k/8]
+  const uint16_t* norms_k;
+  const uint8_t* sketch;     // [batch][n_kv_heads][cap_tok][d/8]
+  const uint16_t* gamma;
+  const float* S;            // [d][d]
+  const int32_t* ctx_lens;
+  int d, batch, n_q_heads, gqa, n_kv_heads, bits_k, cap_tok;
+  int with_sketch;
+  int* dev_status;
+  float* out;                // [batch][n_q_heads][cap_tok]
+};
+cudaError_t launch_qjl_scores(const QjlScoresArgs& a, const Codebook& cb, const SignMask& sm,
+                              cudaStream_t stream);
+
 // Workspace of tq_attend: a counter region (zero on first use; every call
 // leaves it zero) followed by partial-result slots. Sized for up to
 // kMaxCtas CTAs, independent of the device.

@@ -71,7 +71,7 @@
 extern "C" {
 #endif
 
-#define TQ_ABI_VERSION 4
+#define TQ_ABI_VERSION 5
 
 /* Tokens per sparse-V block; split boundaries are multiples of this. */
 #define TQ_SPARSE_V_BLOCK 64
@@ -353,6 +353,68 @@ int tq_attend_partial(const void* q, int q_dtype,
 int tq_attend_combine(const float* partials, int n_parts, int batch, int n_q_heads,
                       int d, uint64_t seed, int* dev_status, void* out, int out_dtype,
                       void* stream);
+
+/*
+ * Stage-2 residual sketch (QJL) and the unbiased inner-product estimate.
+ * "We Built a Python Library That Cuts LLM Memory Usage by 80%", section
+ * "Why not both stages?": the method has a second stage, a one-bit
+ * correction of the stage-1 residual that makes inner products unbiased;
+ * that page leaves it out of softmax attention because its variance hurts
+ * there. The library therefore offers it for keys, as a score estimate, not
+ * inside tq_attend. The page gives nothing more; the library's definition:
+ *   r~    = R·x - nK·c[idx]/sqrt(d)   the key's stage-1 residual in rotated
+ *                                      coordinates (= R·(x - x_hat)),
+ *                                      R = H·diag(D)/sqrt(d), nK the stored
+ *                                      fp16 norm, c the N(0,1) codebook
+ *   S     d x d, i.i.d. N(0,1), supplied by the caller (one per model or
+ *         layer; the same S for encode and scores)
+ *   bit_i = 1 iff (S·r~)_i >= 0, i = 0..d-1, LSB-first, d/8 bytes per row
+ *   gamma = ||r~||, fp16 round-to-nearest-even, saturated at 65504
+ *   estimate <q, x> ~ <q~, nK·c[idx]/sqrt(d)> + gamma·sqrt(pi/2)/d·<S·q~, 2·bit - 1>
+ * with q~ = R·q. For s ~ N(0, I), E[sign(s·r)(s·q)] = sqrt(2/pi)·<q, r>/|r|,
+ * so the correction is unbiased for <q, x - x_hat> over the draw of S (up
+ * to the fp16 rounding of gamma).
+ *
+ * tq_qjl_encode — sketch rows of n_tok keys of one sequence.
+ *   k           [n_tok][n_kv_heads][d] fp16/bf16 keys (dtype), 16-byte aligned.
+ *   projection  float [d][d], row i = projection vector i, 16-byte aligned.
+ *   packed_k, norms_k  the keys' stage-1 cache (tq_encode's output for the
+ *               same keys, seed and bits_k), rows tok_offset .. + n_tok - 1
+ *               are read; packed_k 16-byte aligned.
+ *   sketch      uint8 [n_kv_heads][cap_tok][d/8], rows tok_offset .. written.
+ *   gamma       fp16 bits [n_kv_heads][cap_tok], same rows written.
+ *   Other arguments as for tq_encode (bits_k 2..4); TQ_DEV_NORM_SATURATED
+ *   reports a gamma above 65504.
+ */
+int tq_qjl_encode(const void* k, int dtype, int n_tok, int n_kv_heads, int d, int bits_k,
+                  uint64_t seed, const float* projection, const uint8_t* packed_k,
+                  const uint16_t* norms_k, uint8_t* sketch, uint16_t* gamma, int cap_tok,
+                  int tok_offset, int* dev_status, void* stream);
+
+/*
+ * tq_qjl_scores — estimated attention scores estimate/sqrt(d) of every query
+ * head against the first L_b = min(ctx_lens[b], cap_tok) cached keys:
+ *   scores[b][h][t] = (<q~, nK_t·c[idx_t]/sqrt(d)>
+ *                      + with_sketch·gamma_t·sqrt(pi/2)/d·<S·q~, 2·bit_t - 1>) / sqrt(d)
+ * for t < L_b; entries t >= L_b are not written.
+ *   q           [batch][n_q_heads][d] of q_dtype (TQ_F16 | TQ_BF16 | TQ_F32),
+ *               16-byte aligned; kv head of query head h is h / gqa_ratio.
+ *   packed_k, norms_k  stage-1 key cache [batch][n_kv_heads][cap_tok][...],
+ *               packed_k 16-byte aligned.
+ *   sketch, gamma  tq_qjl_encode's rows [batch][n_kv_heads][cap_tok][...],
+ *               sketch 8-byte aligned; unused (may be NULL) when with_sketch = 0.
+ *   projection  the S given to tq_qjl_encode; may be NULL when with_sketch = 0.
+ *   with_sketch 1: the unbiased estimate; 0: the stage-1 score only.
+ *   scores      float [batch][n_q_heads][cap_tok].
+ *   ctx_lens, batch, n_q_heads, gqa_ratio (1..8), d, bits_k, seed, cap_tok,
+ *   dev_status  as for tq_attend (ctx > cap_tok clamped with
+ *               TQ_DEV_CTX_CLAMPED; ctx <= 0 writes nothing, TQ_DEV_CTX_EMPTY).
+ */
+int tq_qjl_scores(const void* q, int q_dtype, const uint8_t* packed_k, const uint16_t* norms_k,
+                  const uint8_t* sketch, const uint16_t* gamma, const float* projection,
+                  const int32_t* ctx_lens, int batch, int n_q_heads, int gqa_ratio, int d,
+                  int bits_k, uint64_t seed, int cap_tok, int with_sketch, int* dev_status,
+                  float* scores, void* stream);
 
 /*
  * tq_attend_noalloc — tq_attend for callers that cannot allocate device

@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_status_strings():
-    assert tq.tq_abi_version() == 4
+    assert tq.tq_abi_version() == 5
     assert tq.status_string(0) == "TQ_OK"
     assert tq.status_string(2) == "TQ_ERR_UNSUPPORTED"
 
