@@ -19,6 +19,8 @@ and the 126 MB L2 cannot hold them. Steps are CUDA-graph replays.
           input): Mtok/s (model tokens/s and token-head vectors/s)
   prefill causal attention of a 1024-token chunk over an 8192-token
           compressed context (tensor cores): TFLOP/s
+  qjl     the stage-2 residual sketch of the keys (tq_qjl_encode) and the
+          estimated scores of 32 query heads (tq_qjl_scores), 8 layer caches
   context_parallel  the same attention split into 4 slices of the context,
           emulated on one GPU: 4 tq_attend_partial launches + tq_attend_combine
           per layer, against the one-pass launch
@@ -56,6 +58,8 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 CP_SLICES = 4            # context-parallel measurement: slices per sequence
+QJL_LAYERS = 8           # residual-sketch measurement: distinct layer caches
+FP32_FMA_TFLOPS = 74.45  # 148 SMs x 128 FMA/clock x 2 FLOP x 1.965 GHz (nominal)
 PREFILL_CTX = 8192       # prefill measurement: context length after the chunk
 PREFILL_TOKENS = 1024    # tokens in the chunk
 
@@ -288,6 +292,59 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize()
     enc_ms = reduce_max(e0.elapsed_time(e1) / enc_steps, device)
     enc_launches = enc_steps * L
+
+    # ---------------- stage-2 residual sketch (QJL) of the keys of QJL_LAYERS
+    # layer caches, and the estimated scores of 32 query heads over them
+    QL = min(QJL_LAYERS, L)
+    proj = torch.from_numpy(S.projection_matrix(d)).to(device)
+    qsk = [torch.empty((1, H, cap, d // 8), dtype=torch.uint8, device=device) for _ in range(QL)]
+    qgm = [torch.empty((1, H, cap), dtype=torch.int16, device=device) for _ in range(QL)]
+    qq = [torch.randn((1, w.n_q_heads, d), generator=gen, device=device).half() for _ in range(QL)]
+    qsc = [torch.empty((1, w.n_q_heads, cap), dtype=torch.float32, device=device) for _ in range(QL)]
+    qctx = torch.full((1,), ctx, dtype=torch.int32, device=device)
+
+    def qjl_encode_all():
+        for l in range(QL):
+            tq.tq_qjl_encode(kv_all[l][0], tq.TQ_F16, ctx, H, d, w.bits_k, seed, proj,
+                             caches.pk[l], caches.nk[l], qsk[l], qgm[l], cap, 0, status, stream)
+
+    def qjl_scores_all():
+        for l in range(QL):
+            tq.tq_qjl_scores(qq[l], tq.TQ_F16, caches.pk[l], caches.nk[l], qsk[l], qgm[l], proj,
+                             qctx, 1, w.n_q_heads, w.gqa, d, w.bits_k, seed, cap, 1, qsc[l],
+                             dev_status=status, stream=stream)
+
+    qjl_ms = {}
+    for name, fn in (("encode", qjl_encode_all), ("scores", qjl_scores_all)):
+        with torch.cuda.stream(stream):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        for _ in range(max(3, args.warmup)):
+            g.replay()
+        torch.cuda.synchronize()
+        q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        qsteps = max(3, min(args.steps, 10))
+        barrier(device)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            q0.record(stream)
+            for _ in range(qsteps):
+                g.replay()
+            q1.record(stream)
+        torch.cuda.synchronize()
+        qjl_ms[name] = reduce_max(q0.elapsed_time(q1) / (qsteps * QL), device)
+        launches += qsteps * QL
+        del g
+    n_keys = ctx * H
+    qjl_enc_flops = n_keys * 2 * d * d
+    qjl_enc_bytes = n_keys * (2 * d + d * w.bits_k // 8 + 2 + d // 8 + 2)
+    qjl_sc_flops = ctx * w.n_q_heads * 4 * d
+    qjl_sc_bytes = n_keys * (d * w.bits_k // 8 + 2 + d // 8 + 2) + ctx * w.n_q_heads * 4 + \
+        w.n_q_heads * d * 2
+    del qsk, qgm, qq, qsc
     del kv_all
     torch.cuda.empty_cache()
 
@@ -563,6 +620,28 @@ def run_gpu(args, rank, world, local_rank):
                                  "peak_kind": "measured dense bf16 (fp16 mma runs at the same rate)",
                                  "flops_per_call": pf_flops},
                     "gpu_launches": pf_steps * pf_layers},
+        "qjl": {
+            "workload": f"{WORKLOAD} keys: {H} kv heads x {ctx} positions, K{w.bits_k}, d={d}; "
+                        f"scores of {w.n_q_heads} query heads; {QL} distinct layer caches",
+            "encode": {"us_per_layer": round(qjl_ms["encode"] * 1e3, 2),
+                       "mkeys_per_s": round(n_keys / (qjl_ms["encode"] * 1e-3) / 1e6, 1),
+                       "gbs": round(qjl_enc_bytes / (qjl_ms["encode"] * 1e-3) / 1e9, 1),
+                       "roofline": {"bound": "tensor",
+                                    "achieved": round(qjl_enc_flops / (qjl_ms["encode"] * 1e-3) / 1e12, 2),
+                                    "peak": measured_tensor_peak(), "unit": "TFLOP/s",
+                                    "frac": round(qjl_enc_flops / (qjl_ms["encode"] * 1e-3) / 1e12 / measured_tensor_peak(), 4),
+                                    "peak_kind": "measured dense bf16 (fp16 mma runs at the same rate)",
+                                    "flops_per_layer": qjl_enc_flops,
+                                    "mma_flops_per_layer": 3 * qjl_enc_flops}},
+            "scores": {"us_per_layer": round(qjl_ms["scores"] * 1e3, 2),
+                       "gbs": round(qjl_sc_bytes / (qjl_ms["scores"] * 1e-3) / 1e9, 1),
+                       "bytes_per_layer": qjl_sc_bytes,
+                       "roofline": {"bound": "fp32 fma",
+                                    "achieved": round(qjl_sc_flops / (qjl_ms["scores"] * 1e-3) / 1e12, 2),
+                                    "peak": FP32_FMA_TFLOPS, "unit": "TFLOP/s",
+                                    "frac": round(qjl_sc_flops / (qjl_ms["scores"] * 1e-3) / 1e12 / FP32_FMA_TFLOPS, 4),
+                                    "hbm_frac": round(qjl_sc_bytes / (qjl_ms["scores"] * 1e-3) / 1e9 / peak, 4),
+                                    "flops_per_layer": qjl_sc_flops}}},
         "context_parallel": {
             "slices": P, "emulated_on_one_gpu": True,
             "per_layer": f"{P} x tq_attend_partial over {ctx // P}-position slices + "

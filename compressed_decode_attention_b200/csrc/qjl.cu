@@ -12,12 +12,13 @@
 //
 // tq_qjl_encode (qjl_encode_kernel): a CTA takes 64 tokens of one kv head.
 //   1. d/32 lanes per key rebuild z = H·(D⊙x) in registers (the encoder's
-//      rotation), read the key's stage-1 row and norm, and leave
-//      r~·sqrt(d) = z - nK·c[idx] in shared memory with gamma.
-//   2. S·r~ as a 64 x d x d fp32 product on the FMA pipe: S is staged 32
-//      columns at a time (transposed) in shared memory; a thread owns 8
-//      consecutive outputs of 64·8/d tokens, so its 8 sign bits form one
-//      byte of each of its tokens' rows.
+//      rotation), read the key's stage-1 row and norm, and leave the
+//      residual z - nK·c[idx], scaled to unit length, in shared memory as
+//      fp16 high/low parts, with gamma.
+//   2. S·r~ on tensor cores (mma.sync m16n8k16, fp32 accumulate) as
+//      Ahi·Bhi + Ahi·Blo + Alo·Bhi (~22 significant bits); S staged 64
+//      columns at a time as fp16 high/low [output][column] tiles. Warp
+//      ballots of the accumulator signs give the row bytes.
 // tq_qjl_scores (qjl_scores_kernel): a CTA takes up to 1024 positions of one
 //   (sequence, kv head). Its prologue rotates the GQA group's queries and
 //   forms p = S·q~ (one warp per output row of S, coalesced); then every
@@ -34,15 +35,67 @@ constexpr int kQjlThreads = 256;
 constexpr int kScorePositions = 1024; // positions per scores CTA
 
 // ------------------------------------------------------------------ encode
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void ldsm4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                        uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, "
+      "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// fp16 high part and the fp16 rounding of the remainder: hi + lo carries
+// about 22 significant bits of x
+__device__ __forceinline__ void split_f16(float x, __half& hi, __half& lo) {
+  hi = __float2half_rn(x);
+  lo = __float2half_rn(x - __half2float(hi));
+}
+// bit 2i of the result = bit i of the 4-bit x
+__device__ __forceinline__ uint32_t spread4(uint32_t x) {
+  return (x & 1u) | ((x & 2u) << 1) | ((x & 4u) << 2) | ((x & 8u) << 3);
+}
+
 template <int D>
 struct QjlEncGeo {
-  static constexpr int RS = D + 4;                 // residual row stride (floats)
-  static constexpr int JC = 32;                    // S columns per staged chunk
-  static constexpr int NO = D / 8;                 // threads across outputs
-  static constexpr int NT = kQjlThreads / NO;      // threads across tokens
-  static constexpr int TPT = kQjlTokens / NT;      // tokens per thread
-  static constexpr size_t SMEM = (size_t)(kQjlTokens * RS + JC * D) * sizeof(float);
+  // S is staged 64 columns at a time for every 64-token unit (72 KB of
+  // shared memory at d = 128: three CTAs per SM). Keeping all of S resident
+  // in a persistent CTA (104 KB, two CTAs per SM) measured slower: the
+  // kernel is latency-bound and gains more from the extra warps.
+  static constexpr int AS = D + 8;                 // A row stride (halves): 16 B pad
+  static constexpr int KC = D < 64 ? D : 64;       // S columns per staged chunk
+  static constexpr int BS = KC + 8;                // S chunk row stride (halves)
+  static constexpr int NT8 = D / 16;               // n-tiles of 8 outputs per warp
+  static constexpr size_t A_BYTES = (size_t)kQjlTokens * AS * 2;
+  static constexpr size_t B_BYTES = (size_t)D * BS * 2;
+  static constexpr size_t SMEM = 2 * A_BYTES + 2 * B_BYTES;
+  static_assert(D % KC == 0, "chunking");
 };
+
+// S[:, kc .. kc + KC) as fp16 high/low parts into [output][column] tiles.
+template <int D, int KC, int BS>
+__device__ __forceinline__ void stage_projection(const float* S, int kc, __half* bhi,
+                                                 __half* blo, int tid) {
+  for (int e = tid; e < D * KC / 4; e += kQjlThreads) {
+    const int o = e / (KC / 4), q4 = e % (KC / 4);
+    const float4 s4 = __ldg(reinterpret_cast<const float4*>(S + (size_t)o * D + kc) + q4);
+    __half hx, lx, hy, ly, hz, lz, hw, lw;
+    split_f16(s4.x, hx, lx);
+    split_f16(s4.y, hy, ly);
+    split_f16(s4.z, hz, lz);
+    split_f16(s4.w, hw, lw);
+    __half2* ph = reinterpret_cast<__half2*>(bhi + o * BS + 4 * q4);
+    __half2* pl = reinterpret_cast<__half2*>(blo + o * BS + 4 * q4);
+    ph[0] = __halves2half2(hx, hy);
+    ph[1] = __halves2half2(hz, hw);
+    pl[0] = __halves2half2(lx, ly);
+    pl[1] = __halves2half2(lz, lw);
+  }
+}
 
 template <int D, int BITS>
 __global__ void __launch_bounds__(kQjlThreads)
@@ -51,18 +104,22 @@ qjl_encode_kernel(const __grid_constant__ QjlEncodeArgs a,
                   const __grid_constant__ SignMask sm) {
   using G = QjlEncGeo<D>;
   constexpr int LPV = D / 32;
-  extern __shared__ __align__(16) float qsm[];
-  float* rs = qsm;                                  // [64][RS] residual · sqrt(d)
-  float* st = qsm + kQjlTokens * G::RS;             // [JC][D] chunk of S^T
-  const int tid = threadIdx.x, lane = tid & 31;
+  constexpr int KC = G::KC;
+  extern __shared__ __align__(128) uint8_t qsm[];
+  __half* ahi = reinterpret_cast<__half*>(qsm);                       // [64][AS]
+  __half* alo = reinterpret_cast<__half*>(qsm + G::A_BYTES);
+  __half* bhi = reinterpret_cast<__half*>(qsm + 2 * G::A_BYTES);      // [D][BS]
+  __half* blo = reinterpret_cast<__half*>(qsm + 2 * G::A_BYTES + G::B_BYTES);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   const int h = blockIdx.y;
   const int tok0 = blockIdx.x * kQjlTokens;
   const int ntok = min(kQjlTokens, a.n_tok - tok0);
 
-  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-  asm volatile("griddepcontrol.wait;\n" ::: "memory");
-
-  // ---- 1. residual of each key in rotated coordinates (times sqrt(d))
+  // ---- 1. residual of each key in rotated coordinates, scaled to unit
+  // length (the signs of S·r~ do not change), as fp16 high/low parts
   {
     const int sub = lane & (LPV - 1);
     const unsigned gmask = ((1u << LPV) - 1u) << (lane & ~(LPV - 1));
@@ -70,10 +127,11 @@ qjl_encode_kernel(const __grid_constant__ QjlEncodeArgs a,
     sign_masks(sm, sub, smask);
     constexpr int rowb = D * BITS / 8;
     for (int v = tid / LPV; v < kQjlTokens; v += kQjlThreads / LPV) {
-      float* dst = rs + v * G::RS + 32 * sub;
+      __half* dh = ahi + v * G::AS + 32 * sub;
+      __half* dl = alo + v * G::AS + 32 * sub;
       if (v >= ntok) {                              // rows past the end: zero
 #pragma unroll
-        for (int i = 0; i < 32; ++i) dst[i] = 0.f;
+        for (int i = 0; i < 32; ++i) dh[i] = dl[i] = __float2half_rn(0.f);
         continue;
       }
       const int tok = tok0 + v;
@@ -90,12 +148,20 @@ qjl_encode_kernel(const __grid_constant__ QjlEncodeArgs a,
       float ss = 0.f;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float r = fmaf(-nk, cb.centroid[field<BITS>(w, i)], x[i]);
-        dst[i] = r;
-        ss = fmaf(r, r, ss);
+        x[i] = fmaf(-nk, cb.centroid[field<BITS>(w, i)], x[i]);   // r~·sqrt(d)
+        ss = fmaf(x[i], x[i], ss);
       }
 #pragma unroll
       for (int o = 1; o < LPV; o <<= 1) ss += __shfl_xor_sync(gmask, ss, o);
+      const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        __half h0, l0, h1, l1;
+        split_f16(x[i] * inv, h0, l0);
+        split_f16(x[i + 1] * inv, h1, l1);
+        *reinterpret_cast<__half2*>(dh + i) = __halves2half2(h0, h1);
+        *reinterpret_cast<__half2*>(dl + i) = __halves2half2(l0, l1);
+      }
       if (sub == 0) {
         // ||r~|| = ||z - nK·c|| / sqrt(d)
         const float gmm = sqrtf(ss) * rsqrtf((float)D);
@@ -105,53 +171,68 @@ qjl_encode_kernel(const __grid_constant__ QjlEncodeArgs a,
     }
   }
 
-  // ---- 2. u = S·r~ (the sign of r~·sqrt(d) is that of r~)
-  const int oo = tid % G::NO, tt = tid / G::NO;
-  float acc[G::TPT][8];
+  // ---- 2. u = S·r~ on tensor cores: warp (mt, nh) takes tokens 16·mt ..
+  // and outputs nh·d/2 .. ; S is staged KC columns at a time as fp16
+  // high/low [output][column]; u = Ahi·Bhi + Ahi·Blo + Alo·Bhi in fp32
+  const int mt = warp & 3, nh = warp >> 2;
+  float acc[G::NT8][4];
 #pragma unroll
-  for (int t = 0; t < G::TPT; ++t)
+  for (int n = 0; n < G::NT8; ++n)
 #pragma unroll
-    for (int k = 0; k < 8; ++k) acc[t][k] = 0.f;
-  for (int j0 = 0; j0 < D; j0 += G::JC) {
-    __syncthreads();                                // residuals ready / chunk free
-    // st[jj][o] = S[o][j0 + jj]: each thread copies float4 runs of rows of S
-    for (int e = tid; e < D * G::JC / 4; e += kQjlThreads) {
-      const int o = e / (G::JC / 4), jq = e % (G::JC / 4);
-      const float4 s4 = __ldg(reinterpret_cast<const float4*>(a.S + (size_t)o * D + j0) + jq);
-      st[(4 * jq + 0) * D + o] = s4.x;
-      st[(4 * jq + 1) * D + o] = s4.y;
-      st[(4 * jq + 2) * D + o] = s4.z;
-      st[(4 * jq + 3) * D + o] = s4.w;
-    }
+    for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
+  // ldmatrix lane addresses: A rows 16·mt + (lane & 15), column +8 for
+  // lanes 16..31; B rows (outputs) n0 + (lane & 7) + 8·(lane >> 4), column
+  // +8 for lanes 8..15 and 24..31
+  const uint32_t a_hi = smem_u32(ahi + (16 * mt + (lane & 15)) * G::AS + ((lane >> 4) << 3));
+  const uint32_t a_lo = smem_u32(alo + (16 * mt + (lane & 15)) * G::AS + ((lane >> 4) << 3));
+  const int brow = nh * (D / 2) + (lane & 7) + ((lane >> 4) << 3);
+  const uint32_t b_hi = smem_u32(bhi + brow * G::BS + (((lane >> 3) & 1) << 3));
+  const uint32_t b_lo = smem_u32(blo + brow * G::BS + (((lane >> 3) & 1) << 3));
+  for (int kc = 0; kc < D; kc += KC) {
+    __syncthreads();                                // A ready / previous chunk used
+    stage_projection<D, KC, G::BS>(a.S, kc, bhi, blo, tid);
     __syncthreads();
-#pragma unroll 4
-    for (int jj = 0; jj < G::JC; ++jj) {
-      const float4 b0 = *reinterpret_cast<const float4*>(st + jj * D + 8 * oo);
-      const float4 b1 = *reinterpret_cast<const float4*>(st + jj * D + 8 * oo + 4);
 #pragma unroll
-      for (int t = 0; t < G::TPT; ++t) {
-        const float r = rs[(tt * G::TPT + t) * G::RS + j0 + jj];
-        acc[t][0] = fmaf(r, b0.x, acc[t][0]);
-        acc[t][1] = fmaf(r, b0.y, acc[t][1]);
-        acc[t][2] = fmaf(r, b0.z, acc[t][2]);
-        acc[t][3] = fmaf(r, b0.w, acc[t][3]);
-        acc[t][4] = fmaf(r, b1.x, acc[t][4]);
-        acc[t][5] = fmaf(r, b1.y, acc[t][5]);
-        acc[t][6] = fmaf(r, b1.z, acc[t][6]);
-        acc[t][7] = fmaf(r, b1.w, acc[t][7]);
+    for (int kk = 0; kk < KC / 16; ++kk) {
+      uint32_t ah[4], al[4];
+      ldsm4(a_hi + 2 * (kc + 16 * kk), ah);
+      ldsm4(a_lo + 2 * (kc + 16 * kk), al);
+#pragma unroll
+      for (int n2 = 0; n2 < G::NT8 / 2; ++n2) {
+        uint32_t bh[4], bl[4];
+        const uint32_t off = 2 * (16 * n2 * G::BS + 16 * kk);
+        ldsm4(b_hi + off, bh);
+        ldsm4(b_lo + off, bl);
+        mma_f16(acc[2 * n2], ah, bh[0], bh[1]);
+        mma_f16(acc[2 * n2], ah, bl[0], bl[1]);
+        mma_f16(acc[2 * n2], al, bh[0], bh[1]);
+        mma_f16(acc[2 * n2 + 1], ah, bh[2], bh[3]);
+        mma_f16(acc[2 * n2 + 1], ah, bl[2], bl[3]);
+        mma_f16(acc[2 * n2 + 1], al, bh[2], bh[3]);
       }
     }
   }
-  // one byte (8 sign bits, LSB first) of each of this thread's tokens
+
+  // ---- 3. sign bits: accumulator (n-tile n, element e) of lane (g, t) is
+  // token 16·mt + g + 8·(e >> 1), output 8·n + 2t + (e & 1) of the warp's
+  // half. Ballots collect the 8 outputs of each n-tile; lane (g, t = 0)
+  // writes token g's byte and lane (g, t = 1) token g + 8's.
+  const int gq = lane >> 2, tq = lane & 3;
 #pragma unroll
-  for (int t = 0; t < G::TPT; ++t) {
-    const int v = tt * G::TPT + t;
-    if (v >= ntok) continue;
-    uint32_t byte = 0;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) byte |= (acc[t][k] >= 0.f ? 1u : 0u) << k;
-    const size_t row = (size_t)h * a.cap_tok + a.tok_offset + tok0 + v;
-    a.sketch[row * (D / 8) + oo] = (uint8_t)byte;
+  for (int n = 0; n < G::NT8; ++n) {
+    const uint32_t m0 = __ballot_sync(0xFFFFFFFFu, acc[n][0] >= 0.f);
+    const uint32_t m1 = __ballot_sync(0xFFFFFFFFu, acc[n][1] >= 0.f);
+    const uint32_t m2 = __ballot_sync(0xFFFFFFFFu, acc[n][2] >= 0.f);
+    const uint32_t m3 = __ballot_sync(0xFFFFFFFFu, acc[n][3] >= 0.f);
+    if (tq < 2) {
+      const uint32_t e0 = tq ? m2 : m0, e1 = tq ? m3 : m1;
+      const uint32_t byte = spread4((e0 >> (4 * gq)) & 15u) | (spread4((e1 >> (4 * gq)) & 15u) << 1);
+      const int v = 16 * mt + gq + 8 * tq;
+      if (v < ntok) {
+        const size_t row = (size_t)h * a.cap_tok + a.tok_offset + tok0 + v;
+        a.sketch[row * (D / 8) + nh * (D / 16) + n] = (uint8_t)byte;
+      }
+    }
   }
 }
 

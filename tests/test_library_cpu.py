@@ -188,3 +188,53 @@ def _partial(**kw):
 ])
 def test_partial_validation(kw, want):
     assert _partial(**kw) == want
+
+
+def _qjl_encode(**kw):
+    a = dict(k=FAKE, dtype=tq.TQ_F16, n=4, H=2, d=128, bits=4, S=FAKE, pk=FAKE, nk=FAKE,
+             sk=FAKE, g=FAKE, cap=8, off=0)
+    a.update(kw)
+    return tq.lib().tq_qjl_encode(a["k"], a["dtype"], a["n"], a["H"], a["d"], a["bits"], 0,
+                                  a["S"], a["pk"], a["nk"], a["sk"], a["g"], a["cap"],
+                                  a["off"], None, 0)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(S=None), tq.TQ_ERR_INVALID_ARG),
+    (dict(sk=None), tq.TQ_ERR_INVALID_ARG),
+    (dict(k=FAKE + 2), tq.TQ_ERR_INVALID_ARG),
+    (dict(S=FAKE + 4), tq.TQ_ERR_INVALID_ARG),
+    (dict(bits=5), tq.TQ_ERR_INVALID_ARG),
+    (dict(d=96), tq.TQ_ERR_INVALID_ARG),
+    (dict(dtype=tq.TQ_F32), tq.TQ_ERR_INVALID_ARG),
+    (dict(off=5), tq.TQ_ERR_INVALID_ARG),                 # 5 + 4 > 8
+    (dict(n=0), tq.TQ_OK),                                # no-op, no launch
+])
+def test_qjl_encode_validation(kw, want):
+    assert _qjl_encode(**kw) == want
+
+
+def _qjl_scores(**kw):
+    a = dict(q=FAKE, pk=FAKE, sk=FAKE, g=FAKE, S=FAKE, ctx=FAKE, B=2, hq=8, gqa=4, d=128,
+             bits=4, cap=256, with_sketch=1, out=FAKE)
+    a.update(kw)
+    return tq.lib().tq_qjl_scores(a["q"], tq.TQ_F16, a["pk"], FAKE, a["sk"], a["g"], a["S"],
+                                  a["ctx"], a["B"], a["hq"], a["gqa"], a["d"], a["bits"], 0,
+                                  a["cap"], a["with_sketch"], None, a["out"], 0)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(S=None), tq.TQ_ERR_INVALID_ARG),                # the sketch term needs S
+    (dict(sk=None), tq.TQ_ERR_INVALID_ARG),
+    (dict(out=None), tq.TQ_ERR_INVALID_ARG),
+    (dict(gqa=3), tq.TQ_ERR_INVALID_ARG),
+    (dict(hq=16, gqa=16), tq.TQ_ERR_UNSUPPORTED),
+    (dict(with_sketch=2), tq.TQ_ERR_INVALID_ARG),
+    (dict(sk=FAKE + 4), tq.TQ_ERR_INVALID_ARG),          # sketch rows need 8-byte alignment
+    (dict(out=FAKE + 2), tq.TQ_ERR_INVALID_ARG),
+    (dict(d=32), tq.TQ_ERR_INVALID_ARG),
+    (dict(bits=1), tq.TQ_ERR_INVALID_ARG),
+    (dict(B=0), tq.TQ_ERR_INVALID_ARG),
+])
+def test_qjl_scores_validation(kw, want):
+    assert _qjl_scores(**kw) == want
