@@ -21,6 +21,8 @@ and the 126 MB L2 cannot hold them. Steps are CUDA-graph replays.
           compressed context (tensor cores): TFLOP/s
   qjl     the stage-2 residual sketch of the keys (tq_qjl_encode) and the
           estimated scores of 32 query heads (tq_qjl_scores), 8 layer caches
+  batched attention at serving scale: 64 sequences of 1024-16384 positions
+          (K4/V3, ~0.5 GB per call)
   context_parallel  the same attention split into 4 slices of the context,
           emulated on one GPU: 4 tq_attend_partial launches + tq_attend_combine
           per layer, against the one-pass launch
@@ -53,6 +55,7 @@ import synthetic as S  # noqa: E402
 METRIC = "decode-attn packed-KV GB/s & % HBM roofline; encode Mtok/s (1×B200)"
 WORKLOAD = "llama3_8b_decode"
 ENCODE_WORKLOAD = "bulk_prefill_encode"
+BATCHED_WORKLOAD = "batched_serving"
 LAYERS = 32
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
@@ -524,6 +527,57 @@ def run_gpu(args, rank, world, local_rank):
         launches += per * L * args.steps
         del g
 
+    # ---------------- attention at serving scale: the batched workload (64
+    # sequences of U{1024..16384} positions, K4/V3, sparse-V gate 1e-6), two
+    # layer caches alternating (2 x 0.97 GB of capacity, > L2). The rows are
+    # random bytes and the norms random values near sqrt(d): timing only.
+    wb = S.WORKLOADS[BATCHED_WORKLOAD]
+    bctx_h = S.ctx_lens(wb)
+    bctx = torch.from_numpy(bctx_h).to(device)
+    bH, bcap, bHq = wb.n_kv_heads, wb.cap_tok, wb.n_q_heads
+    brk, brv = d * wb.bits_k // 8, d * wb.bits_v // 8
+    bcache = []
+    for _ in range(2):
+        bpk = torch.randint(0, 256, (wb.batch, bH, bcap, brk), dtype=torch.uint8, device=device,
+                            generator=gen)
+        bpv = torch.randint(0, 256, (wb.batch, bH, bcap, brv), dtype=torch.uint8, device=device,
+                            generator=gen)
+        bnk = (11.3 + torch.randn((wb.batch, bH, bcap), generator=gen, device=device)) \
+            .half().view(torch.int16)
+        bnv = (11.3 + torch.randn((wb.batch, bH, bcap), generator=gen, device=device)) \
+            .half().view(torch.int16)
+        bcache.append((bpk, bnk, bpv, bnv))
+    bq = [torch.randn((wb.batch, bHq, d), generator=gen, device=device).half() for _ in range(2)]
+    bout = torch.empty((wb.batch, bHq, d), dtype=torch.float16, device=device)
+    bws_bytes = tq.tq_attend_workspace_size(wb.batch, bHq, bcap, d)
+    bws = torch.zeros(bws_bytes, dtype=torch.uint8, device=device)
+
+    def batched_all():
+        for i in range(2):
+            bpk, bnk, bpv, bnv = bcache[i]
+            tq.tq_attend(bq[i], tq.TQ_F16, bpk, bnk, bpv, bnv, bctx, wb.batch, bHq, wb.gqa, d,
+                         wb.bits_k, wb.bits_v, seed, bcap, wb.tau, 0, bws, bws_bytes, bout,
+                         tq.TQ_F16, dev_status=status, stream=stream)
+
+    bgraph = capture(batched_all)
+    for _ in range(args.warmup):
+        bgraph.replay()
+    torch.cuda.synchronize()
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(device)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        b0.record(stream)
+        for _ in range(args.steps):
+            bgraph.replay()
+        b1.record(stream)
+    torch.cuda.synchronize()
+    batched_ms = reduce_max(b0.elapsed_time(b1) / (2 * args.steps), device)
+    launches += 2 * args.steps
+    batched_bytes = int(bctx_h.astype(np.int64).sum()) * bH * (brk + brv + 4) + \
+        wb.batch * bHq * d * (2 + 2)
+    del bgraph, bcache, bq, bout, bws
+
     # ---------------- end to end: host inputs in, host output back, every step
     q_host = torch.empty((L, 1, w.n_q_heads, d), dtype=torch.float16).pin_memory()
     kv_host = torch.empty((L, 2, 1, H, d), dtype=torch.int16).pin_memory()
@@ -642,6 +696,16 @@ def run_gpu(args, rank, world, local_rank):
                                     "frac": round(qjl_sc_flops / (qjl_ms["scores"] * 1e-3) / 1e12 / FP32_FMA_TFLOPS, 4),
                                     "hbm_frac": round(qjl_sc_bytes / (qjl_ms["scores"] * 1e-3) / 1e9 / peak, 4),
                                     "flops_per_layer": qjl_sc_flops}}},
+        "batched": {
+            "workload": f"{BATCHED_WORKLOAD}: {wb.batch} sequences, ctx U{{{wb.ctx_range[0]}.."
+                        f"{wb.ctx_range[1]}}}, {bHq} q / {bH} kv heads, d={d}, "
+                        f"K{wb.bits_k}/V{wb.bits_v}, sparse-V gate {wb.tau}; 2 layer caches "
+                        "alternating (rows random bytes: timing only)",
+            "us_per_call": round(batched_ms * 1e3, 2),
+            "bytes_per_call": batched_bytes,
+            "gbs": round(batched_bytes / (batched_ms * 1e-3) / 1e9, 1),
+            "frac": round(batched_bytes / (batched_ms * 1e-3) / 1e9 / peak, 4),
+            "frac_of_nominal_8tbs": round(batched_bytes / (batched_ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 4)},
         "context_parallel": {
             "slices": P, "emulated_on_one_gpu": True,
             "per_layer": f"{P} x tq_attend_partial over {ctx // P}-position slices + "
