@@ -398,9 +398,14 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.empty_cache()
 
     # ---------------- decode step graphs
-    q = [torch.randn((1, w.n_q_heads, d), generator=gen, device=device).half() for _ in range(L)]
-    kv_new = [device_kv(w, l, 1, gen) for l in range(L)]
-    outs = [torch.empty((1, w.n_q_heads, d), dtype=torch.float16, device=device) for _ in range(L)]
+    # per-layer queries, new K/V and outputs are views of three contiguous
+    # buffers, so that the end-to-end step moves each with one copy
+    q_all = torch.randn((L, 1, w.n_q_heads, d), generator=gen, device=device).half()
+    kv_all_new = torch.stack([device_kv(w, l, 1, gen) for l in range(L)])   # [L][2][1][H][d]
+    outs_all = torch.empty((L, 1, w.n_q_heads, d), dtype=torch.float16, device=device)
+    q = [q_all[l] for l in range(L)]
+    kv_new = [kv_all_new[l] for l in range(L)]
+    outs = [outs_all[l] for l in range(L)]
     ctx_dev = torch.full((1,), ctx, dtype=torch.int32, device=device)
     ws_bytes = tq.tq_attend_workspace_size(1, w.n_q_heads, cap, d)
     ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=device)
@@ -582,18 +587,18 @@ def run_gpu(args, rank, world, local_rank):
     q_host = torch.empty((L, 1, w.n_q_heads, d), dtype=torch.float16).pin_memory()
     kv_host = torch.empty((L, 2, 1, H, d), dtype=torch.int16).pin_memory()
     out_host = torch.empty((L, 1, w.n_q_heads, d), dtype=torch.float16).pin_memory()
-    q_host.copy_(torch.stack([x.cpu() for x in q]))
-    kv_host.copy_(torch.stack([x.cpu() for x in kv_new]))
+    q_host.copy_(q_all.cpu())
+    kv_host.copy_(kv_all_new.cpu())
     e2e_graph = capture(step)
     torch.cuda.synchronize()
 
     def e2e_step():
-        for l in range(L):
-            q[l].copy_(q_host[l], non_blocking=True)
-            kv_new[l].copy_(kv_host[l], non_blocking=True)
+        # one host-to-device copy each of every layer's query and new K/V,
+        # the step's launches, one device-to-host copy of every output
+        q_all.copy_(q_host, non_blocking=True)
+        kv_all_new.copy_(kv_host, non_blocking=True)
         e2e_graph.replay()
-        for l in range(L):
-            out_host[l].copy_(outs[l], non_blocking=True)
+        out_host.copy_(outs_all, non_blocking=True)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
