@@ -42,17 +42,23 @@ struct PfGeo {
   static constexpr int VROWS = RV % 16 == 0 ? 1 : 16 / (RV % 16);
   static constexpr int QH = 0;                               // [128 rows][kTS] fp16
   static constexpr int QL = QH + kPfRows * kTS * 2;
+  // two buffers of dequantized chunk tiles: K high, K low, V ([64 positions]
+  // [kTS] fp16 each) and the K / V norms as floats
   static constexpr int KH = QL + kPfRows * kTS * 2;          // [64 positions][kTS]
   static constexpr int KL = KH + kPfChunk * kTS * 2;
   static constexpr int VT = KL + kPfChunk * kTS * 2;
-  static constexpr int STG = VT + kPfChunk * kTS * 2;        // two staging slots
+  static constexpr int NKF = VT + kPfChunk * kTS * 2;        // float [64]
+  static constexpr int NVF = NKF + kPfChunk * 4;             // float [64]
+  static constexpr int TBUF = NVF + kPfChunk * 4 - KH;       // bytes per buffer
+  static constexpr int STG = KH + 2 * TBUF;                  // two staging slots
   static constexpr int SLOT = kPfChunk * (RK + RV) + 2 * kPfChunk * 2;
   static constexpr int LUTK = STG + 2 * SLOT;                // uint2 per pair code
   static constexpr int LUTV = LUTK + (1 << (2 * BK)) * 8;    // uint32 per pair code
   static constexpr int SINV = LUTV + (1 << (2 * BV)) * 4;    // float per row
   static constexpr int MBAR = SINV + kPfRows * 4;
   static constexpr int SMEM = MBAR + 16;
-  static_assert(SLOT % 16 == 0 && STG % 16 == 0 && MBAR % 8 == 0, "alignment");
+  static_assert(SLOT % 16 == 0 && STG % 16 == 0 && TBUF % 16 == 0 && MBAR % 8 == 0,
+                "alignment");
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
@@ -142,6 +148,7 @@ prefill_kernel(const __grid_constant__ PrefillArgs a,
              2 * nrows, bar);
   };
   if (tid == 0 && nchunks > 0) issue(0);
+  if (tid == 0 && nchunks > 1) issue(1);
 
   // ---- rotated queries: warp w rotates its rows 16w .. 16w + 15 one by one
   // (row r = token r / GQ of the tile, head r % GQ of the group)
@@ -219,48 +226,70 @@ prefill_kernel(const __grid_constant__ PrefillArgs a,
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   bool stalled = false;
 
-  for (int c = 0; c < nchunks; ++c) {
-    if (tid == 0 && c + 1 < nchunks) issue(c + 1);  // its slot was drained last round
-    if (!__syncthreads_and(mbar_wait(bar0 + 8 * (c & 1), (uint32_t)(c >> 1) & 1u))) {
-      stalled = true;                                // a copy never completed
-      if (tid == 0 && a.dev_status) atomicOr(a.dev_status, TQ_DEV_WAIT_TIMEOUT);
-      if (tid == 0 && c + 1 < nchunks) mbar_wait(bar0 + 8 * ((c + 1) & 1), (uint32_t)((c + 1) >> 1) & 1u);
-      break;
-    }
-    // ---- dequantize the chunk: thread t -> position t / 4, coordinates
-    // 32·(t % 4) .. + 31
-    {
-      const uint8_t* st = smem + G::STG + (c & 1) * G::SLOT;
-      const int pos = tid >> 2, qd = tid & 3;
-      uint32_t kw[(4 * BK + 3) / 4 + 1], vw[(4 * BV + 3) / 4 + 1];
-      load_chunk<4 * BK>(st, pos * G::RK + 4 * BK * qd, kw);
-      load_chunk<4 * BV>(st, kPfChunk * G::RK + pos * G::RV + 4 * BV * qd, vw);
-      uint32_t hi[16], lo[16], vv[16];
+  // Chunk c: its packed rows arrive in staging slot c & 1 (issued two
+  // chunks ahead), are dequantized into tile buffer c & 1, and are consumed
+  // by the MMAs of the next round. A warp that finishes the MMAs of chunk c
+  // goes on to dequantize chunk c + 1 into the other buffer while the rest
+  // still multiply; one barrier per chunk separates the rounds.
+  auto dequant = [&](int c) {
+    const uint8_t* st = smem + G::STG + (c & 1) * G::SLOT;
+    uint8_t* tb = smem + (c & 1) * G::TBUF;        // buffer c & 1 (add G::KH etc.)
+    const int pos = tid >> 2, qd = tid & 3;
+    uint32_t kw[(4 * BK + 3) / 4 + 1], vw[(4 * BV + 3) / 4 + 1];
+    load_chunk<4 * BK>(st, pos * G::RK + 4 * BK * qd, kw);
+    load_chunk<4 * BV>(st, kPfChunk * G::RK + pos * G::RV + 4 * BV * qd, vw);
+    uint32_t hi[16], lo[16], vv[16];
 #pragma unroll
-      for (int p = 0; p < 16; ++p) {
-        const uint2 e = lds<uint2>(smem, G::LUTK + pair_code_shifted<BK, 3>(kw, p));
-        hi[p] = e.x;
-        lo[p] = e.y;
-        vv[p] = lds<uint32_t>(smem, G::LUTV + pair_code_shifted<BV, 2>(vw, p));
-      }
-      const int off = 2 * (pos * kTS + 32 * qd);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        *reinterpret_cast<uint4*>(smem + G::KH + off + 16 * k) =
-            make_uint4(hi[4 * k], hi[4 * k + 1], hi[4 * k + 2], hi[4 * k + 3]);
-        *reinterpret_cast<uint4*>(smem + G::KL + off + 16 * k) =
-            make_uint4(lo[4 * k], lo[4 * k + 1], lo[4 * k + 2], lo[4 * k + 3]);
-        *reinterpret_cast<uint4*>(smem + G::VT + off + 16 * k) =
-            make_uint4(vv[4 * k], vv[4 * k + 1], vv[4 * k + 2], vv[4 * k + 3]);
-      }
+    for (int p = 0; p < 16; ++p) {
+      const uint2 e = lds<uint2>(smem, G::LUTK + pair_code_shifted<BK, 3>(kw, p));
+      hi[p] = e.x;
+      lo[p] = e.y;
+      vv[p] = lds<uint32_t>(smem, G::LUTV + pair_code_shifted<BV, 2>(vw, p));
     }
-    __syncthreads();
-
+    const int off = 2 * (pos * kTS + 32 * qd);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      *reinterpret_cast<uint4*>(tb + G::KH + off + 16 * k) =
+          make_uint4(hi[4 * k], hi[4 * k + 1], hi[4 * k + 2], hi[4 * k + 3]);
+      *reinterpret_cast<uint4*>(tb + G::KL + off + 16 * k) =
+          make_uint4(lo[4 * k], lo[4 * k + 1], lo[4 * k + 2], lo[4 * k + 3]);
+      *reinterpret_cast<uint4*>(tb + G::VT + off + 16 * k) =
+          make_uint4(vv[4 * k], vv[4 * k + 1], vv[4 * k + 2], vv[4 * k + 3]);
+    }
+    if (qd == 0) {
+      // norms as floats; 0 past the sequence end (the copied norm runs stop
+      // at a multiple of 8 positions: the rest of the slot is stale)
+      const bool live = c * kPfChunk + pos < L;
+      const uint16_t* nsrc = reinterpret_cast<const uint16_t*>(st + kPfChunk * (G::RK + G::RV));
+      reinterpret_cast<float*>(tb + G::NKF)[pos] =
+          live ? __half2float(__ushort_as_half(nsrc[pos])) : 0.f;
+      reinterpret_cast<float*>(tb + G::NVF)[pos] =
+          live ? __half2float(__ushort_as_half(nsrc[kPfChunk + pos])) : 0.f;
+    }
+  };
+  // the first chunk: its data, its tiles, then slot 0 is free for chunk 2
+  int issued = nchunks > 0 ? (nchunks > 1 ? 2 : 1) : 0;   // chunks 0, 1 in flight
+  if (nchunks > 0) {
+    const bool ok = mbar_wait(bar0, 0u);
+    if (ok) dequant(0);
+    if (!__syncthreads_and(ok)) {                  // the first copy never completed
+      stalled = true;
+      if (tid == 0) {
+        if (a.dev_status) atomicOr(a.dev_status, TQ_DEV_WAIT_TIMEOUT);
+        for (int k = 0; k < issued; ++k) mbar_wait(bar0 + 8 * (k & 1), (uint32_t)(k >> 1) & 1u);
+      }
+    } else {
+      if (tid == 0 && nchunks > 2) issue(2);
+      issued = min(nchunks, 3);
+    }
+  }
+  for (int c = 0; c < nchunks && !stalled; ++c) {
+    const uint8_t* tb = smem + (c & 1) * G::TBUF;
+    const uint32_t tbs = sbase + (c & 1) * G::TBUF;
     // ---- scores of the warp's 16 rows x 64 positions
     const int t0 = c * kPfChunk;
-    const uint16_t* nks = reinterpret_cast<const uint16_t*>(
-        smem + G::STG + (c & 1) * G::SLOT + kPfChunk * (G::RK + G::RV));
-    const uint16_t* nvs = nks + kPfChunk;
+    const float* nkf = reinterpret_cast<const float*>(tb + G::NKF);
+    const float* nvf = reinterpret_cast<const float*>(tb + G::NVF);
     float s[8][4];
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
@@ -273,8 +302,8 @@ prefill_kernel(const __grid_constant__ PrefillArgs a,
         for (int ks = 0; ks < 8; ++ks) {
           uint32_t bh0, bh1, bh2, bh3, bl0, bl1, bl2, bl3;
           const uint32_t o2 = 2 * ((16 * n2 + prow) * kTS + 16 * ks + pcol);
-          ldsm_x4(sbase + G::KH + o2, bh0, bh1, bh2, bh3);
-          ldsm_x4(sbase + G::KL + o2, bl0, bl1, bl2, bl3);
+          ldsm_x4(tbs + G::KH + o2, bh0, bh1, bh2, bh3);
+          ldsm_x4(tbs + G::KL + o2, bl0, bl1, bl2, bl3);
           mma16816(s[2 * n2], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], bh0, bh1);
           mma16816(s[2 * n2], qb[ks][0], qb[ks][1], qb[ks][2], qb[ks][3], bh0, bh1);
           mma16816(s[2 * n2], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], bl0, bl1);
@@ -291,7 +320,7 @@ prefill_kernel(const __grid_constant__ PrefillArgs a,
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int pl = 8 * nt + 2 * tq + e, pos = t0 + pl;
-        const float nk = __half2float(__ushort_as_half(nks[pl]));
+        const float nk = nkf[pl];
         float v0 = s[nt][e] * (si0 * nk), v1 = s[nt][2 + e] * (si1 * nk);
         if (pos > p0) v0 = -INFINITY;
         if (pos > p1) v1 = -INFINITY;
@@ -326,7 +355,7 @@ prefill_kernel(const __grid_constant__ PrefillArgs a,
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int pl = 8 * nt + 2 * tq + e;
-        const float nv = __half2float(__ushort_as_half(nvs[pl]));
+        const float nv = nvf[pl];
         const float w0 = s[nt][e] == -INFINITY ? 0.f : fast_exp2(s[nt][e] - mn0);
         const float w1 = s[nt][2 + e] == -INFINITY ? 0.f : fast_exp2(s[nt][2 + e] - mn1);
         l0 += w0;
@@ -346,13 +375,30 @@ prefill_kernel(const __grid_constant__ PrefillArgs a,
 #pragma unroll
         for (int j2 = 0; j2 < 8; ++j2) {
           uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(sbase + G::VT + 2 * ((16 * kk + vrow) * kTS + 16 * j2 + vcol), b0, b1, b2, b3);
+          ldsm_x4_t(tbs + G::VT + 2 * ((16 * kk + vrow) * kTS + 16 * j2 + vcol), b0, b1, b2, b3);
           mma16816(o[2 * j2], pa[kk][0], pa[kk][1], pa[kk][2], pa[kk][3], b0, b1);
           mma16816(o[2 * j2 + 1], pa[kk][0], pa[kk][1], pa[kk][2], pa[kk][3], b2, b3);
         }
       }
     }
-    __syncthreads();                                 // tiles and slot c are free
+    // ---- the next chunk into the other buffer (its last readers were the
+    // MMAs of chunk c - 1, finished before the previous barrier)
+    if (c + 1 < nchunks) {
+      const bool ok = mbar_wait(bar0 + 8 * ((c + 1) & 1), (uint32_t)((c + 1) >> 1) & 1u);
+      if (ok) dequant(c + 1);
+      if (!__syncthreads_and(ok)) {                // a copy never completed
+        stalled = true;
+        if (tid == 0 && a.dev_status) atomicOr(a.dev_status, TQ_DEV_WAIT_TIMEOUT);
+        // wait (bounded) for the copies still in flight, then stop
+        if (tid == 0)
+          for (int k = c + 1; k < issued; ++k)
+            mbar_wait(bar0 + 8 * (k & 1), (uint32_t)(k >> 1) & 1u);
+        break;
+      }
+      // slot (c + 1) & 1 is consumed: chunk c + 3 goes there
+      if (tid == 0 && c + 3 < nchunks) issue(c + 3);
+      if (c + 3 < nchunks) issued = c + 4;
+    }
   }
 
   // ---- per-row sums, normalization, inverse rotation, store
