@@ -178,3 +178,45 @@ def test_per_layer_bit_choice_in_one_step():
         want, _ = oracle_attend(codec.promote(qs[l], "f16"), gk, gnk, gv, gnv, ctx, gqa, bk, bv,
                                 seed)
         assert np.abs(host(outs[l]) - want).max() <= ATOL, (bk, bv)
+
+
+def test_append_full_workload_bench_configuration():
+    """The bench's decode step at full size: the Llama-3-8B-shaped layer
+    (8 kv heads, 32768 positions, K4/V2, GQA 4, one CTA per SM) with its
+    last row replaced by the new token, fp16 output as timed."""
+    import torch
+    import compressed_decode_attention_b200 as tq
+    from gpu_support import oracle_cache
+    w = S.WORKLOADS["llama3_8b_decode"]
+    pk, nk, pv, nv, ctx = oracle_cache("llama3_8b_decode")
+    B, H, cap, d = pk.shape[0], pk.shape[1], pk.shape[2], w.d
+    rng = np.random.default_rng(31)
+    new = rng.standard_normal((2, B, H, d))
+    new_bits = S.f16_bits(new)
+    qb = S.query_bits(w, step=3)
+    c = [dev(x) for x in (pk, nk, pv, nv)]
+    ws_bytes = tq.tq_attend_workspace_size(B, w.n_q_heads, cap, d)
+    ws = torch.zeros(ws_bytes // 4, dtype=torch.float32, device="cuda")
+    out = torch.empty((B, w.n_q_heads, d), dtype=torch.int16, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq.tq_attend_append(dev(qb), tq.TQ_F16, dev(new_bits), tq.TQ_F16, c[0], c[1], c[2], c[3],
+                        dev(ctx), B, w.n_q_heads, w.gqa, d, w.bits_k, w.bits_v, 0, cap, 0.0, 0,
+                        ws, ws_bytes, out, tq.TQ_F16, dev_status=st)
+    torch.cuda.synchronize()
+    gk, gnk, gv, gnv = [host(x) for x in c]
+    L = int(ctx[0])
+    for which, bits, rows, norms in ((0, w.bits_k, gk, gnk), (1, w.bits_v, gv, gnv)):
+        x = codec.promote(new_bits[which, 0], "f16")
+        idx, _, nbits, _, margin = codec.encode(x, bits, 0)
+        check_indices(codec.unpack(rows[0, :, L - 1], bits, d), idx, margin)
+        check_norms(norms[0, :, L - 1], nbits)
+    keep = np.ones(cap, bool)
+    keep[L - 1] = False
+    np.testing.assert_array_equal(gk[0][:, keep], pk[0][:, keep])
+    np.testing.assert_array_equal(gv[0][:, keep], pv[0][:, keep])
+    want, _ = oracle_attend(codec.promote(qb, "f16"), gk, gnk, gv, gnv, ctx, w.gqa, w.bits_k,
+                            w.bits_v, 0)
+    got = host(out).view(np.float16).astype(np.float64)
+    # fp16 output: its own rounding (2^-11 relative) on top of the bound
+    assert np.max(np.abs(got - want) - 2.0 ** -11 * np.abs(want)) <= ATOL
+    assert int(st.item()) == 0

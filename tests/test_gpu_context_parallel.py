@@ -170,3 +170,39 @@ def test_odd_record_count_alignment():
     """batch x heads odd (3 x 5): row p of the gathered buffer is only 8-byte
     aligned, which the records allow."""
     _run(4, 2, [300, 200, 129], 320, 1, 5, 128, 3, rng_seed=9)
+
+
+def test_full_workload_four_slices_as_timed():
+    """The bench's context-parallel line: the Llama-3-8B-shaped layer (8 kv
+    heads x 32768 positions) split into 4 slices that are views of one
+    cache (row offset, cap_tok kept as the head stride), merged by
+    tq_attend_combine; against the oracle over the whole context."""
+    import torch
+    import compressed_decode_attention_b200 as tq
+    from compressed_decode_attention_b200.context_parallel import slice_bounds
+    from gpu_support import oracle_cache
+    w = S.WORKLOADS["llama3_8b_decode"]
+    pk, nk, pv, nv, ctx = oracle_cache("llama3_8b_decode")
+    B, H, cap, d = pk.shape[0], pk.shape[1], pk.shape[2], w.d
+    qb = S.query_bits(w, step=5)
+    c = [dev(x) for x in (pk, nk, pv, nv)]
+    rk, rv = d * w.bits_k // 8, d * w.bits_v // 8
+    P = 4
+    rec = torch.empty((P, B, w.n_q_heads, d + 2), dtype=torch.float32, device="cuda")
+    ws_bytes = tq.tq_attend_workspace_size(B, w.n_q_heads, cap, d)
+    ws = torch.zeros(ws_bytes // 4, dtype=torch.float32, device="cuda")
+    qd = dev(qb)
+    for r in range(P):
+        a, b = slice_bounds(int(ctx[0]), P, r)
+        lens = dev(np.array([b - a], np.int32))
+        tq.tq_attend_partial(qd, tq.TQ_F16, c[0].data_ptr() + a * rk, c[1].data_ptr() + 2 * a,
+                             c[2].data_ptr() + a * rv, c[3].data_ptr() + 2 * a, lens, B,
+                             w.n_q_heads, w.gqa, d, w.bits_k, w.bits_v, 0, cap, 0.0, 0, ws,
+                             ws_bytes, rec[r])
+    out = torch.empty((B, w.n_q_heads, d), dtype=torch.int16, device="cuda")
+    tq.tq_attend_combine(rec, P, B, w.n_q_heads, d, 0, out, tq.TQ_F16)
+    torch.cuda.synchronize()
+    want, _ = oracle_attend(codec.promote(qb, "f16"), pk, nk, pv, nv, ctx, w.gqa, w.bits_k,
+                            w.bits_v, 0)
+    got = host(out).view(np.float16).astype(np.float64)
+    assert np.max(np.abs(got - want) - 2.0 ** -11 * np.abs(want)) <= ATOL

@@ -147,3 +147,50 @@ def test_gpu_sketch_rows_feed_the_scores():
     want = qjl.scores(codec.promote(qb, "f16"), host(pk)[None], host(nk)[None], host(sk)[None],
                       host(gk)[None], np.array([n]), gqa, bits, seed, Sm.astype(np.float64))
     assert np.abs(host(out) - want).max() <= ATOL
+
+
+def _oracle_head_sketch(kx, pk_h, nk_h, bits, seed, Sm):
+    """Worker: oracle sketch rows / gamma / projections of one kv head."""
+    from oracle import qjl as oq
+    r_rot = oq.residual_rotated(kx, bits, seed)[2]
+    rows, u, gb = oq.sketch(r_rot, Sm)
+    return rows, gb, u, np.sqrt(np.sum(r_rot ** 2, axis=1))
+
+
+def test_full_workload_sketch_and_scores():
+    """The bench's QJL line at full size: the Llama-3-8B-shaped layer's keys
+    (8 kv heads x 32768) sketched on the GPU against the oracle, then the
+    scores of its 32 query heads from the GPU's own rows."""
+    import torch
+    import compressed_decode_attention_b200 as tq
+    from gpu_support import oracle_cache, pool
+    w = S.WORKLOADS["llama3_8b_decode"]
+    pk, nk, pv, nv, ctx = oracle_cache("llama3_8b_decode")
+    H, cap, d, bits, n = w.n_kv_heads, w.cap_tok, w.d, w.bits_k, int(ctx[0])
+    kv = S.kv_bits(w, 0, n)                               # [2][n][H][d], the cached keys
+    Sm = S.projection_matrix(d)
+    sk = torch.zeros((1, H, cap, d // 8), dtype=torch.uint8, device="cuda")
+    gk = torch.zeros((1, H, cap), dtype=torch.int16, device="cuda")
+    tq.tq_qjl_encode(dev(np.ascontiguousarray(kv[0])), tq.TQ_F16, n, H, d, bits, 0, dev(Sm),
+                     dev(pk[0]), dev(nk[0]), sk, gk, cap, 0)
+    torch.cuda.synchronize()
+    got_rows, got_g = host(sk)[0], host(gk)[0]
+    futs = [pool().submit(_oracle_head_sketch, codec.promote(kv[0, :, h], "f16"), pk[0, h],
+                          nk[0, h], bits, 0, Sm.astype(np.float64)) for h in (0, 5)]
+    snorm = np.linalg.norm(Sm.astype(np.float64), axis=1)
+    for h, f in zip((0, 5), futs):
+        rows, gb, u, rr = f.result()
+        gbits = np.unpackbits(got_rows[h, :n], axis=-1, bitorder="little")
+        wbits = np.unpackbits(rows, axis=-1, bitorder="little")
+        margin = np.abs(u) / (snorm[None, :] * np.maximum(rr[:, None], 1e-30))
+        assert not ((gbits != wbits) & (margin >= 1e-4)).any()
+        assert (gbits != wbits).mean() <= 1e-3
+        assert np.abs(got_g[h, :n].astype(np.int64) - gb.astype(np.int64)).max() <= 1
+    qb = S.query_bits(w, step=7)
+    out = torch.empty((1, w.n_q_heads, cap), dtype=torch.float32, device="cuda")
+    tq.tq_qjl_scores(dev(qb), tq.TQ_F16, dev(pk), dev(nk), sk, gk, dev(Sm), dev(ctx), 1,
+                     w.n_q_heads, w.gqa, d, bits, 0, cap, 1, out)
+    torch.cuda.synchronize()
+    want = qjl.scores(codec.promote(qb, "f16"), pk, nk, got_rows[None], got_g[None], ctx, w.gqa,
+                      bits, 0, Sm.astype(np.float64))
+    assert np.abs(host(out) - want).max() <= ATOL
