@@ -120,3 +120,33 @@ def test_prefill_long_context_sharp_queries():
     """1500 cached positions (24 chunks), queries x4 (sharper softmax)."""
     err, st = _run(4, 2, [1500], 1536, 2, 4, 33, 0, 11, qscale=4.0)
     assert err <= ATOL
+
+
+def test_prefill_full_workload_sampled():
+    """The bench's prefill line: a 1024-token chunk at the end of an
+    8192-position context, 32 query / 8 kv heads, K4/V2, fp16 output;
+    tokens sampled across the tiles (first, tile edges, last) against the
+    oracle."""
+    import torch
+    import compressed_decode_attention_b200 as tq
+    rng = np.random.default_rng(41)
+    B, Hkv, gqa, T, L, bk, bv, seed = 1, 8, 4, 1024, 8192, 4, 2, 0
+    Hq = Hkv * gqa
+    pk, nk, pv, nv = _cache(bk, bv, B, Hkv, L, np.array([L]), seed, rng)
+    qb = S.f16_bits(rng.standard_normal((B, T, Hq, D)))
+    q64 = codec.promote(qb, "f16")
+    out = torch.empty((B, T, Hq, D), dtype=torch.int16, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq.tq_prefill_attend(dev(qb), tq.TQ_F16, dev(pk), dev(nk), dev(pv), dev(nv),
+                         dev(np.array([L], np.int32)), B, T, Hq, gqa, D, bk, bv, seed, L, out,
+                         tq.TQ_F16, dev_status=st)
+    torch.cuda.synchronize()
+    got = host(out).view(np.float16).astype(np.float64)
+    sample = [0, 1, 31, 32, 511, 512, 1000, 1023]
+    futs = {t: pool().submit(_oracle_token, q64[0, t], pk[0], nk[0], pv[0], nv[0], L - T + t,
+                             gqa, bk, bv, seed) for t in sample}
+    for t, f in futs.items():
+        want = f.result()
+        err = np.max(np.abs(got[0, t] - want) - 2.0 ** -11 * np.abs(want))
+        assert err <= ATOL, (t, err)
+    assert int(st.item()) == 0
