@@ -127,15 +127,34 @@ __device__ __forceinline__ void encode_vector(
 
   // words[w] accumulates bits(v) << off = (kMagic + idx) << off; the kMagic
   // parts are removed after the loop
+  // With three or more positive thresholds the count is two-level: one
+  // compare (ALU pipe) against the middle threshold picks the half of the
+  // table, and only that half's HALF thresholds take a saturated FMA. Below
+  // the middle, its indicator and the upper half's are all 1; above, the
+  // lower half's are all 0.
+  constexpr int HALF = NTH / 2;
+  const float tmid = (n > 0.f ? n : 1.f) * cb.threshold[kHalf + HALF];
+
   uint32_t words[BITS] = {};
 #pragma unroll
   for (int i = 0; i < 32; i += 2) {
-    float2 w2 = make_float2(kOdd, kOdd);
     const float a0 = fabsf(x[i]), a1 = fabsf(x[i + 1]);
+    float2 w2;
+    if constexpr (NTH >= 3) {
+      const bool p0 = a0 < tmid, p1 = a1 < tmid;
+      w2 = make_float2(p0 ? kOdd - 2.f * (HALF + 1) : kOdd, p1 ? kOdd - 2.f * (HALF + 1) : kOdd);
 #pragma unroll
-    for (int k = 0; k < NTH; ++k)
-      w2 = f2fma(make_float2(fma_sat(a0, -big, C[k]), fma_sat(a1, -big, C[k])),
-                 make_float2(-2.f, -2.f), w2);
+      for (int k = 0; k < HALF; ++k)
+        w2 = f2fma(make_float2(fma_sat(a0, -big, p0 ? C[k] : C[k + HALF + 1]),
+                               fma_sat(a1, -big, p1 ? C[k] : C[k + HALF + 1])),
+                   make_float2(-2.f, -2.f), w2);
+    } else {
+      w2 = make_float2(kOdd, kOdd);
+#pragma unroll
+      for (int k = 0; k < NTH; ++k)
+        w2 = f2fma(make_float2(fma_sat(a0, -big, C[k]), fma_sat(a1, -big, C[k])),
+                   make_float2(-2.f, -2.f), w2);
+    }
     const float2 sg = f2add(make_float2(x[i], x[i + 1]), make_float2(0.f, 0.f));
     const float2 u = f2add(make_float2(copysignf(w2.x, sg.x), copysignf(w2.y, sg.y)),
                            make_float2(kOdd, kOdd));
