@@ -776,6 +776,10 @@ attend_kernel(const __grid_constant__ AttendArgs a,
     uint8_t* app_k = smem + Gm::APPOFF;
     uint8_t* app_v = app_k + D / 2;
     uint16_t* app_n = reinterpret_cast<uint16_t*>(app_k + D);
+    __syncthreads();
+    // The owner warp encodes after the CTA barrier: no other warp needs the
+    // new row (only this warp's last chunk holds position L - 1), and the
+    // encode overlaps the wait for the warp's first staged chunk.
     if (app) {
       constexpr int LPV = D / 32;                     // lanes per vector
       if (lane < 2 * LPV) {
@@ -805,7 +809,6 @@ attend_kernel(const __grid_constant__ AttendArgs a,
         a.norms_v[row] = app_n[1];
       }
     }
-    __syncthreads();
 
     // ---- query fragments (B operand of the score MMA), column n = gq.
     //   NT = 1: columns 0-3 hold the high part of heads 0-3, 4-7 their low part.

@@ -67,12 +67,16 @@ encode_kernel(const __grid_constant__ EncodeArgs a,
 template <int D>
 cudaError_t launch_encode_d(const EncodeArgs& a, const Codebook& cbk, const Codebook& cbv,
                             const SignMask& sm, cudaStream_t stream) {
-  static int sms = 0;
-  if (!sms) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      sms = 148;
+  // SM count of the current device, looked up once per device
+  static int cached[64] = {0};
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) {
+    if (!cached[dev]) {
+      int n = 0;
+      cached[dev] = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) ==
+                            cudaSuccess && n > 0 ? n : 148;
+    }
+    sms = cached[dev];
   }
   // grid.x: enough tile blocks that all (head, K/V) pairs cover every SM
   // about eight times; each block strides over its head's tiles

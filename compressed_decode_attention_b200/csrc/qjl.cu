@@ -384,13 +384,16 @@ template <int D, int BITS>
 cudaError_t launch_encode_db(const QjlEncodeArgs& a, const Codebook& cb, const SignMask& sm,
                              cudaStream_t stream) {
   using G = QjlEncGeo<D>;
-  static bool attr_set = false;
-  if (!attr_set) {
+  // the shared-memory opt-in is per device
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !configured[dev]) {
     const cudaError_t e = cudaFuncSetAttribute(qjl_encode_kernel<D, BITS>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                (int)G::SMEM);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    if (dev >= 0 && dev < 64) configured[dev] = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((a.n_tok + kQjlTokens - 1) / kQjlTokens, a.n_kv_heads, 1);
