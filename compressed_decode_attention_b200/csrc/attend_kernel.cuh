@@ -443,6 +443,14 @@ attend_kernel(const __grid_constant__ AttendArgs a,
     for (size_t off = ((size_t)cta * kThreads + tid) * 128; off < qbytes;
          off += (size_t)Gc * kThreads * 128)
       asm volatile("prefetch.global.L2 [%0];\n" ::"l"(qc + off));
+    // likewise the decode step's new K/V rows, encoded later by the owner warps
+    if (a.new_kv) {
+      const size_t kvbytes = (size_t)2 * B * H * D * 2;
+      const char* kc = reinterpret_cast<const char*>(a.new_kv);
+      for (size_t off = ((size_t)cta * kThreads + tid) * 128; off < kvbytes;
+           off += (size_t)Gc * kThreads * 128)
+        asm volatile("prefetch.global.L2 [%0];\n" ::"l"(kc + off));
+    }
   }
 
   // Segment search (warp 0): the first sequence whose flat block range holds
