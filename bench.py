@@ -400,8 +400,14 @@ def run_gpu(args, rank, world, local_rank):
     # ---------------- decode step graphs
     # per-layer queries, new K/V and outputs are views of three contiguous
     # buffers, so that the end-to-end step moves each with one copy
-    q_all = torch.randn((L, 1, w.n_q_heads, d), generator=gen, device=device).half()
-    kv_all_new = torch.stack([device_kv(w, l, 1, gen) for l in range(L)])   # [L][2][1][H][d]
+    # the step's inputs (every layer's query, then every layer's new K/V)
+    # share one device buffer of 16-bit words
+    nq16, nkv16 = L * w.n_q_heads * d, L * 2 * H * d
+    inputs = torch.empty(nq16 + nkv16, dtype=torch.int16, device=device)
+    q_all = inputs[:nq16].view(torch.float16).view(L, 1, w.n_q_heads, d)
+    kv_all_new = inputs[nq16:].view(L, 2, 1, H, d)
+    q_all.copy_(torch.randn((L, 1, w.n_q_heads, d), generator=gen, device=device).half())
+    kv_all_new.copy_(torch.stack([device_kv(w, l, 1, gen) for l in range(L)]))
     outs_all = torch.empty((L, 1, w.n_q_heads, d), dtype=torch.float16, device=device)
     q = [q_all[l] for l in range(L)]
     kv_new = [kv_all_new[l] for l in range(L)]
@@ -584,19 +590,16 @@ def run_gpu(args, rank, world, local_rank):
     del bgraph, bcache, bq, bout, bws
 
     # ---------------- end to end: host inputs in, host output back, every step
-    q_host = torch.empty((L, 1, w.n_q_heads, d), dtype=torch.float16).pin_memory()
-    kv_host = torch.empty((L, 2, 1, H, d), dtype=torch.int16).pin_memory()
+    in_host = torch.empty(nq16 + nkv16, dtype=torch.int16).pin_memory()
     out_host = torch.empty((L, 1, w.n_q_heads, d), dtype=torch.float16).pin_memory()
-    q_host.copy_(q_all.cpu())
-    kv_host.copy_(kv_all_new.cpu())
+    in_host.copy_(inputs.cpu())
     e2e_graph = capture(step)
     torch.cuda.synchronize()
 
     def e2e_step():
-        # one host-to-device copy each of every layer's query and new K/V,
-        # the step's launches, one device-to-host copy of every output
-        q_all.copy_(q_host, non_blocking=True)
-        kv_all_new.copy_(kv_host, non_blocking=True)
+        # one host-to-device copy of every layer's query and new K/V, the
+        # step's launches, one device-to-host copy of every output
+        inputs.copy_(in_host, non_blocking=True)
         e2e_graph.replay()
         out_host.copy_(outs_all, non_blocking=True)
 
@@ -654,7 +657,7 @@ def run_gpu(args, rank, world, local_rank):
                      "traffic": traffic["traffic_bytes_per_launch"] if traffic else None},
         "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 4),
-                "h2d_bytes_per_step": int(q_host.numel() * 2 + kv_host.numel() * 2),
+                "h2d_bytes_per_step": int(in_host.numel() * 2),
                 "d2h_bytes_per_step": int(out_host.numel() * 2)},
         "gpu_launches": launches,
         "clocks": clk.summary(),
