@@ -366,12 +366,17 @@ def run_gpu(args, rank, world, local_rank):
               for _ in range(pf_layers)]
     pf_ctx_dev = torch.full((1,), pf_ctx, dtype=torch.int32, device=device)
 
+    pf_splits = tq.tq_prefill_splits(1, pf_T, w.n_q_heads, w.gqa)
+    pf_wsb = tq.tq_prefill_workspace_size(1, pf_T, w.n_q_heads, d, pf_splits)
+    pf_ws = torch.empty(max(pf_wsb, 16), dtype=torch.uint8, device=device)
+
     def prefill_all():
         for l in range(pf_layers):
-            tq.tq_prefill_attend(pf_q[l], tq.TQ_F16, pf.pk[l], pf.nk[l], pf.pv[l], pf.nv[l],
-                                 pf_ctx_dev, 1, pf_T, w.n_q_heads, w.gqa, d, w.bits_k, w.bits_v,
-                                 seed, pf_ctx, pf_out[l], tq.TQ_F16, dev_status=status,
-                                 stream=stream)
+            tq.tq_prefill_attend_split(pf_q[l], tq.TQ_F16, pf.pk[l], pf.nk[l], pf.pv[l],
+                                       pf.nv[l], pf_ctx_dev, 1, pf_T, w.n_q_heads, w.gqa, d,
+                                       w.bits_k, w.bits_v, seed, pf_ctx, pf_splits, pf_ws,
+                                       pf_wsb, pf_out[l], tq.TQ_F16, dev_status=status,
+                                       stream=stream)
 
     with torch.cuda.stream(stream):
         prefill_all()
@@ -394,7 +399,7 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize()
     pf_ms = reduce_max(p0.elapsed_time(p1) / (pf_steps * pf_layers), device)
     pf_flops = prefill_flops(w, pf_ctx, pf_T)
-    del pf_graph, pf, pf_q, pf_out
+    del pf_graph, pf, pf_q, pf_out, pf_ws
     torch.cuda.empty_cache()
 
     # ---------------- decode step graphs
@@ -681,7 +686,8 @@ def run_gpu(args, rank, world, local_rank):
                                  "frac": round(pf_flops / (pf_ms * 1e-3) / 1e12 / measured_tensor_peak(), 4),
                                  "peak_kind": "measured dense bf16 (fp16 mma runs at the same rate)",
                                  "flops_per_call": pf_flops},
-                    "gpu_launches": pf_steps * pf_layers},
+                    "context_splits": pf_splits,
+                    "gpu_launches": pf_steps * pf_layers * (2 if pf_splits > 1 else 1)},
         "qjl": {
             "workload": f"{WORKLOAD} keys: {H} kv heads x {ctx} positions, K{w.bits_k}, d={d}; "
                         f"scores of {w.n_q_heads} query heads; {QL} distinct layer caches",

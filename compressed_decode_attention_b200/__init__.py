@@ -62,6 +62,13 @@ def lib() -> ctypes.CDLL:
         L.tq_prefill_attend.restype = I
         L.tq_prefill_attend.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, I, U64, I, P, P,
                                         I, P]
+        L.tq_prefill_attend_split.restype = I
+        L.tq_prefill_attend_split.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, I, U64, I,
+                                              I, P, SZ, P, P, I, P]
+        L.tq_prefill_workspace_size.restype = SZ
+        L.tq_prefill_workspace_size.argtypes = [I, I, I, I, I]
+        L.tq_prefill_splits.restype = I
+        L.tq_prefill_splits.argtypes = [I, I, I, I]
         L.tq_attend_partial.restype = I
         L.tq_attend_partial.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F, I,
                                         P, SZ, P, P, P, P]
@@ -227,6 +234,27 @@ def tq_qjl_scores(q, q_dtype, packed_k, norms_k, sketch, gamma, projection, ctx_
         _ptr(q), q_dtype, _ptr(packed_k), _ptr(norms_k), _ptr(sketch), _ptr(gamma),
         _ptr(projection), _ptr(ctx_lens), batch, n_q_heads, gqa_ratio, d, bits_k, seed, cap_tok,
         int(with_sketch), _ptr(dev_status), _ptr(scores), _stream(stream)))
+
+
+def tq_prefill_attend_split(q, q_dtype, packed_k, norms_k, packed_v, norms_v, ctx_lens, batch,
+                            n_tok, n_q_heads, gqa_ratio, d, bits_k, bits_v, seed, cap_tok,
+                            n_splits, workspace, workspace_bytes, out, out_dtype,
+                            dev_status=None, stream=None):
+    """tq_prefill_attend with each query tile's context split n_splits ways
+    (records in the workspace, merged into out by a second launch)."""
+    _check("tq_prefill_attend_split", lib().tq_prefill_attend_split(
+        _ptr(q), q_dtype, _ptr(packed_k), _ptr(norms_k), _ptr(packed_v), _ptr(norms_v),
+        _ptr(ctx_lens), batch, n_tok, n_q_heads, gqa_ratio, d, bits_k, bits_v, seed, cap_tok,
+        n_splits, _ptr(workspace), workspace_bytes, _ptr(dev_status), _ptr(out), out_dtype,
+        _stream(stream)))
+
+
+def tq_prefill_workspace_size(batch, n_tok, n_q_heads, d, n_splits) -> int:
+    return lib().tq_prefill_workspace_size(batch, n_tok, n_q_heads, d, n_splits)
+
+
+def tq_prefill_splits(batch, n_tok, n_q_heads, gqa_ratio) -> int:
+    return lib().tq_prefill_splits(batch, n_tok, n_q_heads, gqa_ratio)
 
 
 def tq_attend_noalloc(q, q_dtype, packed_k, norms_k, packed_v, norms_v, ctx_lens,

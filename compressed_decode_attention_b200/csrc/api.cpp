@@ -268,6 +268,58 @@ int tq_prefill_attend(const void* q, int q_dtype, const uint8_t* packed_k,
                       int n_tok, int n_q_heads, int gqa_ratio, int d, int bits_k,
                       int bits_v, uint64_t seed, int cap_tok, int* dev_status, void* out,
                       int out_dtype, void* stream) {
+  return tq_prefill_attend_split(q, q_dtype, packed_k, norms_k, packed_v, norms_v, ctx_lens,
+                                 batch, n_tok, n_q_heads, gqa_ratio, d, bits_k, bits_v, seed,
+                                 cap_tok, 1, nullptr, 0, dev_status, out, out_dtype, stream);
+}
+
+int tq_prefill_splits(int batch, int n_tok, int n_q_heads, int gqa_ratio) {
+  if (batch < 1 || n_tok < 1 || n_q_heads < 1 || gqa_ratio < 1 || n_q_heads % gqa_ratio ||
+      gqa_ratio > kMaxGroup)
+    return 1;
+  // CTAs of one split (one per SM: 128 query rows each); pick the split
+  // count that minimizes rounds of the SMs per unit of work, ceil(n·S/SMs)/S
+  const long long rows_per_tile = 128 / gqa_ratio;
+  const long long ctas = (long long)batch * (n_q_heads / gqa_ratio) *
+                         ((n_tok + rows_per_tile - 1) / rows_per_tile);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      sms <= 0)
+    sms = 148;
+  int best = 1;
+  double best_cost = (double)((ctas + sms - 1) / sms);
+  for (int sp = 2; sp <= kMaxPrefillSplits; ++sp) {
+    // a small charge per split for the records and the combine
+    const double cost = (double)((ctas * sp + sms - 1) / sms) / sp + 0.02 * (sp - 1);
+    if (cost < best_cost - 1e-9) {
+      best = sp;
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
+size_t tq_prefill_workspace_size(int batch, int n_tok, int n_q_heads, int d, int n_splits) {
+  if (batch < 1 || n_tok < 1 || n_q_heads < 1 || n_splits <= 1 || check_head_dim(d) != TQ_OK)
+    return 0;
+  return (size_t)n_splits * batch * n_tok * n_q_heads * (d + 2) * sizeof(float);
+}
+
+int tq_prefill_attend_split(const void* q, int q_dtype, const uint8_t* packed_k,
+                            const uint16_t* norms_k, const uint8_t* packed_v,
+                            const uint16_t* norms_v, const int32_t* ctx_lens, int batch,
+                            int n_tok, int n_q_heads, int gqa_ratio, int d, int bits_k,
+                            int bits_v, uint64_t seed, int cap_tok, int n_splits,
+                            void* workspace, size_t workspace_bytes, int* dev_status,
+                            void* out, int out_dtype, void* stream) {
+  if (n_splits < 1 || n_splits > kMaxPrefillSplits) return TQ_ERR_INVALID_ARG;
+  if (n_splits > 1 &&
+      (!workspace || ((uintptr_t)workspace & 15u) || n_tok < 1 ||
+       workspace_bytes < tq_prefill_workspace_size(batch, n_tok, n_q_heads, d, n_splits)))
+    return TQ_ERR_INVALID_ARG;
+  if (n_splits > 1 && (long long)batch * n_tok * n_q_heads > (1LL << 30))
+    return TQ_ERR_UNSUPPORTED;
   if (batch < 1 || n_tok < 1 || n_q_heads < 1 || gqa_ratio < 1 || cap_tok < 1)
     return TQ_ERR_INVALID_ARG;
   if (n_q_heads % gqa_ratio) return TQ_ERR_INVALID_ARG;
@@ -307,6 +359,8 @@ int tq_prefill_attend(const void* q, int q_dtype, const uint8_t* packed_k,
   a.dev_status = dev_status;
   a.out = out;
   a.out_dtype = out_dtype;
+  a.n_splits = n_splits;
+  a.records = n_splits > 1 ? (float*)workspace : nullptr;
   return from_cuda(launch_prefill(a, *cbk, *cbv, sign_mask(seed), (cudaStream_t)stream));
 }
 

@@ -88,9 +88,14 @@ prefill_kernel(const __grid_constant__ PrefillArgs a,
   const int GQ = a.gqa, H = a.n_kv_heads, T = a.n_tok;
   const int TQ = kPfRows / GQ;                     // query tokens per tile
   const int tiles = (T + TQ - 1) / TQ;
-  const int tile = blockIdx.x % tiles;
-  const int g = (blockIdx.x / tiles) % H;
-  const int b = blockIdx.x / (tiles * H);
+  // split s of n_splits takes the s-th share of the tile's chunks and leaves
+  // log-sum-exp records for the combine kernel instead of the output
+  const int S = a.n_splits > 1 ? a.n_splits : 1;
+  const int split = blockIdx.x % S;
+  const int unit = blockIdx.x / S;
+  const int tile = unit % tiles;
+  const int g = (unit / tiles) % H;
+  const int b = unit / (tiles * H);
   const int i0 = tile * TQ, nq = min(TQ, T - i0);
   const int R = nq * GQ;                           // valid rows
   float* sinv = reinterpret_cast<float*>(smem + G::SINV);
@@ -124,16 +129,20 @@ prefill_kernel(const __grid_constant__ PrefillArgs a,
   const int raw = a.ctx_lens[b];
   const int L = min(max(raw, 0), a.cap_tok);
   const int start = L - T;                         // absolute position of token 0
-  if (tile == 0 && g == 0 && tid == 0 && a.dev_status) {
+  if (tile == 0 && g == 0 && split == 0 && tid == 0 && a.dev_status) {
     if (raw > a.cap_tok) atomicOr(a.dev_status, TQ_DEV_CTX_CLAMPED);
     if (L < T) atomicOr(a.dev_status, TQ_DEV_CTX_EMPTY);
   }
   const int p_last = start + i0 + nq - 1;          // last query position of the tile
-  const int nchunks = p_last >= 0 ? p_last / kPfChunk + 1 : 0;
+  const int nch_tile = p_last >= 0 ? p_last / kPfChunk + 1 : 0;
+  // this CTA's chunks: absolute chunks cbase .. cbase + nchunks - 1 (local
+  // index c = 0 .. nchunks - 1 for staging slots and barrier phases)
+  const int cbase = (int)((long long)split * nch_tile / S);
+  const int nchunks = (int)((long long)(split + 1) * nch_tile / S) - cbase;
 
   const size_t seq_row = ((size_t)b * H + g) * a.cap_tok;
   auto issue = [&](int c) {                        // thread 0
-    const int t0 = c * kPfChunk;
+    const int t0 = (cbase + c) * kPfChunk;
     const int rows = min(kPfChunk, L - t0);
     const int krows = min(kPfChunk, (rows + G::KROWS - 1) / G::KROWS * G::KROWS);
     const int vrows = min(kPfChunk, (rows + G::VROWS - 1) / G::VROWS * G::VROWS);
@@ -259,7 +268,7 @@ prefill_kernel(const __grid_constant__ PrefillArgs a,
     if (qd == 0) {
       // norms as floats; 0 past the sequence end (the copied norm runs stop
       // at a multiple of 8 positions: the rest of the slot is stale)
-      const bool live = c * kPfChunk + pos < L;
+      const bool live = (cbase + c) * kPfChunk + pos < L;
       const uint16_t* nsrc = reinterpret_cast<const uint16_t*>(st + kPfChunk * (G::RK + G::RV));
       reinterpret_cast<float*>(tb + G::NKF)[pos] =
           live ? __half2float(__ushort_as_half(nsrc[pos])) : 0.f;
@@ -287,7 +296,7 @@ prefill_kernel(const __grid_constant__ PrefillArgs a,
     const uint8_t* tb = smem + (c & 1) * G::TBUF;
     const uint32_t tbs = sbase + (c & 1) * G::TBUF;
     // ---- scores of the warp's 16 rows x 64 positions
-    const int t0 = c * kPfChunk;
+    const int t0 = (cbase + c) * kPfChunk;
     const float* nkf = reinterpret_cast<const float*>(tb + G::NKF);
     const float* nvf = reinterpret_cast<const float*>(tb + G::NVF);
     float s[8][4];
@@ -407,6 +416,30 @@ prefill_kernel(const __grid_constant__ PrefillArgs a,
     l0 += __shfl_xor_sync(0xFFFFFFFFu, l0, o2);
     l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, o2);
   }
+  if (S > 1) {
+    // records of this split: the unnormalized value sum (rotated domain),
+    // the base-2 running maximum and the sum, per row (empty: 0, -inf, 0)
+#pragma unroll
+    for (int rsel = 0; rsel < 2; ++rsel) {
+      const int r = rsel ? r1 : r0;
+      if (r >= R) continue;
+      const int t = r / GQ, h = r - t * GQ;
+      const size_t rec = (size_t)split * ((size_t)a.batch * T * a.n_q_heads) +
+                         ((size_t)b * T + i0 + t) * a.n_q_heads + (size_t)g * GQ + h;
+      float* dst = a.records + rec * (D + 2);
+      const float m = stalled ? -INFINITY : (rsel ? m1 : m0);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float v0 = stalled || m == -INFINITY ? 0.f : o[j][2 * rsel];
+        const float v1 = stalled || m == -INFINITY ? 0.f : o[j][2 * rsel + 1];
+        *reinterpret_cast<float2*>(dst + 8 * j + 2 * tq) = make_float2(v0, v1);
+      }
+      if (tq == 0)
+        *reinterpret_cast<float2*>(dst + D) =
+            make_float2(m, m == -INFINITY ? 0.f : (rsel ? l1 : l0));
+    }
+    return;
+  }
   const float il0 = l0 > 0.f && !stalled ? 1.f / l0 : 0.f;
   const float il1 = l1 > 0.f && !stalled ? 1.f / l1 : 0.f;
   // x[k][e]: coordinate 8k + 2tq + e of row r0 (y: row r1)
@@ -488,7 +521,8 @@ cudaError_t launch_prefill_bits(const PrefillArgs& a, const Codebook& cbk, const
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }
   const int tq = kPfRows / a.gqa;
-  const long long grid = (long long)a.batch * a.n_kv_heads * ((a.n_tok + tq - 1) / tq);
+  const int S = a.n_splits > 1 ? a.n_splits : 1;
+  const long long grid = (long long)a.batch * a.n_kv_heads * ((a.n_tok + tq - 1) / tq) * S;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
@@ -500,7 +534,18 @@ cudaError_t launch_prefill_bits(const PrefillArgs& a, const Codebook& cbk, const
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, prefill_kernel<BK, BV>, a, cbk, cbv, sm);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_kernel<BK, BV>, a, cbk, cbv, sm);
+  if (e != cudaSuccess || S == 1) return e;
+  // merge the splits' records and rotate back (the context-parallel combine)
+  CombineArgs c;
+  c.partials = a.records;
+  c.n_parts = S;
+  c.n_rec = a.batch * a.n_tok * a.n_q_heads;
+  c.d = 128;
+  c.dev_status = a.dev_status;
+  c.out = a.out;
+  c.out_dtype = a.out_dtype;
+  return launch_combine(c, sm, stream);
 }
 
 }  // namespace

@@ -113,7 +113,13 @@ struct PrefillArgs {
   int* dev_status;
   void* out;                 // [batch][n_tok][n_q_heads][d]
   int out_dtype;
+  // n_splits > 1: every tile's context is split n_splits ways; the splits
+  // write log-sum-exp records [n_splits][batch*n_tok*n_q_heads][d + 2] and
+  // a combine launch merges them into out
+  int n_splits;
+  float* records;
 };
+constexpr int kMaxPrefillSplits = 8;
 cudaError_t launch_prefill(const PrefillArgs& a, const Codebook& cbk, const Codebook& cbv,
                            const SignMask& sm, cudaStream_t stream);
 

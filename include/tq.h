@@ -71,7 +71,7 @@
 extern "C" {
 #endif
 
-#define TQ_ABI_VERSION 5
+#define TQ_ABI_VERSION 6
 
 /* Tokens per sparse-V block; split boundaries are multiples of this. */
 #define TQ_SPARSE_V_BLOCK 64
@@ -292,6 +292,41 @@ int tq_prefill_attend(const void* q, int q_dtype,
                       int gqa_ratio, int d, int bits_k, int bits_v, uint64_t seed,
                       int cap_tok, int* dev_status, void* out, int out_dtype,
                       void* stream);
+
+/*
+ * tq_prefill_attend_split — tq_prefill_attend with every query tile's
+ * context split n_splits ways. Each split attends over its share of the
+ * tile's 64-position chunks and leaves log-sum-exp records (the layout of
+ * tq_attend_partial, one per (sequence, token, query head)) in the
+ * workspace; a merge launch (tq_attend_combine's kernel) then writes out.
+ * The result equals tq_prefill_attend's within the attention tolerance.
+ * Splitting keeps all SMs busy when the tiles do not fill whole waves (one
+ * CTA of 128 query rows per SM): 256 tiles on 148 SMs take two waves, four
+ * splits of them seven quarter-waves.
+ *   n_splits    1 .. 8; 1 is tq_prefill_attend (no workspace needed).
+ *   workspace, workspace_bytes  >= tq_prefill_workspace_size(batch, n_tok,
+ *               n_q_heads, d, n_splits) bytes, 16-byte aligned, for
+ *               n_splits > 1; scratch (no state between calls).
+ *   batch · n_tok · n_q_heads <= 2^30 when n_splits > 1 (TQ_ERR_UNSUPPORTED).
+ * All other arguments and errors as for tq_prefill_attend.
+ */
+int tq_prefill_attend_split(const void* q, int q_dtype,
+                            const uint8_t* packed_k, const uint16_t* norms_k,
+                            const uint8_t* packed_v, const uint16_t* norms_v,
+                            const int32_t* ctx_lens, int batch, int n_tok, int n_q_heads,
+                            int gqa_ratio, int d, int bits_k, int bits_v, uint64_t seed,
+                            int cap_tok, int n_splits, void* workspace,
+                            size_t workspace_bytes, int* dev_status, void* out,
+                            int out_dtype, void* stream);
+
+/* Workspace bytes of tq_prefill_attend_split: n_splits · batch · n_tok ·
+ * n_q_heads · (d + 2) floats; 0 for n_splits <= 1 or invalid arguments. */
+size_t tq_prefill_workspace_size(int batch, int n_tok, int n_q_heads, int d, int n_splits);
+
+/* A split count for tq_prefill_attend_split on the current device: the
+ * n in 1..8 that minimizes ceil(tiles·n / SMs) / n (rounds of the SMs per
+ * unit of work) plus a small charge per split. Host only; 1 on bad input. */
+int tq_prefill_splits(int batch, int n_tok, int n_q_heads, int gqa_ratio);
 
 /*
  * Context parallelism: the positions of every sequence are split over the

@@ -46,7 +46,7 @@ def _oracle_token(q, pk, nk, pv, nv, p, gqa, bk, bv, seed):
 
 
 def _run(bk, bv, ctx, cap, Hkv, gqa, T, seed, rng_seed, q_dtype="f16", out_dtype="f32",
-         qscale=1.0):
+         qscale=1.0, n_splits=1):
     import torch
     import compressed_decode_attention_b200 as tq
     rng = np.random.default_rng(rng_seed)
@@ -62,9 +62,16 @@ def _run(bk, bv, ctx, cap, Hkv, gqa, T, seed, rng_seed, q_dtype="f16", out_dtype
     else:
         out = torch.empty((B, T, Hq, D), dtype=torch.int16, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    tq.tq_prefill_attend(dev(qb), enum[q_dtype], dev(pk), dev(nk), dev(pv), dev(nv), dev(ctx),
-                         B, T, Hq, gqa, D, bk, bv, seed, cap, out, enum[out_dtype],
-                         dev_status=st)
+    if n_splits == 1:
+        tq.tq_prefill_attend(dev(qb), enum[q_dtype], dev(pk), dev(nk), dev(pv), dev(nv),
+                             dev(ctx), B, T, Hq, gqa, D, bk, bv, seed, cap, out, enum[out_dtype],
+                             dev_status=st)
+    else:
+        wsb = tq.tq_prefill_workspace_size(B, T, Hq, D, n_splits)
+        ws = torch.full((wsb // 4,), float("nan"), dtype=torch.float32, device="cuda")
+        tq.tq_prefill_attend_split(dev(qb), enum[q_dtype], dev(pk), dev(nk), dev(pv), dev(nv),
+                                   dev(ctx), B, T, Hq, gqa, D, bk, bv, seed, cap, n_splits, ws,
+                                   wsb, out, enum[out_dtype], dev_status=st)
     torch.cuda.synchronize()
     got = host(out)
     if out_dtype == "f16":
@@ -143,6 +150,63 @@ def test_prefill_full_workload_sampled():
     torch.cuda.synchronize()
     got = host(out).view(np.float16).astype(np.float64)
     sample = [0, 1, 31, 32, 511, 512, 1000, 1023]
+    futs = {t: pool().submit(_oracle_token, q64[0, t], pk[0], nk[0], pv[0], nv[0], L - T + t,
+                             gqa, bk, bv, seed) for t in sample}
+    for t, f in futs.items():
+        want = f.result()
+        err = np.max(np.abs(got[0, t] - want) - 2.0 ** -11 * np.abs(want))
+        assert err <= ATOL, (t, err)
+    assert int(st.item()) == 0
+
+
+@pytest.mark.parametrize("n_splits,bk,bv,gqa,T", [
+    (2, 4, 2, 4, 40),
+    (3, 3, 2, 5, 30),
+    (4, 4, 3, 8, 20),
+    (8, 2, 4, 1, 130),
+])
+def test_prefill_split_context_matches_oracle(n_splits, bk, bv, gqa, T):
+    """The context of every tile split n ways (records merged by the combine
+    kernel), including splits with no chunk: the oracle bar as unsplit."""
+    err, st = _run(bk, bv, [300, 180], 320, 2, gqa, T, 0, 100 + bk * 10 + n_splits,
+                   n_splits=n_splits)
+    assert err <= ATOL
+    assert st == 0
+
+
+def test_prefill_split_short_context_and_dtypes():
+    """ctx = 5 < 12 tokens with 4 splits: tokens without positions give 0 and
+    TQ_DEV_CTX_EMPTY through the merge; bf16 output."""
+    err, st = _run(4, 2, [5, 70], 128, 2, 4, 12, 0, 9, n_splits=4)
+    assert err <= ATOL
+    assert st == 4
+    err, _ = _run(4, 2, [200], 256, 1, 4, 24, 3, 7, out_dtype="bf16", n_splits=3)
+    assert err <= ATOL
+
+
+def test_prefill_split_full_workload_sampled():
+    """The bench's prefill line with the split count the library picks for
+    this device (4 on 148 SMs)."""
+    import torch
+    import compressed_decode_attention_b200 as tq
+    rng = np.random.default_rng(43)
+    B, Hkv, gqa, T, L, bk, bv, seed = 1, 8, 4, 1024, 8192, 4, 2, 0
+    Hq = Hkv * gqa
+    pk, nk, pv, nv = _cache(bk, bv, B, Hkv, L, np.array([L]), seed, rng)
+    qb = S.f16_bits(rng.standard_normal((B, T, Hq, D)))
+    q64 = codec.promote(qb, "f16")
+    n_splits = tq.tq_prefill_splits(B, T, Hq, gqa)
+    assert n_splits >= 1
+    wsb = tq.tq_prefill_workspace_size(B, T, Hq, D, n_splits)
+    ws = torch.empty(max(wsb, 16) // 4, dtype=torch.float32, device="cuda")
+    out = torch.empty((B, T, Hq, D), dtype=torch.int16, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq.tq_prefill_attend_split(dev(qb), tq.TQ_F16, dev(pk), dev(nk), dev(pv), dev(nv),
+                               dev(np.array([L], np.int32)), B, T, Hq, gqa, D, bk, bv, seed, L,
+                               n_splits, ws, wsb, out, tq.TQ_F16, dev_status=st)
+    torch.cuda.synchronize()
+    got = host(out).view(np.float16).astype(np.float64)
+    sample = [0, 31, 32, 500, 1023]
     futs = {t: pool().submit(_oracle_token, q64[0, t], pk[0], nk[0], pv[0], nv[0], L - T + t,
                              gqa, bk, bv, seed) for t in sample}
     for t, f in futs.items():

@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol():
 def test_abi_version_and_status_strings():
     hdr = open(os.path.join(ROOT, "include", "tq.h")).read()
     assert tq.tq_abi_version() == int(re.search(r"#define TQ_ABI_VERSION (\d+)", hdr).group(1))
-    assert tq.tq_abi_version() == 5
+    assert tq.tq_abi_version() == 6
     assert tq.status_string(0) == "TQ_OK"
     assert tq.status_string(2) == "TQ_ERR_UNSUPPORTED"
 
