@@ -240,3 +240,32 @@ def _qjl_scores(**kw):
 ])
 def test_qjl_scores_validation(kw, want):
     assert _qjl_scores(**kw) == want
+
+
+def _prefill_split(**kw):
+    a = dict(q=FAKE, n=2, ws=FAKE, wsb=1 << 30, d=128, ntok=16)
+    a.update(kw)
+    return tq.lib().tq_prefill_attend_split(a["q"], tq.TQ_F16, FAKE, FAKE, FAKE, FAKE, FAKE, 1,
+                                            a["ntok"], 8, 4, a["d"], 4, 2, 0, 256, a["n"],
+                                            a["ws"], a["wsb"], None, FAKE, tq.TQ_F32, 0)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(n=0), tq.TQ_ERR_INVALID_ARG),
+    (dict(n=9), tq.TQ_ERR_INVALID_ARG),                  # at most 8 splits
+    (dict(ws=None), tq.TQ_ERR_INVALID_ARG),              # splits need a workspace
+    (dict(ws=FAKE + 8), tq.TQ_ERR_INVALID_ARG),          # 16-byte aligned
+    (dict(wsb=1024), tq.TQ_ERR_INVALID_ARG),             # too small
+    (dict(d=64), tq.TQ_ERR_UNSUPPORTED),                 # prefill is built for d = 128
+    (dict(q=None), tq.TQ_ERR_INVALID_ARG),
+])
+def test_prefill_split_validation(kw, want):
+    assert _prefill_split(**kw) == want
+
+
+def test_prefill_workspace_size_and_split_choice():
+    assert tq.tq_prefill_workspace_size(2, 16, 8, 128, 3) == 3 * 2 * 16 * 8 * 130 * 4
+    assert tq.tq_prefill_workspace_size(2, 16, 8, 128, 1) == 0
+    assert tq.tq_prefill_workspace_size(2, 16, 8, 96, 3) == 0
+    assert 1 <= tq.tq_prefill_splits(1, 1024, 32, 4) <= 8
+    assert tq.tq_prefill_splits(0, 1024, 32, 4) == 1
