@@ -77,6 +77,7 @@ constexpr int kMiscLast = 8;     // last-CTA flag
 constexpr int kMiscNB = 9;       // flat block count (lo, hi), common length
 constexpr int kMiscState = 12;   // scan state: sb, sP (lo, hi)
 constexpr int kMiscQInv = 16;    // 8 floats: 1/(query scale · kKScale)
+constexpr int kMiscApp = 24;     // decode-step append: segment count + 1 once encoded
 constexpr int kMiscM = 32;       // 8 floats: merged max
 constexpr int kMiscL = 40;       // 8 floats: merged sum
 constexpr int kMiscCb = 64;      // 32 words: staged codebooks
@@ -205,6 +206,16 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity) {
   const long long t0 = clock64();
   while (!mbar_try(bar, parity))
     if (clock64() - t0 > kWaitLimitCycles) return false;
+  return true;
+}
+// Waits (bounded, out of line) until the shared word at `flag` equals
+// `want`; false if it does not within kWaitLimitCycles.
+__device__ __noinline__ bool wait_flag_slow(const int* flag, int want) {
+  const long long t0 = clock64();
+  while (*reinterpret_cast<const volatile int*>(flag) != want) {
+    if (clock64() - t0 > kWaitLimitCycles) return false;
+    __nanosleep(64);
+  }
   return true;
 }
 // Waits for the phase with the given parity to complete; false if it does
@@ -543,6 +554,7 @@ attend_kernel(const __grid_constant__ AttendArgs a,
       misc[kMiscState + 1] = 0;
       misc[kMiscState + 2] = 0;
       misc[kMiscSeg + 3] = 0;
+      misc[kMiscApp] = 0;
     }
     __syncwarp();
     const int ge = effective_ctas(nbt, common);
@@ -627,6 +639,7 @@ attend_kernel(const __grid_constant__ AttendArgs a,
   };
 
   bool first = true;
+  int seg_iter = 0;                                   // segments this CTA has done
   while (pos < r1) {
     if (!first) {
       if (warp == 0) find_segment(pos, r1);
@@ -776,19 +789,37 @@ attend_kernel(const __grid_constant__ AttendArgs a,
       }
       fill_ring();
     }
-    // ---- decode-step append: the warp whose range ends at the sequence's
-    // last position encodes the new token of (b, g) (lanes 0-3: K, 4-7: V;
-    // the encode kernel's per-vector code), stores it in cache row L - 1 and
-    // keeps a copy to patch into its staged last chunk.
-    const bool app = a.new_kv != nullptr && blk0 + nseg == nbl && nw > 0 && wp1 == L;
+    // ---- decode-step append. The owner warp (its range ends at the
+    // sequence's last position) patches the new row into its staged last
+    // chunk. The encode of the new token of (b, g) (lanes 0-3: K, 4-7: V;
+    // the encode kernel's per-vector code), the store of cache row L - 1 and
+    // the copy for the patch are done by a helper warp with the fewest
+    // blocks, which hands the row over through shared memory.
+    const bool app_cta = a.new_kv != nullptr && blk0 + nseg == nbl && sp1 == L && nun > 0;
+    const bool app = app_cta && nw > 0 && wp1 == L;
+    int helper = -1;
+    if (app_cta) {
+      int owner_w = 0, best = 1 << 30;
+#pragma unroll 1
+      for (int w = 0; w < kWarps; ++w)
+        if ((long long)nun * (w + 1) / kWarps > (long long)nun * w / kWarps) owner_w = w;
+#pragma unroll 1
+      for (int w = 0; w < kWarps; ++w) {
+        const int cw = (int)((long long)nun * (w + 1) / kWarps - (long long)nun * w / kWarps);
+        if (w != owner_w && cw < best) {
+          best = cw;
+          helper = w;
+        }
+      }
+      if (helper < 0) helper = owner_w;
+    }
     uint8_t* app_k = smem + Gm::APPOFF;
     uint8_t* app_v = app_k + D / 2;
     uint16_t* app_n = reinterpret_cast<uint16_t*>(app_k + D);
     __syncthreads();
-    // The owner warp encodes after the CTA barrier: no other warp needs the
-    // new row (only this warp's last chunk holds position L - 1), and the
-    // encode overlaps the wait for the warp's first staged chunk.
-    if (app) {
+    // The helper encodes after the CTA barrier: only the owner needs the new
+    // row, for its last chunk, and the helper has the fewest blocks.
+    if (app_cta && warp == helper) {
       constexpr int LPV = D / 32;                     // lanes per vector
       if (lane < 2 * LPV) {
         const int sub = lane & (LPV - 1);
@@ -815,6 +846,8 @@ attend_kernel(const __grid_constant__ AttendArgs a,
       if (lane == 0) {
         a.norms_k[row] = app_n[0];
         a.norms_v[row] = app_n[1];
+        __threadfence_block();                        // the row before the flag
+        *reinterpret_cast<volatile int*>(misc + kMiscApp) = seg_iter + 1;
       }
     }
 
@@ -853,6 +886,13 @@ attend_kernel(const __grid_constant__ AttendArgs a,
       const int cend = min(wp1, t0 + kBlk);
       const bool partial = cend < t0 + kBlk;
       if (app && cend == L) {                       // the staged row L - 1 is stale
+        if (lane == 0) {                              // wait (bounded) for the helper
+          if (*reinterpret_cast<volatile int*>(misc + kMiscApp) != seg_iter + 1 &&
+              !wait_flag_slow(misc + kMiscApp, seg_iter + 1) && a.dev_status)
+            atomicOr(a.dev_status, TQ_DEV_WAIT_TIMEOUT);
+          __threadfence_block();
+        }
+        __syncwarp();
         const int r = L - 1 - t0;
         for (int w = lane; w < Gm::RK / 4; w += 32)
           *reinterpret_cast<uint32_t*>(smem + st + r * Gm::RK + 4 * w) =
@@ -1220,6 +1260,7 @@ attend_kernel(const __grid_constant__ AttendArgs a,
       }
     }
     pos += nseg;
+    ++seg_iter;
     __syncthreads();                                  // misc / fin / q~ reuse
   }
 
