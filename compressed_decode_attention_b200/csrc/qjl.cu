@@ -22,7 +22,8 @@
 // tq_qjl_scores (qjl_scores_kernel): a CTA takes up to 1024 positions of one
 //   (sequence, kv head). Its prologue rotates the GQA group's queries and
 //   forms p = S·q~ (one warp per output row of S, coalesced); then every
-//   thread scores its positions against the group from shared memory.
+//   thread scores two positions at a time against the group, reading the
+//   group's weights as 16-byte shared-memory broadcasts.
 #include <math.h>
 
 #include "encode_common.cuh"
@@ -32,7 +33,15 @@ namespace {
 
 constexpr int kQjlTokens = 64;        // tokens per encode CTA
 constexpr int kQjlThreads = 256;
-constexpr int kScorePositions = 1024; // positions per scores CTA
+#ifndef TQ_SCORE_THREADS
+#define TQ_SCORE_THREADS 256
+#endif
+#ifndef TQ_SCORE_POSITIONS
+#define TQ_SCORE_POSITIONS 512
+#endif
+constexpr int kScoreThreads = TQ_SCORE_THREADS;     // threads per scores CTA
+constexpr int kScorePositions = TQ_SCORE_POSITIONS; // positions per scores CTA
+static_assert(kScorePositions % kScoreThreads == 0, "whole positions per thread");
 
 // ------------------------------------------------------------------ encode
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -238,12 +247,12 @@ qjl_encode_kernel(const __grid_constant__ QjlEncodeArgs a,
 
 // ------------------------------------------------------------------ scores
 template <int D, int BITS, int GMAX>
-__global__ void __launch_bounds__(kQjlThreads)
+__global__ void __launch_bounds__(kScoreThreads)
 qjl_scores_kernel(const __grid_constant__ QjlScoresArgs a,
                   const __grid_constant__ Codebook cb,
                   const __grid_constant__ SignMask sm) {
   constexpr int Q = D / 32;
-  constexpr int NW = kQjlThreads / 32;
+  constexpr int NW = kScoreThreads / 32;
   constexpr int ROWB = D * BITS / 8;                // packed row bytes
   __shared__ __align__(16) float qt[GMAX][D];       // q~ = R·q
   __shared__ __align__(16) float qs[GMAX][D];       // q~ / d: stage-1 weights
@@ -294,89 +303,158 @@ qjl_scores_kernel(const __grid_constant__ QjlScoresArgs a,
     }
   }
   __syncthreads();
-  // ps = 2·scale·S·q~: warp w takes rows w, w + NW, ...; lanes split a row
-  // (coalesced reads of S); the butterfly leaves the sum in every lane
+  // ps = 2·scale·S·q~: thread (o, j) takes row o of S against heads j·HPT ..
+  // (j + 1)·HPT - 1. The row's 16-byte loads are independent of each other
+  // (one round trip to L2, not one per row); q~ is read as broadcasts.
   const float scale = sqrtf(0.5f * 3.14159265358979f) / ((float)D * sqrtf((float)D));
-  for (int o = warp; a.with_sketch && o < D; o += NW) {
-    float part[GMAX];
+  constexpr int TPR = kScoreThreads >= D ? kScoreThreads / D : 1;   // threads per row of S
+  constexpr int HPT = (GMAX + TPR - 1) / TPR;                     // heads per thread
+  for (int e = tid; a.with_sketch && e < D * TPR; e += kScoreThreads) {
+    const int o = e / TPR, h0 = (e % TPR) * HPT;
+    const float4* srow = reinterpret_cast<const float4*>(a.S + (size_t)o * D);
+    float part[HPT];
 #pragma unroll
-    for (int hh = 0; hh < GMAX; ++hh) part[hh] = 0.f;
+    for (int k = 0; k < HPT; ++k) part[k] = 0.f;
+#pragma unroll 8
+    for (int j4 = 0; j4 < D / 4; ++j4) {
+      const float4 s4 = __ldg(srow + j4);
 #pragma unroll
-    for (int k = 0; k < Q; ++k) {
-      const int j = lane + 32 * k;
-      const float s = __ldg(a.S + (size_t)o * D + j);
-#pragma unroll
-      for (int hh = 0; hh < GMAX; ++hh) part[hh] = fmaf(s, qt[hh][j], part[hh]);
+      for (int k = 0; k < HPT; ++k) {
+        if (h0 + k < GMAX) {
+          const float4 q4 = reinterpret_cast<const float4*>(&qt[h0 + k][0])[j4];
+          part[k] = fmaf(s4.x, q4.x, part[k]);
+          part[k] = fmaf(s4.y, q4.y, part[k]);
+          part[k] = fmaf(s4.z, q4.z, part[k]);
+          part[k] = fmaf(s4.w, q4.w, part[k]);
+        }
+      }
     }
 #pragma unroll
-    for (int hh = 0; hh < GMAX; ++hh) {
-      float v = part[hh];
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
-      if (lane == 0) ps[hh][o] = 2.f * scale * v;
-    }
+    for (int k = 0; k < HPT; ++k)
+      if (h0 + k < GMAX) ps[h0 + k][o] = 2.f * scale * part[k];
   }
   __syncthreads();
-  if (a.with_sketch && warp < GMAX) {               // sum_i p_i (the -1 half of 2b - 1)
+  for (int hh = warp; a.with_sketch && hh < GMAX; hh += NW) {   // sum_i p_i (the -1 half of 2b - 1)
     float v = 0.f;
-    for (int i = lane; i < D; i += 32) v += ps[warp][i];
+    for (int i = lane; i < D; i += 32) v += ps[hh][i];
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
-    if (lane == 0) psum[warp] = 0.5f * v;
+    if (lane == 0) psum[hh] = 0.5f * v;
   }
   __syncthreads();
 
-  // ---- one position per thread:
+  // ---- PP positions per thread (t, t + kScoreThreads, ...), so each
+  // 16-byte broadcast read of qs / ps serves all of them:
   //   score = nK·sum_i qs_i·c[idx_i] + gamma·(sum_{bit_i = 1} ps_i - psum)
+  // Every sum runs over i in ascending order, as in a one-position loop.
   const size_t hrow = ((size_t)b * a.n_kv_heads + g) * a.cap_tok;
   const int tend = min(L, t0 + kScorePositions);
-  for (int t = t0 + tid; t < tend; t += kQjlThreads) {
-    const size_t row = hrow + t;
-    uint32_t w[ROWB / 4];
-    {
-      const uint2* pr = reinterpret_cast<const uint2*>(a.packed_k + row * ROWB);
+  const float4* qs4 = reinterpret_cast<const float4*>(&qs[0][0]);
+  const float4* ps4 = reinterpret_cast<const float4*>(&ps[0][0]);
+  constexpr int PP = kScorePositions / kScoreThreads;
+  for (int tb = t0 + tid; tb < tend; tb += PP * kScoreThreads) {
+    bool ok[PP];
+    size_t row[PP];
+    uint32_t w[PP][ROWB / 4];
+    float nk[PP];
+#pragma unroll
+    for (int u = 0; u < PP; ++u) {
+      const int t = tb + u * kScoreThreads;
+      ok[u] = t < tend;
+      row[u] = hrow + (ok[u] ? t : tb);             // a valid row either way
+      const uint2* pr = reinterpret_cast<const uint2*>(a.packed_k + row[u] * ROWB);
 #pragma unroll
       for (int k = 0; k < ROWB / 8; ++k) {
         const uint2 v = __ldg(pr + k);
-        w[2 * k] = v.x;
-        w[2 * k + 1] = v.y;
+        w[u][2 * k] = v.x;
+        w[u][2 * k + 1] = v.y;
+      }
+      nk[u] = __half2float(__ushort_as_half(a.norms_k[row[u]]));
+    }
+    float s1[PP][GMAX];
+#pragma unroll
+    for (int u = 0; u < PP; ++u)
+#pragma unroll
+      for (int hh = 0; hh < GMAX; ++hh) s1[u][hh] = 0.f;
+#pragma unroll
+    for (int i4 = 0; i4 < D / 4; ++i4) {
+      float c[PP][4];
+#pragma unroll
+      for (int u = 0; u < PP; ++u)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) c[u][e] = cs[field<BITS>(w[u], 4 * i4 + e)];
+#pragma unroll
+      for (int hh = 0; hh < GMAX; ++hh) {
+        const float4 q = qs4[hh * (D / 4) + i4];
+#pragma unroll
+        for (int u = 0; u < PP; ++u) {
+          s1[u][hh] = fmaf(q.x, c[u][0], s1[u][hh]);
+          s1[u][hh] = fmaf(q.y, c[u][1], s1[u][hh]);
+          s1[u][hh] = fmaf(q.z, c[u][2], s1[u][hh]);
+          s1[u][hh] = fmaf(q.w, c[u][3], s1[u][hh]);
+        }
       }
     }
-    const float nk = __half2float(__ushort_as_half(a.norms_k[row]));
-    float s1[GMAX], s2[GMAX];
+    float score[PP][GMAX];
 #pragma unroll
-    for (int hh = 0; hh < GMAX; ++hh) s1[hh] = s2[hh] = 0.f;
+    for (int u = 0; u < PP; ++u)
 #pragma unroll
-    for (int i = 0; i < D; ++i) {
-      const float c = cs[field<BITS>(w, i)];
-#pragma unroll
-      for (int hh = 0; hh < GMAX; ++hh) s1[hh] = fmaf(qs[hh][i], c, s1[hh]);
-    }
-    float score[GMAX];
-#pragma unroll
-    for (int hh = 0; hh < GMAX; ++hh) score[hh] = nk * s1[hh];
+      for (int hh = 0; hh < GMAX; ++hh) score[u][hh] = nk[u] * s1[u][hh];
     if (a.with_sketch) {
-      uint32_t sk[D / 32];
-      const uint2* pk = reinterpret_cast<const uint2*>(a.sketch + row * (D / 8));
+      uint32_t sk[PP][D / 32];
+      float gm[PP];
 #pragma unroll
-      for (int k = 0; k < D / 64; ++k) {
-        const uint2 v = __ldg(pk + k);
-        sk[2 * k] = v.x;
-        sk[2 * k + 1] = v.y;
+      for (int u = 0; u < PP; ++u) {
+        const uint2* pk = reinterpret_cast<const uint2*>(a.sketch + row[u] * (D / 8));
+#pragma unroll
+        for (int k = 0; k < D / 64; ++k) {
+          const uint2 v = __ldg(pk + k);
+          sk[u][2 * k] = v.x;
+          sk[u][2 * k + 1] = v.y;
+        }
+        gm[u] = __half2float(__ushort_as_half(a.gamma[row[u]]));
       }
-      const float gm = __half2float(__ushort_as_half(a.gamma[row]));
+      float s2[PP][GMAX];
 #pragma unroll
-      for (int i = 0; i < D; ++i) {
-        const float bit = ((sk[i >> 5] >> (i & 31)) & 1u) ? 1.f : 0.f;
+      for (int u = 0; u < PP; ++u)
 #pragma unroll
-        for (int hh = 0; hh < GMAX; ++hh) s2[hh] = fmaf(bit, ps[hh][i], s2[hh]);
+        for (int hh = 0; hh < GMAX; ++hh) s2[u][hh] = 0.f;
+#pragma unroll
+      for (int i4 = 0; i4 < D / 4; ++i4) {
+        float bit[PP][4];
+#pragma unroll
+        for (int u = 0; u < PP; ++u)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 4 * i4 + e;
+            bit[u][e] = ((sk[u][i >> 5] >> (i & 31)) & 1u) ? 1.f : 0.f;
+          }
+#pragma unroll
+        for (int hh = 0; hh < GMAX; ++hh) {
+          const float4 pv = ps4[hh * (D / 4) + i4];
+#pragma unroll
+          for (int u = 0; u < PP; ++u) {
+            s2[u][hh] = fmaf(bit[u][0], pv.x, s2[u][hh]);
+            s2[u][hh] = fmaf(bit[u][1], pv.y, s2[u][hh]);
+            s2[u][hh] = fmaf(bit[u][2], pv.z, s2[u][hh]);
+            s2[u][hh] = fmaf(bit[u][3], pv.w, s2[u][hh]);
+          }
+        }
       }
 #pragma unroll
-      for (int hh = 0; hh < GMAX; ++hh) score[hh] = fmaf(gm, s2[hh] - psum[hh], score[hh]);
+      for (int u = 0; u < PP; ++u)
+#pragma unroll
+        for (int hh = 0; hh < GMAX; ++hh)
+          score[u][hh] = fmaf(gm[u], s2[u][hh] - psum[hh], score[u][hh]);
     }
 #pragma unroll
-    for (int hh = 0; hh < GMAX; ++hh)
-      if (hh < G) a.out[((size_t)b * a.n_q_heads + (size_t)g * G + hh) * a.cap_tok + t] = score[hh];
+    for (int u = 0; u < PP; ++u) {
+      if (!ok[u]) continue;
+      const int t = tb + u * kScoreThreads;
+#pragma unroll
+      for (int hh = 0; hh < GMAX; ++hh)
+        if (hh < G) a.out[((size_t)b * a.n_q_heads + (size_t)g * G + hh) * a.cap_tok + t] = score[u][hh];
+    }
   }
 }
 
@@ -424,7 +502,7 @@ cudaError_t launch_scores_dbg(const QjlScoresArgs& a, const Codebook& cb, const 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((a.cap_tok + kScorePositions - 1) / kScorePositions, a.n_kv_heads,
                      a.batch);
-  cfg.blockDim = dim3(kQjlThreads);
+  cfg.blockDim = dim3(kScoreThreads);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
