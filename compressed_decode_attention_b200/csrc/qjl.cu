@@ -19,11 +19,13 @@
 //      Ahi·Bhi + Ahi·Blo + Alo·Bhi (~22 significant bits); S staged 64
 //      columns at a time as fp16 high/low [output][column] tiles. Warp
 //      ballots of the accumulator signs give the row bytes.
-// tq_qjl_scores (qjl_scores_kernel): a CTA takes up to 1024 positions of one
+// tq_qjl_scores (qjl_scores_kernel): a CTA takes up to 512 positions of one
 //   (sequence, kv head). Its prologue rotates the GQA group's queries and
-//   forms p = S·q~ (one warp per output row of S, coalesced); then every
-//   thread scores two positions at a time against the group, reading the
-//   group's weights as 16-byte shared-memory broadcasts.
+//   forms p = S·q~ (a thread per row of S and group of heads); then every
+//   thread scores two positions against the group, reading the group's
+//   weights as 16-byte shared-memory broadcasts. Measured: 256 or 128
+//   positions per CTA repeat the prologue too often, 1024 leave too few
+//   CTAs for the latency-bound loop.
 #include <math.h>
 
 #include "encode_common.cuh"
@@ -33,14 +35,8 @@ namespace {
 
 constexpr int kQjlTokens = 64;        // tokens per encode CTA
 constexpr int kQjlThreads = 256;
-#ifndef TQ_SCORE_THREADS
-#define TQ_SCORE_THREADS 256
-#endif
-#ifndef TQ_SCORE_POSITIONS
-#define TQ_SCORE_POSITIONS 512
-#endif
-constexpr int kScoreThreads = TQ_SCORE_THREADS;     // threads per scores CTA
-constexpr int kScorePositions = TQ_SCORE_POSITIONS; // positions per scores CTA
+constexpr int kScoreThreads = 256;     // threads per scores CTA
+constexpr int kScorePositions = 512;   // positions per scores CTA
 static_assert(kScorePositions % kScoreThreads == 0, "whole positions per thread");
 
 // ------------------------------------------------------------------ encode
