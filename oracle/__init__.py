@@ -22,6 +22,10 @@ Modules:
   codebook   Lloyd-Max quantizer for N(0,1)
   rotation   SplitMix64 sign vector, Sylvester Hadamard matrix, rotation
   codec      norm / rotate / index / pack, unpack / dequantize
-  attention  compressed-domain decode attention with the sparse-V gate
+  attention  compressed-domain decode attention with the sparse-V gate, the
+             per-slice log-sum-exp records of a split context and their
+             combine
+  qjl        stage-2 residual sketch of the keys and the unbiased score
+             estimate
 """
-from . import codebook, rotation, codec, attention  # noqa: F401
+from . import codebook, rotation, codec, attention, qjl  # noqa: F401
