@@ -152,3 +152,41 @@ def test_sketch_of_the_unrotated_residual(monkeypatch):
     import test_oracle_qjl as tq
     _fails(tq.test_residual_is_the_original_space_difference)
     _fails(tq.test_rotated_sketch_equals_original_space_sketch_with_S_R)
+
+
+def test_centroid_at_cell_midpoint(monkeypatch):
+    # the centroid step takes the middle of the cell instead of E[X | cell]
+    def midpoint(a, b):
+        return a + 1.0 if b == float("inf") else 0.5 * (a + b)
+    monkeypatch.setattr(codebook, "cell_centroid", midpoint)
+    monkeypatch.setattr(codec, "_CB_CACHE", {})
+    _fails(tcb.test_matches_max_1960_table, 3)
+
+
+def test_dequant_without_the_norm(monkeypatch):
+    # the original-space reconstruction forgets to scale the unit vector
+    monkeypatch.setattr(codec, "dequant", lambda idx, nb, bits, seed:
+                        rotation.unrotate(codec.dequant_rotated(idx, bits), seed))
+    _fails(tc.test_codec_statistics_match_printed_benchmark, 4)
+
+
+def test_gated_positions_dropped_from_the_sum(monkeypatch):
+    # the softmax sum runs over the positions that pass the gate only
+    def dropped(qs, idx_k, nk_bits, idx_v, nv_bits, bits_k, bits_v, seed, tau):
+        qs = np.asarray(qs, dtype=np.float64)
+        g, d = qs.shape
+        L = idx_k.shape[0]
+        nk = np.asarray(nk_bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+        nv = np.asarray(nv_bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+        s = (rotation.rotate(qs, seed) @ codec.dequant_rotated(idx_k, bits_k).T) * nk / np.sqrt(d)
+        w = np.exp(s - s.max(axis=1, keepdims=True))
+        nblk = (L + attention.GATE_BLOCK - 1) // attention.GATE_BLOCK
+        pad = np.full((g, nblk * attention.GATE_BLOCK), -np.inf)
+        pad[:, :L] = s
+        mblk = pad.reshape(g, nblk, attention.GATE_BLOCK).max(axis=2)
+        gated = np.exp(s - np.repeat(mblk, attention.GATE_BLOCK, axis=1)[:, :L]) < tau
+        kept = np.where(gated, 0.0, w)
+        acc = (kept * nv) @ codec.dequant_rotated(idx_v, bits_v)
+        return rotation.unrotate(acc / kept.sum(axis=1, keepdims=True), seed), gated
+    monkeypatch.setattr(attention, "attend_head_group", dropped)
+    _fails(ta.test_gate_matches_brute_force, 0.05)
