@@ -56,6 +56,11 @@ METRIC = "decode-attn packed-KV GB/s & % HBM roofline; encode Mtok/s (1×B200)"
 WORKLOAD = "llama3_8b_decode"
 ENCODE_WORKLOAD = "bulk_prefill_encode"
 BATCHED_WORKLOAD = "batched_serving"
+QWEN_WORKLOAD = "qwen14b_decode"
+QWEN_LAYERS = 8          # long-context measurement: distinct layer caches (705 MB > L2)
+# The pages' codec figures for random vectors (TQAI §The CLI), beside ours.
+PAGES_CODEC = {"k4": {"nmse": 0.009287, "snr_db": 20.3, "cos": 0.9954},
+               "v2": {"nmse": 0.115653, "snr_db": 9.4, "cos": 0.9408}}
 LAYERS = 32
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
@@ -240,15 +245,58 @@ class LayerCaches:
 
 
 def device_kv(w, layer, n_tok, gen):
-    """fp16 K/V [2][n][H][d] on the device: N(0,1) with the workload's x20
-    outlier K channels (same recipe as synthetic.kv_f32, torch's generator)."""
+    """K/V [2][n][H][d] as 16-bit patterns of the workload's dtype on the
+    device: N(0,1), with the workload's outlier K channels (x20, or values
+    replaced by Laplace(0,1) draws); the recipe of synthetic.kv_f32 drawn
+    with torch's generator."""
     import torch
     x = torch.randn((2, n_tok, w.n_kv_heads, w.d), generator=gen, device="cuda",
                     dtype=torch.float32)
     ch = S.outlier_channels(w, layer)
     for h in range(w.n_kv_heads):
-        x[0, :, h, torch.as_tensor(ch[h], device="cuda")] *= 20.0
-    return x.half().view(torch.int16)
+        idx = torch.as_tensor(ch[h], device="cuda")
+        if w.outlier == "x20":
+            x[0, :, h, idx] *= 20.0
+        elif w.outlier == "laplace":        # inverse CDF of Laplace(0, 1)
+            u = torch.rand((n_tok, len(ch[h])), generator=gen, device="cuda") - 0.5
+            x[0, :, h, idx] = -torch.sign(u) * torch.log1p(-2.0 * u.abs())
+    return (x.bfloat16() if w.dtype == "bf16" else x.half()).view(torch.int16)
+
+
+class Nvtx:
+    """NVTX range around a timed region (visible in profilers; no effect
+    on the timing)."""
+
+    def __init__(self, name):
+        self.name = name
+
+    def __enter__(self):
+        import torch
+        torch.cuda.nvtx.range_push(self.name)
+        return self
+
+    def __exit__(self, *exc):
+        import torch
+        torch.cuda.nvtx.range_pop()
+
+
+def codec_quality(x16, dtype, xhat, nhat):
+    """Sums over vectors of the codec's errors, on the device.
+
+    x16: [n][H][d] 16-bit patterns of the encoder input; xhat: [H][n][d]
+    float32 from tq_dequant (original domain); nhat: [H][n] stored fp16 norms.
+    Returns (rotated-domain squared error ||y - y^||^2 with y = R x/||x||
+    and y^ the codebook point, which equals ||x/||x|| - x^/n^||^2 since R is
+    orthonormal; NMSE ||x - x^||^2/||x||^2; cosine) summed over vectors."""
+    import torch
+    x = (x16.view(torch.bfloat16) if dtype == "bf16" else x16.view(torch.float16)).float()
+    x = x.permute(1, 0, 2)
+    nx = x.norm(dim=-1, keepdim=True)
+    nh = nhat.view(torch.float16).float().unsqueeze(-1)
+    rot = ((x / nx - xhat / nh) ** 2).sum(-1)
+    nmse = ((x - xhat) ** 2).sum(-1) / (nx.squeeze(-1) ** 2)
+    cos = (x * xhat).sum(-1) / (nx.squeeze(-1) * xhat.norm(dim=-1))
+    return float(rot.double().sum()), float(nmse.double().sum()), float(cos.double().sum())
 
 
 def run_gpu(args, rank, world, local_rank):
@@ -288,13 +336,64 @@ def run_gpu(args, rank, world, local_rank):
     barrier(device)
     torch.cuda.synchronize()
     e0.record(stream)
-    with torch.cuda.stream(stream):
+    with Nvtx("encode"), torch.cuda.stream(stream):
         for _ in range(enc_steps):
             encode_all()
     e1.record(stream)
     torch.cuda.synchronize()
     enc_ms = reduce_max(e0.elapsed_time(e1) / enc_steps, device)
     enc_launches = enc_steps * L
+
+    # ---------------- encode -> dequant round trip of the bulk workload: every
+    # layer's K and V dequantized to the original domain (tq_dequant, timed)
+    # and compared with the encoder input: the codec's quality
+    dq = torch.empty((H, ctx, d), dtype=torch.float32, device=device)
+    quality = {"k": [0.0, 0.0, 0.0], "v": [0.0, 0.0, 0.0]}
+    streams_ = (("k", 0, w.bits_k, caches.pk, caches.nk), ("v", 1, w.bits_v, caches.pv, caches.nv))
+    for l in range(L):
+        for name, which, bits, pks, nks in streams_:
+            with torch.cuda.stream(stream):
+                tq.tq_dequant(pks[l], nks[l], ctx, H, d, bits, seed, cap, 0, dq, stream)
+            stream.synchronize()
+            r = codec_quality(kv_all[l][which], we.dtype, dq, nks[l][0])
+            quality[name] = [a_ + b_ for a_, b_ in zip(quality[name], r)]
+
+    def dequant_all():
+        for l in range(L):
+            for name, which, bits, pks, nks in streams_:
+                tq.tq_dequant(pks[l], nks[l], ctx, H, d, bits, seed, cap, 0, dq, stream)
+
+    with torch.cuda.stream(stream):
+        dequant_all()
+    torch.cuda.synchronize()
+    dq0, dq1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(device)
+    torch.cuda.synchronize()
+    dq0.record(stream)
+    with Nvtx("dequant"), torch.cuda.stream(stream):
+        dequant_all()
+    dq1.record(stream)
+    torch.cuda.synchronize()
+    dq_ms = reduce_max(dq0.elapsed_time(dq1) / L, device)     # per layer, K and V
+    launches += 2 * L
+    n_vec = L * ctx * H
+    round_trip = {"workload": ENCODE_WORKLOAD, "vectors_per_stream": n_vec,
+                  "note": "rotated_mse = mean ||y - y^||^2 with y = R x/||x|| (per-coordinate "
+                          "MSE in N(0,1) units); K has 4 outlier channels x20 per head, so its "
+                          "rotated coordinates are not N(0,1) and its MSE departs from the "
+                          "codebook's; V is plain N(0,1)"}
+    for name, bits in (("k", w.bits_k), ("v", w.bits_v)):
+        rot, nmse, cos = (v_ / n_vec for v_ in quality[name])
+        dmse = tq.tq_build_codebook(bits, 1)[2]
+        round_trip[name] = {"bits": bits, "rotated_mse": round(rot, 6),
+                            "codebook_mse": round(dmse, 6), "ratio": round(rot / dmse, 4),
+                            "nmse": round(nmse, 6), "snr_db": round(-10 * np.log10(nmse), 2),
+                            "cos": round(cos, 5)}
+    round_trip["pages_random_vectors"] = dict(PAGES_CODEC, source="TQAI §The CLI")
+    round_trip["dequant_us_per_layer"] = round(dq_ms * 1e3, 2)
+    round_trip["dequant_gbs"] = round(H * ctx * ((w.d * (w.bits_k + w.bits_v)) // 8 + 4 + 2 * w.d * 4)
+                                      / (dq_ms * 1e-3) / 1e9, 1)
+    del dq
 
     # ---------------- stage-2 residual sketch (QJL) of the keys of QJL_LAYERS
     # layer caches, and the estimated scores of 32 query heads over them
@@ -456,7 +555,7 @@ def run_gpu(args, rank, world, local_rank):
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(device)
     torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clk:
+    with ClockSampler(local_rank) as clk, Nvtx("decode_step"):
         with torch.cuda.stream(stream):
             t0.record(stream)
             for _ in range(args.steps):
@@ -480,7 +579,7 @@ def run_gpu(args, rank, world, local_rank):
     a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(device)
     torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
+    with Nvtx("attend"), torch.cuda.stream(stream):
         a0.record(stream)
         for _ in range(args.steps):
             attend_graph.replay()
@@ -545,8 +644,8 @@ def run_gpu(args, rank, world, local_rank):
 
     # ---------------- attention at serving scale: the batched workload (64
     # sequences of U{1024..16384} positions, K4/V3, sparse-V gate 1e-6), two
-    # layer caches alternating (2 x 0.97 GB of capacity, > L2). The rows are
-    # random bytes and the norms random values near sqrt(d): timing only.
+    # layer caches alternating (2 x 0.97 GB of capacity, > L2), each encoded
+    # by tq_encode from the workload's recipe (N(0,1) fp16 K/V)
     wb = S.WORKLOADS[BATCHED_WORKLOAD]
     bctx_h = S.ctx_lens(wb)
     bctx = torch.from_numpy(bctx_h).to(device)
@@ -554,15 +653,17 @@ def run_gpu(args, rank, world, local_rank):
     brk, brv = d * wb.bits_k // 8, d * wb.bits_v // 8
     bcache = []
     for _ in range(2):
-        bpk = torch.randint(0, 256, (wb.batch, bH, bcap, brk), dtype=torch.uint8, device=device,
-                            generator=gen)
-        bpv = torch.randint(0, 256, (wb.batch, bH, bcap, brv), dtype=torch.uint8, device=device,
-                            generator=gen)
-        bnk = (11.3 + torch.randn((wb.batch, bH, bcap), generator=gen, device=device)) \
-            .half().view(torch.int16)
-        bnv = (11.3 + torch.randn((wb.batch, bH, bcap), generator=gen, device=device)) \
-            .half().view(torch.int16)
+        bpk = torch.zeros((wb.batch, bH, bcap, brk), dtype=torch.uint8, device=device)
+        bpv = torch.zeros((wb.batch, bH, bcap, brv), dtype=torch.uint8, device=device)
+        bnk = torch.zeros((wb.batch, bH, bcap), dtype=torch.int16, device=device)
+        bnv = torch.zeros((wb.batch, bH, bcap), dtype=torch.int16, device=device)
+        for b in range(wb.batch):
+            kvb = device_kv(wb, 0, int(bctx_h[b]), gen)
+            tq.tq_encode(kvb, tq.TQ_F16, int(bctx_h[b]), bH, d, wb.bits_k, wb.bits_v, seed,
+                         bpk[b], bpv[b], bnk[b], bnv[b], bcap, 0, status, stream)
+        torch.cuda.synchronize()
         bcache.append((bpk, bnk, bpv, bnv))
+    skipped = torch.zeros(1, dtype=torch.int64, device=device)
     bq = [torch.randn((wb.batch, bHq, d), generator=gen, device=device).half() for _ in range(2)]
     bout = torch.empty((wb.batch, bHq, d), dtype=torch.float16, device=device)
     bws_bytes = tq.tq_attend_workspace_size(wb.batch, bHq, bcap, d)
@@ -573,7 +674,7 @@ def run_gpu(args, rank, world, local_rank):
             bpk, bnk, bpv, bnv = bcache[i]
             tq.tq_attend(bq[i], tq.TQ_F16, bpk, bnk, bpv, bnv, bctx, wb.batch, bHq, wb.gqa, d,
                          wb.bits_k, wb.bits_v, seed, bcap, wb.tau, 0, bws, bws_bytes, bout,
-                         tq.TQ_F16, dev_status=status, stream=stream)
+                         tq.TQ_F16, dev_status=status, sparse_v_skipped=skipped, stream=stream)
 
     bgraph = capture(batched_all)
     for _ in range(args.warmup):
@@ -582,7 +683,8 @@ def run_gpu(args, rank, world, local_rank):
     b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(device)
     torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
+    skipped.zero_()
+    with Nvtx("batched"), torch.cuda.stream(stream):
         b0.record(stream)
         for _ in range(args.steps):
             bgraph.replay()
@@ -590,9 +692,57 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize()
     batched_ms = reduce_max(b0.elapsed_time(b1) / (2 * args.steps), device)
     launches += 2 * args.steps
+    batched_skipped = int(skipped.item()) // args.steps
     batched_bytes = int(bctx_h.astype(np.int64).sum()) * bH * (brk + brv + 4) + \
         wb.batch * bHq * d * (2 + 2)
     del bgraph, bcache, bq, bout, bws
+    torch.cuda.empty_cache()
+
+    # ---------------- the Qwen-14B-shaped long-context layer (40 q / 8 kv
+    # heads, GQA 5, ctx 131072, K3/V2, bf16 with Laplace(0,1) values on 3 K
+    # channels per head): QWEN_LAYERS layer caches encoded by tq_encode from
+    # the recipe, a CUDA graph of their tq_attend launches (time / layers)
+    wq = S.WORKLOADS[QWEN_WORKLOAD]
+    QLAY = min(QWEN_LAYERS, L)
+    qcache = LayerCaches(wq, QLAY, stream)
+    for l in range(QLAY):
+        kvq = device_kv(wq, l, wq.ctx, gen)
+        tq.tq_encode(kvq, tq.TQ_BF16, wq.ctx, wq.n_kv_heads, d, wq.bits_k, wq.bits_v, seed,
+                     qcache.pk[l], qcache.pv[l], qcache.nk[l], qcache.nv[l], wq.cap_tok, 0,
+                     status, stream)
+        torch.cuda.synchronize()
+        del kvq
+    qw_q = torch.randn((QLAY, 1, wq.n_q_heads, d), generator=gen, device=device).bfloat16()
+    qw_out = torch.empty((QLAY, 1, wq.n_q_heads, d), dtype=torch.bfloat16, device=device)
+    qw_ctx = torch.full((1,), wq.ctx, dtype=torch.int32, device=device)
+    qw_wsb = tq.tq_attend_workspace_size(1, wq.n_q_heads, wq.cap_tok, d)
+    qw_ws = torch.zeros(qw_wsb, dtype=torch.uint8, device=device)
+
+    def qwen_all():
+        for l in range(QLAY):
+            tq.tq_attend(qw_q[l], tq.TQ_BF16, qcache.pk[l], qcache.nk[l], qcache.pv[l],
+                         qcache.nv[l], qw_ctx, 1, wq.n_q_heads, wq.gqa, d, wq.bits_k, wq.bits_v,
+                         seed, wq.cap_tok, 0.0, 0, qw_ws, qw_wsb, qw_out[l], tq.TQ_BF16,
+                         dev_status=status, stream=stream)
+
+    qgraph = capture(qwen_all)
+    for _ in range(args.warmup):
+        qgraph.replay()
+    torch.cuda.synchronize()
+    w0_, w1_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(device)
+    torch.cuda.synchronize()
+    with Nvtx("qwen14b"), torch.cuda.stream(stream):
+        w0_.record(stream)
+        for _ in range(args.steps):
+            qgraph.replay()
+        w1_.record(stream)
+    torch.cuda.synchronize()
+    qwen_ms = reduce_max(w0_.elapsed_time(w1_) / (QLAY * args.steps), device)
+    launches += QLAY * args.steps
+    qwen_bytes = attend_bytes(wq, wq.ctx)
+    del qgraph, qcache, qw_q, qw_out, qw_ws
+    torch.cuda.empty_cache()
 
     # ---------------- end to end: host inputs in, host output back, every step
     in_host = torch.empty(nq16 + nkv16, dtype=torch.int16).pin_memory()
@@ -614,7 +764,7 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier(device)
     x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
+    with Nvtx("e2e"), torch.cuda.stream(stream):
         x0.record(stream)
         for _ in range(args.steps):
             e2e_step()
@@ -643,15 +793,13 @@ def run_gpu(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f32",
+        "dtype": "f16",
+        "dtype_detail": "tensor-core mma.sync with fp16 operands and fp32 accumulation: scores "
+                        "from fp16 high+low pairs of the query and of the K codebook (~22 "
+                        "significant bits), P.V with fp16 weights x V norm and fp16 V levels; "
+                        "softmax, merges and the inverse rotation in fp32",
         "data": "synthetic (seeded N(0,1) fp16 K/V with x20 outlier K channels; torch generator on device)",
-        "config": {"workload": WORKLOAD, "layers": L, "batch": w.batch, "n_q_heads": w.n_q_heads,
-                   "n_kv_heads": H, "d": d, "ctx": ctx, "bits": f"K{w.bits_k}/V{w.bits_v}",
-                   "kv_dtype": "fp16", "q_out_dtype": "fp16", "per_gpu": "one model replica",
-                   "l2": f"inputs larger than L2: {L} distinct layer caches, "
-                         f"{L * per_layer_attend / 1e6:.0f} MB per step",
-                   "step": "per layer: tq_attend_append (append the new token, attend over "
-                           "ctx positions; one launch), CUDA graph"},
+        "config": config_of(w, L),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                      "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
@@ -714,12 +862,26 @@ def run_gpu(args, rank, world, local_rank):
             "workload": f"{BATCHED_WORKLOAD}: {wb.batch} sequences, ctx U{{{wb.ctx_range[0]}.."
                         f"{wb.ctx_range[1]}}}, {bHq} q / {bH} kv heads, d={d}, "
                         f"K{wb.bits_k}/V{wb.bits_v}, sparse-V gate {wb.tau}; 2 layer caches "
-                        "alternating (rows random bytes: timing only)",
+                        "alternating, each encoded by tq_encode from seeded N(0,1) fp16 K/V",
+            "sparse_v_skipped_per_call": batched_skipped,
             "us_per_call": round(batched_ms * 1e3, 2),
             "bytes_per_call": batched_bytes,
             "gbs": round(batched_bytes / (batched_ms * 1e-3) / 1e9, 1),
             "frac": round(batched_bytes / (batched_ms * 1e-3) / 1e9 / peak, 4),
             "frac_of_nominal_8tbs": round(batched_bytes / (batched_ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 4)},
+        "qwen14b": {
+            "workload": f"{QWEN_WORKLOAD}: batch 1, {wq.n_q_heads} q / {wq.n_kv_heads} kv heads "
+                        f"(GQA {wq.gqa}), d={d}, ctx {wq.ctx}, K{wq.bits_k}/V{wq.bits_v}, bf16 "
+                        f"q/K/V, Laplace(0,1) values on {wq.n_outlier} K channels per head; "
+                        f"{QLAY} distinct layer caches ({QLAY * qwen_bytes / 1e6:.0f} MB > L2), "
+                        "CUDA graph of their tq_attend launches",
+            "us_per_launch": round(qwen_ms * 1e3, 2),
+            "bytes_per_launch": qwen_bytes,
+            "roofline": {"bound": "hbm", "achieved": round(qwen_bytes / (qwen_ms * 1e-3) / 1e9, 1),
+                         "peak": peak, "unit": "GB/s",
+                         "frac": round(qwen_bytes / (qwen_ms * 1e-3) / 1e9 / peak, 4),
+                         "frac_of_nominal_8tbs": round(qwen_bytes / (qwen_ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 4)}},
+        "round_trip": round_trip,
         "context_parallel": {
             "slices": P, "emulated_on_one_gpu": True,
             "per_layer": f"{P} x tq_attend_partial over {ctx // P}-position slices + "
@@ -736,63 +898,102 @@ def run_gpu(args, rank, world, local_rank):
 
 
 # ------------------------------------------------------------------ CPU oracle arm
-def oracle_sample(budget_s=12.0):
+def config_of(w, layers):
+    """The `config` object of the bench line (shared by both arms)."""
+    return {"workload": WORKLOAD, "layers": layers, "batch": w.batch, "n_q_heads": w.n_q_heads,
+            "n_kv_heads": w.n_kv_heads, "d": w.d, "ctx": w.ctx,
+            "bits": f"K{w.bits_k}/V{w.bits_v}", "kv_dtype": "fp16", "q_out_dtype": "fp16",
+            "per_gpu": "one model replica",
+            "l2": f"inputs larger than L2: {layers} distinct layer caches, "
+                  f"{layers * attend_bytes(w, w.ctx) / 1e6:.0f} MB per step",
+            "step": "per layer: tq_attend_append (append the new token, attend over "
+                    "ctx positions; one launch), CUDA graph"}
+
+
+def oracle_sample(budget_s=12.0, threads=None):
     """Time the oracle on a bounded sample of the decode workload: whole
     (kv head, query group) units of one layer at full context, plus a block of
-    encode vectors. Returns dict with GB/s and Mtok/s on the same byte basis."""
+    encode vectors. `threads` caps numpy's BLAS pool (None: its default).
+    Returns GB/s on the bench's byte basis, the units and seconds timed."""
     import threadpoolctl
     from oracle import attention, codec
     w = S.WORKLOADS[WORKLOAD]
-    cores = max(i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()) \
-        if threadpoolctl.threadpool_info() else 1
-    # inputs (not timed): one kv head's K/V at full context, encoded by the oracle
-    kv = S.kv_bits(w, 0, w.ctx)[:, :, :1]
-    x_k = codec.promote(kv[0, :, 0], w.dtype)
-    x_v = codec.promote(kv[1, :, 0], w.dtype)
-    t = time.perf_counter()
-    rk, nk = codec.encode_rows(x_k, w.bits_k, S.SIGN_SEED)
-    rv, nv = codec.encode_rows(x_v, w.bits_v, S.SIGN_SEED)
-    enc_s = time.perf_counter() - t
-    enc_vecs = 2 * w.ctx
-    qb = S.query_bits(w)[:, :w.gqa]
-    q64 = codec.promote(qb, w.dtype)
-    units, att_s = 0, 0.0
-    while att_s < budget_s and units < 64:
+    with threadpoolctl.threadpool_limits(threads):
+        info = threadpoolctl.threadpool_info()
+        cores = max((i.get("num_threads", 1) for i in info), default=1)
+        # inputs (not timed): one kv head's K/V at full context
+        kv = S.kv_bits(w, 0, w.ctx)[:, :, :1]
+        x_k = codec.promote(kv[0, :, 0], w.dtype)
+        x_v = codec.promote(kv[1, :, 0], w.dtype)
         t = time.perf_counter()
-        attention.attend(q64, rk[None, None], nk[None, None], rv[None, None], nv[None, None],
-                         np.array([w.ctx]), w.gqa, w.bits_k, w.bits_v, S.SIGN_SEED)
-        att_s += time.perf_counter() - t
-        units += 1
+        rk, nk = codec.encode_rows(x_k, w.bits_k, S.SIGN_SEED)
+        rv, nv = codec.encode_rows(x_v, w.bits_v, S.SIGN_SEED)
+        enc_s = time.perf_counter() - t
+        enc_vecs = 2 * w.ctx
+        qb = S.query_bits(w)[:, :w.gqa]
+        q64 = codec.promote(qb, w.dtype)
+        units, att_s = 0, 0.0
+        while units < 1 or (att_s < budget_s and units < 64):
+            t = time.perf_counter()
+            attention.attend(q64, rk[None, None], nk[None, None], rv[None, None], nv[None, None],
+                             np.array([w.ctx]), w.gqa, w.bits_k, w.bits_v, S.SIGN_SEED)
+            att_s += time.perf_counter() - t
+            units += 1
     unit_bytes = w.ctx * (w.d * w.bits_k // 8 + w.d * w.bits_v // 8 + 4) + w.gqa * w.d * 4
     return {"attend_gbs": units * unit_bytes / att_s / 1e9, "attend_units": units,
-            "attend_s": att_s, "encode_mtoks": (enc_vecs / 2 / w.n_kv_heads) / enc_s / 1e6,
+            "attend_s": att_s, "encode_s": enc_s,
+            "encode_mtoks": (enc_vecs / 2 / w.n_kv_heads) / enc_s / 1e6,
             "encode_vectors_per_s": enc_vecs / enc_s, "cores": cores,
             "sample": f"{units} x (1 kv head + its {w.gqa} query heads, ctx {w.ctx}) attention; "
                       f"{enc_vecs} vector encodes"}
 
 
+def cpu_baseline_both(budget_s):
+    """The oracle timed single-threaded and with numpy's default thread pool."""
+    one = oracle_sample(budget_s / 2, threads=1)
+    allc = oracle_sample(budget_s / 2)
+    return {"value": round(allc["attend_gbs"], 4), "unit": "GB/s", "cores": allc["cores"],
+            "nproc": os.cpu_count(), "kind": "oracle", "sample": allc["sample"],
+            "encode_mtoks": round(allc["encode_mtoks"], 6),
+            "single_thread": {"value": round(one["attend_gbs"], 4), "unit": "GB/s", "threads": 1,
+                              "sample": one["sample"],
+                              "encode_mtoks": round(one["encode_mtoks"], 6)}}
+
+
 def run_reference(args, rank, world):
+    """The oracle as the reference arm. A step is one bounded sample of the
+    workload (see oracle_sample); value is GB/s over the timed samples and
+    ms_per_step the measured wall time of one sample step."""
     if rank != 0:
         return None
     w = S.WORKLOADS[WORKLOAD]
     per_step = []
     o = None
     for i in range(args.warmup + args.steps):
-        o = oracle_sample(budget_s=2.0)
+        t = time.perf_counter()
+        o = oracle_sample(budget_s=1.0)
+        o["step_s"] = time.perf_counter() - t
         if i >= args.warmup:
             per_step.append(o)
-    gbs = float(np.mean([p["attend_gbs"] for p in per_step]))
-    step_bytes = LAYERS * (attend_bytes(w, w.ctx) + encode_bytes(w, w.n_kv_heads))
+    att_bytes = sum(p["attend_units"] for p in per_step) * \
+        (w.ctx * (w.d * w.bits_k // 8 + w.d * w.bits_v // 8 + 4) + w.gqa * w.d * 4)
+    att_s = sum(p["attend_s"] for p in per_step)
+    gbs = att_bytes / att_s / 1e9
+    step_ms = 1e3 * float(np.mean([p["step_s"] for p in per_step]))
+    full_step_bytes = LAYERS * (attend_bytes(w, w.ctx) + encode_bytes(w, w.n_kv_heads))
     return {
         "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(step_bytes / (gbs * 1e9) * 1e3, 3), "higher_is_better": True,
+        "ms_per_step": round(step_ms, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "layers": LAYERS, "batch": w.batch,
-                   "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "d": w.d,
-                   "ctx": w.ctx, "bits": f"K{w.bits_k}/V{w.bits_v}"},
+        "config": config_of(w, LAYERS),
+        "step": "one bounded sample per step: " + o["sample"] + " (timed wall clock, host cores)",
+        "units_timed_per_step": {"attention_units": round(float(np.mean([p["attend_units"] for p in per_step])), 2),
+                                 "encode_vectors": 2 * w.ctx},
+        "projection_ms_per_full_decode_step": round(full_step_bytes / (gbs * 1e9) * 1e3, 1),
         "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": o["cores"],
-                         "kind": "oracle", "sample": "per step: " + o["sample"]},
+                         "nproc": os.cpu_count(), "kind": "oracle",
+                         "sample": "per step: " + o["sample"]},
         "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -823,10 +1024,7 @@ def main(argv=None):
     res = run_gpu(args, rank, world, local_rank)
     if rank == 0:
         if not args.no_cpu_baseline:
-            o = oracle_sample()
-            res["cpu_baseline"] = {"value": round(o["attend_gbs"], 4), "unit": "GB/s",
-                                   "cores": o["cores"], "kind": "oracle", "sample": o["sample"],
-                                   "encode_mtoks": round(o["encode_mtoks"], 6)}
+            res["cpu_baseline"] = cpu_baseline_both(16.0)
         print(json.dumps(res), flush=True)
     import torch.distributed as dist
     if dist.is_initialized():

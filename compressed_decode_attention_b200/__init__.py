@@ -38,51 +38,60 @@ def lib() -> ctypes.CDLL:
         if not os.path.exists(LIB_PATH):
             raise ImportError(f"{LIB_PATH} is not built; run "
                               "`python -m compressed_decode_attention_b200.build`")
-        L = ctypes.CDLL(LIB_PATH)
-        P, I, U64, SZ, F, D = (ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64,
-                               ctypes.c_size_t, ctypes.c_float, ctypes.POINTER(ctypes.c_double))
-        L.tq_abi_version.restype = I
-        L.tq_abi_version.argtypes = []
-        L.tq_status_string.restype = ctypes.c_char_p
-        L.tq_status_string.argtypes = [I]
-        L.tq_build_codebook.restype = I
-        L.tq_build_codebook.argtypes = [I, I, D, D, D]
-        L.tq_encode.restype = I
-        L.tq_encode.argtypes = [P, I, I, I, I, I, I, U64, P, P, P, P, I, I, P, P]
-        L.tq_dequant.restype = I
-        L.tq_dequant.argtypes = [P, P, I, I, I, I, U64, I, I, P, P]
-        L.tq_attend_workspace_size.restype = SZ
-        L.tq_attend_workspace_size.argtypes = [I, I, I, I]
-        L.tq_attend.restype = I
-        L.tq_attend.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F, I,
-                                P, SZ, P, P, P, I, P]
-        L.tq_attend_append.restype = I
-        L.tq_attend_append.argtypes = [P, I, P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F,
-                                       I, P, SZ, P, P, P, I, P]
-        L.tq_prefill_attend.restype = I
-        L.tq_prefill_attend.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, I, U64, I, P, P,
-                                        I, P]
-        L.tq_prefill_attend_split.restype = I
-        L.tq_prefill_attend_split.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, I, U64, I,
-                                              I, P, SZ, P, P, I, P]
-        L.tq_prefill_workspace_size.restype = SZ
-        L.tq_prefill_workspace_size.argtypes = [I, I, I, I, I]
-        L.tq_prefill_splits.restype = I
-        L.tq_prefill_splits.argtypes = [I, I, I, I]
-        L.tq_attend_partial.restype = I
-        L.tq_attend_partial.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F, I,
-                                        P, SZ, P, P, P, P]
-        L.tq_attend_combine.restype = I
-        L.tq_attend_combine.argtypes = [P, I, I, I, I, U64, P, P, I, P]
-        L.tq_qjl_encode.restype = I
-        L.tq_qjl_encode.argtypes = [P, I, I, I, I, I, U64, P, P, P, P, P, I, I, P, P]
-        L.tq_qjl_scores.restype = I
-        L.tq_qjl_scores.argtypes = [P, I, P, P, P, P, P, P, I, I, I, I, I, U64, I, I, P, P, P]
-        L.tq_attend_noalloc.restype = I
-        L.tq_attend_noalloc.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F, I,
-                                        P, P, P, I, P]
-        _lib = L
+        _lib = load_library(LIB_PATH)
     return _lib
+
+
+def load_library(path: str) -> ctypes.CDLL:
+    """Open a build of the library at `path` with the C ABI's argument types
+    declared (lib() uses it for libtq.so; tests use it for test builds)."""
+    L = ctypes.CDLL(path)
+    P, I, U64, SZ, F, D = (ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64,
+                           ctypes.c_size_t, ctypes.c_float, ctypes.POINTER(ctypes.c_double))
+    L.tq_abi_version.restype = I
+    L.tq_abi_version.argtypes = []
+    L.tq_status_string.restype = ctypes.c_char_p
+    L.tq_status_string.argtypes = [I]
+    L.tq_build_codebook.restype = I
+    L.tq_build_codebook.argtypes = [I, I, D, D, D]
+    L.tq_encode.restype = I
+    L.tq_encode.argtypes = [P, I, I, I, I, I, I, U64, P, P, P, P, I, I, P, P]
+    L.tq_dequant.restype = I
+    L.tq_dequant.argtypes = [P, P, I, I, I, I, U64, I, I, P, P]
+    L.tq_attend_workspace_size.restype = SZ
+    L.tq_attend_workspace_size.argtypes = [I, I, I, I]
+    L.tq_attend.restype = I
+    L.tq_attend.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F, I,
+                            P, SZ, P, P, P, I, P]
+    L.tq_attend_gate_counts.restype = I
+    L.tq_attend_gate_counts.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F, I,
+                                        P, SZ, P, P, P, P, I, P]
+    L.tq_attend_append.restype = I
+    L.tq_attend_append.argtypes = [P, I, P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F,
+                                   I, P, SZ, P, P, P, I, P]
+    L.tq_prefill_attend.restype = I
+    L.tq_prefill_attend.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, I, U64, I, P, P,
+                                    I, P]
+    L.tq_prefill_attend_split.restype = I
+    L.tq_prefill_attend_split.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, I, U64, I,
+                                          I, P, SZ, P, P, I, P]
+    L.tq_prefill_workspace_size.restype = SZ
+    L.tq_prefill_workspace_size.argtypes = [I, I, I, I, I]
+    L.tq_prefill_splits.restype = I
+    L.tq_prefill_splits.argtypes = [I, I, I, I]
+    L.tq_attend_partial.restype = I
+    L.tq_attend_partial.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F, I,
+                                    P, SZ, P, P, P, P]
+    L.tq_attend_combine.restype = I
+    L.tq_attend_combine.argtypes = [P, I, I, I, I, U64, P, P, I, P]
+    L.tq_qjl_encode.restype = I
+    L.tq_qjl_encode.argtypes = [P, I, I, I, I, I, U64, P, P, P, P, P, I, I, P, P]
+    L.tq_qjl_scores.restype = I
+    L.tq_qjl_scores.argtypes = [P, I, P, P, P, P, P, P, I, I, I, I, I, U64, I, I, P, P, P]
+    L.tq_attend_noalloc.restype = I
+    L.tq_attend_noalloc.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F, I,
+                                    P, P, P, I, P]
+    return L
 
 
 def _ptr(x):
@@ -163,6 +172,21 @@ def tq_attend(q, q_dtype, packed_k, norms_k, packed_v, norms_v, ctx_lens, batch,
         bits_v, seed, cap_tok, float(sparse_v_thresh), n_ctas,
         _ptr(workspace), workspace_bytes, _ptr(dev_status),
         _ptr(sparse_v_skipped), _ptr(out), out_dtype, _stream(stream)))
+
+
+def tq_attend_gate_counts(q, q_dtype, packed_k, norms_k, packed_v, norms_v, ctx_lens, batch,
+                          n_q_heads, gqa_ratio, d, bits_k, bits_v, seed, cap_tok,
+                          sparse_v_thresh, n_ctas, workspace, workspace_bytes, head_skipped,
+                          out, out_dtype, dev_status=None, sparse_v_skipped=None,
+                          stream=None):
+    """tq_attend plus per (sequence, query head) sparse-V gate counts added
+    into head_skipped (uint32 [batch][n_q_heads], zeroed by the caller)."""
+    _check("tq_attend_gate_counts", lib().tq_attend_gate_counts(
+        _ptr(q), q_dtype, _ptr(packed_k), _ptr(norms_k), _ptr(packed_v),
+        _ptr(norms_v), _ptr(ctx_lens), batch, n_q_heads, gqa_ratio, d, bits_k,
+        bits_v, seed, cap_tok, float(sparse_v_thresh), n_ctas,
+        _ptr(workspace), workspace_bytes, _ptr(dev_status),
+        _ptr(sparse_v_skipped), _ptr(head_skipped), _ptr(out), out_dtype, _stream(stream)))
 
 
 def tq_attend_append(q, q_dtype, new_kv, kv_dtype, packed_k, norms_k, packed_v, norms_v,

@@ -1,8 +1,14 @@
 """Build the library in-tree: csrc/*.cu, csrc/*.cpp -> libtq.so (sm_100a).
 
 Usage: python -m compressed_decode_attention_b200.build [--force] [--verbose]
+       [--waittest]
 Objects go to _build/ beside this file; the shared library is written next
 to this file so it travels with the source tree.
+
+--waittest (build(variant="waittest")) builds libtq_waittest.so, a test-only
+build of the same sources with TQ_TEST_INJECT_WAIT_FAULTS: short bounded
+waits and two waits made to run out, for the test of the kernels' give-up
+path (tests/test_gpu_wait_timeout.py). Only that test loads it.
 """
 from __future__ import annotations
 
@@ -37,12 +43,16 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def _compile(src, verbose):
-    obj = os.path.join(OBJ, os.path.basename(src) + ".o")
+VARIANTS = {None: ("libtq.so", "", []),
+            "waittest": ("libtq_waittest.so", "waittest", ["-DTQ_TEST_INJECT_WAIT_FAULTS"])}
+
+
+def _compile(src, verbose, obj_dir=None, defines=()):
+    obj = os.path.join(obj_dir or OBJ, os.path.basename(src) + ".o")
     if not _stale(obj, [src] + _headers()):
         return obj
-    cmd = [NVCC] + ARCH + COMMON + (CUDA_ONLY if src.endswith(".cu") else ["-x", "cu"] + CUDA_ONLY) + \
-        ["-c", src, "-o", obj]
+    cmd = [NVCC] + ARCH + COMMON + list(defines) + \
+        (CUDA_ONLY if src.endswith(".cu") else ["-x", "cu"] + CUDA_ONLY) + ["-c", src, "-o", obj]
     if verbose:
         cmd += ["-Xptxas", "-v"]
         print(" ".join(cmd), flush=True)
@@ -54,21 +64,25 @@ def _compile(src, verbose):
     return obj
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    os.makedirs(OBJ, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, variant=None) -> str:
+    name, sub, defines = VARIANTS[variant]
+    out = OUT if variant is None else os.path.join(HERE, name)
+    obj_dir = os.path.join(OBJ, sub) if sub else OBJ
+    os.makedirs(obj_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
     if force:
-        for f in glob.glob(os.path.join(OBJ, "*.o")):
+        for f in glob.glob(os.path.join(obj_dir, "*.o")):
             os.remove(f)
     with ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose), srcs))
-    if force or _stale(OUT, objs):
-        cmd = [NVCC] + ARCH + ["-shared", "-o", OUT] + objs + ["-lcudart"]
+        objs = list(ex.map(lambda s: _compile(s, verbose, obj_dir, defines), srcs))
+    if force or _stale(out, objs):
+        cmd = [NVCC] + ARCH + ["-shared", "-o", out] + objs + ["-lcudart"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    return OUT
+    return out
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv,
+                variant="waittest" if "--waittest" in sys.argv else None))

@@ -37,7 +37,8 @@ int attend_common(const void* q, int q_dtype, const void* new_kv, int kv_dtype,
                   int gqa_ratio, int d, int bits_k, int bits_v, uint64_t seed, int cap_tok,
                   float sparse_v_thresh, int n_ctas, void* workspace, size_t workspace_bytes,
                   int* dev_status, unsigned long long* sparse_v_skipped, void* out,
-                  int out_dtype, int partial_out, void* stream) {
+                  int out_dtype, int partial_out, void* stream,
+                  unsigned int* head_skipped = nullptr) {
   if (batch < 1 || n_q_heads < 1 || gqa_ratio < 1 || cap_tok < 1)
     return TQ_ERR_INVALID_ARG;
   if (n_q_heads % gqa_ratio) return TQ_ERR_INVALID_ARG;
@@ -58,7 +59,7 @@ int attend_common(const void* q, int q_dtype, const void* new_kv, int kv_dtype,
   if (!aligned16(q) || !out_ok || !aligned16(packed_k) || !aligned16(packed_v) ||
       !aligned16(norms_k) || !aligned16(norms_v) || !aligned16(workspace) ||
       ((uintptr_t)ctx_lens & 3u) || ((uintptr_t)sparse_v_skipped & 7u) ||
-      ((uintptr_t)dev_status & 3u))
+      ((uintptr_t)dev_status & 3u) || ((uintptr_t)head_skipped & 3u))
     return TQ_ERR_INVALID_ARG;
   if (workspace_bytes < attend_workspace_bytes(batch, n_q_heads, d)) return TQ_ERR_INVALID_ARG;
   const Codebook* cbk = codebook_for(bits_k);
@@ -87,6 +88,7 @@ int attend_common(const void* q, int q_dtype, const void* new_kv, int kv_dtype,
   a.slots = (float*)((uint8_t*)workspace + attend_counter_bytes(batch, n_q_heads));
   a.dev_status = dev_status;
   a.skipped = sparse_v_skipped;
+  a.head_skipped = head_skipped;
   a.out = out;
   a.out_dtype = out_dtype;
   a.partial_out = partial_out;
@@ -206,6 +208,23 @@ int tq_attend(const void* q, int q_dtype, const uint8_t* packed_k,
                            gqa_ratio, d, bits_k, bits_v, seed, cap_tok, sparse_v_thresh,
                            n_ctas, workspace, workspace_bytes, dev_status, sparse_v_skipped,
                            out, out_dtype, 0, stream);
+}
+
+int tq_attend_gate_counts(const void* q, int q_dtype, const uint8_t* packed_k,
+                          const uint16_t* norms_k, const uint8_t* packed_v,
+                          const uint16_t* norms_v, const int32_t* ctx_lens, int batch,
+                          int n_q_heads, int gqa_ratio, int d, int bits_k, int bits_v,
+                          uint64_t seed, int cap_tok, float sparse_v_thresh, int n_ctas,
+                          void* workspace, size_t workspace_bytes, int* dev_status,
+                          unsigned long long* sparse_v_skipped, unsigned int* head_skipped,
+                          void* out, int out_dtype, void* stream) {
+  if (!head_skipped) return TQ_ERR_INVALID_ARG;
+  return tq::attend_common(q, q_dtype, nullptr, TQ_F16, const_cast<uint8_t*>(packed_k),
+                           const_cast<uint16_t*>(norms_k), const_cast<uint8_t*>(packed_v),
+                           const_cast<uint16_t*>(norms_v), ctx_lens, batch, n_q_heads,
+                           gqa_ratio, d, bits_k, bits_v, seed, cap_tok, sparse_v_thresh,
+                           n_ctas, workspace, workspace_bytes, dev_status, sparse_v_skipped,
+                           out, out_dtype, 0, stream, head_skipped);
 }
 
 int tq_attend_append(const void* q, int q_dtype, const void* new_kv, int kv_dtype,

@@ -11,18 +11,20 @@
 // output values per lane, d/16 k-steps per score MMA chain and d/16 PV
 // coordinate tiles.
 //
-// Work decomposition. The cache is a flat list of 64-position blocks in
-// (batch, kv head, block) order; CTA c of Geff owns blocks
-// [c·NB/Geff, (c+1)·NB/Geff). Geff = min(grid, #blocks), except that when all
-// S (batch, kv head) segments have the same block count and S <= grid, Geff
-// is the largest multiple of S within the grid (at most one CTA per block),
-// so every CTA stays inside one segment. A CTA walks the (batch, kv head)
-// segments of its range. Its 12 warps split each segment in whole blocks,
-// merge in shared memory, and
-// either write the output (segment = whole sequence) or leave a partial in a
-// workspace slot; the last CTA to finish a sequence (atomic counter, no
-// waiting) merges the partials and writes the output. No separate combine
-// launch, no spin-waits on other CTAs.
+// Work decomposition. The cache is a list of (batch, kv head) segments of
+// 64-position blocks. Each segment costs its blocks plus a fixed overhead
+// (kSegCost block units: query rotation, first-chunk latency, merges), and
+// CTA c of Geff owns the blocks in the cost range [c·C/Geff, (c+1)·C/Geff)
+// of the total cost C, so CTAs whose range holds many short segments get
+// fewer blocks. Geff = min(grid, #blocks), except that when all S segments
+// have the same block count and S <= grid, Geff is the largest multiple of
+// S within the grid (at most one CTA per block) and the overhead is 0, so
+// every CTA stays inside one segment. A CTA walks the segments of its
+// range. Its warps split each segment in whole units, merge in shared
+// memory, and either write the output (segment = whole sequence) or leave a
+// partial in a workspace slot; the last CTA to finish a sequence (atomic
+// counter, no waiting) merges the partials and writes the output. No
+// separate combine launch, no spin-waits on other CTAs.
 //
 // Per warp and chunk of up to 64 positions (GQA group of g <= 8 query heads),
 // in four 16-position steps:
@@ -44,7 +46,10 @@
 //           of a 4-entry register table; V3/V4: pair table + movmatrix.
 // Output, once per (batch, query head): D⊙(H·(acc/l))/d with shuffles.
 #pragma once
+#include <atomic>
 #include <math.h>
+
+#include <type_traits>
 
 #include "encode_common.cuh"
 
@@ -62,8 +67,20 @@ constexpr float kKScale = 256.f;                // K codebook scale inside the M
 // each CTA's share is reserved by the system).
 constexpr int smem_budget(int per_sm) { return per_sm == 1 ? 227 * 1024 : 228 * 1024 / per_sm - 1024; }
 constexpr int kMaxStages = 3;                   // ring slots per warp
+#ifdef TQ_TEST_INJECT_WAIT_FAULTS
+// Test build only (libtq_waittest.so, for the test of the give-up path):
+// waits give up after ~50 us, and two waits are made to run out without any
+// invalid access: in tq_attend, every warp arms the ring slot of its first
+// chunk for 16 bytes more than its bulk copies deliver (all their bytes
+// still land, so nothing is in flight when it stops), and in the decode step
+// the helper warp never raises the flag its owner waits for.
+constexpr long long kWaitLimitCycles = 100000LL;
+constexpr bool kInjectWaitFaults = true;
+#else
 // Give up on a staged-data wait after this many cycles (~1 s at 2 GHz).
 constexpr long long kWaitLimitCycles = 2000000000LL;
+constexpr bool kInjectWaitFaults = false;
+#endif
 
 constexpr int ceil_pow2(int x) {
   int p = 1;
@@ -72,7 +89,12 @@ constexpr int ceil_pow2(int x) {
 }
 
 // misc words
-constexpr int kMiscSeg = 0;      // b, g, blk0, nseg, nb, L
+constexpr int kMiscCost = 0;     // total cost (lo, hi), per-segment overhead sig
+constexpr int kMiscDesc = 48;    // segment: b, g, blk0, nseg, nb, L, cost of block 0 (lo, hi)
+// Cost of one (sequence, kv head) segment in the CTA split, in 64-position
+// block units, on top of its blocks: the query rotation, the first chunk's
+// latency, the merges and the share of a last round of blocks.
+constexpr int kSegCost = 16;
 constexpr int kMiscLast = 8;     // last-CTA flag
 constexpr int kMiscNB = 9;       // flat block count (lo, hi), common length
 constexpr int kMiscState = 12;   // scan state: sb, sP (lo, hi)
@@ -102,8 +124,8 @@ struct Dm {
   static_assert(M >= kMaxGroup * D, "merge buffer holds GQ x D outputs");
 };
 
-template <int BK, int BV, int D>
-struct Geo {
+template <int BK, int BV, int D, bool WIDE>
+struct GeoL {
   static constexpr int RK = D * BK / 8;                 // packed K row bytes
   static constexpr int RV = D * BV / 8;
   // rows per 16-byte multiple of a bulk copy of K / V rows
@@ -117,14 +139,21 @@ struct Geo {
   static constexpr int VB = kBlk * RVS;
   static constexpr int NKOFF = KB + VB;
   static constexpr int STAGE = KB + VB + 2 * kBlk * 2;
-  // K table: uint2 (high pair, low pair) per (pair code, lane & 15): 128 B per code.
-  static constexpr int LUTK = (1 << (2 * BK)) * 128;
+  // K table: uint2 (high pair, low pair) per (pair code, lane & 15): 128 B per
+  // code. In the wide layout (4-bit K: the pair code is a whole byte) codes
+  // are 256 B apart, so that one byte permute of the packed word and the
+  // lane offset forms the entry's address; the V table (3/4 bits) then sits
+  // in the other 128 B of each code's row.
+  static constexpr bool KWIDE = WIDE;
+  static constexpr int KSTRIDE = WIDE ? 256 : 128;
+  static constexpr int LUTK = (1 << (2 * BK)) * KSTRIDE;
   // V table (3/4 bits): uint32 fp16 pair per (pair code, lane): 128 B per code.
-  static constexpr int LUTV = BV == 2 ? 0 : (1 << (2 * BV)) * 128;
-  // The V table sits at a power-of-two offset no smaller than either table,
-  // so entry addresses are formed with OR.
-  static constexpr int LUTV_OFF = BV == 2 ? LUTK : ceil_pow2(LUTK > LUTV ? LUTK : LUTV);
-  static constexpr int QOFF = LUTV_OFF + LUTV;
+  static constexpr int LUTV = BV == 2 || WIDE ? 0 : (1 << (2 * BV)) * 128;
+  // Narrow layout: the V table sits at a power-of-two offset no smaller
+  // than either table, so entry addresses are formed with OR.
+  static constexpr int LUTV_OFF = WIDE ? 128 : BV == 2 ? LUTK : ceil_pow2(LUTK > LUTV ? LUTK : LUTV);
+  static constexpr int VSHIFT = WIDE ? 8 : 7;           // log2 of the V code stride
+  static constexpr int QOFF = WIDE ? LUTK : LUTV_OFF + LUTV;
   static constexpr int QS = kMaxGroup * D * 2 * 2;      // q~ high and low, fp16
   static constexpr int MISC = 1024;                     // kMiscWords words
   static constexpr int MBAR = kMaxWarps * kMaxStages * 8;  // per-warp ring barriers
@@ -142,8 +171,15 @@ struct Geo {
   static constexpr int MERGE = NW * Dm<D>::STRIDE * 4;
   static constexpr int RING = NSTAGE * NW * STAGE;
   static constexpr int SMEM = FIXED + (RING > MERGE ? RING : MERGE);
-  static_assert(NSTAGE >= 1, "stage ring does not fit");
-  static_assert(SMEM <= BUDGET, "shared memory budget");
+  static_assert(NSTAGE >= 1 || WIDE, "stage ring does not fit");
+  static_assert(SMEM <= BUDGET || WIDE, "shared memory budget");
+};
+
+// The wide K table wherever it keeps the ring as deep as the narrow one.
+template <int BK, int BV, int D>
+struct Geo : GeoL<BK, BV, D, (BK == 4 && GeoL<BK, BV, D, true>::NSTAGE >= 1 &&
+                              GeoL<BK, BV, D, true>::NSTAGE >= GeoL<BK, BV, D, false>::NSTAGE)> {
+  static_assert(!Geo::KWIDE || (BK == 4 && BV <= BK), "wide layout: byte pair codes, V codes fit");
 };
 
 
@@ -247,8 +283,8 @@ __device__ __forceinline__ int seq_blocks(const AttendArgs& a, int b) {
   return (L + kBlk - 1) / kBlk;
 }
 
-// CTA owning flat block `blk` when NB blocks are split over G CTAs as
-// [c·NB/G, (c+1)·NB/G): the largest c with floor(c·NB/G) <= blk.
+// CTA owning the block at cost `blk` when a total cost NB is split over G
+// CTAs as [c·NB/G, (c+1)·NB/G): the largest c with floor(c·NB/G) <= blk.
 __device__ __forceinline__ int cta_of(long long blk, long long nb, int g) {
   return (int)(((blk + 1) * g - 1) / nb);
 }
@@ -419,12 +455,12 @@ attend_kernel(const __grid_constant__ AttendArgs a,
     uint2 v;
     v.x = (c0 & 0xFFFFu) | (c1 << 16);                // high parts (even, odd coord)
     v.y = (c0 >> 16) | (c1 & 0xFFFF0000u);            // low parts
-    *reinterpret_cast<uint2*>(lutK + code * 128 + copy * 8) = v;
+    *reinterpret_cast<uint2*>(lutK + code * Gm::KSTRIDE + copy * 8) = v;
   }
   if (BV != 2) {
     for (int e = tid; e < (1 << (2 * BV)) * 32; e += kThreads) {
       const int code = e >> 5, copy = e & 31;
-      *reinterpret_cast<uint32_t*>(lutV + code * 128 + copy * 4) =
+      *reinterpret_cast<uint32_t*>(lutV + (code << Gm::VSHIFT) + copy * 4) =
           cbs[16 + (code & ((1 << BV) - 1))] | (cbs[16 + (code >> BV)] << 16);
     }
   }
@@ -438,6 +474,125 @@ attend_kernel(const __grid_constant__ AttendArgs a,
       vt_hi |= (h >> 8) << (8 * j);
     }
   }
+
+  // Segment search (warp 0) in cost units. The CTAs split a list of
+  // (sequence, kv head) segments (sequences in order, kv heads in order
+  // within one); a segment of nb > 0 blocks costs nb + sig units, a fixed
+  // per-segment overhead sig first, then one unit per block. Finds the first
+  // segment holding a block of cost >= at, continuing from the scan state in
+  // misc, and writes its descriptor at misc[slot]: b, g, the first block and
+  // the number of its blocks with cost in [at, end) (0: none), the segment's
+  // block count and length, and the cost of its block 0.
+  // len0: this lane's length among the first 32 sequences.
+  auto find_segment = [&](long long at, long long end, int len0, int slot) {
+    const int sig = misc[kMiscCost + 2];
+    int sb = misc[kMiscState];
+    long long sP = (long long)(unsigned)misc[kMiscState + 1] | ((long long)misc[kMiscState + 2] << 32);
+    while (true) {
+      if (sb >= B) {                      // inconsistent lengths: stop this CTA
+        if (lane == 0) misc[slot + 3] = 0;
+        break;
+      }
+      const int bb = sb + lane;
+      const int len = sb == 0 ? len0 : (bb < B ? min(max(a.ctx_lens[bb], 0), a.cap_tok) : 0);
+      const int nb = (len + kBlk - 1) / kBlk;
+      const int cst = nb > 0 ? nb + sig : 0;          // cost of one kv head of sequence bb
+      int incl = cst;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const long long segend = (long long)H * (sP + incl);
+      const unsigned hit = __ballot_sync(0xFFFFFFFFu, segend > at && bb < B);
+      if (hit) {
+        const int l = __ffs(hit) - 1;
+        const int nbl = __shfl_sync(0xFFFFFFFFu, nb, l);
+        const int lenl = __shfl_sync(0xFFFFFFFFu, len, l);
+        const int excl = __shfl_sync(0xFFFFFFFFu, incl - cst, l);
+        sb += l;
+        sP += excl;
+        if (lane == 0) {
+          const int cl = nbl + sig;
+          const long long rel = at - (long long)H * sP;
+          const int g = (int)(rel / cl), off = (int)(rel % cl);
+          const long long first = (long long)H * sP + (long long)g * cl + sig;
+          const int blk0 = max(0, off - sig);
+          const long long bend = min((long long)nbl, end - first);
+          misc[slot + 0] = sb;
+          misc[slot + 1] = g;
+          misc[slot + 2] = blk0;
+          misc[slot + 3] = (int)max(0LL, bend - blk0);
+          misc[slot + 4] = nbl;
+          misc[slot + 5] = lenl;
+          misc[slot + 6] = (int)(first & 0xFFFFFFFF);
+          misc[slot + 7] = (int)(first >> 32);
+          misc[kMiscState] = sb;
+          misc[kMiscState + 1] = (int)(sP & 0xFFFFFFFF);
+          misc[kMiscState + 2] = (int)(sP >> 32);
+        }
+        break;
+      }
+      sP += __shfl_sync(0xFFFFFFFFu, incl, 31);
+      sb += 32;
+    }
+  };
+
+  // Balanced split over Geff CTAs, each owning at least one block (the
+  // partial count of a sequence relies on it): min(grid, NB), or, when every
+  // (sequence, kv head) segment has the same block count and there are no
+  // more segments than CTAs, a multiple of the segment count so that no CTA
+  // spans two segments.
+  auto effective_ctas = [&](long long nbt, int common) {
+    int ge = (int)min((long long)Gc, nbt);
+    const long long S = (long long)B * H;
+    if (common > 0 && S <= Gc) ge = (int)(S * min((long long)(Gc / S), (long long)common));
+    return ge;
+  };
+
+  // Warp 0: flat block count, whether all sequences have the same length,
+  // and the first segment of this CTA (into misc).
+  auto plan_cta = [&](int len0) {
+    long long tot = 0;
+    int nmin = 0x7FFFFFFF, nmax = 0, live = 0;
+    for (int b0 = 0; b0 < B; b0 += 32) {
+      const bool in = b0 + lane < B;
+      const int nb = b0 == 0 ? (len0 + kBlk - 1) / kBlk : (in ? seq_blocks(a, b0 + lane) : 0);
+      int sum = nb, lo = in ? nb : 0x7FFFFFFF, hi = nb, nz = nb > 0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+        lo = min(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, o));
+        hi = max(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, o));
+        nz += __shfl_xor_sync(0xFFFFFFFFu, nz, o);
+      }
+      tot += sum;
+      live += nz;
+      nmin = min(nmin, lo);
+      nmax = max(nmax, hi);
+    }
+    const long long nbt = tot * H;
+    const int common = nmin == nmax ? nmax : -1;
+    // no per-segment overhead when every CTA gets a piece of one segment
+    const int sig = common > 0 && (long long)B * H <= Gc ? 0 : kSegCost;
+    const long long ctot = (tot + (long long)sig * live) * H;
+    if (lane == 0) {
+      misc[kMiscCost] = (int)(ctot & 0xFFFFFFFF);
+      misc[kMiscCost + 1] = (int)(ctot >> 32);
+      misc[kMiscCost + 2] = sig;
+      misc[kMiscNB] = (int)(nbt & 0xFFFFFFFF);
+      misc[kMiscNB + 1] = (int)(nbt >> 32);
+      misc[kMiscNB + 2] = common;
+      misc[kMiscState] = 0;
+      misc[kMiscState + 1] = 0;
+      misc[kMiscState + 2] = 0;
+      misc[kMiscDesc + 3] = 0;
+      misc[kMiscApp] = 0;
+    }
+    __syncwarp();
+    const int ge = effective_ctas(nbt, common);
+    if (cta < ge) find_segment(ctot * cta / ge, ctot * (cta + 1) / ge, len0, kMiscDesc);
+  };
 
   // Everything below reads inputs that an earlier launch may have written.
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
@@ -464,108 +619,14 @@ attend_kernel(const __grid_constant__ AttendArgs a,
     }
   }
 
-  // Segment search (warp 0): the first sequence whose flat block range holds
-  // flat block `at`, continuing from the scan state in misc. Writes the
-  // segment (b, g, first block, block count, blocks of the sequence, length).
-  auto find_segment = [&](long long at, long long end) {
-    int sb = misc[kMiscState];
-    long long sP = (long long)(unsigned)misc[kMiscState + 1] | ((long long)misc[kMiscState + 2] << 32);
-    while (true) {
-      if (sb >= B) {                      // inconsistent lengths: stop this CTA
-        if (lane == 0) misc[kMiscSeg + 3] = 0;
-        break;
-      }
-      const int bb = sb + lane;
-      const int len = sb == 0 ? len0 : (bb < B ? min(max(a.ctx_lens[bb], 0), a.cap_tok) : 0);
-      const int nb = (len + kBlk - 1) / kBlk;
-      int incl = nb;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      const long long segend = (long long)H * (sP + incl);
-      const unsigned hit = __ballot_sync(0xFFFFFFFFu, segend > at && bb < B);
-      if (hit) {
-        const int l = __ffs(hit) - 1;
-        const int nbl = __shfl_sync(0xFFFFFFFFu, nb, l);
-        const int lenl = __shfl_sync(0xFFFFFFFFu, len, l);
-        const int excl = __shfl_sync(0xFFFFFFFFu, incl - nb, l);
-        sb += l;
-        sP += excl;
-        if (lane == 0) {
-          const long long rel = at - (long long)H * sP;
-          const int g = (int)(rel / nbl), blk0 = (int)(rel % nbl);
-          misc[kMiscSeg + 0] = sb;
-          misc[kMiscSeg + 1] = g;
-          misc[kMiscSeg + 2] = blk0;
-          misc[kMiscSeg + 3] = (int)min((long long)(nbl - blk0), end - at);
-          misc[kMiscSeg + 4] = nbl;
-          misc[kMiscSeg + 5] = lenl;
-          misc[kMiscState] = sb;
-          misc[kMiscState + 1] = (int)(sP & 0xFFFFFFFF);
-          misc[kMiscState + 2] = (int)(sP >> 32);
-        }
-        break;
-      }
-      sP += __shfl_sync(0xFFFFFFFFu, incl, 31);
-      sb += 32;
-    }
-  };
-
-  // Balanced split over Geff CTAs, each owning at least one block (the
-  // partial count of a sequence relies on it): min(grid, NB), or, when every
-  // (sequence, kv head) segment has the same block count and there are no
-  // more segments than CTAs, a multiple of the segment count so that no CTA
-  // spans two segments.
-  auto effective_ctas = [&](long long nbt, int common) {
-    int ge = (int)min((long long)Gc, nbt);
-    const long long S = (long long)B * H;
-    if (common > 0 && S <= Gc) ge = (int)(S * min((long long)(Gc / S), (long long)common));
-    return ge;
-  };
-
-  if (warp == 0) {
-    // ---- flat block count, whether all sequences have the same length, and
-    // the first segment of this CTA
-    long long tot = 0;
-    int nmin = 0x7FFFFFFF, nmax = 0;
-    for (int b0 = 0; b0 < B; b0 += 32) {
-      const bool in = b0 + lane < B;
-      const int nb = b0 == 0 ? (len0 + kBlk - 1) / kBlk : (in ? seq_blocks(a, b0 + lane) : 0);
-      int sum = nb, lo = in ? nb : 0x7FFFFFFF, hi = nb;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-        lo = min(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, o));
-        hi = max(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, o));
-      }
-      tot += sum;
-      nmin = min(nmin, lo);
-      nmax = max(nmax, hi);
-    }
-    const long long nbt = tot * H;
-    const int common = nmin == nmax ? nmax : -1;
-    if (lane == 0) {
-      misc[kMiscNB] = (int)(nbt & 0xFFFFFFFF);
-      misc[kMiscNB + 1] = (int)(nbt >> 32);
-      misc[kMiscNB + 2] = common;
-      misc[kMiscState] = 0;
-      misc[kMiscState + 1] = 0;
-      misc[kMiscState + 2] = 0;
-      misc[kMiscSeg + 3] = 0;
-      misc[kMiscApp] = 0;
-    }
-    __syncwarp();
-    const int ge = effective_ctas(nbt, common);
-    if (cta < ge) find_segment(nbt * cta / ge, nbt * (cta + 1) / ge);
-  }
+  if (warp == 0) plan_cta(len0);
   __syncthreads();
 
   const long long NB = (long long)(unsigned)misc[kMiscNB] | ((long long)misc[kMiscNB + 1] << 32);
   const int Geff = effective_ctas(NB, misc[kMiscNB + 2]);
-  const long long r0 = cta < Geff ? NB * cta / Geff : 0;
-  const long long r1 = cta < Geff ? NB * (cta + 1) / Geff : 0;
+  const long long Ctot = (long long)(unsigned)misc[kMiscCost] | ((long long)misc[kMiscCost + 1] << 32);
+  const long long r0 = cta < Geff ? Ctot * cta / Geff : 0;   // this CTA's cost range
+  const long long r1 = cta < Geff ? Ctot * (cta + 1) / Geff : 0;
   long long pos = r0;
   unsigned nskip = 0;
   const float log2tau = a.tau > 0.f ? log2f(a.tau) : -INFINITY;
@@ -638,19 +699,35 @@ attend_kernel(const __grid_constant__ AttendArgs a,
     __syncthreads();
   };
 
-  bool first = true;
+  // Warps split a segment into ranges of whole units: 64-position blocks
+  // with the sparse-V gate (its block maximum needs the whole block) and in
+  // the decode step (the warp that encodes the new token needs the slack of
+  // a block fewer), else 32 positions, which evens out the shares when a
+  // segment has only a few blocks per warp. A warp walks its range in
+  // chunks of up to 64 positions starting at wp0. The range of warp w in the
+  // segment described at misc[slot]:
+  const int unit = a.tau > 0.f || a.new_kv ? kBlk : kBlk / 2;
+  auto warp_share = [&](int slot, int w, int& wp0, int& wp1) {
+    const int blk0 = misc[slot + 2], nseg = misc[slot + 3], L = misc[slot + 5];
+    const int sp0 = blk0 * kBlk, sp1 = min(L, (blk0 + nseg) * kBlk);
+    const int nun = nseg > 0 ? (sp1 - sp0 + unit - 1) / unit : 0;
+    wp0 = sp0 + unit * (int)((long long)nun * w / kWarps);
+    wp1 = min(sp1, sp0 + unit * (int)((long long)nun * (w + 1) / kWarps));
+  };
+
   int seg_iter = 0;                                   // segments this CTA has done
   while (pos < r1) {
-    if (!first) {
-      if (warp == 0) find_segment(pos, r1);
+    if (seg_iter > 0) {
+      if (warp == 0) find_segment(pos, r1, len0, kMiscDesc);
       __syncthreads();
     }
-    first = false;
-    const int b = misc[kMiscSeg + 0], g = misc[kMiscSeg + 1], blk0 = misc[kMiscSeg + 2];
-    const int nseg = misc[kMiscSeg + 3], nbl = misc[kMiscSeg + 4], L = misc[kMiscSeg + 5];
+    const int cs = kMiscDesc;
+    const int b = misc[cs + 0], g = misc[cs + 1], blk0 = misc[cs + 2];
+    const int nseg = misc[cs + 3], nbl = misc[cs + 4], L = misc[cs + 5];
     if (nseg <= 0) break;
-    const long long sP_seg = (long long)(unsigned)misc[kMiscState + 1] | ((long long)misc[kMiscState + 2] << 32);
-    const long long seg_first = (long long)H * sP_seg + (long long)g * nbl;
+    // cost of the segment's block 0, and the cost just past this CTA's piece
+    const long long seg_first = (long long)(unsigned)misc[cs + 6] | ((long long)misc[cs + 7] << 32);
+    const long long next_pos = seg_first + blk0 + nseg;
 
     // query values of the group (warp h < g loads head h), issued before the
     // block loads
@@ -681,23 +758,18 @@ attend_kernel(const __grid_constant__ AttendArgs a,
     for (int k = 0; k < QPL; ++k) qraw[k] = 0.f;
     if (warp < GQ) load_q(warp, qraw);
 
-    // ---- this warp's blocks of the segment
-    // The warps split the segment in whole 64-position blocks (the sparse-V
-    // gate's block maximum needs the full block; measured, a 16-position
-    // split was no faster without the gate either: the SM is throughput
-    // bound in this phase). A warp walks its range in chunks of up to 64
-    // positions starting at wp0.
+    // ---- this warp's share of the segment
     const int sp0 = blk0 * kBlk, sp1 = min(L, (blk0 + nseg) * kBlk);
-    const int unit = kBlk;
     const int nun = (sp1 - sp0 + unit - 1) / unit;
-    const int wp0 = sp0 + unit * (int)((long long)nun * warp / kWarps);
-    const int wp1 = min(sp1, sp0 + unit * (int)((long long)nun * (warp + 1) / kWarps));
+    int wp0, wp1;
+    warp_share(cs, warp, wp0, wp1);
     const int nw = wp1 > wp0 ? (wp1 - wp0 + kBlk - 1) / kBlk : 0;
 
     float acc[NPV][4];
 #pragma unroll
     for (int r = 0; r < NPV; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
     float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+    unsigned nsk0 = 0, nsk1 = 0;               // gated positions of heads hs0, hs0 + 1
 
     const size_t seq_row = ((size_t)b * H + g) * a.cap_tok;
     const uint8_t* gk = a.packed_k + seq_row * Gm::RK;
@@ -705,17 +777,19 @@ attend_kernel(const __grid_constant__ AttendArgs a,
     const uint16_t* gnk = a.norms_k + seq_row;
     const uint16_t* gnv = a.norms_v + seq_row;
     const uint32_t wring = Gm::FIXED + warp * Gm::NSTAGE * Gm::STAGE;   // smem offset
-    const uint32_t wring_s = smem_addr(smem) + wring;                    // shared address
 
     // Bulk copies of chunk c of the warp's range (its j-th staged chunk)
     // into ring slot j % NSTAGE, issued by lane 0: K rows, V rows and the
     // two norm runs are contiguous in global memory. Rows past the range are
     // not copied; their slot bytes are stale and masked out below (norms are
     // copied in whole 16-byte runs, which stay inside cap_tok).
-    auto issue = [&](int c, int j) {
+    // ... of chunk c of warp v's range [v0, v1) into slot j % NSTAGE of v's
+    // ring (v = this warp, or in the first segment a query-rotating warp
+    // whose first copies another warp issues)
+    auto issue_for = [&](int v, int v0, int v1, int c, int j) {
       if (lane == 0) {
-        const int t0 = wp0 + c * kBlk;
-        const int rows = min(kBlk, wp1 - t0);
+        const int t0 = v0 + c * kBlk;
+        const int rows = min(kBlk, v1 - t0);
         // A bulk copy moves a multiple of 16 bytes: row counts are rounded up
         // to Gm::KROWS / VROWS (2 for the 24-byte rows at d = 64 and 3 bits,
         // else 1) and norm runs to 8; every bound stays inside cap_tok, a
@@ -724,15 +798,18 @@ attend_kernel(const __grid_constant__ AttendArgs a,
         const int vrows = min(kBlk, (rows + Gm::VROWS - 1) / Gm::VROWS * Gm::VROWS);
         const int nrows = min(kBlk, (rows + 7) & ~7);
         const int slot = j % Gm::NSTAGE;
-        const uint32_t dst = wring_s + slot * Gm::STAGE, bar = wbar + 8 * slot;
+        const uint32_t dst = smem_addr(smem) + Gm::FIXED + (v * Gm::NSTAGE + slot) * Gm::STAGE;
+        const uint32_t bar = smem_addr(smem) + Gm::QOFF + Gm::QS + Gm::MISC + (v * kMaxStages + slot) * 8;
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-        mbar_expect(bar, krows * Gm::RK + vrows * Gm::RV + 4 * nrows);
+        const uint32_t extra = kInjectWaitFaults && a.new_kv == nullptr && j == 0 ? 16u : 0u;
+        mbar_expect(bar, krows * Gm::RK + vrows * Gm::RV + 4 * nrows + extra);
         bulk_g2s(dst, gk + (size_t)t0 * Gm::RK, krows * Gm::RK, bar);
         bulk_g2s(dst + Gm::KB, gv + (size_t)t0 * Gm::RV, vrows * Gm::RV, bar);
         bulk_g2s(dst + Gm::NKOFF, gnk + t0, 2 * nrows, bar);
         bulk_g2s(dst + Gm::NKOFF + 2 * kBlk, gnv + t0, 2 * nrows, bar);
       }
     };
+    auto issue = [&](int c, int j) { issue_for(warp, wp0, wp1, c, j); };
 
     // every slot of the ring gets a block (or an empty group); the warps
     // that rotate the query fill theirs afterwards, so that the query loads
@@ -745,7 +822,20 @@ attend_kernel(const __grid_constant__ AttendArgs a,
     int issued = stalled ? 0 : min(nw, Gm::NSTAGE);
     auto bar_of = [&](int jj) { return wbar + 8 * (jj % Gm::NSTAGE); };
     auto par_of = [&](int jj) { return (uint32_t)(jj / Gm::NSTAGE) & 1u; };
-    if (warp >= GQ) fill_ring();
+    // In the first segment every ring starts at chunk 0, so the warps that
+    // do not rotate the query also issue the first chunks of those that do
+    // (query warp v by warp GQ + v % (warps - GQ)): all rings fill at once.
+    const bool proxy_fill = seg_iter == 0 && GQ < kWarps;
+    if (warp >= GQ) {
+      fill_ring();
+      if (proxy_fill)
+        for (int v = warp - GQ; v < GQ; v += kWarps - GQ) {
+          int v0, v1;
+          warp_share(cs, v, v0, v1);
+          const int nv_ = v1 > v0 ? (v1 - v0 + kBlk - 1) / kBlk : 0;
+          for (int p = 0; p < Gm::NSTAGE && p < nv_; ++p) issue_for(v, v0, v1, p, p);
+        }
+    }
     // ---- rotated query of the group: warp w handles query heads w, w +
     // kWarps, ... (the first one's values are already loaded)
     auto rotate_q = [&](int h, const float (&qr)[QPL]) {
@@ -787,7 +877,7 @@ attend_kernel(const __grid_constant__ AttendArgs a,
         load_q(h, q2);
         rotate_q(h, q2);
       }
-      fill_ring();
+      if (!proxy_fill) fill_ring();
     }
     // ---- decode-step append. The owner warp (its range ends at the
     // sequence's last position) patches the new row into its staged last
@@ -847,7 +937,7 @@ attend_kernel(const __grid_constant__ AttendArgs a,
         a.norms_k[row] = app_n[0];
         a.norms_v[row] = app_n[1];
         __threadfence_block();                        // the row before the flag
-        *reinterpret_cast<volatile int*>(misc + kMiscApp) = seg_iter + 1;
+        if (!kInjectWaitFaults) *reinterpret_cast<volatile int*>(misc + kMiscApp) = seg_iter + 1;
       }
     }
 
@@ -867,8 +957,12 @@ attend_kernel(const __grid_constant__ AttendArgs a,
         qb[t][s][1] = ok ? *reinterpret_cast<const uint32_t*>(src + head * D + c0 + 2) : 0u;
       }
     }
-    const float sinv0 = hv0 ? miscf[kMiscQInv + hs0] : 0.f;
-    const float sinv1 = hv1 ? miscf[kMiscQInv + hs0 + 1] : 0.f;
+    // Query scale of heads hs0, hs0 + 1. A head beyond the group has a zero
+    // query and scale 1: its scores are 0 and its weights finite, and its
+    // accumulator columns are never read.
+    const float2 sinv = make_float2(hv0 ? miscf[kMiscQInv + hs0] : 1.f,
+                                    hv1 ? miscf[kMiscQInv + hs0 + 1] : 1.f);
+    const bool gate = a.tau > 0.f;
 
     for (int i = 0; i < nw && !stalled; ++i) {
       const int j = jdone + i;
@@ -933,8 +1027,16 @@ attend_kernel(const __grid_constant__ AttendArgs a,
         for (int s2 = 0; s2 < KS; ++s2) {
 #pragma unroll
           for (int gr = 0; gr < 2; ++gr) {
-            const uint2 e0 = lds<uint2>(smem, k_entry<BK>(kw[gr], 2 * s2) + lbK);
-            const uint2 e1 = lds<uint2>(smem, k_entry<BK>(kw[gr], 2 * s2 + 1) + lbK);
+            uint32_t a0, a1;
+            if constexpr (Gm::KWIDE) {               // (code << 8) | lane offset
+              a0 = __byte_perm(kw[gr][s2 >> 1], lbK, 0x7604u | (uint32_t)((2 * s2) & 3) << 4);
+              a1 = __byte_perm(kw[gr][s2 >> 1], lbK, 0x7604u | (uint32_t)((2 * s2 + 1) & 3) << 4);
+            } else {
+              a0 = k_entry<BK>(kw[gr], 2 * s2) + lbK;
+              a1 = k_entry<BK>(kw[gr], 2 * s2 + 1) + lbK;
+            }
+            const uint2 e0 = lds<uint2>(smem, a0);
+            const uint2 e1 = lds<uint2>(smem, a1);
 #pragma unroll
             for (int t = 0; t < NT; ++t)
               mma16816(d[gr][t], e0.x, e0.y, e1.x, e1.y, qb[t][s2][0], qb[t][s2][1]);
@@ -959,66 +1061,99 @@ attend_kernel(const __grid_constant__ AttendArgs a,
           }
         }
       }
-      // -- scale by the K norm and query scale, mask, block maximum per head
-      float mb0 = -INFINITY, mb1 = -INFINITY;
+      // -- scores x = (MMA sum) · n_K per position and head (the query scale
+      // is applied below), masked past the chunk; block maximum per head
+      auto scale_scores = [&](auto part_c) {          // sc <- x, in place
+        constexpr bool PART = decltype(part_c)::value;
+        float2 xm = make_float2(-INFINITY, -INFINITY);
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt)
+        for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-        for (int rr = 0; rr < NR; ++rr) {
-          const int p = pos_of(mt, rr);
-          const float nk = __half2float(__ushort_as_half(lds<uint16_t>(smem, st + Gm::NKOFF + 2 * p)));
-          float v0 = sc[mt][rr][0] * (sinv0 * nk);
-          float v1 = sc[mt][rr][1] * (sinv1 * nk);
-          if (partial && t0 + p >= cend) v0 = v1 = -INFINITY;
-          sc[mt][rr][0] = v0;
-          sc[mt][rr][1] = v1;
-          mb0 = fmaxf(mb0, v0);
-          mb1 = fmaxf(mb1, v1);
-        }
+          for (int rr = 0; rr < NR; ++rr) {
+            const int p = pos_of(mt, rr);
+            const float nk = __half2float(__ushort_as_half(lds<uint16_t>(smem, st + Gm::NKOFF + 2 * p)));
+            float2 x = __fmul2_rn(make_float2(sc[mt][rr][0], sc[mt][rr][1]), make_float2(nk, nk));
+            if (PART && t0 + p >= cend) x = make_float2(-INFINITY, -INFINITY);
+            sc[mt][rr][0] = x.x;
+            sc[mt][rr][1] = x.y;
+            xm.x = fmaxf(xm.x, x.x);
+            xm.y = fmaxf(xm.y, x.y);
+          }
+        return xm;
+      };
+      float2 xm = partial ? scale_scores(std::true_type{}) : scale_scores(std::false_type{});
       // lanes holding the same heads: NT = 1 -> lane bits 1-4; NT = 2 -> bits 2-4
 #pragma unroll
       for (int o = (NT == 1 ? 2 : 4); o < 32; o <<= 1) {
-        mb0 = fmaxf(mb0, __shfl_xor_sync(0xFFFFFFFFu, mb0, o));
-        mb1 = fmaxf(mb1, __shfl_xor_sync(0xFFFFFFFFu, mb1, o));
+        xm.x = fmaxf(xm.x, __shfl_xor_sync(0xFFFFFFFFu, xm.x, o));
+        xm.y = fmaxf(xm.y, __shfl_xor_sync(0xFFFFFFFFu, xm.y, o));
       }
-      const float mn0 = fmaxf(m_run[0], mb0), mn1 = fmaxf(m_run[1], mb1);
+      // block maximum of the scores s = x · scale (the scale is positive, so
+      // the maximum of the rounded products is the rounded product of the maximum)
+      const float2 mb = __fmul2_rn(xm, sinv);
+      const float mn0 = fmaxf(m_run[0], mb.x), mn1 = fmaxf(m_run[1], mb.y);
       const float al0 = fast_exp2(m_run[0] - mn0), al1 = fast_exp2(m_run[1] - mn1);
       m_run[0] = mn0;
       m_run[1] = mn1;
       l_run[0] *= al0;
       l_run[1] *= al1;
 
-      // -- weights, gate, P' = w · nV packed as fp16 pairs (heads hs0, hs0+1)
+      // -- weights w = 2^(s - m), P' = w · n_V packed as fp16 pairs (heads hs0,
+      // hs0+1). With the sparse-V gate, P' = 0 where 2^(s - M_blk) < tau.
       uint32_t pk[4][NR];
+      auto weights = [&](auto gate_c, auto part_c) {
+        constexpr bool GATE = decltype(gate_c)::value, PART = decltype(part_c)::value;
+        const float2 negm = make_float2(-mn0, -mn1);
+        float2 lsum = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt)
+        for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-        for (int rr = 0; rr < NR; ++rr) {
-          const int p = pos_of(mt, rr);
-          const float nv = __half2float(__ushort_as_half(lds<uint16_t>(smem, st + Gm::NKOFF + 2 * kBlk + 2 * p)));
-          const float s0 = sc[mt][rr][0], s1 = sc[mt][rr][1];
-          const float w0 = fast_exp2(s0 - mn0), w1 = fast_exp2(s1 - mn1);
-          l_run[0] += w0;
-          l_run[1] += w1;
-          float p0 = w0 * nv, p1 = w1 * nv;
-          const bool g0 = s0 - mb0 < log2tau, g1 = s1 - mb1 < log2tau;   // exp(s - M_blk) < tau
-          if (g0) p0 = 0.f;
-          if (g1) p1 = 0.f;
-          if (partial && t0 + p >= cend) p0 = p1 = 0.f;   // stale slot bytes
-          nskip += (g0 && hv0 && s0 != -INFINITY) + (g1 && hv1 && s1 != -INFINITY);
-          pk[mt][rr] = pack_half2(hv0 ? p0 : 0.f, hv1 ? p1 : 0.f);
-        }
+          for (int rr = 0; rr < NR; ++rr) {
+            const int p = pos_of(mt, rr);
+            const float nv = __half2float(__ushort_as_half(lds<uint16_t>(smem, st + Gm::NKOFF + 2 * kBlk + 2 * p)));
+            float2 e, sv;
+            if (GATE) {                             // the rounded score, as the gate compares it
+              sv = __fmul2_rn(make_float2(sc[mt][rr][0], sc[mt][rr][1]), sinv);
+              e = __fadd2_rn(sv, negm);
+            } else {
+              e = __ffma2_rn(make_float2(sc[mt][rr][0], sc[mt][rr][1]), sinv, negm);
+            }
+            const float2 w = make_float2(fast_exp2(e.x), fast_exp2(e.y));
+            lsum = __fadd2_rn(lsum, w);
+            float2 pp = __fmul2_rn(w, make_float2(nv, nv));
+            if (GATE) {
+              const bool g0 = sv.x - mb.x < log2tau, g1 = sv.y - mb.y < log2tau;   // exp(s - M_blk) < tau
+              if (g0) pp.x = 0.f;
+              if (g1) pp.y = 0.f;
+              nsk0 += g0 && hv0 && sv.x != -INFINITY;
+              nsk1 += g1 && hv1 && sv.y != -INFINITY;
+            }
+            if (PART && t0 + p >= cend) pp = make_float2(0.f, 0.f);   // stale slot bytes
+            pk[mt][rr] = pack_half2(pp.x, pp.y);
+          }
+        l_run[0] += lsum.x;
+        l_run[1] += lsum.y;
+      };
+      if (gate) {
+        if (partial) weights(std::true_type{}, std::true_type{});
+        else weights(std::true_type{}, std::false_type{});
+      } else {
+        if (partial) weights(std::false_type{}, std::true_type{});
+        else weights(std::false_type{}, std::false_type{});
+      }
       // rescale the PV accumulators (PV layout: heads 2tq, 2tq+1)
       {
-        float a0 = al0, a1 = al1;
-        if (NT == 1 && tq >= 2) a0 = a1 = 1.f;      // heads 4-7: padding
-        if (__any_sync(0xFFFFFFFFu, a0 != 1.f || a1 != 1.f)) {
+        float2 al = make_float2(al0, al1);
+        if (NT == 1 && tq >= 2) al = make_float2(1.f, 1.f);   // heads 4-7: padding
+        if (__any_sync(0xFFFFFFFFu, al.x != 1.f || al.y != 1.f)) {
 #pragma unroll
           for (int r = 0; r < NPV; ++r) {
-            acc[r][0] *= a0;
-            acc[r][1] *= a1;
-            acc[r][2] *= a0;
-            acc[r][3] *= a1;
+            const float2 u = __fmul2_rn(make_float2(acc[r][0], acc[r][1]), al);
+            const float2 v = __fmul2_rn(make_float2(acc[r][2], acc[r][3]), al);
+            acc[r][0] = u.x;
+            acc[r][1] = u.y;
+            acc[r][2] = v.x;
+            acc[r][3] = v.y;
           }
         }
       }
@@ -1026,6 +1161,7 @@ attend_kernel(const __grid_constant__ AttendArgs a,
       // -- P·V over the four 16-position steps
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
+        if (16 * mt >= cend - t0) break;     // steps past the chunk
         uint32_t x0, x1;   // P' of positions 0-7 / 8-15 x heads 0-7, standard layout
         if (NT == 1) {
           const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, pk[mt][0], 2);
@@ -1035,7 +1171,7 @@ attend_kernel(const __grid_constant__ AttendArgs a,
           x0 = pk[mt][0];
           x1 = pk[mt][NR - 1];
         }
-        if (!__any_sync(0xFFFFFFFFu, (x0 | x1) != 0u)) continue;   // whole step gated
+        if (gate && !__any_sync(0xFFFFFFFFu, (x0 | x1) != 0u)) continue;   // whole step gated
         const uint32_t b0 = transpose8x8(x0), b1 = transpose8x8(x1);
         if (BV == 2) {
           // lane gq reads D/32 bytes (D/8 coordinates) of the rows of
@@ -1091,10 +1227,10 @@ attend_kernel(const __grid_constant__ AttendArgs a,
           load_chunk<CBV>(smem, r0p + 8 * Gm::RVS, v1);
 #pragma unroll
           for (int r = 0; r < NPV; ++r) {
-            const uint32_t y0 = lds<uint32_t>(smem, pair_code_shifted<BV, 7>(v0, 2 * r) | lbV);
-            const uint32_t y1 = lds<uint32_t>(smem, pair_code_shifted<BV, 7>(v0, 2 * r + 1) | lbV);
-            const uint32_t y2 = lds<uint32_t>(smem, pair_code_shifted<BV, 7>(v1, 2 * r) | lbV);
-            const uint32_t y3 = lds<uint32_t>(smem, pair_code_shifted<BV, 7>(v1, 2 * r + 1) | lbV);
+            const uint32_t y0 = lds<uint32_t>(smem, pair_code_shifted<BV, Gm::VSHIFT>(v0, 2 * r) | lbV);
+            const uint32_t y1 = lds<uint32_t>(smem, pair_code_shifted<BV, Gm::VSHIFT>(v0, 2 * r + 1) | lbV);
+            const uint32_t y2 = lds<uint32_t>(smem, pair_code_shifted<BV, Gm::VSHIFT>(v1, 2 * r) | lbV);
+            const uint32_t y3 = lds<uint32_t>(smem, pair_code_shifted<BV, Gm::VSHIFT>(v1, 2 * r + 1) | lbV);
             mma16816(acc[r], transpose8x8(y0), transpose8x8(y1), transpose8x8(y2),
                      transpose8x8(y3), b0, b1);
           }
@@ -1107,6 +1243,19 @@ attend_kernel(const __grid_constant__ AttendArgs a,
       }
     }
     jdone += nw;
+    nskip += nsk0 + nsk1;
+    if (a.head_skipped && gate) {             // per (sequence, query head) gate counts
+#pragma unroll
+      for (int o = (NT == 1 ? 2 : 4); o < 32; o <<= 1) {
+        nsk0 += __shfl_xor_sync(0xFFFFFFFFu, nsk0, o);
+        nsk1 += __shfl_xor_sync(0xFFFFFFFFu, nsk1, o);
+      }
+      if (gq == 0 && (NT == 2 || tq < 2)) {
+        unsigned int* hk = a.head_skipped + (size_t)b * a.n_q_heads + (size_t)g * GQ + hs0;
+        if (hv0 && nsk0) atomicAdd(hk, nsk0);
+        if (hv1 && nsk1) atomicAdd(hk + 1, nsk1);
+      }
+    }
 
     // ---- per-warp softmax sums over the lanes holding the same heads
 #pragma unroll
@@ -1143,7 +1292,7 @@ attend_kernel(const __grid_constant__ AttendArgs a,
     if (!finalize) {
       const int sigma = b * H + g;
       const long long last = seg_first + nbl - 1;
-      const int c_first = cta_of(seg_first, NB, Geff), c_last = cta_of(last, NB, Geff);
+      const int c_first = cta_of(seg_first, Ctot, Geff), c_last = cta_of(last, Ctot, Geff);
       const int n_parts = c_last - c_first + 1;
       float* slot = a.slots + (size_t)(cta + sigma) * GQ * (D + 2);
       for (int i = tid; i < GQ * D; i += kThreads) slot[i] = fin[i];
@@ -1259,7 +1408,7 @@ attend_kernel(const __grid_constant__ AttendArgs a,
         }
       }
     }
-    pos += nseg;
+    pos = next_pos;
     ++seg_iter;
     __syncthreads();                                  // misc / fin / q~ reuse
   }
@@ -1272,7 +1421,7 @@ attend_kernel(const __grid_constant__ AttendArgs a,
 }
 
 inline int sm_count() {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
   if (!cached[dev]) {
@@ -1288,7 +1437,8 @@ template <int BK, int BV, int NT, int D>
 cudaError_t launch_one(const AttendArgs& a, const Codebook& cbk, const Codebook& cbv,
                        const SignMask& sm, int n_ctas, cudaStream_t stream) {
   using Gm = Geo<BK, BV, D>;
-  static bool configured[64] = {false};
+  // set once per device (idempotent; atomic so that concurrent first calls do not race)
+  static std::atomic<bool> configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || !configured[dev]) {
@@ -1328,6 +1478,11 @@ cudaError_t launch_pair(const AttendArgs& a, const Codebook& cbk, const Codebook
 template <int D>
 cudaError_t launch_attend_d(const AttendArgs& a, const Codebook& cbk, const Codebook& cbv,
                             const SignMask& sm, int n_ctas, cudaStream_t stream) {
+#ifdef TQ_TEST_INJECT_WAIT_FAULTS
+  // the wait test build holds K4/V2 only
+  if (a.bits_k * 8 + a.bits_v != 4 * 8 + 2) return cudaErrorNotSupported;
+  return launch_pair<4, 2, D>(a, cbk, cbv, sm, n_ctas, stream);
+#else
   switch (a.bits_k * 8 + a.bits_v) {
     case 4 * 8 + 2: return launch_pair<4, 2, D>(a, cbk, cbv, sm, n_ctas, stream);
     case 3 * 8 + 2: return launch_pair<3, 2, D>(a, cbk, cbv, sm, n_ctas, stream);
@@ -1340,6 +1495,7 @@ cudaError_t launch_attend_d(const AttendArgs& a, const Codebook& cbk, const Code
     case 3 * 8 + 4: return launch_pair<3, 4, D>(a, cbk, cbv, sm, n_ctas, stream);
     default: return cudaErrorInvalidValue;
   }
+#endif
 }
 
 }  // namespace tq

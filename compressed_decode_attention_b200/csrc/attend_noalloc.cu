@@ -7,10 +7,14 @@
 // host application that owns all device allocations. For them this entry
 // point takes its scratch from one fixed array compiled into the library.
 //
-// The array lives for as long as the library is loaded, on every device that
-// loads it, and is shared by every call on that device. Its size caps the
-// problem: batch · n_q_heads <= 54530 / 23887 / 8033 at d = 64 / 128 / 256
-// (see kNoAllocScratchBytes).
+// The array is created on a device together with the library's device code.
+// Under CUDA's default lazy module loading that happens on the first use of
+// that code on the device, which for a caller of this entry point alone is
+// the address lookup of its first call: that first call can allocate (the
+// module and the array) and belongs in initialization, outside any stream
+// capture. The array is kept until the process exits and is shared by every
+// call on that device. Its size caps the problem: batch · n_q_heads <= 54530
+// / 23887 / 8033 at d = 64 / 128 / 256 (see kNoAllocScratchBytes).
 #include <mutex>
 
 #include "tq.h"
@@ -30,7 +34,9 @@ std::mutex g_scratch_mutex;
 
 // Device address of the scratch array on the current device. The name of a
 // __device__ array in host code only stands in for it; the address has to be
-// queried once per device with that device current.
+// queried once per device with that device current. It is kept for the life
+// of the process, so the entry point must not be used on a device after
+// cudaDeviceReset (which unloads the module and frees the array).
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

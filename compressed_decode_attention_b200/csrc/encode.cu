@@ -15,6 +15,7 @@
 //   index   zeta = z/n compared as z against n·t (symmetric half table),
 //           counted with compare-and-set results
 //   pack    the lane's 32 indices are 4·bits contiguous bytes of the row
+#include <atomic>
 #include "encode_common.cuh"
 
 namespace tq {
@@ -68,7 +69,7 @@ template <int D>
 cudaError_t launch_encode_d(const EncodeArgs& a, const Codebook& cbk, const Codebook& cbv,
                             const SignMask& sm, cudaStream_t stream) {
   // SM count of the current device, looked up once per device
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64] = {};
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) {
     if (!cached[dev]) {

@@ -24,6 +24,7 @@
 //   PV       A = softmax weight x V norm (fp16, from the score registers),
 //            B = V tile (ldmatrix.trans)
 // Output per row: D⊙(H·(acc/l))/d with in-register and shuffle stages.
+#include <atomic>
 #include "attend_kernel.cuh"
 
 namespace tq {
@@ -511,7 +512,8 @@ template <int BK, int BV>
 cudaError_t launch_prefill_bits(const PrefillArgs& a, const Codebook& cbk, const Codebook& cbv,
                                 const SignMask& sm, cudaStream_t stream) {
   using G = PfGeo<BK, BV>;
-  static bool configured[64] = {false};
+  // set once per device (idempotent; atomic so that concurrent first calls do not race)
+  static std::atomic<bool> configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || !configured[dev]) {

@@ -26,6 +26,7 @@
 //   weights as 16-byte shared-memory broadcasts. Measured: 256 or 128
 //   positions per CTA repeat the prologue too often, 1024 leave too few
 //   CTAs for the latency-bound loop.
+#include <atomic>
 #include <math.h>
 
 #include "encode_common.cuh"
@@ -459,7 +460,8 @@ cudaError_t launch_encode_db(const QjlEncodeArgs& a, const Codebook& cb, const S
                              cudaStream_t stream) {
   using G = QjlEncGeo<D>;
   // the shared-memory opt-in is per device
-  static bool configured[64] = {false};
+  // set once per device (idempotent; atomic so that concurrent first calls do not race)
+  static std::atomic<bool> configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || !configured[dev]) {

@@ -84,6 +84,7 @@ struct AttendArgs {
   float* slots;              // partial (acc[gqa][d], m/l[gqa][2]) per slot
   int* dev_status;
   unsigned long long* skipped;
+  unsigned int* head_skipped;  // [batch][n_q_heads] gated positions per head, or nullptr
   void* out;
   int out_dtype;
   // Context-parallel slice: out is float [batch][n_q_heads][d + 2] of

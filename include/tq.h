@@ -71,7 +71,7 @@
 extern "C" {
 #endif
 
-#define TQ_ABI_VERSION 6
+#define TQ_ABI_VERSION 7
 
 /* Tokens per sparse-V block; split boundaries are multiples of this. */
 #define TQ_SPARSE_V_BLOCK 64
@@ -229,6 +229,29 @@ int tq_attend(const void* q, int q_dtype,
               void* workspace, size_t workspace_bytes, int* dev_status,
               unsigned long long* sparse_v_skipped,
               void* out, int out_dtype, void* stream);
+
+/*
+ * tq_attend_gate_counts — tq_attend that also reports, for every (sequence,
+ * query head), how many positions the sparse-V gate left out of that head's
+ * V accumulation [TQPLUS §2 Sparse V; the gate rule is frozen above]. Meant
+ * for verifying the gate head by head; the attention itself is tq_attend's.
+ *
+ *   head_skipped  uint32 [batch][n_q_heads] on the device, 4-byte aligned,
+ *               not NULL (TQ_ERR_INVALID_ARG): entry (b, h) is atomically
+ *               incremented by the number of positions t < L_b gated for
+ *               head h (the caller zeroes it). Nothing is added with the
+ *               gate off (sparse_v_thresh <= 0).
+ * All other arguments, results and errors are tq_attend's.
+ */
+int tq_attend_gate_counts(const void* q, int q_dtype,
+                          const uint8_t* packed_k, const uint16_t* norms_k,
+                          const uint8_t* packed_v, const uint16_t* norms_v,
+                          const int32_t* ctx_lens, int batch, int n_q_heads,
+                          int gqa_ratio, int d, int bits_k, int bits_v, uint64_t seed,
+                          int cap_tok, float sparse_v_thresh, int n_ctas,
+                          void* workspace, size_t workspace_bytes, int* dev_status,
+                          unsigned long long* sparse_v_skipped, unsigned int* head_skipped,
+                          void* out, int out_dtype, void* stream);
 
 /*
  * tq_attend_append — one decode step in one launch: append the new token of
@@ -460,14 +483,21 @@ int tq_qjl_scores(const void* q, int q_dtype, const uint8_t* packed_k, const uin
  *
  * Same arguments and results as tq_attend, without workspace and
  * workspace_bytes: the scratch is one fixed 16 MiB device array inside the
- * library, allocated when the library is loaded, on every device that loads
- * it, and kept until the process exits. This call allocates and frees no
- * memory.
+ * library, created on each device together with the library's device code
+ * and kept until the process exits. The call itself allocates and frees no
+ * memory, with one exception on each device's first use:
+ *   - Under CUDA's default lazy module loading, a device gets the library's
+ *     device code, and with it the 16 MiB array, only when that code is
+ *     first used there. The first tq_attend_noalloc call on a device looks
+ *     up the array's address, which loads the module if nothing else has.
+ *     Make that first call during initialization, before any stream capture
+ *     (or set CUDA_MODULE_LOADING=EAGER, which creates the array with the
+ *     CUDA context). Later calls reuse the address.
+ *   - The address is kept for the life of the process: do not use this
+ *     entry point on a device after cudaDeviceReset.
  *   - Limit: the problem's tq_attend_workspace_size must fit 16 MiB, i.e.
  *     batch · n_q_heads <= 54530 / 23887 / 8033 at d = 64 / 128 / 256;
  *     larger problems return TQ_ERR_UNSUPPORTED.
- *   - The first call on a device looks up the array's device address (a
- *     host-side set-up); make that first call before any stream capture.
  *   - Every call on a device shares the array. Each call first clears the
  *     array's counter region on `stream`; calls whose execution overlaps on
  *     the GPU (other streams, other threads) race on it and give undefined

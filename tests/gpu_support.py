@@ -154,9 +154,69 @@ def gpu_encode(kv_bits, dtype, bits_k, bits_v, seed, cap=None, tok_offset=0,
     return host(pk), host(nk), host(pv), host(nv), int(st.item())
 
 
+# Error bound of the kernel's fp32 scores against the oracle's float64 ones,
+# used to find the positions where the two may take the sparse-V gate
+# decision differently. A score s_t = (nK_t/sqrt d)·sum_i q~_i·c_i/sqrt(d) is
+# formed on tensor cores from fp16 high+low parts of q~ and of the codebook
+# values (the missing low x low term and the rounding of the low parts leave
+# < 3·2^-22 of each product), accumulated in fp32 over 128 products, eight
+# k-steps and three partial products (about ten roundings of at most 2^-23
+# of the running magnitude), then scaled twice by exact factors with one
+# rounding each: < 2^-19 of the sum S_t of the products' magnitudes in all.
+# So |ds_t| <= SCORE_EPS_ABS·S_t + SCORE_EPS_REL·|s_t|, with a factor of 8
+# to spare in the first term.
+SCORE_EPS_ABS = 2.0 ** -16
+SCORE_EPS_REL = 2.0 ** -22
+
+
+def _gate_table(q, pk, nk, L, gqa, bk, seed, tau):
+    """Worker: (gated count, ambiguous count) per query head of one kv head.
+    A position is ambiguous when its float64 gate value exp(s - M_blk) lies
+    within the score error bound (relative, in the log domain) of tau."""
+    from oracle import attention, codec, rotation
+    d = q.shape[-1]
+    idx = codec.unpack(pk, bk, d)
+    gv = attention.gate_values(q, idx, nk, bk, seed)             # [g, L]
+    nkf = nk.view(np.float16).astype(np.float64)
+    q_rot = rotation.rotate(q, seed)
+    k_rot = codec.dequant_rotated(idx, bk)
+    s = (q_rot @ k_rot.T) * nkf / np.sqrt(d)
+    mag = (np.abs(q_rot) @ np.abs(k_rot).T) * nkf / np.sqrt(d)
+    bound = SCORE_EPS_ABS * mag + SCORE_EPS_REL * np.abs(s)
+    nblk = (L + attention.GATE_BLOCK - 1) // attention.GATE_BLOCK
+    pad = np.zeros((q.shape[0], nblk * attention.GATE_BLOCK))
+    pad[:, :L] = bound
+    bmax = np.repeat(pad.reshape(q.shape[0], nblk, -1).max(axis=2), attention.GATE_BLOCK, axis=1)[:, :L]
+    with np.errstate(divide="ignore"):
+        amb = np.abs(np.log(gv) - np.log(tau)) <= bound + bmax
+    return (gv < tau).sum(axis=1), amb.sum(axis=1)
+
+
+def oracle_gate_table(q64, pk, nk, ctx, gqa, bk, seed, tau):
+    """Per (sequence, query head): the oracle's gated-position count and the
+    number of positions whose decision the score error bound leaves open."""
+    B, H = pk.shape[:2]
+    Hq = q64.shape[1]
+    cnt = np.zeros((B, Hq), np.int64)
+    amb = np.zeros((B, Hq), np.int64)
+    futs = []
+    for b in range(B):
+        L = int(min(max(int(ctx[b]), 0), pk.shape[2]))
+        for g in range(H):
+            if L > 0:
+                hs = slice(g * gqa, (g + 1) * gqa)
+                futs.append((b, hs, pool().submit(_gate_table, q64[b, hs], pk[b, g, :L],
+                                                  nk[b, g, :L], L, gqa, bk, seed, tau)))
+    for b, hs, f in futs:
+        cnt[b, hs], amb[b, hs] = f.result()
+    return cnt, amb
+
+
 def gpu_attend(q_bits, q_dtype, pk, nk, pv, nv, ctx, gqa, bk, bv, seed, tau=0.0,
-               n_ctas=0, out_dtype=None, workspace=None):
-    """tq_attend on host arrays; returns (out float32/bits, status, skipped)."""
+               n_ctas=0, out_dtype=None, workspace=None, head_counts=False):
+    """tq_attend on host arrays; returns (out float32/bits, status, skipped),
+    plus the per (sequence, query head) gate counts of tq_attend_gate_counts
+    when head_counts is set."""
     import torch
     import compressed_decode_attention_b200 as tq
     B, H, cap = pk.shape[:3]
@@ -174,10 +234,16 @@ def gpu_attend(q_bits, q_dtype, pk, nk, pv, nv, ctx, gqa, bk, bv, seed, tau=0.0,
     sk = torch.zeros(1, dtype=torch.int64, device="cuda")
     qt = dev(q_bits)
     q_enum = {"f16": tq.TQ_F16, "bf16": tq.TQ_BF16, "f32": tq.TQ_F32}[q_dtype]
-    tq.tq_attend(qt, q_enum, dev(pk), dev(nk), dev(pv), dev(nv),
-                 dev(np.asarray(ctx, np.int32)), B, Hq, gqa, d, bk, bv, seed, cap, tau,
-                 n_ctas, ws, ws_bytes, out, out_dtype, dev_status=st, sparse_v_skipped=sk)
+    args = (qt, q_enum, dev(pk), dev(nk), dev(pv), dev(nv), dev(np.asarray(ctx, np.int32)),
+            B, Hq, gqa, d, bk, bv, seed, cap, tau, n_ctas, ws, ws_bytes)
+    if head_counts:
+        hk = torch.zeros((B, Hq), dtype=torch.int32, device="cuda")
+        tq.tq_attend_gate_counts(*args, hk, out, out_dtype, dev_status=st, sparse_v_skipped=sk)
+    else:
+        tq.tq_attend(*args, out, out_dtype, dev_status=st, sparse_v_skipped=sk)
     torch.cuda.synchronize()
+    if head_counts:
+        return host(out), int(st.item()), int(sk.item()), hk.cpu().numpy().astype(np.int64)
     return host(out), int(st.item()), int(sk.item())
 
 

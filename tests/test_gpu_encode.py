@@ -55,22 +55,51 @@ def test_encode_k4v3_batched_serving_sequence():
              count_rule=True)
 
 
-@pytest.mark.parametrize("layer", [0, 31])
-def test_encode_bulk_prefill_layer_sampled(layer):
-    """Full-size layer launch (32768 tokens x 8 heads), oracle on a sample."""
+@pytest.mark.parametrize("layer", [0, 1, 30, 31])
+def test_encode_bulk_prefill_whole_layer(layer):
+    """Four whole layers of the bulk-encode workload (32768 tokens x 8 kv
+    heads each, the bench's launch), every vector checked against the
+    oracle; the exempted near-threshold count is bounded per layer."""
     w = S.WORKLOADS["bulk_prefill_encode"]
     kv = S.kv_bits(w, 0, w.ctx, layer=layer)
     pk, nk, pv, nv, st = gpu_encode(kv, w.dtype, w.bits_k, w.bits_v, SEED)
-    rng = np.random.default_rng(layer)
-    toks = np.sort(rng.choice(w.ctx, size=2048, replace=False))
-    sub = kv[:, toks]
-    stats = []
+    assert st == 0
+    _compare(kv, w.dtype, w.bits_k, w.bits_v, SEED, pk, nk, pv, nv, parallel=True,
+             count_rule=True)
+
+
+def test_round_trip_bulk_layer_quality():
+    """Encode -> dequant on the GPU over one whole bulk layer: the mean
+    rotated-domain squared error ||y - y^||^2 (y = R x/||x||, per-coordinate
+    MSE in N(0,1) units) equals the oracle's on the same vectors, and for V
+    (plain N(0,1) input) it lies within [0.95, 1.01] of the codebook MSE D_2
+    (the finite-d marginal has lighter tails than N(0,1))."""
+    import torch
+    import compressed_decode_attention_b200 as tq
+    from oracle import codebook as ocb, rotation
+    w = S.WORKLOADS["bulk_prefill_encode"]
+    kv = S.kv_bits(w, 0, w.ctx, layer=2)
+    pk, nk, pv, nv, st = gpu_encode(kv, w.dtype, w.bits_k, w.bits_v, SEED)
+    H, n, d = w.n_kv_heads, w.ctx, w.d
     for which, bits, rows, nb in ((0, w.bits_k, pk, nk), (1, w.bits_v, pv, nv)):
-        idx_o, nb_o, mg = oracle_encode_heads(sub, w.dtype, which, bits, SEED)
-        idx_g = codec.unpack(rows[:, toks].reshape(-1, rows.shape[-1]), bits, w.d)
-        stats.append(check_indices(idx_g.reshape(idx_o.shape), idx_o, mg))
-        check_norms(nb[:, toks], nb_o)
-    check_near_fraction(stats)
+        out = torch.empty((H, n, d), dtype=torch.float32, device="cuda")
+        tq.tq_dequant(dev(rows), dev(nb), n, H, d, bits, SEED, n, 1, out)
+        torch.cuda.synchronize()
+        yhat_g = host(out).astype(np.float64)
+        idx_o, _, _ = oracle_encode_parallel(kv, w.dtype, which, bits, SEED)
+        mse_g, mse_o = 0.0, 0.0
+        for h in range(H):
+            x = codec.promote(kv[which, :, h], w.dtype)
+            y = rotation.rotate(x / np.linalg.norm(x, axis=1, keepdims=True), SEED)
+            mse_g += np.sum((y - yhat_g[h]) ** 2)
+            mse_o += np.sum((y - codec.dequant_rotated(idx_o[h].astype(np.int64), bits)) ** 2)
+        mse_g /= H * n
+        mse_o /= H * n
+        print(f"bits {bits}: rotated MSE gpu {mse_g:.6f} oracle {mse_o:.6f}")
+        assert abs(mse_g - mse_o) <= 1e-6 * mse_o
+        if which == 1:
+            c, t = ocb.lloyd_max_normal(bits)
+            assert 0.95 <= mse_g / ocb.quantizer_mse(c, t) <= 1.01
 
 
 @pytest.mark.parametrize("bk,bv", [(2, 2), (3, 3), (4, 4), (2, 4), (3, 2)])

@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol():
 def test_abi_version_and_status_strings():
     hdr = open(os.path.join(ROOT, "include", "tq.h")).read()
     assert tq.tq_abi_version() == int(re.search(r"#define TQ_ABI_VERSION (\d+)", hdr).group(1))
-    assert tq.tq_abi_version() == 6
+    assert tq.tq_abi_version() == 7
     assert tq.status_string(0) == "TQ_OK"
     assert tq.status_string(2) == "TQ_ERR_UNSUPPORTED"
 
@@ -269,3 +269,17 @@ def test_prefill_workspace_size_and_split_choice():
     assert tq.tq_prefill_workspace_size(2, 16, 8, 96, 3) == 0
     assert 1 <= tq.tq_prefill_splits(1, 1024, 32, 4) <= 8
     assert tq.tq_prefill_splits(0, 1024, 32, 4) == 1
+
+
+@pytest.mark.parametrize("head_skipped,want", [
+    (None, tq.TQ_ERR_INVALID_ARG),          # the counts array is required
+    (FAKE + 2, tq.TQ_ERR_INVALID_ARG),      # not 4-byte aligned
+])
+def test_gate_counts_rejects_bad_count_array(head_skipped, want):
+    """tq_attend_gate_counts checks its per-head count array on the host,
+    before any CUDA call; every other argument is valid."""
+    ws = tq.tq_attend_workspace_size(1, 8, 64, 128)
+    st = tq.lib().tq_attend_gate_counts(FAKE, tq.TQ_F16, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 4,
+                                         128, 4, 2, 0, 64, 1e-3, 0, FAKE, ws, None, None,
+                                         head_skipped, FAKE, tq.TQ_F32, None)
+    assert st == want
