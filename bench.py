@@ -257,8 +257,9 @@ def device_kv(w, layer, n_tok, gen):
         idx = torch.as_tensor(ch[h], device="cuda")
         if w.outlier == "x20":
             x[0, :, h, idx] *= 20.0
-        elif w.outlier == "laplace":        # inverse CDF of Laplace(0, 1)
-            u = torch.rand((n_tok, len(ch[h])), generator=gen, device="cuda") - 0.5
+        elif w.outlier == "laplace":        # inverse CDF of Laplace(0, 1), u in (-1/2, 1/2)
+            u = torch.rand((n_tok, len(ch[h])), generator=gen, device="cuda") * (1 - 2.0 ** -23) \
+                + (2.0 ** -24 - 0.5)
             x[0, :, h, idx] = -torch.sign(u) * torch.log1p(-2.0 * u.abs())
     return (x.bfloat16() if w.dtype == "bf16" else x.half()).view(torch.int16)
 
@@ -999,6 +1000,60 @@ def run_reference(args, rank, world):
     }
 
 
+def profile_case(name, reps):
+    """A few eager launches of one kernel's workload for an ncu capture
+    (prints no bench line): 'llama' = tq_attend over 8 Llama-3-8B-shaped
+    layer caches, 'batched' = one serving-scale call, 'qwen' = tq_attend over
+    2 Qwen-14B-shaped layers, 'encode' = tq_encode of 4 bulk-prefill layers.
+    Caches hold tq_encode'd seeded data."""
+    import torch
+    import compressed_decode_attention_b200 as tq
+    torch.cuda.set_device(0)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(S.DATA_SEED)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    seed = S.SIGN_SEED
+    if name == "encode":
+        w = S.WORKLOADS[ENCODE_WORKLOAD]
+        caches = LayerCaches(w, 4, None)
+        kvs = [device_kv(w, l, w.ctx, gen) for l in range(4)]
+        for _ in range(reps):
+            for l in range(4):
+                tq.tq_encode(kvs[l], tq.TQ_F16, w.ctx, w.n_kv_heads, w.d, w.bits_k, w.bits_v, seed,
+                             caches.pk[l], caches.pv[l], caches.nk[l], caches.nv[l], w.cap_tok, 0,
+                             status)
+        torch.cuda.synchronize()
+        return
+    w = S.WORKLOADS[{"llama": WORKLOAD, "batched": BATCHED_WORKLOAD, "qwen": QWEN_WORKLOAD}[name]]
+    layers = {"llama": 8, "batched": 1, "qwen": 2}[name]
+    ctx_h = S.ctx_lens(w)
+    B, H, d, cap = w.batch, w.n_kv_heads, w.d, w.cap_tok
+    rk, rv = d * w.bits_k // 8, d * w.bits_v // 8
+    kvdt = tq.TQ_BF16 if w.dtype == "bf16" else tq.TQ_F16
+    cs = []
+    for _ in range(layers):
+        pk = torch.zeros((B, H, cap, rk), dtype=torch.uint8, device="cuda")
+        pv = torch.zeros((B, H, cap, rv), dtype=torch.uint8, device="cuda")
+        nk = torch.zeros((B, H, cap), dtype=torch.int16, device="cuda")
+        nv = torch.zeros((B, H, cap), dtype=torch.int16, device="cuda")
+        for b in range(B):
+            kvb = device_kv(w, 0, int(ctx_h[b]), gen)
+            tq.tq_encode(kvb, kvdt, int(ctx_h[b]), H, d, w.bits_k, w.bits_v, seed, pk[b], pv[b],
+                         nk[b], nv[b], cap, 0, status)
+        cs.append((pk, nk, pv, nv))
+    q = torch.randn((B, w.n_q_heads, d), generator=gen, device="cuda")
+    q = q.bfloat16() if w.dtype == "bf16" else q.half()
+    out = torch.empty_like(q)
+    ctx = torch.from_numpy(ctx_h).cuda()
+    wsb = tq.tq_attend_workspace_size(B, w.n_q_heads, cap, d)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    for _ in range(reps):
+        for pk, nk, pv, nv in cs:
+            tq.tq_attend(q, kvdt, pk, nk, pv, nv, ctx, B, w.n_q_heads, w.gqa, d, w.bits_k,
+                         w.bits_v, seed, cap, w.tau, 0, ws, wsb, out, kvdt, dev_status=status)
+    torch.cuda.synchronize()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1007,7 +1062,12 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=["llama", "batched", "qwen", "encode"],
+                    help="only launch one kernel's workload a few times (for ncu captures)")
     args = ap.parse_args(argv)
+    if args.profile_case:
+        profile_case(args.profile_case, args.steps)
+        return 0
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     rank, world, local_rank = dist_env()

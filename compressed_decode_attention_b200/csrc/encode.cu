@@ -79,6 +79,12 @@ cudaError_t launch_encode_d(const EncodeArgs& a, const Codebook& cbk, const Code
     }
     sms = cached[dev];
   }
+  // d = 128 with a few tiles of tokens: the tensor-core encode (the FWHT
+  // kernel below when the driver's tensor-map call is unavailable)
+  if (encode_tc_applies(a)) {
+    const cudaError_t e = launch_encode_tc(a, cbk, cbv, sm, sms, stream);
+    if (e != cudaErrorNotSupported) return e;
+  }
   // grid.x: enough tile blocks that all (head, K/V) pairs cover every SM
   // about eight times; each block strides over its head's tiles
   constexpr int kTokens = kEncThreads / (D / 32);

@@ -83,24 +83,15 @@ __device__ __forceinline__ void rotate_vector(float (&x)[32], int sub, unsigned 
   }
 }
 
-template <int BITS, int LPV>
-__device__ __forceinline__ void encode_vector(
-    float (&x)[32], const Codebook& cb, int sub, unsigned gmask,
-    uint8_t* row_dst, uint16_t* norm_dst, int* dev_status) {
+// Lloyd-Max indices of 32 rotated coordinates z (unnormalized Hadamard
+// domain, z = H·(D⊙x)) of a vector whose norm is n, packed LSB-first into
+// BITS words: idx = #{j : z/n >= t_j}. Shared by the FWHT encode (4 lanes
+// per vector) and the tensor-core encode (one thread per vector, four calls),
+// so the two take their decisions with the same arithmetic.
+template <int BITS>
+__device__ __forceinline__ void quantize_pack(const float (&x)[32], float n, const Codebook& cb,
+                                              uint32_t (&words)[BITS]) {
   constexpr int kHalf = 1 << (BITS - 1);
-  // ||x||^2 over the group of LPV lanes (pairs of coordinates per fma)
-  float2 ss2 = make_float2(0.f, 0.f);
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const float2 v = make_float2(x[2 * j], x[2 * j + 1]);
-    ss2 = f2fma(v, v, ss2);
-  }
-  float ss = ss2.x + ss2.y;
-#pragma unroll
-  for (int o = 1; o < LPV; o <<= 1) ss += __shfl_xor_sync(gmask, ss, o);
-  const float n = sqrtf(ss);
-
-  rotate_vector<LPV>(x, sub, gmask);
 
   // idx = #{j : z/n >= t_j} over the symmetric table (t_{half-1} = 0), on
   // the FMA pipe. With a = |z| and the positive thresholds t_k (k = 1 ..
@@ -135,7 +126,8 @@ __device__ __forceinline__ void encode_vector(
   constexpr int HALF = NTH / 2;
   const float tmid = (n > 0.f ? n : 1.f) * cb.threshold[kHalf + HALF];
 
-  uint32_t words[BITS] = {};
+#pragma unroll
+  for (int w = 0; w < BITS; ++w) words[w] = 0;
 #pragma unroll
   for (int i = 0; i < 32; i += 2) {
     const float a0 = fabsf(x[i]), a1 = fabsf(x[i + 1]);
@@ -177,6 +169,27 @@ __device__ __forceinline__ void encode_vector(
     }
     words[w] -= c;
   }
+}
+
+template <int BITS, int LPV>
+__device__ __forceinline__ void encode_vector(
+    float (&x)[32], const Codebook& cb, int sub, unsigned gmask,
+    uint8_t* row_dst, uint16_t* norm_dst, int* dev_status) {
+  // ||x||^2 over the group of LPV lanes (pairs of coordinates per fma)
+  float2 ss2 = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const float2 v = make_float2(x[2 * j], x[2 * j + 1]);
+    ss2 = f2fma(v, v, ss2);
+  }
+  float ss = ss2.x + ss2.y;
+#pragma unroll
+  for (int o = 1; o < LPV; o <<= 1) ss += __shfl_xor_sync(gmask, ss, o);
+  const float n = sqrtf(ss);
+
+  rotate_vector<LPV>(x, sub, gmask);
+  uint32_t words[BITS];
+  quantize_pack<BITS>(x, n, cb, words);
 
   if constexpr (BITS == 4) {
     *reinterpret_cast<uint4*>(row_dst + 16 * sub) =

@@ -51,6 +51,10 @@ struct EncodeArgs {
 cudaError_t launch_encode(const EncodeArgs& a, const Codebook& cbk,
                           const Codebook& cbv, const SignMask& sm,
                           cudaStream_t stream);
+// Tensor-core encode (encode_tc.cu): d = 128 and enough tokens to fill tiles.
+bool encode_tc_applies(const EncodeArgs& a);
+cudaError_t launch_encode_tc(const EncodeArgs& a, const Codebook& cbk, const Codebook& cbv,
+                             const SignMask& sm, int sms, cudaStream_t stream);
 
 struct DequantArgs {
   int d;

@@ -12,13 +12,12 @@ import pytest
 
 import synthetic as S
 from gpu_support import (check_indices, check_norms, dev, gpu_attend, gpu_encode, host,
-                         oracle_attend, oracle_encode_heads)
-from oracle import attention, codec
+                         oracle_attend, oracle_encode_heads, oracle_gate_table)
+from oracle import codec
 
 pytestmark = pytest.mark.gpu
 SEED = S.SIGN_SEED
 ATOL = 2e-3
-GATE_WINDOW = 1e-3
 DIMS = [64, 256]
 
 
@@ -94,21 +93,6 @@ def _cache(bk, bv, B, Hkv, cap, ctx, seed, rng, d):
     return pk, nk, pv, nv
 
 
-def _gate_ambiguous(q64, pk, nk, ctx, gqa, bk, seed, tau):
-    n = 0
-    B, H = pk.shape[:2]
-    d = q64.shape[-1]
-    for b in range(B):
-        L = int(min(ctx[b], pk.shape[2]))
-        for g in range(H):
-            if L <= 0:
-                continue
-            idx = codec.unpack(pk[b, g, :L], bk, d)
-            gv = attention.gate_values(q64[b, g * gqa:(g + 1) * gqa], idx, nk[b, g, :L], bk, seed)
-            n += int(np.sum(np.abs(gv / tau - 1.0) < GATE_WINDOW))
-    return n
-
-
 @pytest.mark.parametrize("d", DIMS)
 @pytest.mark.parametrize("bk,bv,gqa,tau,qscale,n_ctas", [
     (4, 2, 4, 0.0, 1.0, 0),
@@ -125,12 +109,17 @@ def test_attend_head_dims(d, bk, bv, gqa, tau, qscale, n_ctas):
     qb = S.f16_bits(rng.standard_normal((len(ctx), Hkv * gqa, d)) * qscale)
     q64 = codec.promote(qb, "f16")
     want, ng_o = oracle_attend(q64, pk, nk, pv, nv, ctx, gqa, bk, bv, SEED, tau)
-    got, st, ng_g = gpu_attend(qb, "f16", pk, nk, pv, nv, ctx, gqa, bk, bv, SEED, tau=tau,
-                               n_ctas=n_ctas)
+    got, st, ng_g, heads_g = gpu_attend(qb, "f16", pk, nk, pv, nv, ctx, gqa, bk, bv, SEED,
+                                        tau=tau, n_ctas=n_ctas, head_counts=True)
     err = np.abs(got - want).max()
     print(f"d={d} K{bk}/V{bv} g={gqa}: max|err| = {err:.3e}, gated {ng_o}/{ng_g}")
     assert err <= ATOL
     assert st == 4                      # the empty sequence
     if tau > 0:
+        # per (sequence, query head): equal outside the score error band
         assert ng_o > 0
-        assert abs(ng_g - ng_o) <= _gate_ambiguous(q64, pk, nk, ctx, gqa, bk, SEED, tau)
+        cnt_o, amb = oracle_gate_table(q64, pk, nk, ctx, gqa, bk, SEED, tau)
+        assert cnt_o.sum() == ng_o and heads_g.sum() == ng_g
+        assert np.all(np.abs(heads_g - cnt_o) <= amb)
+    else:
+        assert ng_g == 0 and not heads_g.any()
