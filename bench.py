@@ -321,6 +321,13 @@ def run_gpu(args, rank, world, local_rank):
     # ---------------- bulk encode (prefill) of every layer: the encode metric
     kv_all = [device_kv(we, l, ctx, gen) for l in range(L)]
     status = torch.zeros(1, dtype=torch.int32, device=device)
+    section_status = {}
+
+    def take_status(name):
+        """The device status bits the section just run set (then cleared)."""
+        section_status[name] = int(status.item())
+        status.zero_()
+
 
     def encode_all():
         for l in range(L):
@@ -345,6 +352,7 @@ def run_gpu(args, rank, world, local_rank):
     enc_ms = reduce_max(e0.elapsed_time(e1) / enc_steps, device)
     enc_launches = enc_steps * L
 
+    take_status("encode")
     # ---------------- encode -> dequant round trip of the bulk workload: every
     # layer's K and V dequantized to the original domain (tq_dequant, timed)
     # and compared with the encoder input: the codec's quality
@@ -396,6 +404,7 @@ def run_gpu(args, rank, world, local_rank):
                                       / (dq_ms * 1e-3) / 1e9, 1)
     del dq
 
+    take_status("round_trip")
     # ---------------- stage-2 residual sketch (QJL) of the keys of QJL_LAYERS
     # layer caches, and the estimated scores of 32 query heads over them
     QL = min(QJL_LAYERS, L)
@@ -451,6 +460,7 @@ def run_gpu(args, rank, world, local_rank):
     del kv_all
     torch.cuda.empty_cache()
 
+    take_status("qjl")
     # ---------------- prefill attention: a 1024-token chunk at the end of an
     # 8192-token context (the chunk's rows are in the cache), 4 layers
     pf_layers, pf_ctx, pf_T = 4, PREFILL_CTX, PREFILL_TOKENS
@@ -502,6 +512,7 @@ def run_gpu(args, rank, world, local_rank):
     del pf_graph, pf, pf_q, pf_out, pf_ws
     torch.cuda.empty_cache()
 
+    take_status("prefill")
     # ---------------- decode step graphs
     # per-layer queries, new K/V and outputs are views of three contiguous
     # buffers, so that the end-to-end step moves each with one copy
@@ -567,6 +578,7 @@ def run_gpu(args, rank, world, local_rank):
     ms_step = reduce_max(ms_total / args.steps, device)
     launches += kernels_per_step * args.steps
 
+    take_status("decode_step")
     # ---------------- the attention kernel alone: per-launch time = a graph
     # of the L layers' launches (distinct caches, larger than L2) / L
     def attend_all():
@@ -589,6 +601,7 @@ def run_gpu(args, rank, world, local_rank):
     attend_ms_mean = reduce_max(a0.elapsed_time(a1) / (args.steps * L), device)
     launches += L * args.steps
 
+    take_status("attend")
     # ---------------- context parallelism, P slices emulated on this GPU: per
     # layer, one tq_attend_partial per slice of whole 64-position blocks
     # (views into the layer cache: row offset, cap_tok kept as the head
@@ -643,6 +656,7 @@ def run_gpu(args, rank, world, local_rank):
         launches += per * L * args.steps
         del g
 
+    take_status("context_parallel")
     # ---------------- attention at serving scale: the batched workload (64
     # sequences of U{1024..16384} positions, K4/V3, sparse-V gate 1e-6), two
     # layer caches alternating (2 x 0.97 GB of capacity, > L2), each encoded
@@ -699,6 +713,7 @@ def run_gpu(args, rank, world, local_rank):
     del bgraph, bcache, bq, bout, bws
     torch.cuda.empty_cache()
 
+    take_status("batched")
     # ---------------- the Qwen-14B-shaped long-context layer (40 q / 8 kv
     # heads, GQA 5, ctx 131072, K3/V2, bf16 with Laplace(0,1) values on 3 K
     # channels per head): QWEN_LAYERS layer caches encoded by tq_encode from
@@ -745,6 +760,7 @@ def run_gpu(args, rank, world, local_rank):
     del qgraph, qcache, qw_q, qw_out, qw_ws
     torch.cuda.empty_cache()
 
+    take_status("qwen14b")
     # ---------------- end to end: host inputs in, host output back, every step
     in_host = torch.empty(nq16 + nkv16, dtype=torch.int16).pin_memory()
     out_host = torch.empty((L, 1, w.n_q_heads, d), dtype=torch.float16).pin_memory()
@@ -773,7 +789,10 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = reduce_max(x0.elapsed_time(x1) / args.steps, device)
     launches += kernels_per_step * args.steps
-    st = int(status.item())
+    take_status("e2e")
+    st = 0
+    for v_ in section_status.values():
+        st |= v_
 
     per_layer_attend = attend_bytes(w, ctx)
     per_layer_encode = encode_bytes(w, H)
@@ -893,6 +912,7 @@ def run_gpu(args, rank, world, local_rank):
             "combine_ms": round(cp_times["combine"], 5),
             "record_bytes_per_slice": int(w.n_q_heads * (d + 2) * 4)},
         "device_status": st,
+        "device_status_by_section": section_status,
     }
     del step_graph, attend_graph, e2e_graph
     return res
@@ -1004,7 +1024,8 @@ def profile_case(name, reps):
     """A few eager launches of one kernel's workload for an ncu capture
     (prints no bench line): 'llama' = tq_attend over 8 Llama-3-8B-shaped
     layer caches, 'batched' = one serving-scale call, 'qwen' = tq_attend over
-    2 Qwen-14B-shaped layers, 'encode' = tq_encode of 4 bulk-prefill layers.
+    2 Qwen-14B-shaped layers, 'encode' = tq_encode of 4 bulk-prefill layers,
+    'prefill' = tq_prefill_attend of the prefill leg's chunk on one layer.
     Caches hold tq_encode'd seeded data."""
     import torch
     import compressed_decode_attention_b200 as tq
@@ -1022,6 +1043,27 @@ def profile_case(name, reps):
                 tq.tq_encode(kvs[l], tq.TQ_F16, w.ctx, w.n_kv_heads, w.d, w.bits_k, w.bits_v, seed,
                              caches.pk[l], caches.pv[l], caches.nk[l], caches.nv[l], w.cap_tok, 0,
                              status)
+        torch.cuda.synchronize()
+        return
+    if name == "prefill":
+        w = S.WORKLOADS[WORKLOAD]
+        ctx, T, H, d = PREFILL_CTX, PREFILL_TOKENS, w.n_kv_heads, w.d
+        caches = LayerCaches(dataclasses.replace(w, ctx=ctx, cap_tok=ctx), 1, None)
+        kv = device_kv(w, 0, ctx, gen)
+        tq.tq_encode(kv, tq.TQ_F16, ctx, H, d, w.bits_k, w.bits_v, seed, caches.pk[0],
+                     caches.pv[0], caches.nk[0], caches.nv[0], ctx, 0, status)
+        del kv
+        q = torch.randn((1, T, w.n_q_heads, d), generator=gen, device="cuda").half()
+        out = torch.empty_like(q)
+        ctx_dev = torch.full((1,), ctx, dtype=torch.int32, device="cuda")
+        splits = tq.tq_prefill_splits(1, T, w.n_q_heads, w.gqa)
+        wsb = tq.tq_prefill_workspace_size(1, T, w.n_q_heads, d, splits)
+        ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device="cuda")
+        for _ in range(reps):
+            tq.tq_prefill_attend_split(q, tq.TQ_F16, caches.pk[0], caches.nk[0], caches.pv[0],
+                                       caches.nv[0], ctx_dev, 1, T, w.n_q_heads, w.gqa, d,
+                                       w.bits_k, w.bits_v, seed, ctx, splits, ws, wsb, out,
+                                       tq.TQ_F16, dev_status=status)
         torch.cuda.synchronize()
         return
     w = S.WORKLOADS[{"llama": WORKLOAD, "batched": BATCHED_WORKLOAD, "qwen": QWEN_WORKLOAD}[name]]
@@ -1062,7 +1104,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-case", choices=["llama", "batched", "qwen", "encode"],
+    ap.add_argument("--profile-case", choices=["llama", "batched", "qwen", "encode",
+                                                      "prefill"],
                     help="only launch one kernel's workload a few times (for ncu captures)")
     args = ap.parse_args(argv)
     if args.profile_case:

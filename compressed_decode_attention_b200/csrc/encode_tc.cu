@@ -31,6 +31,7 @@
 #include <mutex>
 
 #include "encode_common.cuh"
+#include "tc_common.cuh"
 
 namespace tq {
 namespace {
@@ -51,67 +52,17 @@ constexpr long long kTcWaitLimit = 2000000000LL;    // cycles (~1 s)
 static_assert(kTmemCols == 512, "one CTA per SM holds all 512 TMEM columns");
 static_assert(kSmem <= 227 * 1024, "shared memory");
 
-__device__ __forceinline__ uint32_t saddr(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
+using tc::bar_arrive;
+using tc::bar_expect;
+using tc::bar_init;
+using tc::saddr;
+using tc::tmem_ld32;
+using tc::umma_desc;
+__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
+  return tc::bar_wait(bar, parity, kTcWaitLimit);
 }
-__device__ __forceinline__ void bar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void bar_expect(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void bar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool bar_try(uint32_t bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(done) : "r"(bar), "r"(parity) : "memory");
-  return done != 0;
-}
-// Bounded wait for the phase of the given parity; false if it gave up.
-__device__ __noinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
-  if (bar_try(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (!bar_try(bar, parity))
-    if (clock64() - t0 > kTcWaitLimit) return false;
-  return true;
-}
-
-// UMMA shared-memory descriptor of a K-major operand in the 128-byte swizzle
-// layout: 8-row groups of 128-byte rows 1024 bytes apart (stride byte
-// offset), start address advanced by 32 bytes per 16-element k-step inside
-// the swizzle row; descriptor version 1, layout type 2 (128-byte swizzle).
-__device__ __forceinline__ uint64_t umma_desc(uint32_t start) {
-  return (uint64_t)((start >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) |
-         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
-// Instruction descriptor of kind::f16: fp32 accumulator, A and B of the
-// input type (0 fp16, 1 bf16), both K-major, N = 128, M = 128.
 __host__ __device__ constexpr uint32_t umma_idesc(uint32_t fmt) {
-  return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(kDim >> 3) << 17) |
-         ((uint32_t)(kTile >> 4) << 24);
-}
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-      "%28, %29, %30, %31}, [%32];\n"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  return tc::umma_idesc(fmt, kTile, kDim);
 }
 
 // Item j of the CTA's list -> (K/V, kv head, tile).

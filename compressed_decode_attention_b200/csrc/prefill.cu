@@ -554,6 +554,11 @@ cudaError_t launch_prefill_bits(const PrefillArgs& a, const Codebook& cbk, const
 
 cudaError_t launch_prefill(const PrefillArgs& a, const Codebook& cbk, const Codebook& cbv,
                            const SignMask& sm, cudaStream_t stream) {
+  return launch_prefill_tc(a, cbk, cbv, sm, stream);
+}
+
+cudaError_t launch_prefill_mma_sync(const PrefillArgs& a, const Codebook& cbk,
+                                    const Codebook& cbv, const SignMask& sm, cudaStream_t stream) {
   switch (a.bits_k * 8 + a.bits_v) {
     case 4 * 8 + 2: return launch_prefill_bits<4, 2>(a, cbk, cbv, sm, stream);
     case 3 * 8 + 2: return launch_prefill_bits<3, 2>(a, cbk, cbv, sm, stream);
