@@ -469,6 +469,7 @@ def run_gpu(args, rank, world, local_rank):
         kv_pf = device_kv(w, l, pf_ctx, gen)
         tq.tq_encode(kv_pf, tq.TQ_F16, pf_ctx, H, d, w.bits_k, w.bits_v, seed, pf.pk[l], pf.pv[l],
                      pf.nk[l], pf.nv[l], pf_ctx, 0, status, stream)
+        torch.cuda.synchronize()       # the input's memory is reused on another stream
         del kv_pf
     pf_q = [torch.randn((1, pf_T, w.n_q_heads, d), generator=gen, device=device).half()
             for _ in range(pf_layers)]
@@ -476,7 +477,7 @@ def run_gpu(args, rank, world, local_rank):
               for _ in range(pf_layers)]
     pf_ctx_dev = torch.full((1,), pf_ctx, dtype=torch.int32, device=device)
 
-    pf_splits = tq.tq_prefill_splits(1, pf_T, w.n_q_heads, w.gqa)
+    pf_splits = tq.tq_prefill_splits(1, pf_T, w.n_q_heads, w.gqa, pf_ctx)
     pf_wsb = tq.tq_prefill_workspace_size(1, pf_T, w.n_q_heads, d, pf_splits)
     pf_ws = torch.empty(max(pf_wsb, 16), dtype=torch.uint8, device=device)
 
@@ -676,7 +677,7 @@ def run_gpu(args, rank, world, local_rank):
             kvb = device_kv(wb, 0, int(bctx_h[b]), gen)
             tq.tq_encode(kvb, tq.TQ_F16, int(bctx_h[b]), bH, d, wb.bits_k, wb.bits_v, seed,
                          bpk[b], bpv[b], bnk[b], bnv[b], bcap, 0, status, stream)
-        torch.cuda.synchronize()
+            torch.cuda.synchronize()   # the input's memory is reused on another stream
         bcache.append((bpk, bnk, bpv, bnv))
     skipped = torch.zeros(1, dtype=torch.int64, device=device)
     bq = [torch.randn((wb.batch, bHq, d), generator=gen, device=device).half() for _ in range(2)]
@@ -1056,7 +1057,7 @@ def profile_case(name, reps):
         q = torch.randn((1, T, w.n_q_heads, d), generator=gen, device="cuda").half()
         out = torch.empty_like(q)
         ctx_dev = torch.full((1,), ctx, dtype=torch.int32, device="cuda")
-        splits = tq.tq_prefill_splits(1, T, w.n_q_heads, w.gqa)
+        splits = tq.tq_prefill_splits(1, T, w.n_q_heads, w.gqa, ctx)
         wsb = tq.tq_prefill_workspace_size(1, T, w.n_q_heads, d, splits)
         ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device="cuda")
         for _ in range(reps):

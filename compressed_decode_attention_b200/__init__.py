@@ -78,7 +78,7 @@ def load_library(path: str) -> ctypes.CDLL:
     L.tq_prefill_workspace_size.restype = SZ
     L.tq_prefill_workspace_size.argtypes = [I, I, I, I, I]
     L.tq_prefill_splits.restype = I
-    L.tq_prefill_splits.argtypes = [I, I, I, I]
+    L.tq_prefill_splits.argtypes = [I, I, I, I, I]
     L.tq_attend_partial.restype = I
     L.tq_attend_partial.argtypes = [P, I, P, P, P, P, P, I, I, I, I, I, I, U64, I, F, I,
                                     P, SZ, P, P, P, P]
@@ -277,8 +277,8 @@ def tq_prefill_workspace_size(batch, n_tok, n_q_heads, d, n_splits) -> int:
     return lib().tq_prefill_workspace_size(batch, n_tok, n_q_heads, d, n_splits)
 
 
-def tq_prefill_splits(batch, n_tok, n_q_heads, gqa_ratio) -> int:
-    return lib().tq_prefill_splits(batch, n_tok, n_q_heads, gqa_ratio)
+def tq_prefill_splits(batch, n_tok, n_q_heads, gqa_ratio, max_ctx=0) -> int:
+    return lib().tq_prefill_splits(batch, n_tok, n_q_heads, gqa_ratio, max_ctx)
 
 
 def tq_attend_noalloc(q, q_dtype, packed_k, norms_k, packed_v, norms_v, ctx_lens,

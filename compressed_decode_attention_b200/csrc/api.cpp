@@ -292,13 +292,14 @@ int tq_prefill_attend(const void* q, int q_dtype, const uint8_t* packed_k,
                                  cap_tok, 1, nullptr, 0, dev_status, out, out_dtype, stream);
 }
 
-int tq_prefill_splits(int batch, int n_tok, int n_q_heads, int gqa_ratio) {
+int tq_prefill_splits(int batch, int n_tok, int n_q_heads, int gqa_ratio, int max_ctx) {
   if (batch < 1 || n_tok < 1 || n_q_heads < 1 || gqa_ratio < 1 || n_q_heads % gqa_ratio ||
       gqa_ratio > kMaxGroup)
     return 1;
   // CTAs of one split (one per SM: 128 query rows each); pick the split
-  // count that minimizes rounds of the SMs per unit of work, ceil(n·S/SMs)/S
+  // count that minimizes rounds of the SMs times the time of one CTA
   const long long rows_per_tile = 128 / gqa_ratio;
+  const double chunks = (double)((max_ctx > n_tok ? max_ctx : n_tok) / 64 + 1);
   const long long ctas = (long long)batch * (n_q_heads / gqa_ratio) *
                          ((n_tok + rows_per_tile - 1) / rows_per_tile);
   int dev = 0, sms = 148;
@@ -307,10 +308,9 @@ int tq_prefill_splits(int batch, int n_tok, int n_q_heads, int gqa_ratio) {
       sms <= 0)
     sms = 148;
   int best = 1;
-  double best_cost = (double)((ctas + sms - 1) / sms);
+  double best_cost = (double)((ctas + sms - 1) / sms) * (chunks + 10.0);
   for (int sp = 2; sp <= kMaxPrefillSplits; ++sp) {
-    // a small charge per split for the records and the combine
-    const double cost = (double)((ctas * sp + sms - 1) / sms) / sp + 0.02 * (sp - 1);
+    const double cost = (double)((ctas * sp + sms - 1) / sms) * (chunks / sp + 10.0);
     if (cost < best_cost - 1e-9) {
       best = sp;
       best_cost = cost;

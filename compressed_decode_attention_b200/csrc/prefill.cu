@@ -1,96 +1,102 @@
-// tq_prefill_attend: causal attention of a chunk of T new query tokens per
-// sequence over the compressed cache (the prefill of a chunk whose K/V rows
-// were appended with tq_encode), on tensor cores.
+// tq_prefill_attend on the B200 tensor cores (tcgen05, TMEM): causal
+// attention of a chunk of T new query tokens over the compressed cache.
 //
 // [TQPLUS §3] reports prefill speed with the compressed cache; the scores
 // and the weighted sum are those of decode ([ADAPTQ §How it works, item 3]:
-// rotated query, codebook lookups of the packed indices, inverse rotation of
-// the output), per query token with the causal length. With many query rows
-// per kv head this is a dense contraction, so unlike decode the cache tile
-// is dequantized once into shared memory and reused by every query row.
+// rotated query, codebook values of the packed indices, inverse rotation of
+// the output). With 128 query rows per kv head and chunk this is a dense
+// contraction, so each 64-position chunk of the cache is dequantized once
+// into shared-memory operand tiles and reused by all rows.
 //
-// Decomposition: one CTA per (sequence, kv head, tile of query rows); a row
-// is a (token, query head of the GQA group) pair, 16·8 = 128 rows per CTA.
-// Per 64-position chunk of the cache:
-//   stage    bulk copies of the packed K/V rows and norms (two slots,
-//            mbarrier, bounded wait)
-//   dequant  all threads: K codebook values as fp16 high/low tiles and V as
-//            an fp16 tile, [position][coordinate], 272-byte rows (ldmatrix
-//            without bank conflicts)
-//   scores   per warp (16 rows): mma.m16n8k16, A = rotated query high/low
-//            (registers), B = K tiles (ldmatrix); Q_hi·K_hi + Q_lo·K_hi +
-//            Q_hi·K_lo keep ~22 significant bits as in decode
-//   softmax  online, fp32, log2 domain, causal mask
-//   PV       A = softmax weight x V norm (fp16, from the score registers),
-//            B = V tile (ldmatrix.trans)
-// Output per row: D⊙(H·(acc/l))/d with in-register and shuffle stages.
+// One CTA per (context split, sequence, kv head, tile of 128 query rows); a
+// row is a (token, query head of the GQA group) pair. Warp roles:
+//   warps 0-3  one thread per row: rotate its query (thread-local FWHT) into
+//              fp16 high/low parts in tensor memory; per chunk read the row
+//              of scores, scale, causal mask, online softmax in the log2
+//              domain, rescale the output row when the maximum grows, and
+//              write the row of P' = weight x V norm (fp16) to tensor memory;
+//              at the end read the output row, normalize, inverse-rotate and
+//              store it (or the split's record)
+//   warps 4-7  dequantize a chunk: K codebook values as fp16 high and low
+//              tiles [64 positions x 128 coordinates] and the norms, then V
+//              [64 positions x 128 coordinates]
+//   warp 8     bulk copies of the packed rows and norms (four slots)
+//   warp 9     tensor memory (512 columns: two score buffers of 64, the
+//              128-column output, the query's high and low parts, two P'
+//              buffers); one thread issues per chunk
+//                S = Q_hi·K_hi + Q_lo·K_hi + Q_hi·K_lo  (M 128, N 64, K 128)
+//                O += P'·V                              (M 128, N 128, K 64)
+//              kind::f16 MMAs with fp32 accumulators, the A operands (Q, P')
+//              in tensor memory, scores one chunk ahead of P'·V
+// K tiles are K-major and V tiles MN-major (position rows of coordinates),
+// both in the 128-byte swizzle layout (tc_common.cuh). A K buffer is free
+// once its scores are done and a V buffer once its P'·V is, so the
+// dequantization of chunk c + 2 overlaps the products of chunk c + 1.
+// The high/low split keeps ~22 significant bits of the scores as in decode;
+// P' and V are fp16 as in decode. Every wait is bounded; a role that gives
+// up sets TQ_DEV_WAIT_TIMEOUT and stops, and the tensor memory is freed
+// after a CTA barrier on every path.
 #include <atomic>
+
 #include "attend_kernel.cuh"
+#include "tc_common.cuh"
 
 namespace tq {
 namespace {
 
-constexpr int kPfWarps = 8;
-constexpr int kPfThreads = 32 * kPfWarps;
-constexpr int kPfRows = 16 * kPfWarps;          // query rows per CTA
-constexpr int kPfChunk = 64;                    // cache positions per chunk
-constexpr int kTS = 136;                        // tile row stride in halves (272 B)
+constexpr int kTRows = 128;                       // query rows per tile (MMA M)
+constexpr int kTChunk = 64;                       // cache positions per chunk
+constexpr int kTD = 128;                          // head dimension
+constexpr int kTWarps = 10;
+constexpr int kTThreads = 32 * kTWarps;
+constexpr int kTStages = 4;                       // staging slots of packed rows
+constexpr int kTNormSlots = 8;                    // ring of per-chunk norms
+constexpr long long kTWait = 2000000000LL;         // cycles (~1 s)
+// tensor-memory columns
+constexpr uint32_t kColS = 0;                     // 2 x 64: scores
+constexpr uint32_t kColO = 128;                   // 128: output accumulator
+constexpr uint32_t kColQH = 256, kColQL = 320;    // 64 each: query parts (fp16 pairs)
+constexpr uint32_t kColP = 384;                   // 2 x 32: P' (fp16 pairs)
+constexpr uint32_t kTTmemCols = 512;
 
 template <int BK, int BV>
-struct PfGeo {
-  static constexpr int RK = 16 * BK, RV = 16 * BV;          // d = 128
-  static constexpr int KROWS = RK % 16 == 0 ? 1 : 16 / (RK % 16);
-  static constexpr int VROWS = RV % 16 == 0 ? 1 : 16 / (RV % 16);
-  static constexpr int QH = 0;                               // [128 rows][kTS] fp16
-  static constexpr int QL = QH + kPfRows * kTS * 2;
-  // two buffers of dequantized chunk tiles: K high, K low, V ([64 positions]
-  // [kTS] fp16 each) and the K / V norms as floats
-  static constexpr int KH = QL + kPfRows * kTS * 2;          // [64 positions][kTS]
-  static constexpr int KL = KH + kPfChunk * kTS * 2;
-  static constexpr int VT = KL + kPfChunk * kTS * 2;
-  static constexpr int NKF = VT + kPfChunk * kTS * 2;        // float [64]
-  static constexpr int NVF = NKF + kPfChunk * 4;             // float [64]
-  static constexpr int TBUF = NVF + kPfChunk * 4 - KH;       // bytes per buffer
-  static constexpr int STG = KH + 2 * TBUF;                  // two staging slots
-  static constexpr int SLOT = kPfChunk * (RK + RV) + 2 * kPfChunk * 2;
-  static constexpr int LUTK = STG + 2 * SLOT;                // uint2 per pair code
-  static constexpr int LUTV = LUTK + (1 << (2 * BK)) * 8;    // uint32 per pair code
-  static constexpr int SINV = LUTV + (1 << (2 * BV)) * 4;    // float per row
-  static constexpr int MBAR = SINV + kPfRows * 4;
-  static constexpr int SMEM = MBAR + 16;
-  static_assert(SLOT % 16 == 0 && STG % 16 == 0 && TBUF % 16 == 0 && MBAR % 8 == 0,
-                "alignment");
+struct TcGeo {
+  static constexpr int RK = 16 * BK, RV = 16 * BV;            // packed row bytes (d = 128)
+  static constexpr int TILE = kTChunk * kTD * 2;              // 16 KB: [64 x 128] fp16
+  static constexpr int KH = 0;                                // 2 K high tiles
+  static constexpr int KL = KH + 2 * TILE;                    // 2 K low tiles
+  static constexpr int VV = KL + 2 * TILE;                    // 2 V tiles
+  static constexpr int SLOT = kTChunk * (RK + RV) + 2 * kTChunk * 2;
+  static constexpr int STG = VV + 2 * TILE;                   // staging slots
+  static constexpr int NKF = STG + kTStages * SLOT;           // norm ring: 64 floats a slot
+  static constexpr int NVF = NKF + kTNormSlots * kTChunk * 4;
+  // codebook tables, one copy per lane group where random lookups of a
+  // warp would collide in shared-memory banks: K (uint2 per pair code) 16
+  // copies unless 2-bit, V (uint32 per pair code) 32 copies unless 2-bit
+  static constexpr int KREP = BK == 2 ? 1 : 16, VREP = BV == 2 ? 1 : 32;
+  static constexpr int KSH = BK == 2 ? 3 : 7, VSH = BV == 2 ? 2 : 7;  // log2 bytes per code
+  static constexpr int LUTK = NVF + kTNormSlots * kTChunk * 4;
+  static constexpr int LUTV = LUTK + (1 << (2 * BK)) * 8 * KREP;
+  static constexpr int BARS = LUTV + (1 << (2 * BV)) * 4 * VREP;  // 24 barriers
+  static constexpr int MISC = BARS + 24 * 8;                  // TMEM address, abort flag
+  static constexpr int SMEM = 1024 + MISC + 16;
+  static_assert(SLOT % 16 == 0 && STG % 1024 == 0 && NKF % 16 == 0 && BARS % 8 == 0, "align");
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                        uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                          uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
-
 template <int BK, int BV>
-__global__ void __launch_bounds__(kPfThreads, 1)
-prefill_kernel(const __grid_constant__ PrefillArgs a,
-               const __grid_constant__ Codebook cbk,
-               const __grid_constant__ Codebook cbv,
-               const __grid_constant__ SignMask sm) {
-  using G = PfGeo<BK, BV>;
-  constexpr int D = 128;
-  extern __shared__ __align__(128) uint8_t smem[];
-  const uint32_t sbase = smem_addr(smem);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int gq = lane >> 2, tq = lane & 3;
+__global__ void __launch_bounds__(kTThreads, 1)
+prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ Codebook cbk,
+                  const __grid_constant__ Codebook cbv, const __grid_constant__ SignMask sm) {
+  using G = TcGeo<BK, BV>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = tc::saddr(smem_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sb - raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int GQ = a.gqa, H = a.n_kv_heads, T = a.n_tok;
-  const int TQ = kPfRows / GQ;                     // query tokens per tile
+  const int TQ = kTRows / GQ;                      // query tokens per tile
   const int tiles = (T + TQ - 1) / TQ;
-  // split s of n_splits takes the s-th share of the tile's chunks and leaves
-  // log-sum-exp records for the combine kernel instead of the output
   const int S = a.n_splits > 1 ? a.n_splits : 1;
   const int split = blockIdx.x % S;
   const int unit = blockIdx.x / S;
@@ -99,12 +105,34 @@ prefill_kernel(const __grid_constant__ PrefillArgs a,
   const int b = unit / (tiles * H);
   const int i0 = tile * TQ, nq = min(TQ, T - i0);
   const int R = nq * GQ;                           // valid rows
-  float* sinv = reinterpret_cast<float*>(smem + G::SINV);
-  const uint32_t bar0 = sbase + G::MBAR;
+  // barriers (chunk c uses slot c & 3 of the four-deep rings and c & 1 of
+  // the two-deep ones): staging full/free and K ready (x4); V ready, scores
+  // full/free, P' ready, P'·V done (x2); query ready
+  const uint32_t bars = sb + G::BARS;
+  auto stage_full = [&](int c) { return bars + 8 * (0 + (c & 3)); };
+  auto stage_free = [&](int c) { return bars + 8 * (4 + (c & 3)); };
+  auto k_ready = [&](int c) { return bars + 8 * (8 + (c & 3)); };
+  auto v_ready = [&](int c) { return bars + 8 * (12 + (c & 1)); };
+  auto s_full = [&](int c) { return bars + 8 * (14 + (c & 1)); };
+  auto s_free = [&](int c) { return bars + 8 * (16 + (c & 1)); };
+  auto p_ready = [&](int c) { return bars + 8 * (18 + (c & 1)); };
+  auto pv_done = [&](int c) { return bars + 8 * (20 + (c & 1)); };
+  const uint32_t q_ready = bars + 8 * 22;
+  // phase parity of chunk c's use of a four- or two-deep ring slot
+  auto par4 = [](int c) { return (uint32_t)((c >> 2) & 1); };
+  auto par2 = [](int c) { return (uint32_t)((c >> 1) & 1); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + G::MISC);
+  int* abort_flag = reinterpret_cast<int*>(smem + G::MISC + 4);
+  auto wait = [&](uint32_t bar, uint32_t parity) {
+    if (*reinterpret_cast<volatile int*>(abort_flag)) return false;
+    if (tc::bar_wait(bar, parity, kTWait)) return true;
+    atomicExch(abort_flag, 1);
+    return false;
+  };
 
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-  // ---- codebook tables from the launch parameters
-  for (int code = tid; code < (1 << (2 * BK)); code += kPfThreads) {
+  // ---- codebook tables (launch parameters): K high/low pairs, V pairs
+  for (int code = tid; code < (1 << (2 * BK)); code += kTThreads) {
     uint32_t hl[2];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
@@ -112,423 +140,507 @@ prefill_kernel(const __grid_constant__ PrefillArgs a,
       const __half h = __float2half_rn(c), l = __float2half_rn(c - __half2float(h));
       hl[e] = (uint32_t)__half_as_ushort(h) | ((uint32_t)__half_as_ushort(l) << 16);
     }
-    *reinterpret_cast<uint2*>(smem + G::LUTK + 8 * code) =
-        make_uint2((hl[0] & 0xFFFFu) | (hl[1] << 16), (hl[0] >> 16) | (hl[1] & 0xFFFF0000u));
+    const uint2 e = make_uint2((hl[0] & 0xFFFFu) | (hl[1] << 16), (hl[0] >> 16) | (hl[1] & 0xFFFF0000u));
+#pragma unroll 1
+    for (int rep = 0; rep < G::KREP; ++rep)
+      *reinterpret_cast<uint2*>(smem + G::LUTK + (code << G::KSH) + 8 * rep) = e;
   }
-  for (int code = tid; code < (1 << (2 * BV)); code += kPfThreads) {
+  for (int code = tid; code < (1 << (2 * BV)); code += kTThreads) {
     const uint32_t v0 = __half_as_ushort(__float2half_rn(cbv.centroid[code & ((1 << BV) - 1)]));
     const uint32_t v1 = __half_as_ushort(__float2half_rn(cbv.centroid[code >> BV]));
-    *reinterpret_cast<uint32_t*>(smem + G::LUTV + 4 * code) = v0 | (v1 << 16);
+#pragma unroll 1
+    for (int rep = 0; rep < G::VREP; ++rep)
+      *reinterpret_cast<uint32_t*>(smem + G::LUTV + (code << G::VSH) + 4 * rep) = v0 | (v1 << 16);
   }
   if (tid == 0) {
-    mbar_init(bar0);
-    mbar_init(bar0 + 8);
+    for (int i = 0; i < 4; ++i) {
+      tc::bar_init(stage_full(i), 1);
+      tc::bar_init(stage_free(i), 4);
+      tc::bar_init(k_ready(i), 4);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::bar_init(v_ready(i), 4);
+      tc::bar_init(s_full(i), 1);
+      tc::bar_init(s_free(i), 4);
+      tc::bar_init(p_ready(i), 4);
+      tc::bar_init(pv_done(i), 1);
+    }
+    tc::bar_init(q_ready, 4);
+    *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
-  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  if (warp == 9) tc::tmem_alloc(tc::saddr(tmem_slot), kTTmemCols);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
 
-  const int raw = a.ctx_lens[b];
-  const int L = min(max(raw, 0), a.cap_tok);
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  const int raw_len = a.ctx_lens[b];
+  const int L = min(max(raw_len, 0), a.cap_tok);
   const int start = L - T;                         // absolute position of token 0
   if (tile == 0 && g == 0 && split == 0 && tid == 0 && a.dev_status) {
-    if (raw > a.cap_tok) atomicOr(a.dev_status, TQ_DEV_CTX_CLAMPED);
+    if (raw_len > a.cap_tok) atomicOr(a.dev_status, TQ_DEV_CTX_CLAMPED);
     if (L < T) atomicOr(a.dev_status, TQ_DEV_CTX_EMPTY);
   }
   const int p_last = start + i0 + nq - 1;          // last query position of the tile
-  const int nch_tile = p_last >= 0 ? p_last / kPfChunk + 1 : 0;
-  // this CTA's chunks: absolute chunks cbase .. cbase + nchunks - 1 (local
-  // index c = 0 .. nchunks - 1 for staging slots and barrier phases)
+  const int nch_tile = p_last >= 0 ? p_last / kTChunk + 1 : 0;
   const int cbase = (int)((long long)split * nch_tile / S);
   const int nchunks = (int)((long long)(split + 1) * nch_tile / S) - cbase;
-
   const size_t seq_row = ((size_t)b * H + g) * a.cap_tok;
-  auto issue = [&](int c) {                        // thread 0
-    const int t0 = (cbase + c) * kPfChunk;
-    const int rows = min(kPfChunk, L - t0);
-    const int krows = min(kPfChunk, (rows + G::KROWS - 1) / G::KROWS * G::KROWS);
-    const int vrows = min(kPfChunk, (rows + G::VROWS - 1) / G::VROWS * G::VROWS);
-    const int nrows = min(kPfChunk, (rows + 7) & ~7);
-    const uint32_t dst = sbase + G::STG + (c & 1) * G::SLOT, bar = bar0 + 8 * (c & 1);
-    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-    mbar_expect(bar, krows * G::RK + vrows * G::RV + 4 * nrows);
-    bulk_g2s(dst, a.packed_k + (seq_row + t0) * G::RK, krows * G::RK, bar);
-    bulk_g2s(dst + kPfChunk * G::RK, a.packed_v + (seq_row + t0) * G::RV, vrows * G::RV, bar);
-    bulk_g2s(dst + kPfChunk * (G::RK + G::RV), a.norms_k + seq_row + t0, 2 * nrows, bar);
-    bulk_g2s(dst + kPfChunk * (G::RK + G::RV) + 2 * kPfChunk, a.norms_v + seq_row + t0,
-             2 * nrows, bar);
-  };
-  if (tid == 0 && nchunks > 0) issue(0);
-  if (tid == 0 && nchunks > 1) issue(1);
 
-  // ---- rotated queries: warp w rotates its rows 16w .. 16w + 15 one by one
-  // (row r = token r / GQ of the tile, head r % GQ of the group)
-  for (int rr = 0; rr < 16; ++rr) {
-    const int r = 16 * warp + rr;
-    __half* qh = reinterpret_cast<__half*>(smem + G::QH) + r * kTS + 4 * lane;
-    __half* ql = reinterpret_cast<__half*>(smem + G::QL) + r * kTS + 4 * lane;
-    if (r >= R) {
-      *reinterpret_cast<uint2*>(qh) = make_uint2(0u, 0u);
-      *reinterpret_cast<uint2*>(ql) = make_uint2(0u, 0u);
-      if (lane == 0) sinv[r] = 0.f;
-      continue;
+  if (warp == 8) {
+    // ---- producer: chunk c into staging slot c & 3
+    if (lane == 0) {
+      int c = 0;
+      for (; c < nchunks; ++c) {
+        if (!wait(stage_free(c), par4(c) ^ 1)) break;
+        const int t0 = (cbase + c) * kTChunk;
+        const int rows = min(kTChunk, L - t0);
+        const int nrows = min(kTChunk, (rows + 7) & ~7);
+        const uint32_t dst = sb + G::STG + (c & 3) * G::SLOT;
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+        tc::bar_expect(stage_full(c), rows * (G::RK + G::RV) + 4 * nrows);
+        tc::bulk_g2s(dst, a.packed_k + (seq_row + t0) * G::RK, rows * G::RK, stage_full(c));
+        tc::bulk_g2s(dst + kTChunk * G::RK, a.packed_v + (seq_row + t0) * G::RV, rows * G::RV,
+                     stage_full(c));
+        tc::bulk_g2s(dst + kTChunk * (G::RK + G::RV), a.norms_k + seq_row + t0, 2 * nrows,
+                     stage_full(c));
+        tc::bulk_g2s(dst + kTChunk * (G::RK + G::RV) + 2 * kTChunk, a.norms_v + seq_row + t0,
+                     2 * nrows, stage_full(c));
+      }
+      // copies still in flight complete before the CTA can end
+      for (int k = c > kTStages ? c - kTStages : 0; k < c; ++k)
+        tc::bar_wait(stage_full(k), par4(k), kTWait);
     }
+  } else if (warp >= 4) {
+    if (warp == 9) {
+      // ---- MMA issue (one thread)
+      if (lane == 0) {
+        constexpr uint32_t idS = tc::umma_idesc(0u, kTRows, kTChunk);
+        constexpr uint32_t idO = tc::umma_idesc(0u, kTRows, kTD) | (1u << 16);  // B MN-major
+        bool ok = nchunks == 0 || wait(q_ready, 0);
+        uint32_t last_bar = 0, last_par = 0;      // the latest commit's barrier and phase
+        // descriptors of buffer 0, k-step 0 (a start address moves the low
+        // field by bytes / 16)
+        const uint64_t kdesc = tc::umma_desc(sb + G::KH);
+        const uint64_t vdesc = tc::umma_desc_mn(sb + G::VV, 64 * 128, 1024);
+        auto scores = [&](int c) {
+          if (!wait(k_ready(c), par4(c)) || !wait(s_free(c), par2(c) ^ 1)) return false;
+          tc::fence_after_sync();
+          const uint32_t d = tmem + kColS + kTChunk * (c & 1);
+          const uint64_t kb = kdesc + (uint32_t)(((c & 1) * G::TILE) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < kTD / 16; ++kk) {
+            const uint32_t koff = (kk >> 2) * (kTChunk * 128) + (kk & 3) * 32;
+            const uint64_t kh = kb + (koff >> 4);
+            const uint64_t kl = kb + ((koff + (G::KL - G::KH)) >> 4);
+            tc::mma_f16_ts(d, tmem + kColQH + 8 * kk, kh, idS, kk > 0);
+            tc::mma_f16_ts(d, tmem + kColQL + 8 * kk, kh, idS, true);
+            tc::mma_f16_ts(d, tmem + kColQH + 8 * kk, kl, idS, true);
+          }
+          tc::mma_commit(s_full(c));
+          last_bar = s_full(c);
+          last_par = par2(c);
+          return true;
+        };
+        auto pv = [&](int c) {
+          if (!wait(v_ready(c), par2(c)) || !wait(p_ready(c), par2(c))) return false;
+          tc::fence_after_sync();
+          const uint64_t vb = vdesc + (uint32_t)(((c & 1) * G::TILE) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < kTChunk / 16; ++kk)
+            tc::mma_f16_ts(tmem + kColO, tmem + kColP + 32 * (c & 1) + 8 * kk,
+                           vb + (uint32_t)(kk * 2048 >> 4), idO, c > 0 || kk > 0);
+          tc::mma_commit(pv_done(c));
+          last_bar = pv_done(c);
+          last_par = par2(c);
+          return true;
+        };
+        if (ok && nchunks > 0) ok = scores(0);
+        for (int c = 0; ok && c < nchunks; ++c) {
+          if (c + 1 < nchunks && !scores(c + 1)) break;
+          if (!pv(c)) break;
+        }
+        // the last committed products (and all before them) complete before
+        // the tensor memory is freed
+        if (last_bar) tc::bar_wait(last_bar, last_par, kTWait);
+      }
+    } else {
+      // ---- dequantization (warps 4-7, thread u): position u & 63,
+      // coordinates 64·(u >> 6) .. + 63 (eight consecutive positions per
+      // quarter warp: the 16-byte tile stores fall in distinct banks)
+      const int u = tid - 128;
+      const int pos = u & 63, half = u >> 6;
+      const uint32_t krep = G::KREP > 1 ? 8 * (lane & 15) : 0;   // this lane's table copies
+      const uint32_t vrep = G::VREP > 1 ? 4 * lane : 0;
+      for (int c = 0; c < nchunks; ++c) {
+        const int i = c & 1;
+        // K buffer i: free once the scores of chunk c - 2 are done
+        bool ok = wait(stage_full(c), par4(c)) && wait(s_full(c), par2(c) ^ 1);
+        if (!__all_sync(0xFFFFFFFFu, ok)) break;
+        const uint8_t* st = smem + G::STG + (c & 3) * G::SLOT;
+        {
+          uint32_t kw[(8 * BK + 3) / 4 + 1];
+          load_chunk<8 * BK>(st, pos * G::RK + 8 * BK * half, kw);
+          uint8_t* khp = smem + G::KH + i * G::TILE;
+          uint8_t* klp = smem + G::KL + i * G::TILE;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {              // 16-byte chunks: 4 pairs
+            uint32_t h4[4], l4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint2 v =
+                  lds<uint2>(smem, G::LUTK + (pair_code_shifted<BK, G::KSH>(kw, 4 * j + e) | krep));
+              h4[e] = v.x;
+              l4[e] = v.y;
+            }
+            const uint32_t off = tc::sw128_offset(kTChunk, pos, 64 * half + 8 * j);
+            *reinterpret_cast<uint4*>(khp + off) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+            *reinterpret_cast<uint4*>(klp + off) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+          }
+        }
+        if (u < kTChunk) {
+          // norms as floats; 0 past the sequence end (the copied norm runs
+          // stop at a multiple of 8 positions: the rest of the slot is stale)
+          const bool live = (cbase + c) * kTChunk + u < L;
+          const uint16_t* ns = reinterpret_cast<const uint16_t*>(st + kTChunk * (G::RK + G::RV));
+          const int slot = (c & (kTNormSlots - 1)) * kTChunk + u;
+          reinterpret_cast<float*>(smem + G::NKF)[slot] =
+              live ? __half2float(__ushort_as_half(ns[u])) : 0.f;
+          reinterpret_cast<float*>(smem + G::NVF)[slot] =
+              live ? __half2float(__ushort_as_half(ns[kTChunk + u])) : 0.f;
+        }
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+        __syncwarp();
+        if (lane == 0) tc::bar_arrive(k_ready(c));
+        // V buffer i: free once the P'·V of chunk c - 2 is done
+        ok = wait(pv_done(c), par2(c) ^ 1);
+        if (!__all_sync(0xFFFFFFFFu, ok)) break;
+        {
+          uint32_t vw[(8 * BV + 3) / 4 + 1];
+          load_chunk<8 * BV>(st, kTChunk * G::RK + pos * G::RV + 8 * BV * half, vw);
+          uint8_t* vp = smem + G::VV + i * G::TILE;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            uint32_t p4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              p4[e] = lds<uint32_t>(smem, G::LUTV + (pair_code_shifted<BV, G::VSH>(vw, 4 * j + e) | vrep));
+            *reinterpret_cast<uint4*>(vp + tc::sw128_offset(kTChunk, pos, 64 * half + 8 * j)) =
+                make_uint4(p4[0], p4[1], p4[2], p4[3]);
+          }
+        }
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          tc::bar_arrive(v_ready(c));
+          tc::bar_arrive(stage_free(c));
+        }
+      }
+    }
+  } else {
+    // ---- warps 0-3: thread r = row r of the tile (TMEM lane r)
+    const int r = tid;
+    const bool live_row = r < R;
     const int t = r / GQ, h = r - t * GQ;
-    const size_t qo = (((size_t)b * T + i0 + t) * a.n_q_heads + (size_t)g * GQ + h) * D + 4 * lane;
-    float x[4];
-    if (a.q_dtype == TQ_F32) {
-      const float4 v = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.q) + qo);
-      x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
-    } else {
-      const uint2 v = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(a.q) + qo);
-      const bool bf = a.q_dtype == TQ_BF16;
-      const float2 f0 = unpack16x2(v.x, bf), f1 = unpack16x2(v.y, bf);
-      x[0] = f0.x; x[1] = f0.y; x[2] = f1.x; x[3] = f1.y;
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int c = 4 * lane + k;
-      x[k] = apply_sign(x[k], sm.w[c >> 5], c & 31);
-    }
-    fwht_warp<4>(x, lane);
-    float amax = 0.f;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      x[k] *= kLog2e / (128.0f * 11.3137084989847603904f);
-      amax = fmaxf(amax, fabsf(x[k]));
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-    const int e = amax > 0.f ? ilogbf(amax) : 0;
-    const float qs = ldexpf(1.f, min(14 - e, 120));
-    uint32_t hw[2], lw[2];
-#pragma unroll
-    for (int k = 0; k < 4; k += 2) {
-      const float v0 = x[k] * qs, v1 = x[k + 1] * qs;
-      const __half h0 = __float2half_rn(v0), h1 = __float2half_rn(v1);
-      hw[k / 2] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
-      lw[k / 2] = pack_half2(v0 - __half2float(h0), v1 - __half2float(h1));
-    }
-    *reinterpret_cast<uint2*>(qh) = make_uint2(hw[0], hw[1]);
-    *reinterpret_cast<uint2*>(ql) = make_uint2(lw[0], lw[1]);
-    if (lane == 0) sinv[r] = 1.f / (qs * kKScale);
-  }
-  __syncthreads();
-
-  // A fragments of the warp's 16 rows (k-step ks: coordinates 16ks..16ks+15)
-  uint32_t qa[8][4], qb[8][4];
-  {
-    const int row = 16 * warp + (lane & 7) + 8 * ((lane >> 3) & 1);
-    const int col = 8 * (lane >> 4);
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      ldsm_x4(sbase + G::QH + 2 * (row * kTS + 16 * ks + col), qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
-      ldsm_x4(sbase + G::QL + 2 * (row * kTS + 16 * ks + col), qb[ks][0], qb[ks][1], qb[ks][2], qb[ks][3]);
-    }
-  }
-  const int r0 = 16 * warp + gq, r1 = r0 + 8;      // this lane's rows
-  const float si0 = sinv[r0], si1 = sinv[r1];
-  const int p0 = r0 < R ? start + i0 + r0 / GQ : -1;   // causal limits (-1: no positions)
-  const int p1 = r1 < R ? start + i0 + r1 / GQ : -1;
-
-  float o[16][4];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  bool stalled = false;
-
-  // Chunk c: its packed rows arrive in staging slot c & 1 (issued two
-  // chunks ahead), are dequantized into tile buffer c & 1, and are consumed
-  // by the MMAs of the next round. A warp that finishes the MMAs of chunk c
-  // goes on to dequantize chunk c + 1 into the other buffer while the rest
-  // still multiply; one barrier per chunk separates the rounds.
-  auto dequant = [&](int c) {
-    const uint8_t* st = smem + G::STG + (c & 1) * G::SLOT;
-    uint8_t* tb = smem + (c & 1) * G::TBUF;        // buffer c & 1 (add G::KH etc.)
-    const int pos = tid >> 2, qd = tid & 3;
-    uint32_t kw[(4 * BK + 3) / 4 + 1], vw[(4 * BV + 3) / 4 + 1];
-    load_chunk<4 * BK>(st, pos * G::RK + 4 * BK * qd, kw);
-    load_chunk<4 * BV>(st, kPfChunk * G::RK + pos * G::RV + 4 * BV * qd, vw);
-    uint32_t hi[16], lo[16], vv[16];
-#pragma unroll
-    for (int p = 0; p < 16; ++p) {
-      const uint2 e = lds<uint2>(smem, G::LUTK + pair_code_shifted<BK, 3>(kw, p));
-      hi[p] = e.x;
-      lo[p] = e.y;
-      vv[p] = lds<uint32_t>(smem, G::LUTV + pair_code_shifted<BV, 2>(vw, p));
-    }
-    const int off = 2 * (pos * kTS + 32 * qd);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      *reinterpret_cast<uint4*>(tb + G::KH + off + 16 * k) =
-          make_uint4(hi[4 * k], hi[4 * k + 1], hi[4 * k + 2], hi[4 * k + 3]);
-      *reinterpret_cast<uint4*>(tb + G::KL + off + 16 * k) =
-          make_uint4(lo[4 * k], lo[4 * k + 1], lo[4 * k + 2], lo[4 * k + 3]);
-      *reinterpret_cast<uint4*>(tb + G::VT + off + 16 * k) =
-          make_uint4(vv[4 * k], vv[4 * k + 1], vv[4 * k + 2], vv[4 * k + 3]);
-    }
-    if (qd == 0) {
-      // norms as floats; 0 past the sequence end (the copied norm runs stop
-      // at a multiple of 8 positions: the rest of the slot is stale)
-      const bool live = (cbase + c) * kPfChunk + pos < L;
-      const uint16_t* nsrc = reinterpret_cast<const uint16_t*>(st + kPfChunk * (G::RK + G::RV));
-      reinterpret_cast<float*>(tb + G::NKF)[pos] =
-          live ? __half2float(__ushort_as_half(nsrc[pos])) : 0.f;
-      reinterpret_cast<float*>(tb + G::NVF)[pos] =
-          live ? __half2float(__ushort_as_half(nsrc[kPfChunk + pos])) : 0.f;
-    }
-  };
-  // the first chunk: its data, its tiles, then slot 0 is free for chunk 2
-  int issued = nchunks > 0 ? (nchunks > 1 ? 2 : 1) : 0;   // chunks 0, 1 in flight
-  if (nchunks > 0) {
-    const bool ok = mbar_wait(bar0, 0u);
-    if (ok) dequant(0);
-    if (!__syncthreads_and(ok)) {                  // the first copy never completed
-      stalled = true;
-      if (tid == 0) {
-        if (a.dev_status) atomicOr(a.dev_status, TQ_DEV_WAIT_TIMEOUT);
-        for (int k = 0; k < issued; ++k) mbar_wait(bar0 + 8 * (k & 1), (uint32_t)(k >> 1) & 1u);
-      }
-    } else {
-      if (tid == 0 && nchunks > 2) issue(2);
-      issued = min(nchunks, 3);
-    }
-  }
-  for (int c = 0; c < nchunks && !stalled; ++c) {
-    const uint8_t* tb = smem + (c & 1) * G::TBUF;
-    const uint32_t tbs = sbase + (c & 1) * G::TBUF;
-    // ---- scores of the warp's 16 rows x 64 positions
-    const int t0 = (cbase + c) * kPfChunk;
-    const float* nkf = reinterpret_cast<const float*>(tb + G::NKF);
-    const float* nvf = reinterpret_cast<const float*>(tb + G::NVF);
-    float s[8][4];
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+    const uint32_t trow = (uint32_t)(32 * warp) << 16;
+    float si;
     {
-      // ldmatrix x4: two n-tiles (positions 16 n2 .. + 15) x (coords lo / hi 8)
-      const int prow = (lane & 7) + 8 * (lane >> 4), pcol = 8 * ((lane >> 3) & 1);
+      // rotated query: q~ = H·(D⊙q)·log2(e)/d^{3/2}, scaled by a power of two
+      // qs that puts its largest value near 2^14, as fp16 high and low parts
+      float x[kTD];
+      if (live_row) {
+        const size_t qo = (((size_t)b * T + i0 + t) * a.n_q_heads + (size_t)g * GQ + h) * kTD;
+        if (a.q_dtype == TQ_F32) {
+          const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.q) + qo);
 #pragma unroll
-      for (int n2 = 0; n2 < 4; ++n2) {
+          for (int k = 0; k < kTD / 4; ++k) {
+            const float4 v = src[k];
+            x[4 * k] = v.x; x[4 * k + 1] = v.y; x[4 * k + 2] = v.z; x[4 * k + 3] = v.w;
+          }
+        } else {
+          const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.q) + qo);
+          const bool bf = a.q_dtype == TQ_BF16;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          uint32_t bh0, bh1, bh2, bh3, bl0, bl1, bl2, bl3;
-          const uint32_t o2 = 2 * ((16 * n2 + prow) * kTS + 16 * ks + pcol);
-          ldsm_x4(tbs + G::KH + o2, bh0, bh1, bh2, bh3);
-          ldsm_x4(tbs + G::KL + o2, bl0, bl1, bl2, bl3);
-          mma16816(s[2 * n2], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], bh0, bh1);
-          mma16816(s[2 * n2], qb[ks][0], qb[ks][1], qb[ks][2], qb[ks][3], bh0, bh1);
-          mma16816(s[2 * n2], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], bl0, bl1);
-          mma16816(s[2 * n2 + 1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], bh2, bh3);
-          mma16816(s[2 * n2 + 1], qb[ks][0], qb[ks][1], qb[ks][2], qb[ks][3], bh2, bh3);
-          mma16816(s[2 * n2 + 1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], bl2, bl3);
+          for (int k = 0; k < kTD / 8; ++k) {
+            const uint4 v = src[k];
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = unpack16x2(w4[e], bf);
+              x[8 * k + 2 * e] = f.x;
+              x[8 * k + 2 * e + 1] = f.y;
+            }
+          }
         }
+#pragma unroll
+        for (int k = 0; k < kTD; ++k) x[k] = apply_sign(x[k], sm.w[k >> 5], k & 31);
+#pragma unroll
+        for (int s = 1; s < kTD; s <<= 1)
+#pragma unroll
+          for (int k = 0; k < kTD; ++k)
+            if (!(k & s)) {
+              const float p = x[k], q = x[k + s];
+              x[k] = p + q;
+              x[k + s] = p - q;
+            }
+      } else {
+#pragma unroll
+        for (int k = 0; k < kTD; ++k) x[k] = 0.f;
       }
-    }
-    // ---- scale, causal mask, online softmax (rows r0: s[.][0..1], r1: [2..3])
-    float mx0 = -INFINITY, mx1 = -INFINITY;
+      float amax = 0.f;
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int pl = 8 * nt + 2 * tq + e, pos = t0 + pl;
-        const float nk = nkf[pl];
-        float v0 = s[nt][e] * (si0 * nk), v1 = s[nt][2 + e] * (si1 * nk);
-        if (pos > p0) v0 = -INFINITY;
-        if (pos > p1) v1 = -INFINITY;
-        s[nt][e] = v0;
-        s[nt][2 + e] = v1;
-        mx0 = fmaxf(mx0, v0);
-        mx1 = fmaxf(mx1, v1);
+      for (int k = 0; k < kTD; ++k) {
+        x[k] *= kLog2e / (128.0f * 11.3137084989847603904f);
+        amax = fmaxf(amax, fabsf(x[k]));
       }
+      const int e = amax > 0.f ? ilogbf(amax) : 0;
+      const float qs = ldexpf(1.f, min(14 - e, 120));
+      // 16 columns (32 coordinates) of each part per store
 #pragma unroll
-    for (int o2 = 1; o2 <= 2; o2 <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xFFFFFFFFu, mx0, o2));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xFFFFFFFFu, mx1, o2));
-    }
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    const float al0 = mn0 == -INFINITY ? 1.f : fast_exp2(m0 - mn0);
-    const float al1 = mn1 == -INFINITY ? 1.f : fast_exp2(m1 - mn1);
-    m0 = mn0;
-    m1 = mn1;
-    l0 *= al0;
-    l1 *= al1;
+      for (int blk = 0; blk < kTD / 32; ++blk) {
+        uint32_t hw[16], lw[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      o[j][0] *= al0;
-      o[j][1] *= al0;
-      o[j][2] *= al1;
-      o[j][3] *= al1;
-    }
-    uint32_t pa[4][4];                              // P' A fragments per 16 positions
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      float w[4];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int pl = 8 * nt + 2 * tq + e;
-        const float nv = nvf[pl];
-        const float w0 = s[nt][e] == -INFINITY ? 0.f : fast_exp2(s[nt][e] - mn0);
-        const float w1 = s[nt][2 + e] == -INFINITY ? 0.f : fast_exp2(s[nt][2 + e] - mn1);
-        l0 += w0;
-        l1 += w1;
-        w[e] = w0 * nv;
-        w[2 + e] = w1 * nv;
-      }
-      const int kk = nt >> 1, hf = nt & 1;
-      pa[kk][2 * hf] = pack_half2(w[0], w[1]);          // row gq
-      pa[kk][2 * hf + 1] = pack_half2(w[2], w[3]);      // row gq + 8
-    }
-    // ---- O += P'·V (k = positions 16kk.., n = coordinates 8j..)
-    {
-      const int vrow = (lane & 7) + 8 * ((lane >> 3) & 1), vcol = 8 * (lane >> 4);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-#pragma unroll
-        for (int j2 = 0; j2 < 8; ++j2) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(tbs + G::VT + 2 * ((16 * kk + vrow) * kTS + 16 * j2 + vcol), b0, b1, b2, b3);
-          mma16816(o[2 * j2], pa[kk][0], pa[kk][1], pa[kk][2], pa[kk][3], b0, b1);
-          mma16816(o[2 * j2 + 1], pa[kk][0], pa[kk][1], pa[kk][2], pa[kk][3], b2, b3);
+        for (int k = 0; k < 16; ++k) {
+          const float v0 = x[32 * blk + 2 * k] * qs, v1 = x[32 * blk + 2 * k + 1] * qs;
+          const __half h0 = __float2half_rn(v0), h1 = __float2half_rn(v1);
+          hw[k] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
+          lw[k] = pack_half2(v0 - __half2float(h0), v1 - __half2float(h1));
         }
+        tc::tmem_st16_nowait(tmem + trow + kColQH + 16 * blk, hw);
+        tc::tmem_st16_nowait(tmem + trow + kColQL + 16 * blk, lw);
       }
+      tc::tmem_wait_st();
+      si = live_row ? 1.f / (qs * kKScale) : 1.f;
     }
-    // ---- the next chunk into the other buffer (its last readers were the
-    // MMAs of chunk c - 1, finished before the previous barrier)
-    if (c + 1 < nchunks) {
-      const bool ok = mbar_wait(bar0 + 8 * ((c + 1) & 1), (uint32_t)((c + 1) >> 1) & 1u);
-      if (ok) dequant(c + 1);
-      if (!__syncthreads_and(ok)) {                // a copy never completed
-        stalled = true;
-        if (tid == 0 && a.dev_status) atomicOr(a.dev_status, TQ_DEV_WAIT_TIMEOUT);
-        // wait (bounded) for the copies still in flight, then stop
-        if (tid == 0)
-          for (int k = c + 1; k < issued; ++k)
-            mbar_wait(bar0 + 8 * (k & 1), (uint32_t)(k >> 1) & 1u);
+    tc::fence_before_sync();
+    __syncwarp();
+    if (lane == 0) tc::bar_arrive(q_ready);
+
+    const int lim = live_row ? start + i0 + t : -1;  // last visible position
+    const float2 si2 = make_float2(si, si);
+    // mu: reference maximum of the unscaled scores (score x K norm). It moves
+    // only when a row's maximum exceeds it by more than 8 in the base-2
+    // exponent, so the output is rarely rescaled; weights are taken as
+    // 2^(si·(v - mu) - 8) <= 1 (the factor cancels in O / l), which keeps P'
+    // within the V norm's range as in decode
+    float mu = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int c = 0; c < nchunks; ++c) {
+      // the scores, and (acquired from the dequantizing warps directly) the
+      // chunk's norms
+      ok = wait(s_full(c), par2(c)) && wait(k_ready(c), par4(c));
+      if (!__all_sync(0xFFFFFFFFu, ok)) {
+        ok = false;
         break;
       }
-      // slot (c + 1) & 1 is consumed: chunk c + 3 goes there
-      if (tid == 0 && c + 3 < nchunks) issue(c + 3);
-      if (c + 3 < nchunks) issued = c + 4;
-    }
-  }
-
-  // ---- per-row sums, normalization, inverse rotation, store
+      tc::fence_after_sync();
+      const int t0 = (cbase + c) * kTChunk;
+      const int ns = (c & (kTNormSlots - 1)) * kTChunk;
+      const float4* nk4 = reinterpret_cast<const float4*>(smem + G::NKF) + ns / 4;
+      const float4* nv4 = reinterpret_cast<const float4*>(smem + G::NVF) + ns / 4;
+      float sv[kTChunk];
+      {
+        float z[32];
+        tc::tmem_ld32(tmem + trow + kColS + kTChunk * (c & 1), z);
 #pragma unroll
-  for (int o2 = 1; o2 <= 2; o2 <<= 1) {
-    l0 += __shfl_xor_sync(0xFFFFFFFFu, l0, o2);
-    l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, o2);
-  }
-  if (S > 1) {
-    // records of this split: the unnormalized value sum (rotated domain),
-    // the base-2 running maximum and the sum, per row (empty: 0, -inf, 0)
+        for (int k = 0; k < 32; ++k) sv[k] = z[k];
+        tc::tmem_ld32(tmem + trow + kColS + kTChunk * (c & 1) + 32, z);
 #pragma unroll
-    for (int rsel = 0; rsel < 2; ++rsel) {
-      const int r = rsel ? r1 : r0;
-      if (r >= R) continue;
-      const int t = r / GQ, h = r - t * GQ;
-      const size_t rec = (size_t)split * ((size_t)a.batch * T * a.n_q_heads) +
-                         ((size_t)b * T + i0 + t) * a.n_q_heads + (size_t)g * GQ + h;
-      float* dst = a.records + rec * (D + 2);
-      const float m = stalled ? -INFINITY : (rsel ? m1 : m0);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float v0 = stalled || m == -INFINITY ? 0.f : o[j][2 * rsel];
-        const float v1 = stalled || m == -INFINITY ? 0.f : o[j][2 * rsel + 1];
-        *reinterpret_cast<float2*>(dst + 8 * j + 2 * tq) = make_float2(v0, v1);
+        for (int k = 0; k < 32; ++k) sv[32 + k] = z[k];
       }
-      if (tq == 0)
-        *reinterpret_cast<float2*>(dst + D) =
-            make_float2(m, m == -INFINITY ? 0.f : (rsel ? l1 : l0));
-    }
-    return;
-  }
-  const float il0 = l0 > 0.f && !stalled ? 1.f / l0 : 0.f;
-  const float il1 = l1 > 0.f && !stalled ? 1.f / l1 : 0.f;
-  // x[k][e]: coordinate 8k + 2tq + e of row r0 (y: row r1)
-  float x[16][2], y[16][2];
+      // the score buffer is free for chunk c + 2
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::bar_arrive(s_free(c));
+      float mx = -INFINITY;
+      const bool masked = t0 + kTChunk - 1 > lim;
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    x[j][0] = o[j][0] * il0; x[j][1] = o[j][1] * il0;
-    y[j][0] = o[j][2] * il1; y[j][1] = o[j][3] * il1;
-  }
-  // Walsh-Hadamard over the 128 coordinates c = 8j + 2tq + e: bit 0 in the
-  // register pair, bits 1-2 across the four lanes tq, bits 3-6 across j.
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    float u = x[j][0], v = x[j][1];
-    x[j][0] = u + v; x[j][1] = u - v;
-    u = y[j][0]; v = y[j][1];
-    y[j][0] = u + v; y[j][1] = u - v;
-  }
-#pragma unroll
-  for (int ob = 1; ob <= 2; ob <<= 1) {
-    const bool upper = tq & ob;
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float px = __shfl_xor_sync(0xFFFFFFFFu, x[j][e], ob);
-        const float py = __shfl_xor_sync(0xFFFFFFFFu, y[j][e], ob);
-        x[j][e] = upper ? px - x[j][e] : x[j][e] + px;
-        y[j][e] = upper ? py - y[j][e] : y[j][e] + py;
-      }
-  }
-#pragma unroll
-  for (int sj = 1; sj < 16; sj <<= 1)
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-      if (!(j & sj))
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          float u = x[j][e], v = x[j + sj][e];
-          x[j][e] = u + v; x[j + sj][e] = u - v;
-          u = y[j][e]; v = y[j + sj][e];
-          y[j][e] = u + v; y[j + sj][e] = u - v;
+      for (int k = 0; k < kTChunk; k += 4) {
+        const float4 n = nk4[k / 4];
+        float2 v0 = __fmul2_rn(make_float2(sv[k], sv[k + 1]), make_float2(n.x, n.y));
+        float2 v1 = __fmul2_rn(make_float2(sv[k + 2], sv[k + 3]), make_float2(n.z, n.w));
+        if (masked) {
+          if (t0 + k > lim) v0.x = -INFINITY;
+          if (t0 + k + 1 > lim) v0.y = -INFINITY;
+          if (t0 + k + 2 > lim) v1.x = -INFINITY;
+          if (t0 + k + 3 > lim) v1.y = -INFINITY;
         }
+        sv[k] = v0.x; sv[k + 1] = v0.y; sv[k + 2] = v1.x; sv[k + 3] = v1.y;
+        mx = fmaxf(mx, fmaxf(fmaxf(v0.x, v0.y), fmaxf(v1.x, v1.y)));
+      }
+      const float mn = fmaxf(mu, mx);
+      // the output row holds earlier chunks' products: rescale it (after the
+      // previous P'·V completes) when the reference maximum moves
+      const bool grow = mu != -INFINITY && si * (mn - mu) > 8.f;
+      const float al = grow ? fast_exp2(si * (mu - mn)) : 1.f;
+      if (__any_sync(0xFFFFFFFFu, grow)) {
+        ok = wait(pv_done(c - 1), par2(c - 1));
+        if (!__all_sync(0xFFFFFFFFu, ok)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+#pragma unroll 1
+        for (int q4 = 0; q4 < kTD / 32; ++q4) {
+          float z[32];
+          tc::tmem_ld32(tmem + trow + kColO + 32 * q4, z);
 #pragma unroll
-  for (int rsel = 0; rsel < 2; ++rsel) {
-    const int r = rsel ? r1 : r0;
-    if (r >= R) continue;
-    const int t = r / GQ, h = r - t * GQ;
-    const size_t ob = (((size_t)b * T + i0 + t) * a.n_q_heads + (size_t)g * GQ + h) * D;
+          for (int k = 0; k < 32; k += 2) {
+            const float2 y = __fmul2_rn(make_float2(z[k], z[k + 1]), make_float2(al, al));
+            z[k] = y.x;
+            z[k + 1] = y.y;
+          }
+          tc::tmem_st32(tmem + trow + kColO + 32 * q4, z);
+        }
+      }
+      if (grow || mu == -INFINITY) mu = mn;
+      // weights 2^(si·v - si·mu - 8) (0 for masked scores), their sum, and P'
+      const float off = mu == -INFINITY ? 0.f : -fmaf(si, mu, 8.f);
+      const float2 off2 = make_float2(off, off);
+      float2 ls = make_float2(0.f, 0.f);
+      uint32_t pw[kTChunk / 2];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int c = 8 * j + 2 * tq;
-      float v0 = rsel ? y[j][0] : x[j][0], v1 = rsel ? y[j][1] : x[j][1];
-      v0 = apply_sign(v0, sm.w[c >> 5], c & 31) * (1.f / D);
-      v1 = apply_sign(v1, sm.w[(c + 1) >> 5], (c + 1) & 31) * (1.f / D);
-      if (a.out_dtype == TQ_F32) {
-        *reinterpret_cast<float2*>(reinterpret_cast<float*>(a.out) + ob + c) = make_float2(v0, v1);
+      for (int k = 0; k < kTChunk; k += 4) {
+        const float4 n = nv4[k / 4];
+        const float2 e0 = __ffma2_rn(make_float2(sv[k], sv[k + 1]), si2, off2);
+        const float2 e1 = __ffma2_rn(make_float2(sv[k + 2], sv[k + 3]), si2, off2);
+        const float2 w0 = make_float2(fast_exp2(e0.x), fast_exp2(e0.y));
+        const float2 w1 = make_float2(fast_exp2(e1.x), fast_exp2(e1.y));
+        ls = __fadd2_rn(ls, __fadd2_rn(w0, w1));
+        const float2 p0 = __fmul2_rn(w0, make_float2(n.x, n.y));
+        const float2 p1 = __fmul2_rn(w1, make_float2(n.z, n.w));
+        pw[k / 2] = pack_half2(p0.x, p0.y);
+        pw[k / 2 + 1] = pack_half2(p1.x, p1.y);
+      }
+      l = l * al + (ls.x + ls.y);
+      // P' row into buffer c & 1 (free once the P'·V of chunk c - 2 is done)
+      ok = wait(pv_done(c), par2(c) ^ 1);
+      if (!__all_sync(0xFFFFFFFFu, ok)) {
+        ok = false;
+        break;
+      }
+      {
+        uint32_t lo[16], hi[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          lo[k] = pw[k];
+          hi[k] = pw[16 + k];
+        }
+        tc::tmem_st16_nowait(tmem + trow + kColP + 32 * (c & 1), lo);
+        tc::tmem_st16_nowait(tmem + trow + kColP + 32 * (c & 1) + 16, hi);
+        tc::tmem_wait_st();
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::bar_arrive(p_ready(c));
+    }
+
+    // ---- output row: acc = O / l, inverse rotation D⊙(H·acc)/d (or the record)
+    if (ok && nchunks > 0) {
+      ok = wait(pv_done(nchunks - 1), par2(nchunks - 1));
+      ok = __all_sync(0xFFFFFFFFu, ok);
+    }
+    if (ok) {
+      float x[kTD];
+      if (nchunks > 0) {
+        tc::fence_after_sync();
+#pragma unroll
+        for (int q4 = 0; q4 < kTD / 32; ++q4) {
+          float z[32];
+          tc::tmem_ld32(tmem + trow + kColO + 32 * q4, z);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) x[32 * q4 + k] = z[k];
+        }
       } else {
-        const bool bf = a.out_dtype == TQ_BF16;
-        const uint32_t h0 = bf ? f32_to_bf16_bits(v0) : f32_to_f16_bits(v0);
-        const uint32_t h1 = bf ? f32_to_bf16_bits(v1) : f32_to_f16_bits(v1);
-        *reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(a.out) + ob + c) = h0 | (h1 << 16);
+#pragma unroll
+        for (int k = 0; k < kTD; ++k) x[k] = 0.f;
+      }
+      if (live_row && S > 1) {
+        // records of this split: the unnormalized value sum (rotated
+        // domain), the base-2 running maximum and the sum (empty: 0, -inf, 0)
+        const size_t rec = (size_t)split * ((size_t)a.batch * T * a.n_q_heads) +
+                           ((size_t)b * T + i0 + t) * a.n_q_heads + (size_t)g * GQ + h;
+        float* dst = a.records + rec * (kTD + 2);
+        const bool empty = mu == -INFINITY;
+#pragma unroll
+        for (int k = 0; k < kTD; k += 2)
+          *reinterpret_cast<float2*>(dst + k) =
+              make_float2(empty ? 0.f : x[k], empty ? 0.f : x[k + 1]);
+        *reinterpret_cast<float2*>(dst + kTD) =
+            make_float2(empty ? -INFINITY : fmaf(si, mu, 8.f), empty ? 0.f : l);
+      } else if (live_row) {
+        const float il = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+        for (int k = 0; k < kTD; ++k) x[k] *= il;
+#pragma unroll
+        for (int s = 1; s < kTD; s <<= 1)
+#pragma unroll
+          for (int k = 0; k < kTD; ++k)
+            if (!(k & s)) {
+              const float p = x[k], q = x[k + s];
+              x[k] = p + q;
+              x[k + s] = p - q;
+            }
+        const size_t ob = (((size_t)b * T + i0 + t) * a.n_q_heads + (size_t)g * GQ + h) * kTD;
+        if (a.out_dtype == TQ_F32) {
+          float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + ob);
+#pragma unroll
+          for (int k = 0; k < kTD; k += 4)
+            o[k / 4] = make_float4(apply_sign(x[k], sm.w[k >> 5], k & 31) * (1.f / kTD),
+                                   apply_sign(x[k + 1], sm.w[k >> 5], (k + 1) & 31) * (1.f / kTD),
+                                   apply_sign(x[k + 2], sm.w[k >> 5], (k + 2) & 31) * (1.f / kTD),
+                                   apply_sign(x[k + 3], sm.w[k >> 5], (k + 3) & 31) * (1.f / kTD));
+        } else {
+          const bool bf = a.out_dtype == TQ_BF16;
+          uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.out) + ob);
+#pragma unroll
+          for (int k = 0; k < kTD; k += 8) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c0 = k + 2 * e;
+              const float v0 = apply_sign(x[c0], sm.w[c0 >> 5], c0 & 31) * (1.f / kTD);
+              const float v1 = apply_sign(x[c0 + 1], sm.w[c0 >> 5], (c0 + 1) & 31) * (1.f / kTD);
+              const uint32_t h0 = bf ? f32_to_bf16_bits(v0) : f32_to_f16_bits(v0);
+              const uint32_t h1 = bf ? f32_to_bf16_bits(v1) : f32_to_f16_bits(v1);
+              w4[e] = h0 | (h1 << 16);
+            }
+            o[k / 8] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
+        }
       }
     }
   }
+  if (tid == 0 && *reinterpret_cast<volatile int*>(abort_flag) && a.dev_status)
+    atomicOr(a.dev_status, TQ_DEV_WAIT_TIMEOUT);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 9) tc::tmem_dealloc(tmem, kTTmemCols);
 }
 
 template <int BK, int BV>
 cudaError_t launch_prefill_bits(const PrefillArgs& a, const Codebook& cbk, const Codebook& cbv,
-                                const SignMask& sm, cudaStream_t stream) {
-  using G = PfGeo<BK, BV>;
-  // set once per device (idempotent; atomic so that concurrent first calls do not race)
+                                   const SignMask& sm, cudaStream_t stream) {
+  using G = TcGeo<BK, BV>;
   static std::atomic<bool> configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || !configured[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(prefill_kernel<BK, BV>,
+    const cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<BK, BV>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }
-  const int tq = kPfRows / a.gqa;
+  const int tq = kTRows / a.gqa;
   const int S = a.n_splits > 1 ? a.n_splits : 1;
   const long long grid = (long long)a.batch * a.n_kv_heads * ((a.n_tok + tq - 1) / tq) * S;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(kPfThreads);
+  cfg.blockDim = dim3(kTThreads);
   cfg.dynamicSmemBytes = G::SMEM;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -536,14 +648,14 @@ cudaError_t launch_prefill_bits(const PrefillArgs& a, const Codebook& cbk, const
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_kernel<BK, BV>, a, cbk, cbv, sm);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_tc_kernel<BK, BV>, a, cbk, cbv, sm);
   if (e != cudaSuccess || S == 1) return e;
   // merge the splits' records and rotate back (the context-parallel combine)
   CombineArgs c;
   c.partials = a.records;
   c.n_parts = S;
   c.n_rec = a.batch * a.n_tok * a.n_q_heads;
-  c.d = 128;
+  c.d = kTD;
   c.dev_status = a.dev_status;
   c.out = a.out;
   c.out_dtype = a.out_dtype;
@@ -553,12 +665,7 @@ cudaError_t launch_prefill_bits(const PrefillArgs& a, const Codebook& cbk, const
 }  // namespace
 
 cudaError_t launch_prefill(const PrefillArgs& a, const Codebook& cbk, const Codebook& cbv,
-                           const SignMask& sm, cudaStream_t stream) {
-  return launch_prefill_tc(a, cbk, cbv, sm, stream);
-}
-
-cudaError_t launch_prefill_mma_sync(const PrefillArgs& a, const Codebook& cbk,
-                                    const Codebook& cbv, const SignMask& sm, cudaStream_t stream) {
+                              const SignMask& sm, cudaStream_t stream) {
   switch (a.bits_k * 8 + a.bits_v) {
     case 4 * 8 + 2: return launch_prefill_bits<4, 2>(a, cbk, cbv, sm, stream);
     case 3 * 8 + 2: return launch_prefill_bits<3, 2>(a, cbk, cbv, sm, stream);

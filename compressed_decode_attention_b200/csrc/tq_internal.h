@@ -127,9 +127,6 @@ struct PrefillArgs {
 constexpr int kMaxPrefillSplits = 8;
 cudaError_t launch_prefill(const PrefillArgs& a, const Codebook& cbk, const Codebook& cbv,
                            const SignMask& sm, cudaStream_t stream);
-// The same on the fifth-generation tensor cores (prefill_tc.cu).
-cudaError_t launch_prefill_tc(const PrefillArgs& a, const Codebook& cbk, const Codebook& cbv,
-                              const SignMask& sm, cudaStream_t stream);
 
 struct CombineArgs {
   const float* partials;     // [n_parts][n_rec][d + 2]

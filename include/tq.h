@@ -71,7 +71,7 @@
 extern "C" {
 #endif
 
-#define TQ_ABI_VERSION 7
+#define TQ_ABI_VERSION 8
 
 /* Tokens per sparse-V block; split boundaries are multiples of this. */
 #define TQ_SPARSE_V_BLOCK 64
@@ -346,10 +346,13 @@ int tq_prefill_attend_split(const void* q, int q_dtype,
  * n_q_heads · (d + 2) floats; 0 for n_splits <= 1 or invalid arguments. */
 size_t tq_prefill_workspace_size(int batch, int n_tok, int n_q_heads, int d, int n_splits);
 
-/* A split count for tq_prefill_attend_split on the current device: the
- * n in 1..8 that minimizes ceil(tiles·n / SMs) / n (rounds of the SMs per
- * unit of work) plus a small charge per split. Host only; 1 on bad input. */
-int tq_prefill_splits(int batch, int n_tok, int n_q_heads, int gqa_ratio);
+/* A split count for tq_prefill_attend_split on the current device, for
+ * sequences of at most max_ctx positions (n_tok if smaller): the n in 1..8
+ * that minimizes ceil(tiles·n / SMs) · (chunks / n + 10), i.e. rounds of
+ * the SMs times the time of one CTA, which handles 1/n of the longest
+ * tile's 64-position chunks after a fixed cost of about 10 chunks (set-up,
+ * pipeline fill and drain). Host only; 1 on bad input. */
+int tq_prefill_splits(int batch, int n_tok, int n_q_heads, int gqa_ratio, int max_ctx);
 
 /*
  * Context parallelism: the positions of every sequence are split over the

@@ -51,6 +51,7 @@ def test_encode_k4v3_batched_serving_sequence():
     n = int(S.ctx_lens(w)[0])
     kv = S.kv_bits(w, 0, n)
     pk, nk, pv, nv, st = gpu_encode(kv, w.dtype, w.bits_k, w.bits_v, SEED, cap=w.cap_tok)
+    assert st == 0
     _compare(kv, w.dtype, w.bits_k, w.bits_v, SEED, pk, nk, pv, nv, parallel=True,
              count_rule=True)
 

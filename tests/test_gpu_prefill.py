@@ -184,9 +184,10 @@ def test_prefill_split_short_context_and_dtypes():
     assert err <= ATOL
 
 
-def test_prefill_split_full_workload_sampled():
-    """The bench's prefill line with the split count the library picks for
-    this device (4 on 148 SMs)."""
+@pytest.mark.parametrize("forced", [0, 4])
+def test_prefill_split_full_workload_sampled(forced):
+    """The bench's prefill chunk with the split count the library picks for
+    this device (forced = 0) and with 4 context splits."""
     import torch
     import compressed_decode_attention_b200 as tq
     rng = np.random.default_rng(43)
@@ -195,7 +196,7 @@ def test_prefill_split_full_workload_sampled():
     pk, nk, pv, nv = _cache(bk, bv, B, Hkv, L, np.array([L]), seed, rng)
     qb = S.f16_bits(rng.standard_normal((B, T, Hq, D)))
     q64 = codec.promote(qb, "f16")
-    n_splits = tq.tq_prefill_splits(B, T, Hq, gqa)
+    n_splits = forced or tq.tq_prefill_splits(B, T, Hq, gqa, L)
     assert n_splits >= 1
     wsb = tq.tq_prefill_workspace_size(B, T, Hq, D, n_splits)
     ws = torch.empty(max(wsb, 16) // 4, dtype=torch.float32, device="cuda")

@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol():
 def test_abi_version_and_status_strings():
     hdr = open(os.path.join(ROOT, "include", "tq.h")).read()
     assert tq.tq_abi_version() == int(re.search(r"#define TQ_ABI_VERSION (\d+)", hdr).group(1))
-    assert tq.tq_abi_version() == 7
+    assert tq.tq_abi_version() == 8
     assert tq.status_string(0) == "TQ_OK"
     assert tq.status_string(2) == "TQ_ERR_UNSUPPORTED"
 
@@ -267,8 +267,8 @@ def test_prefill_workspace_size_and_split_choice():
     assert tq.tq_prefill_workspace_size(2, 16, 8, 128, 3) == 3 * 2 * 16 * 8 * 130 * 4
     assert tq.tq_prefill_workspace_size(2, 16, 8, 128, 1) == 0
     assert tq.tq_prefill_workspace_size(2, 16, 8, 96, 3) == 0
-    assert 1 <= tq.tq_prefill_splits(1, 1024, 32, 4) <= 8
-    assert tq.tq_prefill_splits(0, 1024, 32, 4) == 1
+    assert 1 <= tq.tq_prefill_splits(1, 1024, 32, 4, 8192) <= 8
+    assert tq.tq_prefill_splits(0, 1024, 32, 4, 8192) == 1
 
 
 @pytest.mark.parametrize("head_skipped,want", [
