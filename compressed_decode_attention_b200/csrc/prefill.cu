@@ -5,33 +5,36 @@
 // and the weighted sum are those of decode ([ADAPTQ §How it works, item 3]:
 // rotated query, codebook values of the packed indices, inverse rotation of
 // the output). With 128 query rows per kv head and chunk this is a dense
-// contraction, so each 64-position chunk of the cache is dequantized once
+// contraction, so each 128-position chunk of the cache is dequantized once
 // into shared-memory operand tiles and reused by all rows.
 //
 // One CTA per (context split, sequence, kv head, tile of 128 query rows); a
 // row is a (token, query head of the GQA group) pair. Warp roles:
-//   warps 0-3  one thread per row: rotate its query (thread-local FWHT) into
-//              fp16 high/low parts in tensor memory; per chunk read the row
-//              of scores, scale, causal mask, online softmax in the log2
-//              domain, rescale the output row when the maximum grows, and
-//              write the row of P' = weight x V norm (fp16) to tensor memory;
-//              at the end read the output row, normalize, inverse-rotate and
-//              store it (or the split's record)
-//   warps 4-7  dequantize a chunk: K codebook values as fp16 high and low
-//              tiles [64 positions x 128 coordinates] and the norms, then V
-//              [64 positions x 128 coordinates]
-//   warp 8     bulk copies of the packed rows and norms (four slots)
-//   warp 9     tensor memory (512 columns: two score buffers of 64, the
-//              128-column output, the query's high and low parts, two P'
-//              buffers); one thread issues per chunk
-//                S = Q_hi·K_hi + Q_lo·K_hi + Q_hi·K_lo  (M 128, N 64, K 128)
-//                O += P'·V                              (M 128, N 128, K 64)
-//              kind::f16 MMAs with fp32 accumulators, the A operands (Q, P')
-//              in tensor memory, scores one chunk ahead of P'·V
-// K tiles are K-major and V tiles MN-major (position rows of coordinates),
-// both in the 128-byte swizzle layout (tc_common.cuh). A K buffer is free
-// once its scores are done and a V buffer once its P'·V is, so the
-// dequantization of chunk c + 2 overlaps the products of chunk c + 1.
+//   warps 0-3   one thread per row: rotate its query (thread-local FWHT)
+//               into fp16 high/low parts in tensor memory; per chunk read
+//               the row of scores (two passes of four 32-column loads:
+//               maximum, then weights), scale, causal mask, online softmax
+//               in the log2 domain, rescale the output row when the
+//               reference maximum moves, and write the row of P' = weight x
+//               V norm (fp16 pairs) over the columns of its own scores; at
+//               the end read the output row, normalize, inverse-rotate and
+//               store it (or the split's record)
+//   warps 4-7   dequantize K: codebook values as fp16 high and low tiles
+//               [128 positions x 128 coordinates], and the chunk's norms
+//   warps 8-9   dequantize V [128 positions x 128 coordinates]
+//   warp 10     bulk copies of the packed rows and norms (two slots)
+//   warp 11     tensor memory (512 columns: two 128-column score buffers,
+//               the 128-column output, the query's high and low parts); one
+//               thread issues per chunk
+//                 S = Q_hi·K_hi + Q_lo·K_hi + Q_hi·K_lo  (M 128, N 128, K 128)
+//                 O += P'·V                              (M 128, N 128, K 128)
+//               kind::f16 MMAs with fp32 accumulators, the A operands (Q,
+//               P') in tensor memory, scores one chunk ahead of P'·V
+// K tiles are K-major and the V tile MN-major (position rows of
+// coordinates), in the 128-byte swizzle layout (tc_common.cuh). K tiles are
+// double-buffered (a buffer is free once its scores are done), the V tile
+// is single (free once its P'·V is done), and a score buffer is reused
+// once the P'·V that read its P' is done.
 // The high/low split keeps ~22 significant bits of the scores as in decode;
 // P' and V are fp16 as in decode. Every wait is bounded; a role that gives
 // up sets TQ_DEV_WAIT_TIMEOUT and stops, and the tensor memory is freed
@@ -45,40 +48,38 @@ namespace tq {
 namespace {
 
 constexpr int kTRows = 128;                       // query rows per tile (MMA M)
-constexpr int kTChunk = 64;                       // cache positions per chunk
+constexpr int kTChunk = 128;                      // cache positions per chunk (MMA N)
 constexpr int kTD = 128;                          // head dimension
-constexpr int kTWarps = 10;
+constexpr int kTWarps = 12;
 constexpr int kTThreads = 32 * kTWarps;
-constexpr int kTStages = 4;                       // staging slots of packed rows
-constexpr int kTNormSlots = 8;                    // ring of per-chunk norms
+constexpr int kTNormSlots = 4;                    // ring of per-chunk norms
 constexpr long long kTWait = 2000000000LL;         // cycles (~1 s)
 // tensor-memory columns
-constexpr uint32_t kColS = 0;                     // 2 x 64: scores
-constexpr uint32_t kColO = 128;                   // 128: output accumulator
-constexpr uint32_t kColQH = 256, kColQL = 320;    // 64 each: query parts (fp16 pairs)
-constexpr uint32_t kColP = 384;                   // 2 x 32: P' (fp16 pairs)
+constexpr uint32_t kColS = 0;                     // 2 x 128: scores, then P' (fp16 pairs)
+constexpr uint32_t kColO = 256;                   // 128: output accumulator
+constexpr uint32_t kColQH = 384, kColQL = 448;    // 64 each: query parts (fp16 pairs)
 constexpr uint32_t kTTmemCols = 512;
 
 template <int BK, int BV>
 struct TcGeo {
   static constexpr int RK = 16 * BK, RV = 16 * BV;            // packed row bytes (d = 128)
-  static constexpr int TILE = kTChunk * kTD * 2;              // 16 KB: [64 x 128] fp16
+  static constexpr int TILE = kTChunk * kTD * 2;              // 32 KB: [128 x 128] fp16
   static constexpr int KH = 0;                                // 2 K high tiles
   static constexpr int KL = KH + 2 * TILE;                    // 2 K low tiles
-  static constexpr int VV = KL + 2 * TILE;                    // 2 V tiles
+  static constexpr int VV = KL + 2 * TILE;                    // the V tile
   static constexpr int SLOT = kTChunk * (RK + RV) + 2 * kTChunk * 2;
-  static constexpr int STG = VV + 2 * TILE;                   // staging slots
-  static constexpr int NKF = STG + kTStages * SLOT;           // norm ring: 64 floats a slot
+  static constexpr int STG = VV + TILE;                       // 2 staging slots
+  static constexpr int NKF = STG + 2 * SLOT;                  // norm ring: 128 floats a slot
   static constexpr int NVF = NKF + kTNormSlots * kTChunk * 4;
-  // codebook tables, one copy per lane group where random lookups of a
-  // warp would collide in shared-memory banks: K (uint2 per pair code) 16
-  // copies unless 2-bit, V (uint32 per pair code) 32 copies unless 2-bit
-  static constexpr int KREP = BK == 2 ? 1 : 16, VREP = BV == 2 ? 1 : 32;
-  static constexpr int KSH = BK == 2 ? 3 : 7, VSH = BV == 2 ? 2 : 7;  // log2 bytes per code
+  // codebook tables, eight copies (one per lane & 7) where random lookups of
+  // a warp would collide in shared-memory banks: K (uint2 per pair code)
+  // unless 2-bit, V (uint32 per pair code) unless 2-bit
+  static constexpr int KREP = BK == 2 ? 1 : 8, VREP = BV == 2 ? 1 : 8;
+  static constexpr int KSH = BK == 2 ? 3 : 6, VSH = BV == 2 ? 2 : 5;  // log2 bytes per code
   static constexpr int LUTK = NVF + kTNormSlots * kTChunk * 4;
   static constexpr int LUTV = LUTK + (1 << (2 * BK)) * 8 * KREP;
-  static constexpr int BARS = LUTV + (1 << (2 * BV)) * 4 * VREP;  // 24 barriers
-  static constexpr int MISC = BARS + 24 * 8;                  // TMEM address, abort flag
+  static constexpr int BARS = LUTV + (1 << (2 * BV)) * 4 * VREP;  // 16 barriers
+  static constexpr int MISC = BARS + 16 * 8;                  // TMEM address, abort flag
   static constexpr int SMEM = 1024 + MISC + 16;
   static_assert(SLOT % 16 == 0 && STG % 1024 == 0 && NKF % 16 == 0 && BARS % 8 == 0, "align");
   static_assert(SMEM <= 227 * 1024, "shared memory");
@@ -105,22 +106,22 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
   const int b = unit / (tiles * H);
   const int i0 = tile * TQ, nq = min(TQ, T - i0);
   const int R = nq * GQ;                           // valid rows
-  // barriers (chunk c uses slot c & 3 of the four-deep rings and c & 1 of
-  // the two-deep ones): staging full/free and K ready (x4); V ready, scores
-  // full/free, P' ready, P'·V done (x2); query ready
+  // barriers (chunk c uses slot c & 1 of the two-deep rings, c & 3 of the
+  // four-deep one): staging full/free, K ready (x4), V ready (x1), scores
+  // full, P' ready, P'·V done, query ready
   const uint32_t bars = sb + G::BARS;
-  auto stage_full = [&](int c) { return bars + 8 * (0 + (c & 3)); };
-  auto stage_free = [&](int c) { return bars + 8 * (4 + (c & 3)); };
-  auto k_ready = [&](int c) { return bars + 8 * (8 + (c & 3)); };
-  auto v_ready = [&](int c) { return bars + 8 * (12 + (c & 1)); };
-  auto s_full = [&](int c) { return bars + 8 * (14 + (c & 1)); };
-  auto s_free = [&](int c) { return bars + 8 * (16 + (c & 1)); };
-  auto p_ready = [&](int c) { return bars + 8 * (18 + (c & 1)); };
-  auto pv_done = [&](int c) { return bars + 8 * (20 + (c & 1)); };
-  const uint32_t q_ready = bars + 8 * 22;
-  // phase parity of chunk c's use of a four- or two-deep ring slot
-  auto par4 = [](int c) { return (uint32_t)((c >> 2) & 1); };
+  auto stage_full = [&](int c) { return bars + 8 * (0 + (c & 1)); };
+  auto stage_free = [&](int c) { return bars + 8 * (2 + (c & 1)); };
+  auto k_ready = [&](int c) { return bars + 8 * (4 + (c & 3)); };
+  const uint32_t v_ready = bars + 8 * 8;
+  auto s_full = [&](int c) { return bars + 8 * (9 + (c & 1)); };
+  auto p_ready = [&](int c) { return bars + 8 * (11 + (c & 1)); };
+  auto pv_done = [&](int c) { return bars + 8 * (13 + (c & 1)); };
+  const uint32_t q_ready = bars + 8 * 15;
+  // phase parity of chunk c's use of a one-, two- or four-deep ring slot
+  auto par1 = [](int c) { return (uint32_t)(c & 1); };
   auto par2 = [](int c) { return (uint32_t)((c >> 1) & 1); };
+  auto par4 = [](int c) { return (uint32_t)((c >> 2) & 1); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + G::MISC);
   int* abort_flag = reinterpret_cast<int*>(smem + G::MISC + 4);
   auto wait = [&](uint32_t bar, uint32_t parity) {
@@ -153,23 +154,20 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
       *reinterpret_cast<uint32_t*>(smem + G::LUTV + (code << G::VSH) + 4 * rep) = v0 | (v1 << 16);
   }
   if (tid == 0) {
-    for (int i = 0; i < 4; ++i) {
-      tc::bar_init(stage_full(i), 1);
-      tc::bar_init(stage_free(i), 4);
-      tc::bar_init(k_ready(i), 4);
-    }
     for (int i = 0; i < 2; ++i) {
-      tc::bar_init(v_ready(i), 4);
+      tc::bar_init(stage_full(i), 1);
+      tc::bar_init(stage_free(i), 6);              // the K and V dequantizing warps
       tc::bar_init(s_full(i), 1);
-      tc::bar_init(s_free(i), 4);
       tc::bar_init(p_ready(i), 4);
       tc::bar_init(pv_done(i), 1);
     }
+    for (int i = 0; i < 4; ++i) tc::bar_init(k_ready(i), 4);
+    tc::bar_init(v_ready, 2);
     tc::bar_init(q_ready, 4);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
-  if (warp == 9) tc::tmem_alloc(tc::saddr(tmem_slot), kTTmemCols);
+  if (warp == 11) tc::tmem_alloc(tc::saddr(tmem_slot), kTTmemCols);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -189,16 +187,16 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
   const int nchunks = (int)((long long)(split + 1) * nch_tile / S) - cbase;
   const size_t seq_row = ((size_t)b * H + g) * a.cap_tok;
 
-  if (warp == 8) {
-    // ---- producer: chunk c into staging slot c & 3
+  if (warp == 10) {
+    // ---- producer: chunk c into staging slot c & 1
     if (lane == 0) {
       int c = 0;
       for (; c < nchunks; ++c) {
-        if (!wait(stage_free(c), par4(c) ^ 1)) break;
+        if (!wait(stage_free(c), par2(c) ^ 1)) break;
         const int t0 = (cbase + c) * kTChunk;
         const int rows = min(kTChunk, L - t0);
         const int nrows = min(kTChunk, (rows + 7) & ~7);
-        const uint32_t dst = sb + G::STG + (c & 3) * G::SLOT;
+        const uint32_t dst = sb + G::STG + (c & 1) * G::SLOT;
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
         tc::bar_expect(stage_full(c), rows * (G::RK + G::RV) + 4 * nrows);
         tc::bulk_g2s(dst, a.packed_k + (seq_row + t0) * G::RK, rows * G::RK, stage_full(c));
@@ -210,133 +208,147 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
                      2 * nrows, stage_full(c));
       }
       // copies still in flight complete before the CTA can end
-      for (int k = c > kTStages ? c - kTStages : 0; k < c; ++k)
-        tc::bar_wait(stage_full(k), par4(k), kTWait);
+      for (int k = c > 2 ? c - 2 : 0; k < c; ++k) tc::bar_wait(stage_full(k), par2(k), kTWait);
+    }
+  } else if (warp == 11) {
+    // ---- MMA issue (one thread)
+    if (lane == 0) {
+      constexpr uint32_t idS = tc::umma_idesc(0u, kTRows, kTChunk);
+      constexpr uint32_t idO = tc::umma_idesc(0u, kTRows, kTD) | (1u << 16);  // B MN-major
+      bool ok = nchunks == 0 || wait(q_ready, 0);
+      uint32_t last_bar = 0, last_par = 0;        // the latest commit's barrier and phase
+      // descriptors of buffer 0, k-step 0 (a start address moves the low
+      // field by bytes / 16)
+      const uint64_t kdesc = tc::umma_desc(sb + G::KH);
+      const uint64_t vdesc = tc::umma_desc_mn(sb + G::VV, kTChunk * 128, 1024);
+      auto scores = [&](int c) {
+        // K buffer c & 1 ready; score buffer c & 1 free once the P'·V of
+        // chunk c - 2 (which read its P') is done
+        if (!wait(k_ready(c), par4(c)) || (c >= 2 && !wait(pv_done(c - 2), par2(c - 2))))
+          return false;
+        tc::fence_after_sync();
+        const uint32_t d = tmem + kColS + kTChunk * (c & 1);
+        const uint64_t kb = kdesc + (uint32_t)(((c & 1) * G::TILE) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < kTD / 16; ++kk) {
+          const uint32_t koff = (kk >> 2) * (kTChunk * 128) + (kk & 3) * 32;
+          const uint64_t kh = kb + (koff >> 4);
+          const uint64_t kl = kb + ((koff + (G::KL - G::KH)) >> 4);
+          tc::mma_f16_ts(d, tmem + kColQH + 8 * kk, kh, idS, kk > 0);
+          tc::mma_f16_ts(d, tmem + kColQL + 8 * kk, kh, idS, true);
+          tc::mma_f16_ts(d, tmem + kColQH + 8 * kk, kl, idS, true);
+        }
+        tc::mma_commit(s_full(c));
+        last_bar = s_full(c);
+        last_par = par2(c);
+        return true;
+      };
+      auto pv = [&](int c) {
+        if (!wait(v_ready, par1(c)) || !wait(p_ready(c), par2(c))) return false;
+        tc::fence_after_sync();
+#pragma unroll
+        for (int kk = 0; kk < kTChunk / 16; ++kk)
+          tc::mma_f16_ts(tmem + kColO, tmem + kColS + kTChunk * (c & 1) + 8 * kk,
+                         vdesc + (uint32_t)(kk * 2048 >> 4), idO, c > 0 || kk > 0);
+        tc::mma_commit(pv_done(c));
+        last_bar = pv_done(c);
+        last_par = par2(c);
+        return true;
+      };
+      if (ok && nchunks > 0) ok = scores(0);
+      for (int c = 0; ok && c < nchunks; ++c) {
+        if (c + 1 < nchunks && !scores(c + 1)) break;
+        if (!pv(c)) break;
+      }
+      // the last committed products (and all before them) complete before
+      // the tensor memory is freed
+      if (last_bar) tc::bar_wait(last_bar, last_par, kTWait);
+    }
+  } else if (warp >= 8) {
+    // ---- V dequantization (warps 8-9, thread v): positions (v & 31) + 32j,
+    // coordinates 64·(v >> 5) .. + 63 (eight consecutive positions per
+    // quarter warp: the 16-byte tile stores fall in distinct banks)
+    const int v = tid - 256;
+    const int half = v >> 5;
+    const uint32_t vrep = G::VREP > 1 ? 4 * (lane & 7) : 0;   // this lane's table copy
+    for (int c = 0; c < nchunks; ++c) {
+      // the V tile is free once the P'·V of chunk c - 1 is done
+      const bool ok = wait(stage_full(c), par2(c)) && (c == 0 || wait(pv_done(c - 1), par2(c - 1)));
+      if (!__all_sync(0xFFFFFFFFu, ok)) break;
+      const uint8_t* st = smem + G::STG + (c & 1) * G::SLOT;
+      uint8_t* vp = smem + G::VV;
+#pragma unroll 1
+      for (int j = 0; j < 4; ++j) {
+        const int pos = (v & 31) + 32 * j;
+        uint32_t vw[(8 * BV + 3) / 4 + 1];
+        load_chunk<8 * BV>(st, kTChunk * G::RK + pos * G::RV + 8 * BV * half, vw);
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          uint32_t p4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            p4[e] = lds<uint32_t>(smem, G::LUTV + (pair_code_shifted<BV, G::VSH>(vw, 4 * jj + e) | vrep));
+          *reinterpret_cast<uint4*>(vp + tc::sw128_offset(kTChunk, pos, 64 * half + 8 * jj)) =
+              make_uint4(p4[0], p4[1], p4[2], p4[3]);
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+      __syncwarp();
+      if (lane == 0) {
+        tc::bar_arrive(v_ready);
+        tc::bar_arrive(stage_free(c));
+      }
     }
   } else if (warp >= 4) {
-    if (warp == 9) {
-      // ---- MMA issue (one thread)
-      if (lane == 0) {
-        constexpr uint32_t idS = tc::umma_idesc(0u, kTRows, kTChunk);
-        constexpr uint32_t idO = tc::umma_idesc(0u, kTRows, kTD) | (1u << 16);  // B MN-major
-        bool ok = nchunks == 0 || wait(q_ready, 0);
-        uint32_t last_bar = 0, last_par = 0;      // the latest commit's barrier and phase
-        // descriptors of buffer 0, k-step 0 (a start address moves the low
-        // field by bytes / 16)
-        const uint64_t kdesc = tc::umma_desc(sb + G::KH);
-        const uint64_t vdesc = tc::umma_desc_mn(sb + G::VV, 64 * 128, 1024);
-        auto scores = [&](int c) {
-          if (!wait(k_ready(c), par4(c)) || !wait(s_free(c), par2(c) ^ 1)) return false;
-          tc::fence_after_sync();
-          const uint32_t d = tmem + kColS + kTChunk * (c & 1);
-          const uint64_t kb = kdesc + (uint32_t)(((c & 1) * G::TILE) >> 4);
+    // ---- K dequantization (warps 4-7, thread u): positions (u & 63) + 64j,
+    // coordinates 64·(u >> 6) .. + 63, and the norms of position u
+    const int u = tid - 128;
+    const int half = u >> 6;
+    const uint32_t krep = G::KREP > 1 ? 8 * (lane & 7) : 0;   // this lane's table copy
+    for (int c = 0; c < nchunks; ++c) {
+      const int i = c & 1;
+      // K buffer i: free once the scores of chunk c - 2 are done
+      const bool ok = wait(stage_full(c), par2(c)) && wait(s_full(c), par2(c) ^ 1);
+      if (!__all_sync(0xFFFFFFFFu, ok)) break;
+      const uint8_t* st = smem + G::STG + i * G::SLOT;
+      uint8_t* khp = smem + G::KH + i * G::TILE;
+      uint8_t* klp = smem + G::KL + i * G::TILE;
+#pragma unroll 1
+      for (int j = 0; j < 2; ++j) {
+        const int pos = (u & 63) + 64 * j;
+        uint32_t kw[(8 * BK + 3) / 4 + 1];
+        load_chunk<8 * BK>(st, pos * G::RK + 8 * BK * half, kw);
 #pragma unroll
-          for (int kk = 0; kk < kTD / 16; ++kk) {
-            const uint32_t koff = (kk >> 2) * (kTChunk * 128) + (kk & 3) * 32;
-            const uint64_t kh = kb + (koff >> 4);
-            const uint64_t kl = kb + ((koff + (G::KL - G::KH)) >> 4);
-            tc::mma_f16_ts(d, tmem + kColQH + 8 * kk, kh, idS, kk > 0);
-            tc::mma_f16_ts(d, tmem + kColQL + 8 * kk, kh, idS, true);
-            tc::mma_f16_ts(d, tmem + kColQH + 8 * kk, kl, idS, true);
+        for (int jj = 0; jj < 8; ++jj) {              // 16-byte chunks: 4 pairs
+          uint32_t h4[4], l4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint2 w =
+                lds<uint2>(smem, G::LUTK + (pair_code_shifted<BK, G::KSH>(kw, 4 * jj + e) | krep));
+            h4[e] = w.x;
+            l4[e] = w.y;
           }
-          tc::mma_commit(s_full(c));
-          last_bar = s_full(c);
-          last_par = par2(c);
-          return true;
-        };
-        auto pv = [&](int c) {
-          if (!wait(v_ready(c), par2(c)) || !wait(p_ready(c), par2(c))) return false;
-          tc::fence_after_sync();
-          const uint64_t vb = vdesc + (uint32_t)(((c & 1) * G::TILE) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < kTChunk / 16; ++kk)
-            tc::mma_f16_ts(tmem + kColO, tmem + kColP + 32 * (c & 1) + 8 * kk,
-                           vb + (uint32_t)(kk * 2048 >> 4), idO, c > 0 || kk > 0);
-          tc::mma_commit(pv_done(c));
-          last_bar = pv_done(c);
-          last_par = par2(c);
-          return true;
-        };
-        if (ok && nchunks > 0) ok = scores(0);
-        for (int c = 0; ok && c < nchunks; ++c) {
-          if (c + 1 < nchunks && !scores(c + 1)) break;
-          if (!pv(c)) break;
+          const uint32_t off = tc::sw128_offset(kTChunk, pos, 64 * half + 8 * jj);
+          *reinterpret_cast<uint4*>(khp + off) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+          *reinterpret_cast<uint4*>(klp + off) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
         }
-        // the last committed products (and all before them) complete before
-        // the tensor memory is freed
-        if (last_bar) tc::bar_wait(last_bar, last_par, kTWait);
       }
-    } else {
-      // ---- dequantization (warps 4-7, thread u): position u & 63,
-      // coordinates 64·(u >> 6) .. + 63 (eight consecutive positions per
-      // quarter warp: the 16-byte tile stores fall in distinct banks)
-      const int u = tid - 128;
-      const int pos = u & 63, half = u >> 6;
-      const uint32_t krep = G::KREP > 1 ? 8 * (lane & 15) : 0;   // this lane's table copies
-      const uint32_t vrep = G::VREP > 1 ? 4 * lane : 0;
-      for (int c = 0; c < nchunks; ++c) {
-        const int i = c & 1;
-        // K buffer i: free once the scores of chunk c - 2 are done
-        bool ok = wait(stage_full(c), par4(c)) && wait(s_full(c), par2(c) ^ 1);
-        if (!__all_sync(0xFFFFFFFFu, ok)) break;
-        const uint8_t* st = smem + G::STG + (c & 3) * G::SLOT;
-        {
-          uint32_t kw[(8 * BK + 3) / 4 + 1];
-          load_chunk<8 * BK>(st, pos * G::RK + 8 * BK * half, kw);
-          uint8_t* khp = smem + G::KH + i * G::TILE;
-          uint8_t* klp = smem + G::KL + i * G::TILE;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {              // 16-byte chunks: 4 pairs
-            uint32_t h4[4], l4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const uint2 v =
-                  lds<uint2>(smem, G::LUTK + (pair_code_shifted<BK, G::KSH>(kw, 4 * j + e) | krep));
-              h4[e] = v.x;
-              l4[e] = v.y;
-            }
-            const uint32_t off = tc::sw128_offset(kTChunk, pos, 64 * half + 8 * j);
-            *reinterpret_cast<uint4*>(khp + off) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
-            *reinterpret_cast<uint4*>(klp + off) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
-          }
-        }
-        if (u < kTChunk) {
-          // norms as floats; 0 past the sequence end (the copied norm runs
-          // stop at a multiple of 8 positions: the rest of the slot is stale)
-          const bool live = (cbase + c) * kTChunk + u < L;
-          const uint16_t* ns = reinterpret_cast<const uint16_t*>(st + kTChunk * (G::RK + G::RV));
-          const int slot = (c & (kTNormSlots - 1)) * kTChunk + u;
-          reinterpret_cast<float*>(smem + G::NKF)[slot] =
-              live ? __half2float(__ushort_as_half(ns[u])) : 0.f;
-          reinterpret_cast<float*>(smem + G::NVF)[slot] =
-              live ? __half2float(__ushort_as_half(ns[kTChunk + u])) : 0.f;
-        }
-        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-        __syncwarp();
-        if (lane == 0) tc::bar_arrive(k_ready(c));
-        // V buffer i: free once the P'·V of chunk c - 2 is done
-        ok = wait(pv_done(c), par2(c) ^ 1);
-        if (!__all_sync(0xFFFFFFFFu, ok)) break;
-        {
-          uint32_t vw[(8 * BV + 3) / 4 + 1];
-          load_chunk<8 * BV>(st, kTChunk * G::RK + pos * G::RV + 8 * BV * half, vw);
-          uint8_t* vp = smem + G::VV + i * G::TILE;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            uint32_t p4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              p4[e] = lds<uint32_t>(smem, G::LUTV + (pair_code_shifted<BV, G::VSH>(vw, 4 * j + e) | vrep));
-            *reinterpret_cast<uint4*>(vp + tc::sw128_offset(kTChunk, pos, 64 * half + 8 * j)) =
-                make_uint4(p4[0], p4[1], p4[2], p4[3]);
-          }
-        }
-        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-        __syncwarp();
-        if (lane == 0) {
-          tc::bar_arrive(v_ready(c));
-          tc::bar_arrive(stage_free(c));
-        }
+      {
+        // norms as floats; 0 past the sequence end (the copied norm runs
+        // stop at a multiple of 8 positions: the rest of the slot is stale)
+        const bool live = (cbase + c) * kTChunk + u < L;
+        const uint16_t* ns = reinterpret_cast<const uint16_t*>(st + kTChunk * (G::RK + G::RV));
+        const int slot = (c & (kTNormSlots - 1)) * kTChunk + u;
+        reinterpret_cast<float*>(smem + G::NKF)[slot] =
+            live ? __half2float(__ushort_as_half(ns[u])) : 0.f;
+        reinterpret_cast<float*>(smem + G::NVF)[slot] =
+            live ? __half2float(__ushort_as_half(ns[kTChunk + u])) : 0.f;
+      }
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+      __syncwarp();
+      if (lane == 0) {
+        tc::bar_arrive(k_ready(c));
+        tc::bar_arrive(stage_free(c));
       }
     }
   } else {
@@ -428,8 +440,8 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
     float mu = -INFINITY, l = 0.f;
     bool ok = true;
     for (int c = 0; c < nchunks; ++c) {
-      // the scores, and (acquired from the dequantizing warps directly) the
-      // chunk's norms
+      // the scores, and (acquired from the K-dequantizing warps directly)
+      // the chunk's norms
       ok = wait(s_full(c), par2(c)) && wait(k_ready(c), par4(c));
       if (!__all_sync(0xFFFFFFFFu, ok)) {
         ok = false;
@@ -440,35 +452,33 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
       const int ns = (c & (kTNormSlots - 1)) * kTChunk;
       const float4* nk4 = reinterpret_cast<const float4*>(smem + G::NKF) + ns / 4;
       const float4* nv4 = reinterpret_cast<const float4*>(smem + G::NVF) + ns / 4;
-      float sv[kTChunk];
-      {
-        float z[32];
-        tc::tmem_ld32(tmem + trow + kColS + kTChunk * (c & 1), z);
-#pragma unroll
-        for (int k = 0; k < 32; ++k) sv[k] = z[k];
-        tc::tmem_ld32(tmem + trow + kColS + kTChunk * (c & 1) + 32, z);
-#pragma unroll
-        for (int k = 0; k < 32; ++k) sv[32 + k] = z[k];
-      }
-      // the score buffer is free for chunk c + 2
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) tc::bar_arrive(s_free(c));
-      float mx = -INFINITY;
+      const uint32_t sbuf = tmem + trow + kColS + kTChunk * (c & 1);
       const bool masked = t0 + kTChunk - 1 > lim;
-#pragma unroll
-      for (int k = 0; k < kTChunk; k += 4) {
-        const float4 n = nk4[k / 4];
-        float2 v0 = __fmul2_rn(make_float2(sv[k], sv[k + 1]), make_float2(n.x, n.y));
-        float2 v1 = __fmul2_rn(make_float2(sv[k + 2], sv[k + 3]), make_float2(n.z, n.w));
+      // v = score x K norm, -inf past the row's last visible position
+      auto scaled = [&](const float (&z)[32], int q, int k, float2& v0, float2& v1) {
+        const float4 n = nk4[8 * q + k / 4];
+        v0 = __fmul2_rn(make_float2(z[k], z[k + 1]), make_float2(n.x, n.y));
+        v1 = __fmul2_rn(make_float2(z[k + 2], z[k + 3]), make_float2(n.z, n.w));
         if (masked) {
-          if (t0 + k > lim) v0.x = -INFINITY;
-          if (t0 + k + 1 > lim) v0.y = -INFINITY;
-          if (t0 + k + 2 > lim) v1.x = -INFINITY;
-          if (t0 + k + 3 > lim) v1.y = -INFINITY;
+          const int p = t0 + 32 * q + k;
+          if (p > lim) v0.x = -INFINITY;
+          if (p + 1 > lim) v0.y = -INFINITY;
+          if (p + 2 > lim) v1.x = -INFINITY;
+          if (p + 3 > lim) v1.y = -INFINITY;
         }
-        sv[k] = v0.x; sv[k + 1] = v0.y; sv[k + 2] = v1.x; sv[k + 3] = v1.y;
-        mx = fmaxf(mx, fmaxf(fmaxf(v0.x, v0.y), fmaxf(v1.x, v1.y)));
+      };
+      // pass 1: the chunk's maximum
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (int q = 0; q < kTChunk / 32; ++q) {
+        float z[32];
+        tc::tmem_ld32(sbuf + 32 * q, z);
+#pragma unroll
+        for (int k = 0; k < 32; k += 4) {
+          float2 v0, v1;
+          scaled(z, q, k, v0, v1);
+          mx = fmaxf(mx, fmaxf(fmaxf(v0.x, v0.y), fmaxf(v1.x, v1.y)));
+        }
       }
       const float mn = fmaxf(mu, mx);
       // the output row holds earlier chunks' products: rescale it (after the
@@ -496,42 +506,36 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
         }
       }
       if (grow || mu == -INFINITY) mu = mn;
-      // weights 2^(si·v - si·mu - 8) (0 for masked scores), their sum, and P'
+      // pass 2: weights 2^(si·v - si·mu - 8) (0 for masked scores), their
+      // sum, and P' over the columns already read: the 16 P' columns of
+      // piece q lie in columns 16q .. 16q + 15 of the buffer
       const float off = mu == -INFINITY ? 0.f : -fmaf(si, mu, 8.f);
       const float2 off2 = make_float2(off, off);
       float2 ls = make_float2(0.f, 0.f);
-      uint32_t pw[kTChunk / 2];
+#pragma unroll 1
+      for (int q = 0; q < kTChunk / 32; ++q) {
+        float z[32];
+        tc::tmem_ld32(sbuf + 32 * q, z);
+        uint32_t pw[16];
 #pragma unroll
-      for (int k = 0; k < kTChunk; k += 4) {
-        const float4 n = nv4[k / 4];
-        const float2 e0 = __ffma2_rn(make_float2(sv[k], sv[k + 1]), si2, off2);
-        const float2 e1 = __ffma2_rn(make_float2(sv[k + 2], sv[k + 3]), si2, off2);
-        const float2 w0 = make_float2(fast_exp2(e0.x), fast_exp2(e0.y));
-        const float2 w1 = make_float2(fast_exp2(e1.x), fast_exp2(e1.y));
-        ls = __fadd2_rn(ls, __fadd2_rn(w0, w1));
-        const float2 p0 = __fmul2_rn(w0, make_float2(n.x, n.y));
-        const float2 p1 = __fmul2_rn(w1, make_float2(n.z, n.w));
-        pw[k / 2] = pack_half2(p0.x, p0.y);
-        pw[k / 2 + 1] = pack_half2(p1.x, p1.y);
-      }
-      l = l * al + (ls.x + ls.y);
-      // P' row into buffer c & 1 (free once the P'·V of chunk c - 2 is done)
-      ok = wait(pv_done(c), par2(c) ^ 1);
-      if (!__all_sync(0xFFFFFFFFu, ok)) {
-        ok = false;
-        break;
-      }
-      {
-        uint32_t lo[16], hi[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          lo[k] = pw[k];
-          hi[k] = pw[16 + k];
+        for (int k = 0; k < 32; k += 4) {
+          float2 v0, v1;
+          scaled(z, q, k, v0, v1);
+          const float4 n = nv4[8 * q + k / 4];
+          const float2 e0 = __ffma2_rn(v0, si2, off2);
+          const float2 e1 = __ffma2_rn(v1, si2, off2);
+          const float2 w0 = make_float2(fast_exp2(e0.x), fast_exp2(e0.y));
+          const float2 w1 = make_float2(fast_exp2(e1.x), fast_exp2(e1.y));
+          ls = __fadd2_rn(ls, __fadd2_rn(w0, w1));
+          const float2 p0 = __fmul2_rn(w0, make_float2(n.x, n.y));
+          const float2 p1 = __fmul2_rn(w1, make_float2(n.z, n.w));
+          pw[k / 2] = pack_half2(p0.x, p0.y);
+          pw[k / 2 + 1] = pack_half2(p1.x, p1.y);
         }
-        tc::tmem_st16_nowait(tmem + trow + kColP + 32 * (c & 1), lo);
-        tc::tmem_st16_nowait(tmem + trow + kColP + 32 * (c & 1) + 16, hi);
-        tc::tmem_wait_st();
+        tc::tmem_st16_nowait(sbuf + 16 * q, pw);
       }
+      tc::tmem_wait_st();
+      l = l * al + (ls.x + ls.y);
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::bar_arrive(p_ready(c));
@@ -559,7 +563,8 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
       }
       if (live_row && S > 1) {
         // records of this split: the unnormalized value sum (rotated
-        // domain), the base-2 running maximum and the sum (empty: 0, -inf, 0)
+        // domain), the base-2 reference maximum of its weights and their
+        // sum (empty: 0, -inf, 0)
         const size_t rec = (size_t)split * ((size_t)a.batch * T * a.n_q_heads) +
                            ((size_t)b * T + i0 + t) * a.n_q_heads + (size_t)g * GQ + h;
         float* dst = a.records + rec * (kTD + 2);
@@ -618,7 +623,7 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  if (warp == 9) tc::tmem_dealloc(tmem, kTTmemCols);
+  if (warp == 11) tc::tmem_dealloc(tmem, kTTmemCols);
 }
 
 template <int BK, int BV>
