@@ -22,7 +22,8 @@
 //   warps 4-7   dequantize K: codebook values as fp16 high and low tiles
 //               [128 positions x 128 coordinates], and the chunk's norms
 //   warps 8-9   dequantize V [128 positions x 128 coordinates]
-//   warp 10     bulk copies of the packed rows and norms (two slots)
+//   warp 10     bulk copies of the packed rows and norms (two K slots and
+//               two V slots)
 //   warp 11     tensor memory (512 columns: two 128-column score buffers,
 //               the 128-column output, the query's high and low parts); one
 //               thread issues per chunk
@@ -67,9 +68,11 @@ struct TcGeo {
   static constexpr int KH = 0;                                // 2 K high tiles
   static constexpr int KL = KH + 2 * TILE;                    // 2 K low tiles
   static constexpr int VV = KL + 2 * TILE;                    // the V tile
-  static constexpr int SLOT = kTChunk * (RK + RV) + 2 * kTChunk * 2;
+  // staging: K slots (packed K rows, then the K and V norms) and V slots
+  static constexpr int KSLOT = kTChunk * RK + 2 * kTChunk * 2, VSLOT = kTChunk * RV;
   static constexpr int STG = VV + TILE;                       // 2 staging slots
-  static constexpr int NKF = STG + 2 * SLOT;                  // norm ring: 128 floats a slot
+  static constexpr int VSTG = STG + 2 * KSLOT;
+  static constexpr int NKF = VSTG + 2 * VSLOT;                // norm ring: 128 floats a slot
   static constexpr int NVF = NKF + kTNormSlots * kTChunk * 4;
   // codebook tables, eight copies (one per lane & 7) where random lookups of
   // a warp would collide in shared-memory banks: K (uint2 per pair code)
@@ -78,10 +81,10 @@ struct TcGeo {
   static constexpr int KSH = BK == 2 ? 3 : 6, VSH = BV == 2 ? 2 : 5;  // log2 bytes per code
   static constexpr int LUTK = NVF + kTNormSlots * kTChunk * 4;
   static constexpr int LUTV = LUTK + (1 << (2 * BK)) * 8 * KREP;
-  static constexpr int BARS = LUTV + (1 << (2 * BV)) * 4 * VREP;  // 16 barriers
-  static constexpr int MISC = BARS + 16 * 8;                  // TMEM address, abort flag
+  static constexpr int BARS = LUTV + (1 << (2 * BV)) * 4 * VREP;  // 20 barriers
+  static constexpr int MISC = BARS + 20 * 8;                  // TMEM address, abort flag
   static constexpr int SMEM = 1024 + MISC + 16;
-  static_assert(SLOT % 16 == 0 && STG % 1024 == 0 && NKF % 16 == 0 && BARS % 8 == 0, "align");
+  static_assert(KSLOT % 16 == 0 && VSLOT % 16 == 0 && STG % 1024 == 0 && NKF % 16 == 0 && BARS % 8 == 0, "align");
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
@@ -110,8 +113,10 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
   // four-deep one): staging full/free, K ready (x4), V ready (x1), scores
   // full, P' ready, P'·V done, query ready
   const uint32_t bars = sb + G::BARS;
-  auto stage_full = [&](int c) { return bars + 8 * (0 + (c & 1)); };
-  auto stage_free = [&](int c) { return bars + 8 * (2 + (c & 1)); };
+  auto kst_full = [&](int c) { return bars + 8 * (0 + (c & 1)); };
+  auto kst_free = [&](int c) { return bars + 8 * (2 + (c & 1)); };
+  auto vst_full = [&](int c) { return bars + 8 * (16 + (c & 1)); };
+  auto vst_free = [&](int c) { return bars + 8 * (18 + (c & 1)); };
   auto k_ready = [&](int c) { return bars + 8 * (4 + (c & 3)); };
   const uint32_t v_ready = bars + 8 * 8;
   auto s_full = [&](int c) { return bars + 8 * (9 + (c & 1)); };
@@ -155,8 +160,10 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
   }
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
-      tc::bar_init(stage_full(i), 1);
-      tc::bar_init(stage_free(i), 6);              // the K and V dequantizing warps
+      tc::bar_init(kst_full(i), 1);
+      tc::bar_init(kst_free(i), 4);                // the K-dequantizing warps
+      tc::bar_init(vst_full(i), 1);
+      tc::bar_init(vst_free(i), 2);                // the V-dequantizing warps
       tc::bar_init(s_full(i), 1);
       tc::bar_init(p_ready(i), 4);
       tc::bar_init(pv_done(i), 1);
@@ -188,27 +195,34 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
   const size_t seq_row = ((size_t)b * H + g) * a.cap_tok;
 
   if (warp == 10) {
-    // ---- producer: chunk c into staging slot c & 1
-    if (lane == 0) {
+    // ---- producer: lane 0 copies chunk c's K rows and norms into K slot
+    // c & 1, lane 1 its V rows into V slot c & 1 (each side runs ahead of
+    // the other as far as its own slots allow)
+    if (lane < 2) {
+      const bool kside = lane == 0;
       int c = 0;
       for (; c < nchunks; ++c) {
-        if (!wait(stage_free(c), par2(c) ^ 1)) break;
+        if (!wait(kside ? kst_free(c) : vst_free(c), par2(c) ^ 1)) break;
         const int t0 = (cbase + c) * kTChunk;
         const int rows = min(kTChunk, L - t0);
         const int nrows = min(kTChunk, (rows + 7) & ~7);
-        const uint32_t dst = sb + G::STG + (c & 1) * G::SLOT;
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-        tc::bar_expect(stage_full(c), rows * (G::RK + G::RV) + 4 * nrows);
-        tc::bulk_g2s(dst, a.packed_k + (seq_row + t0) * G::RK, rows * G::RK, stage_full(c));
-        tc::bulk_g2s(dst + kTChunk * G::RK, a.packed_v + (seq_row + t0) * G::RV, rows * G::RV,
-                     stage_full(c));
-        tc::bulk_g2s(dst + kTChunk * (G::RK + G::RV), a.norms_k + seq_row + t0, 2 * nrows,
-                     stage_full(c));
-        tc::bulk_g2s(dst + kTChunk * (G::RK + G::RV) + 2 * kTChunk, a.norms_v + seq_row + t0,
-                     2 * nrows, stage_full(c));
+        if (kside) {
+          const uint32_t dst = sb + G::STG + (c & 1) * G::KSLOT;
+          tc::bar_expect(kst_full(c), rows * G::RK + 4 * nrows);
+          tc::bulk_g2s(dst, a.packed_k + (seq_row + t0) * G::RK, rows * G::RK, kst_full(c));
+          tc::bulk_g2s(dst + kTChunk * G::RK, a.norms_k + seq_row + t0, 2 * nrows, kst_full(c));
+          tc::bulk_g2s(dst + kTChunk * G::RK + 2 * kTChunk, a.norms_v + seq_row + t0, 2 * nrows,
+                       kst_full(c));
+        } else {
+          const uint32_t dst = sb + G::VSTG + (c & 1) * G::VSLOT;
+          tc::bar_expect(vst_full(c), rows * G::RV);
+          tc::bulk_g2s(dst, a.packed_v + (seq_row + t0) * G::RV, rows * G::RV, vst_full(c));
+        }
       }
       // copies still in flight complete before the CTA can end
-      for (int k = c > 2 ? c - 2 : 0; k < c; ++k) tc::bar_wait(stage_full(k), par2(k), kTWait);
+      for (int k = c > 2 ? c - 2 : 0; k < c; ++k)
+        tc::bar_wait(kside ? kst_full(k) : vst_full(k), par2(k), kTWait);
     }
   } else if (warp == 11) {
     // ---- MMA issue (one thread)
@@ -273,30 +287,31 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
     const uint32_t vrep = G::VREP > 1 ? 4 * (lane & 7) : 0;   // this lane's table copy
     for (int c = 0; c < nchunks; ++c) {
       // the V tile is free once the P'·V of chunk c - 1 is done
-      const bool ok = wait(stage_full(c), par2(c)) && (c == 0 || wait(pv_done(c - 1), par2(c - 1)));
+      const bool ok = wait(vst_full(c), par2(c)) && (c == 0 || wait(pv_done(c - 1), par2(c - 1)));
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
-      const uint8_t* st = smem + G::STG + (c & 1) * G::SLOT;
+      const uint8_t* st = smem + G::VSTG + (c & 1) * G::VSLOT;
       uint8_t* vp = smem + G::VV;
 #pragma unroll 1
       for (int j = 0; j < 4; ++j) {
         const int pos = (v & 31) + 32 * j;
         uint32_t vw[(8 * BV + 3) / 4 + 1];
-        load_chunk<8 * BV>(st, kTChunk * G::RK + pos * G::RV + 8 * BV * half, vw);
+        load_chunk<8 * BV>(st, pos * G::RV + 8 * BV * half, vw);
+        // every table load of the unit before its stores (a store would
+        // otherwise hold back the loads that follow it)
+        uint32_t p[32];
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          uint32_t p4[4];
+        for (int e = 0; e < 32; ++e)
+          p[e] = lds<uint32_t>(smem, G::LUTV + (pair_code_shifted<BV, G::VSH>(vw, e) | vrep));
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            p4[e] = lds<uint32_t>(smem, G::LUTV + (pair_code_shifted<BV, G::VSH>(vw, 4 * jj + e) | vrep));
+        for (int jj = 0; jj < 8; ++jj)
           *reinterpret_cast<uint4*>(vp + tc::sw128_offset(kTChunk, pos, 64 * half + 8 * jj)) =
-              make_uint4(p4[0], p4[1], p4[2], p4[3]);
-        }
+              make_uint4(p[4 * jj], p[4 * jj + 1], p[4 * jj + 2], p[4 * jj + 3]);
       }
       asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
       __syncwarp();
       if (lane == 0) {
         tc::bar_arrive(v_ready);
-        tc::bar_arrive(stage_free(c));
+        tc::bar_arrive(vst_free(c));
       }
     }
   } else if (warp >= 4) {
@@ -308,9 +323,9 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
     for (int c = 0; c < nchunks; ++c) {
       const int i = c & 1;
       // K buffer i: free once the scores of chunk c - 2 are done
-      const bool ok = wait(stage_full(c), par2(c)) && wait(s_full(c), par2(c) ^ 1);
+      const bool ok = wait(kst_full(c), par2(c)) && wait(s_full(c), par2(c) ^ 1);
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
-      const uint8_t* st = smem + G::STG + i * G::SLOT;
+      const uint8_t* st = smem + G::STG + i * G::KSLOT;
       uint8_t* khp = smem + G::KH + i * G::TILE;
       uint8_t* klp = smem + G::KL + i * G::TILE;
 #pragma unroll 1
@@ -318,26 +333,25 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
         const int pos = (u & 63) + 64 * j;
         uint32_t kw[(8 * BK + 3) / 4 + 1];
         load_chunk<8 * BK>(st, pos * G::RK + 8 * BK * half, kw);
+        // every table load of the unit before its stores
+        uint2 p[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          p[e] = lds<uint2>(smem, G::LUTK + (pair_code_shifted<BK, G::KSH>(kw, e) | krep));
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {              // 16-byte chunks: 4 pairs
-          uint32_t h4[4], l4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint2 w =
-                lds<uint2>(smem, G::LUTK + (pair_code_shifted<BK, G::KSH>(kw, 4 * jj + e) | krep));
-            h4[e] = w.x;
-            l4[e] = w.y;
-          }
           const uint32_t off = tc::sw128_offset(kTChunk, pos, 64 * half + 8 * jj);
-          *reinterpret_cast<uint4*>(khp + off) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
-          *reinterpret_cast<uint4*>(klp + off) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+          *reinterpret_cast<uint4*>(khp + off) =
+              make_uint4(p[4 * jj].x, p[4 * jj + 1].x, p[4 * jj + 2].x, p[4 * jj + 3].x);
+          *reinterpret_cast<uint4*>(klp + off) =
+              make_uint4(p[4 * jj].y, p[4 * jj + 1].y, p[4 * jj + 2].y, p[4 * jj + 3].y);
         }
       }
       {
         // norms as floats; 0 past the sequence end (the copied norm runs
         // stop at a multiple of 8 positions: the rest of the slot is stale)
         const bool live = (cbase + c) * kTChunk + u < L;
-        const uint16_t* ns = reinterpret_cast<const uint16_t*>(st + kTChunk * (G::RK + G::RV));
+        const uint16_t* ns = reinterpret_cast<const uint16_t*>(st + kTChunk * G::RK);
         const int slot = (c & (kTNormSlots - 1)) * kTChunk + u;
         reinterpret_cast<float*>(smem + G::NKF)[slot] =
             live ? __half2float(__ushort_as_half(ns[u])) : 0.f;
@@ -348,7 +362,7 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
       __syncwarp();
       if (lane == 0) {
         tc::bar_arrive(k_ready(c));
-        tc::bar_arrive(stage_free(c));
+        tc::bar_arrive(kst_free(c));
       }
     }
   } else {
@@ -467,19 +481,23 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
           if (p + 3 > lim) v1.y = -INFINITY;
         }
       };
-      // pass 1: the chunk's maximum
-      float mx = -INFINITY;
+      // pass 1: the chunk's maximum (pieces loaded two at a time: one wait
+      // for both)
+      float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll 1
-      for (int q = 0; q < kTChunk / 32; ++q) {
-        float z[32];
-        tc::tmem_ld32(sbuf + 32 * q, z);
+      for (int qp = 0; qp < kTChunk / 64; ++qp) {
+        float za[32], zb[32];
+        tc::tmem_ld32x2(sbuf + 64 * qp, sbuf + 64 * qp + 32, za, zb);
 #pragma unroll
         for (int k = 0; k < 32; k += 4) {
-          float2 v0, v1;
-          scaled(z, q, k, v0, v1);
-          mx = fmaxf(mx, fmaxf(fmaxf(v0.x, v0.y), fmaxf(v1.x, v1.y)));
+          float2 v0, v1, v2, v3;
+          scaled(za, 2 * qp, k, v0, v1);
+          scaled(zb, 2 * qp + 1, k, v2, v3);
+          mx0 = fmaxf(mx0, fmaxf(fmaxf(v0.x, v0.y), fmaxf(v1.x, v1.y)));
+          mx1 = fmaxf(mx1, fmaxf(fmaxf(v2.x, v2.y), fmaxf(v3.x, v3.y)));
         }
       }
+      const float mx = fmaxf(mx0, mx1);
       const float mn = fmaxf(mu, mx);
       // the output row holds earlier chunks' products: rescale it (after the
       // previous P'·V completes) when the reference maximum moves
@@ -513,26 +531,32 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
       const float2 off2 = make_float2(off, off);
       float2 ls = make_float2(0.f, 0.f);
 #pragma unroll 1
-      for (int q = 0; q < kTChunk / 32; ++q) {
-        float z[32];
-        tc::tmem_ld32(sbuf + 32 * q, z);
-        uint32_t pw[16];
+      for (int qp = 0; qp < kTChunk / 64; ++qp) {
+        float z[2][32];
+        tc::tmem_ld32x2(sbuf + 64 * qp, sbuf + 64 * qp + 32, z[0], z[1]);
+        uint32_t pw[2][16];
 #pragma unroll
-        for (int k = 0; k < 32; k += 4) {
-          float2 v0, v1;
-          scaled(z, q, k, v0, v1);
-          const float4 n = nv4[8 * q + k / 4];
-          const float2 e0 = __ffma2_rn(v0, si2, off2);
-          const float2 e1 = __ffma2_rn(v1, si2, off2);
-          const float2 w0 = make_float2(fast_exp2(e0.x), fast_exp2(e0.y));
-          const float2 w1 = make_float2(fast_exp2(e1.x), fast_exp2(e1.y));
-          ls = __fadd2_rn(ls, __fadd2_rn(w0, w1));
-          const float2 p0 = __fmul2_rn(w0, make_float2(n.x, n.y));
-          const float2 p1 = __fmul2_rn(w1, make_float2(n.z, n.w));
-          pw[k / 2] = pack_half2(p0.x, p0.y);
-          pw[k / 2 + 1] = pack_half2(p1.x, p1.y);
+        for (int hq = 0; hq < 2; ++hq) {
+          const int q = 2 * qp + hq;
+#pragma unroll
+          for (int k = 0; k < 32; k += 4) {
+            float2 v0, v1;
+            scaled(z[hq], q, k, v0, v1);
+            const float4 n = nv4[8 * q + k / 4];
+            const float2 e0 = __ffma2_rn(v0, si2, off2);
+            const float2 e1 = __ffma2_rn(v1, si2, off2);
+            const float2 w0 = make_float2(fast_exp2(e0.x), fast_exp2(e0.y));
+            const float2 w1 = make_float2(fast_exp2(e1.x), fast_exp2(e1.y));
+            ls = __fadd2_rn(ls, __fadd2_rn(w0, w1));
+            const float2 p0 = __fmul2_rn(w0, make_float2(n.x, n.y));
+            const float2 p1 = __fmul2_rn(w1, make_float2(n.z, n.w));
+            pw[hq][k / 2] = pack_half2(p0.x, p0.y);
+            pw[hq][k / 2 + 1] = pack_half2(p1.x, p1.y);
+          }
         }
-        tc::tmem_st16_nowait(sbuf + 16 * q, pw);
+        // both pieces read: P' of piece q to columns 16q .. 16q + 15
+        tc::tmem_st16_nowait(sbuf + 32 * qp, pw[0]);
+        tc::tmem_st16_nowait(sbuf + 32 * qp + 16, pw[1]);
       }
       tc::tmem_wait_st();
       l = l * al + (ls.x + ls.y);
