@@ -74,12 +74,17 @@ struct TcGeo {
   static constexpr int VSTG = STG + 2 * KSLOT;
   static constexpr int NKF = VSTG + 2 * VSLOT;                // norm ring: 128 floats a slot
   static constexpr int NVF = NKF + kTNormSlots * kTChunk * 4;
-  // codebook tables, eight copies (one per lane & 7) where random lookups of
-  // a warp would collide in shared-memory banks: K (uint2 per pair code)
-  // unless 2-bit, V (uint32 per pair code) unless 2-bit
-  static constexpr int KREP = BK == 2 ? 1 : 8, VREP = BV == 2 ? 1 : 8;
-  static constexpr int KSH = BK == 2 ? 3 : 6, VSH = BV == 2 ? 2 : 5;  // log2 bytes per code
+  // codebook tables, several copies where a warp's random lookups would
+  // collide in shared-memory banks (lane l reads copy l % KREP): K (uint2
+  // per pair code) 16 copies where they fit (conflict-free: a 64-bit load
+  // serves 16 lanes at a time), else 8, 1 at 2 bits; V (uint32 per pair
+  // code) 8 copies unless 2-bit
   static constexpr int LUTK = NVF + kTNormSlots * kTChunk * 4;
+  static constexpr int VREP = BV == 2 ? 1 : 8;
+  static constexpr bool K16 = LUTK + (1 << (2 * BK)) * 8 * 16 + (1 << (2 * BV)) * 4 * VREP +
+                              20 * 8 + 16 + 1024 <= 227 * 1024;
+  static constexpr int KREP = BK == 2 ? 1 : K16 ? 16 : 8;
+  static constexpr int KSH = BK == 2 ? 3 : K16 ? 7 : 6, VSH = BV == 2 ? 2 : 5;  // log2 bytes per code
   static constexpr int LUTV = LUTK + (1 << (2 * BK)) * 8 * KREP;
   static constexpr int BARS = LUTV + (1 << (2 * BV)) * 4 * VREP;  // 20 barriers
   static constexpr int MISC = BARS + 20 * 8;                  // TMEM address, abort flag
@@ -319,7 +324,7 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
     // coordinates 64·(u >> 6) .. + 63, and the norms of position u
     const int u = tid - 128;
     const int half = u >> 6;
-    const uint32_t krep = G::KREP > 1 ? 8 * (lane & 7) : 0;   // this lane's table copy
+    const uint32_t krep = 8 * (lane & (G::KREP - 1));        // this lane's table copy
     for (int c = 0; c < nchunks; ++c) {
       const int i = c & 1;
       // K buffer i: free once the scores of chunk c - 2 are done
