@@ -299,7 +299,10 @@ int tq_prefill_splits(int batch, int n_tok, int n_q_heads, int gqa_ratio, int ma
   // CTAs of one split (one per SM: 128 query rows each); pick the split
   // count that minimizes rounds of the SMs times the time of one CTA
   const long long rows_per_tile = 128 / gqa_ratio;
-  const double chunks = (double)((max_ctx > n_tok ? max_ctx : n_tok) / 64 + 1);
+  // the longest tile's 128-position chunks; a split of fewer chunks than
+  // splits would leave some empty
+  const int nch = ((max_ctx > n_tok ? max_ctx : n_tok) + 127) / 128;
+  const double chunks = (double)nch;
   const long long ctas = (long long)batch * (n_q_heads / gqa_ratio) *
                          ((n_tok + rows_per_tile - 1) / rows_per_tile);
   int dev = 0, sms = 148;
@@ -308,9 +311,9 @@ int tq_prefill_splits(int batch, int n_tok, int n_q_heads, int gqa_ratio, int ma
       sms <= 0)
     sms = 148;
   int best = 1;
-  double best_cost = (double)((ctas + sms - 1) / sms) * (chunks + 10.0);
-  for (int sp = 2; sp <= kMaxPrefillSplits; ++sp) {
-    const double cost = (double)((ctas * sp + sms - 1) / sms) * (chunks / sp + 10.0);
+  double best_cost = (double)((ctas + sms - 1) / sms) * (chunks + 5.0);
+  for (int sp = 2; sp <= kMaxPrefillSplits && sp <= nch; ++sp) {
+    const double cost = (double)((ctas * sp + sms - 1) / sms) * (chunks / sp + 5.0);
     if (cost < best_cost - 1e-9) {
       best = sp;
       best_cost = cost;

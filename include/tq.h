@@ -347,11 +347,11 @@ int tq_prefill_attend_split(const void* q, int q_dtype,
 size_t tq_prefill_workspace_size(int batch, int n_tok, int n_q_heads, int d, int n_splits);
 
 /* A split count for tq_prefill_attend_split on the current device, for
- * sequences of at most max_ctx positions (n_tok if smaller): the n in 1..8
- * that minimizes ceil(tiles·n / SMs) · (chunks / n + 10), i.e. rounds of
- * the SMs times the time of one CTA, which handles 1/n of the longest
- * tile's 64-position chunks after a fixed cost of about 10 chunks (set-up,
- * pipeline fill and drain). Host only; 1 on bad input. */
+ * sequences of at most max_ctx positions (n_tok if smaller): the n in
+ * 1..min(8, chunks) that minimizes ceil(tiles·n / SMs) · (chunks / n + 5),
+ * i.e. rounds of the SMs times the time of one CTA, which handles 1/n of
+ * the longest tile's 128-position chunks after a fixed cost of about 5
+ * chunks (set-up, pipeline fill and drain). Host only; 1 on bad input. */
 int tq_prefill_splits(int batch, int n_tok, int n_q_heads, int gqa_ratio, int max_ctx);
 
 /*

@@ -271,6 +271,21 @@ def test_prefill_workspace_size_and_split_choice():
     assert tq.tq_prefill_splits(0, 1024, 32, 4, 8192) == 1
 
 
+def test_prefill_split_choice_follows_the_measured_sweep():
+    """On a 148-SM device (the host default without a GPU) the split count
+    is the fastest one measured for these chunk shapes (8 kv heads, GQA 4):
+    1 for 1024 tokens over 8192 (256 tiles already fill the SMs), 4 for 128
+    tokens over 8192 (32 tiles), 1 for 4096 tokens over 16384."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("the choice depends on the device's SM count")
+    assert tq.tq_prefill_splits(1, 1024, 32, 4, 8192) == 1
+    assert tq.tq_prefill_splits(1, 128, 32, 4, 8192) == 4
+    assert tq.tq_prefill_splits(1, 4096, 32, 4, 16384) == 1
+    # a short context leaves little to split: one chunk per tile
+    assert tq.tq_prefill_splits(1, 128, 32, 4, 128) == 1
+
+
 @pytest.mark.parametrize("head_skipped,want", [
     (None, tq.TQ_ERR_INVALID_ARG),          # the counts array is required
     (FAKE + 2, tq.TQ_ERR_INVALID_ARG),      # not 4-byte aligned
