@@ -486,13 +486,15 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
           if (p + 3 > lim) v1.y = -INFINITY;
         }
       };
-      // pass 1: the chunk's maximum (pieces loaded two at a time: one wait
-      // for both)
+      // pass 1: v = score x K norm (masked) written back over the scores,
+      // and the chunk's maximum (pieces loaded two at a time: one wait for
+      // both)
       float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll 1
       for (int qp = 0; qp < kTChunk / 64; ++qp) {
         float za[32], zb[32];
         tc::tmem_ld32x2(sbuf + 64 * qp, sbuf + 64 * qp + 32, za, zb);
+        uint32_t va[32], vb[32];
 #pragma unroll
         for (int k = 0; k < 32; k += 4) {
           float2 v0, v1, v2, v3;
@@ -500,8 +502,15 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
           scaled(zb, 2 * qp + 1, k, v2, v3);
           mx0 = fmaxf(mx0, fmaxf(fmaxf(v0.x, v0.y), fmaxf(v1.x, v1.y)));
           mx1 = fmaxf(mx1, fmaxf(fmaxf(v2.x, v2.y), fmaxf(v3.x, v3.y)));
+          va[k] = __float_as_uint(v0.x); va[k + 1] = __float_as_uint(v0.y);
+          va[k + 2] = __float_as_uint(v1.x); va[k + 3] = __float_as_uint(v1.y);
+          vb[k] = __float_as_uint(v2.x); vb[k + 1] = __float_as_uint(v2.y);
+          vb[k + 2] = __float_as_uint(v3.x); vb[k + 3] = __float_as_uint(v3.y);
         }
+        tc::tmem_st32_nowait(sbuf + 64 * qp, va);
+        tc::tmem_st32_nowait(sbuf + 64 * qp + 32, vb);
       }
+      tc::tmem_wait_st();
       const float mx = fmaxf(mx0, mx1);
       const float mn = fmaxf(mu, mx);
       // the output row holds earlier chunks' products: rescale it (after the
@@ -545,8 +554,9 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
           const int q = 2 * qp + hq;
 #pragma unroll
           for (int k = 0; k < 32; k += 4) {
-            float2 v0, v1;
-            scaled(z[hq], q, k, v0, v1);
+            // v, as pass 1 left it
+            const float2 v0 = make_float2(z[hq][k], z[hq][k + 1]);
+            const float2 v1 = make_float2(z[hq][k + 2], z[hq][k + 3]);
             const float4 n = nv4[8 * q + k / 4];
             const float2 e0 = __ffma2_rn(v0, si2, off2);
             const float2 e1 = __ffma2_rn(v1, si2, off2);
