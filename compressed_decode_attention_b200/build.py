@@ -1,7 +1,7 @@
 """Build the library in-tree: csrc/*.cu, csrc/*.cpp -> libtq.so (sm_100a).
 
 Usage: python -m compressed_decode_attention_b200.build [--force] [--verbose]
-       [--waittest]
+       [--waittest | --debug]
 Objects go to _build/ beside this file; the shared library is written next
 to this file so it travels with the source tree.
 
@@ -9,6 +9,11 @@ to this file so it travels with the source tree.
 build of the same sources with TQ_TEST_INJECT_WAIT_FAULTS: short bounded
 waits and two waits made to run out, for the test of the kernels' give-up
 path (tests/test_gpu_wait_timeout.py). Only that test loads it.
+
+--debug (build(variant="debug")) builds libtq_debug.so, the bounds-checked
+build (TQ_DEBUG): the copy and store index checks of the kernels are live
+and report TQ_DEV_DEBUG_CHECK instead of touching memory out of range
+(tests/test_gpu_debug_build.py runs it).
 """
 from __future__ import annotations
 
@@ -44,7 +49,8 @@ def _stale(target, deps):
 
 
 VARIANTS = {None: ("libtq.so", "", []),
-            "waittest": ("libtq_waittest.so", "waittest", ["-DTQ_TEST_INJECT_WAIT_FAULTS"])}
+            "waittest": ("libtq_waittest.so", "waittest", ["-DTQ_TEST_INJECT_WAIT_FAULTS"]),
+            "debug": ("libtq_debug.so", "debug", ["-DTQ_DEBUG"])}
 
 
 def _compile(src, verbose, obj_dir=None, defines=()):
@@ -85,4 +91,5 @@ def build(force: bool = False, verbose: bool = False, variant=None) -> str:
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv,
-                variant="waittest" if "--waittest" in sys.argv else None))
+                variant="waittest" if "--waittest" in sys.argv else
+                "debug" if "--debug" in sys.argv else None))

@@ -802,11 +802,17 @@ attend_kernel(const __grid_constant__ AttendArgs a,
         const uint32_t bar = smem_addr(smem) + Gm::QOFF + Gm::QS + Gm::MISC + (v * kMaxStages + slot) * 8;
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
         const uint32_t extra = kInjectWaitFaults && a.new_kv == nullptr && j == 0 ? 16u : 0u;
-        mbar_expect(bar, krows * Gm::RK + vrows * Gm::RV + 4 * nrows + extra);
-        bulk_g2s(dst, gk + (size_t)t0 * Gm::RK, krows * Gm::RK, bar);
-        bulk_g2s(dst + Gm::KB, gv + (size_t)t0 * Gm::RV, vrows * Gm::RV, bar);
-        bulk_g2s(dst + Gm::NKOFF, gnk + t0, 2 * nrows, bar);
-        bulk_g2s(dst + Gm::NKOFF + 2 * kBlk, gnv + t0, 2 * nrows, bar);
+        // the rows lie in the sequence's capacity (checked in the
+        // bounds-checked build; a skipped copy still completes the phase)
+        const bool inb = tq_check(t0 >= 0 && rows > 0 &&
+                                  t0 + max(krows, max(vrows, nrows)) <= a.cap_tok, a.dev_status);
+        mbar_expect(bar, inb ? krows * Gm::RK + vrows * Gm::RV + 4 * nrows + extra : 0u);
+        if (inb) {
+          bulk_g2s(dst, gk + (size_t)t0 * Gm::RK, krows * Gm::RK, bar);
+          bulk_g2s(dst + Gm::KB, gv + (size_t)t0 * Gm::RV, vrows * Gm::RV, bar);
+          bulk_g2s(dst + Gm::NKOFF, gnk + t0, 2 * nrows, bar);
+          bulk_g2s(dst + Gm::NKOFF + 2 * kBlk, gnv + t0, 2 * nrows, bar);
+        }
       }
     };
     auto issue = [&](int c, int j) { issue_for(warp, wp0, wp1, c, j); };

@@ -11,6 +11,20 @@
 
 namespace tq {
 
+// Index check of the bounds-checked build (compiled with TQ_DEBUG): a failed
+// check sets TQ_DEV_DEBUG_CHECK and the caller skips the access (no trap: the
+// context stays usable). Without TQ_DEBUG every check is the constant true.
+__device__ __forceinline__ bool tq_check(bool ok, int* dev_status) {
+#ifdef TQ_DEBUG
+  if (!ok && dev_status) atomicOr(dev_status, TQ_DEV_DEBUG_CHECK);
+  return ok;
+#else
+  (void)ok;
+  (void)dev_status;
+  return true;
+#endif
+}
+
 __device__ __forceinline__ float2 unpack16x2(uint32_t w, bool bf16) {
   if (bf16) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));

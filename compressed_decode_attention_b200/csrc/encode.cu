@@ -54,6 +54,8 @@ encode_kernel(const __grid_constant__ EncodeArgs a,
   const size_t tok_stride = (size_t)a.n_kv_heads * D;
   for (int tok = blockIdx.x * kTokens + threadIdx.x / LPV; tok < a.n_tok;
        tok += gridDim.x * kTokens) {
+    // the destination row lies in the cache (bounds-checked build)
+    if (!tq_check(a.tok_offset + tok < a.cap_tok, a.dev_status)) continue;
     float x[32];
     load_signed(src0 + tok * tok_stride, sub, a.is_bf16, smask, x);
     if (bits == 4)

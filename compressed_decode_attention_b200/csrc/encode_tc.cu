@@ -268,7 +268,8 @@ encode_tc_kernel(const __grid_constant__ EncodeArgs a, const __grid_constant__ C
       asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
       const TcItem it = item_of(j);
       const int tok = it.t * kTile + r;
-      const bool valid = tok < a.n_tok;
+      // (and, in the bounds-checked build, its row lies in the cache)
+      const bool valid = tok < a.n_tok && tq_check(a.tok_offset + tok < a.cap_tok, a.dev_status);
       const int bits = it.kv ? a.bits_v : a.bits_k;
       const size_t rb = (size_t)kDim * bits / 8;
       const size_t rowi = (size_t)it.h * a.cap_tok + a.tok_offset + (valid ? tok : 0);

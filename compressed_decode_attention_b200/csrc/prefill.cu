@@ -212,17 +212,23 @@ prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__
         const int rows = min(kTChunk, L - t0);
         const int nrows = min(kTChunk, (rows + 7) & ~7);
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+        // the rows lie in the sequence's capacity (checked in the
+        // bounds-checked build; a skipped copy still completes the phase)
+        const bool inb = tq_check(t0 >= 0 && rows > 0 && t0 + nrows <= a.cap_tok, a.dev_status);
         if (kside) {
           const uint32_t dst = sb + G::STG + (c & 1) * G::KSLOT;
-          tc::bar_expect(kst_full(c), rows * G::RK + 4 * nrows);
-          tc::bulk_g2s(dst, a.packed_k + (seq_row + t0) * G::RK, rows * G::RK, kst_full(c));
-          tc::bulk_g2s(dst + kTChunk * G::RK, a.norms_k + seq_row + t0, 2 * nrows, kst_full(c));
-          tc::bulk_g2s(dst + kTChunk * G::RK + 2 * kTChunk, a.norms_v + seq_row + t0, 2 * nrows,
-                       kst_full(c));
+          tc::bar_expect(kst_full(c), inb ? rows * G::RK + 4 * nrows : 0u);
+          if (inb) {
+            tc::bulk_g2s(dst, a.packed_k + (seq_row + t0) * G::RK, rows * G::RK, kst_full(c));
+            tc::bulk_g2s(dst + kTChunk * G::RK, a.norms_k + seq_row + t0, 2 * nrows, kst_full(c));
+            tc::bulk_g2s(dst + kTChunk * G::RK + 2 * kTChunk, a.norms_v + seq_row + t0, 2 * nrows,
+                         kst_full(c));
+          }
         } else {
           const uint32_t dst = sb + G::VSTG + (c & 1) * G::VSLOT;
-          tc::bar_expect(vst_full(c), rows * G::RV);
-          tc::bulk_g2s(dst, a.packed_v + (seq_row + t0) * G::RV, rows * G::RV, vst_full(c));
+          tc::bar_expect(vst_full(c), inb ? rows * G::RV : 0u);
+          if (inb)
+            tc::bulk_g2s(dst, a.packed_v + (seq_row + t0) * G::RV, rows * G::RV, vst_full(c));
         }
       }
       // copies still in flight complete before the CTA can end

@@ -91,6 +91,8 @@ typedef enum { TQ_F16 = 0, TQ_BF16 = 1, TQ_F32 = 2 } tq_dtype;
 #define TQ_DEV_NORM_SATURATED 2  /* some norm > 65504; stored as 65504      */
 #define TQ_DEV_CTX_EMPTY      4  /* some ctx_lens[b] <= 0; output set to 0  */
 #define TQ_DEV_WAIT_TIMEOUT   8  /* a wait for staged cache data gave up    */
+#define TQ_DEV_DEBUG_CHECK   16  /* bounds-checked build (TQ_DEBUG) only: an
+                                    index check failed; the access was skipped */
                                  /* after ~1 s; the output is not valid     */
 
 /* Library ABI version (TQ_ABI_VERSION of the build). */

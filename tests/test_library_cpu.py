@@ -35,6 +35,20 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(tq, n), f"binding lacks {n}"
 
 
+@pytest.mark.parametrize("variant", ["libtq_debug.so", "libtq_waittest.so"])
+def test_checked_and_test_builds_export_the_same_abi(variant):
+    """The bounds-checked (TQ_DEBUG) and wait-fault test builds are the same
+    library: every declared symbol, the same ABI version."""
+    path = os.path.join(os.path.dirname(tq.LIB_PATH), variant)
+    if not os.path.exists(path):
+        pytest.skip(f"{variant} not built (build() of __graft_entry__ builds it)")
+    lib = ctypes.CDLL(path)
+    for n in _declared_functions():
+        assert hasattr(lib, n), n
+    lib.tq_abi_version.restype = ctypes.c_int
+    assert lib.tq_abi_version() == tq.tq_abi_version()
+
+
 def test_abi_version_and_status_strings():
     hdr = open(os.path.join(ROOT, "include", "tq.h")).read()
     assert tq.tq_abi_version() == int(re.search(r"#define TQ_ABI_VERSION (\d+)", hdr).group(1))
