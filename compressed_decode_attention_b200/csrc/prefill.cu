@@ -11,14 +11,16 @@
 // One CTA per (context split, sequence, kv head, tile of 128 query rows); a
 // row is a (token, query head of the GQA group) pair. Warp roles:
 //   warps 0-3   one thread per row: rotate its query (thread-local FWHT)
-//               into fp16 high/low parts in tensor memory; per chunk read
-//               the row of scores (two passes of four 32-column loads:
-//               maximum, then weights), scale, causal mask, online softmax
-//               in the log2 domain, rescale the output row when the
-//               reference maximum moves, and write the row of P' = weight x
-//               V norm (fp16 pairs) over the columns of its own scores; at
-//               the end read the output row, normalize, inverse-rotate and
-//               store it (or the split's record)
+//               into fp16 high/low parts in tensor memory; per chunk two
+//               passes over the row of scores (32-column loads, two per
+//               wait): the first scales them by the K norms, masks them
+//               causally, writes them back and takes the maximum; the
+//               second takes the weights (online softmax in the log2
+//               domain; the output row is rescaled when the reference
+//               maximum moves) and writes the row of P' = weight x V norm
+//               (fp16 pairs) over the columns of its own scores; at the end
+//               read the output row, normalize, inverse-rotate and store it
+//               (or the split's record)
 //   warps 4-7   dequantize K: codebook values as fp16 high and low tiles
 //               [128 positions x 128 coordinates], and the chunk's norms
 //   warps 8-9   dequantize V [128 positions x 128 coordinates]
