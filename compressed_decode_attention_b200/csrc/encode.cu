@@ -12,8 +12,8 @@
 //           D applied by one XOR per fp16 pair
 //   norm    16 paired FMAs + 2 shuffles
 //   rotate  1 scalar + 4 paired butterfly stages, 2 cross-lane stages
-//   index   zeta = z/n compared as z against n·t (symmetric half table),
-//           counted with compare-and-set results
+//   index   zeta = z/n compared as |z| against n·t (symmetric half table)
+//           by a binary search of saturated FMAs
 //   pack    the lane's 32 indices are 4·bits contiguous bytes of the row
 #include <atomic>
 #include "encode_common.cuh"

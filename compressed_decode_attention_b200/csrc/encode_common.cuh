@@ -94,13 +94,15 @@ __device__ __forceinline__ void quantize_pack(const float (&x)[32], float n, con
   constexpr int kHalf = 1 << (BITS - 1);
 
   // idx = #{j : z/n >= t_j} over the symmetric table (t_{half-1} = 0), on
-  // the FMA pipe. With a = |z| and the positive thresholds t_k (k = 1 ..
-  // half-1, N(0,1) units), each indicator [a < n·t_k] is the saturated
-  //   y_k = sat(t_k·2^24 - a·(2^24/n))
-  // (1 below the threshold, 0 at or above it, fractional only within
-  // 2^-24 of it in zeta = z/n: inside the comparison window, where either
-  // index is acceptable). With the odd number
-  // w = 2·count + 1 = (2·half - 1) - 2·sum_k y_k:
+  // the FMA pipe. With a = |z| and the positive thresholds t_1 < .. < t_m
+  // (m = half - 1, N(0,1) units), count = #{k : a >= n·t_k} is found by
+  // binary search: each step's indicator [a >= n·t] is the saturated
+  //   b = sat(a·(2^24/n) - t·2^24)
+  // (1 at or above the threshold, 0 below it, fractional only within 2^-24
+  // of it in zeta = z/n: inside the comparison window, where any index is
+  // acceptable), and the next step's threshold is picked by the bits found
+  // so far as a product-sum (exact for bits 0/1, off by at most an ulp of
+  // t·2^24, i.e. ~2^-24 in zeta). With the odd number w = 2·count + 1:
   //   z >= 0: 2·idx = 2·(half + count)     = (2·half - 1) + w
   //   z <  0: 2·idx = 2·(half - 1 - count) = (2·half - 1) - w
   // so u = copysign(w, z) + (2·half - 1) = 2·idx, and 2^24 + u rounds to
@@ -109,43 +111,44 @@ __device__ __forceinline__ void quantize_pack(const float (&x)[32], float n, con
   // idx = half: its scale uses n = 1.
   constexpr float kTwo24 = 16777216.f;
   constexpr int NTH = kHalf - 1;                      // positive thresholds
+  static_assert(NTH == 1 || NTH == 3 || NTH == 7, "2, 3 or 4 bits");
   const float big = __frcp_rn(n > 0.f ? n : 1.f) * kTwo24;
-  float C[NTH];
+  float T[NTH];                                       // t_{k+1}·2^24
 #pragma unroll
-  for (int k = 0; k < NTH; ++k) C[k] = cb.threshold[kHalf + k] * kTwo24;
+  for (int k = 0; k < NTH; ++k) T[k] = cb.threshold[kHalf + k] * kTwo24;
   constexpr float kOdd = (float)(2 * kHalf - 1);
   constexpr uint32_t kMagic = 0x4B800000u;            // bits of 2^24
+  // the binary search's threshold differences, negated (-t·2^24 enters the
+  // saturated FMA as its addend)
+  const float2 one = make_float2(1.f, 1.f);
+  auto ind = [&](float a0, float a1, float2 nt) {    // [a >= t] for both lanes
+    return make_float2(fma_sat(a0, big, nt.x), fma_sat(a1, big, nt.y));
+  };
+  auto dup = [](float v) { return make_float2(v, v); };
 
   // words[w] accumulates bits(v) << off = (kMagic + idx) << off; the kMagic
   // parts are removed after the loop
-  // With three or more positive thresholds the count is two-level: one
-  // compare (ALU pipe) against the middle threshold picks the half of the
-  // table, and only that half's HALF thresholds take a saturated FMA. Below
-  // the middle, its indicator and the upper half's are all 1; above, the
-  // lower half's are all 0.
-  constexpr int HALF = NTH / 2;
-  const float tmid = (n > 0.f ? n : 1.f) * cb.threshold[kHalf + HALF];
-
 #pragma unroll
   for (int w = 0; w < BITS; ++w) words[w] = 0;
 #pragma unroll
   for (int i = 0; i < 32; i += 2) {
     const float a0 = fabsf(x[i]), a1 = fabsf(x[i + 1]);
     float2 w2;
-    if constexpr (NTH >= 3) {
-      const bool p0 = a0 < tmid, p1 = a1 < tmid;
-      w2 = make_float2(p0 ? kOdd - 2.f * (HALF + 1) : kOdd, p1 ? kOdd - 2.f * (HALF + 1) : kOdd);
-#pragma unroll
-      for (int k = 0; k < HALF; ++k)
-        w2 = f2fma(make_float2(fma_sat(a0, -big, p0 ? C[k] : C[k + HALF + 1]),
-                               fma_sat(a1, -big, p1 ? C[k] : C[k + HALF + 1])),
-                   make_float2(-2.f, -2.f), w2);
+    if constexpr (NTH == 7) {
+      const float2 b2 = ind(a0, a1, dup(-T[3]));                               // a >= t4
+      const float2 b1 = ind(a0, a1, f2fma(b2, dup(T[1] - T[5]), dup(-T[1])));  // t6 or t2
+      // t7, t5, t3 or t1: -t1 - b2·(t5 - t1) - b1·(t3 - t1) - b2·b1·(t7 - t5 - t3 + t1)
+      float2 nt = f2fma(b2, dup(T[0] - T[4]), dup(-T[0]));
+      nt = f2fma(b1, dup(T[0] - T[2]), nt);
+      nt = f2fma(f2mul(b2, b1), dup((T[4] - T[6]) + (T[2] - T[0])), nt);
+      const float2 b0 = ind(a0, a1, nt);
+      w2 = f2fma(b2, dup(8.f), f2fma(b1, dup(4.f), f2fma(b0, dup(2.f), one)));
+    } else if constexpr (NTH == 3) {
+      const float2 b1 = ind(a0, a1, dup(-T[1]));                               // a >= t2
+      const float2 b0 = ind(a0, a1, f2fma(b1, dup(T[0] - T[2]), dup(-T[0])));  // t3 or t1
+      w2 = f2fma(b1, dup(4.f), f2fma(b0, dup(2.f), one));
     } else {
-      w2 = make_float2(kOdd, kOdd);
-#pragma unroll
-      for (int k = 0; k < NTH; ++k)
-        w2 = f2fma(make_float2(fma_sat(a0, -big, C[k]), fma_sat(a1, -big, C[k])),
-                   make_float2(-2.f, -2.f), w2);
+      w2 = f2fma(ind(a0, a1, dup(-T[0])), dup(2.f), one);
     }
     const float2 sg = f2add(make_float2(x[i], x[i + 1]), make_float2(0.f, 0.f));
     const float2 u = f2add(make_float2(copysignf(w2.x, sg.x), copysignf(w2.y, sg.y)),
