@@ -81,15 +81,19 @@ template <int BITS>
 __device__ __forceinline__ void epilogue_row(uint32_t tacc, const Codebook& cb, uint8_t* row,
                                              uint16_t* norm, bool valid, int* dev_status) {
   float z[32];
-  // pass 1: ||z||^2 = d·||x||^2 (H·H = d·I)
-  float2 ss = make_float2(0.f, 0.f);
+  // pass 1: ||z||^2 = d·||x||^2 (H·H = d·I); 64 columns per wait
+  float2 ss = make_float2(0.f, 0.f), ss1 = ss;
 #pragma unroll 1
-  for (int c = 0; c < kDim / 32; ++c) {
-    tmem_ld32(tacc + 32 * c, z);
+  for (int c = 0; c < kDim / 64; ++c) {
+    float zb[32];
+    tc::tmem_ld32x2(tacc + 64 * c, tacc + 64 * c + 32, z, zb);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) ss = f2fma(make_float2(z[2 * j], z[2 * j + 1]),
-                                            make_float2(z[2 * j], z[2 * j + 1]), ss);
+    for (int j = 0; j < 16; ++j) {
+      ss = f2fma(make_float2(z[2 * j], z[2 * j + 1]), make_float2(z[2 * j], z[2 * j + 1]), ss);
+      ss1 = f2fma(make_float2(zb[2 * j], zb[2 * j + 1]), make_float2(zb[2 * j], zb[2 * j + 1]), ss1);
+    }
   }
+  ss = f2add(ss, ss1);
   const float n = sqrtf((ss.x + ss.y) * (1.f / kDim));
   // pass 2: indices of 32 coordinates at a time, BITS words each
 #pragma unroll 1
