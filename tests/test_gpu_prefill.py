@@ -109,6 +109,15 @@ def test_prefill_matches_oracle(bk, bv, gqa, T, q_dtype):
     assert st == 0
 
 
+@pytest.mark.parametrize("bk,bv", [(bk, bv) for bk in (2, 3, 4) for bv in (2, 3, 4)])
+def test_prefill_every_bit_pair(bk, bv):
+    """Every (b_K, b_V) instantiation of the kernel (each has its own
+    shared-memory layout and table copies), on a chunk of two partial tiles."""
+    err, st = _run(bk, bv, [150], 160, 1, 4, 40, 0, 300 + 10 * bk + bv)
+    assert err <= ATOL
+    assert st == 0
+
+
 @pytest.mark.parametrize("out_dtype", ["f16", "bf16"])
 def test_prefill_output_dtypes(out_dtype):
     err, _ = _run(4, 2, [200], 256, 1, 4, 24, 3, 7, out_dtype=out_dtype)
