@@ -1026,6 +1026,7 @@ def profile_case(name, reps):
     (prints no bench line): 'llama' = tq_attend over 8 Llama-3-8B-shaped
     layer caches, 'batched' = one serving-scale call, 'qwen' = tq_attend over
     2 Qwen-14B-shaped layers, 'encode' = tq_encode of 4 bulk-prefill layers,
+    'dequant' = tq_dequant (original domain) of one bulk-prefill layer's K,
     'prefill' = tq_prefill_attend of the prefill leg's chunk on one layer.
     Caches hold tq_encode'd seeded data."""
     import torch
@@ -1044,6 +1045,19 @@ def profile_case(name, reps):
                 tq.tq_encode(kvs[l], tq.TQ_F16, w.ctx, w.n_kv_heads, w.d, w.bits_k, w.bits_v, seed,
                              caches.pk[l], caches.pv[l], caches.nk[l], caches.nv[l], w.cap_tok, 0,
                              status)
+        torch.cuda.synchronize()
+        return
+    if name == "dequant":
+        w = S.WORKLOADS[ENCODE_WORKLOAD]
+        caches = LayerCaches(w, 1, None)
+        kv = device_kv(w, 0, w.ctx, gen)
+        tq.tq_encode(kv, tq.TQ_F16, w.ctx, w.n_kv_heads, w.d, w.bits_k, w.bits_v, seed,
+                     caches.pk[0], caches.pv[0], caches.nk[0], caches.nv[0], w.cap_tok, 0, status)
+        del kv
+        out = torch.empty((w.n_kv_heads, w.ctx, w.d), dtype=torch.float32, device="cuda")
+        for _ in range(reps):
+            tq.tq_dequant(caches.pk[0], caches.nk[0], w.ctx, w.n_kv_heads, w.d, w.bits_k, seed,
+                          w.cap_tok, 0, out)
         torch.cuda.synchronize()
         return
     if name == "prefill":
@@ -1106,7 +1120,7 @@ def main(argv=None):
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", choices=["llama", "batched", "qwen", "encode",
-                                                      "prefill"],
+                                                      "dequant", "prefill"],
                     help="only launch one kernel's workload a few times (for ncu captures)")
     args = ap.parse_args(argv)
     if args.profile_case:
