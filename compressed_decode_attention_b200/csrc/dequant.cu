@@ -5,7 +5,7 @@
 // per lane, 256/(d/32) tokens of one kv head per 256-thread block. Levels
 // come from a shared-memory copy of the codebook; each warp's rows are
 // staged in shared memory and stored whole.
-#include "device_common.cuh"
+#include "encode_common.cuh"
 
 namespace tq {
 namespace {
@@ -64,18 +64,29 @@ dequant_kernel(const __grid_constant__ DequantArgs a,
     for (int i = 0; i < 32; ++i) c[i] = 0.f;
   }
 
-  float scale;
+  // y_i = c_i · scale_i: scale_i = 1/sqrt(d) in the rotated domain; in the
+  // original space c = H·c[idx] (the encoder's butterflies, two-wide) and
+  // scale_i = D_i · n / d (a sign flip commutes exactly with the product)
   if (a.domain == 1) {
     // 1/sqrt(d), correctly rounded
-    scale = D == 64 ? 0.125f : D == 128 ? 0.0883883476483184405501f : 0.0625f;
+    const float scale = D == 64 ? 0.125f : D == 128 ? 0.0883883476483184405501f : 0.0625f;
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      const float2 y = f2mul(make_float2(c[i], c[i + 1]), make_float2(scale, scale));
+      c[i] = y.x;
+      c[i + 1] = y.y;
+    }
   } else {
-    fwht_registers<32>(c);
-#pragma unroll
-    for (int o = 1; o < LPV; o <<= 1) fwht_cross_lane<32>(c, gmask, o, (sub & o) != 0);
+    rotate_vector<LPV>(c, sub, gmask);
     const uint32_t m = sm.w[sub];
+    const float scale = valid ? __half2float(__ushort_as_half(a.norms[row])) / (float)D : 0.f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) c[i] = apply_sign(c[i], m, i);
-    scale = valid ? __half2float(__ushort_as_half(a.norms[row])) / (float)D : 0.f;
+    for (int i = 0; i < 32; i += 2) {
+      const float2 y = f2mul(make_float2(c[i], c[i + 1]),
+                             make_float2(apply_sign(scale, m, i), apply_sign(scale, m, i + 1)));
+      c[i] = y.x;
+      c[i + 1] = y.y;
+    }
   }
   // Chunk q = 8·sub + k of token t's row sits at q ^ s, s = lane & 7: the
   // eight lanes of each quarter-warp store to eight different bank groups,
@@ -86,8 +97,7 @@ dequant_kernel(const __grid_constant__ DequantArgs a,
 #pragma unroll
   for (int k = 0; k < 8; ++k)
     st[t * kChunks + ((8 * sub + k) ^ s)] =
-        make_float4(c[4 * k] * scale, c[4 * k + 1] * scale, c[4 * k + 2] * scale,
-                    c[4 * k + 3] * scale);
+        make_float4(c[4 * k], c[4 * k + 1], c[4 * k + 2], c[4 * k + 3]);
   __syncwarp();
   float4* dst = reinterpret_cast<float4*>(a.out + ((size_t)h * a.n_tok + tok0) * D);
 #pragma unroll
